@@ -1,0 +1,282 @@
+"""CPU oracle for the SmoothQuant W8A8 path and the LLM.int8() decomposition.
+
+TEST INFRASTRUCTURE ONLY. Tests, ``__graft_entry__.smoke()`` and the CPU
+baseline leg of ``bench.py`` may import this package; the product package
+never does. The arithmetic lives in ``sq_oracle.c`` (plain loops, fp64/int64
+where the method has an exact definition, correctly rounded fp32 where a
+quantised code is decided). This module only marshals numpy arrays.
+
+Functions whose exact fp32 bits depend on the reduction order convention
+(the normalisation sums) are marked "parity unpinned" in ``sq_oracle.c``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "sq_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+CFLAGS = ["-O2", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared", "-std=c11"]
+
+
+def build(force: bool = False) -> str:
+    """Compile liboracle.so with gcc (strict IEEE flags)."""
+    hdr = os.path.join(_HERE, "sq_oracle.h")
+    fresh = os.path.exists(_LIB) and os.path.getmtime(_LIB) >= max(
+        os.path.getmtime(_SRC), os.path.getmtime(hdr))
+    if force or not fresh:
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", *CFLAGS, "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        _lib = ctypes.CDLL(build())
+        _declare(_lib)
+    return _lib
+
+
+_p = ctypes.c_void_p
+_i64 = ctypes.c_int64
+_i = ctypes.c_int
+_f = ctypes.c_float
+_d = ctypes.c_double
+
+
+def _declare(L):
+    L.or_col_absmax.argtypes = [_p, _i64, _i64, _i64, _p]
+    L.or_smooth_scales.argtypes = [_p, _p, _i64, _d, _p]
+    L.or_fold_weight.argtypes = [_p, _i64, _i64, _p, _i, _p]
+    L.or_fold_norm.argtypes = [_p, _p, _p, _i64, _i, _p, _p]
+    L.or_quantize_weight.argtypes = [_p, _i64, _i64, _i, _p, _p]
+    L.or_quantize_act.argtypes = [_p, _i64, _i64, _i64, _p, _i, _p, _p, _p]
+    L.or_scale_from_absmax.argtypes = [_p, _i64]
+    L.or_scale_from_absmax.restype = _f
+    L.or_norm_smooth_quant.argtypes = [_p, _i64, _i64, _i64, _i, _p, _p, _f, _i, _p, _p, _p, _p, _p]
+    L.or_norm_f64.argtypes = [_p, _i64, _i64, _i, _p, _p, _d, _p]
+    L.or_gemm_i8.argtypes = [_p, _p, _i64, _i64, _i64, _i64, _i64, _p]
+    L.or_dequant.argtypes = [_p, _i64, _i64, _i64, _p, _i, _p, _i, _p, _p]
+    L.or_round_bf16.argtypes = [_d]
+    L.or_round_bf16.restype = ctypes.c_uint16
+    L.or_round_fp16.argtypes = [_d]
+    L.or_round_fp16.restype = ctypes.c_uint16
+    L.or_llmint8_outliers.argtypes = [_p, _i64, _i64, _i64, _f, _d, _p]
+    L.or_llmint8_outliers.restype = _i64
+    L.or_llmint8_quant_rows.argtypes = [_p, _i64, _i64, _i64, _p, _i64, _p, _p]
+    L.or_llmint8_quant_weight.argtypes = [_p, _i64, _i64, _p, _i64, _p, _p]
+    L.or_llmint8_combine.argtypes = [_p, _i64, _i64, _i64, _i64, _p, _p, _p, _i64, _p, _p, _i64, _p]
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def f32(a):
+    """fp32 image of an array-like (exact for fp16/bf16 sources)."""
+    try:
+        import torch
+
+        if isinstance(a, torch.Tensor):
+            return a.detach().to("cpu", torch.float32).contiguous().numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return _c(a, np.float32)
+
+
+# ---------------------------------------------------------------- a1 / a2
+def col_absmax(X, running=None):
+    X = f32(X)
+    M, K = X.shape
+    io = np.zeros(K, np.float32) if running is None else _c(running, np.float32).copy()
+    lib().or_col_absmax(_ptr(X), M, K, K, _ptr(io))
+    return io
+
+
+# ---------------------------------------------------------------- a3
+def smooth_scales(x, w, alpha):
+    x, w = f32(x), f32(w)
+    s = np.empty_like(x)
+    lib().or_smooth_scales(_ptr(x), _ptr(w), x.size, float(alpha), _ptr(s))
+    return s
+
+
+def fold_weight(W, s, round_f32=True):
+    W = _c(f32(W) if round_f32 else W, np.float64)
+    s = _c(s, np.float64)
+    N, K = W.shape
+    out = np.empty_like(W)
+    lib().or_fold_weight(_ptr(W), N, K, _ptr(s), int(round_f32), _ptr(out))
+    return out.astype(np.float32) if round_f32 else out
+
+
+def fold_norm(gamma, beta, s, round_f32=True):
+    g = _c(gamma, np.float64)
+    b = None if beta is None else _c(beta, np.float64)
+    s = _c(s, np.float64)
+    go = np.empty_like(g)
+    bo = None if b is None else np.empty_like(b)
+    lib().or_fold_norm(_ptr(g), _ptr(b), _ptr(s), g.size, int(round_f32), _ptr(go), _ptr(bo))
+    if round_f32:
+        return go.astype(np.float32), (None if bo is None else bo.astype(np.float32))
+    return go, bo
+
+
+# ---------------------------------------------------------------- a4
+def quantize_weight(Wp, per_channel=True):
+    Wp = f32(Wp)
+    N, K = Wp.shape
+    Wq = np.empty((N, K), np.int8)
+    qs = np.empty(N if per_channel else 1, np.float32)
+    lib().or_quantize_weight(_ptr(Wp), N, K, int(per_channel), _ptr(Wq), _ptr(qs))
+    return Wq, qs
+
+
+# ---------------------------------------------------------------- a5'
+def quantize_act(X, s=None, per_token=True, static_qs=None):
+    X = f32(X)
+    M, K = X.shape
+    s = None if s is None else f32(s)
+    st = None if static_qs is None else np.array([static_qs], np.float32)
+    Xq = np.empty((M, K), np.int8)
+    qs = np.empty(M if per_token else 1, np.float32)
+    lib().or_quantize_act(_ptr(X), M, K, K, _ptr(s), int(per_token), _ptr(st), _ptr(Xq), _ptr(qs))
+    return Xq, qs
+
+
+def scale_from_absmax(absmax):
+    a = f32(absmax).ravel()
+    return np.float32(lib().or_scale_from_absmax(_ptr(a), a.size))
+
+
+# ---------------------------------------------------------------- a5
+LAYERNORM, RMSNORM = 0, 1
+
+
+def norm_smooth_quant(H, norm, gamma, beta=None, eps=1e-5, per_token=True, static_qs=None,
+                      quantize=True, absmax=None, want_v=False):
+    H = f32(H)
+    M, K = H.shape
+    g = f32(gamma)
+    b = None if beta is None else f32(beta)
+    st = None if static_qs is None else np.array([static_qs], np.float32)
+    Xq = np.empty((M, K), np.int8) if quantize else None
+    qs = np.empty(M if per_token else 1, np.float32) if quantize else None
+    am = None if absmax is None else _c(absmax, np.float32).copy()
+    V = np.empty((M, K), np.float32) if want_v else None
+    lib().or_norm_smooth_quant(_ptr(H), M, K, K, int(norm), _ptr(g), _ptr(b), float(eps),
+                               int(per_token), _ptr(st), _ptr(Xq), _ptr(qs), _ptr(am), _ptr(V))
+    return {"Xq": Xq, "qs": qs, "absmax": am, "V": V}
+
+
+def norm_f64(H, norm, gamma, beta=None, eps=1e-5):
+    H = _c(H, np.float64)
+    M, K = H.shape
+    g = _c(gamma, np.float64)
+    b = None if beta is None else _c(beta, np.float64)
+    V = np.empty((M, K), np.float64)
+    lib().or_norm_f64(_ptr(H), M, K, int(norm), _ptr(g), _ptr(b), float(eps), _ptr(V))
+    return V
+
+
+# ---------------------------------------------------------------- a6
+def gemm_i8(Xq, Wq, rows=None):
+    Xq, Wq = _c(Xq, np.int8), _c(Wq, np.int8)
+    M, K = Xq.shape
+    N = Wq.shape[0]
+    r0, r1 = (0, M) if rows is None else rows
+    acc = np.empty((r1 - r0, N), np.int64)
+    lib().or_gemm_i8(_ptr(Xq), _ptr(Wq), M, N, K, r0, r1, _ptr(acc))
+    return acc
+
+
+def dequant(acc, qs_x, qs_w, bias=None, rows=None):
+    acc = _c(acc, np.int64)
+    qs_x, qs_w = _c(qs_x, np.float32).ravel(), _c(qs_w, np.float32).ravel()
+    n_rows, N = acc.shape
+    r0 = 0 if rows is None else rows[0]
+    b = None if bias is None else _c(f32(bias), np.float64)
+    y = np.empty((n_rows, N), np.float64)
+    # qs_x is the full per-token vector (indexed by absolute row) or one scale
+    lib().or_dequant(_ptr(acc), r0, r0 + n_rows, N, _ptr(qs_x), int(qs_x.size > 1), _ptr(qs_w),
+                     int(qs_w.size > 1), _ptr(b), _ptr(y))
+    return y
+
+
+def round_bf16_bits(y):
+    y = np.asarray(y, np.float64)
+    f = lib().or_round_bf16
+    return np.array([f(float(v)) for v in y.ravel()], np.uint16).reshape(y.shape)
+
+
+def round_fp16_bits(y):
+    y = np.asarray(y, np.float64)
+    f = lib().or_round_fp16
+    return np.array([f(float(v)) for v in y.ravel()], np.uint16).reshape(y.shape)
+
+
+# ---------------------------------------------------------------- a7-a9
+def llmint8_outliers(X, thr=6.0, min_ratio=0.0):
+    X = f32(X)
+    M, K = X.shape
+    idx = np.empty(max(K, 1), np.int32)
+    n = lib().or_llmint8_outliers(_ptr(X), M, K, K, float(thr), float(min_ratio), _ptr(idx))
+    return idx[:n].copy()
+
+
+def llmint8_quant_rows(X, idx):
+    X = f32(X)
+    M, K = X.shape
+    idx = _c(idx, np.int32)
+    Xq = np.empty((M, K), np.int8)
+    qs = np.empty(M, np.float32)
+    lib().or_llmint8_quant_rows(_ptr(X), M, K, K, _ptr(idx), idx.size, _ptr(Xq), _ptr(qs))
+    return Xq, qs
+
+
+def llmint8_quant_weight(W, idx):
+    W = f32(W)
+    N, K = W.shape
+    idx = _c(idx, np.int32)
+    Wq = np.empty((N, K), np.int8)
+    qs = np.empty(N, np.float32)
+    lib().or_llmint8_quant_weight(_ptr(W), N, K, _ptr(idx), idx.size, _ptr(Wq), _ptr(qs))
+    return Wq, qs
+
+
+def llmint8_combine(acc, qs_x, qs_w, X, W, idx, rows=None):
+    acc = _c(acc, np.int64)
+    X, W = f32(X), f32(W)
+    M, K = X.shape
+    N = W.shape[0]
+    idx = _c(idx, np.int32)
+    n_rows = acc.shape[0]
+    r0 = 0 if rows is None else rows[0]
+    y = np.empty((n_rows, N), np.float64)
+    lib().or_llmint8_combine(_ptr(acc), r0, r0 + n_rows, N, K, _ptr(_c(qs_x, np.float32)),
+                             _ptr(_c(qs_w, np.float32)), _ptr(X), K, _ptr(W), _ptr(idx), idx.size, _ptr(y))
+    return y
+
+
+def llmint8_matmul(X, W, thr=6.0, min_ratio=0.0, rows=None):
+    """Whole decomposition: returns (y fp64, idx, Xq, qs_x, Wq, qs_w)."""
+    idx = llmint8_outliers(X, thr, min_ratio)
+    Xq, qs_x = llmint8_quant_rows(X, idx)
+    Wq, qs_w = llmint8_quant_weight(W, idx)
+    acc = gemm_i8(Xq, Wq, rows)
+    y = llmint8_combine(acc, qs_x, qs_w, X, W, idx, rows)
+    return y, idx, Xq, qs_x, Wq, qs_w

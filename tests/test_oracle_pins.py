@@ -1,0 +1,416 @@
+"""Pins for the CPU oracle: it is checked against what the pages and the
+mathematics fix, never against itself or the GPU path.
+
+Each test names the fact it pins. A plausible slip in the oracle (a dropped
+clamp, a transposed fold, a wrong rounding mode, a wrong comparison) fails at
+least one of them.
+"""
+import itertools
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _load(name):
+    with open(os.path.join(GOLD, name)) as f:
+        return json.load(f)
+
+
+# ------------------------------------------------------------------ a3 pins
+def test_closed_form_scales(orc):
+    """"大语言模型量化技术（四）：SmoothQuant", section 缩放因子: closed forms of
+    s_j = x^a / w^(1-a) at powers of two, including a = 0 and a = 1."""
+    for c in _load("closed_forms_scale.json")["cases"]:
+        s = orc.smooth_scales([c["x"]], [c["w"]], c["alpha"])
+        assert s[0] == np.float32(c["s"]), c
+
+
+def test_worked_example(orc):
+    """Same page, section 缩放的效果: the two-channel example. s_A = 100,
+    s_B ~ 7.07; a value 0.4 in channel B quantises to 1 before smoothing and
+    to 7 after; the error drops from 0.387 to about 0.010 (about 2.5%)."""
+    g = _load("worked_example_wangyu.json")
+    p = g["printed"]
+    s = orc.smooth_scales(g["x_max"], g["w_max"], g["alpha"])
+    assert s[0] == np.float32(100.0)
+    assert abs(s[1] - p["s_B"]) < 5e-3
+    # an activation tensor whose channel maxima are 100 and 0.5, holding 0.4
+    X = np.array([[100.0, 0.5], [0.0, 0.4]], np.float32)
+    Xq, qs = orc.quantize_act(X, None, per_token=False)
+    assert abs(1.0 / qs[0] - p["delta_before"]) < 5e-4
+    assert Xq[1, 1] == p["q_before"]
+    deq = Xq[1, 1] / qs[0]
+    assert abs(deq - p["dequant_before"]) < 5e-4
+    assert abs(deq - 0.4 - p["abs_error_before"]) < 5e-4
+    Xq2, qs2 = orc.quantize_act(X, s, per_token=False)
+    assert abs(1.0 / qs2[0] - p["delta_after"]) < 5e-6
+    assert Xq2[1, 1] == p["q_after"]
+    deq2 = Xq2[1, 1] / qs2[0] * s[1]
+    assert abs(deq2 - p["dequant_after"]) < 1e-3
+    assert abs(deq2 - 0.4) == pytest.approx(p["abs_error_after"], abs=5e-4)
+    assert 100 * abs(deq2 - 0.4) / 0.4 == pytest.approx(p["rel_error_after_percent"], abs=0.1)
+    # the smoothed channel B maximum equals the smoothed weight maximum
+    assert abs(0.5 / s[1] - p["channel_B_max_after"]) < 5e-4
+    assert abs(s[1] * 0.01 - p["channel_B_max_after"]) < 5e-4
+
+
+def test_clamps(orc):
+    """lpnh.cn SmoothQuant article §3.2: clamp(min=1e-5) on both statistics and
+    on s. A zero statistic must not produce 0, inf or nan."""
+    s = orc.smooth_scales([0.0, 1e-5, 1e-7, 4.0], [1e5, 0.0, 4.0, 0.0], 0.5)
+    assert np.all(np.isfinite(s)) and np.all(s >= np.float32(1e-5))
+    assert s[0] == np.float32(1e-5)  # sqrt(1e-5 / 1e5) = 1e-5 exactly at the clamp
+    assert s[1] == np.float32(1.0)   # both clamped to 1e-5
+    # x = 4, w clamped to 1e-5: sqrt(4 / 1e-5)
+    assert s[3] == np.float32(np.sqrt(np.float64(np.float32(4.0)) / np.float64(np.float32(1e-5))))
+
+
+def test_balance_alpha_half(orc):
+    """Section 缩放因子: at a = 0.5 the smoothed maxima match,
+    x_j / s_j = s_j * w_j (to fp32 rounding of s)."""
+    rng = np.random.default_rng(3)
+    x = (rng.random(4096) * 300 + 1e-3).astype(np.float32)
+    w = (rng.random(4096) * 0.2 + 1e-4).astype(np.float32)
+    s = orc.smooth_scales(x, w, 0.5).astype(np.float64)
+    a = x.astype(np.float64) / s
+    b = s * w.astype(np.float64)
+    assert np.max(np.abs(a - b) / b) < 4 * 2.0 ** -24
+
+
+def test_power_law_general_alpha(orc):
+    """s_j against an independent evaluation of the formula through logs
+    (exp(a ln x - (1-a) ln w)), relative 1e-6, for a in {0.4, 0.6}."""
+    rng = np.random.default_rng(4)
+    x = (rng.random(2000) * 100 + 1e-2).astype(np.float32)
+    w = (rng.random(2000) * 0.1 + 1e-3).astype(np.float32)
+    for a in (0.4, 0.6, 0.75):
+        s = orc.smooth_scales(x, w, a).astype(np.float64)
+        ref = np.exp(a * np.log(x.astype(np.float64)) - (1 - a) * np.log(w.astype(np.float64)))
+        assert np.max(np.abs(s - ref) / ref) < 1e-6
+
+
+# ------------------------------------------------------------------ fold pins
+def test_equivalence_identity_fp64(orc):
+    """"SmoothQuant 的原理": Y = XW = (X S^-1)(S W), exact in the reals. In fp64
+    with the oracle's own fold (input channel j of W times s_j) the two
+    products agree to 1e-12 relative (max-norm)."""
+    rng = np.random.default_rng(5)
+    M, K, N = 24, 96, 40
+    X = rng.normal(size=(M, K))
+    X[:, 3] *= 80.0
+    W = rng.normal(scale=0.02, size=(N, K))
+    x = np.abs(X).max(0).astype(np.float32)
+    w = np.abs(W).max(0).astype(np.float32)
+    for a in (0.4, 0.5, 0.6):
+        s = orc.smooth_scales(x, w, a).astype(np.float64)
+        Wp = orc.fold_weight(W, s, round_f32=False)
+        Y = X @ W.T
+        Y2 = (X / s) @ Wp.T
+        assert np.max(np.abs(Y2 - Y)) / np.max(np.abs(Y)) < 1e-12
+    # a fold along the wrong axis breaks the identity (the test has power)
+    Wbad = W * s[:N, None] if N <= K else None
+    assert np.max(np.abs((X / s) @ Wbad.T - Y)) / np.max(np.abs(Y)) > 1e-3
+
+
+def test_fold_f32_is_one_rounding(orc):
+    """The fp32 fold is the fp32 product: fp64 product of two fp32 values is
+    exact, so rounding it once equals the IEEE fp32 multiply."""
+    rng = np.random.default_rng(6)
+    W = rng.normal(scale=0.02, size=(17, 33)).astype(np.float32)
+    s = (rng.random(33) * 10).astype(np.float32)
+    Wp = orc.fold_weight(W, s, round_f32=True)
+    assert np.array_equal(Wp, (W * s[None, :]).astype(np.float32))
+
+
+def test_norm_fold_identity_fp64(orc):
+    """"融入 LayerNorm": with gamma' = gamma/s and beta' = beta/s the norm output
+    is y/s (fp64, 1e-12), for LayerNorm and RMSNorm."""
+    rng = np.random.default_rng(7)
+    M, K = 8, 256
+    H = rng.normal(size=(M, K))
+    H[:, 5] *= 50
+    gamma = 1 + 0.1 * rng.normal(size=K)
+    beta = 0.1 * rng.normal(size=K)
+    s = (rng.random(K) * 20 + 0.05)
+    gp, bp = orc.fold_norm(gamma, beta, s, round_f32=False)
+    for norm, b, bpp in ((orc.LAYERNORM, beta, bp), (orc.RMSNORM, None, None)):
+        V = orc.norm_f64(H, norm, gamma, b, 1e-5)
+        V2 = orc.norm_f64(H, norm, gp, bpp, 1e-5)
+        assert np.max(np.abs(V2 - V / s)) / np.max(np.abs(V / s)) < 1e-12
+
+
+# ------------------------------------------------------------------ norm pins
+@pytest.mark.parametrize("K", [1024, 7168, 1000, 8])
+def test_norm_fp32_matches_fp64(orc, K):
+    """The fp32 fused path (fixed reduction order) agrees with the fp64 norm
+    to 1e-6 relative per row, LayerNorm and RMSNorm."""
+    rng = np.random.default_rng(K)
+    M = 6
+    H = rng.normal(size=(M, K)).astype(np.float32)
+    H[:, min(3, K - 1)] *= 60
+    gamma = (1 + 0.1 * rng.normal(size=K)).astype(np.float32)
+    beta = (0.1 * rng.normal(size=K)).astype(np.float32)
+    for norm, b, eps in ((orc.LAYERNORM, beta, 1e-5), (orc.RMSNORM, None, 1e-6)):
+        r = orc.norm_smooth_quant(H, norm, gamma, b, eps, quantize=False, want_v=True)
+        V64 = orc.norm_f64(H, norm, gamma, b, eps)
+        err = np.max(np.abs(r["V"] - V64), axis=1) / np.max(np.abs(V64), axis=1)
+        assert np.all(err < 1e-6), err
+
+
+def test_norm_special_rows(orc):
+    """Closed forms: an alternating row +-c has mean 0 and variance c^2, so
+    LayerNorm gives +-1/sqrt(1 + eps/c^2) (times gamma, plus beta); a
+    constant row c gives RMSNorm c/sqrt(c^2 + eps)."""
+    K = 512
+    c = 3.0
+    row = np.tile([c, -c], K // 2).astype(np.float32)
+    gamma = np.full(K, 2.0, np.float32)
+    beta = np.full(K, 0.5, np.float32)
+    r = orc.norm_smooth_quant(row[None], orc.LAYERNORM, gamma, beta, 1e-5, quantize=False, want_v=True)
+    expect = np.sign(row) * 2.0 / np.sqrt(1 + 1e-5 / c ** 2) + 0.5
+    assert np.max(np.abs(r["V"][0] - expect)) < 1e-6
+    const = np.full(K, -c, np.float32)
+    r = orc.norm_smooth_quant(const[None], orc.RMSNORM, gamma, None, 1e-6, quantize=False, want_v=True)
+    assert np.max(np.abs(r["V"][0] - (-c) * 2.0 / np.sqrt(c * c + 1e-6))) < 1e-6
+
+
+def test_norm_quant_per_token_scale(orc):
+    """Per-token quantisation of the norm output: the largest |v| of every
+    row maps to +-127 and qs = 127 / max|v| ("8位量化" §2.1)."""
+    rng = np.random.default_rng(8)
+    H = rng.normal(size=(16, 256)).astype(np.float32)
+    gamma = (1 + 0.1 * rng.normal(size=256)).astype(np.float32)
+    r = orc.norm_smooth_quant(H, orc.RMSNORM, gamma, None, 1e-6, want_v=True)
+    for i in range(16):
+        m = np.max(np.abs(r["V"][i]))
+        assert r["qs"][i] == np.float32(127.0) / np.float32(m)
+        assert np.max(np.abs(r["Xq"][i].astype(np.int32))) == 127
+
+
+def test_norm_absmax_calibration(orc):
+    """Calibration mode keeps a running per-channel max of |v| across batches."""
+    rng = np.random.default_rng(9)
+    gamma = np.ones(64, np.float32)
+    am = np.zeros(64, np.float32)
+    Vs = []
+    for b in range(3):
+        H = rng.normal(size=(5, 64)).astype(np.float32)
+        r = orc.norm_smooth_quant(H, orc.RMSNORM, gamma, None, 1e-6, quantize=False, absmax=am,
+                                  want_v=True)
+        am = r["absmax"]
+        Vs.append(r["V"])
+    assert np.array_equal(am, np.abs(np.concatenate(Vs)).max(0))
+
+
+# ------------------------------------------------------------------ quant pins
+def test_round_half_even_and_clip(orc):
+    """"8位量化" §2.1: q = clip(round(x * scale), -127, 127) with numpy's
+    round (half to even)."""
+    X = np.array([[2.5, -2.5, 3.5, 0.5, 1.5, -0.5, 127.4, 200.0, -300.0, 126.5]], np.float32)
+    Xq, qs = orc.quantize_act(X, None, per_token=False, static_qs=1.0)
+    assert Xq.tolist() == [[2, -2, 4, 0, 2, 0, 127, 127, -127, 126]]
+    assert qs[0] == 1.0
+    # per token: the row max maps to 127; 63.5 ties to 64
+    Xq, qs = orc.quantize_act(np.array([[127.0, 63.5, -0.5]], np.float32), None, per_token=True)
+    assert qs[0] == 1.0 and Xq.tolist() == [[127, 64, 0]]
+
+
+def test_zero_row_scale_floor(orc):
+    """An all-zero row takes the 1e-8 floor of quantize_vectorwise and gives 0."""
+    Xq, qs = orc.quantize_act(np.zeros((2, 16), np.float32), None, per_token=True)
+    assert np.all(Xq == 0) and np.all(qs == np.float32(127.0) / np.float32(1e-8))
+
+
+def test_weight_quant_group_scaling_invariance(orc):
+    """"缩放的代价": relative quantisation error is unchanged when a whole
+    quantisation group is scaled. With per-output-channel groups and power of
+    two factors, codes are identical and scales divide exactly."""
+    rng = np.random.default_rng(10)
+    W = rng.normal(scale=0.02, size=(32, 128)).astype(np.float32)
+    f = (2.0 ** rng.integers(-6, 7, size=32)).astype(np.float32)
+    Wq, qs = orc.quantize_weight(W, per_channel=True)
+    Wq2, qs2 = orc.quantize_weight(W * f[:, None], per_channel=True)
+    assert np.array_equal(Wq, Wq2)
+    assert np.array_equal(qs2, (qs / f).astype(np.float32))
+    e1 = np.abs(W - Wq / qs[:, None]).max(1) / np.abs(W).max(1)
+    e2 = np.abs(W * f[:, None] - Wq2 / qs2[:, None]).max(1) / np.abs(W * f[:, None]).max(1)
+    assert np.allclose(e1, e2, rtol=1e-6)
+
+
+def test_weight_quant_per_tensor(orc):
+    W = np.array([[0.5, -1.0], [0.25, 2.0]], np.float32)
+    Wq, qs = orc.quantize_weight(W, per_channel=False)
+    assert qs[0] == np.float32(63.5)
+    assert Wq.tolist() == [[32, -64], [16, 127]]  # 31.75 -> 32, 15.875 -> 16
+
+
+# ------------------------------------------------------------------ GEMM pins
+def test_gemm_bruteforce_random(orc):
+    rng = np.random.default_rng(11)
+    for (M, N, K) in [(1, 1, 1), (3, 5, 7), (17, 9, 64), (33, 40, 130)]:
+        X = rng.integers(-127, 128, size=(M, K)).astype(np.int8)
+        W = rng.integers(-127, 128, size=(N, K)).astype(np.int8)
+        ref = X.astype(np.int64) @ W.astype(np.int64).T
+        assert np.array_equal(orc.gemm_i8(X, W), ref)
+        r = orc.gemm_i8(X, W, rows=(M // 2, M))
+        assert np.array_equal(r, ref[M // 2:])
+
+
+@pytest.mark.parametrize("K", [1, 2, 3])
+def test_gemm_exhaustive_small_k(orc, K):
+    vals = [-127, -1, 0, 1, 127]
+    rows = np.array(list(itertools.product(vals, repeat=K)), np.int8)
+    acc = orc.gemm_i8(rows, rows)
+    ref = np.array([[sum(int(a) * int(b) for a, b in zip(r1, r2)) for r2 in rows] for r1 in rows])
+    assert np.array_equal(acc, ref)
+
+
+def test_gemm_no_overflow_bound(orc):
+    """"8位量化" §2.1: int32 accumulation does not overflow. |acc| <= 127^2 K;
+    at the largest K here (49152) all-127 operands give exactly 792,772,608."""
+    K = 49152
+    X = np.full((2, K), 127, np.int8)
+    X[1] = -127
+    W = np.full((1, K), 127, np.int8)
+    acc = orc.gemm_i8(X, W)
+    assert acc[0, 0] == 792_772_608 and acc[1, 0] == -792_772_608
+    assert abs(int(acc[0, 0])) < 2 ** 31
+    assert 127 * 127 * 133_144 < 2 ** 31 < 127 * 127 * 133_145
+
+
+def test_dequant_closed_form(orc):
+    """out = acc / (c_x * c_w) + bias ("8位量化" §2.1 outer-product dequant)."""
+    acc = np.array([[127 * 127, -127 * 64]], np.int64)
+    y = orc.dequant(acc, np.array([63.5], np.float32), np.array([254.0, 127.0], np.float32),
+                    bias=np.array([0.25, -1.0], np.float32))
+    assert y[0, 0] == 16129 / (63.5 * 254) + 0.25
+    assert y[0, 1] == -127 * 64 / (63.5 * 127) - 1.0
+
+
+def test_dequant_row_and_column_scales(orc):
+    """Scales factor out only per row (token) and per column (output channel):
+    Y = diag(dX) Xq Wq^T diag(dW) ("为什么激活不能用逐通道量化")."""
+    rng = np.random.default_rng(12)
+    X = rng.integers(-127, 128, size=(5, 32)).astype(np.int8)
+    W = rng.integers(-127, 128, size=(7, 32)).astype(np.int8)
+    qx = (rng.random(5) * 10 + 1).astype(np.float32)
+    qw = (rng.random(7) * 10 + 1).astype(np.float32)
+    y = orc.dequant(orc.gemm_i8(X, W), qx, qw)
+    ref = np.diag(1 / qx.astype(np.float64)) @ (X.astype(np.float64) @ W.astype(np.float64).T) \
+        @ np.diag(1 / qw.astype(np.float64))
+    assert np.max(np.abs(y - ref) / (np.abs(ref) + 1e-30)) < 1e-14
+
+
+# ------------------------------------------------------------------ rounding pins
+def test_round_bf16_matches_torch_on_fp32(orc):
+    rng = np.random.default_rng(13)
+    v = np.concatenate([rng.normal(size=2000) * 10.0 ** rng.integers(-20, 20, size=2000),
+                        [0.0, -0.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, 3.3e38, -3.4e38]]).astype(np.float32)
+    ref = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(orc.round_bf16_bits(v.astype(np.float64)), ref)
+
+
+def test_round_fp16_matches_numpy(orc):
+    rng = np.random.default_rng(14)
+    v = np.concatenate([rng.normal(size=3000) * 10.0 ** rng.integers(-9, 5, size=3000),
+                        [0.0, -0.0, 1 + 2 ** -11, 1 + 3 * 2 ** -11, 65504.0, 65519.9, 65520.0,
+                         2 ** -25, 3 * 2 ** -26, 1e-9]])
+    ref = v.astype(np.float16).view(np.uint16)
+    assert np.array_equal(orc.round_fp16_bits(v), ref)
+
+
+# ------------------------------------------------------------------ LLM.int8 pins
+def test_outliers_bruteforce(orc):
+    """"8位量化" §2.2 split_outliers: columns where the share of |x| > alpha
+    exceeds min_ratio; §4.1: any value over the threshold marks the column."""
+    rng = np.random.default_rng(15)
+    X = rng.normal(size=(32, 40)).astype(np.float32)
+    X[3, 7] = 6.0         # not > 6.0
+    X[5, 9] = 6.00390625  # next fp16 above 6: counts
+    X[0:2, 20] = -7.0     # 2/32 = 0.0625
+    X[0:3, 30] = 9.0      # 3/32
+    X[:, 7] = np.clip(X[:, 7], -5, 5); X[3, 7] = 6.0
+    for thr, mr in [(6.0, 0.0), (6.0, 0.06), (6.0, 0.0625), (2.0, 0.1), (100.0, 0.0)]:
+        ref = [j for j in range(40) if np.mean(np.abs(X[:, j]) > thr) > mr]
+        assert orc.llmint8_outliers(X, thr, mr).tolist() == ref
+    assert 9 in orc.llmint8_outliers(X, 6.0, 0.0).tolist()
+    assert 7 not in orc.llmint8_outliers(X, 6.0, 0.0).tolist()
+    assert 20 in orc.llmint8_outliers(X, 6.0, 0.06).tolist()
+    assert 20 not in orc.llmint8_outliers(X, 6.0, 0.0625).tolist()
+
+
+def test_decomposition_identity_fp64():
+    """§2.2: X_O W_O + X_notO W_notO = X W (exact split of the inner product)."""
+    rng = np.random.default_rng(16)
+    X = rng.normal(size=(9, 50))
+    W = rng.normal(size=(50, 11))
+    O = [3, 17, 44]
+    m = np.ones(50, bool)
+    m[O] = False
+    assert np.max(np.abs(X[:, O] @ W[O] + X[:, m] @ W[m] - X @ W)) < 1e-12
+
+
+def test_llmint8_no_outliers_reduces_to_vectorwise(orc):
+    """With O empty the decomposition is the vector-wise int8 path."""
+    rng = np.random.default_rng(17)
+    X = rng.normal(size=(12, 64)).astype(np.float32)
+    W = rng.normal(scale=0.02, size=(20, 64)).astype(np.float32)
+    y, idx, Xq, qx, Wq, qw = orc.llmint8_matmul(X, W, 6.0)
+    assert idx.size == 0
+    Xq2, qx2 = orc.quantize_act(X, None, per_token=True)
+    Wq2, qw2 = orc.quantize_weight(W, per_channel=True)
+    assert np.array_equal(Xq, Xq2) and np.array_equal(Wq, Wq2)
+    assert np.array_equal(y, orc.dequant(orc.gemm_i8(Xq2, Wq2), qx2, qw2))
+
+
+def test_llmint8_planted_and_accuracy(orc):
+    """Planted outlier dims are found exactly; outlier columns are zero in both
+    int8 operands; the result is close to the exact product, and much closer
+    than plain vector-wise int8 on the same data."""
+    rng = np.random.default_rng(18)
+    M, K, N = 64, 256, 48
+    X = np.clip(rng.normal(size=(M, K)), -5.9, 5.9).astype(np.float32)
+    dims = [11, 100, 200]
+    for d in dims:
+        X[rng.permutation(M)[:16], d] = 30.0
+    W = rng.normal(scale=0.02, size=(N, K)).astype(np.float32)
+    y, idx, Xq, qx, Wq, qw = orc.llmint8_matmul(X, W, 6.0)
+    assert idx.tolist() == dims
+    assert np.all(Xq[:, dims] == 0) and np.all(Wq[:, dims] == 0)
+    ref = X.astype(np.float64) @ W.astype(np.float64).T
+    err = np.max(np.abs(y - ref)) / np.max(np.abs(ref))
+    Xv, qxv = orc.quantize_act(X, None, per_token=True)
+    Wv, qwv = orc.quantize_weight(W, per_channel=True)
+    err_v = np.max(np.abs(orc.dequant(orc.gemm_i8(Xv, Wv), qxv, qwv) - ref)) / np.max(np.abs(ref))
+    assert err < 2e-2 and err < err_v / 2
+
+
+def test_vectorwise_toy_magnitude(orc):
+    """"8位量化" §2.1 toy: X(4x8), W(8x16) from default_rng(0), X[0,3] = 40;
+    vector-wise int8 gives a relative error of order 1e-3..1e-2. A magnitude
+    check only: the page prints no tensors."""
+    rng = np.random.default_rng(0)
+    X = rng.normal(0, 1, (4, 8)).astype(np.float16)
+    W = rng.normal(0, 1, (8, 16)).astype(np.float16)
+    X[0, 3] = 40.0
+    Xq, qx = orc.quantize_act(X.astype(np.float32), None, per_token=True)
+    Wq, qw = orc.quantize_weight(W.T.astype(np.float32), per_channel=True)
+    y = orc.dequant(orc.gemm_i8(Xq, Wq), qx, qw)
+    ref = X.astype(np.float32).astype(np.float64) @ W.astype(np.float32).astype(np.float64)
+    err = np.abs(y - ref).max() / np.abs(ref).max()
+    assert 1e-4 < err < 5e-2
+
+
+def test_col_absmax_bruteforce(orc):
+    rng = np.random.default_rng(19)
+    X = rng.normal(size=(37, 29)).astype(np.float32)
+    prev = np.abs(rng.normal(size=29)).astype(np.float32) * 2
+    got = orc.col_absmax(X, prev)
+    ref = np.array([max(prev[j], max(abs(float(X[i, j])) for i in range(37))) for j in range(29)],
+                   np.float32)
+    assert np.array_equal(got, ref)
