@@ -1,0 +1,421 @@
+"""Benchmark of the SmoothQuant W8A8 linear-layer path on B200.
+
+One step = one pass of every hot-path row over one batch of synthetic input
+shaped like a Qwen3-0.6B decoder layer at 2048 tokens (hidden 1024; q/k/v
+fused 1024->4096, o 2048->1024, gate/up fused 1024->6144, down 3072->1024;
+6 activation channels x20..x100):
+  a5 norm pass producing the linear input (RMSNorm, original gamma)     x2
+  a1 calibration absmax of that input                                   x2
+  a2 weight absmax over the fused consumers                             x2
+  a3 smoothing factors, gamma' = gamma / s                              x2
+  a4 weight fold + int8 quantisation (per output channel)               x4
+  a5 fused RMSNorm + smoothing + per-token int8                         x2
+  a6 int8 GEMM + dequant epilogue to bf16                               x4
+  a7-a9 LLM.int8 decomposition of the q/k/v projection (bf16)           x1
+The step is captured once in a CUDA graph and replayed. L2 is flushed (a
+256 MB write) before every timed step, outside the timed interval; each step is
+bracketed by CUDA events on the stream it runs on.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0). With torchrun (N > 1) every rank runs its own
+replica of the step on its own GPU (no data-path collective; weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+M_TOKENS, HIDDEN = 2048, 1024
+WORKLOAD = "qwen3-0.6b-shaped decoder layer linear stack, 2048 tokens, hidden 1024, bf16 in/out, int8 GEMMs"
+METRIC = "W8A8 GEMM TOPS & tokens/s at 1 B200; % of INT8 TC peak / HBM GB/s"
+# GEMM (M, N, K) of one step: qkv, o, gate/up, down, LLM.int8 q/k/v
+GEMMS = [(2048, 4096, 1024), (2048, 1024, 2048), (2048, 6144, 1024), (2048, 1024, 3072), (2048, 4096, 1024)]
+# our kernels per call of each entry point used in the step
+LAUNCHES_PER_STEP = (2 * 1 + 2 * 1 + 2 * 1 + 2 * 2 + 4 * 1 + 2 * 1 + 4 * 1 + 5)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    Q = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.proc = None
+        self.index = index
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(index), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "20"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 8]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if "Active" in r[5 + i] and "Not" not in r[5 + i]})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ GPU arm
+class Layer:
+    """Device buffers and the step for the Qwen3-0.6B-shaped layer."""
+
+    def __init__(self, dev):
+        import torch
+
+        import w8a8_post_quantization_sq_b200 as sq
+        from w8a8_post_quantization_sq_b200 import inputs
+
+        self.sq, self.torch = sq, torch
+        d = inputs.c2_qwen3_06b(device=dev)
+        self.d = d
+        M, K = M_TOKENS, HIDDEN
+        e = lambda *s, dt=torch.float32: torch.empty(s, dtype=dt, device=dev)  # noqa: E731
+        self.h = {"attn": d["h_attn"], "mlp": d["h_mlp"]}
+        self.gamma = {"attn": d["gamma_attn"].float().contiguous(), "mlp": d["gamma_mlp"].float().contiguous()}
+        self.W = d["W"]
+        self.V = {k: e(M, K, dt=torch.bfloat16) for k in ("attn", "mlp")}
+        self.xmax = {k: e(K) for k in ("attn", "mlp")}
+        self.wmax = {k: e(K) for k in ("attn", "mlp")}
+        self.s = {k: e(K) for k in ("attn", "mlp")}
+        self.gp = {k: e(K) for k in ("attn", "mlp")}
+        self.Wq = {k: e(*self.W[k].shape, dt=torch.int8) for k in self.W}
+        self.qw = {k: e(self.W[k].shape[0]) for k in self.W}
+        self.Xq = {k: e(M, K, dt=torch.int8) for k in ("attn", "mlp")}
+        self.qx = {k: e(M) for k in ("attn", "mlp")}
+        xo, so = d["o_in"]
+        xd, sd = d["down_in"]
+        self.act_in = {"o": (xo, so), "down": (xd, sd)}
+        self.Y = {k: e(M, self.W[k].shape[0], dt=torch.bfloat16) for k in self.W}
+        self.Y["llm"] = e(M, 4096, dt=torch.bfloat16)
+        self.ws = sq.workspace(sq.SQ_OP_LLMINT8, M, 4096, K, device=dev)
+        self.ws_gemm = {k: sq.workspace(sq.SQ_OP_GEMM, M, 4096, K, device=dev) for k in ("qkv", "o", "gateup", "down")}
+        self.llm = sq.llmint8_weight_state(self.W["qkv"])
+        self.idx = e(K, dt=torch.int32)
+        self.nidx = e(1, dt=torch.int32)
+        self.gemm_events = None
+
+    def step(self, gemm_ev=None):
+        sq, d = self.sq, self.d
+        eps = d["eps"]
+        for k in ("attn", "mlp"):
+            # a5 (calibration pass) -> linear input; a1 on it
+            sq.sq_norm_smooth_quant(self.h[k], sq.SQ_RMSNORM, self.gamma[k], None, eps, True, None, None, None,
+                                    None, self.V[k])
+            self.xmax[k].zero_()
+            sq.sq_calib_absmax(self.V[k], self.xmax[k])
+        for k, w in (("attn", "qkv"), ("mlp", "gateup")):
+            self.wmax[k].zero_()
+            sq.sq_weight_absmax(self.W[w], self.wmax[k])                       # a2
+            sq.sq_smooth_scales(self.xmax[k], self.wmax[k], d["alpha"], self.s[k])  # a3
+            sq.sq_fold_norm(self.gamma[k], None, self.s[k], self.gp[k])
+        sq.sq_quantize_weight(self.W["qkv"], self.s["attn"], True, self.Wq["qkv"], self.qw["qkv"])  # a4
+        sq.sq_quantize_weight(self.W["gateup"], self.s["mlp"], True, self.Wq["gateup"], self.qw["gateup"])
+        sq.sq_quantize_weight(self.W["o"], None, True, self.Wq["o"], self.qw["o"])
+        sq.sq_quantize_weight(self.W["down"], None, True, self.Wq["down"], self.qw["down"])
+        for k in ("attn", "mlp"):                                              # a5
+            sq.sq_norm_smooth_quant(self.h[k], sq.SQ_RMSNORM, self.gp[k], None, eps, True, None, self.Xq[k],
+                                    self.qx[k], None, None)
+        plan = [("qkv", self.Xq["attn"], self.qx["attn"]), ("o", *self.act_in["o"]),
+                ("gateup", self.Xq["mlp"], self.qx["mlp"]), ("down", *self.act_in["down"])]
+        for i, (w, xq, qx) in enumerate(plan):                                 # a6
+            if gemm_ev is not None:
+                gemm_ev[i][0].record()
+            sq.sq_gemm_w8a8(xq, self.Wq[w], qx, self.qw[w], None, self.Y[w], self.ws_gemm[w])
+            if gemm_ev is not None:
+                gemm_ev[i][1].record()
+        sq.sq_llmint8_matmul(self.V["attn"], self.llm, 6.0, 0.0, self.Y["llm"], self.idx, self.nidx, self.ws)
+
+    def outputs(self):
+        return [self.Y[k] for k in ("qkv", "o", "gateup", "down", "llm")]
+
+
+def run_ours(args, rank, world, dev):
+    import torch
+    import torch.distributed as dist
+
+    torch.cuda.set_device(dev)
+    L = Layer(dev)
+    stream = torch.cuda.Stream()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        L.step()
+        L.step()
+    stream.synchronize()
+    # capture the step, with events around the GEMMs so their share is measured live
+    n_g = 4
+    # external events are re-recorded by every replay of the graph
+    gemm_ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)] for _ in range(n_g)]
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        L.step(gemm_ev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    for _ in range(max(args.warmup, 3)):
+        graph.replay()
+    torch.cuda.synchronize()
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    gemm_ms = []
+    clocks = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    time.sleep(0.05)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            ev[i][0].record(stream)
+            graph.replay()
+            ev[i][1].record(stream)
+            if i < 64:
+                stream.synchronize()
+                gemm_ms.append([gemm_ev[j][0].elapsed_time(gemm_ev[j][1]) for j in range(n_g)])
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop() if clocks else None
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = sum(step_ms)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+
+    # e2e through the public API with host buffers: H2D of the inputs, the
+    # step, D2H of every output, all inside the timed region
+    h_host = {k: L.h[k].cpu().pin_memory() for k in L.h}
+    outs = L.outputs()
+    o_host = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+    h2d = sum(v.numel() * v.element_size() for v in h_host.values())
+    d2h = sum(o.numel() * o.element_size() for o in outs)
+    e2e_steps = max(3, min(args.steps, 50))
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            for k in L.h:
+                L.h[k].copy_(h_host[k], non_blocking=True)
+            graph.replay()
+            for o, oh in zip(outs, o_host):
+                oh.copy_(o, non_blocking=True)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = torch.tensor([e0.elapsed_time(e1) / e2e_steps], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_ms = float(e2e_ms.item())
+
+    gm = np.array(gemm_ms)  # [steps, 4]
+    gemm_ops = [2.0 * m * n * k for (m, n, k) in GEMMS[:4]]
+    gemm_avg_ms = gm.mean(axis=0)
+    gemm_tops = sum(gemm_ops) / (gemm_avg_ms.sum() * 1e-3) / 1e12
+    pk, src = peaks()
+    i8_peak = 2.0 * pk["bf16_tflops"]  # dense int8 = 2 x dense bf16 (nominal 4.5 vs 2.25 PFLOP/s)
+    del graph
+    return {
+        "ms_per_step": ms_per_step, "e2e_ms": e2e_ms, "h2d": h2d, "d2h": d2h, "clocks": clk,
+        "gemm_avg_ms": gemm_avg_ms.tolist(), "gemm_tops": gemm_tops, "i8_peak": i8_peak, "peak_src": src,
+        "step_ms_median": statistics.median(step_ms),
+    }
+
+
+# ------------------------------------------------------------------ CPU arm
+def cpu_step_sample(rows):
+    """The oracle, as it stands, on the same step for `rows` tokens of the
+    workload (weights in full). Returns (seconds of weight-side work,
+    seconds of per-token work for `rows` tokens)."""
+    import torch
+
+    import oracle
+    from w8a8_post_quantization_sq_b200 import inputs
+
+    oracle.lib()
+    d = inputs.c2_qwen3_06b(device="cpu")
+    sl = slice(0, rows)
+    h = {"attn": d["h_attn"][sl], "mlp": d["h_mlp"][sl]}
+    gamma = {"attn": d["gamma_attn"].numpy(), "mlp": d["gamma_mlp"].numpy()}
+    W = {k: oracle.f32(v) for k, v in d["W"].items()}
+    t_rows = 0.0
+    t_w = 0.0
+    t0 = time.perf_counter()
+    V = {k: oracle.norm_smooth_quant(h[k], oracle.RMSNORM, gamma[k], None, d["eps"], quantize=False,
+                                     want_v=True)["V"] for k in h}
+    V16 = {k: torch.from_numpy(V[k]).to(torch.bfloat16) for k in V}
+    xmax = {k: oracle.col_absmax(V16[k]) for k in V}
+    t_rows += time.perf_counter() - t0
+    t0 = time.perf_counter()
+    s, gp = {}, {}
+    for k, w in (("attn", "qkv"), ("mlp", "gateup")):
+        wmax = oracle.col_absmax(W[w])
+        s[k] = oracle.smooth_scales(xmax[k], wmax, d["alpha"])
+        gp[k], _ = oracle.fold_norm(gamma[k], None, s[k])
+    Wq, qw = {}, {}
+    for w, k in (("qkv", "attn"), ("gateup", "mlp"), ("o", None), ("down", None)):
+        Wp = oracle.fold_weight(W[w], s[k]) if k else W[w]
+        Wq[w], qw[w] = oracle.quantize_weight(Wp, True)
+    t_w += time.perf_counter() - t0
+    t0 = time.perf_counter()
+    Xq, qx = {}, {}
+    for k in h:
+        r = oracle.norm_smooth_quant(h[k], oracle.RMSNORM, gp[k], None, d["eps"], True)
+        Xq[k], qx[k] = r["Xq"], r["qs"]
+    xo, so = d["o_in"]
+    xd, sd = d["down_in"]
+    plan = [("qkv", Xq["attn"], qx["attn"]), ("o", xo[sl].numpy(), so[sl].numpy()),
+            ("gateup", Xq["mlp"], qx["mlp"]), ("down", xd[sl].numpy(), sd[sl].numpy())]
+    for w, xq, q in plan:
+        y = oracle.dequant(oracle.gemm_i8(xq, Wq[w]), q, qw[w])
+        oracle.round_bf16_bits(y)
+    t_rows += time.perf_counter() - t0
+    # LLM.int8 of the q/k/v projection: outlier set over the sample rows,
+    # row quantisation, weight requantisation, GEMM + outlier term
+    t0 = time.perf_counter()
+    idx = oracle.llmint8_outliers(V16["attn"], 6.0, 0.0)
+    Xq8, qx8 = oracle.llmint8_quant_rows(V16["attn"], idx)
+    t_rows += time.perf_counter() - t0
+    t0 = time.perf_counter()
+    Wq8, qw8 = oracle.llmint8_quant_weight(d["W"]["qkv"], idx)
+    t_w += time.perf_counter() - t0
+    t0 = time.perf_counter()
+    y = oracle.llmint8_combine(oracle.gemm_i8(Xq8, Wq8), qx8, qw8, V16["attn"], d["W"]["qkv"], idx)
+    oracle.round_bf16_bits(y)
+    t_rows += time.perf_counter() - t0
+    return t_w, t_rows
+
+
+def cpu_baseline(rows):
+    t_w, t_rows = cpu_step_sample(rows)
+    step_s = t_w + t_rows * (M_TOKENS / rows)
+    return {"value": M_TOKENS / step_s, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{rows} of {M_TOKENS} tokens through every step (weights in full: {t_w:.2f} s; "
+                      f"token rows: {t_rows:.2f} s), extrapolated linearly in tokens",
+            "step_s": step_s}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    rows = 64
+    times = []
+    for _ in range(max(args.warmup, 0) and 1):
+        cpu_step_sample(16)
+    for _ in range(args.steps):
+        t_w, t_rows = cpu_step_sample(rows)
+        times.append(t_w + t_rows * (M_TOKENS / rows))
+    step_s = sum(times) / len(times)
+    v = M_TOKENS / step_s
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "i8", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "tokens": M_TOKENS, "hidden": HIDDEN},
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": f"each step: {rows} of {M_TOKENS} tokens, weights in full, extrapolated"},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-rows", type=int, default=256, help="token rows of the CPU baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    from w8a8_post_quantization_sq_b200 import build
+
+    if rank == 0:
+        build.build()
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+
+        torch.cuda.set_device(dev)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+        dist.barrier()
+    r = run_ours(args, rank, world, dev)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    value = M_TOKENS * world / (r["ms_per_step"] * 1e-3)
+    e2e = M_TOKENS * world / (r["e2e_ms"] * 1e-3)
+    gemm_avg_s = sum(r["gemm_avg_ms"]) * 1e-3
+    gemm_ops = sum(2.0 * m * n * k for (m, n, k) in GEMMS[:4])
+    achieved = gemm_ops / gemm_avg_s / 1e12
+    traffic = None
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": r["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "i8", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "tokens": M_TOKENS, "hidden": HIDDEN, "parallelism": f"replicas x{world}",
+                   "l2": "flushed before every timed step (256 MB write, outside the timed interval)",
+                   "graph": "one CUDA graph per step"},
+        "gemm_tops": r["gemm_tops"], "gemm_avg_us": [x * 1e3 for x in r["gemm_avg_ms"]],
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": r["i8_peak"], "unit": "TOPS",
+                     "frac": achieved / r["i8_peak"], "traffic": traffic,
+                     "kernel": "gemm_w8a8_kernel", "peak_source": f"{r['peak_src']} bf16 burst x 2 (int8 nominal ratio)"},
+        "e2e": {"value": e2e, "unit": "tokens/s", "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
+        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "clocks": r["clocks"],
+    }
+    if not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = {k: v for k, v in cpu_baseline(args.cpu_rows).items() if k != "step_s"}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,276 @@
+/*
+ * sq_api.h — C ABI of the SmoothQuant W8A8 linear-layer library for NVIDIA
+ * B200 (sm_100a), plus the LLM.int8() mixed-precision decomposition.
+ *
+ * Sources (page title, section) cited below:
+ *   [SQ-p1] lpnh.cn SmoothQuant practice article (§2.1 scale formula, §3.2
+ *           calibrate, §3.3 apply_smoothquant)
+ *   [SQ-p2] "大语言模型量化技术（四）：SmoothQuant" (wangyu.me): sections
+ *           为什么激活不能用逐通道量化, SmoothQuant 的原理, 缩放因子, 缩放的代价,
+ *           缩放的效果, 融入 LayerNorm
+ *   [SQ-p4] "如何通过 SmoothQuant 解决激活值离群点难题：实现端侧 LLM 全量化推理的关键"
+ *           (tbr8.org) §3 smooth_layer_weights, §4 deployment notes
+ *   [SQ-p5] "8位量化：异常值与混合精度分解实战" (xdnf.cn) §2.1 absmax and
+ *           vector-wise quantisation, §2.2 mixed-precision decomposition,
+ *           §2.3 threshold 6.0, §4.1 threshold semantics
+ *
+ * Conventions (all entry points)
+ *   - Pointers are DEVICE pointers owned by the caller unless stated. The
+ *     library never allocates device memory; where an operation needs scratch
+ *     it takes a caller-provided `workspace` of at least sq_workspace_size()
+ *     bytes, 256-byte aligned.
+ *   - Matrices are row-major. Activations X are [M,K] (tokens x input
+ *     channels) with row stride ldx elements. Weights are [N,K] (output x
+ *     input channel, K contiguous), the torch nn.Linear layout; the pages'
+ *     W[K,N] is its transpose. Outputs Y are [M,N] with row stride ldy.
+ *   - Every call is asynchronous on `stream` (0 = legacy default stream) and
+ *     never synchronises it, except sq_workspace_status().
+ *   - Return value: SQ_OK, or an error code with no kernel launched and no
+ *     output touched (argument errors), or SQ_ERR_CUDA if a launch failed.
+ *     sq_last_error_string() (thread-local) describes the last error.
+ *   - M == 0 (no rows) is valid and launches nothing. K == 0 and N == 0 are
+ *     rejected with SQ_ERR_UNSUPPORTED_SHAPE.
+ *   - Results are deterministic: the same inputs give bit-identical outputs
+ *     on every call, whatever the launch order of the blocks.
+ *   - The library is built for sm_100a only; calls on another device return
+ *     SQ_ERR_CUDA ("no kernel image").
+ */
+#ifndef SQ_API_H
+#define SQ_API_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SQ_API __attribute__((visibility("default")))
+#else
+#define SQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* sq_stream_t; /* a cudaStream_t */
+
+typedef enum {
+    SQ_OK = 0,
+    SQ_ERR_INVALID_ARG = 1,       /* null pointer, bad enum, negative size */
+    SQ_ERR_UNSUPPORTED_SHAPE = 2, /* size outside what the kernels handle  */
+    SQ_ERR_ALIGNMENT = 3,         /* pointer or stride not 16-byte aligned */
+    SQ_ERR_CUDA = 4,              /* a CUDA runtime/driver call failed     */
+    SQ_ERR_TIMEOUT = 5            /* a bounded device-side wait gave up    */
+} sq_status_t;
+
+typedef enum { SQ_F32 = 0, SQ_F16 = 1, SQ_BF16 = 2, SQ_I32 = 3, SQ_I8 = 4 } sq_dtype_t;
+
+typedef enum { SQ_LAYERNORM = 0, SQ_RMSNORM = 1 } sq_norm_t;
+
+typedef enum {
+    SQ_OP_GEMM = 0,           /* sq_gemm_w8a8                               */
+    SQ_OP_QUANT_ACT = 1,      /* sq_quantize_act (per-tensor dynamic)       */
+    SQ_OP_QUANT_WEIGHT = 2,   /* sq_quantize_weight (per-tensor)            */
+    SQ_OP_LLMINT8_DETECT = 3, /* sq_llmint8_detect                          */
+    SQ_OP_LLMINT8 = 4         /* sq_llmint8_matmul                          */
+} sq_op_t;
+
+/* Bytes of workspace an operation needs for the given sizes (0 if none is
+ * needed; callers may still pass one). Never fails; unknown op -> 0. */
+SQ_API size_t sq_workspace_size(sq_op_t op, int64_t M, int64_t N, int64_t K);
+
+/* Description of the last error on this host thread ("" if none). */
+SQ_API const char* sq_last_error_string(void);
+
+/* Synchronises `stream`, reads the status word that bounded device waits
+ * write into `workspace`, clears it and returns SQ_OK or SQ_ERR_TIMEOUT.
+ * Applies to workspaces passed to sq_gemm_w8a8 and sq_llmint8_matmul. */
+SQ_API sq_status_t sq_workspace_status(void* workspace, sq_stream_t stream);
+
+/* Library version as an integer (major*10000 + minor*100 + patch). */
+SQ_API int sq_version(void);
+
+/* --------------------------------------------------------------------------
+ * a1 / a2  Calibration absmax                      [SQ-p2] 缩放因子;
+ *          [SQ-p1] §3.2 (act.abs().amax over tokens; weight.abs().amax(dim=0));
+ *          [SQ-p4] §3 (max over batch and sequence; max over output dim).
+ *
+ * sq_calib_absmax:  xmax[j] = max(xmax[j], max_i |X[i,j]|)  over i < M.
+ *   Running maximum across calls: call once per calibration batch after the
+ *   caller has zero-filled xmax once. X: [M,K] of dtype dt in {F16, BF16,
+ *   F32}, row stride ldx >= K. xmax: [K] fp32, read and written.
+ * sq_weight_absmax: wmax[j] = max(wmax[j], max_n |W[n,j]|), W [N,K] (torch
+ *   layout: the max runs over output channels). For an input shared by
+ *   several linears (q/k/v, gate/up) call it on each, or on their
+ *   concatenation; the result is one scale per input channel.
+ * Requirements: X (W) 16-byte aligned; K and ldx multiples of 8 (16-bit)
+ * or 4 (fp32). NaN inputs give an unspecified result.
+ * ------------------------------------------------------------------------ */
+SQ_API sq_status_t sq_calib_absmax(const void* X, sq_dtype_t dt, int64_t M, int64_t K, int64_t ldx,
+                            float* xmax_inout, sq_stream_t stream);
+SQ_API sq_status_t sq_weight_absmax(const void* W, sq_dtype_t dt, int64_t N, int64_t K, int64_t ldw,
+                             float* wmax_inout, sq_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * a3  Smoothing factors                            [SQ-p2] 缩放因子;
+ *     [SQ-p1] §2.1, §3.2; [SQ-p4] §3.
+ *   s[j] = max(1e-5, x^alpha / w^(1-alpha)),  x = max(xmax[j], 1e-5),
+ *   w = max(wmax[j], 1e-5), evaluated in fp64 and rounded once to fp32.
+ *   alpha in [0, 1]; alpha = 0, 0.5, 1 use the closed forms 1/w, sqrt(x/w), x.
+ *   Outside [0,1] -> SQ_ERR_INVALID_ARG. xmax, wmax, s: [K] fp32.
+ * ------------------------------------------------------------------------ */
+SQ_API sq_status_t sq_smooth_scales(const float* xmax, const float* wmax, int64_t K, double alpha,
+                             float* s_out, sq_stream_t stream);
+
+/* a3 fold  W' = diag(s) W in the pages' notation: input channel k of every
+ * output row times s[k]      [SQ-p2] SmoothQuant 的原理; [SQ-p4] §3
+ * (weight.mul_(s.view(1,-1))).  W: [N,K] of dt in {F16, BF16, F32};
+ * Wp_out: [N,K] fp32 (one fp32 rounding per product). K % 8 == 0. */
+SQ_API sq_status_t sq_fold_weight(const void* W, sq_dtype_t dt, int64_t N, int64_t K, const float* s,
+                           float* Wp_out, sq_stream_t stream);
+
+/* a3 fold into the norm  gamma' = gamma / s, beta' = beta / s  (fp32 IEEE
+ * division)                  [SQ-p2] 融入 LayerNorm.
+ * beta / beta_out may both be NULL (RMSNorm). All [K] fp32. In-place
+ * (gamma_out == gamma) is allowed. */
+SQ_API sq_status_t sq_fold_norm(const float* gamma, const float* beta, const float* s, int64_t K,
+                         float* gamma_out, float* beta_out, sq_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * a4  Weight quantisation (offline)     [SQ-p5] §2.1; [SQ-p2]
+ *     为什么激活不能用逐通道量化 (weight scales per output channel).
+ *   W' = fp32(W) * s[k]  (s may be NULL: W' = fp32(W)), then
+ *   m = max |W'| over the row (per_channel != 0) or the tensor;
+ *   qs = 127 / max(m, 1e-8)  (fp32);  Wq = clip(rne(W' * qs), -127, 127).
+ *   W: [N,K] of dt in {F16, BF16, F32}. Wq: [N,K] int8. qs_w: [N] or [1].
+ *   Per-tensor needs workspace (SQ_OP_QUANT_WEIGHT). K % 16 == 0.
+ * ------------------------------------------------------------------------ */
+SQ_API sq_status_t sq_quantize_weight(const void* W, sq_dtype_t dt, int64_t N, int64_t K,
+                               const float* s, int per_channel, int8_t* Wq, float* qs_w,
+                               void* workspace, size_t ws_bytes, sq_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * a5'  Activation quantisation without a norm     [SQ-p4] §3 (input / s);
+ *      [SQ-p1] §3.3; [SQ-p5] §2.1.
+ *   v = fp32(X[i,j]) / s[j]  (IEEE division; s may be NULL: v = X),
+ *   per_token != 0: qs_x[i] = 127 / max(max_j |v[i,j]|, 1e-8);
+ *   per_token == 0: qs_x[0] = *static_qs if static_qs != NULL, else
+ *                   127 / max(max_ij |v|, 1e-8) (needs workspace);
+ *   Xq[i,j] = clip(rne(v * qs), -127, 127).
+ *   X: [M,K] dt in {F16, BF16, F32}, stride ldx. Xq: [M,K] contiguous.
+ *   K % 16 == 0.
+ * ------------------------------------------------------------------------ */
+SQ_API sq_status_t sq_quantize_act(const void* X, sq_dtype_t dt, int64_t M, int64_t K, int64_t ldx,
+                            const float* s, int per_token, const float* static_qs,
+                            int8_t* Xq, float* qs_x, void* workspace, size_t ws_bytes,
+                            sq_stream_t stream);
+
+/* Static per-tensor scale from calibration maxima: qs = 127 / max(max_j
+ * absmax[j], 1e-8), written to qs_out[0]. absmax: [n] fp32. */
+SQ_API sq_status_t sq_scale_from_absmax(const float* absmax, int64_t n, float* qs_out,
+                                 sq_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * a5  Fused norm + smoothing + int8           [SQ-p2] 融入 LayerNorm;
+ *     [SQ-p4] §4 item 2; [SQ-p5] §2.1.
+ *   LayerNorm: mu = S(x)/K, d = x - mu, var = S(d*d)/K, r = 1/sqrt(var+eps),
+ *              v = (d*r)*gamma' + beta'  (beta' may be NULL)
+ *   RMSNorm:   r = 1/sqrt(S(x*x)/K + eps),  v = (x*r)*gamma'
+ *   Every step is one correctly rounded fp32 operation. S() is a sum in a
+ *   fixed order: 128 lanes; lane t folds 8-element chunks t, t+128, ... with
+ *   fma in index order; each 32-lane group combines by the xor butterfly
+ *   (16, 8, 4, 2, 1); the four group totals add as (G0+G1)+(G2+G3).
+ *   Then, if Xq != NULL: per_token != 0 -> qs_x[i] = 127/max(max_j|v|,1e-8);
+ *   per_token == 0 -> qs = *static_qs (required), qs_x[0] = qs;
+ *   Xq = clip(rne(v*qs), -127, 127).
+ *   Optional outputs: absmax_inout [K] fp32 running max of |v| per channel
+ *   (calibration mode); V_out [M,K] (stride K) v rounded to dt.
+ *   gamma_p (and beta_p) are the folded parameters from sq_fold_norm, or the
+ *   original ones to calibrate. H: [M,K] dt in {F16, BF16}, stride ldh.
+ *   K % 8 == 0, 8 <= K <= 16384.
+ * ------------------------------------------------------------------------ */
+SQ_API sq_status_t sq_norm_smooth_quant(const void* H, sq_dtype_t dt, int64_t M, int64_t K, int64_t ldh,
+                                 sq_norm_t norm, const float* gamma_p, const float* beta_p,
+                                 float eps, int per_token, const float* static_qs,
+                                 int8_t* Xq, float* qs_x, float* absmax_inout, void* V_out,
+                                 sq_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * a6  INT8 GEMM with dequantisation epilogue   [SQ-p5] §2.1 (int32
+ *     accumulation, out / (c_x outer c_w)); [SQ-p2] 为什么激活不能用逐通道量化
+ *     (Y = diag(dX) Xq Wq diag(dW)).
+ *   acc[i,j] = sum_k Xq[i,k] * Wq[j,k]   (exact int32; |acc| <= 127^2 K)
+ *   out_dt = SQ_I32: Y = acc.
+ *   otherwise: Y = acc / (qs_x[i or 0] * qs_w[j or 0]) + bias[j], computed in
+ *   fp32 as acc * ((1/qs_x) * (1/qs_w)) (+ bias), rounded once to out_dt in
+ *   {F32, F16, BF16}. bias: [N] fp32 or NULL.
+ *   Xq: [M,K] int8 contiguous; Wq: [N,K] int8 contiguous; Y: [M,N] stride ldy.
+ *   K % 16 == 0, K <= 133144 (int32 bound); Xq, Wq 16-byte aligned.
+ *   Workspace (SQ_OP_GEMM) holds the status word of the bounded waits; zero
+ *   it once before first use.
+ * ------------------------------------------------------------------------ */
+SQ_API sq_status_t sq_gemm_w8a8(const int8_t* Xq, const int8_t* Wq, int64_t M, int64_t N, int64_t K,
+                         const float* qs_x, int x_per_token, const float* qs_w, int w_per_channel,
+                         const float* bias, sq_dtype_t out_dt, void* Y, int64_t ldy,
+                         void* workspace, size_t ws_bytes, sq_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * a7-a9  LLM.int8() mixed-precision decomposition     [SQ-p5] §2.2, §2.3,
+ *        §4.1.
+ * ------------------------------------------------------------------------ */
+
+/* a7: outlier dimensions O = { j : count_i(|X[i,j]| > threshold) / M >
+ * min_ratio } in ascending order (fp64 ratio and comparison; the threshold
+ * test is strict, in fp32). min_ratio = 0 marks a column on any single
+ * value over the threshold. X: [M,K] dt in {F16, BF16}, stride ldx.
+ * outlier_idx: [K] int32 (first *n_outliers entries valid); n_outliers: [1]
+ * int32, device. Workspace: SQ_OP_LLMINT8_DETECT. K % 8 == 0. */
+SQ_API sq_status_t sq_llmint8_detect(const void* X, sq_dtype_t dt, int64_t M, int64_t K, int64_t ldx,
+                              float threshold, double min_ratio, int32_t* outlier_idx,
+                              int32_t* n_outliers, void* workspace, size_t ws_bytes,
+                              sq_stream_t stream);
+
+/* a8: vector-wise row quantisation over the columns not in O:
+ * qs_x[i] = 127 / max(max_{j not in O} |X[i,j]|, 1e-8);
+ * Xq[i,j] = 0 for j in O, else clip(rne(X*qs), -127, 127).
+ * idx / n_idx: device outlier list (as written by sq_llmint8_detect). */
+SQ_API sq_status_t sq_llmint8_quant_rows(const void* X, sq_dtype_t dt, int64_t M, int64_t K, int64_t ldx,
+                                  const int32_t* idx, const int32_t* n_idx, int8_t* Xq,
+                                  float* qs_x, sq_stream_t stream);
+
+/* a9 weight side: vector-wise quantisation of W over the input channels not
+ * in O (one scale per output channel): qs_w[n] = 127/max(max_{k not in O}
+ * |W[n,k]|, 1e-8); Wq[n,k] = 0 for k in O. W: [N,K] dt in {F16, BF16}. */
+SQ_API sq_status_t sq_llmint8_quant_weight(const void* W, sq_dtype_t dt, int64_t N, int64_t K,
+                                    const int32_t* idx, const int32_t* n_idx, int8_t* Wq,
+                                    float* qs_w, sq_stream_t stream);
+
+/* Weight state for sq_llmint8_matmul. W is the caller's 16-bit weight [N,K]
+ * (same dtype as X). Wq [N,K] int8, qs_w [N] fp32, cached_idx [K] int32 and
+ * cached_n [1] int32 are caller-allocated device buffers that the library
+ * maintains: they hold the int8 weight for the outlier set in cached_idx.
+ * Set *cached_n = -1 (device) before the first call to mark the cache empty. */
+typedef struct {
+    const void* W;
+    int64_t N;
+    int8_t* Wq;
+    float* qs_w;
+    int32_t* cached_idx;
+    int32_t* cached_n;
+} sq_llmint8_weight_t;
+
+/* a7-a9 in one call: detect O on X; if O differs from the cached set,
+ * requantise the weight for O (on the device, no host synchronisation);
+ * quantise the rows of X; then one GEMM whose epilogue forms
+ *   Y[i,j] = acc[i,j] / (qs_x[i] * qs_w[j]) + sum_{o in O ascending} X[i,o] * W[j,o]
+ * in fp32 (the 16-bit products are exact in fp32) and rounds once to dt.
+ * X, Y: dt in {F16, BF16}; Y [M,N] stride ldy. idx_out [K], n_out [1]
+ * receive O. Workspace: SQ_OP_LLMINT8. K % 16 == 0. */
+SQ_API sq_status_t sq_llmint8_matmul(const void* X, sq_dtype_t dt, int64_t M, int64_t K, int64_t ldx,
+                              const sq_llmint8_weight_t* w, float threshold, double min_ratio,
+                              void* Y, int64_t ldy, int32_t* idx_out, int32_t* n_out,
+                              void* workspace, size_t ws_bytes, sq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SQ_API_H */

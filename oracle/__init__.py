@@ -71,6 +71,8 @@ def _declare(L):
     L.or_round_bf16.restype = ctypes.c_uint16
     L.or_round_fp16.argtypes = [_d]
     L.or_round_fp16.restype = ctypes.c_uint16
+    L.or_round_bf16_array.argtypes = [_p, _i64, _p]
+    L.or_round_fp16_array.argtypes = [_p, _i64, _p]
     L.or_llmint8_outliers.argtypes = [_p, _i64, _i64, _i64, _f, _d, _p]
     L.or_llmint8_outliers.restype = _i64
     L.or_llmint8_quant_rows.argtypes = [_p, _i64, _i64, _i64, _p, _i64, _p, _p]
@@ -218,15 +220,19 @@ def dequant(acc, qs_x, qs_w, bias=None, rows=None):
 
 
 def round_bf16_bits(y):
-    y = np.asarray(y, np.float64)
-    f = lib().or_round_bf16
-    return np.array([f(float(v)) for v in y.ravel()], np.uint16).reshape(y.shape)
+    """Bits of the bf16 nearest to each fp64 value (ties to even)."""
+    y = _c(y, np.float64)
+    out = np.empty(y.shape, np.uint16)
+    lib().or_round_bf16_array(_ptr(y), y.size, _ptr(out))
+    return out
 
 
 def round_fp16_bits(y):
-    y = np.asarray(y, np.float64)
-    f = lib().or_round_fp16
-    return np.array([f(float(v)) for v in y.ravel()], np.uint16).reshape(y.shape)
+    """Bits of the fp16 nearest to each fp64 value (ties to even)."""
+    y = _c(y, np.float64)
+    out = np.empty(y.shape, np.uint16)
+    lib().or_round_fp16_array(_ptr(y), y.size, _ptr(out))
+    return out
 
 
 # ---------------------------------------------------------------- a7-a9

@@ -409,6 +409,14 @@ uint16_t or_round_fp16(double y) {
     return sign | (uint16_t)((E + 15) << 10) | mant;
 }
 
+void or_round_bf16_array(const double* y, int64_t n, uint16_t* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = or_round_bf16(y[i]);
+}
+
+void or_round_fp16_array(const double* y, int64_t n, uint16_t* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = or_round_fp16(y[i]);
+}
+
 /* ------------------------------------------------------------------ a7
  * Outlier dimensions   [SQ-p5] §2.2 split_outliers (over = |x| > alpha;
  * ratio = over.mean(axis=0); keep ratio > min_ratio), §4.1 (any value over

@@ -87,6 +87,8 @@ void or_dequant(const int64_t* acc, int64_t r0, int64_t r1, int64_t N,
 /* Round fp64 to the nearest bf16 / fp16 (ties to even); returns the bits. */
 uint16_t or_round_bf16(double y);
 uint16_t or_round_fp16(double y);
+void or_round_bf16_array(const double* y, int64_t n, uint16_t* out);
+void or_round_fp16_array(const double* y, int64_t n, uint16_t* out);
 
 /* LLM.int8 outlier set: columns j with count_i(|X_ij| > thr) / M > min_ratio,
  * ascending. Returns |O|. */

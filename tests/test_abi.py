@@ -1,0 +1,115 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the
+public header declares, validates arguments before touching the device, and
+the product path has no route to the oracle."""
+import ctypes
+import glob
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+PKG = os.path.join(ROOT, "w8a8_post_quantization_sq_b200")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from w8a8_post_quantization_sq_b200 import build
+
+    build.build()
+    from w8a8_post_quantization_sq_b200 import _lib
+
+    return _lib.lib()
+
+
+def declared_symbols():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        txt = open(h, encoding="utf-8").read()
+        names |= set(re.findall(r"^SQ_API\s+[\w\s\*]+?\b(sq_\w+)\s*\(", txt, flags=re.M))
+    return names
+
+
+def test_header_declares_the_boundary():
+    need = {"sq_calib_absmax", "sq_weight_absmax", "sq_smooth_scales", "sq_fold_weight", "sq_fold_norm",
+            "sq_quantize_weight", "sq_quantize_act", "sq_scale_from_absmax", "sq_norm_smooth_quant",
+            "sq_gemm_w8a8", "sq_llmint8_detect", "sq_llmint8_quant_rows", "sq_llmint8_quant_weight",
+            "sq_llmint8_matmul", "sq_workspace_size", "sq_last_error_string", "sq_workspace_status",
+            "sq_version"}
+    assert need <= declared_symbols()
+
+
+def test_library_exports_every_declared_symbol(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", os.path.join(PKG, "libsq_b200.so")],
+                         capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (sq_\w+)", out))
+    missing = declared_symbols() - exported
+    assert not missing, missing
+    for name in declared_symbols():
+        assert getattr(L, name) is not None
+
+
+def test_binding_covers_every_symbol():
+    from w8a8_post_quantization_sq_b200 import _lib
+
+    assert declared_symbols() <= set(_lib.SIGNATURES)
+
+
+def test_no_oracle_in_product():
+    """The library links nothing from the oracle and the package never imports it."""
+    out = subprocess.run(["nm", "-D", os.path.join(PKG, "libsq_b200.so")], capture_output=True, text=True).stdout
+    assert "or_" not in " ".join(re.findall(r"\b[UT] (\w+)", out)).replace("error", "")
+    for f in glob.glob(os.path.join(PKG, "**", "*.py"), recursive=True):
+        src = open(f, encoding="utf-8").read()
+        assert not re.search(r"^\s*(import|from)\s+oracle\b", src, flags=re.M), f
+    for f in glob.glob(os.path.join(PKG, "csrc", "*")):
+        assert "sq_oracle" not in open(f, encoding="utf-8").read(), f
+
+
+def test_workspace_sizes(L):
+    assert L.sq_workspace_size(0, 2048, 4096, 1024) >= 256
+    det = L.sq_workspace_size(3, 2048, 0, 4096)
+    assert det >= 256 + 16 * 4096 * 4
+    full = L.sq_workspace_size(4, 2048, 16384, 4096)
+    assert full >= det + 2048 * 4096 + 2048 * 4
+    assert L.sq_workspace_size(99, 1, 1, 1) == 0
+    assert L.sq_version() >= 100
+
+
+def _expect(L, status, code, fragment):
+    assert status == code, (status, L.sq_last_error_string())
+    assert fragment in L.sq_last_error_string().decode()
+
+
+def test_argument_validation_without_gpu(L):
+    """Each check returns before any CUDA call, so these run on a CPU host."""
+    p = ctypes.c_void_p(16)  # a fake, aligned, non-null address: never dereferenced
+    odd = ctypes.c_void_p(18)
+    # null pointers
+    _expect(L, L.sq_gemm_w8a8(None, p, 16, 16, 16, p, 1, p, 1, None, 2, p, 16, p, 256, None), 1, "null")
+    # K not a multiple of 16
+    _expect(L, L.sq_gemm_w8a8(p, p, 16, 16, 24, p, 1, p, 1, None, 2, p, 16, p, 256, None), 2, "multiple of 16")
+    # K beyond the int32 bound
+    _expect(L, L.sq_gemm_w8a8(p, p, 16, 16, 133152, p, 1, p, 1, None, 2, p, 16, p, 256, None), 2, "overflow")
+    # misaligned operand
+    _expect(L, L.sq_gemm_w8a8(odd, p, 16, 16, 16, p, 1, p, 1, None, 2, p, 16, p, 256, None), 3, "aligned")
+    # missing workspace
+    _expect(L, L.sq_gemm_w8a8(p, p, 16, 16, 16, p, 1, p, 1, None, 2, p, 16, None, 0, None), 1, "workspace")
+    # norm: bad K, bad dtype, per-tensor without a static scale
+    _expect(L, L.sq_norm_smooth_quant(p, 2, 4, 12, 12, 1, p, None, 1e-6, 1, None, p, p, None, None, None), 2, "K")
+    _expect(L, L.sq_norm_smooth_quant(p, 0, 4, 16, 16, 1, p, None, 1e-6, 1, None, p, p, None, None, None), 1,
+            "dtype")
+    _expect(L, L.sq_norm_smooth_quant(p, 2, 4, 16, 16, 1, p, None, 1e-6, 0, None, p, p, None, None, None), 1,
+            "static")
+    # smoothing: alpha out of range
+    _expect(L, L.sq_smooth_scales(p, p, 16, 1.5, p, None), 1, "alpha")
+    # absmax: stride smaller than K
+    _expect(L, L.sq_calib_absmax(p, 2, 4, 16, 8, p, None), 2, "sizes")
+    # quantize_act: dynamic per-tensor without workspace
+    _expect(L, L.sq_quantize_act(p, 2, 4, 16, 16, None, 0, None, p, p, None, 0, None), 1, "workspace")
+    # llmint8: workspace too small
+    _expect(L, L.sq_llmint8_detect(p, 1, 256, 64, 64, 6.0, 0.0, p, p, p, 16, None), 1, "workspace")
+    # M == 0 is a valid empty call (nothing launched)
+    assert L.sq_gemm_w8a8(p, p, 0, 16, 16, p, 1, p, 1, None, 2, p, 16, p, 256, None) == 0
+    assert L.sq_calib_absmax(p, 2, 0, 16, 16, p, None) == 0

@@ -1,0 +1,508 @@
+"""GPU parity: every hot-path step through the C ABI against the CPU oracle.
+
+Bit-exact for int8 codes, scales, int32 accumulators, calibration maxima,
+smoothing factors and outlier sets. Dequantised outputs:
+  fp32  |gpu - y| <= 1e-6 * (|acc/(qx qw)| + |h| + |bias|)   (y = oracle fp64)
+  16-bit  within 1 ulp of RN16(y), plus the same fp32 allowance where terms
+          cancel (bias or the LLM.int8 outlier term).
+The fp32 epilogue computes acc * ((1/qx) * (1/qw)) with four roundings, at most
+about 3e-7 relative, so 1e-6 is the bound the arithmetic gives.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import w8a8_post_quantization_sq_b200 as sq
+from w8a8_post_quantization_sq_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _setup():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    sq.lib()
+    oracle.lib()
+
+
+def npf(t):
+    return t.detach().to("cpu", torch.float32).numpy()
+
+
+def npu16(t):
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def ord16(bits):
+    b = bits.astype(np.int64)
+    return np.where(b & 0x8000, -(b & 0x7FFF), b)
+
+
+def ulp16(bits, dtype):
+    """Spacing of the 16-bit grid at each value (bits of a finite value)."""
+    v = torch.from_numpy(bits.view(np.int16)).view(dtype).double().numpy()
+    nxt = torch.from_numpy((bits.astype(np.int32) + 1).astype(np.uint16).view(np.int16)).view(dtype).double().numpy()
+    return np.abs(nxt - v)
+
+
+def assert_close_16(got, y, dtype, terms=None):
+    """got: torch 16-bit tensor; y: oracle fp64; terms: sum of |terms| (fp64)."""
+    gb = npu16(got)
+    rb = oracle.round_bf16_bits(y) if dtype == torch.bfloat16 else oracle.round_fp16_bits(y)
+    d = np.abs(ord16(gb) - ord16(rb))
+    ok = d <= 1
+    if terms is not None:
+        g = npf(got).astype(np.float64)
+        ok |= np.abs(g - y) <= ulp16(rb, dtype) + 2.0 ** -20 * terms
+    bad = np.argwhere(~ok)
+    assert bad.size == 0, f"{bad.shape[0]} outputs beyond tolerance, first {bad[:5].tolist()} d={d[~ok][:5]}"
+
+
+def assert_close_f32(got, y, terms):
+    g = npf(got).astype(np.float64)
+    err = np.abs(g - y)
+    bad = err > 1e-6 * terms
+    assert not bad.any(), f"max rel {np.max(err / np.maximum(terms, 1e-300))}"
+
+
+def rnd(shape, seed, dtype=torch.float32, scale=1.0):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(shape, generator=g) * scale).to(dtype)
+
+
+# ---------------------------------------------------------------- a1 / a2
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("M,K", [(1, 8), (37, 1000), (300, 2056), (1029, 4104)])
+def test_calib_absmax(dtype, M, K):
+    if dtype == torch.float32 and K % 4:
+        pytest.skip()
+    X1 = rnd((M, K), 1, dtype, 3.0)
+    X2 = rnd((M + 5, K), 2, dtype, 3.0)
+    X2[:, K // 3] *= 100
+    xmax = torch.zeros(K, device=DEV)
+    sq.sq_calib_absmax(X1.to(DEV), xmax)
+    sq.sq_calib_absmax(X2.to(DEV), xmax)
+    ref = oracle.col_absmax(X2, oracle.col_absmax(X1))
+    assert np.array_equal(npf(xmax), ref)
+
+
+def test_calib_absmax_strided_and_weight():
+    X = rnd((64, 1024), 3, torch.bfloat16)
+    view = X.to(DEV)[:, 256:768]  # ld = 1024, K = 512
+    xmax = torch.zeros(512, device=DEV)
+    sq.sq_calib_absmax(view, xmax)
+    assert np.array_equal(npf(xmax), oracle.col_absmax(X[:, 256:768]))
+    W = rnd((3000, 520), 4, torch.float32, 0.02)
+    wmax = torch.zeros(520, device=DEV)
+    sq.sq_weight_absmax(W.to(DEV), wmax)
+    assert np.array_equal(npf(wmax), oracle.col_absmax(W))
+
+
+# ---------------------------------------------------------------- a3
+@pytest.mark.parametrize("alpha", [0.0, 0.4, 0.5, 0.6, 0.75, 1.0])
+def test_smooth_scales(alpha):
+    K = 12288
+    g = torch.Generator().manual_seed(5)
+    x = torch.rand(K, generator=g) * 200
+    w = torch.rand(K, generator=g) * 0.3
+    x[:7] = torch.tensor([0.0, 1e-7, 1e-5, 1.0, 4.0, 100.0, 32.0])
+    w[:7] = torch.tensor([0.0, 1.0, 1e-5, 0.0, 4.0, 0.01, 32.0])
+    s = torch.empty(K, device=DEV)
+    sq.sq_smooth_scales(x.to(DEV), w.to(DEV), alpha, s)
+    ref = oracle.smooth_scales(x, w, alpha)
+    got = npf(s)
+    mism = np.nonzero(got != ref)[0]
+    assert mism.size == 0, f"alpha={alpha}: {mism.size} mismatches, e.g. {mism[:3]} {got[mism[:3]]} {ref[mism[:3]]}"
+
+
+def test_fold_weight_and_norm():
+    N, K = 333, 1032
+    for dtype in (torch.float16, torch.bfloat16, torch.float32):
+        W = rnd((N, K), 6, dtype, 0.03)
+        s = (torch.rand(K, generator=torch.Generator().manual_seed(7)) * 20 + 0.01)
+        Wp = torch.empty((N, K), device=DEV)
+        sq.sq_fold_weight(W.to(DEV), s.to(DEV), Wp)
+        assert np.array_equal(npf(Wp), oracle.fold_weight(W.float().numpy(), s.numpy(), round_f32=True))
+    gamma = 1 + 0.1 * rnd(K, 8)
+    beta = 0.1 * rnd(K, 9)
+    go = torch.empty(K, device=DEV)
+    bo = torch.empty(K, device=DEV)
+    sq.sq_fold_norm(gamma.to(DEV), beta.to(DEV), s.to(DEV), go, bo)
+    rg, rb = oracle.fold_norm(gamma.numpy(), beta.numpy(), s.numpy(), round_f32=True)
+    assert np.array_equal(npf(go), rg) and np.array_equal(npf(bo), rb)
+
+
+# ---------------------------------------------------------------- a4
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("per_channel", [True, False])
+@pytest.mark.parametrize("with_s", [True, False])
+def test_quantize_weight(dtype, per_channel, with_s):
+    N, K = 517, 2064
+    W = rnd((N, K), 10, dtype, 0.02)
+    s = torch.rand(K, generator=torch.Generator().manual_seed(11)) * 30 + 0.05 if with_s else None
+    Wq = torch.empty((N, K), dtype=torch.int8, device=DEV)
+    qs = torch.empty(N if per_channel else 1, device=DEV)
+    ws = sq.workspace(sq.SQ_OP_QUANT_WEIGHT, 0, N, K)
+    sq.sq_quantize_weight(W.to(DEV), None if s is None else s.to(DEV), per_channel, Wq, qs, ws)
+    Wp = oracle.fold_weight(W.float().numpy(), s.numpy(), True) if with_s else W.float().numpy()
+    rq, rs = oracle.quantize_weight(Wp, per_channel)
+    assert np.array_equal(npf(qs), rs)
+    assert np.array_equal(Wq.cpu().numpy(), rq)
+
+
+# ---------------------------------------------------------------- a5'
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("mode", ["token", "tensor_dynamic", "tensor_static"])
+def test_quantize_act(dtype, mode):
+    M, K = 77, 1040
+    X = rnd((M, K), 12, dtype)
+    X[:, 5] *= 50
+    s = torch.rand(K, generator=torch.Generator().manual_seed(13)) * 8 + 0.1
+    per_token = mode == "token"
+    static = torch.tensor([3.7]) if mode == "tensor_static" else None
+    Xq = torch.empty((M, K), dtype=torch.int8, device=DEV)
+    qs = torch.empty(M if per_token else 1, device=DEV)
+    ws = sq.workspace(sq.SQ_OP_QUANT_ACT, M, 0, K)
+    sq.sq_quantize_act(X.to(DEV), s.to(DEV), per_token, None if static is None else static.to(DEV), Xq, qs, ws)
+    rq, rs = oracle.quantize_act(X, s.numpy(), per_token, None if static is None else 3.7)
+    assert np.array_equal(npf(qs), rs)
+    assert np.array_equal(Xq.cpu().numpy(), rq)
+
+
+def test_quantize_act_config1_worked_path():
+    """Single linear, p4 toy shapes: X [16,1024] ch0 x50, per-tensor, s from X itself."""
+    d = inputs.c1_single_linear()
+    X, W = d["X"], d["W"]
+    xmax = torch.zeros(1024, device=DEV)
+    wmax = torch.zeros(1024, device=DEV)
+    sq.sq_calib_absmax(X.to(DEV), xmax)
+    sq.sq_weight_absmax(W.to(DEV), wmax)
+    s = torch.empty(1024, device=DEV)
+    sq.sq_smooth_scales(xmax, wmax, 0.5, s)
+    rs = oracle.smooth_scales(oracle.col_absmax(X), oracle.col_absmax(W), 0.5)
+    assert np.array_equal(npf(s), rs)
+    Xq = torch.empty((16, 1024), dtype=torch.int8, device=DEV)
+    qx = torch.empty(1, device=DEV)
+    ws = sq.workspace(sq.SQ_OP_QUANT_ACT, 16, 0, 1024)
+    sq.sq_quantize_act(X.to(DEV), s, False, None, Xq, qx, ws)
+    rq, rqs = oracle.quantize_act(X, rs, False)
+    assert np.array_equal(Xq.cpu().numpy(), rq) and np.array_equal(npf(qx), rqs)
+
+
+# ---------------------------------------------------------------- a5
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("norm", ["ln", "rms"])
+@pytest.mark.parametrize("K", [8, 1000, 1024, 3072, 7168, 12288, 16384])
+def test_norm_smooth_quant_per_token(dtype, norm, K):
+    M = 37 if K >= 7168 else 129
+    H = rnd((M, K), K, dtype)
+    H[:, K // 5] *= 60
+    gamma = 1 + 0.1 * rnd(K, 1)
+    beta = 0.1 * rnd(K, 2) if norm == "ln" else None
+    eps = 1e-5 if norm == "ln" else 1e-6
+    nt = sq.SQ_LAYERNORM if norm == "ln" else sq.SQ_RMSNORM
+    Xq = torch.empty((M, K), dtype=torch.int8, device=DEV)
+    qs = torch.empty(M, device=DEV)
+    V = torch.empty((M, K), dtype=dtype, device=DEV)
+    sq.sq_norm_smooth_quant(H.to(DEV), nt, gamma.to(DEV), None if beta is None else beta.to(DEV), eps, True, None,
+                            Xq, qs, None, V)
+    r = oracle.norm_smooth_quant(H, oracle.LAYERNORM if norm == "ln" else oracle.RMSNORM, gamma.numpy(),
+                                 None if beta is None else beta.numpy(), eps, True, want_v=True)
+    assert np.array_equal(npf(qs), r["qs"])
+    assert np.array_equal(Xq.cpu().numpy(), r["Xq"])
+    assert np.array_equal(npu16(V), npu16(torch.from_numpy(r["V"]).to(dtype)))
+
+
+@pytest.mark.parametrize("norm", ["ln", "rms"])
+def test_norm_static_and_calibration(norm):
+    """Calibration mode (running per-channel max of |v| over batches) and the
+    static per-tensor scale taken from it, the OPT-30B-style path."""
+    M, K = 200, 7168
+    nt = sq.SQ_LAYERNORM if norm == "ln" else sq.SQ_RMSNORM
+    on = oracle.LAYERNORM if norm == "ln" else oracle.RMSNORM
+    gamma = 1 + 0.1 * rnd(K, 3)
+    beta = 0.1 * rnd(K, 4) if norm == "ln" else None
+    am = torch.zeros(K, device=DEV)
+    ram = np.zeros(K, np.float32)
+    for b in range(3):
+        H = rnd((M, K), 20 + b, torch.float16)
+        H[:, 11] *= 60
+        sq.sq_norm_smooth_quant(H.to(DEV), nt, gamma.to(DEV), None if beta is None else beta.to(DEV), 1e-5, True,
+                                None, None, None, am, None)
+        ram = oracle.norm_smooth_quant(H, on, gamma.numpy(), None if beta is None else beta.numpy(), 1e-5,
+                                       quantize=False, absmax=ram)["absmax"]
+    assert np.array_equal(npf(am), ram)
+    qs_static = torch.empty(1, device=DEV)
+    sq.sq_scale_from_absmax(am, qs_static)
+    rqs = oracle.scale_from_absmax(ram)
+    assert npf(qs_static)[0] == rqs
+    H = rnd((M, K), 99, torch.float16, 1.3)  # values beyond the calibrated range clip
+    H[:, 11] *= 80
+    Xq = torch.empty((M, K), dtype=torch.int8, device=DEV)
+    qx = torch.empty(1, device=DEV)
+    sq.sq_norm_smooth_quant(H.to(DEV), nt, gamma.to(DEV), None if beta is None else beta.to(DEV), 1e-5, False,
+                            qs_static, Xq, qx, None, None)
+    r = oracle.norm_smooth_quant(H, on, gamma.numpy(), None if beta is None else beta.numpy(), 1e-5,
+                                 per_token=False, static_qs=float(rqs))
+    assert np.array_equal(Xq.cpu().numpy(), r["Xq"])
+    assert npf(qx)[0] == rqs
+
+
+# ---------------------------------------------------------------- a6
+GEMM_SHAPES = [(1, 16, 16), (16, 1024, 1024), (200, 300, 272), (257, 513, 1040), (128, 256, 128),
+               (640, 2048, 384), (129, 4096, 1024)]
+
+
+def rand_i8(shape, seed):
+    g = torch.Generator().manual_seed(seed)
+    return torch.randint(-127, 128, shape, generator=g, dtype=torch.int32).to(torch.int8)
+
+
+@pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
+def test_gemm_int32_exact(M, N, K):
+    Xq, Wq = rand_i8((M, K), M + 1), rand_i8((N, K), N + 2)
+    Y = torch.empty((M, N), dtype=torch.int32, device=DEV)
+    ws = sq.workspace(sq.SQ_OP_GEMM, M, N, K)
+    sq.sq_gemm_w8a8(Xq.to(DEV), Wq.to(DEV), None, None, None, Y, ws)
+    torch.cuda.synchronize()
+    sq.sq_workspace_status(ws)
+    ref = oracle.gemm_i8(Xq.numpy(), Wq.numpy())
+    assert np.all(np.abs(ref) < 2 ** 31)
+    assert np.array_equal(Y.cpu().numpy().astype(np.int64), ref)
+
+
+def test_gemm_int32_extremes():
+    """All-127 operands at the largest K of the workloads: no overflow."""
+    K = 49152
+    Xq = torch.full((130, K), 127, dtype=torch.int8)
+    Xq[1::2] = -127
+    Wq = torch.full((260, K), 127, dtype=torch.int8)
+    Wq[5] = -127
+    Y = torch.empty((130, 260), dtype=torch.int32, device=DEV)
+    sq.sq_gemm_w8a8(Xq.to(DEV), Wq.to(DEV), None, None, None, Y, sq.workspace(0, 130, 260, K))
+    y = Y.cpu().numpy().astype(np.int64)
+    expect = np.where((np.arange(130)[:, None] % 2 == 1) ^ (np.arange(260)[None, :] == 5), -1, 1) * 792_772_608
+    assert np.array_equal(y, expect)
+
+
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float16, torch.float32])
+@pytest.mark.parametrize("per_token,per_channel,with_bias", [(True, True, False), (False, False, False),
+                                                             (True, False, True), (False, True, True)])
+def test_gemm_dequant(out_dtype, per_token, per_channel, with_bias):
+    M, N, K = 300, 520, 1040
+    Xq, Wq = rand_i8((M, K), 31), rand_i8((N, K), 32)
+    g = torch.Generator().manual_seed(33)
+    qx = torch.rand(M if per_token else 1, generator=g) * 100 + 1
+    qw = torch.rand(N if per_channel else 1, generator=g) * 5000 + 100
+    bias = torch.randn(N, generator=g) if with_bias else None
+    Y = torch.empty((M, N), dtype=out_dtype, device=DEV)
+    sq.sq_gemm_w8a8(Xq.to(DEV), Wq.to(DEV), qx.to(DEV), qw.to(DEV), None if bias is None else bias.to(DEV), Y,
+                    sq.workspace(0, M, N, K))
+    acc = oracle.gemm_i8(Xq.numpy(), Wq.numpy())
+    y = oracle.dequant(acc, qx.numpy(), qw.numpy(), None if bias is None else bias.numpy())
+    terms = np.abs(oracle.dequant(acc, qx.numpy(), qw.numpy()))
+    if bias is not None:
+        terms = terms + np.abs(bias.numpy().astype(np.float64))[None, :]
+    if out_dtype == torch.float32:
+        assert_close_f32(Y, y, terms)
+    else:
+        assert_close_16(Y, y, out_dtype, terms if bias is not None else None)
+
+
+def test_gemm_strided_output_untouched_tail():
+    """Outputs beyond N (ldy > N) keep their contents; rows past M are never written."""
+    M, N, K = 131, 200, 256
+    Xq, Wq = rand_i8((M, K), 41), rand_i8((N, K), 42)
+    big = torch.full((M + 3, 264), 7.0, dtype=torch.bfloat16, device=DEV)
+    Y = big[:M, :N]
+    qx = torch.full((M,), 50.0, device=DEV)
+    qw = torch.full((N,), 400.0, device=DEV)
+    sq.sq_gemm_w8a8(Xq.to(DEV), Wq.to(DEV), qx, qw, None, Y, sq.workspace(0, M, N, K))
+    b = big.cpu()
+    assert torch.all(b[:, N:] == 7.0) and torch.all(b[M:] == 7.0)
+    y = oracle.dequant(oracle.gemm_i8(Xq.numpy(), Wq.numpy()), np.full(M, 50, np.float32), np.full(N, 400, np.float32))
+    assert_close_16(b[:M, :N].contiguous(), y, torch.bfloat16)
+
+
+def test_gemm_deterministic():
+    M, N, K = 1024, 2048, 2048
+    Xq, Wq = rand_i8((M, K), 51).to(DEV), rand_i8((N, K), 52).to(DEV)
+    qx = torch.rand(M, device=DEV) + 1
+    qw = torch.rand(N, device=DEV) + 100
+    ws = sq.workspace(0, M, N, K)
+    outs = []
+    for _ in range(2):
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=DEV)
+        sq.sq_gemm_w8a8(Xq, Wq, qx, qw, None, Y, ws)
+        outs.append(Y)
+    assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
+
+
+@pytest.mark.parametrize("M,N,K", [(4096, 36864, 12288), (1024, 28672, 7168), (2048, 16384, 4096)])
+def test_gemm_full_size_sampled(M, N, K):
+    """Full-size shapes in the launch configuration the benchmark times:
+    all outputs against torch._int_mm (a library cross-check, test only) and
+    sampled rows against the oracle."""
+    g = torch.Generator(device=DEV).manual_seed(M + N)
+    Xq = torch.randint(-127, 128, (M, K), generator=g, device=DEV, dtype=torch.int8)
+    Wq = torch.randint(-127, 128, (N, K), generator=g, device=DEV, dtype=torch.int8)
+    Y = torch.empty((M, N), dtype=torch.int32, device=DEV)
+    ws = sq.workspace(0, M, N, K)
+    sq.sq_gemm_w8a8(Xq, Wq, None, None, None, Y, ws)
+    ref = torch._int_mm(Xq, Wq.t())
+    assert torch.equal(Y, ref)
+    rows = [0, 1, 127, 128, M // 2 + 3, M - 1]
+    Xs = Xq[rows].cpu().numpy()
+    acc = oracle.gemm_i8(Xs, Wq.cpu().numpy())
+    assert np.array_equal(Y[rows].cpu().numpy().astype(np.int64), acc)
+    del Xq, Wq, Y, ref
+    torch.cuda.empty_cache()
+
+
+# ---------------------------------------------------------------- a7 - a9
+def _llm_case(M, K, N, n_out, seed, dtype=torch.float16):
+    d = inputs.c4_llmint8(device="cpu", M=M, K=K, N=N, n_out=n_out, seed=seed)
+    return d["X"].to(dtype), d["W"].to(dtype), d["dims"]
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("M,K,N,n_out", [(256, 512, 384, 3), (300, 1024, 520, 6), (64, 256, 128, 0)])
+def test_llmint8_steps_and_matmul(dtype, M, K, N, n_out):
+    X, W, dims = _llm_case(M, K, N, n_out, seed=M + n_out, dtype=dtype)
+    Xd, Wd = X.to(DEV), W.to(DEV)
+    idx = torch.empty(K, dtype=torch.int32, device=DEV)
+    n = torch.empty(1, dtype=torch.int32, device=DEV)
+    wsd = sq.workspace(sq.SQ_OP_LLMINT8_DETECT, M, N, K)
+    sq.sq_llmint8_detect(Xd, 6.0, 0.0, idx, n, wsd)
+    ridx = oracle.llmint8_outliers(X, 6.0, 0.0)
+    assert ridx.tolist() == dims.tolist()
+    nn_ = int(n.item())
+    assert nn_ == ridx.size and idx[:nn_].cpu().numpy().tolist() == ridx.tolist()
+    Xq = torch.empty((M, K), dtype=torch.int8, device=DEV)
+    qx = torch.empty(M, device=DEV)
+    sq.sq_llmint8_quant_rows(Xd, idx, n, Xq, qx)
+    rXq, rqx = oracle.llmint8_quant_rows(X, ridx)
+    assert np.array_equal(Xq.cpu().numpy(), rXq) and np.array_equal(npf(qx), rqx)
+    Wq = torch.empty((N, K), dtype=torch.int8, device=DEV)
+    qw = torch.empty(N, device=DEV)
+    sq.sq_llmint8_quant_weight(Wd, idx, n, Wq, qw)
+    rWq, rqw = oracle.llmint8_quant_weight(W, ridx)
+    assert np.array_equal(Wq.cpu().numpy(), rWq) and np.array_equal(npf(qw), rqw)
+    # the fused call
+    st = sq.llmint8_weight_state(Wd)
+    Y = torch.empty((M, N), dtype=dtype, device=DEV)
+    idx2 = torch.empty(K, dtype=torch.int32, device=DEV)
+    n2 = torch.empty(1, dtype=torch.int32, device=DEV)
+    ws = sq.workspace(sq.SQ_OP_LLMINT8, M, N, K)
+    sq.sq_llmint8_matmul(Xd, st, 6.0, 0.0, Y, idx2, n2, ws)
+    torch.cuda.synchronize()
+    sq.sq_workspace_status(ws)
+    assert int(n2.item()) == ridx.size and idx2[:ridx.size].cpu().numpy().tolist() == ridx.tolist()
+    assert np.array_equal(st["Wq"].cpu().numpy(), rWq) and np.array_equal(npf(st["qs_w"]), rqw)
+    acc = oracle.gemm_i8(rXq, rWq)
+    y = oracle.llmint8_combine(acc, rqx, rqw, X, W, ridx)
+    Xf, Wf = npf(X).astype(np.float64), npf(W).astype(np.float64)
+    terms = np.abs(oracle.dequant(acc, rqx, rqw)) + np.abs(Xf[:, ridx]) @ np.abs(Wf[:, ridx]).T
+    assert_close_16(Y, y, dtype, terms)
+    # second call, same O: the cached weight is reused and the result repeats
+    Y2 = torch.empty_like(Y)
+    sq.sq_llmint8_matmul(Xd, st, 6.0, 0.0, Y2, idx2, n2, ws)
+    assert int(ws[4:8].view(torch.int32).item()) == 0  # O unchanged
+    assert torch.equal(Y.view(torch.int16), Y2.view(torch.int16))
+
+
+def test_llmint8_cache_follows_outlier_set():
+    M, K, N = 128, 512, 256
+    X1, W, _ = _llm_case(M, K, N, 3, seed=1)
+    X2, _, _ = _llm_case(M, K, N, 5, seed=2)
+    Wd = W.to(DEV)
+    st = sq.llmint8_weight_state(Wd)
+    ws = sq.workspace(sq.SQ_OP_LLMINT8, M, N, K)
+    idx = torch.empty(K, dtype=torch.int32, device=DEV)
+    n = torch.empty(1, dtype=torch.int32, device=DEV)
+    for X in (X1, X2, X1):
+        Y = torch.empty((M, N), dtype=torch.float16, device=DEV)
+        sq.sq_llmint8_matmul(X.to(DEV), st, 6.0, 0.0, Y, idx, n, ws)
+        ridx = oracle.llmint8_outliers(X, 6.0, 0.0)
+        assert int(ws[4:8].view(torch.int32).item()) == 1  # O changed each time
+        rWq, rqw = oracle.llmint8_quant_weight(W, ridx)
+        assert np.array_equal(st["Wq"].cpu().numpy(), rWq)
+        rXq, rqx = oracle.llmint8_quant_rows(X, ridx)
+        acc = oracle.gemm_i8(rXq, rWq)
+        y = oracle.llmint8_combine(acc, rqx, rqw, X, W, ridx)
+        Xf, Wf = npf(X).astype(np.float64), npf(W).astype(np.float64)
+        terms = np.abs(oracle.dequant(acc, rqx, rqw)) + np.abs(Xf[:, ridx]) @ np.abs(Wf[:, ridx]).T
+        assert_close_16(Y, y, torch.float16, terms)
+
+
+def test_llmint8_min_ratio():
+    M, K = 200, 256
+    X = rnd((M, K), 61, torch.float16).clamp(-5, 5)
+    X[:13, 10] = 7.0   # 13/200 = 0.065 > 0.06
+    X[:12, 20] = -9.0  # 12/200 = 0.06, not > 0.06
+    X[:1, 30] = 6.5
+    idx = torch.empty(K, dtype=torch.int32, device=DEV)
+    n = torch.empty(1, dtype=torch.int32, device=DEV)
+    ws = sq.workspace(sq.SQ_OP_LLMINT8_DETECT, M, 0, K)
+    for mr in (0.0, 0.06, 0.1):
+        sq.sq_llmint8_detect(X.to(DEV), 6.0, mr, idx, n, ws)
+        ref = oracle.llmint8_outliers(X, 6.0, mr).tolist()
+        assert idx[: int(n.item())].cpu().tolist() == ref
+
+
+def test_llmint8_full_size_sampled():
+    """The 6.7B-shaped case ([2048,4096] x [16384,4096]) in the benchmark's
+    launch configuration; outlier set exact, sampled rows against the oracle."""
+    d = inputs.c4_llmint8(device=DEV)
+    X, W = d["X"], d["W"]
+    M, K = X.shape
+    N = W.shape[0]
+    st = sq.llmint8_weight_state(W)
+    Y = torch.empty((M, N), dtype=torch.float16, device=DEV)
+    idx = torch.empty(K, dtype=torch.int32, device=DEV)
+    n = torch.empty(1, dtype=torch.int32, device=DEV)
+    ws = sq.workspace(sq.SQ_OP_LLMINT8, M, N, K)
+    sq.sq_llmint8_matmul(X, st, 6.0, 0.0, Y, idx, n, ws)
+    torch.cuda.synchronize()
+    Xc, Wc = X.cpu(), W.cpu()
+    ridx = oracle.llmint8_outliers(Xc, 6.0, 0.0)
+    assert ridx.tolist() == d["dims"].tolist()
+    assert idx[: int(n.item())].cpu().tolist() == ridx.tolist()
+    rWq, rqw = oracle.llmint8_quant_weight(Wc, ridx)
+    assert np.array_equal(st["qs_w"].cpu().numpy(), rqw)
+    assert np.array_equal(st["Wq"].cpu().numpy(), rWq)
+    rows = np.array([0, 5, 511, 1024, 2047])
+    rXq, rqx = oracle.llmint8_quant_rows(Xc[rows], ridx)
+    acc = oracle.gemm_i8(rXq, rWq)
+    y = oracle.llmint8_combine(acc, rqx, rqw, Xc[rows], Wc, ridx)
+    Xf, Wf = npf(Xc[rows]).astype(np.float64), npf(Wc).astype(np.float64)
+    terms = np.abs(oracle.dequant(acc, rqx, rqw)) + np.abs(Xf[:, ridx]) @ np.abs(Wf[:, ridx]).T
+    assert_close_16(Y[rows].contiguous(), y, torch.float16, terms)
+
+
+# ---------------------------------------------------------------- edges
+def test_empty_inputs():
+    ws = sq.workspace(0, 1, 16, 16)
+    e = torch.empty((0, 16), dtype=torch.int8, device=DEV)
+    W = rand_i8((16, 16), 1).to(DEV)
+    Y = torch.empty((0, 16), dtype=torch.bfloat16, device=DEV)
+    sq.sq_gemm_w8a8(e, W, torch.ones(1, device=DEV), torch.ones(1, device=DEV), None, Y, ws)
+    xmax = torch.full((16,), 3.0, device=DEV)
+    sq.sq_calib_absmax(torch.empty((0, 16), dtype=torch.bfloat16, device=DEV), xmax)
+    assert torch.all(xmax == 3.0)
+    n = torch.full((1,), 99, dtype=torch.int32, device=DEV)
+    idx = torch.empty(16, dtype=torch.int32, device=DEV)
+    sq.sq_llmint8_detect(torch.empty((0, 16), dtype=torch.float16, device=DEV), 6.0, 0.0, idx, n,
+                         sq.workspace(3, 0, 0, 16))
+    assert int(n.item()) == 0
+
+
+def test_errors_raise():
+    with pytest.raises(sq.SqError) as ei:
+        sq.sq_gemm_w8a8(torch.zeros((4, 24), dtype=torch.int8, device=DEV),
+                        torch.zeros((4, 24), dtype=torch.int8, device=DEV), None, None, None,
+                        torch.empty((4, 4), dtype=torch.int32, device=DEV), sq.workspace(0, 4, 4, 24))
+    assert ei.value.status == 2

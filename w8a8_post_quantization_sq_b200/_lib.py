@@ -1,0 +1,270 @@
+"""ctypes binding of libsq_b200.so: argument marshalling only.
+
+Every function here has the name of the C entry point it calls, takes torch
+tensors that already live on the GPU (torch provides device memory and the
+current stream), checks dtype/contiguity, passes raw pointers and sizes, and
+raises SqError when the call returns a non-zero status. No arithmetic of the
+method happens in Python, and there is no fallback: if the shared library is
+missing or cannot be loaded, the first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsq_b200.so")
+
+SQ_F32, SQ_F16, SQ_BF16, SQ_I32, SQ_I8 = 0, 1, 2, 3, 4
+SQ_LAYERNORM, SQ_RMSNORM = 0, 1
+SQ_OP_GEMM, SQ_OP_QUANT_ACT, SQ_OP_QUANT_WEIGHT, SQ_OP_LLMINT8_DETECT, SQ_OP_LLMINT8 = 0, 1, 2, 3, 4
+
+STATUS = {0: "SQ_OK", 1: "SQ_ERR_INVALID_ARG", 2: "SQ_ERR_UNSUPPORTED_SHAPE", 3: "SQ_ERR_ALIGNMENT",
+          4: "SQ_ERR_CUDA", 5: "SQ_ERR_TIMEOUT"}
+
+_DT = {torch.float32: SQ_F32, torch.float16: SQ_F16, torch.bfloat16: SQ_BF16, torch.int32: SQ_I32,
+       torch.int8: SQ_I8}
+
+
+class SqError(RuntimeError):
+    def __init__(self, name, status, msg):
+        super().__init__(f"{name}: {STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+class LLMInt8Weight(ctypes.Structure):
+    _fields_ = [("W", ctypes.c_void_p), ("N", ctypes.c_int64), ("Wq", ctypes.c_void_p),
+                ("qs_w", ctypes.c_void_p), ("cached_idx", ctypes.c_void_p), ("cached_n", ctypes.c_void_p)]
+
+
+_p, _i64, _i, _f, _d, _sz = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_double,
+                             ctypes.c_size_t)
+
+SIGNATURES = {
+    "sq_workspace_size": ([_i, _i64, _i64, _i64], _sz),
+    "sq_last_error_string": ([], ctypes.c_char_p),
+    "sq_workspace_status": ([_p, _p], _i),
+    "sq_version": ([], _i),
+    "sq_calib_absmax": ([_p, _i, _i64, _i64, _i64, _p, _p], _i),
+    "sq_weight_absmax": ([_p, _i, _i64, _i64, _i64, _p, _p], _i),
+    "sq_smooth_scales": ([_p, _p, _i64, _d, _p, _p], _i),
+    "sq_fold_weight": ([_p, _i, _i64, _i64, _p, _p, _p], _i),
+    "sq_fold_norm": ([_p, _p, _p, _i64, _p, _p, _p], _i),
+    "sq_quantize_weight": ([_p, _i, _i64, _i64, _p, _i, _p, _p, _p, _sz, _p], _i),
+    "sq_quantize_act": ([_p, _i, _i64, _i64, _i64, _p, _i, _p, _p, _p, _p, _sz, _p], _i),
+    "sq_scale_from_absmax": ([_p, _i64, _p, _p], _i),
+    "sq_norm_smooth_quant": ([_p, _i, _i64, _i64, _i64, _i, _p, _p, _f, _i, _p, _p, _p, _p, _p, _p], _i),
+    "sq_gemm_w8a8": ([_p, _p, _i64, _i64, _i64, _p, _i, _p, _i, _p, _i, _p, _i64, _p, _sz, _p], _i),
+    "sq_llmint8_detect": ([_p, _i, _i64, _i64, _i64, _f, _d, _p, _p, _p, _sz, _p], _i),
+    "sq_llmint8_quant_rows": ([_p, _i, _i64, _i64, _i64, _p, _p, _p, _p, _p], _i),
+    "sq_llmint8_quant_weight": ([_p, _i, _i64, _i64, _p, _p, _p, _p, _p], _i),
+    "sq_llmint8_matmul": ([_p, _i, _i64, _i64, _i64, ctypes.POINTER(LLMInt8Weight), _f, _d, _p, _i64, _p, _p, _p,
+                           _sz, _p], _i),
+}
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libsq_b200.so (once). Raises if it is not built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is not built; run `python -m w8a8_post_quantization_sq_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = L
+    return _lib
+
+
+def _check(name, status):
+    if status != 0:
+        raise SqError(name, status, lib().sq_last_error_string().decode())
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensor must be on a CUDA device")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dt(t):
+    return _DT[t.dtype]
+
+
+def _ld(t):
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError("expected a 2-D tensor with unit inner stride")
+    return t.stride(0)
+
+
+def _vec(t, dtype, n=None):
+    if t is None:
+        return None
+    if t.dtype != dtype or not t.is_contiguous() or (n is not None and t.numel() != n):
+        raise ValueError(f"expected a contiguous {dtype} tensor of {n} elements")
+    return _ptr(t)
+
+
+# ---------------------------------------------------------------- workspace
+def sq_workspace_size(op, M, N, K):
+    return int(lib().sq_workspace_size(op, M, N, K))
+
+
+def workspace(op, M, N, K, device=None):
+    """A zeroed workspace tensor sized for `op` (allocated by torch)."""
+    n = max(sq_workspace_size(op, M, N, K), 256)
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def sq_workspace_status(ws, stream=None):
+    _check("sq_workspace_status", lib().sq_workspace_status(_ptr(ws), _stream(stream)))
+
+
+def sq_version():
+    return int(lib().sq_version())
+
+
+# ---------------------------------------------------------------- a1 / a2
+def sq_calib_absmax(X, xmax, stream=None):
+    _check("sq_calib_absmax", lib().sq_calib_absmax(_ptr(X), _dt(X), X.shape[0], X.shape[1], _ld(X),
+                                                    _vec(xmax, torch.float32, X.shape[1]), _stream(stream)))
+
+
+def sq_weight_absmax(W, wmax, stream=None):
+    _check("sq_weight_absmax", lib().sq_weight_absmax(_ptr(W), _dt(W), W.shape[0], W.shape[1], _ld(W),
+                                                      _vec(wmax, torch.float32, W.shape[1]), _stream(stream)))
+
+
+# ---------------------------------------------------------------- a3
+def sq_smooth_scales(xmax, wmax, alpha, s_out, stream=None):
+    K = xmax.numel()
+    _check("sq_smooth_scales", lib().sq_smooth_scales(_vec(xmax, torch.float32, K), _vec(wmax, torch.float32, K), K,
+                                                      float(alpha), _vec(s_out, torch.float32, K), _stream(stream)))
+
+
+def sq_fold_weight(W, s, Wp_out, stream=None):
+    N, K = W.shape
+    if not W.is_contiguous() or not Wp_out.is_contiguous() or Wp_out.dtype != torch.float32:
+        raise ValueError("W and Wp_out must be contiguous; Wp_out fp32")
+    _check("sq_fold_weight", lib().sq_fold_weight(_ptr(W), _dt(W), N, K, _vec(s, torch.float32, K), _ptr(Wp_out),
+                                                  _stream(stream)))
+
+
+def sq_fold_norm(gamma, beta, s, gamma_out, beta_out=None, stream=None):
+    K = gamma.numel()
+    _check("sq_fold_norm", lib().sq_fold_norm(_vec(gamma, torch.float32, K), _vec(beta, torch.float32, K),
+                                              _vec(s, torch.float32, K), K, _vec(gamma_out, torch.float32, K),
+                                              _vec(beta_out, torch.float32, K), _stream(stream)))
+
+
+# ---------------------------------------------------------------- a4
+def sq_quantize_weight(W, s, per_channel, Wq, qs_w, ws=None, stream=None):
+    N, K = W.shape
+    if not W.is_contiguous() or not Wq.is_contiguous() or Wq.dtype != torch.int8:
+        raise ValueError("W and Wq must be contiguous; Wq int8")
+    _check("sq_quantize_weight", lib().sq_quantize_weight(
+        _ptr(W), _dt(W), N, K, _vec(s, torch.float32, K), int(per_channel), _ptr(Wq),
+        _vec(qs_w, torch.float32, N if per_channel else 1), _ptr(ws), 0 if ws is None else ws.numel(),
+        _stream(stream)))
+
+
+# ---------------------------------------------------------------- a5'
+def sq_quantize_act(X, s, per_token, static_qs, Xq, qs_x, ws=None, stream=None):
+    M, K = X.shape
+    if not Xq.is_contiguous() or Xq.dtype != torch.int8:
+        raise ValueError("Xq must be contiguous int8")
+    _check("sq_quantize_act", lib().sq_quantize_act(
+        _ptr(X), _dt(X), M, K, _ld(X), _vec(s, torch.float32, K), int(per_token), _vec(static_qs, torch.float32, 1),
+        _ptr(Xq), _vec(qs_x, torch.float32, M if per_token else 1), _ptr(ws), 0 if ws is None else ws.numel(),
+        _stream(stream)))
+
+
+def sq_scale_from_absmax(absmax, qs_out, stream=None):
+    _check("sq_scale_from_absmax", lib().sq_scale_from_absmax(_vec(absmax, torch.float32), absmax.numel(),
+                                                              _vec(qs_out, torch.float32, 1), _stream(stream)))
+
+
+# ---------------------------------------------------------------- a5
+def sq_norm_smooth_quant(H, norm, gamma, beta, eps, per_token, static_qs, Xq, qs_x, absmax=None, V=None,
+                         stream=None):
+    M, K = H.shape
+    if Xq is not None and (not Xq.is_contiguous() or Xq.dtype != torch.int8):
+        raise ValueError("Xq must be contiguous int8")
+    if V is not None and (V.dtype != H.dtype or not V.is_contiguous()):
+        raise ValueError("V must be contiguous with the dtype of H")
+    _check("sq_norm_smooth_quant", lib().sq_norm_smooth_quant(
+        _ptr(H), _dt(H), M, K, _ld(H), int(norm), _vec(gamma, torch.float32, K), _vec(beta, torch.float32, K),
+        float(eps), int(per_token), _vec(static_qs, torch.float32, 1), _ptr(Xq),
+        None if qs_x is None else _vec(qs_x, torch.float32), _vec(absmax, torch.float32, K), _ptr(V),
+        _stream(stream)))
+
+
+# ---------------------------------------------------------------- a6
+def sq_gemm_w8a8(Xq, Wq, qs_x, qs_w, bias, Y, ws, stream=None):
+    M, K = Xq.shape
+    N = Wq.shape[0]
+    if Xq.dtype != torch.int8 or Wq.dtype != torch.int8 or not Xq.is_contiguous() or not Wq.is_contiguous():
+        raise ValueError("Xq and Wq must be contiguous int8")
+    if Wq.shape[1] != K or Y.shape[0] != M or Y.shape[1] != N:
+        raise ValueError("shape mismatch")
+    _check("sq_gemm_w8a8", lib().sq_gemm_w8a8(
+        _ptr(Xq), _ptr(Wq), M, N, K, _vec(qs_x, torch.float32), int(qs_x is not None and qs_x.numel() > 1),
+        _vec(qs_w, torch.float32), int(qs_w is not None and qs_w.numel() > 1), _vec(bias, torch.float32, N),
+        _dt(Y), _ptr(Y), _ld(Y), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+# ---------------------------------------------------------------- a7 - a9
+def sq_llmint8_detect(X, threshold, min_ratio, idx, n, ws, stream=None):
+    M, K = X.shape
+    _check("sq_llmint8_detect", lib().sq_llmint8_detect(
+        _ptr(X), _dt(X), M, K, _ld(X), float(threshold), float(min_ratio), _vec(idx, torch.int32, K),
+        _vec(n, torch.int32, 1), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def sq_llmint8_quant_rows(X, idx, n, Xq, qs_x, stream=None):
+    M, K = X.shape
+    _check("sq_llmint8_quant_rows", lib().sq_llmint8_quant_rows(
+        _ptr(X), _dt(X), M, K, _ld(X), _vec(idx, torch.int32), _vec(n, torch.int32, 1), _ptr(Xq),
+        _vec(qs_x, torch.float32, M), _stream(stream)))
+
+
+def sq_llmint8_quant_weight(W, idx, n, Wq, qs_w, stream=None):
+    N, K = W.shape
+    if not W.is_contiguous():
+        raise ValueError("W must be contiguous")
+    _check("sq_llmint8_quant_weight", lib().sq_llmint8_quant_weight(
+        _ptr(W), _dt(W), N, K, _vec(idx, torch.int32), _vec(n, torch.int32, 1), _ptr(Wq),
+        _vec(qs_w, torch.float32, N), _stream(stream)))
+
+
+def llmint8_weight_state(W):
+    """Device buffers of the int8 weight cache for sq_llmint8_matmul (torch
+    allocates them; cached_n = -1 marks the cache empty)."""
+    N, K = W.shape
+    st = {"W": W, "Wq": torch.empty((N, K), dtype=torch.int8, device=W.device),
+          "qs_w": torch.empty(N, dtype=torch.float32, device=W.device),
+          "cached_idx": torch.zeros(K, dtype=torch.int32, device=W.device),
+          "cached_n": torch.full((1,), -1, dtype=torch.int32, device=W.device)}
+    st["c"] = LLMInt8Weight(W.data_ptr(), N, st["Wq"].data_ptr(), st["qs_w"].data_ptr(),
+                            st["cached_idx"].data_ptr(), st["cached_n"].data_ptr())
+    return st
+
+
+def sq_llmint8_matmul(X, wstate, threshold, min_ratio, Y, idx, n, ws, stream=None):
+    M, K = X.shape
+    _check("sq_llmint8_matmul", lib().sq_llmint8_matmul(
+        _ptr(X), _dt(X), M, K, _ld(X), ctypes.byref(wstate["c"]), float(threshold), float(min_ratio), _ptr(Y),
+        _ld(Y), _vec(idx, torch.int32, K), _vec(n, torch.int32, 1), _ptr(ws), ws.numel(), _stream(stream)))

@@ -1,0 +1,124 @@
+// a1 / a2: per-input-channel absmax for calibration.
+//
+// x_j = max_i |X_ij| over the calibration tokens and w_j = max over output
+// channels of |W| in input channel j ("大语言模型量化技术（四）：SmoothQuant",
+// section 缩放因子; lpnh.cn SmoothQuant article §3.2; "如何通过 SmoothQuant
+// 解决激活值离群点难题" §3). With W stored [N,K] both are the same operation: a
+// column max over the rows of a row-major matrix, kept as a running max.
+//
+// Bandwidth kernel. A block of 8 warps covers 32 lanes x one 16-byte vector
+// of columns (256 columns of a 16-bit matrix, 128 of an fp32 one) and a band
+// of rows; warp w reads rows w, w+8, ... so every warp-wide load is one
+// contiguous 512-byte segment. Each lane keeps the running max of its vector
+// in registers, the 8 warps combine in shared memory, and one atomicMax per
+// column per block publishes the result. max and |.| are exact, so the
+// result does not depend on the order.
+#include "sq_common.cuh"
+
+namespace sq {
+namespace {
+
+constexpr int kWarps = 8;
+constexpr int kUnroll = 4;
+
+template <typename T>
+__global__ void __launch_bounds__(kWarps * 32)
+col_absmax_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, int rows_per_block,
+                  float* __restrict__ out) {
+    constexpr int V = Vec<T>::N;
+    constexpr int COLS = 32 * V;
+    __shared__ float red[kWarps][COLS];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t c0 = (int64_t)blockIdx.x * COLS + lane * V;
+    const int64_t r_begin = (int64_t)blockIdx.y * rows_per_block;
+    const int64_t r_end = min(M, r_begin + rows_per_block);
+    float m[V];
+#pragma unroll
+    for (int e = 0; e < V; ++e) m[e] = 0.0f;
+    if (c0 < K) {
+        const T* base = X + c0;
+        int64_t r = r_begin + warp;
+        for (; r + (kUnroll - 1) * kWarps < r_end; r += kUnroll * kWarps) {
+            uint4 raw[kUnroll];
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) raw[u] = ldg_nc_v4(base + (r + u * kWarps) * ld);
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                float f[V];
+                unpack<T>(raw[u], f);
+#pragma unroll
+                for (int e = 0; e < V; ++e) m[e] = fmaxf(m[e], fabsf(f[e]));
+            }
+        }
+        for (; r < r_end; r += kWarps) {
+            float f[V];
+            unpack<T>(ldg_nc_v4(base + r * ld), f);
+#pragma unroll
+            for (int e = 0; e < V; ++e) m[e] = fmaxf(m[e], fabsf(f[e]));
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < V; ++e) red[warp][lane * V + e] = m[e];
+    __syncthreads();
+    for (int c = threadIdx.x; c < COLS; c += kWarps * 32) {
+        float v = red[0][c];
+#pragma unroll
+        for (int w = 1; w < kWarps; ++w) v = fmaxf(v, red[w][c]);
+        const int64_t col = (int64_t)blockIdx.x * COLS + c;
+        if (col < K) atomic_max_nonneg(out + col, v);
+    }
+}
+
+template <typename T>
+sq_status_t launch(const void* X, int64_t M, int64_t K, int64_t ld, float* out, cudaStream_t s,
+                   const char* name) {
+    constexpr int COLS = 32 * Vec<T>::N;
+    const int64_t col_blocks = (K + COLS - 1) / COLS;
+    // about 8 blocks per SM in one wave; rows per block a multiple of the warp count
+    const int64_t target = (int64_t)num_sms() * 8;
+    int64_t rpb = (M * col_blocks + target - 1) / target;
+    rpb = ((rpb + kWarps - 1) / kWarps) * kWarps;
+    if (rpb < kWarps * kUnroll) rpb = kWarps * kUnroll;
+    const int64_t row_blocks = (M + rpb - 1) / rpb;
+    SQ_REQUIRE(row_blocks <= 65535, SQ_ERR_UNSUPPORTED_SHAPE, "%s: too many rows (M=%lld)", name,
+               (long long)M);
+    dim3 grid((unsigned)col_blocks, (unsigned)row_blocks);
+    col_absmax_kernel<T><<<grid, kWarps * 32, 0, s>>>(static_cast<const T*>(X), M, K, ld, (int)rpb, out);
+    return check_launch(name);
+}
+
+sq_status_t col_absmax(const void* X, sq_dtype_t dt, int64_t M, int64_t K, int64_t ld, float* out,
+                       sq_stream_t stream, const char* name) {
+    SQ_REQUIRE(X && out, SQ_ERR_INVALID_ARG, "%s: null pointer", name);
+    SQ_REQUIRE(M >= 0 && K > 0 && ld >= K, SQ_ERR_UNSUPPORTED_SHAPE, "%s: bad sizes M=%lld K=%lld ld=%lld",
+               name, (long long)M, (long long)K, (long long)ld);
+    SQ_REQUIRE(dt == SQ_F16 || dt == SQ_BF16 || dt == SQ_F32, SQ_ERR_INVALID_ARG, "%s: dtype must be F16, BF16 or F32",
+               name);
+    const int v = dt == SQ_F32 ? 4 : 8;
+    SQ_REQUIRE(K % v == 0 && ld % v == 0, SQ_ERR_UNSUPPORTED_SHAPE, "%s: K and ld must be multiples of %d", name, v);
+    SQ_REQUIRE(aligned16(X), SQ_ERR_ALIGNMENT, "%s: input not 16-byte aligned", name);
+    if (M == 0) return SQ_OK;
+    cudaStream_t s = as_cuda(stream);
+    switch (dt) {
+        case SQ_F16: return launch<__half>(X, M, K, ld, out, s, name);
+        case SQ_BF16: return launch<__nv_bfloat16>(X, M, K, ld, out, s, name);
+        default: return launch<float>(X, M, K, ld, out, s, name);
+    }
+}
+
+}  // namespace
+}  // namespace sq
+
+extern "C" {
+
+sq_status_t sq_calib_absmax(const void* X, sq_dtype_t dt, int64_t M, int64_t K, int64_t ldx,
+                            float* xmax_inout, sq_stream_t stream) {
+    return sq::col_absmax(X, dt, M, K, ldx, xmax_inout, stream, "sq_calib_absmax");
+}
+
+sq_status_t sq_weight_absmax(const void* W, sq_dtype_t dt, int64_t N, int64_t K, int64_t ldw,
+                             float* wmax_inout, sq_stream_t stream) {
+    return sq::col_absmax(W, dt, N, K, ldw, wmax_inout, stream, "sq_weight_absmax");
+}
+
+}  // extern "C"

@@ -1,0 +1,521 @@
+// a6: INT8 x INT8 -> INT32 GEMM on the 5th-generation tensor cores with a
+// dequantising epilogue, and (a9) the LLM.int8 16-bit outlier term fused into
+// the same epilogue.
+//
+// What it computes ("8位量化：异常值与混合精度分解实战" §2.1; "大语言模型量化技术
+// （四）：SmoothQuant", 为什么激活不能用逐通道量化):
+//   acc[i,j] = sum_k Xq[i,k] * Wq[j,k]            exact in int32
+//   Y[i,j]   = acc * ((1/qs_x[i]) * (1/qs_w[j])) (+ h[i,j]) (+ bias[j])
+// where h is the outlier term sum_{o in O} X16[i,o] * W16[j,o] of §2.2
+// (fp32 fma in ascending o; the 16-bit products are exact in fp32).
+//
+// Design (sm_100a):
+//   - persistent: one 192-thread CTA per SM loops over 128 x BN output tiles,
+//     M index fastest so the CTAs running together share weight tiles in L2;
+//   - warp 0 (one lane) issues TMA loads of 128 x 128 int8 tiles of Xq and
+//     BN x 128 tiles of Wq (128-byte swizzle) into a 4-stage shared-memory
+//     ring guarded by mbarriers;
+//   - warp 1 (one lane) issues tcgen05.mma.cta_group::1.kind::i8 (M=128,
+//     N=BN, K=32 each, four per stage) into a double-buffered int32
+//     accumulator in tensor memory (2 x BN of the 512 columns), and frees
+//     ring stages and accumulator buffers with tcgen05.commit;
+//   - warps 2..5 read the accumulator with tcgen05.ld (warp w owns TMEM lanes
+//     32*(w%4)..+31 = tile rows), dequantise in fp32 and store the row
+//     segments, while the next tile's MMAs run in the other buffer.
+// Every wait is bounded (about 2 s of %globaltimer); on expiry the kernel
+// records code 0x6E1 + role in the status word, drains its own TMA copies and
+// MMAs, frees its tensor memory and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "sq_common.cuh"
+#include "sq_internal.h"
+
+namespace sq {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 128;  // one 128-byte swizzle row of int8
+constexpr int UMMA_K = 32;
+constexpr int STAGES = 4;
+constexpr int kThreads = 192;
+constexpr uint64_t kTimeoutNs = 2000000000ull;
+
+template <int BN>
+struct Cfg {
+    static constexpr uint32_t A_BYTES = BM * BK;
+    static constexpr uint32_t B_BYTES = BN * BK;
+    static constexpr uint32_t A_OFF = 0;
+    static constexpr uint32_t B_OFF = STAGES * A_BYTES;
+    static constexpr uint32_t BAR_OFF = B_OFF + STAGES * B_BYTES;
+    // full[S], empty[S], tfull[2], tempty[2], drain
+    static constexpr uint32_t NBAR = 2 * STAGES + 5;
+    static constexpr uint32_t MISC_OFF = BAR_OFF + NBAR * 8;  // tmem base, abort flag
+    static constexpr uint32_t RW_OFF = (MISC_OFF + 16 + 15) / 16 * 16;  // 1/qs_w and bias of a tile
+    static constexpr uint32_t SMEM = RW_OFF + 4 * 2 * BN * 4;  // per epilogue warp
+    static constexpr uint32_t SMEM_ALLOC = SMEM + 1024;  // slack to align the base to 1024
+    static constexpr uint32_t TMEM_COLS = 2 * BN;
+    // kind::i8, D = s32 (bits 4-5 = 2), A = B = signed 8-bit (bits 7-9, 10-12 = 1),
+    // both K-major, N >> 3 at bit 17, M >> 4 at bit 24
+    static constexpr uint32_t IDESC =
+        (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+};
+
+struct Params {
+    int M, N, K;
+    int num_m, num_n, num_kb;
+    GemmEpilogue ep;
+    int* status;
+};
+
+// ---------------------------------------------------------------- PTX helpers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait for the phase of `parity` to complete. Gives up when another role has
+// aborted or after kTimeoutNs, recording `code` in the status word.
+__device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          int* status, int code) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t n = 1;; ++n) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if ((n & 31u) == 0 && global_ns() - t0 > kTimeoutNs) {
+            *abort_flag = 1;
+            atomicExch(status, code);
+            return false;
+        }
+    }
+}
+
+// Short bounded wait used while draining after an abort (ignores the flag).
+__device__ __noinline__ void wait_drain(uint32_t bar, uint32_t parity) {
+    const uint64_t t0 = global_ns();
+    while (!mbar_try_wait(bar, parity))
+        if (global_ns() - t0 > kTimeoutNs / 4) return;
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+        : "memory");
+}
+
+// UMMA shared-memory descriptor, K-major operand with 128-byte swizzle: rows of
+// 128 bytes, 8-row groups 1024 bytes apart (SBO), version 1, layout 2.
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr) {
+    uint64_t d = (uint64_t)((saddr & 0x3FFFFu) >> 4);
+    d |= (uint64_t)1 << 16;
+    d |= (uint64_t)(1024 >> 4) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+
+__device__ __forceinline__ void umma_i8(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ float load16(const void* base, int64_t idx, int bf16) {
+    const uint16_t u = static_cast<const uint16_t*>(base)[idx];
+    if (bf16) return __uint_as_float((uint32_t)u << 16);
+    return __half2float(__ushort_as_half(u));
+}
+
+// Store 32 consecutive outputs of one row.
+__device__ __forceinline__ void store_row32(const GemmEpilogue& ep, int64_t row, int col0, int N, const float* y,
+                                            const uint32_t* acc_raw) {
+    const bool full = col0 + 32 <= N;
+    if (ep.out_dt == SQ_I32 || ep.out_dt == SQ_F32) {
+        uint32_t* dst = static_cast<uint32_t*>(ep.Y) + row * ep.ldy + col0;
+        const bool vec = full && ((reinterpret_cast<uintptr_t>(dst) & 15u) == 0);
+        uint32_t v[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = ep.out_dt == SQ_I32 ? acc_raw[e] : __float_as_uint(y[e]);
+        if (vec) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 4)
+                *reinterpret_cast<uint4*>(dst + e) = make_uint4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+        } else {
+            for (int e = 0; e < 32 && col0 + e < N; ++e) dst[e] = v[e];
+        }
+    } else {
+        uint16_t* dst = static_cast<uint16_t*>(ep.Y) + row * ep.ldy + col0;
+        const bool vec = full && ((reinterpret_cast<uintptr_t>(dst) & 15u) == 0);
+        uint32_t p[16];
+        if (ep.out_dt == SQ_BF16) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+                p[e] = (uint32_t)to16<__nv_bfloat16>(y[2 * e]) | ((uint32_t)to16<__nv_bfloat16>(y[2 * e + 1]) << 16);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+                p[e] = (uint32_t)to16<__half>(y[2 * e]) | ((uint32_t)to16<__half>(y[2 * e + 1]) << 16);
+        }
+        if (vec) {
+#pragma unroll
+            for (int e = 0; e < 16; e += 4)
+                *reinterpret_cast<uint4*>(dst + 2 * e) = make_uint4(p[e], p[e + 1], p[e + 2], p[e + 3]);
+        } else {
+            for (int e = 0; e < 32 && col0 + e < N; ++e)
+                dst[e] = (uint16_t)(e & 1 ? (p[e >> 1] >> 16) : (p[e >> 1] & 0xffffu));
+        }
+    }
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                 const Params p) {
+    using C = Cfg<BN>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bar0 = sbase + C::BAR_OFF;
+    auto full_bar = [&](int s) { return bar0 + 8u * s; };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+    auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
+    auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
+    const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
+    float* rw_s = reinterpret_cast<float*>(smem + C::RW_OFF);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(tfull_bar(a), 1);
+            mbar_init(tempty_bar(a), 4);
+        }
+        mbar_init(drain_bar, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_holder)),
+                     "r"(C::TMEM_COLS));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    if (warp == 0 && lane == 0) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_a)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_b)) : "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+
+    const int num_tiles = p.num_m * p.num_n;
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------------------------------------------- TMA producer
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t issued_phase[STAGES];
+            bool issued[STAGES];
+            for (int s = 0; s < STAGES; ++s) issued[s] = false, issued_phase[s] = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+                const int m0 = (tile % p.num_m) * BM;
+                const int n0 = (tile / p.num_m) * BN;
+                for (int kb = 0; kb < p.num_kb; ++kb) {
+                    if (!wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, p.status, 0x6E1)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_expect_tx(full_bar(stage), C::A_BYTES + C::B_BYTES);
+                    tma_load_2d(sbase + C::A_OFF + stage * C::A_BYTES, &tmap_a, full_bar(stage), kb * BK, m0);
+                    tma_load_2d(sbase + C::B_OFF + stage * C::B_BYTES, &tmap_b, full_bar(stage), kb * BK, n0);
+                    issued[stage] = true;
+                    issued_phase[stage] = phase;
+                    if (++stage == STAGES) stage = 0, phase ^= 1u;
+                }
+            }
+            if (!ok) {
+                // make sure no copy still lands in shared memory after we leave
+                for (int s = 0; s < STAGES; ++s)
+                    if (issued[s]) wait_drain(full_bar(s), issued_phase[s]);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---------------------------------------------------- MMA issuer
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            int local = 0;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
+                const int acc = local & 1;
+                const uint32_t acc_phase = (uint32_t)(local >> 1) & 1u;
+                if (!wait_bounded(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p.status, 0x6E2)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+                for (int kb = 0; kb < p.num_kb; ++kb) {
+                    if (!wait_bounded(full_bar(stage), phase, abort_flag, p.status, 0x6E3)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_addr = sbase + C::A_OFF + stage * C::A_BYTES;
+                    const uint32_t b_addr = sbase + C::B_OFF + stage * C::B_BYTES;
+#pragma unroll
+                    for (int k = 0; k < BK / UMMA_K; ++k)
+                        umma_i8(d_tmem, sdesc(a_addr + k * UMMA_K), sdesc(b_addr + k * UMMA_K), C::IDESC,
+                                (kb | k) != 0 ? 1u : 0u);
+                    umma_commit(empty_bar(stage));
+                    if (++stage == STAGES) stage = 0, phase ^= 1u;
+                }
+                if (!ok) break;
+                umma_commit(tfull_bar(acc));
+            }
+            // all MMAs issued by this thread complete before tensor memory is freed
+            umma_commit(drain_bar);
+            wait_drain(drain_bar, 0);
+        }
+    } else {
+        // -------------------------------------------------------- epilogue
+        // No block-level barrier is used here: an abort can make one warp leave
+        // early, so each warp stages its own per-column factors and decides
+        // collectively (all lanes) whether to go on.
+        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const GemmEpilogue& ep = p.ep;
+        const bool outl = ep.idx != nullptr;
+        const int n_out = outl ? *ep.n_out : 0;
+        float* rw_w = rw_s + (warp - 2) * 2 * BN;  // this warp's 1/qs_w and bias
+        float* bias_w = rw_w + BN;
+        int local = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
+            const int m0 = (tile % p.num_m) * BM;
+            const int n0 = (tile / p.num_m) * BN;
+            __syncwarp();
+            for (int c = lane; c < BN; c += 32) {
+                const int col = n0 + c;
+                float rw = 0.0f, b = 0.0f;
+                if (col < p.N && ep.out_dt != SQ_I32) {
+                    rw = __frcp_rn(ep.w_per_channel ? ep.qs_w[col] : ep.qs_w[0]);
+                    if (ep.bias) b = ep.bias[col];
+                }
+                rw_w[c] = rw;
+                bias_w[c] = b;
+            }
+            __syncwarp();
+            const int acc = local & 1;
+            const uint32_t acc_phase = (uint32_t)(local >> 1) & 1u;
+            const bool ok = wait_bounded(tfull_bar(acc), acc_phase, abort_flag, p.status, 0x6E4);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc_fence_after();
+            const int row_in = q * 32 + lane;
+            const int64_t row = (int64_t)m0 + row_in;
+            const bool row_ok = row < p.M;
+            float rx = 0.0f;
+            if (row_ok && ep.out_dt != SQ_I32) rx = __frcp_rn(ep.x_per_token ? ep.qs_x[row] : ep.qs_x[0]);
+            const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32(t_row + (uint32_t)(c * 32), r);
+                const int col0 = n0 + c * 32;
+                if (row_ok && col0 < p.N) {
+                    float y[32];
+                    if (ep.out_dt != SQ_I32) {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            y[e] = __fmul_rn((float)(int)r[e], __fmul_rn(rx, rw_w[c * 32 + e]));
+                        if (outl) {
+                            float h[32];
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) h[e] = 0.0f;
+                            for (int o = 0; o < n_out; ++o) {
+                                const int ko = ep.idx[o];
+                                const float xo = load16(ep.x16, row * ep.ldx16 + ko, ep.in16_bf16);
+#pragma unroll
+                                for (int e = 0; e < 32; ++e) {
+                                    const int col = min(col0 + e, p.N - 1);
+                                    h[e] = __fmaf_rn(xo, load16(ep.w16, (int64_t)col * p.K + ko, ep.in16_bf16), h[e]);
+                                }
+                            }
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) y[e] = __fadd_rn(y[e], h[e]);
+                        }
+                        if (ep.bias) {
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) y[e] = __fadd_rn(y[e], bias_w[c * 32 + e]);
+                        }
+                    }
+                    store_row32(ep, row, col0, p.N, y, r);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty_bar(acc));
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(C::TMEM_COLS));
+    }
+}
+
+// ---------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// 2-D int8 tensor [rows, K] row-major, box BK x box_rows, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t K, int box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)K};
+    cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int BN>
+sq_status_t launch_bn(const int8_t* Xq, const int8_t* Wq, int64_t M, int64_t N, int64_t K, const GemmEpilogue& ep,
+                      int* status, cudaStream_t stream) {
+    using C = Cfg<BN>;
+    CUtensorMap ta, tb;
+    if (!make_map(&ta, Xq, M, K, BM) || !make_map(&tb, Wq, N, K, BN))
+        return set_error(SQ_ERR_CUDA, "sq_gemm_w8a8: cuTensorMapEncodeTiled failed");
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+        if (cudaFuncSetAttribute(gemm_w8a8_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)C::SMEM_ALLOC) != cudaSuccess)
+            return check_launch("sq_gemm_w8a8: set shared memory size");
+        attr_set[dev] = true;
+    }
+    Params p;
+    p.M = (int)M;
+    p.N = (int)N;
+    p.K = (int)K;
+    p.num_m = (int)((M + BM - 1) / BM);
+    p.num_n = (int)((N + BN - 1) / BN);
+    p.num_kb = (int)((K + BK - 1) / BK);
+    p.ep = ep;
+    p.status = status;
+    const int tiles = p.num_m * p.num_n;
+    const int grid = tiles < num_sms() ? tiles : num_sms();
+    gemm_w8a8_kernel<BN><<<grid, kThreads, C::SMEM_ALLOC, stream>>>(ta, tb, p);
+    return check_launch("sq_gemm_w8a8");
+}
+
+}  // namespace
+
+sq_status_t launch_gemm_w8a8(const int8_t* Xq, const int8_t* Wq, int64_t M, int64_t N, int64_t K,
+                             const GemmEpilogue& ep, int* status_word, cudaStream_t stream) {
+    // narrow N tiles when wide ones would leave most SMs idle
+    const int64_t tiles256 = ((M + BM - 1) / BM) * ((N + 255) / 256);
+    if (tiles256 < (int64_t)num_sms() && N > 128)
+        return launch_bn<128>(Xq, Wq, M, N, K, ep, status_word, stream);
+    return launch_bn<256>(Xq, Wq, M, N, K, ep, status_word, stream);
+}
+
+}  // namespace sq
+
+extern "C" sq_status_t sq_gemm_w8a8(const int8_t* Xq, const int8_t* Wq, int64_t M, int64_t N, int64_t K,
+                                    const float* qs_x, int x_per_token, const float* qs_w, int w_per_channel,
+                                    const float* bias, sq_dtype_t out_dt, void* Y, int64_t ldy, void* workspace,
+                                    size_t ws_bytes, sq_stream_t stream) {
+    const char* name = "sq_gemm_w8a8";
+    SQ_REQUIRE(Xq && Wq && Y, SQ_ERR_INVALID_ARG, "%s: null Xq, Wq or Y", name);
+    SQ_REQUIRE(out_dt == SQ_I32 || (qs_x && qs_w), SQ_ERR_INVALID_ARG, "%s: dequantising output needs qs_x and qs_w",
+               name);
+    SQ_REQUIRE(out_dt == SQ_I32 || out_dt == SQ_F32 || out_dt == SQ_F16 || out_dt == SQ_BF16, SQ_ERR_INVALID_ARG,
+               "%s: out dtype must be I32, F32, F16 or BF16", name);
+    SQ_REQUIRE(workspace && ws_bytes >= sq::kStatusBytes, SQ_ERR_INVALID_ARG, "%s: needs a workspace of %zu bytes",
+               name, sq::kStatusBytes);
+    SQ_REQUIRE(M >= 0 && N > 0 && K > 0 && ldy >= N, SQ_ERR_UNSUPPORTED_SHAPE, "%s: need N > 0, K > 0, ldy >= N", name);
+    SQ_REQUIRE(K % 16 == 0, SQ_ERR_UNSUPPORTED_SHAPE, "%s: K must be a multiple of 16 (TMA row stride)", name);
+    SQ_REQUIRE(K <= 133144, SQ_ERR_UNSUPPORTED_SHAPE, "%s: K > 133144 could overflow the int32 accumulator", name);
+    SQ_REQUIRE(M < (1ll << 31) && N < (1ll << 31), SQ_ERR_UNSUPPORTED_SHAPE, "%s: M and N must be < 2^31", name);
+    SQ_REQUIRE(sq::aligned16(Xq) && sq::aligned16(Wq), SQ_ERR_ALIGNMENT, "%s: Xq and Wq must be 16-byte aligned", name);
+    if (M == 0) return SQ_OK;
+    sq::GemmEpilogue ep;
+    ep.qs_x = qs_x;
+    ep.x_per_token = x_per_token;
+    ep.qs_w = qs_w;
+    ep.w_per_channel = w_per_channel;
+    ep.bias = bias;
+    ep.out_dt = out_dt;
+    ep.Y = Y;
+    ep.ldy = ldy;
+    return sq::launch_gemm_w8a8(Xq, Wq, M, N, K, ep, static_cast<int*>(workspace), sq::as_cuda(stream));
+}

@@ -1,0 +1,327 @@
+// a7-a9: the LLM.int8() mixed-precision decomposition
+// ("8位量化：异常值与混合精度分解实战" §2.2 split_outliers / mixed_precision_matmul,
+// §2.3 threshold 6.0, §4.1 any value over the threshold marks its dimension).
+//
+//   O = { j : count_i(|X_ij| > threshold) / M > min_ratio }, ascending;
+//   the columns of X in O take a 16-bit product with the matching input
+//   channels of W; the other columns take the vector-wise int8 path (row
+//   scales for X, per-output-channel scales for W over the channels not in O);
+//   the two results are summed.
+//
+// Kernels:
+//   count_kernel      one pass over X; a block owns 256 columns x 128 rows and
+//                     writes its per-column counts to its own slot of the
+//                     workspace (no atomics, nothing to zero beforehand);
+//   compact_kernel    one block sums the slots, applies the ratio test in
+//                     fp64, and writes O in ascending order with a block-wide
+//                     prefix sum; it also compares O with the set the cached
+//                     int8 weight was built for and updates that record;
+//   masked_quant_kernel  row-wise absmax int8 over the columns not in O (used
+//                     for the rows of X and for the output channels of W; the
+//                     weight pass returns at once when O is unchanged);
+//   the tcgen05 GEMM, whose epilogue adds the 16-bit outlier term.
+// Nothing here synchronises with the host, so a whole call can be captured in
+// a CUDA graph.
+#include "sq_common.cuh"
+#include "sq_internal.h"
+
+namespace sq {
+
+size_t detect_workspace_bytes(int64_t M, int64_t K) {
+    const int64_t rb = (M + kDetectRows - 1) / kDetectRows;
+    const size_t counts = (size_t)(rb > 0 ? rb : 1) * (size_t)K * sizeof(int32_t);
+    return kStatusBytes + (counts + 255) / 256 * 256;
+}
+
+// header + counts | Xq [M,K] int8 | qs_x [M] fp32
+size_t llmint8_workspace_bytes(int64_t M, int64_t K) {
+    return detect_workspace_bytes(M, K) + ((size_t)M * (size_t)K + 255) / 256 * 256 + ((size_t)M * 4 + 255) / 256 * 256;
+}
+
+namespace {
+
+constexpr int kWarps = 8;
+constexpr int kCompactThreads = 1024;
+
+template <typename T>
+__global__ void __launch_bounds__(kWarps * 32)
+count_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, float thr, int32_t* __restrict__ partial) {
+    __shared__ int32_t red[kWarps][256];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t c0 = (int64_t)blockIdx.x * 256 + lane * 8;
+    const int64_t r0 = (int64_t)blockIdx.y * kDetectRows;
+    const int64_t r1 = min(M, r0 + kDetectRows);
+    int32_t cnt[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    if (c0 < K) {
+        for (int64_t r = r0 + warp; r < r1; r += kWarps) {
+            float f[8];
+            unpack<T>(ldg_nc_v4(X + r * ld + c0), f);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) cnt[e] += fabsf(f[e]) > thr ? 1 : 0;
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) red[warp][lane * 8 + e] = cnt[e];
+    __syncthreads();
+    for (int c = threadIdx.x; c < 256; c += kWarps * 32) {
+        int32_t s = 0;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) s += red[w][c];
+        const int64_t col = (int64_t)blockIdx.x * 256 + c;
+        if (col < K) partial[(int64_t)blockIdx.y * K + col] = s;
+    }
+}
+
+// flags word 1 of the workspace header: 1 when O differs from the cached set.
+__global__ void __launch_bounds__(kCompactThreads)
+compact_kernel(const int32_t* __restrict__ partial, int64_t row_blocks, int64_t M, int64_t K, double min_ratio,
+               int32_t* __restrict__ idx, int32_t* __restrict__ n_out, int32_t* __restrict__ cached_idx,
+               int32_t* __restrict__ cached_n, int32_t* __restrict__ changed) {
+    __shared__ int32_t warp_tot[kCompactThreads / 32];
+    __shared__ int32_t base_sh;
+    __shared__ int32_t diff_sh;
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    if (t == 0) base_sh = 0, diff_sh = 0;
+    __syncthreads();
+    for (int64_t j0 = 0; j0 < K; j0 += kCompactThreads) {
+        const int64_t j = j0 + t;
+        bool flag = false;
+        if (j < K) {
+            int64_t total = 0;
+            for (int64_t b = 0; b < row_blocks; ++b) total += partial[b * K + j];
+            const double ratio = M > 0 ? __ddiv_rn((double)total, (double)M) : 0.0;
+            flag = ratio > min_ratio;
+        }
+        const unsigned bal = __ballot_sync(0xffffffffu, flag);
+        const int before_in_warp = __popc(bal & ((1u << lane) - 1u));
+        if (lane == 0) warp_tot[warp] = __popc(bal);
+        __syncthreads();
+        int before = base_sh;
+        for (int w = 0; w < warp; ++w) before += warp_tot[w];
+        if (flag) idx[before + before_in_warp] = (int32_t)j;
+        __syncthreads();
+        if (t == 0) {
+            int s = 0;
+            for (int w = 0; w < kCompactThreads / 32; ++w) s += warp_tot[w];
+            base_sh += s;
+        }
+        __syncthreads();
+    }
+    const int n = base_sh;
+    if (t == 0) *n_out = n;
+    if (cached_n) {
+        const int cn = *cached_n;
+        if (cn != n) diff_sh = 1;
+        __syncthreads();
+        if (!diff_sh)
+            for (int o = t; o < n; o += kCompactThreads)
+                if (cached_idx[o] != idx[o]) diff_sh = 1;
+        __syncthreads();
+        const int d = diff_sh;
+        if (d) {
+            for (int o = t; o < n; o += kCompactThreads) cached_idx[o] = idx[o];
+            if (t == 0) *cached_n = n;
+        }
+        if (t == 0) *changed = d;
+    }
+}
+
+// Row-wise int8 over the columns not in O (zeros in O). When `only_if` is
+// given and *only_if == 0 the kernel does nothing.
+template <typename T>
+__global__ void __launch_bounds__(256)
+masked_quant_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, const int32_t* __restrict__ idx,
+                    const int32_t* __restrict__ n_idx, const int32_t* __restrict__ only_if, int8_t* __restrict__ Q,
+                    float* __restrict__ qs_out) {
+    extern __shared__ uint32_t mask[];  // K bits
+    __shared__ float sh[8];
+    if (only_if && *only_if == 0) return;
+    const int64_t words = (K + 31) / 32;
+    for (int64_t w = threadIdx.x; w < words; w += blockDim.x) mask[w] = 0u;
+    __syncthreads();
+    const int n = *n_idx;
+    for (int o = threadIdx.x; o < n; o += blockDim.x) {
+        const int j = idx[o];
+        atomicOr(&mask[j >> 5], 1u << (j & 31));
+    }
+    __syncthreads();
+    for (int64_t row = blockIdx.x; row < M; row += gridDim.x) {
+        const T* x = X + row * ld;
+        float m = 0.0f;
+        for (int64_t k0 = threadIdx.x * 8; k0 < K; k0 += 256 * 8) {
+            float f[8];
+            unpack<T>(ldg_v4(x + k0), f);
+            const uint32_t bits = (mask[k0 >> 5] >> (k0 & 31)) & 0xffu;
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                if (!((bits >> e) & 1u)) m = fmaxf(m, fabsf(f[e]));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        __syncthreads();
+        if ((threadIdx.x & 31) == 0) sh[threadIdx.x >> 5] = m;
+        __syncthreads();
+        float mm = sh[0];
+#pragma unroll
+        for (int w = 1; w < 8; ++w) mm = fmaxf(mm, sh[w]);
+        const float qs = __fdiv_rn(127.0f, fmaxf(mm, 1e-8f));
+        if (threadIdx.x == 0) qs_out[row] = qs;
+        int8_t* q = Q + row * K;
+        for (int64_t k0 = threadIdx.x * 8; k0 < K; k0 += 256 * 8) {
+            float f[8];
+            unpack<T>(ldg_v4(x + k0), f);
+            const uint32_t bits = (mask[k0 >> 5] >> (k0 & 31)) & 0xffu;
+            int c[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) c[e] = ((bits >> e) & 1u) ? 0 : quant_code(__fmul_rn(f[e], qs));
+            *reinterpret_cast<uint2*>(q + k0) = make_uint2(pack4_i8(c[0], c[1], c[2], c[3]), pack4_i8(c[4], c[5], c[6], c[7]));
+        }
+    }
+}
+
+sq_status_t launch_detect(const void* X, sq_dtype_t dt, int64_t M, int64_t K, int64_t ldx, float thr,
+                          double min_ratio, int32_t* idx, int32_t* n_out, int32_t* cached_idx, int32_t* cached_n,
+                          void* ws, cudaStream_t s) {
+    char* wsb = static_cast<char*>(ws);
+    int32_t* changed = reinterpret_cast<int32_t*>(wsb + 4);
+    int32_t* partial = reinterpret_cast<int32_t*>(wsb + kStatusBytes);
+    const int64_t rb = (M + kDetectRows - 1) / kDetectRows;
+    if (rb > 0) {
+        SQ_REQUIRE(rb <= 65535, SQ_ERR_UNSUPPORTED_SHAPE, "sq_llmint8_detect: M too large");
+        dim3 grid((unsigned)((K + 255) / 256), (unsigned)rb);
+        if (dt == SQ_BF16)
+            count_kernel<__nv_bfloat16><<<grid, kWarps * 32, 0, s>>>(static_cast<const __nv_bfloat16*>(X), M, K, ldx,
+                                                                      thr, partial);
+        else
+            count_kernel<__half><<<grid, kWarps * 32, 0, s>>>(static_cast<const __half*>(X), M, K, ldx, thr, partial);
+    }
+    compact_kernel<<<1, kCompactThreads, 0, s>>>(partial, rb, M, K, min_ratio, idx, n_out, cached_idx, cached_n,
+                                                 changed);
+    return check_launch("sq_llmint8_detect");
+}
+
+sq_status_t launch_masked_quant(const void* X, sq_dtype_t dt, int64_t M, int64_t K, int64_t ldx, const int32_t* idx,
+                                const int32_t* n_idx, const int32_t* only_if, int8_t* Q, float* qs, cudaStream_t s,
+                                const char* name) {
+    const size_t smem = (size_t)((K + 31) / 32) * 4;
+    int64_t grid = (int64_t)num_sms() * 8;
+    if (grid > M) grid = M;
+    if (grid < 1) return SQ_OK;
+    if (dt == SQ_BF16) {
+        auto k = masked_quant_kernel<__nv_bfloat16>;
+        if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        k<<<(unsigned)grid, 256, smem, s>>>(static_cast<const __nv_bfloat16*>(X), M, K, ldx, idx, n_idx, only_if, Q, qs);
+    } else {
+        auto k = masked_quant_kernel<__half>;
+        if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        k<<<(unsigned)grid, 256, smem, s>>>(static_cast<const __half*>(X), M, K, ldx, idx, n_idx, only_if, Q, qs);
+    }
+    return check_launch(name);
+}
+
+sq_status_t check_x(const char* name, const void* X, sq_dtype_t dt, int64_t M, int64_t K, int64_t ldx) {
+    SQ_REQUIRE(X, SQ_ERR_INVALID_ARG, "%s: null input", name);
+    SQ_REQUIRE(dt == SQ_F16 || dt == SQ_BF16, SQ_ERR_INVALID_ARG, "%s: dtype must be F16 or BF16", name);
+    SQ_REQUIRE(M >= 0 && K > 0 && ldx >= K && K % 8 == 0 && ldx % 8 == 0, SQ_ERR_UNSUPPORTED_SHAPE,
+               "%s: need K > 0, K %% 8 == 0, ldx >= K, ldx %% 8 == 0", name);
+    SQ_REQUIRE(K <= (1 << 20), SQ_ERR_UNSUPPORTED_SHAPE, "%s: K too large", name);
+    SQ_REQUIRE(aligned16(X), SQ_ERR_ALIGNMENT, "%s: input not 16-byte aligned", name);
+    return SQ_OK;
+}
+
+}  // namespace
+}  // namespace sq
+
+extern "C" {
+
+sq_status_t sq_llmint8_detect(const void* X, sq_dtype_t dt, int64_t M, int64_t K, int64_t ldx, float threshold,
+                              double min_ratio, int32_t* outlier_idx, int32_t* n_outliers, void* workspace,
+                              size_t ws_bytes, sq_stream_t stream) {
+    const char* name = "sq_llmint8_detect";
+    sq_status_t st = sq::check_x(name, X, dt, M, K, ldx);
+    if (st != SQ_OK) return st;
+    SQ_REQUIRE(outlier_idx && n_outliers, SQ_ERR_INVALID_ARG, "%s: null output", name);
+    SQ_REQUIRE(min_ratio >= 0.0 && threshold >= 0.0f, SQ_ERR_INVALID_ARG, "%s: threshold and min_ratio must be >= 0",
+               name);
+    SQ_REQUIRE(workspace && ws_bytes >= sq::detect_workspace_bytes(M, K), SQ_ERR_INVALID_ARG,
+               "%s: needs a workspace of %zu bytes", name, sq::detect_workspace_bytes(M, K));
+    return sq::launch_detect(X, dt, M, K, ldx, threshold, min_ratio, outlier_idx, n_outliers, nullptr, nullptr,
+                             workspace, sq::as_cuda(stream));
+}
+
+sq_status_t sq_llmint8_quant_rows(const void* X, sq_dtype_t dt, int64_t M, int64_t K, int64_t ldx,
+                                  const int32_t* idx, const int32_t* n_idx, int8_t* Xq, float* qs_x,
+                                  sq_stream_t stream) {
+    const char* name = "sq_llmint8_quant_rows";
+    sq_status_t st = sq::check_x(name, X, dt, M, K, ldx);
+    if (st != SQ_OK) return st;
+    SQ_REQUIRE(idx && n_idx && Xq && qs_x, SQ_ERR_INVALID_ARG, "%s: null pointer", name);
+    SQ_REQUIRE(sq::aligned16(Xq), SQ_ERR_ALIGNMENT, "%s: Xq not 16-byte aligned", name);
+    if (M == 0) return SQ_OK;
+    return sq::launch_masked_quant(X, dt, M, K, ldx, idx, n_idx, nullptr, Xq, qs_x, sq::as_cuda(stream), name);
+}
+
+sq_status_t sq_llmint8_quant_weight(const void* W, sq_dtype_t dt, int64_t N, int64_t K, const int32_t* idx,
+                                    const int32_t* n_idx, int8_t* Wq, float* qs_w, sq_stream_t stream) {
+    const char* name = "sq_llmint8_quant_weight";
+    sq_status_t st = sq::check_x(name, W, dt, N, K, K);
+    if (st != SQ_OK) return st;
+    SQ_REQUIRE(idx && n_idx && Wq && qs_w, SQ_ERR_INVALID_ARG, "%s: null pointer", name);
+    SQ_REQUIRE(sq::aligned16(Wq), SQ_ERR_ALIGNMENT, "%s: Wq not 16-byte aligned", name);
+    if (N == 0) return SQ_OK;
+    return sq::launch_masked_quant(W, dt, N, K, K, idx, n_idx, nullptr, Wq, qs_w, sq::as_cuda(stream), name);
+}
+
+sq_status_t sq_llmint8_matmul(const void* X, sq_dtype_t dt, int64_t M, int64_t K, int64_t ldx,
+                              const sq_llmint8_weight_t* w, float threshold, double min_ratio, void* Y, int64_t ldy,
+                              int32_t* idx_out, int32_t* n_out, void* workspace, size_t ws_bytes,
+                              sq_stream_t stream) {
+    const char* name = "sq_llmint8_matmul";
+    sq_status_t st = sq::check_x(name, X, dt, M, K, ldx);
+    if (st != SQ_OK) return st;
+    SQ_REQUIRE(w && w->W && w->Wq && w->qs_w && w->cached_idx && w->cached_n, SQ_ERR_INVALID_ARG,
+               "%s: incomplete weight state", name);
+    SQ_REQUIRE(Y && idx_out && n_out, SQ_ERR_INVALID_ARG, "%s: null output", name);
+    SQ_REQUIRE(w->N > 0 && ldy >= w->N, SQ_ERR_UNSUPPORTED_SHAPE, "%s: need N > 0 and ldy >= N", name);
+    SQ_REQUIRE(K % 16 == 0 && K <= 133144, SQ_ERR_UNSUPPORTED_SHAPE, "%s: K must be a multiple of 16, <= 133144",
+               name);
+    SQ_REQUIRE(M < (1ll << 31) && w->N < (1ll << 31), SQ_ERR_UNSUPPORTED_SHAPE, "%s: M and N must be < 2^31", name);
+    SQ_REQUIRE(sq::aligned16(w->W) && sq::aligned16(w->Wq), SQ_ERR_ALIGNMENT, "%s: weights not 16-byte aligned", name);
+    const size_t need = sq::llmint8_workspace_bytes(M, K);
+    SQ_REQUIRE(workspace && ws_bytes >= need, SQ_ERR_INVALID_ARG, "%s: needs a workspace of %zu bytes", name, need);
+    cudaStream_t s = sq::as_cuda(stream);
+    char* wsb = static_cast<char*>(workspace);
+    const size_t det = sq::detect_workspace_bytes(M, K);
+    int8_t* Xq = reinterpret_cast<int8_t*>(wsb + det);
+    float* qs_x = reinterpret_cast<float*>(wsb + det + ((size_t)M * K + 255) / 256 * 256);
+    int32_t* changed = reinterpret_cast<int32_t*>(wsb + 4);
+    // a7: O, and whether the cached int8 weight was built for it
+    st = sq::launch_detect(X, dt, M, K, ldx, threshold, min_ratio, idx_out, n_out, w->cached_idx, w->cached_n, workspace,
+                           s);
+    if (st != SQ_OK) return st;
+    // weight side for O (returns at once when O is unchanged)
+    st = sq::launch_masked_quant(w->W, dt, w->N, K, K, idx_out, n_out, changed, w->Wq, w->qs_w, s, name);
+    if (st != SQ_OK) return st;
+    if (M == 0) return SQ_OK;
+    // a8
+    st = sq::launch_masked_quant(X, dt, M, K, ldx, idx_out, n_out, nullptr, Xq, qs_x, s, name);
+    if (st != SQ_OK) return st;
+    // a9: int8 GEMM + 16-bit outlier term in the epilogue
+    sq::GemmEpilogue ep;
+    ep.qs_x = qs_x;
+    ep.x_per_token = 1;
+    ep.qs_w = w->qs_w;
+    ep.w_per_channel = 1;
+    ep.out_dt = dt;
+    ep.Y = Y;
+    ep.ldy = ldy;
+    ep.x16 = X;
+    ep.ldx16 = ldx;
+    ep.w16 = w->W;
+    ep.idx = idx_out;
+    ep.n_out = n_out;
+    ep.in16_bf16 = dt == SQ_BF16;
+    return sq::launch_gemm_w8a8(Xq, w->Wq, M, w->N, K, ep, static_cast<int*>(workspace), s);
+}
+
+}  // extern "C"

@@ -1,0 +1,229 @@
+// a4 / a5': symmetric absmax int8 quantisation of weights and of activations
+// that do not come out of a norm.
+//
+// "8位量化：异常值与混合精度分解实战" §2.1: scale = 127 / max(|x|, 1e-8) over the
+// quantisation group, q = clip(round(x * scale), -127, 127), round half to
+// even. Groups are one row (a token of X, an output channel of W) or the
+// whole tensor: these are the only granularities whose scales factor out of
+// the GEMM ("大语言模型量化技术（四）：SmoothQuant", 为什么激活不能用逐通道量化).
+// The weight is smoothed on the fly, W' = fp32(W) * s_k (section SmoothQuant
+// 的原理); the activation is divided by s, X' = X / s ("如何通过 SmoothQuant
+// 解决激活值离群点难题" §3). All arithmetic is fp32 with correctly rounded
+// operations, so codes and scales are bit-exact against a plain CPU loop.
+//
+// Row mode: one 256-thread block per row, the row read twice (the second read
+// hits L1/L2): pass 1 reduces max |v|, pass 2 writes the codes. Tensor mode:
+// a grid-wide absmax into the workspace, then the quantising pass.
+#include "sq_common.cuh"
+#include "sq_internal.h"
+
+namespace sq {
+namespace {
+
+constexpr int kThreads = 256;
+enum SMode { kNoScale = 0, kMul = 1, kDiv = 2 };
+
+// Load 8 consecutive elements as fp32.
+template <typename T>
+__device__ __forceinline__ void load8(const T* p, float* f) {
+    if constexpr (sizeof(T) == 2) {
+        unpack<T>(ldg_v4(p), f);
+    } else {
+        unpack<float>(ldg_v4(p), f);
+        unpack<float>(ldg_v4(p + 4), f + 4);
+    }
+}
+
+template <int SM>
+__device__ __forceinline__ void apply_s(float* f, const float* __restrict__ s, int64_t k0) {
+    if constexpr (SM != kNoScale) {
+        const float4 a = *reinterpret_cast<const float4*>(s + k0);
+        const float4 b = *reinterpret_cast<const float4*>(s + k0 + 4);
+        const float sv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) f[e] = SM == kMul ? __fmul_rn(f[e], sv[e]) : __fdiv_rn(f[e], sv[e]);
+    }
+}
+
+__device__ __forceinline__ float block_max(float v, float* sh) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    __syncthreads();  // sh may still be read from a previous use
+    if (lane == 0) sh[warp] = v;
+    __syncthreads();
+    float m = sh[0];
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, sh[w]);
+    return m;
+}
+
+__device__ __forceinline__ float scale_of(float m) { return __fdiv_rn(127.0f, fmaxf(m, 1e-8f)); }
+
+__device__ __forceinline__ uint2 codes8(const float* v, float qs) {
+    int q[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) q[e] = quant_code(__fmul_rn(v[e], qs));
+    return make_uint2(pack4_i8(q[0], q[1], q[2], q[3]), pack4_i8(q[4], q[5], q[6], q[7]));
+}
+
+// per_row != 0: scale per row from the row's absmax; else *tensor_qs for all.
+template <typename T, int SM>
+__global__ void __launch_bounds__(kThreads)
+row_quant_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, const float* __restrict__ s,
+                 int per_row, const float* __restrict__ tensor_qs, int8_t* __restrict__ Q,
+                 float* __restrict__ qs_out) {
+    __shared__ float sh[kThreads / 32];
+    for (int64_t row = blockIdx.x; row < M; row += gridDim.x) {
+        const T* x = X + row * ld;
+        float qs;
+        if (per_row) {
+            float m = 0.0f;
+            for (int64_t k0 = threadIdx.x * 8; k0 < K; k0 += kThreads * 8) {
+                float f[8];
+                load8<T>(x + k0, f);
+                apply_s<SM>(f, s, k0);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(f[e]));
+            }
+            m = block_max(m, sh);
+            qs = scale_of(m);
+            if (threadIdx.x == 0) qs_out[row] = qs;
+        } else {
+            qs = *tensor_qs;
+            if (row == 0 && threadIdx.x == 0) qs_out[0] = qs;
+        }
+        int8_t* q = Q + row * K;
+        for (int64_t k0 = threadIdx.x * 8; k0 < K; k0 += kThreads * 8) {
+            float f[8];
+            load8<T>(x + k0, f);
+            apply_s<SM>(f, s, k0);
+            *reinterpret_cast<uint2*>(q + k0) = codes8(f, qs);
+        }
+    }
+}
+
+// Grid-wide max |v| over the tensor into *out (non-negative float bits).
+template <typename T, int SM>
+__global__ void __launch_bounds__(kThreads)
+tensor_absmax_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld,
+                     const float* __restrict__ s, float* __restrict__ out) {
+    __shared__ float sh[kThreads / 32];
+    const int64_t vecs_per_row = K / 8;
+    const int64_t nvec = M * vecs_per_row;
+    float m = 0.0f;
+    for (int64_t v = blockIdx.x * (int64_t)kThreads + threadIdx.x; v < nvec; v += (int64_t)gridDim.x * kThreads) {
+        const int64_t row = v / vecs_per_row;
+        const int64_t k0 = (v - row * vecs_per_row) * 8;
+        float f[8];
+        load8<T>(X + row * ld + k0, f);
+        apply_s<SM>(f, s, k0);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(f[e]));
+    }
+    m = block_max(m, sh);
+    if (threadIdx.x == 0) atomic_max_nonneg(out, m);
+}
+
+// qs = 127 / max(max_j a[j], 1e-8) into *qs (one block).
+__global__ void __launch_bounds__(kThreads)
+scale_from_absmax_kernel(const float* __restrict__ a, int64_t n, float* __restrict__ qs) {
+    __shared__ float sh[kThreads / 32];
+    float m = 0.0f;
+    for (int64_t j = threadIdx.x; j < n; j += kThreads) m = fmaxf(m, a[j]);
+    m = block_max(m, sh);
+    if (threadIdx.x == 0) *qs = scale_of(m);
+}
+
+int row_grid(int64_t M) {
+    const int64_t cap = (int64_t)num_sms() * 8;
+    return (int)(M < cap ? M : cap);
+}
+
+int vec_grid(int64_t nvec) {
+    int64_t b = (nvec + kThreads - 1) / kThreads;
+    const int64_t cap = (int64_t)num_sms() * 8;
+    return (int)(b < 1 ? 1 : (b > cap ? cap : b));
+}
+
+template <typename T, int SM>
+sq_status_t quantize(const void* Xv, int64_t M, int64_t K, int64_t ld, const float* s, int per_row,
+                     const float* static_qs, int8_t* Q, float* qs_out, void* ws, cudaStream_t st,
+                     const char* name) {
+    const T* X = static_cast<const T*>(Xv);
+    const float* tensor_qs = static_qs;
+    if (!per_row && !static_qs) {
+        // grid-wide absmax into the workspace, then qs from it
+        float* wmax = reinterpret_cast<float*>(static_cast<char*>(ws) + 16);
+        float* wqs = wmax + 1;
+        if (cudaMemsetAsync(wmax, 0, sizeof(float), st) != cudaSuccess) return check_launch(name);
+        tensor_absmax_kernel<T, SM><<<vec_grid(M * K / 8), kThreads, 0, st>>>(X, M, K, ld, s, wmax);
+        scale_from_absmax_kernel<<<1, kThreads, 0, st>>>(wmax, 1, wqs);
+        tensor_qs = wqs;
+    }
+    row_quant_kernel<T, SM><<<row_grid(M), kThreads, 0, st>>>(X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
+    return check_launch(name);
+}
+
+template <int SM>
+sq_status_t quantize_dt(sq_dtype_t dt, const void* X, int64_t M, int64_t K, int64_t ld, const float* s,
+                        int per_row, const float* static_qs, int8_t* Q, float* qs_out, void* ws,
+                        cudaStream_t st, const char* name) {
+    switch (dt) {
+        case SQ_F16: return quantize<__half, SM>(X, M, K, ld, s, per_row, static_qs, Q, qs_out, ws, st, name);
+        case SQ_BF16:
+            return quantize<__nv_bfloat16, SM>(X, M, K, ld, s, per_row, static_qs, Q, qs_out, ws, st, name);
+        case SQ_F32: return quantize<float, SM>(X, M, K, ld, s, per_row, static_qs, Q, qs_out, ws, st, name);
+        default: return set_error(SQ_ERR_INVALID_ARG, "%s: dtype must be F16, BF16 or F32", name);
+    }
+}
+
+}  // namespace
+}  // namespace sq
+
+extern "C" {
+
+sq_status_t sq_quantize_weight(const void* W, sq_dtype_t dt, int64_t N, int64_t K, const float* s,
+                               int per_channel, int8_t* Wq, float* qs_w, void* workspace, size_t ws_bytes,
+                               sq_stream_t stream) {
+    const char* name = "sq_quantize_weight";
+    SQ_REQUIRE(W && Wq && qs_w, SQ_ERR_INVALID_ARG, "%s: null pointer", name);
+    SQ_REQUIRE(N >= 0 && K > 0 && K % 16 == 0, SQ_ERR_UNSUPPORTED_SHAPE, "%s: need K > 0 and K %% 16 == 0", name);
+    SQ_REQUIRE(sq::aligned16(W) && sq::aligned16(Wq) && (!s || sq::aligned16(s)), SQ_ERR_ALIGNMENT,
+               "%s: W, Wq and s must be 16-byte aligned", name);
+    SQ_REQUIRE(per_channel || (workspace && ws_bytes >= sq::kStatusBytes), SQ_ERR_INVALID_ARG,
+               "%s: per-tensor quantisation needs a workspace of %zu bytes", name, sq::kStatusBytes);
+    if (N == 0) return SQ_OK;
+    cudaStream_t st = sq::as_cuda(stream);
+    if (s)
+        return sq::quantize_dt<sq::kMul>(dt, W, N, K, K, s, per_channel, nullptr, Wq, qs_w, workspace, st, name);
+    return sq::quantize_dt<sq::kNoScale>(dt, W, N, K, K, nullptr, per_channel, nullptr, Wq, qs_w, workspace, st,
+                                         name);
+}
+
+sq_status_t sq_quantize_act(const void* X, sq_dtype_t dt, int64_t M, int64_t K, int64_t ldx, const float* s,
+                            int per_token, const float* static_qs, int8_t* Xq, float* qs_x, void* workspace,
+                            size_t ws_bytes, sq_stream_t stream) {
+    const char* name = "sq_quantize_act";
+    SQ_REQUIRE(X && Xq && qs_x, SQ_ERR_INVALID_ARG, "%s: null pointer", name);
+    SQ_REQUIRE(M >= 0 && K > 0 && K % 16 == 0 && ldx >= K && ldx % 8 == 0, SQ_ERR_UNSUPPORTED_SHAPE,
+               "%s: need K > 0, K %% 16 == 0, ldx >= K, ldx %% 8 == 0", name);
+    SQ_REQUIRE(sq::aligned16(X) && sq::aligned16(Xq) && (!s || sq::aligned16(s)), SQ_ERR_ALIGNMENT,
+               "%s: X, Xq and s must be 16-byte aligned", name);
+    SQ_REQUIRE(per_token || static_qs || (workspace && ws_bytes >= sq::kStatusBytes), SQ_ERR_INVALID_ARG,
+               "%s: dynamic per-tensor quantisation needs a workspace of %zu bytes", name, sq::kStatusBytes);
+    if (M == 0) return SQ_OK;
+    cudaStream_t st = sq::as_cuda(stream);
+    if (s)
+        return sq::quantize_dt<sq::kDiv>(dt, X, M, K, ldx, s, per_token, static_qs, Xq, qs_x, workspace, st, name);
+    return sq::quantize_dt<sq::kNoScale>(dt, X, M, K, ldx, nullptr, per_token, static_qs, Xq, qs_x, workspace, st,
+                                         name);
+}
+
+sq_status_t sq_scale_from_absmax(const float* absmax, int64_t n, float* qs_out, sq_stream_t stream) {
+    SQ_REQUIRE(absmax && qs_out, SQ_ERR_INVALID_ARG, "sq_scale_from_absmax: null pointer");
+    SQ_REQUIRE(n > 0, SQ_ERR_UNSUPPORTED_SHAPE, "sq_scale_from_absmax: n must be > 0");
+    sq::scale_from_absmax_kernel<<<1, sq::kThreads, 0, sq::as_cuda(stream)>>>(absmax, n, qs_out);
+    return sq::check_launch("sq_scale_from_absmax");
+}
+
+}  // extern "C"

@@ -1,0 +1,129 @@
+// Internal helpers shared by the CUDA translation units of the library.
+// Host side: status/error reporting and argument checks. Device side: 16-byte
+// vector loads, 16-bit <-> fp32 conversion, and the int8 rounding step.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <cstdarg>
+#include <cstdio>
+
+#include "../../include/sq_api.h"
+
+namespace sq {
+
+// ----------------------------------------------------------------- host side
+sq_status_t set_error(sq_status_t st, const char* fmt, ...);
+sq_status_t check_launch(const char* what);
+
+inline cudaStream_t as_cuda(sq_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline int dtype_bytes(sq_dtype_t dt) {
+    switch (dt) {
+        case SQ_F32: return 4;
+        case SQ_F16: return 2;
+        case SQ_BF16: return 2;
+        case SQ_I32: return 4;
+        case SQ_I8: return 1;
+    }
+    return 0;
+}
+
+int num_sms();  // SM count of the current device (cached per device)
+
+#define SQ_REQUIRE(cond, status, ...) \
+    do {                              \
+        if (!(cond)) return ::sq::set_error(status, __VA_ARGS__); \
+    } while (0)
+
+// ---------------------------------------------------------------- device side
+// Element count of one 16-byte vector.
+template <typename T> struct Vec;
+template <> struct Vec<__half> { static constexpr int N = 8; };
+template <> struct Vec<__nv_bfloat16> { static constexpr int N = 8; };
+template <> struct Vec<float> { static constexpr int N = 4; };
+
+__device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ uint4 ldg_v4(const void* p) {
+    return *reinterpret_cast<const uint4*>(p);
+}
+
+// Unpack a 16-byte vector into fp32 (exact for 16-bit sources).
+template <typename T>
+__device__ __forceinline__ void unpack(const uint4& r, float* f);
+
+template <>
+__device__ __forceinline__ void unpack<__nv_bfloat16>(const uint4& r, float* f) {
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+
+template <>
+__device__ __forceinline__ void unpack<__half>(const uint4& r, float* f) {
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        __half2 h = *reinterpret_cast<const __half2*>(&w[i]);
+        float2 v = __half22float2(h);
+        f[2 * i] = v.x;
+        f[2 * i + 1] = v.y;
+    }
+}
+
+template <>
+__device__ __forceinline__ void unpack<float>(const uint4& r, float* f) {
+    f[0] = __uint_as_float(r.x);
+    f[1] = __uint_as_float(r.y);
+    f[2] = __uint_as_float(r.z);
+    f[3] = __uint_as_float(r.w);
+}
+
+// fp32 -> 16-bit, round to nearest even.
+template <typename T> __device__ __forceinline__ uint16_t to16(float v);
+template <> __device__ __forceinline__ uint16_t to16<__nv_bfloat16>(float v) {
+    __nv_bfloat16 b = __float2bfloat16_rn(v);
+    return *reinterpret_cast<uint16_t*>(&b);
+}
+template <> __device__ __forceinline__ uint16_t to16<__half>(float v) {
+    __half h = __float2half_rn(v);
+    return *reinterpret_cast<uint16_t*>(&h);
+}
+
+// int8 code of t: clip to [-127, 127], then round half to even. Clipping
+// first gives the same code as rounding first (127.5 -> 127 either way) and
+// keeps |t| small enough for the 1.5 * 2^23 shifter: in [2^23, 2^24) fp32
+// values are consecutive integers, so one RN add rounds t to an integer
+// (ties to even, because the shifter is even) and the low bits hold it.
+__device__ __forceinline__ int quant_code(float t) {
+    t = fminf(fmaxf(t, -127.0f), 127.0f);
+    float r = __fadd_rn(t, 12582912.0f);
+    return __float_as_int(r) - 0x4B400000;
+}
+
+// max on non-negative floats through their bit patterns (monotone for >= 0).
+__device__ __forceinline__ void atomic_max_nonneg(float* addr, float v) {
+    atomicMax(reinterpret_cast<int*>(addr), __float_as_int(v));
+}
+
+__device__ __forceinline__ uint32_t pack4_i8(int a, int b, int c, int d) {
+    return (uint32_t(a) & 0xffu) | ((uint32_t(b) & 0xffu) << 8) | ((uint32_t(c) & 0xffu) << 16) |
+           ((uint32_t(d) & 0xffu) << 24);
+}
+
+}  // namespace sq

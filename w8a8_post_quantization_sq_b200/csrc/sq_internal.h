@@ -1,0 +1,43 @@
+// Declarations shared between the library's translation units (not public).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/sq_api.h"
+
+namespace sq {
+
+// Every workspace-taking operation keeps a 256-byte header; word 0 is the
+// status word written by bounded device waits (0 = fine).
+constexpr size_t kStatusBytes = 256;
+
+// Rows per block of the outlier-count pass of sq_llmint8_detect.
+constexpr int kDetectRows = 128;
+size_t detect_workspace_bytes(int64_t M, int64_t K);
+size_t llmint8_workspace_bytes(int64_t M, int64_t K);
+
+// Epilogue description of the int8 GEMM.
+struct GemmEpilogue {
+    const float* qs_x = nullptr;
+    int x_per_token = 0;
+    const float* qs_w = nullptr;
+    int w_per_channel = 0;
+    const float* bias = nullptr;
+    sq_dtype_t out_dt = SQ_BF16;
+    void* Y = nullptr;
+    int64_t ldy = 0;
+    // LLM.int8 16-bit outlier term: sum over o < *n_out of
+    // X16[i, idx[o]] * W16[j, idx[o]] (null idx = no outlier term).
+    const void* x16 = nullptr;
+    int64_t ldx16 = 0;
+    const void* w16 = nullptr;
+    const int32_t* idx = nullptr;
+    const int32_t* n_out = nullptr;
+    int in16_bf16 = 0;
+};
+
+sq_status_t launch_gemm_w8a8(const int8_t* Xq, const int8_t* Wq, int64_t M, int64_t N, int64_t K,
+                             const GemmEpilogue& ep, int* status_word, cudaStream_t stream);
+
+}  // namespace sq

@@ -1,0 +1,80 @@
+// Host-side status handling, workspace sizing and device queries.
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "sq_common.cuh"
+#include "sq_internal.h"
+
+namespace sq {
+
+static thread_local std::string g_last_error;
+
+sq_status_t set_error(sq_status_t st, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return st;
+}
+
+sq_status_t check_launch(const char* what) {
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return set_error(SQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+    return SQ_OK;
+}
+
+int num_sms() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cache[dev] == 0) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        cache[dev] = n > 0 ? n : 148;
+    }
+    return cache[dev];
+}
+
+}  // namespace sq
+
+extern "C" {
+
+const char* sq_last_error_string(void) { return sq::g_last_error.c_str(); }
+
+int sq_version(void) { return 100; }
+
+size_t sq_workspace_size(sq_op_t op, int64_t M, int64_t N, int64_t K) {
+    (void)N;
+    switch (op) {
+        case SQ_OP_GEMM: return sq::kStatusBytes;
+        case SQ_OP_QUANT_ACT: return sq::kStatusBytes;
+        case SQ_OP_QUANT_WEIGHT: return sq::kStatusBytes;
+        case SQ_OP_LLMINT8_DETECT: return sq::detect_workspace_bytes(M, K);
+        case SQ_OP_LLMINT8: return sq::llmint8_workspace_bytes(M, K);
+    }
+    return 0;
+}
+
+sq_status_t sq_workspace_status(void* workspace, sq_stream_t stream) {
+    SQ_REQUIRE(workspace != nullptr, SQ_ERR_INVALID_ARG, "sq_workspace_status: null workspace");
+    cudaStream_t s = sq::as_cuda(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess)
+        return sq::set_error(SQ_ERR_CUDA, "sq_workspace_status: %s",
+                             cudaGetErrorString(cudaGetLastError()));
+    int word = 0;
+    if (cudaMemcpy(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return sq::set_error(SQ_ERR_CUDA, "sq_workspace_status: copy failed");
+    if (word != 0) {
+        int zero = 0;
+        cudaMemcpy(workspace, &zero, sizeof(int), cudaMemcpyHostToDevice);
+        return sq::set_error(SQ_ERR_TIMEOUT,
+                             "a bounded device wait timed out (code %d); results of that call are invalid",
+                             word);
+    }
+    return SQ_OK;
+}
+
+}  // extern "C"
