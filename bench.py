@@ -354,8 +354,90 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ single kernels
+def run_kernel(args):
+    """Time one entry point alone on one shape (L2 flushed between launches):
+    gemm M,N,K | norm M,K | absmax M,K | quant_weight N,K | llmint8 M,K,N."""
+    import torch
+
+    import w8a8_post_quantization_sq_b200 as sq
+    from w8a8_post_quantization_sq_b200 import build
+
+    build.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    shape = [int(x) for x in args.shape.split(",")]
+    g = torch.Generator(device=dev).manual_seed(0)
+    pk, src = peaks()
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    out = {"kernel": args.kernel, "shape": shape}
+    if args.kernel == "gemm":
+        M, N, K = shape
+        Xq = torch.randint(-127, 128, (M, K), generator=g, device=dev, dtype=torch.int8)
+        Wq = torch.randint(-127, 128, (N, K), generator=g, device=dev, dtype=torch.int8)
+        qx = torch.rand(M, generator=g, device=dev) + 1
+        qw = torch.rand(N, generator=g, device=dev) + 100
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        ws = sq.workspace(sq.SQ_OP_GEMM, M, N, K, device=dev)
+        fn = lambda: sq.sq_gemm_w8a8(Xq, Wq, qx, qw, None, Y, ws)  # noqa: E731
+        work, unit, peak = 2.0 * M * N * K / 1e12, "TOPS", 2.0 * pk["bf16_tflops"]
+    elif args.kernel == "norm":
+        M, K = shape
+        H = torch.randn((M, K), generator=g, device=dev).to(torch.bfloat16)
+        gamma = torch.rand(K, generator=g, device=dev) + 0.5
+        Xq = torch.empty((M, K), dtype=torch.int8, device=dev)
+        qs = torch.empty(M, device=dev)
+        fn = lambda: sq.sq_norm_smooth_quant(H, sq.SQ_RMSNORM, gamma, None, 1e-6, True, None, Xq, qs)  # noqa: E731
+        work, unit, peak = (3.0 * M * K + 4 * M) / 1e9, "GB/s", pk["hbm_gbs"]
+    elif args.kernel == "absmax":
+        M, K = shape
+        X = torch.randn((M, K), generator=g, device=dev).to(torch.bfloat16)
+        xmax = torch.zeros(K, device=dev)
+        fn = lambda: sq.sq_calib_absmax(X, xmax)  # noqa: E731
+        work, unit, peak = 2.0 * M * K / 1e9, "GB/s", pk["hbm_gbs"]
+    elif args.kernel == "quant_weight":
+        N, K = shape
+        W = (torch.randn((N, K), generator=g, device=dev) * 0.02).to(torch.bfloat16)
+        s_ = torch.rand(K, generator=g, device=dev) * 10 + 0.1
+        Wq = torch.empty((N, K), dtype=torch.int8, device=dev)
+        qw = torch.empty(N, device=dev)
+        fn = lambda: sq.sq_quantize_weight(W, s_, True, Wq, qw)  # noqa: E731
+        work, unit, peak = (3.0 * N * K + 4 * N) / 1e9, "GB/s", pk["hbm_gbs"]
+    elif args.kernel == "llmint8":
+        from w8a8_post_quantization_sq_b200 import inputs
+
+        M, K, N = shape
+        d = inputs.c4_llmint8(device=dev, M=M, K=K, N=N)
+        st = sq.llmint8_weight_state(d["W"])
+        Y = torch.empty((M, N), dtype=torch.float16, device=dev)
+        idx = torch.empty(K, dtype=torch.int32, device=dev)
+        n = torch.empty(1, dtype=torch.int32, device=dev)
+        ws = sq.workspace(sq.SQ_OP_LLMINT8, M, N, K, device=dev)
+        fn = lambda: sq.sq_llmint8_matmul(d["X"], st, 6.0, 0.0, Y, idx, n, ws)  # noqa: E731
+        work, unit, peak = 2.0 * M * N * K / 1e12, "TOPS", 2.0 * pk["bf16_tflops"]
+    else:
+        raise SystemExit(f"unknown kernel {args.kernel}")
+    for _ in range(max(args.warmup, 3)):
+        fn()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for a, b in ev:
+        flush.fill_(1)
+        a.record()
+        fn()
+        b.record()
+    torch.cuda.synchronize()
+    ms = [a.elapsed_time(b) for a, b in ev]
+    avg = sum(ms) / len(ms)
+    out.update({"avg_us": avg * 1e3, "min_us": min(ms) * 1e3, "achieved": work / (avg * 1e-3), "unit": unit,
+                "peak": peak, "frac": work / (avg * 1e-3) / peak, "peak_source": src})
+    print(json.dumps(out), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
+    ap.add_argument("--kernel", default=None, help="time one entry point alone: gemm|norm|absmax|quant_weight|llmint8")
+    ap.add_argument("--shape", default="4096,36864,12288")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
@@ -363,6 +445,9 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=256, help="token rows of the CPU baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
+    if args.kernel:
+        run_kernel(args)
+        return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -139,8 +139,9 @@ def test_fold_weight_and_norm():
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16, torch.float32])
 @pytest.mark.parametrize("per_channel", [True, False])
 @pytest.mark.parametrize("with_s", [True, False])
-def test_quantize_weight(dtype, per_channel, with_s):
-    N, K = 517, 2064
+@pytest.mark.parametrize("K", [1024, 2064, 12288, 20480])
+def test_quantize_weight(dtype, per_channel, with_s, K):
+    N = 517 if K <= 2064 else 131
     W = rnd((N, K), 10, dtype, 0.02)
     s = torch.rand(K, generator=torch.Generator().manual_seed(11)) * 30 + 0.05 if with_s else None
     Wq = torch.empty((N, K), dtype=torch.int8, device=DEV)
@@ -156,8 +157,9 @@ def test_quantize_weight(dtype, per_channel, with_s):
 # ---------------------------------------------------------------- a5'
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16, torch.float32])
 @pytest.mark.parametrize("mode", ["token", "tensor_dynamic", "tensor_static"])
-def test_quantize_act(dtype, mode):
-    M, K = 77, 1040
+@pytest.mark.parametrize("K", [256, 1040, 4096, 16400])
+def test_quantize_act(dtype, mode, K):
+    M = 77
     X = rnd((M, K), 12, dtype)
     X[:, 5] *= 50
     s = torch.rand(K, generator=torch.Generator().manual_seed(13)) * 8 + 0.1
@@ -217,10 +219,11 @@ def test_norm_smooth_quant_per_token(dtype, norm, K):
 
 
 @pytest.mark.parametrize("norm", ["ln", "rms"])
-def test_norm_static_and_calibration(norm):
+@pytest.mark.parametrize("K", [1024, 7168])
+def test_norm_static_and_calibration(norm, K):
     """Calibration mode (running per-channel max of |v| over batches) and the
     static per-tensor scale taken from it, the OPT-30B-style path."""
-    M, K = 200, 7168
+    M = 200
     nt = sq.SQ_LAYERNORM if norm == "ln" else sq.SQ_RMSNORM
     on = oracle.LAYERNORM if norm == "ln" else oracle.RMSNORM
     gamma = 1 + 0.1 * rnd(K, 3)

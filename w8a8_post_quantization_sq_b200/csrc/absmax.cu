@@ -74,9 +74,12 @@ sq_status_t launch(const void* X, int64_t M, int64_t K, int64_t ld, float* out, 
                    const char* name) {
     constexpr int COLS = 32 * Vec<T>::N;
     const int64_t col_blocks = (K + COLS - 1) / COLS;
-    // about 8 blocks per SM in one wave; rows per block a multiple of the warp count
+    // one full wave of about 8 blocks per SM: as many row bands as fit beside
+    // the column blocks; rows per band a multiple of the warp count
     const int64_t target = (int64_t)num_sms() * 8;
-    int64_t rpb = (M * col_blocks + target - 1) / target;
+    int64_t bands = target / col_blocks;
+    if (bands < 1) bands = 1;
+    int64_t rpb = (M + bands - 1) / bands;
     rpb = ((rpb + kWarps - 1) / kWarps) * kWarps;
     if (rpb < kWarps * kUnroll) rpb = kWarps * kUnroll;
     const int64_t row_blocks = (M + rpb - 1) / rpb;
@@ -89,7 +92,7 @@ sq_status_t launch(const void* X, int64_t M, int64_t K, int64_t ld, float* out, 
 
 sq_status_t col_absmax(const void* X, sq_dtype_t dt, int64_t M, int64_t K, int64_t ld, float* out,
                        sq_stream_t stream, const char* name) {
-    SQ_REQUIRE(X && out, SQ_ERR_INVALID_ARG, "%s: null pointer", name);
+    SQ_REQUIRE((X || M == 0) && out, SQ_ERR_INVALID_ARG, "%s: null pointer", name);
     SQ_REQUIRE(M >= 0 && K > 0 && ld >= K, SQ_ERR_UNSUPPORTED_SHAPE, "%s: bad sizes M=%lld K=%lld ld=%lld",
                name, (long long)M, (long long)K, (long long)ld);
     SQ_REQUIRE(dt == SQ_F16 || dt == SQ_BF16 || dt == SQ_F32, SQ_ERR_INVALID_ARG, "%s: dtype must be F16, BF16 or F32",

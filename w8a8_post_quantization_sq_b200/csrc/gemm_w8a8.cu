@@ -40,6 +40,11 @@ constexpr int UMMA_K = 32;
 constexpr int STAGES = 4;
 constexpr int kThreads = 192;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
+// staging row strides: 64 B (16-bit) / 128 B (32-bit) of data + 16 B pad
+constexpr int kStg16 = 80;
+constexpr int kStg32 = 144;
+constexpr int kStgWarpBytes = 32 * kStg32;
+enum OutKind { kOutBF16 = 0, kOutF16 = 1, kOutF32 = 2, kOutI32 = 3 };
 
 template <int BN>
 struct Cfg {
@@ -51,8 +56,13 @@ struct Cfg {
     // full[S], empty[S], tfull[2], tempty[2], drain
     static constexpr uint32_t NBAR = 2 * STAGES + 5;
     static constexpr uint32_t MISC_OFF = BAR_OFF + NBAR * 8;  // tmem base, abort flag
-    static constexpr uint32_t RW_OFF = (MISC_OFF + 16 + 15) / 16 * 16;  // 1/qs_w and bias of a tile
-    static constexpr uint32_t SMEM = RW_OFF + 4 * 2 * BN * 4;  // per epilogue warp
+    // per epilogue warp: 1/qs_w and bias of the tile's columns
+    static constexpr uint32_t RW_OFF = (MISC_OFF + 16 + 15) / 16 * 16;
+    static constexpr uint32_t RW_BYTES = 4 * 2 * BN * 4;
+    // per epilogue warp: a 32 x 32 output chunk (rows padded to avoid bank conflicts)
+    static constexpr uint32_t STG_OFF = RW_OFF + RW_BYTES;
+    static constexpr uint32_t STG_BYTES = 4 * kStgWarpBytes;
+    static constexpr uint32_t SMEM = STG_OFF + STG_BYTES;
     static constexpr uint32_t SMEM_ALLOC = SMEM + 1024;  // slack to align the base to 1024
     static constexpr uint32_t TMEM_COLS = 2 * BN;
     // kind::i8, D = s32 (bits 4-5 = 2), A = B = signed 8-bit (bits 7-9, 10-12 = 1),
@@ -64,9 +74,25 @@ struct Cfg {
 struct Params {
     int M, N, K;
     int num_m, num_n, num_kb;
+    int group_m;    // m-blocks per raster group
+    int vec_store;  // Y rows start on 16-byte boundaries
     GemmEpilogue ep;
     int* status;
 };
+
+// Raster: groups of group_m m-blocks; inside a group, n-major then m. The
+// CTAs running together then share the group's rows of Xq (kept in L2) and a
+// few weight tiles, and each weight tile is fetched once per group.
+__device__ __forceinline__ void tile_coords(int tile, const Params& p, int bn, int& m0, int& n0) {
+    const int per_group = p.group_m * p.num_n;
+    const int g = tile / per_group;
+    const int r = tile - g * per_group;
+    const int gm0 = g * p.group_m;
+    const int gsize = min(p.group_m, p.num_m - gm0);
+    const int nb = r / gsize;
+    m0 = (gm0 + (r - nb * gsize)) * BM;
+    n0 = nb * bn;
+}
 
 // ---------------------------------------------------------------- PTX helpers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -173,48 +199,18 @@ __device__ __forceinline__ float load16(const void* base, int64_t idx, int bf16)
     return __half2float(__ushort_as_half(u));
 }
 
-// Store 32 consecutive outputs of one row.
-__device__ __forceinline__ void store_row32(const GemmEpilogue& ep, int64_t row, int col0, int N, const float* y,
-                                            const uint32_t* acc_raw) {
-    const bool full = col0 + 32 <= N;
-    if (ep.out_dt == SQ_I32 || ep.out_dt == SQ_F32) {
-        uint32_t* dst = static_cast<uint32_t*>(ep.Y) + row * ep.ldy + col0;
-        const bool vec = full && ((reinterpret_cast<uintptr_t>(dst) & 15u) == 0);
-        uint32_t v[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) v[e] = ep.out_dt == SQ_I32 ? acc_raw[e] : __float_as_uint(y[e]);
-        if (vec) {
-#pragma unroll
-            for (int e = 0; e < 32; e += 4)
-                *reinterpret_cast<uint4*>(dst + e) = make_uint4(v[e], v[e + 1], v[e + 2], v[e + 3]);
-        } else {
-            for (int e = 0; e < 32 && col0 + e < N; ++e) dst[e] = v[e];
-        }
+template <int OUT>
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+    if constexpr (OUT == kOutBF16) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+        return *reinterpret_cast<uint32_t*>(&h);
     } else {
-        uint16_t* dst = static_cast<uint16_t*>(ep.Y) + row * ep.ldy + col0;
-        const bool vec = full && ((reinterpret_cast<uintptr_t>(dst) & 15u) == 0);
-        uint32_t p[16];
-        if (ep.out_dt == SQ_BF16) {
-#pragma unroll
-            for (int e = 0; e < 16; ++e)
-                p[e] = (uint32_t)to16<__nv_bfloat16>(y[2 * e]) | ((uint32_t)to16<__nv_bfloat16>(y[2 * e + 1]) << 16);
-        } else {
-#pragma unroll
-            for (int e = 0; e < 16; ++e)
-                p[e] = (uint32_t)to16<__half>(y[2 * e]) | ((uint32_t)to16<__half>(y[2 * e + 1]) << 16);
-        }
-        if (vec) {
-#pragma unroll
-            for (int e = 0; e < 16; e += 4)
-                *reinterpret_cast<uint4*>(dst + 2 * e) = make_uint4(p[e], p[e + 1], p[e + 2], p[e + 3]);
-        } else {
-            for (int e = 0; e < 32 && col0 + e < N; ++e)
-                dst[e] = (uint16_t)(e & 1 ? (p[e >> 1] >> 16) : (p[e >> 1] & 0xffffu));
-        }
+        __half2 h = __floats2half2_rn(a, b);
+        return *reinterpret_cast<uint32_t*>(&h);
     }
 }
 
-template <int BN>
+template <int BN, int OUT, bool OUTL>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                  const Params p) {
@@ -272,8 +268,8 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
             for (int s = 0; s < STAGES; ++s) issued[s] = false, issued_phase[s] = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-                const int m0 = (tile % p.num_m) * BM;
-                const int n0 = (tile / p.num_m) * BN;
+                int m0, n0;
+                tile_coords(tile, p, BN, m0, n0);
                 for (int kb = 0; kb < p.num_kb; ++kb) {
                     if (!wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, p.status, 0x6E1)) {
                         ok = false;
@@ -334,74 +330,168 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
     } else {
         // -------------------------------------------------------- epilogue
         // No block-level barrier is used here: an abort can make one warp leave
-        // early, so each warp stages its own per-column factors and decides
-        // collectively (all lanes) whether to go on.
+        // early, so each warp stages its own per-column factors and output
+        // chunks and decides collectively (all lanes) whether to go on.
         const int q = warp & 3;  // TMEM lane quarter this warp may access
         const GemmEpilogue& ep = p.ep;
-        const bool outl = ep.idx != nullptr;
-        const int n_out = outl ? *ep.n_out : 0;
+        const int n_out = OUTL ? *ep.n_out : 0;
+        const bool compact = n_out <= kOutlierCap;
         float* rw_w = rw_s + (warp - 2) * 2 * BN;  // this warp's 1/qs_w and bias
         float* bias_w = rw_w + BN;
+        uint8_t* stg = smem + C::STG_OFF + (warp - 2) * kStgWarpBytes;
         int local = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
-            const int m0 = (tile % p.num_m) * BM;
-            const int n0 = (tile / p.num_m) * BN;
-            __syncwarp();
-            for (int c = lane; c < BN; c += 32) {
-                const int col = n0 + c;
-                float rw = 0.0f, b = 0.0f;
-                if (col < p.N && ep.out_dt != SQ_I32) {
-                    rw = __frcp_rn(ep.w_per_channel ? ep.qs_w[col] : ep.qs_w[0]);
-                    if (ep.bias) b = ep.bias[col];
+            int m0, n0;
+            tile_coords(tile, p, BN, m0, n0);
+            if constexpr (OUT != kOutI32) {
+                __syncwarp();
+                for (int c = lane; c < BN; c += 32) {
+                    const int col = n0 + c;
+                    float rw = 0.0f, b = 0.0f;
+                    if (col < p.N) {
+                        rw = __frcp_rn(ep.w_per_channel ? ep.qs_w[col] : ep.qs_w[0]);
+                        if (ep.bias) b = ep.bias[col];
+                    }
+                    rw_w[c] = rw;
+                    bias_w[c] = b;
                 }
-                rw_w[c] = rw;
-                bias_w[c] = b;
+                __syncwarp();
             }
-            __syncwarp();
             const int acc = local & 1;
             const uint32_t acc_phase = (uint32_t)(local >> 1) & 1u;
             const bool ok = wait_bounded(tfull_bar(acc), acc_phase, abort_flag, p.status, 0x6E4);
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
-            const int row_in = q * 32 + lane;
-            const int64_t row = (int64_t)m0 + row_in;
+            const int row0 = m0 + q * 32;  // first row of this warp
+            const int64_t row = (int64_t)row0 + lane;
             const bool row_ok = row < p.M;
             float rx = 0.0f;
-            if (row_ok && ep.out_dt != SQ_I32) rx = __frcp_rn(ep.x_per_token ? ep.qs_x[row] : ep.qs_x[0]);
+            if constexpr (OUT != kOutI32)
+                if (row_ok) rx = __frcp_rn(ep.x_per_token ? ep.qs_x[row] : ep.qs_x[0]);
             const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+            if (row0 < p.M) {
 #pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32(t_row + (uint32_t)(c * 32), r);
-                const int col0 = n0 + c * 32;
-                if (row_ok && col0 < p.N) {
-                    float y[32];
-                    if (ep.out_dt != SQ_I32) {
+                for (int c = 0; c < BN / 32; ++c) {
+                    const int col0 = n0 + c * 32;
+                    if (col0 >= p.N) break;
+                    uint32_t r[32];
+                    tmem_ld32(t_row + (uint32_t)(c * 32), r);
+                    // 1) this thread's row of the chunk into the warp's staging buffer
+                    if constexpr (OUT == kOutI32) {
+                        uint4* dst = reinterpret_cast<uint4*>(stg + lane * kStg32);
 #pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            y[e] = __fmul_rn((float)(int)r[e], __fmul_rn(rx, rw_w[c * 32 + e]));
-                        if (outl) {
+                        for (int e = 0; e < 8; ++e) dst[e] = make_uint4(r[4 * e], r[4 * e + 1], r[4 * e + 2], r[4 * e + 3]);
+                    } else {
+                        float y[32];
+                        const float4* rw4 = reinterpret_cast<const float4*>(rw_w + c * 32);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const float4 w = rw4[e];
+                            y[4 * e + 0] = __fmul_rn((float)(int)r[4 * e + 0], __fmul_rn(rx, w.x));
+                            y[4 * e + 1] = __fmul_rn((float)(int)r[4 * e + 1], __fmul_rn(rx, w.y));
+                            y[4 * e + 2] = __fmul_rn((float)(int)r[4 * e + 2], __fmul_rn(rx, w.z));
+                            y[4 * e + 3] = __fmul_rn((float)(int)r[4 * e + 3], __fmul_rn(rx, w.w));
+                        }
+                        if constexpr (OUTL) {
                             float h[32];
 #pragma unroll
                             for (int e = 0; e < 32; ++e) h[e] = 0.0f;
-                            for (int o = 0; o < n_out; ++o) {
-                                const int ko = ep.idx[o];
-                                const float xo = load16(ep.x16, row * ep.ldx16 + ko, ep.in16_bf16);
+                            if (compact) {
+                                for (int o = 0; o < n_out; ++o) {
+                                    const float xo = row_ok ? ep.xo[row * kOutlierCap + o] : 0.0f;
+                                    const float4* w4 = reinterpret_cast<const float4*>(ep.wo + (int64_t)o * ep.wo_ld + col0);
 #pragma unroll
-                                for (int e = 0; e < 32; ++e) {
-                                    const int col = min(col0 + e, p.N - 1);
-                                    h[e] = __fmaf_rn(xo, load16(ep.w16, (int64_t)col * p.K + ko, ep.in16_bf16), h[e]);
+                                    for (int e = 0; e < 8; ++e) {
+                                        const float4 w = __ldg(w4 + e);
+                                        h[4 * e + 0] = __fmaf_rn(xo, w.x, h[4 * e + 0]);
+                                        h[4 * e + 1] = __fmaf_rn(xo, w.y, h[4 * e + 1]);
+                                        h[4 * e + 2] = __fmaf_rn(xo, w.z, h[4 * e + 2]);
+                                        h[4 * e + 3] = __fmaf_rn(xo, w.w, h[4 * e + 3]);
+                                    }
+                                }
+                            } else {
+                                for (int o = 0; o < n_out; ++o) {
+                                    const int ko = ep.idx[o];
+                                    const float xo = row_ok ? load16(ep.x16, row * ep.ldx16 + ko, ep.in16_bf16) : 0.0f;
+#pragma unroll
+                                    for (int e = 0; e < 32; ++e) {
+                                        const int col = min(col0 + e, p.N - 1);
+                                        h[e] = __fmaf_rn(xo, load16(ep.w16, (int64_t)col * p.K + ko, ep.in16_bf16), h[e]);
+                                    }
                                 }
                             }
 #pragma unroll
                             for (int e = 0; e < 32; ++e) y[e] = __fadd_rn(y[e], h[e]);
                         }
                         if (ep.bias) {
+                            const float4* b4 = reinterpret_cast<const float4*>(bias_w + c * 32);
 #pragma unroll
-                            for (int e = 0; e < 32; ++e) y[e] = __fadd_rn(y[e], bias_w[c * 32 + e]);
+                            for (int e = 0; e < 8; ++e) {
+                                const float4 b = b4[e];
+                                y[4 * e + 0] = __fadd_rn(y[4 * e + 0], b.x);
+                                y[4 * e + 1] = __fadd_rn(y[4 * e + 1], b.y);
+                                y[4 * e + 2] = __fadd_rn(y[4 * e + 2], b.z);
+                                y[4 * e + 3] = __fadd_rn(y[4 * e + 3], b.w);
+                            }
+                        }
+                        if constexpr (OUT == kOutF32) {
+                            uint4* dst = reinterpret_cast<uint4*>(stg + lane * kStg32);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e)
+                                dst[e] = make_uint4(__float_as_uint(y[4 * e]), __float_as_uint(y[4 * e + 1]),
+                                                    __float_as_uint(y[4 * e + 2]), __float_as_uint(y[4 * e + 3]));
+                        } else {
+                            uint4* dst = reinterpret_cast<uint4*>(stg + lane * kStg16);
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                dst[e] = make_uint4(pack2<OUT>(y[8 * e], y[8 * e + 1]), pack2<OUT>(y[8 * e + 2], y[8 * e + 3]),
+                                                    pack2<OUT>(y[8 * e + 4], y[8 * e + 5]), pack2<OUT>(y[8 * e + 6], y[8 * e + 7]));
                         }
                     }
-                    store_row32(ep, row, col0, p.N, y, r);
+                    __syncwarp();
+                    // 2) copy out with whole row segments per group of lanes
+                    if constexpr (OUT == kOutBF16 || OUT == kOutF16) {
+                        const int part = lane & 3;
+#pragma unroll
+                        for (int it = 0; it < 4; ++it) {
+                            const int rr = it * 8 + (lane >> 2);
+                            const int64_t grow = (int64_t)row0 + rr;
+                            const int col = col0 + part * 8;
+                            const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * kStg16 + part * 16);
+                            if (grow < p.M && col < p.N) {
+                                uint16_t* dst = static_cast<uint16_t*>(ep.Y) + grow * ep.ldy + col;
+                                if (p.vec_store && col + 8 <= p.N) {
+                                    *reinterpret_cast<uint4*>(dst) = v;
+                                } else {
+                                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                                    for (int e = 0; e < 8; ++e)
+                                        if (col + e < p.N) dst[e] = (uint16_t)(w[e >> 1] >> (16 * (e & 1)));
+                                }
+                            }
+                        }
+                    } else {
+                        const int part = lane & 7;
+#pragma unroll
+                        for (int it = 0; it < 8; ++it) {
+                            const int rr = it * 4 + (lane >> 3);
+                            const int64_t grow = (int64_t)row0 + rr;
+                            const int col = col0 + part * 4;
+                            const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * kStg32 + part * 16);
+                            if (grow < p.M && col < p.N) {
+                                uint32_t* dst = static_cast<uint32_t*>(ep.Y) + grow * ep.ldy + col;
+                                if (p.vec_store && col + 4 <= p.N) {
+                                    *reinterpret_cast<uint4*>(dst) = v;
+                                } else {
+                                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                                    for (int e = 0; e < 4; ++e)
+                                        if (col + e < p.N) dst[e] = w[e];
+                                }
+                            }
+                        }
+                    }
+                    __syncwarp();
                 }
             }
             tc_fence_before();
@@ -446,6 +536,18 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t K, int box
     return r == CUDA_SUCCESS;
 }
 
+using KernelFn = void (*)(const CUtensorMap, const CUtensorMap, const Params);
+
+template <int BN>
+KernelFn pick_kernel(sq_dtype_t out_dt, bool outl) {
+    switch (out_dt) {
+        case SQ_BF16: return outl ? gemm_w8a8_kernel<BN, kOutBF16, true> : gemm_w8a8_kernel<BN, kOutBF16, false>;
+        case SQ_F16: return outl ? gemm_w8a8_kernel<BN, kOutF16, true> : gemm_w8a8_kernel<BN, kOutF16, false>;
+        case SQ_F32: return gemm_w8a8_kernel<BN, kOutF32, false>;
+        default: return gemm_w8a8_kernel<BN, kOutI32, false>;
+    }
+}
+
 template <int BN>
 sq_status_t launch_bn(const int8_t* Xq, const int8_t* Wq, int64_t M, int64_t N, int64_t K, const GemmEpilogue& ep,
                       int* status, cudaStream_t stream) {
@@ -453,15 +555,13 @@ sq_status_t launch_bn(const int8_t* Xq, const int8_t* Wq, int64_t M, int64_t N, 
     CUtensorMap ta, tb;
     if (!make_map(&ta, Xq, M, K, BM) || !make_map(&tb, Wq, N, K, BN))
         return set_error(SQ_ERR_CUDA, "sq_gemm_w8a8: cuTensorMapEncodeTiled failed");
-    static bool attr_set[64] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-        if (cudaFuncSetAttribute(gemm_w8a8_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)C::SMEM_ALLOC) != cudaSuccess)
-            return check_launch("sq_gemm_w8a8: set shared memory size");
-        attr_set[dev] = true;
-    }
+    const bool outl = ep.idx != nullptr;
+    if (outl && ep.out_dt != SQ_BF16 && ep.out_dt != SQ_F16)
+        return set_error(SQ_ERR_INVALID_ARG, "sq_gemm_w8a8: the outlier term needs a 16-bit output");
+    KernelFn fn = pick_kernel<BN>(ep.out_dt, outl);
+    // the shared-memory opt-in is per kernel and per device; it is cheap, so set it every time
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM_ALLOC) != cudaSuccess)
+        return check_launch("sq_gemm_w8a8: set shared memory size");
     Params p;
     p.M = (int)M;
     p.N = (int)N;
@@ -469,11 +569,17 @@ sq_status_t launch_bn(const int8_t* Xq, const int8_t* Wq, int64_t M, int64_t N, 
     p.num_m = (int)((M + BM - 1) / BM);
     p.num_n = (int)((N + BN - 1) / BN);
     p.num_kb = (int)((K + BK - 1) / BK);
+    // rows of Xq per raster group kept within about 48 MB of L2
+    const int64_t per_mblock = (int64_t)BM * K;
+    int64_t g = (48ll << 20) / per_mblock;
+    p.group_m = (int)(g < 1 ? 1 : (g > p.num_m ? p.num_m : g));
+    const int eb = (ep.out_dt == SQ_BF16 || ep.out_dt == SQ_F16) ? 2 : 4;
+    p.vec_store = ((reinterpret_cast<uintptr_t>(ep.Y) & 15u) == 0) && ((ep.ldy * eb) % 16 == 0);
     p.ep = ep;
     p.status = status;
     const int tiles = p.num_m * p.num_n;
     const int grid = tiles < num_sms() ? tiles : num_sms();
-    gemm_w8a8_kernel<BN><<<grid, kThreads, C::SMEM_ALLOC, stream>>>(ta, tb, p);
+    fn<<<grid, kThreads, C::SMEM_ALLOC, stream>>>(ta, tb, p);
     return check_launch("sq_gemm_w8a8");
 }
 
@@ -495,7 +601,7 @@ extern "C" sq_status_t sq_gemm_w8a8(const int8_t* Xq, const int8_t* Wq, int64_t 
                                     const float* bias, sq_dtype_t out_dt, void* Y, int64_t ldy, void* workspace,
                                     size_t ws_bytes, sq_stream_t stream) {
     const char* name = "sq_gemm_w8a8";
-    SQ_REQUIRE(Xq && Wq && Y, SQ_ERR_INVALID_ARG, "%s: null Xq, Wq or Y", name);
+    SQ_REQUIRE((Xq || M == 0) && Wq && (Y || M == 0), SQ_ERR_INVALID_ARG, "%s: null Xq, Wq or Y", name);
     SQ_REQUIRE(out_dt == SQ_I32 || (qs_x && qs_w), SQ_ERR_INVALID_ARG, "%s: dequantising output needs qs_x and qs_w",
                name);
     SQ_REQUIRE(out_dt == SQ_I32 || out_dt == SQ_F32 || out_dt == SQ_F16 || out_dt == SQ_BF16, SQ_ERR_INVALID_ARG,

@@ -33,9 +33,13 @@ size_t detect_workspace_bytes(int64_t M, int64_t K) {
     return kStatusBytes + (counts + 255) / 256 * 256;
 }
 
-// header + counts | Xq [M,K] int8 | qs_x [M] fp32
-size_t llmint8_workspace_bytes(int64_t M, int64_t K) {
-    return detect_workspace_bytes(M, K) + ((size_t)M * (size_t)K + 255) / 256 * 256 + ((size_t)M * 4 + 255) / 256 * 256;
+static size_t r256(size_t b) { return (b + 255) / 256 * 256; }
+static int64_t wo_ld_of(int64_t N) { return (N + 255) / 256 * 256; }
+
+// header + counts | Xq [M,K] int8 | qs_x [M] fp32 | X_O [M, cap] fp32 | W_O [cap, N256] fp32
+size_t llmint8_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+    return detect_workspace_bytes(M, K) + r256((size_t)M * (size_t)K) + r256((size_t)M * 4) +
+           r256((size_t)M * kOutlierCap * 4) + r256((size_t)kOutlierCap * (size_t)wo_ld_of(N) * 4);
 }
 
 namespace {
@@ -132,9 +136,8 @@ template <typename T>
 __global__ void __launch_bounds__(256)
 masked_quant_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, const int32_t* __restrict__ idx,
                     const int32_t* __restrict__ n_idx, const int32_t* __restrict__ only_if, int8_t* __restrict__ Q,
-                    float* __restrict__ qs_out) {
+                    float* __restrict__ qs_out, float* __restrict__ xo) {
     extern __shared__ uint32_t mask[];  // K bits
-    __shared__ float sh[8];
     if (only_if && *only_if == 0) return;
     const int64_t words = (K + 31) / 32;
     for (int64_t w = threadIdx.x; w < words; w += blockDim.x) mask[w] = 0u;
@@ -145,10 +148,13 @@ masked_quant_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, c
         atomicOr(&mask[j >> 5], 1u << (j & 31));
     }
     __syncthreads();
-    for (int64_t row = blockIdx.x; row < M; row += gridDim.x) {
+    const int lane = threadIdx.x & 31;
+    const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < M; row += nwarps) {
         const T* x = X + row * ld;
         float m = 0.0f;
-        for (int64_t k0 = threadIdx.x * 8; k0 < K; k0 += 256 * 8) {
+#pragma unroll 4
+        for (int64_t k0 = lane * 8; k0 < K; k0 += 256) {
             float f[8];
             unpack<T>(ldg_v4(x + k0), f);
             const uint32_t bits = (mask[k0 >> 5] >> (k0 & 31)) & 0xffu;
@@ -158,25 +164,47 @@ masked_quant_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, c
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        __syncthreads();
-        if ((threadIdx.x & 31) == 0) sh[threadIdx.x >> 5] = m;
-        __syncthreads();
-        float mm = sh[0];
-#pragma unroll
-        for (int w = 1; w < 8; ++w) mm = fmaxf(mm, sh[w]);
-        const float qs = __fdiv_rn(127.0f, fmaxf(mm, 1e-8f));
-        if (threadIdx.x == 0) qs_out[row] = qs;
+        const float qs = __fdiv_rn(127.0f, fmaxf(m, 1e-8f));
+        if (lane == 0) qs_out[row] = qs;
+        if (xo)  // fp32 copy of the outlier columns of this row, for the GEMM epilogue
+            for (int o = lane; o < n && o < kOutlierCap; o += 32) {
+                const uint16_t u = reinterpret_cast<const uint16_t*>(x)[idx[o]];
+                float f[8];
+                uint4 v = make_uint4(u, 0, 0, 0);
+                unpack<T>(v, f);
+                xo[row * kOutlierCap + o] = f[0];
+            }
         int8_t* q = Q + row * K;
-        for (int64_t k0 = threadIdx.x * 8; k0 < K; k0 += 256 * 8) {
+#pragma unroll 4
+        for (int64_t k0 = lane * 8; k0 < K; k0 += 256) {
             float f[8];
             unpack<T>(ldg_v4(x + k0), f);
             const uint32_t bits = (mask[k0 >> 5] >> (k0 & 31)) & 0xffu;
-            int c[8];
+            uint32_t c[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) c[e] = ((bits >> e) & 1u) ? 0 : quant_code(__fmul_rn(f[e], qs));
-            *reinterpret_cast<uint2*>(q + k0) = make_uint2(pack4_i8(c[0], c[1], c[2], c[3]), pack4_i8(c[4], c[5], c[6], c[7]));
+            for (int e = 0; e < 8; ++e) c[e] = ((bits >> e) & 1u) ? 0u : quant_bits_noclip(__fmul_rn(f[e], qs));
+            *reinterpret_cast<uint2*>(q + k0) =
+                make_uint2(pack_low_bytes(c[0], c[1], c[2], c[3]), pack_low_bytes(c[4], c[5], c[6], c[7]));
         }
     }
+}
+
+// W_O[o, j] = W[j, idx[o]] for o < min(n, cap), j < N; zero for N <= j < ld.
+template <typename T>
+__global__ void gather_wo_kernel(const T* __restrict__ W, int64_t N, int64_t K, const int32_t* __restrict__ idx,
+                                 const int32_t* __restrict__ n_idx, float* __restrict__ wo, int64_t ld) {
+    const int n = min(*n_idx, kOutlierCap);
+    for (int64_t j = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; j < ld; j += (int64_t)gridDim.x * blockDim.x)
+        for (int o = 0; o < n; ++o) {
+            float v = 0.0f;
+            if (j < N) {
+                const uint16_t u = reinterpret_cast<const uint16_t*>(W)[j * K + idx[o]];
+                float f[8];
+                unpack<T>(make_uint4(u, 0, 0, 0), f);
+                v = f[0];
+            }
+            wo[(int64_t)o * ld + j] = v;
+        }
 }
 
 sq_status_t launch_detect(const void* X, sq_dtype_t dt, int64_t M, int64_t K, int64_t ldx, float thr,
@@ -202,25 +230,25 @@ sq_status_t launch_detect(const void* X, sq_dtype_t dt, int64_t M, int64_t K, in
 
 sq_status_t launch_masked_quant(const void* X, sq_dtype_t dt, int64_t M, int64_t K, int64_t ldx, const int32_t* idx,
                                 const int32_t* n_idx, const int32_t* only_if, int8_t* Q, float* qs, cudaStream_t s,
-                                const char* name) {
+                                const char* name, float* xo = nullptr) {
     const size_t smem = (size_t)((K + 31) / 32) * 4;
-    int64_t grid = (int64_t)num_sms() * 8;
-    if (grid > M) grid = M;
+    int64_t grid = (M + 7) / 8;  // one warp per row, 8 warps per block
+    if (grid > (int64_t)num_sms() * 8) grid = (int64_t)num_sms() * 8;
     if (grid < 1) return SQ_OK;
     if (dt == SQ_BF16) {
         auto k = masked_quant_kernel<__nv_bfloat16>;
         if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        k<<<(unsigned)grid, 256, smem, s>>>(static_cast<const __nv_bfloat16*>(X), M, K, ldx, idx, n_idx, only_if, Q, qs);
+        k<<<(unsigned)grid, 256, smem, s>>>(static_cast<const __nv_bfloat16*>(X), M, K, ldx, idx, n_idx, only_if, Q, qs, xo);
     } else {
         auto k = masked_quant_kernel<__half>;
         if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        k<<<(unsigned)grid, 256, smem, s>>>(static_cast<const __half*>(X), M, K, ldx, idx, n_idx, only_if, Q, qs);
+        k<<<(unsigned)grid, 256, smem, s>>>(static_cast<const __half*>(X), M, K, ldx, idx, n_idx, only_if, Q, qs, xo);
     }
     return check_launch(name);
 }
 
 sq_status_t check_x(const char* name, const void* X, sq_dtype_t dt, int64_t M, int64_t K, int64_t ldx) {
-    SQ_REQUIRE(X, SQ_ERR_INVALID_ARG, "%s: null input", name);
+    SQ_REQUIRE(X || M == 0, SQ_ERR_INVALID_ARG, "%s: null input", name);
     SQ_REQUIRE(dt == SQ_F16 || dt == SQ_BF16, SQ_ERR_INVALID_ARG, "%s: dtype must be F16 or BF16", name);
     SQ_REQUIRE(M >= 0 && K > 0 && ldx >= K && K % 8 == 0 && ldx % 8 == 0, SQ_ERR_UNSUPPORTED_SHAPE,
                "%s: need K > 0, K %% 8 == 0, ldx >= K, ldx %% 8 == 0", name);
@@ -255,7 +283,7 @@ sq_status_t sq_llmint8_quant_rows(const void* X, sq_dtype_t dt, int64_t M, int64
     const char* name = "sq_llmint8_quant_rows";
     sq_status_t st = sq::check_x(name, X, dt, M, K, ldx);
     if (st != SQ_OK) return st;
-    SQ_REQUIRE(idx && n_idx && Xq && qs_x, SQ_ERR_INVALID_ARG, "%s: null pointer", name);
+    SQ_REQUIRE(idx && n_idx && ((Xq && qs_x) || M == 0), SQ_ERR_INVALID_ARG, "%s: null pointer", name);
     SQ_REQUIRE(sq::aligned16(Xq), SQ_ERR_ALIGNMENT, "%s: Xq not 16-byte aligned", name);
     if (M == 0) return SQ_OK;
     return sq::launch_masked_quant(X, dt, M, K, ldx, idx, n_idx, nullptr, Xq, qs_x, sq::as_cuda(stream), name);
@@ -266,7 +294,7 @@ sq_status_t sq_llmint8_quant_weight(const void* W, sq_dtype_t dt, int64_t N, int
     const char* name = "sq_llmint8_quant_weight";
     sq_status_t st = sq::check_x(name, W, dt, N, K, K);
     if (st != SQ_OK) return st;
-    SQ_REQUIRE(idx && n_idx && Wq && qs_w, SQ_ERR_INVALID_ARG, "%s: null pointer", name);
+    SQ_REQUIRE(idx && n_idx && ((Wq && qs_w) || N == 0), SQ_ERR_INVALID_ARG, "%s: null pointer", name);
     SQ_REQUIRE(sq::aligned16(Wq), SQ_ERR_ALIGNMENT, "%s: Wq not 16-byte aligned", name);
     if (N == 0) return SQ_OK;
     return sq::launch_masked_quant(W, dt, N, K, K, idx, n_idx, nullptr, Wq, qs_w, sq::as_cuda(stream), name);
@@ -281,19 +309,26 @@ sq_status_t sq_llmint8_matmul(const void* X, sq_dtype_t dt, int64_t M, int64_t K
     if (st != SQ_OK) return st;
     SQ_REQUIRE(w && w->W && w->Wq && w->qs_w && w->cached_idx && w->cached_n, SQ_ERR_INVALID_ARG,
                "%s: incomplete weight state", name);
-    SQ_REQUIRE(Y && idx_out && n_out, SQ_ERR_INVALID_ARG, "%s: null output", name);
+    SQ_REQUIRE((Y || M == 0) && idx_out && n_out, SQ_ERR_INVALID_ARG, "%s: null output", name);
     SQ_REQUIRE(w->N > 0 && ldy >= w->N, SQ_ERR_UNSUPPORTED_SHAPE, "%s: need N > 0 and ldy >= N", name);
     SQ_REQUIRE(K % 16 == 0 && K <= 133144, SQ_ERR_UNSUPPORTED_SHAPE, "%s: K must be a multiple of 16, <= 133144",
                name);
     SQ_REQUIRE(M < (1ll << 31) && w->N < (1ll << 31), SQ_ERR_UNSUPPORTED_SHAPE, "%s: M and N must be < 2^31", name);
     SQ_REQUIRE(sq::aligned16(w->W) && sq::aligned16(w->Wq), SQ_ERR_ALIGNMENT, "%s: weights not 16-byte aligned", name);
-    const size_t need = sq::llmint8_workspace_bytes(M, K);
+    const size_t need = sq::llmint8_workspace_bytes(M, w->N, K);
     SQ_REQUIRE(workspace && ws_bytes >= need, SQ_ERR_INVALID_ARG, "%s: needs a workspace of %zu bytes", name, need);
     cudaStream_t s = sq::as_cuda(stream);
     char* wsb = static_cast<char*>(workspace);
     const size_t det = sq::detect_workspace_bytes(M, K);
-    int8_t* Xq = reinterpret_cast<int8_t*>(wsb + det);
-    float* qs_x = reinterpret_cast<float*>(wsb + det + ((size_t)M * K + 255) / 256 * 256);
+    size_t off = det;
+    int8_t* Xq = reinterpret_cast<int8_t*>(wsb + off);
+    off += sq::r256((size_t)M * K);
+    float* qs_x = reinterpret_cast<float*>(wsb + off);
+    off += sq::r256((size_t)M * 4);
+    float* xo = reinterpret_cast<float*>(wsb + off);
+    off += sq::r256((size_t)M * sq::kOutlierCap * 4);
+    float* wo = reinterpret_cast<float*>(wsb + off);
+    const int64_t wo_ld = sq::wo_ld_of(w->N);
     int32_t* changed = reinterpret_cast<int32_t*>(wsb + 4);
     // a7: O, and whether the cached int8 weight was built for it
     st = sq::launch_detect(X, dt, M, K, ldx, threshold, min_ratio, idx_out, n_out, w->cached_idx, w->cached_n, workspace,
@@ -303,9 +338,22 @@ sq_status_t sq_llmint8_matmul(const void* X, sq_dtype_t dt, int64_t M, int64_t K
     st = sq::launch_masked_quant(w->W, dt, w->N, K, K, idx_out, n_out, changed, w->Wq, w->qs_w, s, name);
     if (st != SQ_OK) return st;
     if (M == 0) return SQ_OK;
-    // a8
-    st = sq::launch_masked_quant(X, dt, M, K, ldx, idx_out, n_out, nullptr, Xq, qs_x, s, name);
+    // a8 (and the fp32 copy of the outlier columns of X)
+    st = sq::launch_masked_quant(X, dt, M, K, ldx, idx_out, n_out, nullptr, Xq, qs_x, s, name, xo);
     if (st != SQ_OK) return st;
+    // fp32 copy of the outlier input channels of W, transposed, for the epilogue
+    {
+        int64_t blocks = (wo_ld + 255) / 256;
+        if (blocks > (int64_t)sq::num_sms() * 4) blocks = (int64_t)sq::num_sms() * 4;
+        if (dt == SQ_BF16)
+            sq::gather_wo_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, s>>>(
+                static_cast<const __nv_bfloat16*>(w->W), w->N, K, idx_out, n_out, wo, wo_ld);
+        else
+            sq::gather_wo_kernel<__half><<<(unsigned)blocks, 256, 0, s>>>(static_cast<const __half*>(w->W), w->N, K,
+                                                                         idx_out, n_out, wo, wo_ld);
+        st = sq::check_launch(name);
+        if (st != SQ_OK) return st;
+    }
     // a9: int8 GEMM + 16-bit outlier term in the epilogue
     sq::GemmEpilogue ep;
     ep.qs_x = qs_x;
@@ -321,6 +369,9 @@ sq_status_t sq_llmint8_matmul(const void* X, sq_dtype_t dt, int64_t M, int64_t K
     ep.idx = idx_out;
     ep.n_out = n_out;
     ep.in16_bf16 = dt == SQ_BF16;
+    ep.xo = xo;
+    ep.wo = wo;
+    ep.wo_ld = wo_ld;
     return sq::launch_gemm_w8a8(Xq, w->Wq, M, w->N, K, ep, static_cast<int*>(workspace), s);
 }
 

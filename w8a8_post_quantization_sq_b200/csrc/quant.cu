@@ -11,9 +11,10 @@
 // 解决激活值离群点难题" §3). All arithmetic is fp32 with correctly rounded
 // operations, so codes and scales are bit-exact against a plain CPU loop.
 //
-// Row mode: one 256-thread block per row, the row read twice (the second read
-// hits L1/L2): pass 1 reduces max |v|, pass 2 writes the codes. Tensor mode:
-// a grid-wide absmax into the workspace, then the quantising pass.
+// Row mode: the row is read once into the registers of one warp (K <= 2048)
+// or one block (K <= 16384), reduced to its absmax and quantised from the
+// registers; longer rows stream twice through a warp. Tensor mode: a
+// grid-wide absmax into the workspace, then the quantising pass.
 #include "sq_common.cuh"
 #include "sq_internal.h"
 
@@ -59,45 +60,110 @@ __device__ __forceinline__ float block_max(float v, float* sh) {
 
 __device__ __forceinline__ float scale_of(float m) { return __fdiv_rn(127.0f, fmaxf(m, 1e-8f)); }
 
-__device__ __forceinline__ uint2 codes8(const float* v, float qs) {
-    int q[8];
+// Eight codes; `clip` is needed only when qs does not come from the group's
+// own absmax (a static per-tensor scale).
+__device__ __forceinline__ uint2 codes8(const float* v, float qs, bool clip) {
+    uint32_t b[8];
+    if (clip) {
 #pragma unroll
-    for (int e = 0; e < 8; ++e) q[e] = quant_code(__fmul_rn(v[e], qs));
-    return make_uint2(pack4_i8(q[0], q[1], q[2], q[3]), pack4_i8(q[4], q[5], q[6], q[7]));
+        for (int e = 0; e < 8; ++e) b[e] = quant_bits_clip(__fmul_rn(v[e], qs));
+    } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) b[e] = quant_bits_noclip(__fmul_rn(v[e], qs));
+    }
+    return make_uint2(pack_low_bytes(b[0], b[1], b[2], b[3]), pack_low_bytes(b[4], b[5], b[6], b[7]));
 }
 
-// per_row != 0: scale per row from the row's absmax; else *tensor_qs for all.
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+// One warp per row, rows strided over the grid. per_row != 0: the row's own
+// scale from its absmax; else *tensor_qs for every row.
 template <typename T, int SM>
 __global__ void __launch_bounds__(kThreads)
 row_quant_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, const float* __restrict__ s,
                  int per_row, const float* __restrict__ tensor_qs, int8_t* __restrict__ Q,
                  float* __restrict__ qs_out) {
-    __shared__ float sh[kThreads / 32];
-    for (int64_t row = blockIdx.x; row < M; row += gridDim.x) {
+    const int lane = threadIdx.x & 31;
+    const int64_t nwarps = (int64_t)gridDim.x * (kThreads / 32);
+    for (int64_t row = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5; row < M; row += nwarps) {
         const T* x = X + row * ld;
         float qs;
         if (per_row) {
             float m = 0.0f;
-            for (int64_t k0 = threadIdx.x * 8; k0 < K; k0 += kThreads * 8) {
+#pragma unroll 4
+            for (int64_t k0 = lane * 8; k0 < K; k0 += 256) {
                 float f[8];
                 load8<T>(x + k0, f);
                 apply_s<SM>(f, s, k0);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(f[e]));
             }
-            m = block_max(m, sh);
-            qs = scale_of(m);
-            if (threadIdx.x == 0) qs_out[row] = qs;
+            qs = scale_of(warp_max(m));
+            if (lane == 0) qs_out[row] = qs;
         } else {
             qs = *tensor_qs;
-            if (row == 0 && threadIdx.x == 0) qs_out[0] = qs;
+            if (row == 0 && lane == 0) qs_out[0] = qs;
         }
         int8_t* q = Q + row * K;
-        for (int64_t k0 = threadIdx.x * 8; k0 < K; k0 += kThreads * 8) {
+#pragma unroll 4
+        for (int64_t k0 = lane * 8; k0 < K; k0 += 256) {
             float f[8];
             load8<T>(x + k0, f);
             apply_s<SM>(f, s, k0);
-            *reinterpret_cast<uint2*>(q + k0) = codes8(f, qs);
+            *reinterpret_cast<uint2*>(q + k0) = codes8(f, qs, !per_row);
+        }
+    }
+}
+
+// The row held in registers by a group of G threads (G = 32: one warp per
+// row, several rows per block; G = 256: the whole block), CH chunks of 8
+// elements per thread: one read of the row from memory, a group max, then the
+// codes from the registers. Used while K <= 8 * G * CH_max.
+template <typename T, int SM, int G, int CH>
+__global__ void __launch_bounds__(kThreads)
+row_quant_reg_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, const float* __restrict__ s,
+                     int per_row, const float* __restrict__ tensor_qs, int8_t* __restrict__ Q,
+                     float* __restrict__ qs_out) {
+    __shared__ float sh[kThreads / 32];
+    constexpr int GPB = kThreads / G;  // groups (rows) per block
+    const int gt = threadIdx.x % G;
+    const int64_t ngroups = (int64_t)gridDim.x * GPB;
+    for (int64_t row = (int64_t)blockIdx.x * GPB + threadIdx.x / G; row < M; row += ngroups) {
+        const T* x = X + row * ld;
+        float v[CH][8];
+        float m = 0.0f;
+#pragma unroll
+        for (int c = 0; c < CH; ++c) {
+            const int64_t k0 = ((int64_t)gt + (int64_t)c * G) * 8;
+            if (k0 < K) {
+                load8<T>(x + k0, v[c]);
+                apply_s<SM>(v[c], s, k0);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(v[c][e]));
+            }
+        }
+        float qs;
+        if (per_row) {
+            if constexpr (G == 32) {
+                m = warp_max(m);
+            } else {
+                m = block_max(m, sh);
+            }
+            qs = scale_of(m);
+            if (gt == 0) qs_out[row] = qs;
+        } else {
+            qs = *tensor_qs;
+            if (row == 0 && gt == 0) qs_out[0] = qs;
+        }
+        int8_t* q = Q + row * K;
+#pragma unroll
+        for (int c = 0; c < CH; ++c) {
+            const int64_t k0 = ((int64_t)gt + (int64_t)c * G) * 8;
+            if (k0 < K) *reinterpret_cast<uint2*>(q + k0) = codes8(v[c], qs, !per_row);
         }
     }
 }
@@ -135,8 +201,9 @@ scale_from_absmax_kernel(const float* __restrict__ a, int64_t n, float* __restri
 }
 
 int row_grid(int64_t M) {
+    const int64_t blocks = (M + kThreads / 32 - 1) / (kThreads / 32);
     const int64_t cap = (int64_t)num_sms() * 8;
-    return (int)(M < cap ? M : cap);
+    return (int)(blocks < cap ? blocks : cap);
 }
 
 int vec_grid(int64_t nvec) {
@@ -160,7 +227,27 @@ sq_status_t quantize(const void* Xv, int64_t M, int64_t K, int64_t ld, const flo
         scale_from_absmax_kernel<<<1, kThreads, 0, st>>>(wmax, 1, wqs);
         tensor_qs = wqs;
     }
-    row_quant_kernel<T, SM><<<row_grid(M), kThreads, 0, st>>>(X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
+    const int64_t cap = (int64_t)num_sms() * 8;
+    auto blocks = [&](int64_t rows_per_block) {
+        int64_t b = (M + rows_per_block - 1) / rows_per_block;
+        return (unsigned)(b < cap ? b : cap);
+    };
+    if (K <= 256)
+        row_quant_reg_kernel<T, SM, 32, 1><<<blocks(8), kThreads, 0, st>>>(X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
+    else if (K <= 512)
+        row_quant_reg_kernel<T, SM, 32, 2><<<blocks(8), kThreads, 0, st>>>(X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
+    else if (K <= 1024)
+        row_quant_reg_kernel<T, SM, 32, 4><<<blocks(8), kThreads, 0, st>>>(X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
+    else if (K <= 2048)
+        row_quant_reg_kernel<T, SM, 32, 8><<<blocks(8), kThreads, 0, st>>>(X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
+    else if (K <= 4096)
+        row_quant_reg_kernel<T, SM, 256, 2><<<blocks(1), kThreads, 0, st>>>(X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
+    else if (K <= 8192)
+        row_quant_reg_kernel<T, SM, 256, 4><<<blocks(1), kThreads, 0, st>>>(X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
+    else if (K <= 16384)
+        row_quant_reg_kernel<T, SM, 256, 8><<<blocks(1), kThreads, 0, st>>>(X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
+    else
+        row_quant_kernel<T, SM><<<row_grid(M), kThreads, 0, st>>>(X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
     return check_launch(name);
 }
 
@@ -186,7 +273,7 @@ sq_status_t sq_quantize_weight(const void* W, sq_dtype_t dt, int64_t N, int64_t 
                                int per_channel, int8_t* Wq, float* qs_w, void* workspace, size_t ws_bytes,
                                sq_stream_t stream) {
     const char* name = "sq_quantize_weight";
-    SQ_REQUIRE(W && Wq && qs_w, SQ_ERR_INVALID_ARG, "%s: null pointer", name);
+    SQ_REQUIRE((W && Wq && qs_w) || N == 0, SQ_ERR_INVALID_ARG, "%s: null pointer", name);
     SQ_REQUIRE(N >= 0 && K > 0 && K % 16 == 0, SQ_ERR_UNSUPPORTED_SHAPE, "%s: need K > 0 and K %% 16 == 0", name);
     SQ_REQUIRE(sq::aligned16(W) && sq::aligned16(Wq) && (!s || sq::aligned16(s)), SQ_ERR_ALIGNMENT,
                "%s: W, Wq and s must be 16-byte aligned", name);
@@ -204,7 +291,7 @@ sq_status_t sq_quantize_act(const void* X, sq_dtype_t dt, int64_t M, int64_t K, 
                             int per_token, const float* static_qs, int8_t* Xq, float* qs_x, void* workspace,
                             size_t ws_bytes, sq_stream_t stream) {
     const char* name = "sq_quantize_act";
-    SQ_REQUIRE(X && Xq && qs_x, SQ_ERR_INVALID_ARG, "%s: null pointer", name);
+    SQ_REQUIRE((X && Xq && qs_x) || M == 0, SQ_ERR_INVALID_ARG, "%s: null pointer", name);
     SQ_REQUIRE(M >= 0 && K > 0 && K % 16 == 0 && ldx >= K && ldx % 8 == 0, SQ_ERR_UNSUPPORTED_SHAPE,
                "%s: need K > 0, K %% 16 == 0, ldx >= K, ldx %% 8 == 0", name);
     SQ_REQUIRE(sq::aligned16(X) && sq::aligned16(Xq) && (!s || sq::aligned16(s)), SQ_ERR_ALIGNMENT,

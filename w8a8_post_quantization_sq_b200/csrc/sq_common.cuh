@@ -116,6 +116,20 @@ __device__ __forceinline__ int quant_code(float t) {
     return __float_as_int(r) - 0x4B400000;
 }
 
+// Same code without the clip, for a scale taken from the group's own absmax:
+// then |t| <= 127 (1 + 2^-23), which rounds to at most 127. Returns the
+// shifter's bit pattern; its low byte is the code (the shifter's low byte is 0).
+__device__ __forceinline__ uint32_t quant_bits_noclip(float t) {
+    return __float_as_uint(__fadd_rn(t, 12582912.0f));
+}
+__device__ __forceinline__ uint32_t quant_bits_clip(float t) {
+    return __float_as_uint(__fadd_rn(fminf(fmaxf(t, -127.0f), 127.0f), 12582912.0f));
+}
+// Low bytes of four words into one word (byte i from word i).
+__device__ __forceinline__ uint32_t pack_low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+
 // max on non-negative floats through their bit patterns (monotone for >= 0).
 __device__ __forceinline__ void atomic_max_nonneg(float* addr, float v) {
     atomicMax(reinterpret_cast<int*>(addr), __float_as_int(v));

@@ -15,7 +15,12 @@ constexpr size_t kStatusBytes = 256;
 // Rows per block of the outlier-count pass of sq_llmint8_detect.
 constexpr int kDetectRows = 128;
 size_t detect_workspace_bytes(int64_t M, int64_t K);
-size_t llmint8_workspace_bytes(int64_t M, int64_t K);
+size_t llmint8_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+// Outlier counts up to this size use compact fp32 copies of the outlier
+// columns (X_O [M, cap], W_O [cap, N padded to 256]) built in the workspace;
+// larger sets read the 16-bit operands directly in the epilogue.
+constexpr int kOutlierCap = 32;
 
 // Epilogue description of the int8 GEMM.
 struct GemmEpilogue {
@@ -35,6 +40,9 @@ struct GemmEpilogue {
     const int32_t* idx = nullptr;
     const int32_t* n_out = nullptr;
     int in16_bf16 = 0;
+    const float* xo = nullptr;  // [M, kOutlierCap] fp32 copies of X[:, O]
+    const float* wo = nullptr;  // [kOutlierCap, wo_ld] fp32 copies of W[:, O]^T
+    int64_t wo_ld = 0;          // multiple of 256, >= N
 };
 
 sq_status_t launch_gemm_w8a8(const int8_t* Xq, const int8_t* Wq, int64_t M, int64_t N, int64_t K,

@@ -47,13 +47,12 @@ const char* sq_last_error_string(void) { return sq::g_last_error.c_str(); }
 int sq_version(void) { return 100; }
 
 size_t sq_workspace_size(sq_op_t op, int64_t M, int64_t N, int64_t K) {
-    (void)N;
     switch (op) {
         case SQ_OP_GEMM: return sq::kStatusBytes;
         case SQ_OP_QUANT_ACT: return sq::kStatusBytes;
         case SQ_OP_QUANT_WEIGHT: return sq::kStatusBytes;
         case SQ_OP_LLMINT8_DETECT: return sq::detect_workspace_bytes(M, K);
-        case SQ_OP_LLMINT8: return sq::llmint8_workspace_bytes(M, K);
+        case SQ_OP_LLMINT8: return sq::llmint8_workspace_bytes(M, N, K);
     }
     return 0;
 }
