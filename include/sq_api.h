@@ -229,6 +229,27 @@ SQ_API sq_status_t sq_llmint8_detect(const void* X, sq_dtype_t dt, int64_t M, in
                               int32_t* n_outliers, void* workspace, size_t ws_bytes,
                               sq_stream_t stream);
 
+/* sq_llmint8_detect_noalloc: sq_llmint8_detect without the workspace
+ * argument. The pages have no counterpart to this entry point; it only changes
+ * where the scratch memory comes from. It is for callers that cannot allocate
+ * device memory or hand scratch to the library: a component that runs where
+ * another layer owns every buffer and passes in only inputs and outputs (an
+ * inference engine's plugin slot, a memory arena planned ahead of time with
+ * nothing to spare), or a service that must not allocate once it is serving.
+ * The scratch is a fixed 4 MiB device array inside this library, one per
+ * device that loads it, held until the process exits. Hence
+ * ceil(M / 128) * K <= 1,048,512 (for example M <= 32768 at K = 4096); larger
+ * sizes return SQ_ERR_UNSUPPORTED_SHAPE and launch nothing.
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * Every call uses the same array: calls that overlap on the GPU (other
+ * streams, other host threads) race, so the caller must serialise them.
+ * Nothing in the array needs clearing; each call writes every count it reads.
+ * Arguments and results are those of sq_llmint8_detect. */
+SQ_API sq_status_t sq_llmint8_detect_noalloc(const void* X, sq_dtype_t dt, int64_t M, int64_t K, int64_t ldx,
+                                             float threshold, double min_ratio, int32_t* outlier_idx,
+                                             int32_t* n_outliers, sq_stream_t stream);
+
 /* a8: vector-wise row quantisation over the columns not in O:
  * qs_x[i] = 127 / max(max_{j not in O} |X[i,j]|, 1e-8);
  * Xq[i,j] = 0 for j in O, else clip(rne(X*qs), -127, 127).

@@ -58,6 +58,7 @@ SIGNATURES = {
     "sq_norm_smooth_quant": ([_p, _i, _i64, _i64, _i64, _i, _p, _p, _f, _i, _p, _p, _p, _p, _p, _p], _i),
     "sq_gemm_w8a8": ([_p, _p, _i64, _i64, _i64, _p, _i, _p, _i, _p, _i, _p, _i64, _p, _sz, _p], _i),
     "sq_llmint8_detect": ([_p, _i, _i64, _i64, _i64, _f, _d, _p, _p, _p, _sz, _p], _i),
+    "sq_llmint8_detect_noalloc": ([_p, _i, _i64, _i64, _i64, _f, _d, _p, _p, _p], _i),
     "sq_llmint8_quant_rows": ([_p, _i, _i64, _i64, _i64, _p, _p, _p, _p, _p], _i),
     "sq_llmint8_quant_weight": ([_p, _i, _i64, _i64, _p, _p, _p, _p, _p], _i),
     "sq_llmint8_matmul": ([_p, _i, _i64, _i64, _i64, ctypes.POINTER(LLMInt8Weight), _f, _d, _p, _i64, _p, _p, _p,
@@ -232,6 +233,14 @@ def sq_llmint8_detect(X, threshold, min_ratio, idx, n, ws, stream=None):
     _check("sq_llmint8_detect", lib().sq_llmint8_detect(
         _ptr(X), _dt(X), M, K, _ld(X), float(threshold), float(min_ratio), _vec(idx, torch.int32, K),
         _vec(n, torch.int32, 1), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def sq_llmint8_detect_noalloc(X, threshold, min_ratio, idx, n, stream=None):
+    """sq_llmint8_detect with the library's own fixed scratch (no workspace)."""
+    M, K = X.shape
+    _check("sq_llmint8_detect_noalloc", lib().sq_llmint8_detect_noalloc(
+        _ptr(X), _dt(X), M, K, _ld(X), float(threshold), float(min_ratio), _vec(idx, torch.int32, K),
+        _vec(n, torch.int32, 1), _stream(stream)))
 
 
 def sq_llmint8_quant_rows(X, idx, n, Xq, qs_x, stream=None):

@@ -22,6 +22,8 @@
 //   the tcgen05 GEMM, whose epilogue adds the 16-bit outlier term.
 // Nothing here synchronises with the host, so a whole call can be captured in
 // a CUDA graph.
+#include <mutex>
+
 #include "sq_common.cuh"
 #include "sq_internal.h"
 
@@ -376,3 +378,64 @@ sq_status_t sq_llmint8_matmul(const void* X, sq_dtype_t dt, int64_t M, int64_t K
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// sq_llmint8_detect_noalloc: the same detection for callers that cannot hand
+// the library any scratch memory. Its scratch (the 256-byte header plus the
+// per-band column counts) is this file-scope device array; each device that
+// loads the library holds one copy until the process exits.
+namespace sq {
+namespace {
+
+constexpr size_t kDetectScratchBytes = size_t(4) << 20;  // 4 MiB
+__device__ __align__(256) unsigned char g_detect_scratch[kDetectScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxDevices] = {};
+
+// Device address of g_detect_scratch on the current device. The name is only
+// a host-side stand-in, so the address is looked up once per device.
+sq_status_t detect_scratch(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return check_launch("sq_llmint8_detect_noalloc: cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices)
+        return set_error(SQ_ERR_CUDA, "sq_llmint8_detect_noalloc: device %d out of range", dev);
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (g_scratch_addr[dev] == nullptr) {
+        void* p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_detect_scratch);
+        if (e != cudaSuccess || p == nullptr)
+            return set_error(SQ_ERR_CUDA, "sq_llmint8_detect_noalloc: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+        g_scratch_addr[dev] = p;
+    }
+    *out = g_scratch_addr[dev];
+    return SQ_OK;
+}
+
+}  // namespace
+}  // namespace sq
+
+extern "C" sq_status_t sq_llmint8_detect_noalloc(const void* X, sq_dtype_t dt, int64_t M, int64_t K, int64_t ldx,
+                                                 float threshold, double min_ratio, int32_t* outlier_idx,
+                                                 int32_t* n_outliers, sq_stream_t stream) {
+    const char* name = "sq_llmint8_detect_noalloc";
+    sq_status_t st = sq::check_x(name, X, dt, M, K, ldx);
+    if (st != SQ_OK) return st;
+    SQ_REQUIRE(outlier_idx && n_outliers, SQ_ERR_INVALID_ARG, "%s: null output", name);
+    SQ_REQUIRE(min_ratio >= 0.0 && threshold >= 0.0f, SQ_ERR_INVALID_ARG, "%s: threshold and min_ratio must be >= 0",
+               name);
+    const size_t need = sq::detect_workspace_bytes(M, K);
+    SQ_REQUIRE(need <= sq::kDetectScratchBytes, SQ_ERR_UNSUPPORTED_SHAPE,
+               "%s: ceil(M/%d) * K = %lld counts need %zu bytes of scratch, more than its fixed %zu bytes; "
+               "use sq_llmint8_detect with a workspace",
+               name, sq::kDetectRows, (long long)(((M + sq::kDetectRows - 1) / sq::kDetectRows) * K), need,
+               sq::kDetectScratchBytes);
+    void* scratch = nullptr;
+    st = sq::detect_scratch(&scratch);
+    if (st != SQ_OK) return st;
+    // every count slot read by the compaction is written by this call first,
+    // so nothing in the scratch has to be cleared between calls
+    return sq::launch_detect(X, dt, M, K, ldx, threshold, min_ratio, outlier_idx, n_outliers, nullptr, nullptr,
+                             scratch, sq::as_cuda(stream));
+}
