@@ -109,8 +109,10 @@ class Layer:
         self.gamma = {"attn": d["gamma_attn"].float().contiguous(), "mlp": d["gamma_mlp"].float().contiguous()}
         self.W = d["W"]
         self.V = {k: e(M, K, dt=torch.bfloat16) for k in ("attn", "mlp")}
-        self.xmax = {k: e(K) for k in ("attn", "mlp")}
-        self.wmax = {k: e(K) for k in ("attn", "mlp")}
+        # the four running maxima share one buffer, cleared by one fill per step
+        self.maxima = e(4, K)
+        self.xmax = {"attn": self.maxima[0], "mlp": self.maxima[1]}
+        self.wmax = {"attn": self.maxima[2], "mlp": self.maxima[3]}
         self.s = {k: e(K) for k in ("attn", "mlp")}
         self.gp = {k: e(K) for k in ("attn", "mlp")}
         self.Wq = {k: e(*self.W[k].shape, dt=torch.int8) for k in self.W}
@@ -132,14 +134,13 @@ class Layer:
     def step(self, gemm_ev=None):
         sq, d = self.sq, self.d
         eps = d["eps"]
+        self.maxima.zero_()
         for k in ("attn", "mlp"):
             # a5 (calibration pass) -> linear input; a1 on it
             sq.sq_norm_smooth_quant(self.h[k], sq.SQ_RMSNORM, self.gamma[k], None, eps, True, None, None, None,
                                     None, self.V[k])
-            self.xmax[k].zero_()
             sq.sq_calib_absmax(self.V[k], self.xmax[k])
         for k, w in (("attn", "qkv"), ("mlp", "gateup")):
-            self.wmax[k].zero_()
             sq.sq_weight_absmax(self.W[w], self.wmax[k])                       # a2
             sq.sq_smooth_scales(self.xmax[k], self.wmax[k], d["alpha"], self.s[k])  # a3
             sq.sq_fold_norm(self.gamma[k], None, self.s[k], self.gp[k])

@@ -25,6 +25,8 @@ template <typename T>
 __global__ void __launch_bounds__(kWarps * 32)
 col_absmax_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, int rows_per_block,
                   float* __restrict__ out) {
+    pdl_wait();
+    pdl_trigger();
     constexpr int V = Vec<T>::N;
     constexpr int COLS = 32 * V;
     __shared__ float red[kWarps][COLS];
@@ -59,6 +61,7 @@ col_absmax_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, int
     }
 #pragma unroll
     for (int e = 0; e < V; ++e) red[warp][lane * V + e] = m[e];
+    __syncwarp();  // lanes may have diverged above; bar.sync needs whole warps
     __syncthreads();
     for (int c = threadIdx.x; c < COLS; c += kWarps * 32) {
         float v = red[0][c];
@@ -86,7 +89,7 @@ sq_status_t launch(const void* X, int64_t M, int64_t K, int64_t ld, float* out, 
     SQ_REQUIRE(row_blocks <= 65535, SQ_ERR_UNSUPPORTED_SHAPE, "%s: too many rows (M=%lld)", name,
                (long long)M);
     dim3 grid((unsigned)col_blocks, (unsigned)row_blocks);
-    col_absmax_kernel<T><<<grid, kWarps * 32, 0, s>>>(static_cast<const T*>(X), M, K, ld, (int)rpb, out);
+    launch_pdl(col_absmax_kernel<T>, dim3(grid), dim3(kWarps * 32), 0, s, static_cast<const T*>(X), M, K, ld, (int)rpb, out);
     return check_launch(name);
 }
 

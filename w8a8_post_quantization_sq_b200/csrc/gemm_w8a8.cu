@@ -6,8 +6,9 @@
 // （四）：SmoothQuant", 为什么激活不能用逐通道量化):
 //   acc[i,j] = sum_k Xq[i,k] * Wq[j,k]            exact in int32
 //   Y[i,j]   = acc * ((1/qs_x[i]) * (1/qs_w[j])) (+ h[i,j]) (+ bias[j])
-// where h is the outlier term sum_{o in O} X16[i,o] * W16[j,o] of §2.2
-// (fp32 fma in ascending o; the 16-bit products are exact in fp32).
+// where h is the outlier term sum_{o in O} X16[i,o] * W16[j,o] of §2.2,
+// added to the dequantised value by fp32 fma in ascending o (the 16-bit
+// products are exact in fp32).
 //
 // Design (sm_100a):
 //   - persistent: one 192-thread CTA per SM loops over 128 x BN output tiles,
@@ -19,9 +20,12 @@
 //     N=BN, K=32 each, four per stage) into a double-buffered int32
 //     accumulator in tensor memory (2 x BN of the 512 columns), and frees
 //     ring stages and accumulator buffers with tcgen05.commit;
-//   - warps 2..5 read the accumulator with tcgen05.ld (warp w owns TMEM lanes
-//     32*(w%4)..+31 = tile rows), dequantise in fp32 and store the row
-//     segments, while the next tile's MMAs run in the other buffer.
+//   - warps 2..9 read the accumulator with tcgen05.ld (warp w owns TMEM lanes
+//     32*(w%4)..+31 = tile rows, and half of the columns), double-buffering
+//     the loads, dequantise in fp32, stage 32 x 32 chunks in shared memory
+//     and write whole row segments, while the next tile's MMAs run in the
+//     other accumulator buffer; the buffer is released right after its
+//     last load.
 // Every wait is bounded (about 2 s of %globaltimer); on expiry the kernel
 // records code 0x6E1 + role in the status word, drains its own TMA copies and
 // MMAs, frees its tensor memory and returns.
@@ -38,12 +42,12 @@ constexpr int BM = 128;
 constexpr int BK = 128;  // one 128-byte swizzle row of int8
 constexpr int UMMA_K = 32;
 constexpr int STAGES = 4;
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;  // two per TMEM lane quarter, each on half the tile's columns
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
-// staging row strides: 64 B (16-bit) / 128 B (32-bit) of data + 16 B pad
-constexpr int kStg16 = 80;
-constexpr int kStg32 = 144;
-constexpr int kStgWarpBytes = 32 * kStg32;
+// staging: 32 rows x 64 B of data (32 16-bit or 16 32-bit values) + 16 B pad
+constexpr int kStgRow = 80;
+constexpr int kStgWarpBytes = 32 * kStgRow;
 enum OutKind { kOutBF16 = 0, kOutF16 = 1, kOutF32 = 2, kOutI32 = 3 };
 
 template <int BN>
@@ -58,10 +62,10 @@ struct Cfg {
     static constexpr uint32_t MISC_OFF = BAR_OFF + NBAR * 8;  // tmem base, abort flag
     // per epilogue warp: 1/qs_w and bias of the tile's columns
     static constexpr uint32_t RW_OFF = (MISC_OFF + 16 + 15) / 16 * 16;
-    static constexpr uint32_t RW_BYTES = 4 * 2 * BN * 4;
+    static constexpr uint32_t RW_BYTES = kEpiWarps * 2 * (BN / 2) * 4;
     // per epilogue warp: a 32 x 32 output chunk (rows padded to avoid bank conflicts)
     static constexpr uint32_t STG_OFF = RW_OFF + RW_BYTES;
-    static constexpr uint32_t STG_BYTES = 4 * kStgWarpBytes;
+    static constexpr uint32_t STG_BYTES = kEpiWarps * kStgWarpBytes;
     static constexpr uint32_t SMEM = STG_OFF + STG_BYTES;
     static constexpr uint32_t SMEM_ALLOC = SMEM + 1024;  // slack to align the base to 1024
     static constexpr uint32_t TMEM_COLS = 2 * BN;
@@ -180,6 +184,31 @@ __device__ __forceinline__ void umma_commit(uint32_t bar) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
+// Issue a 32-column TMEM load without waiting; tmem_wait(r) completes it. The
+// wait names the destination registers so no use of them moves above it.
+__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t* r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait(uint32_t* r) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                   "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+                   "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
+                   "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+                 :
+                 : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
@@ -210,6 +239,130 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
     }
 }
 
+
+// One 32-column chunk of one warp's 32 rows: dequantise (and add the outlier
+// term and bias), stage the chunk in shared memory, then write it out as
+// whole 64-byte row segments (four lanes per row for 16-bit outputs; 32-bit
+// outputs go out in two 16-column halves).
+template <int OUT, bool OUTL>
+__device__ __forceinline__ void epi_chunk(const Params& p, const uint32_t* r, int cw, int col0, int row0, int64_t row,
+                                          bool row_ok, float rx, const float* rw_w, const float* bias_w, uint8_t* stg,
+                                          int lane, int n_out, bool compact) {
+    const GemmEpilogue& ep = p.ep;
+    float y[32];
+    if constexpr (OUT == kOutI32) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) y[e] = __int_as_float((int)r[e]);  // raw bits, stored unchanged
+    } else {
+        const float4* rw4 = reinterpret_cast<const float4*>(rw_w + cw);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float4 w = rw4[e];
+            y[4 * e + 0] = __fmul_rn((float)(int)r[4 * e + 0], __fmul_rn(rx, w.x));
+            y[4 * e + 1] = __fmul_rn((float)(int)r[4 * e + 1], __fmul_rn(rx, w.y));
+            y[4 * e + 2] = __fmul_rn((float)(int)r[4 * e + 2], __fmul_rn(rx, w.z));
+            y[4 * e + 3] = __fmul_rn((float)(int)r[4 * e + 3], __fmul_rn(rx, w.w));
+        }
+        if constexpr (OUTL) {
+            // the 16-bit outlier term, added term by term in ascending o with
+            // fma (the 16-bit products are exact in fp32)
+            if (compact) {
+                for (int o = 0; o < n_out; ++o) {
+                    const float xo = row_ok ? ep.xo[row * kOutlierCap + o] : 0.0f;
+                    const float4* w4 = reinterpret_cast<const float4*>(ep.wo + (int64_t)o * ep.wo_ld + col0);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float4 w = __ldg(w4 + e);
+                        y[4 * e + 0] = __fmaf_rn(xo, w.x, y[4 * e + 0]);
+                        y[4 * e + 1] = __fmaf_rn(xo, w.y, y[4 * e + 1]);
+                        y[4 * e + 2] = __fmaf_rn(xo, w.z, y[4 * e + 2]);
+                        y[4 * e + 3] = __fmaf_rn(xo, w.w, y[4 * e + 3]);
+                    }
+                }
+            } else {
+                for (int o = 0; o < n_out; ++o) {
+                    const int ko = ep.idx[o];
+                    const float xo = row_ok ? load16(ep.x16, row * ep.ldx16 + ko, ep.in16_bf16) : 0.0f;
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int col = min(col0 + e, p.N - 1);
+                        y[e] = __fmaf_rn(xo, load16(ep.w16, (int64_t)col * p.K + ko, ep.in16_bf16), y[e]);
+                    }
+                }
+            }
+        }
+        if (ep.bias) {
+            const float4* b4 = reinterpret_cast<const float4*>(bias_w + cw);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float4 b = b4[e];
+                y[4 * e + 0] = __fadd_rn(y[4 * e + 0], b.x);
+                y[4 * e + 1] = __fadd_rn(y[4 * e + 1], b.y);
+                y[4 * e + 2] = __fadd_rn(y[4 * e + 2], b.z);
+                y[4 * e + 3] = __fadd_rn(y[4 * e + 3], b.w);
+            }
+        }
+    }
+    if constexpr (OUT == kOutBF16 || OUT == kOutF16) {
+        uint4* dst = reinterpret_cast<uint4*>(stg + lane * kStgRow);
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            dst[e] = make_uint4(pack2<OUT>(y[8 * e], y[8 * e + 1]), pack2<OUT>(y[8 * e + 2], y[8 * e + 3]),
+                                pack2<OUT>(y[8 * e + 4], y[8 * e + 5]), pack2<OUT>(y[8 * e + 6], y[8 * e + 7]));
+        __syncwarp();
+        const int part = lane & 3;
+#pragma unroll
+        for (int it = 0; it < 4; ++it) {
+            const int rr = it * 8 + (lane >> 2);
+            const int64_t grow = (int64_t)row0 + rr;
+            const int col = col0 + part * 8;
+            const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * kStgRow + part * 16);
+            if (grow < p.M && col < p.N) {
+                uint16_t* out = static_cast<uint16_t*>(ep.Y) + grow * ep.ldy + col;
+                if (p.vec_store && col + 8 <= p.N) {
+                    *reinterpret_cast<uint4*>(out) = v;
+                } else {
+                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        if (col + e < p.N) out[e] = (uint16_t)(w[e >> 1] >> (16 * (e & 1)));
+                }
+            }
+        }
+        __syncwarp();
+    } else {
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            uint4* dst = reinterpret_cast<uint4*>(stg + lane * kStgRow);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                dst[e] = make_uint4(__float_as_uint(y[16 * hh + 4 * e]), __float_as_uint(y[16 * hh + 4 * e + 1]),
+                                    __float_as_uint(y[16 * hh + 4 * e + 2]), __float_as_uint(y[16 * hh + 4 * e + 3]));
+            __syncwarp();
+            const int part = lane & 3;
+#pragma unroll
+            for (int it = 0; it < 4; ++it) {
+                const int rr = it * 8 + (lane >> 2);
+                const int64_t grow = (int64_t)row0 + rr;
+                const int col = col0 + 16 * hh + part * 4;
+                const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * kStgRow + part * 16);
+                if (grow < p.M && col < p.N) {
+                    uint32_t* out = static_cast<uint32_t*>(ep.Y) + grow * ep.ldy + col;
+                    if (p.vec_store && col + 4 <= p.N) {
+                        *reinterpret_cast<uint4*>(out) = v;
+                    } else {
+                        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            if (col + e < p.N) out[e] = w[e];
+                    }
+                }
+            }
+            __syncwarp();
+        }
+    }
+}
+
 template <int BN, int OUT, bool OUTL>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
@@ -236,7 +389,7 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(tfull_bar(a), 1);
-            mbar_init(tempty_bar(a), 4);
+            mbar_init(tempty_bar(a), kEpiWarps);
         }
         mbar_init(drain_bar, 1);
         *abort_flag = 0;
@@ -252,10 +405,16 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_a)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_b)) : "memory");
     }
+    // bar.sync is an aligned barrier: every warp must reach it converged
+    __syncwarp();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
+    // the set-up above touches only this CTA's shared and tensor memory; wait
+    // here for the previous kernel in the stream before any global access
+    pdl_wait();
+    pdl_trigger();
 
     const int num_tiles = p.num_m * p.num_n;
     if (warp == 0) {
@@ -329,24 +488,30 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
         }
     } else {
         // -------------------------------------------------------- epilogue
-        // No block-level barrier is used here: an abort can make one warp leave
-        // early, so each warp stages its own per-column factors and output
-        // chunks and decides collectively (all lanes) whether to go on.
-        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        // Eight warps: warp w reads TMEM lanes 32*(w%4)..+31 (its tile rows)
+        // and half h = (w-2)/4 of the tile's columns. No block-level barrier
+        // is used here: an abort can make one warp leave early, so each warp
+        // stages its own column factors and output chunks and decides
+        // collectively (all lanes) whether to go on.
+        const int q = warp & 3;
+        const int half = (warp - 2) >> 2;
+        constexpr int HC = BN / 2;        // columns per warp
+        constexpr int NCH = HC / 32;      // 32-column chunks per warp
         const GemmEpilogue& ep = p.ep;
         const int n_out = OUTL ? *ep.n_out : 0;
         const bool compact = n_out <= kOutlierCap;
-        float* rw_w = rw_s + (warp - 2) * 2 * BN;  // this warp's 1/qs_w and bias
-        float* bias_w = rw_w + BN;
+        float* rw_w = rw_s + (warp - 2) * 2 * HC;  // this warp's 1/qs_w and bias
+        float* bias_w = rw_w + HC;
         uint8_t* stg = smem + C::STG_OFF + (warp - 2) * kStgWarpBytes;
         int local = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
             int m0, n0;
             tile_coords(tile, p, BN, m0, n0);
+            const int c_base = n0 + half * HC;  // first column of this warp
             if constexpr (OUT != kOutI32) {
                 __syncwarp();
-                for (int c = lane; c < BN; c += 32) {
-                    const int col = n0 + c;
+                for (int c = lane; c < HC; c += 32) {
+                    const int col = c_base + c;
                     float rw = 0.0f, b = 0.0f;
                     if (col < p.N) {
                         rw = __frcp_rn(ep.w_per_channel ? ep.qs_w[col] : ep.qs_w[0]);
@@ -368,138 +533,69 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
             float rx = 0.0f;
             if constexpr (OUT != kOutI32)
                 if (row_ok) rx = __frcp_rn(ep.x_per_token ? ep.qs_x[row] : ep.qs_x[0]);
-            const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-            if (row0 < p.M) {
-#pragma unroll 1
-                for (int c = 0; c < BN / 32; ++c) {
-                    const int col0 = n0 + c * 32;
-                    if (col0 >= p.N) break;
-                    uint32_t r[32];
-                    tmem_ld32(t_row + (uint32_t)(c * 32), r);
-                    // 1) this thread's row of the chunk into the warp's staging buffer
-                    if constexpr (OUT == kOutI32) {
-                        uint4* dst = reinterpret_cast<uint4*>(stg + lane * kStg32);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) dst[e] = make_uint4(r[4 * e], r[4 * e + 1], r[4 * e + 2], r[4 * e + 3]);
-                    } else {
-                        float y[32];
-                        const float4* rw4 = reinterpret_cast<const float4*>(rw_w + c * 32);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const float4 w = rw4[e];
-                            y[4 * e + 0] = __fmul_rn((float)(int)r[4 * e + 0], __fmul_rn(rx, w.x));
-                            y[4 * e + 1] = __fmul_rn((float)(int)r[4 * e + 1], __fmul_rn(rx, w.y));
-                            y[4 * e + 2] = __fmul_rn((float)(int)r[4 * e + 2], __fmul_rn(rx, w.z));
-                            y[4 * e + 3] = __fmul_rn((float)(int)r[4 * e + 3], __fmul_rn(rx, w.w));
-                        }
-                        if constexpr (OUTL) {
-                            float h[32];
-#pragma unroll
-                            for (int e = 0; e < 32; ++e) h[e] = 0.0f;
-                            if (compact) {
-                                for (int o = 0; o < n_out; ++o) {
-                                    const float xo = row_ok ? ep.xo[row * kOutlierCap + o] : 0.0f;
-                                    const float4* w4 = reinterpret_cast<const float4*>(ep.wo + (int64_t)o * ep.wo_ld + col0);
-#pragma unroll
-                                    for (int e = 0; e < 8; ++e) {
-                                        const float4 w = __ldg(w4 + e);
-                                        h[4 * e + 0] = __fmaf_rn(xo, w.x, h[4 * e + 0]);
-                                        h[4 * e + 1] = __fmaf_rn(xo, w.y, h[4 * e + 1]);
-                                        h[4 * e + 2] = __fmaf_rn(xo, w.z, h[4 * e + 2]);
-                                        h[4 * e + 3] = __fmaf_rn(xo, w.w, h[4 * e + 3]);
-                                    }
-                                }
-                            } else {
-                                for (int o = 0; o < n_out; ++o) {
-                                    const int ko = ep.idx[o];
-                                    const float xo = row_ok ? load16(ep.x16, row * ep.ldx16 + ko, ep.in16_bf16) : 0.0f;
-#pragma unroll
-                                    for (int e = 0; e < 32; ++e) {
-                                        const int col = min(col0 + e, p.N - 1);
-                                        h[e] = __fmaf_rn(xo, load16(ep.w16, (int64_t)col * p.K + ko, ep.in16_bf16), h[e]);
-                                    }
-                                }
-                            }
-#pragma unroll
-                            for (int e = 0; e < 32; ++e) y[e] = __fadd_rn(y[e], h[e]);
-                        }
-                        if (ep.bias) {
-                            const float4* b4 = reinterpret_cast<const float4*>(bias_w + c * 32);
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) {
-                                const float4 b = b4[e];
-                                y[4 * e + 0] = __fadd_rn(y[4 * e + 0], b.x);
-                                y[4 * e + 1] = __fadd_rn(y[4 * e + 1], b.y);
-                                y[4 * e + 2] = __fadd_rn(y[4 * e + 2], b.z);
-                                y[4 * e + 3] = __fadd_rn(y[4 * e + 3], b.w);
-                            }
-                        }
-                        if constexpr (OUT == kOutF32) {
-                            uint4* dst = reinterpret_cast<uint4*>(stg + lane * kStg32);
-#pragma unroll
-                            for (int e = 0; e < 8; ++e)
-                                dst[e] = make_uint4(__float_as_uint(y[4 * e]), __float_as_uint(y[4 * e + 1]),
-                                                    __float_as_uint(y[4 * e + 2]), __float_as_uint(y[4 * e + 3]));
-                        } else {
-                            uint4* dst = reinterpret_cast<uint4*>(stg + lane * kStg16);
-#pragma unroll
-                            for (int e = 0; e < 4; ++e)
-                                dst[e] = make_uint4(pack2<OUT>(y[8 * e], y[8 * e + 1]), pack2<OUT>(y[8 * e + 2], y[8 * e + 3]),
-                                                    pack2<OUT>(y[8 * e + 4], y[8 * e + 5]), pack2<OUT>(y[8 * e + 6], y[8 * e + 7]));
-                        }
+            const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + half * HC);
+            // chunks that hold at least one valid column; none when the rows are past M
+            int nch = 0;
+            if (row0 < p.M && c_base < p.N) nch = min(NCH, (p.N - c_base + 31) / 32);
+            // Double-buffered TMEM loads only where the variant keeps every
+            // value in registers (no spill may sit between a load and its wait).
+            constexpr bool kPipe = !OUTL && OUT != kOutF32;
+            uint32_t ra[32];
+            if constexpr (kPipe) {
+                uint32_t rb[32];
+                if (nch > 0) {
+                    tmem_ld32_async(t_row, ra);
+                    tmem_wait(ra);
+                }
+                for (int c = 0; c < nch; c += 2) {
+                    // chunk c is in ra; fetch chunk c+1 into rb while ra is used
+                    const bool more = c + 1 < nch;
+                    if (more) tmem_ld32_async(t_row + (uint32_t)((c + 1) * 32), rb);
+                    else {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(tempty_bar(acc));  // accumulator read in full
                     }
-                    __syncwarp();
-                    // 2) copy out with whole row segments per group of lanes
-                    if constexpr (OUT == kOutBF16 || OUT == kOutF16) {
-                        const int part = lane & 3;
-#pragma unroll
-                        for (int it = 0; it < 4; ++it) {
-                            const int rr = it * 8 + (lane >> 2);
-                            const int64_t grow = (int64_t)row0 + rr;
-                            const int col = col0 + part * 8;
-                            const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * kStg16 + part * 16);
-                            if (grow < p.M && col < p.N) {
-                                uint16_t* dst = static_cast<uint16_t*>(ep.Y) + grow * ep.ldy + col;
-                                if (p.vec_store && col + 8 <= p.N) {
-                                    *reinterpret_cast<uint4*>(dst) = v;
-                                } else {
-                                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                                    for (int e = 0; e < 8; ++e)
-                                        if (col + e < p.N) dst[e] = (uint16_t)(w[e >> 1] >> (16 * (e & 1)));
-                                }
-                            }
-                        }
-                    } else {
-                        const int part = lane & 7;
-#pragma unroll
-                        for (int it = 0; it < 8; ++it) {
-                            const int rr = it * 4 + (lane >> 3);
-                            const int64_t grow = (int64_t)row0 + rr;
-                            const int col = col0 + part * 4;
-                            const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * kStg32 + part * 16);
-                            if (grow < p.M && col < p.N) {
-                                uint32_t* dst = static_cast<uint32_t*>(ep.Y) + grow * ep.ldy + col;
-                                if (p.vec_store && col + 4 <= p.N) {
-                                    *reinterpret_cast<uint4*>(dst) = v;
-                                } else {
-                                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                                    for (int e = 0; e < 4; ++e)
-                                        if (col + e < p.N) dst[e] = w[e];
-                                }
-                            }
-                        }
+                    epi_chunk<OUT, OUTL>(p, ra, c * 32, c_base + c * 32, row0, row, row_ok, rx, rw_w, bias_w, stg,
+                                         lane, n_out, compact);
+                    if (!more) break;
+                    tmem_wait(rb);
+                    const bool more2 = c + 2 < nch;
+                    if (more2) tmem_ld32_async(t_row + (uint32_t)((c + 2) * 32), ra);
+                    else {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(tempty_bar(acc));
                     }
-                    __syncwarp();
+                    epi_chunk<OUT, OUTL>(p, rb, (c + 1) * 32, c_base + (c + 1) * 32, row0, row, row_ok, rx, rw_w,
+                                         bias_w, stg, lane, n_out, compact);
+                    if (more2) tmem_wait(ra);
+                }
+            } else {
+                for (int c = 0; c < nch; ++c) {
+                    tmem_ld32(t_row + (uint32_t)(c * 32), ra);
+                    if (c + 1 == nch) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(tempty_bar(acc));  // accumulator read in full
+                    }
+                    epi_chunk<OUT, OUTL>(p, ra, c * 32, c_base + c * 32, row0, row, row_ok, rx, rw_w, bias_w, stg,
+                                         lane, n_out, compact);
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(tempty_bar(acc));
+            if (nch == 0) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(tempty_bar(acc));
+            }
         }
     }
 
+    // Lanes 1..31 of warps 0 and 1 reach this point long before their lane 0
+    // finishes its role loop; reconverge each warp first, because bar.sync is
+    // an aligned barrier and must be executed by whole warps. Only then is
+    // every MMA drained and every TMEM read done before the dealloc.
+    __syncwarp();
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -579,7 +675,7 @@ sq_status_t launch_bn(const int8_t* Xq, const int8_t* Wq, int64_t M, int64_t N, 
     p.status = status;
     const int tiles = p.num_m * p.num_n;
     const int grid = tiles < num_sms() ? tiles : num_sms();
-    fn<<<grid, kThreads, C::SMEM_ALLOC, stream>>>(ta, tb, p);
+    launch_pdl(fn, dim3(grid), dim3(kThreads), C::SMEM_ALLOC, stream, ta, tb, p);
     return check_launch("sq_gemm_w8a8");
 }
 

@@ -52,6 +52,8 @@ constexpr int kCompactThreads = 1024;
 template <typename T>
 __global__ void __launch_bounds__(kWarps * 32)
 count_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, float thr, int32_t* __restrict__ partial) {
+    pdl_wait();
+    pdl_trigger();
     __shared__ int32_t red[kWarps][256];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t c0 = (int64_t)blockIdx.x * 256 + lane * 8;
@@ -68,6 +70,7 @@ count_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, float th
     }
 #pragma unroll
     for (int e = 0; e < 8; ++e) red[warp][lane * 8 + e] = cnt[e];
+    __syncwarp();  // lanes may have diverged above; bar.sync needs whole warps
     __syncthreads();
     for (int c = threadIdx.x; c < 256; c += kWarps * 32) {
         int32_t s = 0;
@@ -83,11 +86,14 @@ __global__ void __launch_bounds__(kCompactThreads)
 compact_kernel(const int32_t* __restrict__ partial, int64_t row_blocks, int64_t M, int64_t K, double min_ratio,
                int32_t* __restrict__ idx, int32_t* __restrict__ n_out, int32_t* __restrict__ cached_idx,
                int32_t* __restrict__ cached_n, int32_t* __restrict__ changed) {
+    pdl_wait();
+    pdl_trigger();
     __shared__ int32_t warp_tot[kCompactThreads / 32];
     __shared__ int32_t base_sh;
     __shared__ int32_t diff_sh;
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     if (t == 0) base_sh = 0, diff_sh = 0;
+    __syncwarp();
     __syncthreads();
     for (int64_t j0 = 0; j0 < K; j0 += kCompactThreads) {
         const int64_t j = j0 + t;
@@ -101,16 +107,19 @@ compact_kernel(const int32_t* __restrict__ partial, int64_t row_blocks, int64_t 
         const unsigned bal = __ballot_sync(0xffffffffu, flag);
         const int before_in_warp = __popc(bal & ((1u << lane) - 1u));
         if (lane == 0) warp_tot[warp] = __popc(bal);
+        __syncwarp();
         __syncthreads();
         int before = base_sh;
         for (int w = 0; w < warp; ++w) before += warp_tot[w];
         if (flag) idx[before + before_in_warp] = (int32_t)j;
+        __syncwarp();
         __syncthreads();
         if (t == 0) {
             int s = 0;
             for (int w = 0; w < kCompactThreads / 32; ++w) s += warp_tot[w];
             base_sh += s;
         }
+        __syncwarp();
         __syncthreads();
     }
     const int n = base_sh;
@@ -118,10 +127,12 @@ compact_kernel(const int32_t* __restrict__ partial, int64_t row_blocks, int64_t 
     if (cached_n) {
         const int cn = *cached_n;
         if (cn != n) diff_sh = 1;
+        __syncwarp();
         __syncthreads();
         if (!diff_sh)
             for (int o = t; o < n; o += kCompactThreads)
                 if (cached_idx[o] != idx[o]) diff_sh = 1;
+        __syncwarp();
         __syncthreads();
         const int d = diff_sh;
         if (d) {
@@ -139,16 +150,20 @@ __global__ void __launch_bounds__(256)
 masked_quant_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, const int32_t* __restrict__ idx,
                     const int32_t* __restrict__ n_idx, const int32_t* __restrict__ only_if, int8_t* __restrict__ Q,
                     float* __restrict__ qs_out, float* __restrict__ xo) {
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ uint32_t mask[];  // K bits
     if (only_if && *only_if == 0) return;
     const int64_t words = (K + 31) / 32;
     for (int64_t w = threadIdx.x; w < words; w += blockDim.x) mask[w] = 0u;
+    __syncwarp();
     __syncthreads();
     const int n = *n_idx;
     for (int o = threadIdx.x; o < n; o += blockDim.x) {
         const int j = idx[o];
         atomicOr(&mask[j >> 5], 1u << (j & 31));
     }
+    __syncwarp();
     __syncthreads();
     const int lane = threadIdx.x & 31;
     const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
@@ -195,6 +210,8 @@ masked_quant_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, c
 template <typename T>
 __global__ void gather_wo_kernel(const T* __restrict__ W, int64_t N, int64_t K, const int32_t* __restrict__ idx,
                                  const int32_t* __restrict__ n_idx, float* __restrict__ wo, int64_t ld) {
+    pdl_wait();
+    pdl_trigger();
     const int n = min(*n_idx, kOutlierCap);
     for (int64_t j = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; j < ld; j += (int64_t)gridDim.x * blockDim.x)
         for (int o = 0; o < n; ++o) {
@@ -220,12 +237,12 @@ sq_status_t launch_detect(const void* X, sq_dtype_t dt, int64_t M, int64_t K, in
         SQ_REQUIRE(rb <= 65535, SQ_ERR_UNSUPPORTED_SHAPE, "sq_llmint8_detect: M too large");
         dim3 grid((unsigned)((K + 255) / 256), (unsigned)rb);
         if (dt == SQ_BF16)
-            count_kernel<__nv_bfloat16><<<grid, kWarps * 32, 0, s>>>(static_cast<const __nv_bfloat16*>(X), M, K, ldx,
+            launch_pdl(count_kernel<__nv_bfloat16>, dim3(grid), dim3(kWarps * 32), 0, s, static_cast<const __nv_bfloat16*>(X), M, K, ldx,
                                                                       thr, partial);
         else
-            count_kernel<__half><<<grid, kWarps * 32, 0, s>>>(static_cast<const __half*>(X), M, K, ldx, thr, partial);
+            launch_pdl(count_kernel<__half>, dim3(grid), dim3(kWarps * 32), 0, s, static_cast<const __half*>(X), M, K, ldx, thr, partial);
     }
-    compact_kernel<<<1, kCompactThreads, 0, s>>>(partial, rb, M, K, min_ratio, idx, n_out, cached_idx, cached_n,
+    launch_pdl(compact_kernel, dim3(1), dim3(kCompactThreads), 0, s, partial, rb, M, K, min_ratio, idx, n_out, cached_idx, cached_n,
                                                  changed);
     return check_launch("sq_llmint8_detect");
 }
@@ -240,11 +257,11 @@ sq_status_t launch_masked_quant(const void* X, sq_dtype_t dt, int64_t M, int64_t
     if (dt == SQ_BF16) {
         auto k = masked_quant_kernel<__nv_bfloat16>;
         if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        k<<<(unsigned)grid, 256, smem, s>>>(static_cast<const __nv_bfloat16*>(X), M, K, ldx, idx, n_idx, only_if, Q, qs, xo);
+        launch_pdl(k, dim3((unsigned)grid), dim3(256), smem, s, static_cast<const __nv_bfloat16*>(X), M, K, ldx, idx, n_idx, only_if, Q, qs, xo);
     } else {
         auto k = masked_quant_kernel<__half>;
         if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        k<<<(unsigned)grid, 256, smem, s>>>(static_cast<const __half*>(X), M, K, ldx, idx, n_idx, only_if, Q, qs, xo);
+        launch_pdl(k, dim3((unsigned)grid), dim3(256), smem, s, static_cast<const __half*>(X), M, K, ldx, idx, n_idx, only_if, Q, qs, xo);
     }
     return check_launch(name);
 }
@@ -348,10 +365,10 @@ sq_status_t sq_llmint8_matmul(const void* X, sq_dtype_t dt, int64_t M, int64_t K
         int64_t blocks = (wo_ld + 255) / 256;
         if (blocks > (int64_t)sq::num_sms() * 4) blocks = (int64_t)sq::num_sms() * 4;
         if (dt == SQ_BF16)
-            sq::gather_wo_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, s>>>(
+            sq::launch_pdl(sq::gather_wo_kernel<__nv_bfloat16>, dim3((unsigned)blocks), dim3(256), 0, s, 
                 static_cast<const __nv_bfloat16*>(w->W), w->N, K, idx_out, n_out, wo, wo_ld);
         else
-            sq::gather_wo_kernel<__half><<<(unsigned)blocks, 256, 0, s>>>(static_cast<const __half*>(w->W), w->N, K,
+            sq::launch_pdl(sq::gather_wo_kernel<__half>, dim3((unsigned)blocks), dim3(256), 0, s, static_cast<const __half*>(w->W), w->N, K,
                                                                          idx_out, n_out, wo, wo_ld);
         st = sq::check_launch(name);
         if (st != SQ_OK) return st;

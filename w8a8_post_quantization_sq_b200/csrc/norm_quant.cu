@@ -50,8 +50,10 @@ __device__ __forceinline__ float canon_block_sum(float p, float* sh) {
     for (int o = 16; o >= 1; o >>= 1) p = __fadd_rn(p, __shfl_xor_sync(0xffffffffu, p, o));
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     if (lane == 0) sh[warp] = p;
+    __syncwarp();
     __syncthreads();
     const float r = __fadd_rn(__fadd_rn(sh[0], sh[1]), __fadd_rn(sh[2], sh[3]));
+    __syncwarp();
     __syncthreads();
     return r;
 }
@@ -61,8 +63,10 @@ __device__ __forceinline__ float block_max4(float v, float* sh) {
     for (int o = 16; o >= 1; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     if (lane == 0) sh[warp] = v;
+    __syncwarp();
     __syncthreads();
     const float r = fmaxf(fmaxf(sh[0], sh[1]), fmaxf(sh[2], sh[3]));
+    __syncwarp();
     __syncthreads();
     return r;
 }
@@ -70,6 +74,8 @@ __device__ __forceinline__ float block_max4(float v, float* sh) {
 template <typename T, bool LN, int CMAX>
 __global__ void __launch_bounds__(kThreads)
 norm_quant_kernel(const T* __restrict__ H, NormArgs a) {
+    pdl_wait();
+    pdl_trigger();
     __shared__ float sh[4];
     extern __shared__ float amax_sh[];  // [K] running max |v| (calibration mode)
     const int t = threadIdx.x;
@@ -213,6 +219,7 @@ norm_quant_kernel(const T* __restrict__ H, NormArgs a) {
         }
     }
     if (a.absmax) {
+        __syncwarp();
         __syncthreads();
         // each column was only touched by its owning thread; publish once per block
         for (int j = t; j < a.K; j += kThreads) atomic_max_nonneg(a.absmax + j, amax_sh[j]);
@@ -224,12 +231,15 @@ norm_quant_kernel(const T* __restrict__ H, NormArgs a) {
 template <typename T, bool LN, int CW>
 __global__ void __launch_bounds__(256)
 norm_quant_warp_kernel(const T* __restrict__ H, NormArgs a) {
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ float amax_sh[];  // [K] running max |v| of the block (calibration mode)
     const int lane = threadIdx.x & 31;
     const int nch = (int)(a.K / 8);
     const float Kf = (float)a.K;
     if (a.absmax) {
         for (int j = threadIdx.x; j < a.K; j += blockDim.x) amax_sh[j] = 0.0f;
+        __syncwarp();
         __syncthreads();
     }
     const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
@@ -350,6 +360,7 @@ norm_quant_warp_kernel(const T* __restrict__ H, NormArgs a) {
         }
     }
     if (a.absmax) {
+        __syncwarp();
         __syncthreads();
         for (int j = threadIdx.x; j < a.K; j += blockDim.x) atomic_max_nonneg(a.absmax + j, amax_sh[j]);
     }
@@ -363,7 +374,7 @@ void launch_warp(const void* H, const NormArgs& a, cudaStream_t s) {
     int64_t blocks = (a.M + 7) / 8;  // 8 rows (warps) per block
     const int64_t cap = (int64_t)num_sms() * (a.absmax ? 2 : 8);
     if (blocks > cap) blocks = cap;
-    kern<<<(unsigned)blocks, 256, smem, s>>>(static_cast<const T*>(H), a);
+    launch_pdl(kern, dim3((unsigned)blocks), dim3(256), smem, s, static_cast<const T*>(H), a);
 }
 
 template <typename T, bool LN, int CMAX>
@@ -376,7 +387,7 @@ void launch_one(const void* H, const NormArgs& a, cudaStream_t s) {
     int64_t grid = (int64_t)num_sms() * per_sm;
     if (a.absmax) grid = (int64_t)num_sms() * 2;  // fewer blocks: one publish of [K] per block
     if (grid > a.M) grid = a.M;
-    kern<<<(unsigned)grid, kThreads, smem, s>>>(static_cast<const T*>(H), a);
+    launch_pdl(kern, dim3((unsigned)grid), dim3(kThreads), smem, s, static_cast<const T*>(H), a);
 }
 
 template <typename T, bool LN>

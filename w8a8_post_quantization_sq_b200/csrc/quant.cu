@@ -50,8 +50,10 @@ __device__ __forceinline__ float block_max(float v, float* sh) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    __syncwarp();
     __syncthreads();  // sh may still be read from a previous use
     if (lane == 0) sh[warp] = v;
+    __syncwarp();
     __syncthreads();
     float m = sh[0];
     for (int w = 1; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, sh[w]);
@@ -87,6 +89,8 @@ __global__ void __launch_bounds__(kThreads)
 row_quant_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, const float* __restrict__ s,
                  int per_row, const float* __restrict__ tensor_qs, int8_t* __restrict__ Q,
                  float* __restrict__ qs_out) {
+    pdl_wait();
+    pdl_trigger();
     const int lane = threadIdx.x & 31;
     const int64_t nwarps = (int64_t)gridDim.x * (kThreads / 32);
     for (int64_t row = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5; row < M; row += nwarps) {
@@ -128,6 +132,8 @@ __global__ void __launch_bounds__(kThreads)
 row_quant_reg_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, const float* __restrict__ s,
                      int per_row, const float* __restrict__ tensor_qs, int8_t* __restrict__ Q,
                      float* __restrict__ qs_out) {
+    pdl_wait();
+    pdl_trigger();
     __shared__ float sh[kThreads / 32];
     constexpr int GPB = kThreads / G;  // groups (rows) per block
     const int gt = threadIdx.x % G;
@@ -173,6 +179,8 @@ template <typename T, int SM>
 __global__ void __launch_bounds__(kThreads)
 tensor_absmax_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld,
                      const float* __restrict__ s, float* __restrict__ out) {
+    pdl_wait();
+    pdl_trigger();
     __shared__ float sh[kThreads / 32];
     const int64_t vecs_per_row = K / 8;
     const int64_t nvec = M * vecs_per_row;
@@ -193,6 +201,8 @@ tensor_absmax_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld,
 // qs = 127 / max(max_j a[j], 1e-8) into *qs (one block).
 __global__ void __launch_bounds__(kThreads)
 scale_from_absmax_kernel(const float* __restrict__ a, int64_t n, float* __restrict__ qs) {
+    pdl_wait();
+    pdl_trigger();
     __shared__ float sh[kThreads / 32];
     float m = 0.0f;
     for (int64_t j = threadIdx.x; j < n; j += kThreads) m = fmaxf(m, a[j]);
@@ -223,8 +233,8 @@ sq_status_t quantize(const void* Xv, int64_t M, int64_t K, int64_t ld, const flo
         float* wmax = reinterpret_cast<float*>(static_cast<char*>(ws) + 16);
         float* wqs = wmax + 1;
         if (cudaMemsetAsync(wmax, 0, sizeof(float), st) != cudaSuccess) return check_launch(name);
-        tensor_absmax_kernel<T, SM><<<vec_grid(M * K / 8), kThreads, 0, st>>>(X, M, K, ld, s, wmax);
-        scale_from_absmax_kernel<<<1, kThreads, 0, st>>>(wmax, 1, wqs);
+        launch_pdl(tensor_absmax_kernel<T, SM>, dim3(vec_grid(M * K / 8)), dim3(kThreads), 0, st, X, M, K, ld, s, wmax);
+        launch_pdl(scale_from_absmax_kernel, dim3(1), dim3(kThreads), 0, st, wmax, 1, wqs);
         tensor_qs = wqs;
     }
     const int64_t cap = (int64_t)num_sms() * 8;
@@ -233,21 +243,21 @@ sq_status_t quantize(const void* Xv, int64_t M, int64_t K, int64_t ld, const flo
         return (unsigned)(b < cap ? b : cap);
     };
     if (K <= 256)
-        row_quant_reg_kernel<T, SM, 32, 1><<<blocks(8), kThreads, 0, st>>>(X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
+        launch_pdl(row_quant_reg_kernel<T, SM, 32, 1>, dim3(blocks(8)), dim3(kThreads), 0, st, X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
     else if (K <= 512)
-        row_quant_reg_kernel<T, SM, 32, 2><<<blocks(8), kThreads, 0, st>>>(X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
+        launch_pdl(row_quant_reg_kernel<T, SM, 32, 2>, dim3(blocks(8)), dim3(kThreads), 0, st, X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
     else if (K <= 1024)
-        row_quant_reg_kernel<T, SM, 32, 4><<<blocks(8), kThreads, 0, st>>>(X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
+        launch_pdl(row_quant_reg_kernel<T, SM, 32, 4>, dim3(blocks(8)), dim3(kThreads), 0, st, X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
     else if (K <= 2048)
-        row_quant_reg_kernel<T, SM, 32, 8><<<blocks(8), kThreads, 0, st>>>(X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
+        launch_pdl(row_quant_reg_kernel<T, SM, 32, 8>, dim3(blocks(8)), dim3(kThreads), 0, st, X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
     else if (K <= 4096)
-        row_quant_reg_kernel<T, SM, 256, 2><<<blocks(1), kThreads, 0, st>>>(X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
+        launch_pdl(row_quant_reg_kernel<T, SM, 256, 2>, dim3(blocks(1)), dim3(kThreads), 0, st, X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
     else if (K <= 8192)
-        row_quant_reg_kernel<T, SM, 256, 4><<<blocks(1), kThreads, 0, st>>>(X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
+        launch_pdl(row_quant_reg_kernel<T, SM, 256, 4>, dim3(blocks(1)), dim3(kThreads), 0, st, X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
     else if (K <= 16384)
-        row_quant_reg_kernel<T, SM, 256, 8><<<blocks(1), kThreads, 0, st>>>(X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
+        launch_pdl(row_quant_reg_kernel<T, SM, 256, 8>, dim3(blocks(1)), dim3(kThreads), 0, st, X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
     else
-        row_quant_kernel<T, SM><<<row_grid(M), kThreads, 0, st>>>(X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
+        launch_pdl(row_quant_kernel<T, SM>, dim3(row_grid(M)), dim3(kThreads), 0, st, X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
     return check_launch(name);
 }
 
@@ -309,7 +319,7 @@ sq_status_t sq_quantize_act(const void* X, sq_dtype_t dt, int64_t M, int64_t K, 
 sq_status_t sq_scale_from_absmax(const float* absmax, int64_t n, float* qs_out, sq_stream_t stream) {
     SQ_REQUIRE(absmax && qs_out, SQ_ERR_INVALID_ARG, "sq_scale_from_absmax: null pointer");
     SQ_REQUIRE(n > 0, SQ_ERR_UNSUPPORTED_SHAPE, "sq_scale_from_absmax: n must be > 0");
-    sq::scale_from_absmax_kernel<<<1, sq::kThreads, 0, sq::as_cuda(stream)>>>(absmax, n, qs_out);
+    sq::launch_pdl(sq::scale_from_absmax_kernel, dim3(1), dim3(sq::kThreads), 0, sq::as_cuda(stream), absmax, n, qs_out);
     return sq::check_launch("sq_scale_from_absmax");
 }
 

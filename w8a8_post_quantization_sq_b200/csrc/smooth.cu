@@ -18,6 +18,8 @@ namespace {
 
 __global__ void smooth_scales_kernel(const float* __restrict__ x, const float* __restrict__ w,
                                      int64_t K, double alpha, float* __restrict__ s) {
+    pdl_wait();
+    pdl_trigger();
     for (int64_t j = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; j < K;
          j += (int64_t)gridDim.x * blockDim.x) {
         const float xc = fmaxf(x[j], 1e-5f);
@@ -38,6 +40,8 @@ __global__ void smooth_scales_kernel(const float* __restrict__ x, const float* _
 template <typename T>
 __global__ void fold_weight_kernel(const T* __restrict__ W, int64_t N, int64_t K,
                                    const float* __restrict__ s, float* __restrict__ Wp) {
+    pdl_wait();
+    pdl_trigger();
     constexpr int V = Vec<T>::N;
     const int64_t nvec = N * K / V;
     for (int64_t v = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; v < nvec;
@@ -57,6 +61,8 @@ __global__ void fold_weight_kernel(const T* __restrict__ W, int64_t N, int64_t K
 
 __global__ void fold_norm_kernel(const float* __restrict__ g, const float* __restrict__ b,
                                  const float* __restrict__ s, int64_t K, float* g_out, float* b_out) {
+    pdl_wait();
+    pdl_trigger();
     for (int64_t j = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; j < K;
          j += (int64_t)gridDim.x * blockDim.x) {
         const float sj = s[j];
@@ -84,7 +90,7 @@ sq_status_t sq_smooth_scales(const float* xmax, const float* wmax, int64_t K, do
     SQ_REQUIRE(xmax && wmax && s_out, SQ_ERR_INVALID_ARG, "sq_smooth_scales: null pointer");
     SQ_REQUIRE(K > 0, SQ_ERR_UNSUPPORTED_SHAPE, "sq_smooth_scales: K must be > 0");
     SQ_REQUIRE(alpha >= 0.0 && alpha <= 1.0, SQ_ERR_INVALID_ARG, "sq_smooth_scales: alpha must be in [0, 1]");
-    sq::smooth_scales_kernel<<<sq::grid_for(K, 256), 256, 0, sq::as_cuda(stream)>>>(xmax, wmax, K, alpha, s_out);
+    sq::launch_pdl(sq::smooth_scales_kernel, dim3(sq::grid_for(K, 256)), dim3(256), 0, sq::as_cuda(stream), xmax, wmax, K, alpha, s_out);
     return sq::check_launch("sq_smooth_scales");
 }
 
@@ -98,15 +104,15 @@ sq_status_t sq_fold_weight(const void* W, sq_dtype_t dt, int64_t N, int64_t K, c
     const int64_t n = N * K;
     switch (dt) {
         case SQ_F16:
-            sq::fold_weight_kernel<__half><<<sq::grid_for(n / 8, 256), 256, 0, st>>>(
+            sq::launch_pdl(sq::fold_weight_kernel<__half>, dim3(sq::grid_for(n / 8, 256)), dim3(256), 0, st, 
                 static_cast<const __half*>(W), N, K, s, Wp_out);
             break;
         case SQ_BF16:
-            sq::fold_weight_kernel<__nv_bfloat16><<<sq::grid_for(n / 8, 256), 256, 0, st>>>(
+            sq::launch_pdl(sq::fold_weight_kernel<__nv_bfloat16>, dim3(sq::grid_for(n / 8, 256)), dim3(256), 0, st, 
                 static_cast<const __nv_bfloat16*>(W), N, K, s, Wp_out);
             break;
         case SQ_F32:
-            sq::fold_weight_kernel<float><<<sq::grid_for(n / 4, 256), 256, 0, st>>>(
+            sq::launch_pdl(sq::fold_weight_kernel<float>, dim3(sq::grid_for(n / 4, 256)), dim3(256), 0, st, 
                 static_cast<const float*>(W), N, K, s, Wp_out);
             break;
         default: return sq::set_error(SQ_ERR_INVALID_ARG, "sq_fold_weight: dtype must be F16, BF16 or F32");
@@ -120,7 +126,7 @@ sq_status_t sq_fold_norm(const float* gamma, const float* beta, const float* s, 
     SQ_REQUIRE((beta == nullptr) == (beta_out == nullptr), SQ_ERR_INVALID_ARG,
                "sq_fold_norm: beta and beta_out must both be given or both be NULL");
     SQ_REQUIRE(K > 0, SQ_ERR_UNSUPPORTED_SHAPE, "sq_fold_norm: K must be > 0");
-    sq::fold_norm_kernel<<<sq::grid_for(K, 256), 256, 0, sq::as_cuda(stream)>>>(gamma, beta, s, K, gamma_out,
+    sq::launch_pdl(sq::fold_norm_kernel, dim3(sq::grid_for(K, 256)), dim3(256), 0, sq::as_cuda(stream), gamma, beta, s, K, gamma_out,
                                                                               beta_out);
     return sq::check_launch("sq_fold_norm");
 }

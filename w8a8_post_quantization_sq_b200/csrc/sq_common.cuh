@@ -10,6 +10,7 @@
 
 #include <cstdarg>
 #include <cstdio>
+#include <utility>
 
 #include "../../include/sq_api.h"
 
@@ -36,12 +37,40 @@ inline int dtype_bytes(sq_dtype_t dt) {
 
 int num_sms();  // SM count of the current device (cached per device)
 
+// Kernels are launched with programmatic stream serialisation: a kernel may
+// start (and run its prologue) while the previous kernel in the stream is
+// finishing. Every kernel executes pdl_wait() before it touches global memory,
+// which blocks until the previous grid has completed and its writes are
+// visible, so stream order is kept. SQ_DISABLE_PDL=1 turns this off.
+bool pdl_enabled();
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_enabled() ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 #define SQ_REQUIRE(cond, status, ...) \
     do {                              \
         if (!(cond)) return ::sq::set_error(status, __VA_ARGS__); \
     } while (0)
 
 // ---------------------------------------------------------------- device side
+// Wait for the previous grid in the stream (no-op without a programmatic
+// launch), then allow the next one to begin launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Element count of one 16-byte vector.
 template <typename T> struct Vec;
 template <> struct Vec<__half> { static constexpr int N = 8; };

@@ -1,4 +1,5 @@
 // Host-side status handling, workspace sizing and device queries.
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -24,6 +25,14 @@ sq_status_t check_launch(const char* what) {
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return set_error(SQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
     return SQ_OK;
+}
+
+bool pdl_enabled() {
+    static const bool on = [] {
+        const char* e = getenv("SQ_DISABLE_PDL");
+        return !(e && e[0] == '1');
+    }();
+    return on;
 }
 
 int num_sms() {
