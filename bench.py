@@ -13,8 +13,9 @@ fused 1024->4096, o 2048->1024, gate/up fused 1024->6144, down 3072->1024;
   a6 int8 GEMM + dequant epilogue to bf16                               x4
   a7-a9 LLM.int8 decomposition of the q/k/v projection (bf16)           x1
 The step is captured once in a CUDA graph and replayed. L2 is flushed (a
-256 MB write) before every timed step, outside the timed interval; each step is
-bracketed by CUDA events on the stream it runs on.
+256 MB write, then a 256 MB read of another buffer so that no dirty line of the
+flush is left to be written back) before every timed step, outside the timed
+interval; each step is bracketed by CUDA events on the stream it runs on.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -91,6 +92,25 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ GPU arm
+class L2Flush:
+    """Evicts L2 before a timed interval: a 256 MB write, then a 256 MB read of
+    another buffer, so the dirty lines of the write are written back before the
+    interval starts rather than inside it."""
+
+    def __init__(self, dev):
+        import torch
+
+        self.w = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+        self.r = torch.ones(64 * 1024 * 1024, dtype=torch.float32, device=dev)
+        self.out = torch.empty((), dtype=torch.float32, device=dev)
+
+    def __call__(self, i=1):
+        import torch
+
+        self.w.fill_(i & 0xFF)
+        torch.sum(self.r, dim=0, out=self.out)
+
+
 class Layer:
     """Device buffers and the step for the Qwen3-0.6B-shaped layer."""
 
@@ -184,7 +204,7 @@ def run_ours(args, rank, world, dev):
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
         L.step(gemm_ev)
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     for _ in range(max(args.warmup, 3)):
         graph.replay()
     torch.cuda.synchronize()
@@ -198,7 +218,7 @@ def run_ours(args, rank, world, dev):
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):
         for i in range(args.steps):
-            flush.fill_(i & 0xFF)
+            flush(i)
             ev[i][0].record(stream)
             graph.replay()
             ev[i][1].record(stream)
@@ -370,8 +390,8 @@ def run_kernel(args):
     shape = [int(x) for x in args.shape.split(",")]
     g = torch.Generator(device=dev).manual_seed(0)
     pk, src = peaks()
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
-    out = {"kernel": args.kernel, "shape": shape}
+    flush = L2Flush(dev)
+    out = {"kernel": args.kernel, "shape": shape, "dtype": args.dtype}
     if args.kernel == "gemm":
         M, N, K = shape
         Xq = torch.randint(-127, 128, (M, K), generator=g, device=dev, dtype=torch.int8)
@@ -384,26 +404,32 @@ def run_kernel(args):
         work, unit, peak = 2.0 * M * N * K / 1e12, "TOPS", 2.0 * pk["bf16_tflops"]
     elif args.kernel == "norm":
         M, K = shape
-        H = torch.randn((M, K), generator=g, device=dev).to(torch.bfloat16)
+        dt16 = torch.float16 if args.dtype == "fp16" else torch.bfloat16
+        H = torch.randn((M, K), generator=g, device=dev).to(dt16)
         gamma = torch.rand(K, generator=g, device=dev) + 0.5
+        beta = torch.randn(K, generator=g, device=dev) * 0.1 if args.norm == "ln" else None
+        nt = sq.SQ_LAYERNORM if args.norm == "ln" else sq.SQ_RMSNORM
         Xq = torch.empty((M, K), dtype=torch.int8, device=dev)
         qs = torch.empty(M, device=dev)
-        fn = lambda: sq.sq_norm_smooth_quant(H, sq.SQ_RMSNORM, gamma, None, 1e-6, True, None, Xq, qs)  # noqa: E731
+        fn = lambda: sq.sq_norm_smooth_quant(H, nt, gamma, beta, 1e-5, True, None, Xq, qs)  # noqa: E731
         work, unit, peak = (3.0 * M * K + 4 * M) / 1e9, "GB/s", pk["hbm_gbs"]
+        out["norm"] = args.norm
     elif args.kernel == "absmax":
         M, K = shape
-        X = torch.randn((M, K), generator=g, device=dev).to(torch.bfloat16)
+        dtx = {"fp16": torch.float16, "bf16": torch.bfloat16, "fp32": torch.float32}[args.dtype]
+        X = torch.randn((M, K), generator=g, device=dev).to(dtx)
         xmax = torch.zeros(K, device=dev)
         fn = lambda: sq.sq_calib_absmax(X, xmax)  # noqa: E731
-        work, unit, peak = 2.0 * M * K / 1e9, "GB/s", pk["hbm_gbs"]
+        work, unit, peak = X.element_size() * M * K / 1e9, "GB/s", pk["hbm_gbs"]
     elif args.kernel == "quant_weight":
         N, K = shape
-        W = (torch.randn((N, K), generator=g, device=dev) * 0.02).to(torch.bfloat16)
+        dtx = {"fp16": torch.float16, "bf16": torch.bfloat16, "fp32": torch.float32}[args.dtype]
+        W = (torch.randn((N, K), generator=g, device=dev) * 0.02).to(dtx)
         s_ = torch.rand(K, generator=g, device=dev) * 10 + 0.1
         Wq = torch.empty((N, K), dtype=torch.int8, device=dev)
         qw = torch.empty(N, device=dev)
         fn = lambda: sq.sq_quantize_weight(W, s_, True, Wq, qw)  # noqa: E731
-        work, unit, peak = (3.0 * N * K + 4 * N) / 1e9, "GB/s", pk["hbm_gbs"]
+        work, unit, peak = ((W.element_size() + 1.0) * N * K + 4 * N) / 1e9, "GB/s", pk["hbm_gbs"]
     elif args.kernel == "llmint8":
         from w8a8_post_quantization_sq_b200 import inputs
 
@@ -430,7 +456,7 @@ def run_kernel(args):
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
         for a, b in ev:
-            flush.fill_(1)
+            flush()
             a.record()
             fn()
             b.record()
@@ -447,6 +473,8 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--kernel", default=None, help="time one entry point alone: gemm|norm|absmax|quant_weight|llmint8")
     ap.add_argument("--shape", default="4096,36864,12288")
+    ap.add_argument("--dtype", default="bf16", help="input dtype of --kernel absmax|quant_weight|norm")
+    ap.add_argument("--norm", default="rms", help="--kernel norm: rms|ln")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
@@ -496,7 +524,7 @@ def main():
         "warmup": args.warmup, "ms_per_step": r["ms_per_step"], "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "i8", "data": "synthetic",
         "config": {"workload": WORKLOAD, "tokens": M_TOKENS, "hidden": HIDDEN, "parallelism": f"replicas x{world}",
-                   "l2": "flushed before every timed step (256 MB write, outside the timed interval)",
+                   "l2": "flushed before every timed step (256 MB write + 256 MB read, outside the timed interval)",
                    "graph": "one CUDA graph per step"},
         "gemm_tops": r["gemm_tops"], "gemm_avg_us": [x * 1e3 for x in r["gemm_avg_ms"]],
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": r["i8_peak"], "unit": "TOPS",

@@ -214,18 +214,19 @@ float or_scale_from_absmax(const float* absmax, int64_t n) {
 
 /* ------------------------------------------------------------------ a5
  * Fixed reduction order of the fp32 normalisation sums (reading R5; the pages
- * give the formula, not an order). With 128 lanes and chunks of 8 consecutive
+ * give the formula, not an order). With 256 lanes and chunks of 8 consecutive
  * elements:
- *   lane t folds chunks t, t+128, t+256, ... in increasing order; inside a
+ *   lane t folds chunks t, t+256, t+512, ... in increasing order; inside a
  *   chunk it folds elements in index order with acc = fma(a_j, b_j, acc);
  *   each group of 32 lanes is combined by the butterfly p[i] += p[i ^ off]
  *   for off = 16, 8, 4, 2, 1 (every lane ends with the same value);
- *   the four group totals G0..G3 combine as (G0 + G1) + (G2 + G3).
- * The GPU kernel reduces in exactly this order, so sums, and with them every
+ *   the eight group totals combine as ((G0+G1)+(G2+G3)) + ((G4+G5)+(G6+G7)).
+ * The GPU kernels reduce in exactly this order, so sums, and with them every
  * int8 code, are bit-identical. Parity of the exact fp32 bits is pinned only by
  * this convention ("parity unpinned" for the bits themselves); the value is
  * pinned to the fp64 normalisation to 1e-6 relative. */
-#define OR_LANES 128
+#define OR_LANES 256
+#define OR_GROUPS (OR_LANES / 32)
 #define OR_CHUNK 8
 static float canon_dot(const float* a, const float* b, int64_t K) {
     float p[OR_LANES];
@@ -239,8 +240,8 @@ static float canon_dot(const float* a, const float* b, int64_t K) {
             }
         p[t] = acc;
     }
-    float g[4];
-    for (int w = 0; w < 4; ++w) {
+    float g[OR_GROUPS];
+    for (int w = 0; w < OR_GROUPS; ++w) {
         float q[32], nq[32];
         for (int i = 0; i < 32; ++i) q[i] = p[32 * w + i];
         for (int off = 16; off >= 1; off >>= 1) {
@@ -249,7 +250,7 @@ static float canon_dot(const float* a, const float* b, int64_t K) {
         }
         g[w] = q[0];
     }
-    return (g[0] + g[1]) + (g[2] + g[3]);
+    return ((g[0] + g[1]) + (g[2] + g[3])) + ((g[4] + g[5]) + (g[6] + g[7]));
 }
 
 /* LayerNorm / RMSNorm with the folded gamma' (and beta'), fused with int8

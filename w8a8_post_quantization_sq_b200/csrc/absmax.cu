@@ -6,20 +6,20 @@
 // 解决激活值离群点难题" §3). With W stored [N,K] both are the same operation: a
 // column max over the rows of a row-major matrix, kept as a running max.
 //
-// Bandwidth kernel. A block of 8 warps covers 32 lanes x one 16-byte vector
-// of columns (256 columns of a 16-bit matrix, 128 of an fp32 one) and a band
-// of rows; warp w reads rows w, w+8, ... so every warp-wide load is one
-// contiguous 512-byte segment. Each lane keeps the running max of its vector
-// in registers, the 8 warps combine in shared memory, and one atomicMax per
-// column per block publishes the result. max and |.| are exact, so the
-// result does not depend on the order.
+// Bandwidth kernel. A block of 8 warps covers 32 lanes x four 16-byte vectors
+// of columns (1024 columns of a 16-bit matrix, 512 of an fp32 one) and a band
+// of rows; warp w reads rows w, w+8, ..., two rows per step, so every warp
+// reads 2 KB contiguous segments. Each lane keeps the running max of its
+// columns in registers, the warps combine with shared-memory atomics, and one
+// atomicMax per column per block publishes the result. max and |.| are exact,
+// so the result does not depend on the order.
 #include "sq_common.cuh"
 
 namespace sq {
 namespace {
 
 constexpr int kWarps = 8;
-constexpr int kUnroll = 4;
+constexpr int kU = 4;  // 16-byte vectors per lane per row: a warp reads 2 KB of a row
 
 template <typename T>
 __global__ void __launch_bounds__(kWarps * 32)
@@ -28,68 +28,88 @@ col_absmax_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, int
     pdl_wait();
     pdl_trigger();
     constexpr int V = Vec<T>::N;
-    constexpr int COLS = 32 * V;
-    __shared__ float red[kWarps][COLS];
+    constexpr int LC = V * kU;     // columns per lane
+    constexpr int COLS = 32 * LC;  // columns per block
+    __shared__ int red[COLS];      // block maxima as non-negative float bits
+    for (int c = threadIdx.x; c < COLS; c += kWarps * 32) red[c] = 0;
+    __syncwarp();
+    __syncthreads();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int64_t c0 = (int64_t)blockIdx.x * COLS + lane * V;
+    const int64_t c0 = (int64_t)blockIdx.x * COLS + lane * LC;
     const int64_t r_begin = (int64_t)blockIdx.y * rows_per_block;
     const int64_t r_end = min(M, r_begin + rows_per_block);
-    float m[V];
+    float m[LC];
 #pragma unroll
-    for (int e = 0; e < V; ++e) m[e] = 0.0f;
-    if (c0 < K) {
+    for (int e = 0; e < LC; ++e) m[e] = 0.0f;
+    int nv = 0;  // whole vectors of this lane inside K
+    if (c0 < K) nv = (int)min((int64_t)kU, (K - c0) / V);
+    if (nv > 0) {
         const T* base = X + c0;
         int64_t r = r_begin + warp;
-        for (; r + (kUnroll - 1) * kWarps < r_end; r += kUnroll * kWarps) {
-            uint4 raw[kUnroll];
+        for (; r + kWarps < r_end; r += 2 * kWarps) {
+            uint4 raw[2][kU];
 #pragma unroll
-            for (int u = 0; u < kUnroll; ++u) raw[u] = ldg_nc_v4(base + (r + u * kWarps) * ld);
+            for (int h = 0; h < 2; ++h)
 #pragma unroll
-            for (int u = 0; u < kUnroll; ++u) {
-                float f[V];
-                unpack<T>(raw[u], f);
+                for (int u = 0; u < kU; ++u)
+                    if (u < nv) raw[h][u] = ldg_nc_v4(base + (r + h * kWarps) * ld + u * V);
 #pragma unroll
-                for (int e = 0; e < V; ++e) m[e] = fmaxf(m[e], fabsf(f[e]));
-            }
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int u = 0; u < kU; ++u)
+                    if (u < nv) {
+                        float f[V];
+                        unpack<T>(raw[h][u], f);
+#pragma unroll
+                        for (int e = 0; e < V; ++e) m[u * V + e] = fmaxf(m[u * V + e], fabsf(f[e]));
+                    }
         }
         for (; r < r_end; r += kWarps) {
-            float f[V];
-            unpack<T>(ldg_nc_v4(base + r * ld), f);
 #pragma unroll
-            for (int e = 0; e < V; ++e) m[e] = fmaxf(m[e], fabsf(f[e]));
+            for (int u = 0; u < kU; ++u)
+                if (u < nv) {
+                    float f[V];
+                    unpack<T>(ldg_nc_v4(base + r * ld + u * V), f);
+#pragma unroll
+                    for (int e = 0; e < V; ++e) m[u * V + e] = fmaxf(m[u * V + e], fabsf(f[e]));
+                }
         }
     }
+    // slot of column lane * LC + e is e * 32 + lane: the 32 lanes of an atomic
+    // hit 32 different banks
 #pragma unroll
-    for (int e = 0; e < V; ++e) red[warp][lane * V + e] = m[e];
-    __syncwarp();  // lanes may have diverged above; bar.sync needs whole warps
+    for (int e = 0; e < LC; ++e)
+        if (e / V < nv) atomicMax(&red[e * 32 + lane], __float_as_int(m[e]));
+    __syncwarp();
     __syncthreads();
     for (int c = threadIdx.x; c < COLS; c += kWarps * 32) {
-        float v = red[0][c];
-#pragma unroll
-        for (int w = 1; w < kWarps; ++w) v = fmaxf(v, red[w][c]);
         const int64_t col = (int64_t)blockIdx.x * COLS + c;
-        if (col < K) atomic_max_nonneg(out + col, v);
+        if (col < K) atomicMax(reinterpret_cast<int*>(out + col), red[(c % LC) * 32 + c / LC]);
     }
 }
 
 template <typename T>
 sq_status_t launch(const void* X, int64_t M, int64_t K, int64_t ld, float* out, cudaStream_t s,
                    const char* name) {
-    constexpr int COLS = 32 * Vec<T>::N;
+    constexpr int COLS = 32 * Vec<T>::N * kU;
     const int64_t col_blocks = (K + COLS - 1) / COLS;
-    // one full wave of about 8 blocks per SM: as many row bands as fit beside
-    // the column blocks; rows per band a multiple of the warp count
-    const int64_t target = (int64_t)num_sms() * 8;
+    // one full wave of resident blocks: as many row bands as fit beside the
+    // column blocks; rows per band a multiple of the warp count
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, col_absmax_kernel<T>, kWarps * 32, 0) != cudaSuccess ||
+        per_sm < 1)
+        per_sm = 1;
+    const int64_t target = (int64_t)num_sms() * per_sm;
     int64_t bands = target / col_blocks;
     if (bands < 1) bands = 1;
     int64_t rpb = (M + bands - 1) / bands;
     rpb = ((rpb + kWarps - 1) / kWarps) * kWarps;
-    if (rpb < kWarps * kUnroll) rpb = kWarps * kUnroll;
+    if (rpb < 2 * kWarps) rpb = 2 * kWarps;
     const int64_t row_blocks = (M + rpb - 1) / rpb;
-    SQ_REQUIRE(row_blocks <= 65535, SQ_ERR_UNSUPPORTED_SHAPE, "%s: too many rows (M=%lld)", name,
-               (long long)M);
+    SQ_REQUIRE(row_blocks <= 65535, SQ_ERR_UNSUPPORTED_SHAPE, "%s: too many rows (M=%lld)", name, (long long)M);
     dim3 grid((unsigned)col_blocks, (unsigned)row_blocks);
-    launch_pdl(col_absmax_kernel<T>, dim3(grid), dim3(kWarps * 32), 0, s, static_cast<const T*>(X), M, K, ld, (int)rpb, out);
+    launch_pdl(col_absmax_kernel<T>, dim3(grid), dim3(kWarps * 32), 0, s, static_cast<const T*>(X), M, K, ld,
+               (int)rpb, out);
     return check_launch(name);
 }
 

@@ -254,14 +254,16 @@ __device__ __forceinline__ void epi_chunk(const Params& p, const uint32_t* r, in
 #pragma unroll
         for (int e = 0; e < 32; ++e) y[e] = __int_as_float((int)r[e]);  // raw bits, stored unchanged
     } else {
+        // y = acc * (rx * rw), each product one fp32 rounding, two lanes per op
         const float4* rw4 = reinterpret_cast<const float4*>(rw_w + cw);
+        const uint64_t rx2 = pk2(rx, rx);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
             const float4 w = rw4[e];
-            y[4 * e + 0] = __fmul_rn((float)(int)r[4 * e + 0], __fmul_rn(rx, w.x));
-            y[4 * e + 1] = __fmul_rn((float)(int)r[4 * e + 1], __fmul_rn(rx, w.y));
-            y[4 * e + 2] = __fmul_rn((float)(int)r[4 * e + 2], __fmul_rn(rx, w.z));
-            y[4 * e + 3] = __fmul_rn((float)(int)r[4 * e + 3], __fmul_rn(rx, w.w));
+            const uint64_t d01 = mul2(rx2, pk2(w.x, w.y));
+            const uint64_t d23 = mul2(rx2, pk2(w.z, w.w));
+            upk2(mul2(pk2((float)(int)r[4 * e + 0], (float)(int)r[4 * e + 1]), d01), y[4 * e + 0], y[4 * e + 1]);
+            upk2(mul2(pk2((float)(int)r[4 * e + 2], (float)(int)r[4 * e + 3]), d23), y[4 * e + 2], y[4 * e + 3]);
         }
         if constexpr (OUTL) {
             // the 16-bit outlier term, added term by term in ascending o with

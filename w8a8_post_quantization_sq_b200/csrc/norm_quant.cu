@@ -10,26 +10,27 @@
 //
 // Exactness: every step is one correctly rounded fp32 operation and the two
 // row sums use a fixed order, so v, the scales and the codes are bit-equal to
-// a CPU evaluation in the same order. The order: 128 lanes (the 128 threads
-// of the block); thread t folds its 8-element chunks t, t+128, ... in index
-// order with fma; each warp combines its 32 partials by the xor butterfly
-// (16, 8, 4, 2, 1), after which every lane holds the same value; the four
-// warp totals add as (G0 + G1) + (G2 + G3).
+// a CPU evaluation in the same order. The order: 256 lanes; lane t folds its
+// 8-element chunks t, t+256, ... in index order with fma; each group of 32
+// lanes combines by the xor butterfly (16, 8, 4, 2, 1), after which every lane
+// of the group holds the same value; the eight group totals add as
+// ((G0 + G1) + (G2 + G3)) + ((G4 + G5) + (G6 + G7)).
 //
 // Bandwidth kernels; the row stays in registers:
 //   K <= 4096: one warp per row (no block barrier). Lane l holds chunks
-//     l, l+32, l+64, ...; chunk c belongs to lane c mod 128 of the order above
-//     (its group is (c / 32) mod 4), so the warp keeps four partials, one per
-//     group, folds each in increasing chunk order, and runs the four group
-//     butterflies itself: bit-identical to the 128-thread order.
-//   4096 < K <= 16384: one 128-thread block per row, thread t = lane t.
+//     l, l+32, l+64, ...; chunk c belongs to lane c mod 256 of the order above,
+//     in group (c / 32) mod 8, so the warp keeps eight partials, one per
+//     group, folds each in increasing chunk order and runs the eight group
+//     butterflies itself: bit-identical to the 256-lane order.
+//   4096 < K <= 16384: one 256-thread block per row, thread t = lane t. Rows
+//     reach shared memory through a ring of buffers, one bulk copy (TMA
+//     engine, cp.async.bulk) per row issued R rows ahead, so several rows per
+//     block are in flight while the block reduces and quantises.
 // The codes are written 8 bytes per chunk, the per-token scale once per row.
 #include "sq_common.cuh"
 
 namespace sq {
 namespace {
-
-constexpr int kThreads = 128;
 
 struct NormArgs {
     int64_t M, K, ldh;
@@ -44,189 +45,91 @@ struct NormArgs {
     void* V;        // [M,K] 16-bit, or null
 };
 
-// Fixed-order block sum of one partial per thread (see file comment).
-__device__ __forceinline__ float canon_block_sum(float p, float* sh) {
+__device__ __forceinline__ float butterfly_sum(float p) {
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) p = __fadd_rn(p, __shfl_xor_sync(0xffffffffu, p, o));
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    if (lane == 0) sh[warp] = p;
-    __syncwarp();
-    __syncthreads();
-    const float r = __fadd_rn(__fadd_rn(sh[0], sh[1]), __fadd_rn(sh[2], sh[3]));
-    __syncwarp();
-    __syncthreads();
-    return r;
+    return p;
 }
 
-__device__ __forceinline__ float block_max4(float v, float* sh) {
+__device__ __forceinline__ float tree8(const float* g) {
+    return __fadd_rn(__fadd_rn(__fadd_rn(g[0], g[1]), __fadd_rn(g[2], g[3])),
+                     __fadd_rn(__fadd_rn(g[4], g[5]), __fadd_rn(g[6], g[7])));
+}
+
+__device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    if (lane == 0) sh[warp] = v;
-    __syncwarp();
-    __syncthreads();
-    const float r = fmaxf(fmaxf(sh[0], sh[1]), fmaxf(sh[2], sh[3]));
-    __syncwarp();
-    __syncthreads();
-    return r;
+    return v;
 }
 
-template <typename T, bool LN, int CMAX>
-__global__ void __launch_bounds__(kThreads)
-norm_quant_kernel(const T* __restrict__ H, NormArgs a) {
-    pdl_wait();
-    pdl_trigger();
-    __shared__ float sh[4];
-    extern __shared__ float amax_sh[];  // [K] running max |v| (calibration mode)
-    const int t = threadIdx.x;
-    const int nch = (int)(a.K / 8);
-    const float Kf = (float)a.K;
-    if (a.absmax)
-        for (int j = t; j < a.K; j += kThreads) amax_sh[j] = 0.0f;
-
-    for (int64_t row = blockIdx.x; row < a.M; row += gridDim.x) {
-        const T* h = H + row * a.ldh;
-        uint4 raw[CMAX];
+// v_j of one 8-element chunk; g holds gamma'_j of the chunk, beta'_j is read
+// from a.beta (LayerNorm with a shift only)
+template <typename T, bool LN>
+__device__ __forceinline__ void compute_v_g(const uint4& rw, int ch, const NormArgs& a, const float* g, float mu,
+                                            float r, float* v) {
+    float f[8];
+    unpack<T>(rw, f);
+    const uint64_t r2 = pk2(r, r);
+    if constexpr (LN) {
+        const uint64_t nmu2 = pk2(-mu, -mu);  // x + (-mu) is the IEEE x - mu
+        if (a.beta) {
+            // the last product feeds an add: keep those two steps scalar
+            const float4 b0 = __ldg(reinterpret_cast<const float4*>(a.beta + ch * 8));
+            const float4 b1 = __ldg(reinterpret_cast<const float4*>(a.beta + ch * 8 + 4));
+            const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-        for (int c = 0; c < CMAX; ++c) {
-            const int ch = t + c * kThreads;
-            if (ch < nch) raw[c] = ldg_nc_v4(h + (int64_t)ch * 8);
-        }
-        float mu = 0.0f, r;
-        if constexpr (LN) {
-            float acc = 0.0f;
-#pragma unroll
-            for (int c = 0; c < CMAX; ++c) {
-                if (t + c * kThreads < nch) {
-                    float f[8];
-                    unpack<T>(raw[c], f);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) acc = __fmaf_rn(f[e], 1.0f, acc);
-                }
+            for (int e = 0; e < 8; e += 2) {
+                float u0, u1;
+                upk2(mul2(add2(pk2(f[e], f[e + 1]), nmu2), r2), u0, u1);
+                v[e] = __fadd_rn(__fmul_rn(u0, g[e]), b[e]);
+                v[e + 1] = __fadd_rn(__fmul_rn(u1, g[e + 1]), b[e + 1]);
             }
-            mu = __fdiv_rn(canon_block_sum(acc, sh), Kf);
-            acc = 0.0f;
-#pragma unroll
-            for (int c = 0; c < CMAX; ++c) {
-                if (t + c * kThreads < nch) {
-                    float f[8];
-                    unpack<T>(raw[c], f);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const float d = __fsub_rn(f[e], mu);
-                        acc = __fmaf_rn(d, d, acc);
-                    }
-                }
-            }
-            const float var = __fdiv_rn(canon_block_sum(acc, sh), Kf);
-            r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(var, a.eps)));
         } else {
-            float acc = 0.0f;
 #pragma unroll
-            for (int c = 0; c < CMAX; ++c) {
-                if (t + c * kThreads < nch) {
-                    float f[8];
-                    unpack<T>(raw[c], f);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) acc = __fmaf_rn(f[e], f[e], acc);
-                }
-            }
-            const float ms = __fdiv_rn(canon_block_sum(acc, sh), Kf);
-            r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, a.eps)));
+            for (int e = 0; e < 8; e += 2)
+                upk2(mul2(mul2(add2(pk2(f[e], f[e + 1]), nmu2), r2), pk2(g[e], g[e + 1])), v[e], v[e + 1]);
         }
-
-        // v_j, computed identically each time it is needed
-        auto compute_v = [&](const uint4& rw, int ch, float* v) {
-            float f[8];
-            unpack<T>(rw, f);
-            const float4 g0 = __ldg(reinterpret_cast<const float4*>(a.gamma + ch * 8));
-            const float4 g1 = __ldg(reinterpret_cast<const float4*>(a.gamma + ch * 8 + 4));
-            const float g[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-            if constexpr (LN) {
-                float b[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-                const bool hb = a.beta != nullptr;
-                if (hb) {
-                    const float4 b0 = __ldg(reinterpret_cast<const float4*>(a.beta + ch * 8));
-                    const float4 b1 = __ldg(reinterpret_cast<const float4*>(a.beta + ch * 8 + 4));
-                    b[0] = b0.x; b[1] = b0.y; b[2] = b0.z; b[3] = b0.w;
-                    b[4] = b1.x; b[5] = b1.y; b[6] = b1.z; b[7] = b1.w;
-                }
+    } else {
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float u = __fmul_rn(__fmul_rn(__fsub_rn(f[e], mu), r), g[e]);
-                    v[e] = hb ? __fadd_rn(u, b[e]) : u;
-                }
-            } else {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) v[e] = __fmul_rn(__fmul_rn(f[e], r), g[e]);
-            }
-        };
-
-        float m = 0.0f;
-        const bool need_max = a.Xq && a.per_token;
-        if (need_max || a.absmax || a.V) {
-#pragma unroll
-            for (int c = 0; c < CMAX; ++c) {
-                const int ch = t + c * kThreads;
-                if (ch < nch) {
-                    float v[8];
-                    compute_v(raw[c], ch, v);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(v[e]));
-                    if (a.absmax) {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) amax_sh[ch * 8 + e] = fmaxf(amax_sh[ch * 8 + e], fabsf(v[e]));
-                    }
-                    if (a.V) {
-                        uint32_t o[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            o[e] = (uint32_t)to16<T>(v[2 * e]) | ((uint32_t)to16<T>(v[2 * e + 1]) << 16);
-                        *reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.V) + row * a.K + ch * 8) =
-                            make_uint4(o[0], o[1], o[2], o[3]);
-                    }
-                }
-            }
-        }
-        if (a.Xq) {
-            float qs;
-            if (a.per_token) {
-                qs = __fdiv_rn(127.0f, fmaxf(block_max4(m, sh), 1e-8f));
-                if (t == 0) a.qs_x[row] = qs;
-            } else {
-                qs = *a.static_qs;
-                if (row == 0 && t == 0) a.qs_x[0] = qs;
-            }
-            int8_t* q = a.Xq + row * a.K;
-#pragma unroll
-            for (int c = 0; c < CMAX; ++c) {
-                const int ch = t + c * kThreads;
-                if (ch < nch) {
-                    float v[8];
-                    compute_v(raw[c], ch, v);
-                    uint32_t b[8];
-                    if (a.per_token) {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) b[e] = quant_bits_noclip(__fmul_rn(v[e], qs));
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) b[e] = quant_bits_clip(__fmul_rn(v[e], qs));
-                    }
-                    *reinterpret_cast<uint2*>(q + ch * 8) =
-                        make_uint2(pack_low_bytes(b[0], b[1], b[2], b[3]), pack_low_bytes(b[4], b[5], b[6], b[7]));
-                }
-            }
-        }
-    }
-    if (a.absmax) {
-        __syncwarp();
-        __syncthreads();
-        // each column was only touched by its owning thread; publish once per block
-        for (int j = t; j < a.K; j += kThreads) atomic_max_nonneg(a.absmax + j, amax_sh[j]);
+        for (int e = 0; e < 8; e += 2) upk2(mul2(mul2(pk2(f[e], f[e + 1]), r2), pk2(g[e], g[e + 1])), v[e], v[e + 1]);
     }
 }
 
+__device__ __forceinline__ void load_gamma(const NormArgs& a, int ch, float* g) {
+    const float4 g0 = __ldg(reinterpret_cast<const float4*>(a.gamma + ch * 8));
+    const float4 g1 = __ldg(reinterpret_cast<const float4*>(a.gamma + ch * 8 + 4));
+    g[0] = g0.x; g[1] = g0.y; g[2] = g0.z; g[3] = g0.w;
+    g[4] = g1.x; g[5] = g1.y; g[6] = g1.z; g[7] = g1.w;
+}
 
+// v_j of one 8-element chunk, gamma'_j read from a.gamma
+template <typename T, bool LN>
+__device__ __forceinline__ void compute_v(const uint4& rw, int ch, const NormArgs& a, float mu, float r, float* v) {
+    float g[8];
+    load_gamma(a, ch, g);
+    compute_v_g<T, LN>(rw, ch, a, g, mu, r, v);
+}
+
+template <typename T>
+__device__ __forceinline__ void store_v16(const NormArgs& a, int64_t row, int ch, const float* v) {
+    uint32_t o[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[e] = (uint32_t)to16<T>(v[2 * e]) | ((uint32_t)to16<T>(v[2 * e + 1]) << 16);
+    *reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.V) + row * a.K + ch * 8) = make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+__device__ __forceinline__ uint2 codes8(const float* v, float qs, bool clip) {
+    uint32_t b[8];
+    if (clip) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) b[e] = quant_bits_clip(__fmul_rn(v[e], qs));
+    } else {
+        quant_bits8_noclip(v, qs, b);
+    }
+    return make_uint2(pack_low_bytes(b[0], b[1], b[2], b[3]), pack_low_bytes(b[4], b[5], b[6], b[7]));
+}
+
+// ------------------------------------------------------------------ K <= 4096
 // One warp per row (K <= 32 * 8 * CW); see the file comment for the order.
 template <typename T, bool LN, int CW>
 __global__ void __launch_bounds__(256)
@@ -249,23 +152,21 @@ norm_quant_warp_kernel(const T* __restrict__ H, NormArgs a) {
 #pragma unroll
         for (int i = 0; i < CW; ++i)
             if (lane + 32 * i < nch) raw[i] = ldg_nc_v4(h + (int64_t)(lane + 32 * i) * 8);
-        // fixed-order sum of f(x) over the row: four group partials per lane
+        // fixed-order sum of term(x) over the row: eight group partials per lane
         auto canon = [&](auto term) {
-            float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            float acc[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
             for (int i = 0; i < CW; ++i) {
                 if (lane + 32 * i < nch) {
                     float f[8];
                     unpack<T>(raw[i], f);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) acc[i & 3] = term(f[e], acc[i & 3]);
+                    for (int e = 0; e < 8; ++e) acc[i & 7] = term(f[e], acc[i & 7]);
                 }
             }
 #pragma unroll
-            for (int w = 0; w < 4; ++w)
-#pragma unroll
-                for (int o = 16; o >= 1; o >>= 1) acc[w] = __fadd_rn(acc[w], __shfl_xor_sync(0xffffffffu, acc[w], o));
-            return __fadd_rn(__fadd_rn(acc[0], acc[1]), __fadd_rn(acc[2], acc[3]));
+            for (int w = 0; w < 8; ++w) acc[w] = butterfly_sum(acc[w]);
+            return tree8(acc);
         };
         float mu = 0.0f, r;
         if constexpr (LN) {
@@ -280,28 +181,6 @@ norm_quant_warp_kernel(const T* __restrict__ H, NormArgs a) {
             const float ms = __fdiv_rn(canon([](float x, float c) { return __fmaf_rn(x, x, c); }), Kf);
             r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, a.eps)));
         }
-        auto compute_v = [&](const uint4& rw, int ch, float* v) {
-            float f[8];
-            unpack<T>(rw, f);
-            const float4 g0 = __ldg(reinterpret_cast<const float4*>(a.gamma + ch * 8));
-            const float4 g1 = __ldg(reinterpret_cast<const float4*>(a.gamma + ch * 8 + 4));
-            const float g[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-            if constexpr (LN) {
-                if (a.beta) {
-                    const float4 b0 = __ldg(reinterpret_cast<const float4*>(a.beta + ch * 8));
-                    const float4 b1 = __ldg(reinterpret_cast<const float4*>(a.beta + ch * 8 + 4));
-                    const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) v[e] = __fadd_rn(__fmul_rn(__fmul_rn(__fsub_rn(f[e], mu), r), g[e]), b[e]);
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) v[e] = __fmul_rn(__fmul_rn(__fsub_rn(f[e], mu), r), g[e]);
-                }
-            } else {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) v[e] = __fmul_rn(__fmul_rn(f[e], r), g[e]);
-            }
-        };
         float m = 0.0f;
         if ((a.Xq && a.per_token) || a.absmax || a.V) {
 #pragma unroll
@@ -309,30 +188,22 @@ norm_quant_warp_kernel(const T* __restrict__ H, NormArgs a) {
                 const int ch = lane + 32 * i;
                 if (ch < nch) {
                     float v[8];
-                    compute_v(raw[i], ch, v);
+                    compute_v<T, LN>(raw[i], ch, a, mu, r, v);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(v[e]));
                     if (a.absmax) {
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) atomicMax(reinterpret_cast<int*>(amax_sh + ch * 8 + e), __float_as_int(fabsf(v[e])));
+                        for (int e = 0; e < 8; ++e)
+                            atomicMax(reinterpret_cast<int*>(amax_sh + ch * 8 + e), __float_as_int(fabsf(v[e])));
                     }
-                    if (a.V) {
-                        uint32_t o[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            o[e] = (uint32_t)to16<T>(v[2 * e]) | ((uint32_t)to16<T>(v[2 * e + 1]) << 16);
-                        *reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.V) + row * a.K + ch * 8) =
-                            make_uint4(o[0], o[1], o[2], o[3]);
-                    }
+                    if (a.V) store_v16<T>(a, row, ch, v);
                 }
             }
         }
         if (a.Xq) {
             float qs;
             if (a.per_token) {
-#pragma unroll
-                for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-                qs = __fdiv_rn(127.0f, fmaxf(m, 1e-8f));
+                qs = __fdiv_rn(127.0f, fmaxf(warp_max(m), 1e-8f));
                 if (lane == 0) a.qs_x[row] = qs;
             } else {
                 qs = *a.static_qs;
@@ -344,17 +215,8 @@ norm_quant_warp_kernel(const T* __restrict__ H, NormArgs a) {
                 const int ch = lane + 32 * i;
                 if (ch < nch) {
                     float v[8];
-                    compute_v(raw[i], ch, v);
-                    uint32_t b[8];
-                    if (a.per_token) {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) b[e] = quant_bits_noclip(__fmul_rn(v[e], qs));
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) b[e] = quant_bits_clip(__fmul_rn(v[e], qs));
-                    }
-                    *reinterpret_cast<uint2*>(q + ch * 8) =
-                        make_uint2(pack_low_bytes(b[0], b[1], b[2], b[3]), pack_low_bytes(b[4], b[5], b[6], b[7]));
+                    compute_v<T, LN>(raw[i], ch, a, mu, r, v);
+                    *reinterpret_cast<uint2*>(q + ch * 8) = codes8(v, qs, !a.per_token);
                 }
             }
         }
@@ -363,6 +225,254 @@ norm_quant_warp_kernel(const T* __restrict__ H, NormArgs a) {
         __syncwarp();
         __syncthreads();
         for (int j = threadIdx.x; j < a.K; j += blockDim.x) atomic_max_nonneg(a.absmax + j, amax_sh[j]);
+    }
+}
+
+// ------------------------------------------------------------------ K > 4096
+constexpr int kBlock = 256;
+constexpr uint64_t kWaitNs = 2000000000ull;
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+// Bounded wait for a row copy; false after about 2 s.
+__device__ __noinline__ bool wait_row(uint32_t bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (!mbar_try_wait(bar, parity))
+        if (global_ns() - t0 > kWaitNs) return false;
+    return true;
+}
+// One row (bytes, a multiple of 16) from global into shared memory, completing
+// on the mbarrier; a plain bulk copy, no multicast.
+__device__ __forceinline__ void issue_row(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst), "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
+// Fixed-order block sum of one partial per thread (thread t = lane t).
+__device__ __forceinline__ float canon_block_sum(float p, float* sh) {
+    p = butterfly_sum(p);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (lane == 0) sh[warp] = p;
+    __syncwarp();
+    __syncthreads();
+    return tree8(sh);
+}
+
+__device__ __forceinline__ float block_max8(float v, float* sh) {
+    v = warp_max(v);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (lane == 0) sh[warp] = v;
+    __syncwarp();
+    __syncthreads();
+    float r = sh[0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) r = fmaxf(r, sh[w]);
+    return r;
+}
+
+// One 256-thread block per row, rows strided over the grid (K <= 256*8*C).
+// Thread t always owns chunks t, t+256, ..., so gamma'_j of its chunks is
+// loaded once into registers. The rows arrive in a ring of R shared-memory
+// buffers, each filled by one bulk copy issued R rows ahead. With KEEPV the
+// values v of the thread's chunks stay in registers from the absmax to the
+// codes and the row's buffer is refilled right after the absmax reduction;
+// otherwise v is formed again from the staged row for the codes and the
+// buffer is refilled after them.
+template <typename T, bool LN, int C, bool KEEPV>
+__global__ void __launch_bounds__(kBlock, 2)
+norm_quant_bulk_kernel(const T* __restrict__ H, NormArgs a, int R) {
+    pdl_wait();
+    pdl_trigger();
+    extern __shared__ __align__(128) uint8_t dsm[];  // R rows, then [K] floats (calibration mode)
+    __shared__ __align__(8) uint64_t bars[8];
+    __shared__ float sh[3][8];
+    const int t = threadIdx.x;
+    const int nch = (int)(a.K / 8);
+    const float Kf = (float)a.K;
+    const uint32_t row_bytes = (uint32_t)(a.K * sizeof(T));
+    float* amax_sh = reinterpret_cast<float*>(dsm + (size_t)R * row_bytes);
+    const int64_t G = gridDim.x;
+    float g[C][8];
+#pragma unroll
+    for (int c = 0; c < C; ++c)
+        if (t + c * kBlock < nch) load_gamma(a, t + c * kBlock, g[c]);
+    if (t == 0) {
+        for (int i = 0; i < R; ++i)
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bars[i])));
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (a.absmax)
+        for (int j = t; j < a.K; j += kBlock) amax_sh[j] = 0.0f;
+    __syncwarp();
+    __syncthreads();
+    if (t == 0)
+        for (int i = 0; i < R; ++i) {
+            const int64_t r = blockIdx.x + i * G;
+            if (r < a.M) issue_row(smem_u32(dsm + (size_t)i * row_bytes), H + r * a.ldh, row_bytes, smem_u32(&bars[i]));
+        }
+    bool aborted = false;
+    int it = 0;
+    for (int64_t row = blockIdx.x; row < a.M; row += G, ++it) {
+        const int slot = it % R;
+        const uint8_t* xs = dsm + (size_t)slot * row_bytes;
+        const bool ok = wait_row(smem_u32(&bars[slot]), (uint32_t)((it / R) & 1));
+        __syncwarp();
+        if (__syncthreads_and(ok) == 0) {  // a copy never landed: give up (not expected)
+            aborted = true;
+            break;
+        }
+        auto chunk = [&](int ch) { return *reinterpret_cast<const uint4*>(xs + (size_t)ch * 16); };
+        auto refill = [&]() {
+            if (t == 0) {
+                const int64_t nr = row + (int64_t)R * G;
+                if (nr < a.M) {
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    issue_row(smem_u32(dsm + (size_t)slot * row_bytes), H + nr * a.ldh, row_bytes,
+                              smem_u32(&bars[slot]));
+                }
+            }
+        };
+        float mu = 0.0f, r;
+        if constexpr (LN) {
+            float acc = 0.0f;
+#pragma unroll
+            for (int c = 0; c < C; ++c) {
+                if (t + c * kBlock < nch) {
+                    float f[8];
+                    unpack<T>(chunk(t + c * kBlock), f);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) acc = __fmaf_rn(f[e], 1.0f, acc);
+                }
+            }
+            mu = __fdiv_rn(canon_block_sum(acc, sh[0]), Kf);
+            acc = 0.0f;
+#pragma unroll
+            for (int c = 0; c < C; ++c) {
+                if (t + c * kBlock < nch) {
+                    float f[8];
+                    unpack<T>(chunk(t + c * kBlock), f);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float d = __fsub_rn(f[e], mu);
+                        acc = __fmaf_rn(d, d, acc);
+                    }
+                }
+            }
+            const float var = __fdiv_rn(canon_block_sum(acc, sh[1]), Kf);
+            r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(var, a.eps)));
+        } else {
+            float acc = 0.0f;
+#pragma unroll
+            for (int c = 0; c < C; ++c) {
+                if (t + c * kBlock < nch) {
+                    float f[8];
+                    unpack<T>(chunk(t + c * kBlock), f);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) acc = __fmaf_rn(f[e], f[e], acc);
+                }
+            }
+            const float ms = __fdiv_rn(canon_block_sum(acc, sh[0]), Kf);
+            r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, a.eps)));
+        }
+        float vk[KEEPV ? C : 1][8];
+        float m = 0.0f;
+        if (KEEPV || (a.Xq && a.per_token) || a.absmax || a.V) {
+#pragma unroll
+            for (int c = 0; c < C; ++c) {
+                const int ch = t + c * kBlock;
+                if (ch < nch) {
+                    float v[8];
+                    compute_v_g<T, LN>(chunk(ch), ch, a, g[c], mu, r, v);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(v[e]));
+                    if (a.absmax) {
+                        float4* am = reinterpret_cast<float4*>(amax_sh + ch * 8);
+                        const float4 o0 = am[0], o1 = am[1];
+                        am[0] = make_float4(fmaxf(o0.x, fabsf(v[0])), fmaxf(o0.y, fabsf(v[1])),
+                                            fmaxf(o0.z, fabsf(v[2])), fmaxf(o0.w, fabsf(v[3])));
+                        am[1] = make_float4(fmaxf(o1.x, fabsf(v[4])), fmaxf(o1.y, fabsf(v[5])),
+                                            fmaxf(o1.z, fabsf(v[6])), fmaxf(o1.w, fabsf(v[7])));
+                    }
+                    if (a.V) store_v16<T>(a, row, ch, v);
+                    if constexpr (KEEPV) {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) vk[c][e] = v[e];
+                    }
+                }
+            }
+        }
+        float mx = 0.0f;
+        if (a.Xq && a.per_token) {
+            mx = block_max8(m, sh[2]);
+        } else if (KEEPV) {
+            __syncwarp();
+            __syncthreads();
+        }
+        if constexpr (KEEPV) refill();  // every thread is past its last read of the slot
+        if (a.Xq) {
+            float qs;
+            if (a.per_token) {
+                qs = __fdiv_rn(127.0f, fmaxf(mx, 1e-8f));
+                if (t == 0) a.qs_x[row] = qs;
+            } else {
+                qs = *a.static_qs;
+                if (row == 0 && t == 0) a.qs_x[0] = qs;
+            }
+            int8_t* q = a.Xq + row * a.K;
+#pragma unroll
+            for (int c = 0; c < C; ++c) {
+                const int ch = t + c * kBlock;
+                if (ch < nch) {
+                    if constexpr (KEEPV) {
+                        *reinterpret_cast<uint2*>(q + ch * 8) = codes8(vk[c], qs, !a.per_token);
+                    } else {
+                        float v[8];
+                        compute_v_g<T, LN>(chunk(ch), ch, a, g[c], mu, r, v);
+                        *reinterpret_cast<uint2*>(q + ch * 8) = codes8(v, qs, !a.per_token);
+                    }
+                }
+            }
+        }
+        if constexpr (!KEEPV) {
+            __syncwarp();
+            __syncthreads();
+            refill();
+        }
+    }
+    if (aborted && t == 0) {
+        // drain copies still in flight before the block's shared memory is released
+        for (int i = 0; i < R; ++i) {
+            const uint64_t t0 = global_ns();
+            for (uint32_t ph = 0; ph < 2; ++ph)
+                while (!mbar_try_wait(smem_u32(&bars[i]), ph))
+                    if (global_ns() - t0 > kWaitNs / 4) break;
+        }
+    }
+    if (a.absmax) {
+        __syncwarp();
+        __syncthreads();
+        for (int j = t; j < a.K; j += kBlock) atomic_max_nonneg(a.absmax + j, amax_sh[j]);
     }
 }
 
@@ -377,17 +487,22 @@ void launch_warp(const void* H, const NormArgs& a, cudaStream_t s) {
     launch_pdl(kern, dim3((unsigned)blocks), dim3(256), smem, s, static_cast<const T*>(H), a);
 }
 
-template <typename T, bool LN, int CMAX>
-void launch_one(const void* H, const NormArgs& a, cudaStream_t s) {
-    const size_t smem = a.absmax ? (size_t)a.K * sizeof(float) : 0;
-    auto kern = norm_quant_kernel<T, LN, CMAX>;
-    if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    // up to 16 resident blocks of 128 threads per SM for the small rows
-    const int per_sm = CMAX <= 2 ? 16 : (CMAX <= 4 ? 8 : 4);
+template <typename T, bool LN, int C, bool KEEPV>
+void launch_block(const void* H, const NormArgs& a, cudaStream_t s) {
+    auto kern = norm_quant_bulk_kernel<T, LN, C, KEEPV>;
+    const size_t row_bytes = (size_t)a.K * sizeof(T);
+    int R = (int)((96 * 1024) / row_bytes);  // about 96 KB of staged rows per block
+    if (R < 2) R = 2;
+    if (R > 8) R = 8;
+    const size_t smem = (size_t)R * row_bytes + (a.absmax ? (size_t)a.K * sizeof(float) : 0);
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kBlock, smem) != cudaSuccess || per_sm < 1)
+        per_sm = 1;
     int64_t grid = (int64_t)num_sms() * per_sm;
-    if (a.absmax) grid = (int64_t)num_sms() * 2;  // fewer blocks: one publish of [K] per block
+    if (a.absmax) grid = (int64_t)num_sms();  // fewer blocks: one publish of [K] per block
     if (grid > a.M) grid = a.M;
-    launch_pdl(kern, dim3((unsigned)grid), dim3(kThreads), smem, s, static_cast<const T*>(H), a);
+    launch_pdl(kern, dim3((unsigned)grid), dim3(kBlock), smem, s, static_cast<const T*>(H), a, R);
 }
 
 template <typename T, bool LN>
@@ -398,8 +513,9 @@ void launch_t(const void* H, const NormArgs& a, cudaStream_t s) {
     else if (nch <= 128) launch_warp<T, LN, 4>(H, a, s);
     else if (nch <= 256) launch_warp<T, LN, 8>(H, a, s);
     else if (nch <= 512) launch_warp<T, LN, 16>(H, a, s);
-    else if (nch <= 1024) launch_one<T, LN, 8>(H, a, s);
-    else launch_one<T, LN, 16>(H, a, s);
+    else if (nch <= 1024) launch_block<T, LN, 4, true>(H, a, s);
+    else if (nch <= 1536) launch_block<T, LN, 6, true>(H, a, s);
+    else launch_block<T, LN, 8, false>(H, a, s);
 }
 
 }  // namespace

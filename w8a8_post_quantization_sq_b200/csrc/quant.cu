@@ -41,8 +41,12 @@ __device__ __forceinline__ void apply_s(float* f, const float* __restrict__ s, i
         const float4 a = *reinterpret_cast<const float4*>(s + k0);
         const float4 b = *reinterpret_cast<const float4*>(s + k0 + 4);
         const float sv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        if constexpr (SM == kMul) {
+            mul8(f, sv);
+        } else {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) f[e] = SM == kMul ? __fmul_rn(f[e], sv[e]) : __fdiv_rn(f[e], sv[e]);
+            for (int e = 0; e < 8; ++e) f[e] = __fdiv_rn(f[e], sv[e]);
+        }
     }
 }
 
@@ -70,8 +74,7 @@ __device__ __forceinline__ uint2 codes8(const float* v, float qs, bool clip) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) b[e] = quant_bits_clip(__fmul_rn(v[e], qs));
     } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) b[e] = quant_bits_noclip(__fmul_rn(v[e], qs));
+        quant_bits8_noclip(v, qs, b);
     }
     return make_uint2(pack_low_bytes(b[0], b[1], b[2], b[3]), pack_low_bytes(b[4], b[5], b[6], b[7]));
 }
@@ -123,10 +126,32 @@ row_quant_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, cons
     }
 }
 
+// Raw 8 elements of a row as loaded (one 16-byte vector for 16-bit data, two
+// for fp32).
+template <typename T> struct Raw8 { uint4 a; };
+template <> struct Raw8<float> { uint4 a, b; };
+
+template <typename T>
+__device__ __forceinline__ void load_raw(const T* p, Raw8<T>& r) {
+    r.a = ldg_nc_v4(p);
+    if constexpr (sizeof(T) == 4) r.b = ldg_nc_v4(p + 4);
+}
+template <typename T>
+__device__ __forceinline__ void unpack_raw(const Raw8<T>& r, float* f) {
+    if constexpr (sizeof(T) == 2) {
+        unpack<T>(r.a, f);
+    } else {
+        unpack<float>(r.a, f);
+        unpack<float>(r.b, f + 4);
+    }
+}
+
 // The row held in registers by a group of G threads (G = 32: one warp per
 // row, several rows per block; G = 256: the whole block), CH chunks of 8
 // elements per thread: one read of the row from memory, a group max, then the
-// codes from the registers. Used while K <= 8 * G * CH_max.
+// codes from the registers. The next row's loads are issued before the group
+// reduction so they land while this row is finished. Used while
+// K <= 8 * G * CH_max.
 template <typename T, int SM, int G, int CH>
 __global__ void __launch_bounds__(kThreads)
 row_quant_reg_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, const float* __restrict__ s,
@@ -138,18 +163,36 @@ row_quant_reg_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, 
     constexpr int GPB = kThreads / G;  // groups (rows) per block
     const int gt = threadIdx.x % G;
     const int64_t ngroups = (int64_t)gridDim.x * GPB;
-    for (int64_t row = (int64_t)blockIdx.x * GPB + threadIdx.x / G; row < M; row += ngroups) {
-        const T* x = X + row * ld;
+    int64_t row = (int64_t)blockIdx.x * GPB + threadIdx.x / G;
+    Raw8<T> raw[CH];
+    if (row < M) {
+#pragma unroll
+        for (int c = 0; c < CH; ++c) {
+            const int64_t k0 = ((int64_t)gt + (int64_t)c * G) * 8;
+            if (k0 < K) load_raw<T>(X + row * ld + k0, raw[c]);
+        }
+    }
+    // G == 256: every thread of the block takes the same rows; G == 32: each
+    // warp takes its own, and only warp-level reductions are used
+    for (; row < M; row += ngroups) {
         float v[CH][8];
         float m = 0.0f;
 #pragma unroll
         for (int c = 0; c < CH; ++c) {
             const int64_t k0 = ((int64_t)gt + (int64_t)c * G) * 8;
             if (k0 < K) {
-                load8<T>(x + k0, v[c]);
+                unpack_raw<T>(raw[c], v[c]);
                 apply_s<SM>(v[c], s, k0);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(v[c][e]));
+            }
+        }
+        const int64_t nxt = row + ngroups;
+        if (nxt < M) {
+#pragma unroll
+            for (int c = 0; c < CH; ++c) {
+                const int64_t k0 = ((int64_t)gt + (int64_t)c * G) * 8;
+                if (k0 < K) load_raw<T>(X + nxt * ld + k0, raw[c]);
             }
         }
         float qs;
@@ -237,25 +280,30 @@ sq_status_t quantize(const void* Xv, int64_t M, int64_t K, int64_t ld, const flo
         launch_pdl(scale_from_absmax_kernel, dim3(1), dim3(kThreads), 0, st, wmax, 1, wqs);
         tensor_qs = wqs;
     }
-    const int64_t cap = (int64_t)num_sms() * 8;
-    auto blocks = [&](int64_t rows_per_block) {
+    // one resident wave of blocks; each group strides over the rows
+    auto go = [&](auto kern, int rows_per_block) {
+        int per_sm = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, 0) != cudaSuccess || per_sm < 1)
+            per_sm = 1;
         int64_t b = (M + rows_per_block - 1) / rows_per_block;
-        return (unsigned)(b < cap ? b : cap);
+        const int64_t cap = (int64_t)num_sms() * per_sm;
+        if (b > cap) b = cap;
+        return launch_pdl(kern, dim3((unsigned)b), dim3(kThreads), 0, st, X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
     };
     if (K <= 256)
-        launch_pdl(row_quant_reg_kernel<T, SM, 32, 1>, dim3(blocks(8)), dim3(kThreads), 0, st, X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
+        go(row_quant_reg_kernel<T, SM, 32, 1>, 8);
     else if (K <= 512)
-        launch_pdl(row_quant_reg_kernel<T, SM, 32, 2>, dim3(blocks(8)), dim3(kThreads), 0, st, X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
+        go(row_quant_reg_kernel<T, SM, 32, 2>, 8);
     else if (K <= 1024)
-        launch_pdl(row_quant_reg_kernel<T, SM, 32, 4>, dim3(blocks(8)), dim3(kThreads), 0, st, X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
+        go(row_quant_reg_kernel<T, SM, 32, 4>, 8);
     else if (K <= 2048)
-        launch_pdl(row_quant_reg_kernel<T, SM, 32, 8>, dim3(blocks(8)), dim3(kThreads), 0, st, X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
+        go(row_quant_reg_kernel<T, SM, 32, 8>, 8);
     else if (K <= 4096)
-        launch_pdl(row_quant_reg_kernel<T, SM, 256, 2>, dim3(blocks(1)), dim3(kThreads), 0, st, X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
+        go(row_quant_reg_kernel<T, SM, 256, 2>, 1);
     else if (K <= 8192)
-        launch_pdl(row_quant_reg_kernel<T, SM, 256, 4>, dim3(blocks(1)), dim3(kThreads), 0, st, X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
+        go(row_quant_reg_kernel<T, SM, 256, 4>, 1);
     else if (K <= 16384)
-        launch_pdl(row_quant_reg_kernel<T, SM, 256, 8>, dim3(blocks(1)), dim3(kThreads), 0, st, X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
+        go(row_quant_reg_kernel<T, SM, 256, 8>, 1);
     else
         launch_pdl(row_quant_kernel<T, SM>, dim3(row_grid(M)), dim3(kThreads), 0, st, X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
     return check_launch(name);

@@ -159,6 +159,40 @@ __device__ __forceinline__ uint32_t pack_low_bytes(uint32_t a, uint32_t b, uint3
     return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
 }
 
+// Packed fp32 pairs (sm_100 f32x2 arithmetic): each lane is one correctly
+// rounded fp32 operation, identical to the scalar __fmul_rn / __fadd_rn.
+__device__ __forceinline__ uint64_t pk2(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void upk2(uint64_t v, float& a, float& b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+// v[e] *= s[e] for 8 values, two at a time
+__device__ __forceinline__ void mul8(float* v, const float* s) {
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) upk2(mul2(pk2(v[e], v[e + 1]), pk2(s[e], s[e + 1])), v[e], v[e + 1]);
+}
+// Packed pairs are used only where a product is not followed by an add that
+// must see it rounded: a packed multiply feeding a packed add has been seen to
+// produce the fused (singly rounded) result, which would change int8 codes at
+// exact ties. The int8 step below therefore stays scalar.
+__device__ __forceinline__ void quant_bits8_noclip(const float* v, float qs, uint32_t* b) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) b[e] = quant_bits_noclip(__fmul_rn(v[e], qs));
+}
+
 // max on non-negative floats through their bit patterns (monotone for >= 0).
 __device__ __forceinline__ void atomic_max_nonneg(float* addr, float v) {
     atomicMax(reinterpret_cast<int*>(addr), __float_as_int(v));
