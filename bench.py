@@ -12,6 +12,9 @@ fused 1024->4096, o 2048->1024, gate/up fused 1024->6144, down 3072->1024;
   a5 fused RMSNorm + smoothing + per-token int8                         x2
   a6 int8 GEMM + dequant epilogue to bf16                               x4
   a7-a9 LLM.int8 decomposition of the q/k/v projection (bf16)           x1
+The independent chains of the step (the attention-side and MLP-side
+calibration/quantisation chains, the weight-side work, the o/down GEMMs and the
+LLM.int8 call) run on their own streams inside the step, joined at its end.
 The step is captured once in a CUDA graph and replayed. L2 is flushed (a
 256 MB write, then a 256 MB read of another buffer so that no dirty line of the
 flush is left to be written back) before every timed step, outside the timed
@@ -150,36 +153,67 @@ class Layer:
         self.idx = e(K, dt=torch.int32)
         self.nidx = e(1, dt=torch.int32)
         self.gemm_events = None
+        self.streams = [torch.cuda.Stream(device=dev) for _ in range(5)]
+        self.events = {n: torch.cuda.Event() for n in ("wmax_attn", "wmax_mlp", "V_attn", "V_mlp", "s_attn", "s_mlp",
+                                                      "wq_qkv", "wq_gateup")}
 
     def step(self, gemm_ev=None):
-        sq, d = self.sq, self.d
+        """One pass of every row. Independent chains run on their own streams
+        (forked from and joined back into the current stream), so the
+        latency-bound small kernels of one chain overlap the others."""
+        sq, d, torch = self.sq, self.d, self.torch
         eps = d["eps"]
+        main = torch.cuda.current_stream()
+        sA, sB, sC, sD, sE = self.streams
+        ev = self.events
         self.maxima.zero_()
-        for k in ("attn", "mlp"):
-            # a5 (calibration pass) -> linear input; a1 on it
-            sq.sq_norm_smooth_quant(self.h[k], sq.SQ_RMSNORM, self.gamma[k], None, eps, True, None, None, None,
-                                    None, self.V[k])
-            sq.sq_calib_absmax(self.V[k], self.xmax[k])
-        for k, w in (("attn", "qkv"), ("mlp", "gateup")):
-            sq.sq_weight_absmax(self.W[w], self.wmax[k])                       # a2
-            sq.sq_smooth_scales(self.xmax[k], self.wmax[k], d["alpha"], self.s[k])  # a3
-            sq.sq_fold_norm(self.gamma[k], None, self.s[k], self.gp[k])
-        sq.sq_quantize_weight(self.W["qkv"], self.s["attn"], True, self.Wq["qkv"], self.qw["qkv"])  # a4
-        sq.sq_quantize_weight(self.W["gateup"], self.s["mlp"], True, self.Wq["gateup"], self.qw["gateup"])
-        sq.sq_quantize_weight(self.W["o"], None, True, self.Wq["o"], self.qw["o"])
-        sq.sq_quantize_weight(self.W["down"], None, True, self.Wq["down"], self.qw["down"])
-        for k in ("attn", "mlp"):                                              # a5
-            sq.sq_norm_smooth_quant(self.h[k], sq.SQ_RMSNORM, self.gp[k], None, eps, True, None, self.Xq[k],
-                                    self.qx[k], None, None)
-        plan = [("qkv", self.Xq["attn"], self.qx["attn"]), ("o", *self.act_in["o"]),
-                ("gateup", self.Xq["mlp"], self.qx["mlp"]), ("down", *self.act_in["down"])]
-        for i, (w, xq, qx) in enumerate(plan):                                 # a6
+        for s_ in self.streams:
+            s_.wait_stream(main)
+
+        def gemm(i, w, xq, qx):                                                  # a6
             if gemm_ev is not None:
                 gemm_ev[i][0].record()
             sq.sq_gemm_w8a8(xq, self.Wq[w], qx, self.qw[w], None, self.Y[w], self.ws_gemm[w])
             if gemm_ev is not None:
                 gemm_ev[i][1].record()
-        sq.sq_llmint8_matmul(self.V["attn"], self.llm, 6.0, 0.0, self.Y["llm"], self.idx, self.nidx, self.ws)
+
+        with torch.cuda.stream(sC):
+            sq.sq_weight_absmax(self.W["qkv"], self.wmax["attn"])                  # a2
+            ev["wmax_attn"].record()
+            sq.sq_weight_absmax(self.W["gateup"], self.wmax["mlp"])
+            ev["wmax_mlp"].record()
+            sq.sq_quantize_weight(self.W["o"], None, True, self.Wq["o"], self.qw["o"])  # a4
+            gemm(1, "o", *self.act_in["o"])
+            sq.sq_quantize_weight(self.W["down"], None, True, self.Wq["down"], self.qw["down"])
+            gemm(3, "down", *self.act_in["down"])
+        chains = (("attn", "qkv", sA, 0), ("mlp", "gateup", sB, 2))
+        for k, w, s_, i in chains:
+            with torch.cuda.stream(s_):
+                # a5 (calibration pass) -> linear input; a1 on it
+                sq.sq_norm_smooth_quant(self.h[k], sq.SQ_RMSNORM, self.gamma[k], None, eps, True, None, None,
+                                        None, None, self.V[k])
+                ev["V_" + k].record()
+                sq.sq_calib_absmax(self.V[k], self.xmax[k])
+                s_.wait_event(ev["wmax_" + k])
+                sq.sq_smooth_scales(self.xmax[k], self.wmax[k], d["alpha"], self.s[k])  # a3
+                ev["s_" + k].record()
+                sq.sq_fold_norm(self.gamma[k], None, self.s[k], self.gp[k])
+                sq.sq_norm_smooth_quant(self.h[k], sq.SQ_RMSNORM, self.gp[k], None, eps, True, None,  # a5
+                                        self.Xq[k], self.qx[k], None, None)
+        with torch.cuda.stream(sD):
+            for k, w, _, _ in chains:
+                sD.wait_event(ev["s_" + k])
+                sq.sq_quantize_weight(self.W[w], self.s[k], True, self.Wq[w], self.qw[w])  # a4
+                ev["wq_" + w].record()
+        for k, w, s_, i in chains:
+            with torch.cuda.stream(s_):
+                s_.wait_event(ev["wq_" + w])
+                gemm(i, w, self.Xq[k], self.qx[k])
+        with torch.cuda.stream(sE):                                                # a7-a9
+            sE.wait_event(ev["V_attn"])
+            sq.sq_llmint8_matmul(self.V["attn"], self.llm, 6.0, 0.0, self.Y["llm"], self.idx, self.nidx, self.ws)
+        for s_ in self.streams:
+            main.wait_stream(s_)
 
     def outputs(self):
         return [self.Y[k] for k in ("qkv", "o", "gateup", "down", "llm")]
