@@ -89,6 +89,24 @@ def test_calib_absmax(dtype, M, K):
     assert np.array_equal(npf(xmax), ref)
 
 
+@pytest.mark.parametrize("dtype,M,K,ld", [(torch.bfloat16, 2061, 5128, 5128), (torch.float16, 1531, 6144, 6160),
+                                           (torch.float32, 1203, 4100, 4100)])
+def test_calib_absmax_bulk(dtype, M, K, ld):
+    """Inputs of 16 MB and more take the bulk-staged kernel: ragged row bands,
+    a short last column block, a row stride wider than K."""
+    X = rnd((M, ld), 11, dtype, 2.0)
+    X[M // 2, K - 1] = 500.0
+    X[M - 1, 7] = -300.0
+    xmax = torch.full((K,), 0.25, device=DEV)  # running max: entries above the data survive
+    xmax[5] = 1000.0
+    view = X.to(DEV)[:, :K]
+    assert view.numel() * view.element_size() >= 16 * 2**20
+    sq.sq_calib_absmax(view, xmax)
+    prev = np.full(K, 0.25, dtype=np.float32)
+    prev[5] = 1000.0
+    assert np.array_equal(npf(xmax), oracle.col_absmax(X[:, :K], prev))
+
+
 def test_calib_absmax_strided_and_weight():
     X = rnd((64, 1024), 3, torch.bfloat16)
     view = X.to(DEV)[:, 256:768]  # ld = 1024, K = 512
@@ -219,7 +237,39 @@ def test_norm_smooth_quant_per_token(dtype, norm, K):
 
 
 @pytest.mark.parametrize("norm", ["ln", "rms"])
-@pytest.mark.parametrize("K", [1024, 7168])
+@pytest.mark.parametrize("K,M,dtype", [(5000, 300, torch.bfloat16), (8192, 300, torch.float16),
+                                       (12288, 2500, torch.bfloat16), (13000, 300, torch.bfloat16),
+                                       (16384, 700, torch.float16)])
+def test_norm_quant_only(norm, K, M, dtype):
+    """Codes and scales without the V output, per token and with a static scale:
+    the quantise-only kernels, with full and ragged chunk sets; at M = 2500
+    every block of the grid cycles its ring of staged rows more than once."""
+    H = rnd((M, K), K + 7, dtype)
+    H[:, K // 3] *= 50
+    gamma = 1 + 0.1 * rnd(K, 5)
+    beta = 0.1 * rnd(K, 6) if norm == "ln" else None
+    eps = 1e-5 if norm == "ln" else 1e-6
+    nt = sq.SQ_LAYERNORM if norm == "ln" else sq.SQ_RMSNORM
+    on = oracle.LAYERNORM if norm == "ln" else oracle.RMSNORM
+    bd = None if beta is None else beta.to(DEV)
+    Hd = H.to(DEV)
+    Xq = torch.empty((M, K), dtype=torch.int8, device=DEV)
+    qs = torch.empty(M, device=DEV)
+    sq.sq_norm_smooth_quant(Hd, nt, gamma.to(DEV), bd, eps, True, None, Xq, qs, None, None)
+    r = oracle.norm_smooth_quant(H, on, gamma.numpy(), None if beta is None else beta.numpy(), eps, True)
+    assert np.array_equal(npf(qs), r["qs"])
+    assert np.array_equal(Xq.cpu().numpy(), r["Xq"])
+    qst = torch.tensor([21.5], device=DEV)
+    qx = torch.empty(1, device=DEV)
+    sq.sq_norm_smooth_quant(Hd, nt, gamma.to(DEV), bd, eps, False, qst, Xq, qx, None, None)
+    r = oracle.norm_smooth_quant(H, on, gamma.numpy(), None if beta is None else beta.numpy(), eps,
+                                 per_token=False, static_qs=21.5)
+    assert np.array_equal(Xq.cpu().numpy(), r["Xq"])
+    assert npf(qx)[0] == np.float32(21.5)
+
+
+@pytest.mark.parametrize("norm", ["ln", "rms"])
+@pytest.mark.parametrize("K", [1024, 7168, 12288])
 def test_norm_static_and_calibration(norm, K):
     """Calibration mode (running per-channel max of |v| over batches) and the
     static per-tensor scale taken from it, the OPT-30B-style path."""

@@ -25,7 +25,8 @@
 //   4096 < K <= 16384: one 256-thread block per row, thread t = lane t. Rows
 //     reach shared memory through a ring of buffers, one bulk copy (TMA
 //     engine, cp.async.bulk) per row issued R rows ahead, so several rows per
-//     block are in flight while the block reduces and quantises.
+//     block are in flight while the block reduces and quantises; gamma' of a
+//     thread's chunks lives in its registers for the whole launch.
 // The codes are written 8 bytes per chunk, the per-token scale once per row.
 #include "sq_common.cuh"
 
@@ -62,13 +63,11 @@ __device__ __forceinline__ float warp_max(float v) {
     return v;
 }
 
-// v_j of one 8-element chunk; g holds gamma'_j of the chunk, beta'_j is read
-// from a.beta (LayerNorm with a shift only)
-template <typename T, bool LN>
-__device__ __forceinline__ void compute_v_g(const uint4& rw, int ch, const NormArgs& a, const float* g, float mu,
+// v_j of one 8-element chunk from its fp32 inputs f (v may alias f); g holds
+// gamma'_j of the chunk, beta'_j is read from a.beta (LayerNorm with a shift)
+template <bool LN>
+__device__ __forceinline__ void compute_v_f(const float* f, int ch, const NormArgs& a, const float* g, float mu,
                                             float r, float* v) {
-    float f[8];
-    unpack<T>(rw, f);
     const uint64_t r2 = pk2(r, r);
     if constexpr (LN) {
         const uint64_t nmu2 = pk2(-mu, -mu);  // x + (-mu) is the IEEE x - mu
@@ -93,6 +92,15 @@ __device__ __forceinline__ void compute_v_g(const uint4& rw, int ch, const NormA
 #pragma unroll
         for (int e = 0; e < 8; e += 2) upk2(mul2(mul2(pk2(f[e], f[e + 1]), r2), pk2(g[e], g[e + 1])), v[e], v[e + 1]);
     }
+}
+
+// the same from the chunk's 16-bit inputs
+template <typename T, bool LN>
+__device__ __forceinline__ void compute_v_g(const uint4& rw, int ch, const NormArgs& a, const float* g, float mu,
+                                            float r, float* v) {
+    float f[8];
+    unpack<T>(rw, f);
+    compute_v_f<LN>(f, ch, a, g, mu, r, v);
 }
 
 __device__ __forceinline__ void load_gamma(const NormArgs& a, int ch, float* g) {
@@ -293,12 +301,15 @@ __device__ __forceinline__ float block_max8(float v, float* sh) {
 // One 256-thread block per row, rows strided over the grid (K <= 256*8*C).
 // Thread t always owns chunks t, t+256, ..., so gamma'_j of its chunks is
 // loaded once into registers. The rows arrive in a ring of R shared-memory
-// buffers, each filled by one bulk copy issued R rows ahead. With KEEPV the
-// values v of the thread's chunks stay in registers from the absmax to the
-// codes and the row's buffer is refilled right after the absmax reduction;
-// otherwise v is formed again from the staged row for the codes and the
-// buffer is refilled after them.
-template <typename T, bool LN, int C, bool KEEPV>
+// buffers, each filled by one bulk copy issued R rows ahead.
+//   KEEPV: the sum pass unpacks the thread's chunks into registers, so the
+//     row's buffer is refilled right after the first reduction, and v is
+//     formed in place and kept there until the codes are written.
+//   otherwise (K > 12288): every pass reads the staged row again and the
+//     buffer is refilled after the codes.
+// FULL: K == 2048 * C, every thread owns exactly C chunks (no tail test).
+// QONLY: codes and scales only (no V output, no calibration maxima).
+template <typename T, bool LN, int C, bool KEEPV, bool FULL, bool QONLY>
 __global__ void __launch_bounds__(kBlock, 2)
 norm_quant_bulk_kernel(const T* __restrict__ H, NormArgs a, int R) {
     pdl_wait();
@@ -312,17 +323,18 @@ norm_quant_bulk_kernel(const T* __restrict__ H, NormArgs a, int R) {
     const uint32_t row_bytes = (uint32_t)(a.K * sizeof(T));
     float* amax_sh = reinterpret_cast<float*>(dsm + (size_t)R * row_bytes);
     const int64_t G = gridDim.x;
+    auto mine = [&](int c) { return FULL || t + c * kBlock < nch; };
     float g[C][8];
 #pragma unroll
     for (int c = 0; c < C; ++c)
-        if (t + c * kBlock < nch) load_gamma(a, t + c * kBlock, g[c]);
+        if (mine(c)) load_gamma(a, t + c * kBlock, g[c]);
     if (t == 0) {
         for (int i = 0; i < R; ++i)
             asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bars[i])));
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
-    if (a.absmax)
+    if (!QONLY && a.absmax)
         for (int j = t; j < a.K; j += kBlock) amax_sh[j] = 0.0f;
     __syncwarp();
     __syncthreads();
@@ -342,7 +354,8 @@ norm_quant_bulk_kernel(const T* __restrict__ H, NormArgs a, int R) {
             aborted = true;
             break;
         }
-        auto chunk = [&](int ch) { return *reinterpret_cast<const uint4*>(xs + (size_t)ch * 16); };
+        auto chunk = [&](int c) { return *reinterpret_cast<const uint4*>(xs + (size_t)(t + c * kBlock) * 16); };
+        // every thread is past its last read of the slot: refill it R rows ahead
         auto refill = [&]() {
             if (t == 0) {
                 const int64_t nr = row + (int64_t)R * G;
@@ -353,25 +366,31 @@ norm_quant_bulk_kernel(const T* __restrict__ H, NormArgs a, int R) {
                 }
             }
         };
+        float vk[KEEPV ? C : 1][8];
+        // pass 1: the sum (LayerNorm: of x; RMSNorm: of x^2) in the lane's order
+        float acc = 0.0f;
+#pragma unroll
+        for (int c = 0; c < C; ++c) {
+            if (mine(c)) {
+                float fl[8];
+                float* f = KEEPV ? vk[c] : fl;
+                unpack<T>(chunk(c), f);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc = LN ? __fmaf_rn(f[e], 1.0f, acc) : __fmaf_rn(f[e], f[e], acc);
+            }
+        }
+        const float sum = canon_block_sum(acc, sh[0]);
+        if constexpr (KEEPV) refill();
         float mu = 0.0f, r;
         if constexpr (LN) {
-            float acc = 0.0f;
-#pragma unroll
-            for (int c = 0; c < C; ++c) {
-                if (t + c * kBlock < nch) {
-                    float f[8];
-                    unpack<T>(chunk(t + c * kBlock), f);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) acc = __fmaf_rn(f[e], 1.0f, acc);
-                }
-            }
-            mu = __fdiv_rn(canon_block_sum(acc, sh[0]), Kf);
+            mu = __fdiv_rn(sum, Kf);
             acc = 0.0f;
 #pragma unroll
             for (int c = 0; c < C; ++c) {
-                if (t + c * kBlock < nch) {
-                    float f[8];
-                    unpack<T>(chunk(t + c * kBlock), f);
+                if (mine(c)) {
+                    float fl[8];
+                    if constexpr (!KEEPV) unpack<T>(chunk(c), fl);
+                    const float* f = KEEPV ? vk[c] : fl;
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const float d = __fsub_rn(f[e], mu);
@@ -382,58 +401,40 @@ norm_quant_bulk_kernel(const T* __restrict__ H, NormArgs a, int R) {
             const float var = __fdiv_rn(canon_block_sum(acc, sh[1]), Kf);
             r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(var, a.eps)));
         } else {
-            float acc = 0.0f;
-#pragma unroll
-            for (int c = 0; c < C; ++c) {
-                if (t + c * kBlock < nch) {
-                    float f[8];
-                    unpack<T>(chunk(t + c * kBlock), f);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) acc = __fmaf_rn(f[e], f[e], acc);
-                }
-            }
-            const float ms = __fdiv_rn(canon_block_sum(acc, sh[0]), Kf);
-            r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, a.eps)));
+            r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(sum, Kf), a.eps)));
         }
-        float vk[KEEPV ? C : 1][8];
+        // pass 2: v, its absmax, the optional outputs
         float m = 0.0f;
-        if (KEEPV || (a.Xq && a.per_token) || a.absmax || a.V) {
+        if (KEEPV || a.per_token || (!QONLY && (a.absmax || a.V))) {
 #pragma unroll
             for (int c = 0; c < C; ++c) {
                 const int ch = t + c * kBlock;
-                if (ch < nch) {
-                    float v[8];
-                    compute_v_g<T, LN>(chunk(ch), ch, a, g[c], mu, r, v);
+                if (mine(c)) {
+                    float vl[8];
+                    float* v = KEEPV ? vk[c] : vl;
+                    if constexpr (KEEPV) compute_v_f<LN>(vk[c], ch, a, g[c], mu, r, v);
+                    else compute_v_g<T, LN>(chunk(c), ch, a, g[c], mu, r, v);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(v[e]));
-                    if (a.absmax) {
-                        float4* am = reinterpret_cast<float4*>(amax_sh + ch * 8);
-                        const float4 o0 = am[0], o1 = am[1];
-                        am[0] = make_float4(fmaxf(o0.x, fabsf(v[0])), fmaxf(o0.y, fabsf(v[1])),
-                                            fmaxf(o0.z, fabsf(v[2])), fmaxf(o0.w, fabsf(v[3])));
-                        am[1] = make_float4(fmaxf(o1.x, fabsf(v[4])), fmaxf(o1.y, fabsf(v[5])),
-                                            fmaxf(o1.z, fabsf(v[6])), fmaxf(o1.w, fabsf(v[7])));
-                    }
-                    if (a.V) store_v16<T>(a, row, ch, v);
-                    if constexpr (KEEPV) {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) vk[c][e] = v[e];
+                    if constexpr (!QONLY) {
+                        if (a.absmax) {
+                            float4* am = reinterpret_cast<float4*>(amax_sh + ch * 8);
+                            const float4 o0 = am[0], o1 = am[1];
+                            am[0] = make_float4(fmaxf(o0.x, fabsf(v[0])), fmaxf(o0.y, fabsf(v[1])),
+                                                fmaxf(o0.z, fabsf(v[2])), fmaxf(o0.w, fabsf(v[3])));
+                            am[1] = make_float4(fmaxf(o1.x, fabsf(v[4])), fmaxf(o1.y, fabsf(v[5])),
+                                                fmaxf(o1.z, fabsf(v[6])), fmaxf(o1.w, fabsf(v[7])));
+                        }
+                        if (a.V) store_v16<T>(a, row, ch, v);
                     }
                 }
             }
         }
-        float mx = 0.0f;
-        if (a.Xq && a.per_token) {
-            mx = block_max8(m, sh[2]);
-        } else if (KEEPV) {
-            __syncwarp();
-            __syncthreads();
-        }
-        if constexpr (KEEPV) refill();  // every thread is past its last read of the slot
-        if (a.Xq) {
+        // pass 3: the codes
+        if (QONLY || a.Xq) {
             float qs;
             if (a.per_token) {
-                qs = __fdiv_rn(127.0f, fmaxf(mx, 1e-8f));
+                qs = __fdiv_rn(127.0f, fmaxf(block_max8(m, sh[2]), 1e-8f));
                 if (t == 0) a.qs_x[row] = qs;
             } else {
                 qs = *a.static_qs;
@@ -443,22 +444,26 @@ norm_quant_bulk_kernel(const T* __restrict__ H, NormArgs a, int R) {
 #pragma unroll
             for (int c = 0; c < C; ++c) {
                 const int ch = t + c * kBlock;
-                if (ch < nch) {
+                if (mine(c)) {
                     if constexpr (KEEPV) {
                         *reinterpret_cast<uint2*>(q + ch * 8) = codes8(vk[c], qs, !a.per_token);
                     } else {
                         float v[8];
-                        compute_v_g<T, LN>(chunk(ch), ch, a, g[c], mu, r, v);
+                        compute_v_g<T, LN>(chunk(c), ch, a, g[c], mu, r, v);
                         *reinterpret_cast<uint2*>(q + ch * 8) = codes8(v, qs, !a.per_token);
                     }
                 }
             }
         }
         if constexpr (!KEEPV) {
+            // the codes read the staged row: refill its buffer once every
+            // thread is done with it
             __syncwarp();
             __syncthreads();
             refill();
         }
+        // (the shared partials of the reductions are next written after the
+        // next row's first barrier, so no barrier is needed here)
     }
     if (aborted && t == 0) {
         // drain copies still in flight before the block's shared memory is released
@@ -469,7 +474,7 @@ norm_quant_bulk_kernel(const T* __restrict__ H, NormArgs a, int R) {
                     if (global_ns() - t0 > kWaitNs / 4) break;
         }
     }
-    if (a.absmax) {
+    if (!QONLY && a.absmax) {
         __syncwarp();
         __syncthreads();
         for (int j = t; j < a.K; j += kBlock) atomic_max_nonneg(a.absmax + j, amax_sh[j]);
@@ -487,9 +492,9 @@ void launch_warp(const void* H, const NormArgs& a, cudaStream_t s) {
     launch_pdl(kern, dim3((unsigned)blocks), dim3(256), smem, s, static_cast<const T*>(H), a);
 }
 
-template <typename T, bool LN, int C, bool KEEPV>
-void launch_block(const void* H, const NormArgs& a, cudaStream_t s) {
-    auto kern = norm_quant_bulk_kernel<T, LN, C, KEEPV>;
+template <typename T, bool LN, int C, bool KEEPV, bool FULL, bool QONLY>
+void launch_block_k(const void* H, const NormArgs& a, cudaStream_t s) {
+    auto kern = norm_quant_bulk_kernel<T, LN, C, KEEPV, FULL, QONLY>;
     const size_t row_bytes = (size_t)a.K * sizeof(T);
     int R = (int)((96 * 1024) / row_bytes);  // about 96 KB of staged rows per block
     if (R < 2) R = 2;
@@ -503,6 +508,19 @@ void launch_block(const void* H, const NormArgs& a, cudaStream_t s) {
     if (a.absmax) grid = (int64_t)num_sms();  // fewer blocks: one publish of [K] per block
     if (grid > a.M) grid = a.M;
     launch_pdl(kern, dim3((unsigned)grid), dim3(kBlock), smem, s, static_cast<const T*>(H), a, R);
+}
+
+template <typename T, bool LN, int C, bool KEEPV>
+void launch_block(const void* H, const NormArgs& a, cudaStream_t s) {
+    const bool full = a.K == 2048 * C;
+    const bool qonly = a.Xq && !a.absmax && !a.V;
+    if (full) {
+        if (qonly) launch_block_k<T, LN, C, KEEPV, true, true>(H, a, s);
+        else launch_block_k<T, LN, C, KEEPV, true, false>(H, a, s);
+    } else {
+        if (qonly) launch_block_k<T, LN, C, KEEPV, false, true>(H, a, s);
+        else launch_block_k<T, LN, C, KEEPV, false, false>(H, a, s);
+    }
 }
 
 template <typename T, bool LN>
