@@ -59,6 +59,10 @@ def _declare(L):
     L.or_smooth_scales.argtypes = [_p, _p, _i64, _d, _p]
     L.or_fold_weight.argtypes = [_p, _i64, _i64, _p, _i, _p]
     L.or_fold_norm.argtypes = [_p, _p, _p, _i64, _i, _p, _p]
+    L.or_fold_prev_linear.argtypes = [_p, _i64, _i64, _p, _p, _i, _p, _p]
+    L.or_expf_array.argtypes = [_p, _i64, _p]
+    L.or_silu_array.argtypes = [_p, _i64, _p]
+    L.or_act_quant.argtypes = [_p, _i64, _i64, _i64, _i, _i, _p, _p, _p, _p, _p]
     L.or_quantize_weight.argtypes = [_p, _i64, _i64, _i, _p, _p]
     L.or_quantize_act.argtypes = [_p, _i64, _i64, _i64, _p, _i, _p, _p, _p]
     L.or_scale_from_absmax.argtypes = [_p, _i64]
@@ -136,6 +140,54 @@ def fold_norm(gamma, beta, s, round_f32=True):
     if round_f32:
         return go.astype(np.float32), (None if bo is None else bo.astype(np.float32))
     return go, bo
+
+
+# ---------------------------------------------------------------- f2
+def fold_prev_linear(W, s, bias=None, round_f32=True):
+    """Output channel n of the previous layer (row n, bias_n) divided by s_n."""
+    W = _c(f32(W) if round_f32 else W, np.float64)
+    s = _c(s, np.float64)
+    b = None if bias is None else _c(f32(bias) if round_f32 else bias, np.float64)
+    N, K = W.shape
+    out = np.empty_like(W)
+    bo = None if b is None else np.empty_like(b)
+    lib().or_fold_prev_linear(_ptr(W), N, K, _ptr(b), _ptr(s), int(round_f32), _ptr(out), _ptr(bo))
+    if round_f32:
+        return out.astype(np.float32), (None if bo is None else bo.astype(np.float32))
+    return out, bo
+
+
+# ---------------------------------------------------------------- f1
+SWIGLU, RELU = 0, 1
+
+
+def expf(x):
+    x = f32(np.atleast_1d(x))
+    out = np.empty_like(x)
+    lib().or_expf_array(_ptr(x), x.size, _ptr(out))
+    return out
+
+
+def silu(x):
+    x = f32(np.atleast_1d(x))
+    out = np.empty_like(x)
+    lib().or_silu_array(_ptr(x), x.size, _ptr(out))
+    return out
+
+
+def act_quant(A, act, per_token=True, static_qs=None, quantize=True, absmax=None, want_h=False):
+    """SwiGLU (A = [gate | up], [M, 2I]) or ReLU (A = [M, I]) then int8."""
+    A = f32(A)
+    M, W = A.shape
+    I = W // 2 if act == SWIGLU else W
+    st = None if static_qs is None else np.array([static_qs], np.float32)
+    Xq = np.empty((M, I), np.int8) if quantize else None
+    qs = np.empty(M if per_token else 1, np.float32) if quantize else None
+    am = None if absmax is None else _c(absmax, np.float32).copy()
+    H = np.empty((M, I), np.float32) if want_h else None
+    lib().or_act_quant(_ptr(A), M, I, W, int(act), int(per_token), _ptr(st), _ptr(Xq), _ptr(qs), _ptr(am),
+                       _ptr(H))
+    return {"Xq": Xq, "qs": qs, "absmax": am, "H": H}
 
 
 # ---------------------------------------------------------------- a4

@@ -42,11 +42,15 @@
  *   R5 the normalisation sums follow a fixed reduction order (below);
  *   R6 LLM.int8: the outlier test is strict (|x| > thr); min_ratio = 0 means
  *      any one element marks the column; the 16-bit path is exact products
- *      summed in ascending outlier order, added to the dequantised int8 path.
+ *      summed in ascending outlier order, added to the dequantised int8 path;
+ *   R7 the MLP activation SiLU is evaluated with a fixed fp32 exponential
+ *      (below, f1); the fold into the previous linear divides its output
+ *      channels by s in fp32 (f2).
  */
 #include "sq_oracle.h"
 
 #include <math.h>
+#include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
 
@@ -132,6 +136,106 @@ void or_fold_norm(const double* gamma, const double* beta, const double* s, int6
             beta_out[j] = round_f32 ? (double)((float)beta[j] / (float)s[j]) : b;
         }
     }
+}
+
+/* ------------------------------------------------------------------ f2
+ * Fold 1/s into the previous linear layer   [SQ-p2] 融入前序线性层的权重 and
+ * the table after it (down_proj: up_proj's output channels; o_proj: v_proj's
+ * output channels): output channel j of the previous layer (row j of W [N,K],
+ * and bias_j) is divided by s_j, so its output, the next layer's input
+ * channel j, arrives divided by s_j; the next layer's weight takes s_j on its
+ * input channel j (or_fold_weight).  round_f32: one fp32 division per value
+ * (an fp64 quotient of two fp32 values rounded once to fp32 is the fp32
+ * quotient).  Pinned by: the fp64 identity down(act(gate) * up) unchanged
+ * under (up / s, down * s), with a negative control folding the wrong axis. */
+void or_fold_prev_linear(const double* W, int64_t N, int64_t K, const double* bias, const double* s,
+                         int round_f32, double* Wp, double* bias_out) {
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t k = 0; k < K; ++k) {
+            double q = W[n * K + k] / s[n];
+            Wp[n * K + k] = round_f32 ? (double)((float)W[n * K + k] / (float)s[n]) : q;
+        }
+        if (bias && bias_out) {
+            double b = bias[n] / s[n];
+            bias_out[n] = round_f32 ? (double)((float)bias[n] / (float)s[n]) : b;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------ f1
+ * The input of down_proj (FC2) is act(gate_proj(x)) * up_proj(x) ([SQ-p2]
+ * 融入前序线性层的权重), or relu(fc1(x)) for a ReLU MLP; with 1/s folded into
+ * up_proj's (fc1's) output channels it arrives already smoothed, and is
+ * quantised to int8 like any activation ([SQ-p5] §2.1).
+ *
+ * The pages name the activation but no way to evaluate it. Reading R7: SiLU,
+ * silu(g) = g / (1 + exp(-g)), with exp evaluated by a fixed sequence of fp32
+ * operations (Cody-Waite reduction x = n ln2 + r with ln 2 in two parts, and
+ * the Taylor polynomial of exp(r) to degree 7 by Horner's rule), the same
+ * sequence the CUDA kernel evaluates, so h and the codes it decides agree bit
+ * for bit. Pinned by: exp within 4 ulp of the fp64 exp on a dense grid;
+ * silu(g) - silu(-g) = g; the fp64 identity of the fold. */
+#define OR_LOG2E 0x1.715476p+0f   /* log2(e) rounded to fp32 */
+#define OR_LN2_HI 0x1.62e000p-1f  /* 2839/4096: ln 2 to 12 bits, so n*LN2_HI is exact */
+#define OR_LN2_LO 0x1.0bfbe8p-15f /* ln 2 - LN2_HI, rounded to fp32 */
+
+float or_expf(float x) {
+    if (x > 88.0f) return (float)INFINITY;
+    if (x < -87.0f) return 0.0f;
+    const float n = rintf(x * OR_LOG2E); /* in [-126, 127] */
+    float r = fmaf(-n, OR_LN2_HI, x);
+    r = fmaf(-n, OR_LN2_LO, r);
+    /* 1/k! for k = 7 .. 0 */
+    float p = 1.0f / 5040.0f;
+    p = fmaf(p, r, 1.0f / 720.0f);
+    p = fmaf(p, r, 1.0f / 120.0f);
+    p = fmaf(p, r, 1.0f / 24.0f);
+    p = fmaf(p, r, 1.0f / 6.0f);
+    p = fmaf(p, r, 0.5f);
+    p = fmaf(p, r, 1.0f);
+    p = fmaf(p, r, 1.0f);
+    union { uint32_t u; float f; } two_n;
+    two_n.u = (uint32_t)((int)n + 127) << 23;
+    return p * two_n.f;
+}
+
+float or_silu(float g) { return g / (1.0f + or_expf(-g)); }
+
+void or_expf_array(const float* x, int64_t n, float* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = or_expf(x[i]);
+}
+void or_silu_array(const float* x, int64_t n, float* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = or_silu(x[i]);
+}
+
+void or_act_quant(const float* A, int64_t M, int64_t I, int64_t ld, int act, int per_token,
+                  const float* static_qs, int8_t* Xq, float* qs_x, float* absmax_io, float* H) {
+    float* h = (float*)malloc(sizeof(float) * (size_t)(I > 0 ? I : 1));
+    for (int64_t i = 0; i < M; ++i) {
+        const float* a = A + i * ld;
+        float m = 0.0f;
+        for (int64_t j = 0; j < I; ++j) {
+            float v;
+            if (act == 0) v = or_silu(a[j]) * a[I + j]; /* gate | up halves of the row */
+            else v = a[j] > 0.0f ? a[j] : 0.0f;
+            h[j] = v;
+            const float av = absf(v);
+            if (av > m) m = av;
+            if (absmax_io && av > absmax_io[j]) absmax_io[j] = av;
+            if (H) H[i * I + j] = v;
+        }
+        if (!Xq) continue;
+        float qs;
+        if (per_token) {
+            qs = scale_of(m);
+            qs_x[i] = qs;
+        } else {
+            qs = *static_qs;
+            if (i == 0) qs_x[0] = qs;
+        }
+        for (int64_t j = 0; j < I; ++j) Xq[i * I + j] = q_clip(h[j] * qs);
+    }
+    free(h);
 }
 
 /* ------------------------------------------------------------------ a4

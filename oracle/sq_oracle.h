@@ -43,6 +43,14 @@ void or_fold_weight(const double* W, int64_t N, int64_t K, const double* s,
 
 /* gamma' = gamma / s, beta' = beta / s (beta may be NULL). Same rounding
  * switch as or_fold_weight. */
+void or_fold_prev_linear(const double* W, int64_t N, int64_t K, const double* bias, const double* s,
+                         int round_f32, double* Wp, double* bias_out);
+float or_expf(float x);
+float or_silu(float g);
+void or_expf_array(const float* x, int64_t n, float* out);
+void or_silu_array(const float* x, int64_t n, float* out);
+void or_act_quant(const float* A, int64_t M, int64_t I, int64_t ld, int act, int per_token,
+                  const float* static_qs, int8_t* Xq, float* qs_x, float* absmax_io, float* H);
 void or_fold_norm(const double* gamma, const double* beta, const double* s, int64_t K,
                   int round_f32, double* gamma_out, double* beta_out);
 

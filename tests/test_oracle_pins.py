@@ -414,3 +414,144 @@ def test_col_absmax_bruteforce(orc):
     ref = np.array([max(prev[j], max(abs(float(X[i, j])) for i in range(37))) for j in range(29)],
                    np.float32)
     assert np.array_equal(got, ref)
+
+
+# ---------------------------------------------------------------- f1 / f2
+def _ulps(got, ref64):
+    """|got - ref| in units of the fp32 spacing at ref."""
+    ref32 = ref64.astype(np.float32)
+    return np.abs(got.astype(np.float64) - ref64) / np.spacing(np.abs(ref32)).astype(np.float64)
+
+
+def test_expf_within_4ulp_of_fp64(orc):
+    """The fixed fp32 exponential against the fp64 exp on a dense grid of its
+    finite range, and its end values."""
+    x = np.linspace(-87.0, 88.0, 400_001).astype(np.float32)
+    e = orc.expf(x)
+    assert np.max(_ulps(e, np.exp(x.astype(np.float64)))) <= 4.0
+    assert orc.expf(0.0)[0] == 1.0
+    assert np.isinf(orc.expf(88.5)[0]) and orc.expf(-87.5)[0] == 0.0
+    # across the 2^n seams of the reduction (x = (n + 1/2) ln 2) the result
+    # stays monotone
+    seams = (np.arange(-120, 120) + 0.5) * np.log(2.0)
+    xs = np.concatenate([np.nextafter(seams.astype(np.float32), -np.inf), seams.astype(np.float32),
+                         np.nextafter(seams.astype(np.float32), np.inf)]).astype(np.float32)
+    xs = np.sort(xs[(xs > -87) & (xs < 88)])
+    assert np.all(np.diff(orc.expf(xs)) >= 0)
+
+
+def test_silu_identities(orc):
+    """silu(g) = g * sigmoid(g): silu(g) - silu(-g) = g; silu(0) = 0; silu(g)
+    = g once exp(-g) vanishes next to 1; within a few ulp of the fp64 value."""
+    g = np.linspace(-60, 60, 240_001).astype(np.float32)
+    s = orc.silu(g).astype(np.float64)
+    sn = orc.silu(-g).astype(np.float64)
+    assert np.max(np.abs((s - sn) - g.astype(np.float64)) / np.maximum(np.abs(g), 1e-3)) < 2e-6
+    g64 = g.astype(np.float64)
+    ref = g64 / (1.0 + np.exp(-g64))
+    big = np.abs(ref) > 1e-30
+    assert np.max(_ulps(orc.silu(g)[big], ref[big])) <= 6.0
+    assert orc.silu(0.0)[0] == 0.0
+    assert orc.silu(30.0)[0] == 30.0 and orc.silu(1000.0)[0] == 1000.0
+    assert orc.silu(-100.0)[0] == 0.0
+
+
+def test_swiglu_quant_against_fp64(orc):
+    """h = silu(gate) * up per element ([gate | up] halves of a row), per-token
+    int8: h within a few ulp of the fp64 value and the codes those of the fp64
+    h wherever the fp64 value is not within 1e-3 of a rounding tie. Swapping
+    the halves (a plausible mistake) is far off."""
+    rng = np.random.default_rng(30)
+    M, I = 40, 96
+    A = (rng.normal(size=(M, 2 * I)) * 3).astype(np.float32)
+    r = orc.act_quant(A, orc.SWIGLU, want_h=True)
+    g64, u64 = A[:, :I].astype(np.float64), A[:, I:].astype(np.float64)
+    h64 = g64 / (1.0 + np.exp(-g64)) * u64
+    big = np.abs(h64) > 1e-20
+    assert np.max(_ulps(r["H"][big], h64[big])) <= 8.0
+    qs64 = 127.0 / np.max(np.abs(h64), axis=1)
+    assert np.max(np.abs(r["qs"] / qs64 - 1)) < 1e-6
+    t = h64 * qs64[:, None]
+    clear = np.abs(np.abs(t - np.floor(t)) - 0.5) > 1e-3
+    assert np.array_equal(r["Xq"][clear], np.rint(t)[clear].astype(np.int8))
+    swapped = u64 / (1.0 + np.exp(-u64)) * g64
+    assert np.max(np.abs(swapped - h64)) > 1.0
+
+
+def test_relu_quant_bruteforce(orc):
+    """ReLU MLP input: h = max(x, 0), then int8 per token or with a static scale."""
+    rng = np.random.default_rng(31)
+    X = rng.normal(size=(7, 24)).astype(np.float32)
+    X[2] = -np.abs(X[2])  # an all-negative row: h = 0, scale from the 1e-8 floor
+    r = orc.act_quant(X, orc.RELU, want_h=True)
+    for i in range(7):
+        h = [max(float(v), 0.0) for v in X[i]]
+        m = max(h)
+        qs = np.float32(127.0) / np.float32(max(m, 1e-8))
+        assert r["qs"][i] == qs
+        for j in range(24):
+            assert r["H"][i, j] == np.float32(h[j])
+            assert r["Xq"][i, j] == int(np.clip(np.rint(np.float32(h[j]) * qs), -127, 127))
+    rs = orc.act_quant(X, orc.RELU, per_token=False, static_qs=40.0)
+    assert rs["qs"][0] == np.float32(40.0)
+    assert np.array_equal(rs["Xq"], np.clip(np.rint(np.maximum(X, 0) * np.float32(40.0)), -127, 127).astype(np.int8))
+
+
+def _silu64(x):
+    return x / (1.0 + np.exp(-x))
+
+
+def test_fold_prev_linear_identity_mlp(orc):
+    """[SQ-p2] 融入前序线性层的权重: up_proj's output channel j divided by s_j and
+    down_proj's input channel j multiplied by s_j leave the FFN output
+    unchanged (fp64, exact folds); folding up_proj on its input axis instead
+    does not."""
+    rng = np.random.default_rng(32)
+    M, D, I = 6, 16, 24
+    x = rng.normal(size=(M, D))
+    Wg, Wu = rng.normal(size=(I, D)), rng.normal(size=(I, D))
+    Wd = rng.normal(size=(D, I))
+    bu = rng.normal(size=I)
+    s = np.exp(rng.normal(size=I))
+    y = (_silu64(x @ Wg.T) * (x @ Wu.T + bu)) @ Wd.T
+    Wu2, bu2 = orc.fold_prev_linear(Wu, s, bu, round_f32=False)
+    Wd2 = orc.fold_weight(Wd, s, round_f32=False)
+    h2 = _silu64(x @ Wg.T) * (x @ Wu2.T + bu2)
+    assert np.allclose(h2, (_silu64(x @ Wg.T) * (x @ Wu.T + bu)) / s, rtol=1e-12, atol=0)
+    y2 = h2 @ Wd2.T
+    assert np.max(np.abs(y2 - y)) / np.max(np.abs(y)) < 1e-12
+    s_in = np.exp(rng.normal(size=D))
+    Wu_bad = orc.fold_weight(Wu, s_in, round_f32=False)  # the input axis: wrong
+    y_bad = (_silu64(x @ Wg.T) * (x @ Wu_bad.T + bu)) @ Wd.T
+    assert np.max(np.abs(y_bad - y)) / np.max(np.abs(y)) > 1e-3
+
+
+def test_fold_prev_linear_identity_attention(orc):
+    """o_proj's input is a convex mix of v_proj's outputs (attention weights P
+    with rows summing to 1), so v_proj rows / s and o_proj columns * s leave
+    the attention output unchanged (fp64)."""
+    rng = np.random.default_rng(33)
+    T, D = 9, 12
+    x = rng.normal(size=(T, D))
+    Wv, Wo = rng.normal(size=(D, D)), rng.normal(size=(D, D))
+    P = np.exp(rng.normal(size=(T, T)))
+    P /= P.sum(axis=1, keepdims=True)
+    s = np.exp(rng.normal(size=D))
+    y = (P @ (x @ Wv.T)) @ Wo.T
+    Wv2, _ = orc.fold_prev_linear(Wv, s, round_f32=False)
+    Wo2 = orc.fold_weight(Wo, s, round_f32=False)
+    y2 = (P @ (x @ Wv2.T)) @ Wo2.T
+    assert np.max(np.abs(y2 - y)) / np.max(np.abs(y)) < 1e-12
+
+
+def test_fold_prev_linear_fp32_is_one_division(orc):
+    """In fp32 each folded value is the correctly rounded quotient: an fp64
+    quotient of fp32 operands rounded once (53 >= 2*24 + 2 bits, so the double
+    rounding is innocuous), equal to numpy's float32 division."""
+    rng = np.random.default_rng(34)
+    W = rng.normal(size=(33, 17)).astype(np.float32)
+    b = rng.normal(size=33).astype(np.float32)
+    s = np.exp(rng.normal(size=33)).astype(np.float32)
+    Wp, bp = orc.fold_prev_linear(W, s, b)
+    assert np.array_equal(Wp, W / s[:, None])
+    assert np.array_equal(bp, b / s)
