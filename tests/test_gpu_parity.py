@@ -394,7 +394,8 @@ def test_gemm_deterministic():
     assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
 
 
-@pytest.mark.parametrize("M,N,K", [(4096, 36864, 12288), (1024, 28672, 7168), (2048, 16384, 4096)])
+@pytest.mark.parametrize("M,N,K", [(4096, 36864, 12288), (1024, 28672, 7168), (2048, 16384, 4096),
+                                   (1024, 7168, 28672)])
 def test_gemm_full_size_sampled(M, N, K):
     """Full-size shapes in the launch configuration the benchmark times:
     all outputs against torch._int_mm (a library cross-check, test only) and

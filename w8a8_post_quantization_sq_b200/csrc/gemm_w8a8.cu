@@ -11,8 +11,12 @@
 // products are exact in fp32).
 //
 // Design (sm_100a):
-//   - persistent: one 192-thread CTA per SM loops over 128 x BN output tiles,
-//     M index fastest so the CTAs running together share weight tiles in L2;
+//   - persistent: one 320-thread CTA per SM loops over 128 x BN output tiles
+//     in a grouped raster (the CTAs running together share Xq rows and weight
+//     tiles in L2); whole tiles only: a stream-K split of the k-loop was
+//     measured slower on this part (pieces at scattered k-offsets lose the
+//     L2 reuse of whole tiles running in lockstep, and cost more than the
+//     idle tail they remove);
 //   - warp 0 (one lane) issues TMA loads of 128 x 128 int8 tiles of Xq and
 //     BN x 128 tiles of Wq (128-byte swizzle) into a 4-stage shared-memory
 //     ring guarded by mbarriers;
