@@ -60,6 +60,15 @@ def _declare(L):
     L.or_fold_weight.argtypes = [_p, _i64, _i64, _p, _i, _p]
     L.or_fold_norm.argtypes = [_p, _p, _p, _i64, _i, _p, _p]
     L.or_fold_prev_linear.argtypes = [_p, _i64, _i64, _p, _p, _i, _p, _p]
+    L.or_e4m3_round.argtypes = [_f]
+    L.or_e4m3_round.restype = _f
+    L.or_e4m3_bits.argtypes = [_f]
+    L.or_e4m3_bits.restype = ctypes.c_uint8
+    L.or_e4m3_value.argtypes = [ctypes.c_uint8]
+    L.or_e4m3_value.restype = _d
+    L.or_quantize_fp8.argtypes = [_p, _i64, _i64, _i64, _p, _i, _i, _p, _p, _p]
+    L.or_gemm_fp8.argtypes = [_p, _p, _i64, _i64, _i64, _i64, _i64, _p]
+    L.or_dequant_f64.argtypes = [_p, _i64, _i64, _i64, _p, _i, _p, _i, _p, _p]
     L.or_expf_array.argtypes = [_p, _i64, _p]
     L.or_silu_array.argtypes = [_p, _i64, _p]
     L.or_act_quant.argtypes = [_p, _i64, _i64, _i64, _i, _i, _p, _p, _p, _p, _p]
@@ -188,6 +197,58 @@ def act_quant(A, act, per_token=True, static_qs=None, quantize=True, absmax=None
     lib().or_act_quant(_ptr(A), M, I, W, int(act), int(per_token), _ptr(st), _ptr(Xq), _ptr(qs), _ptr(am),
                        _ptr(H))
     return {"Xq": Xq, "qs": qs, "absmax": am, "H": H}
+
+
+# ---------------------------------------------------------------- f3
+def e4m3_round(x):
+    return np.float32(lib().or_e4m3_round(float(x)))
+
+
+def e4m3_bits(v):
+    return int(lib().or_e4m3_bits(float(v)))
+
+
+def e4m3_value(b):
+    return float(lib().or_e4m3_value(int(b)))
+
+
+def quantize_fp8(X, s=None, s_div=False, per_row=True, static_qs=None):
+    """E4M3 codes (uint8) and scales of fp32(X) (* s or / s per column)."""
+    X = f32(X)
+    M, K = X.shape
+    sv = None if s is None else f32(s)
+    st = None if static_qs is None else np.array([static_qs], np.float32)
+    Q = np.empty((M, K), np.uint8)
+    qs = np.empty(M if per_row else 1, np.float32)
+    lib().or_quantize_fp8(_ptr(X), M, K, K, _ptr(sv), int(s_div), int(per_row), _ptr(st), _ptr(Q), _ptr(qs))
+    return Q, qs
+
+
+def gemm_fp8(A, B, rows=None):
+    """fp64 sums of the decoded E4M3 products (rows: optional row subset)."""
+    A, B = _c(A, np.uint8), _c(B, np.uint8)
+    M, K = A.shape
+    N = B.shape[0]
+    if rows is None:
+        acc = np.empty((M, N), np.float64)
+        lib().or_gemm_fp8(_ptr(A), _ptr(B), M, N, K, 0, M, _ptr(acc))
+        return acc
+    out = np.empty((len(rows), N), np.float64)
+    for n, r in enumerate(rows):
+        lib().or_gemm_fp8(_ptr(A), _ptr(B), M, N, K, int(r), int(r) + 1, _ptr(out[n:n + 1]))
+    return out
+
+
+def dequant_f64(acc, qs_x, qs_w, bias=None, rows=None):
+    acc = _c(acc, np.float64)
+    R, N = acc.shape
+    qx, qw = f32(qs_x), f32(qs_w)
+    if rows is not None:
+        qx = f32(np.asarray(qs_x)[list(rows)]) if qx.size > 1 else qx
+    b = None if bias is None else f32(bias)
+    y = np.empty_like(acc)
+    lib().or_dequant_f64(_ptr(acc), 0, R, N, _ptr(qx), int(qx.size > 1), _ptr(qw), int(qw.size > 1), _ptr(b), _ptr(y))
+    return y
 
 
 # ---------------------------------------------------------------- a4

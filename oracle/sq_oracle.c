@@ -43,9 +43,10 @@
  *   R6 LLM.int8: the outlier test is strict (|x| > thr); min_ratio = 0 means
  *      any one element marks the column; the 16-bit path is exact products
  *      summed in ascending outlier order, added to the dequantised int8 path;
- *   R7 the MLP activation SiLU is evaluated with a fixed fp32 exponential
- *      (below, f1); the fold into the previous linear divides its output
- *      channels by s in fp32 (f2).
+ *   R9 the MLP activation SiLU is evaluated with a fixed fp32 exponential
+ *      (below, f1); R10 the fold into the previous linear divides its output
+ *      channels by s in fp32 (f2); R11 FP8 is OCP E4M3 with the absmax rule
+ *      scaled to its largest value 448 (f3).
  */
 #include "sq_oracle.h"
 
@@ -168,7 +169,7 @@ void or_fold_prev_linear(const double* W, int64_t N, int64_t K, const double* bi
  * up_proj's (fc1's) output channels it arrives already smoothed, and is
  * quantised to int8 like any activation ([SQ-p5] §2.1).
  *
- * The pages name the activation but no way to evaluate it. Reading R7: SiLU,
+ * The pages name the activation but no way to evaluate it. Reading R9: SiLU,
  * silu(g) = g / (1 + exp(-g)), with exp evaluated by a fixed sequence of fp32
  * operations (Cody-Waite reduction x = n ln2 + r with ln 2 in two parts, and
  * the Taylor polynomial of exp(r) to degree 7 by Horner's rule), the same
@@ -236,6 +237,118 @@ void or_act_quant(const float* A, int64_t M, int64_t I, int64_t ld, int act, int
         for (int64_t j = 0; j < I; ++j) Xq[i * I + j] = q_clip(h[j] * qs);
     }
     free(h);
+}
+
+/* ------------------------------------------------------------------ f3
+ * The same W8A8 path on FP8 units   [SQ-p3] 技術原理與特性 (the smoothed
+ * model can run on INT8 or FP8 compute units). The pages give no FP8
+ * details. Reading R11: the format is OCP FP8 E4M3 (1 sign bit, 4 exponent
+ * bits with bias 7, 3 mantissa bits; largest finite value 448, subnormals
+ * spaced 2^-9, no infinities); the absmax rule of [SQ-p5] §2.1 keeps its form
+ * with the format's largest value: qs = 448 / max(m, 1e-8); q = the E4M3
+ * value nearest to fl32(v * qs), ties to the even mantissa, magnitudes past
+ * 448 saturated to 448; the GEMM accumulates the exact products; the
+ * dequantisation divides by qs_x * qs_w as for int8.  Pinned by: every one of
+ * the 254 finite codes decodes and re-encodes to itself; midpoints between
+ * neighbours go to the even code; torch's float8_e4m3fn conversion agrees
+ * inside the finite range; the GEMM by brute force. */
+float or_e4m3_round(float x) {
+    const double a = fabs((double)x);
+    if (a >= 448.0) return x < 0 ? -448.0f : 448.0f;
+    if (a == 0.0) return x;
+    int e;
+    frexp(a, &e); /* a in [2^(e-1), 2^e) */
+    int ex = e - 1;
+    if (ex < -6) ex = -6; /* below the smallest normal: the spacing stays 2^-9 */
+    const double q = ldexp(1.0, ex - 3);
+    double v = nearbyint(a / q) * q; /* a / q is exact; ties to even */
+    if (v > 448.0) v = 448.0;
+    return (float)(x < 0 ? -v : v);
+}
+
+/* bits of an E4M3 value (already representable) */
+uint8_t or_e4m3_bits(float v) {
+    uint8_t sign = v < 0 ? 0x80 : 0;
+    double a = fabs((double)v);
+    if (a == 0.0) return sign;
+    int e;
+    frexp(a, &e);
+    int ex = e - 1;
+    if (ex < -6) return (uint8_t)(sign | (int)(a / ldexp(1.0, -9))); /* subnormal: E = 0 */
+    const int m = (int)((a / ldexp(1.0, ex) - 1.0) * 8.0);
+    return (uint8_t)(sign | ((ex + 7) << 3) | m);
+}
+
+double or_e4m3_value(uint8_t b) {
+    const int E = (b >> 3) & 15, m = b & 7;
+    const double mag = E == 0 ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, E - 7);
+    return (b & 0x80) ? -mag : mag;
+}
+
+static float scale_fp8(float m) {
+    float d = m > 1e-8f ? m : 1e-8f;
+    return 448.0f / d;
+}
+
+/* FP8 quantisation of rows: v = fp32(X) (optionally * s_k or / s_k as in
+ * the int8 weight / activation paths), then per row or one static scale. */
+void or_quantize_fp8(const float* X, int64_t M, int64_t K, int64_t ld, const float* s, int s_div,
+                     int per_row, const float* static_qs, uint8_t* Q, float* qs) {
+    float* v = (float*)malloc(sizeof(float) * (size_t)(K > 0 ? K : 1));
+    float gmax = 0.0f;
+    if (!per_row && !static_qs) {
+        for (int64_t i = 0; i < M; ++i)
+            for (int64_t j = 0; j < K; ++j) {
+                float x = X[i * ld + j];
+                if (s) x = s_div ? x / s[j] : x * s[j];
+                if (absf(x) > gmax) gmax = absf(x);
+            }
+    }
+    for (int64_t i = 0; i < M; ++i) {
+        float m = 0.0f;
+        for (int64_t j = 0; j < K; ++j) {
+            float x = X[i * ld + j];
+            if (s) x = s_div ? x / s[j] : x * s[j];
+            v[j] = x;
+            if (absf(x) > m) m = absf(x);
+        }
+        float q;
+        if (per_row) {
+            q = scale_fp8(m);
+            qs[i] = q;
+        } else {
+            q = static_qs ? *static_qs : scale_fp8(gmax);
+            qs[0] = q;
+        }
+        for (int64_t j = 0; j < K; ++j) Q[i * K + j] = or_e4m3_bits(or_e4m3_round(v[j] * q));
+    }
+    free(v);
+}
+
+/* acc[i - r0, j] = sum_k A[i,k] * B[j,k] of E4M3 codes, in fp64 (each product
+ * is exact; the sum is exact to fp64 rounding). */
+void or_gemm_fp8(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t K, int64_t r0, int64_t r1,
+                 double* acc) {
+    (void)M;
+    for (int64_t i = r0; i < r1; ++i)
+        for (int64_t j = 0; j < N; ++j) {
+            double t = 0.0;
+            for (int64_t k = 0; k < K; ++k) t += or_e4m3_value(A[i * K + k]) * or_e4m3_value(B[j * K + k]);
+            acc[(i - r0) * N + j] = t;
+        }
+}
+
+/* y = acc / (qs_x[i or 0] * qs_w[j or 0]) (+ bias_j) in fp64 for an fp64
+ * accumulator (the FP8 GEMM's exact sums). */
+void or_dequant_f64(const double* acc, int64_t r0, int64_t r1, int64_t N, const float* qs_x, int x_per_token,
+                    const float* qs_w, int w_per_channel, const float* bias, double* y) {
+    for (int64_t i = r0; i < r1; ++i)
+        for (int64_t j = 0; j < N; ++j) {
+            const double d = (double)qs_x[x_per_token ? i : 0] * (double)qs_w[w_per_channel ? j : 0];
+            double v = acc[(i - r0) * N + j] / d;
+            if (bias) v += (double)bias[j];
+            y[(i - r0) * N + j] = v;
+        }
 }
 
 /* ------------------------------------------------------------------ a4

@@ -45,6 +45,15 @@ void or_fold_weight(const double* W, int64_t N, int64_t K, const double* s,
  * switch as or_fold_weight. */
 void or_fold_prev_linear(const double* W, int64_t N, int64_t K, const double* bias, const double* s,
                          int round_f32, double* Wp, double* bias_out);
+float or_e4m3_round(float x);
+uint8_t or_e4m3_bits(float v);
+double or_e4m3_value(uint8_t b);
+void or_quantize_fp8(const float* X, int64_t M, int64_t K, int64_t ld, const float* s, int s_div,
+                     int per_row, const float* static_qs, uint8_t* Q, float* qs);
+void or_gemm_fp8(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t K, int64_t r0, int64_t r1,
+                 double* acc);
+void or_dequant_f64(const double* acc, int64_t r0, int64_t r1, int64_t N, const float* qs_x, int x_per_token,
+                    const float* qs_w, int w_per_channel, const float* bias, double* y);
 float or_expf(float x);
 float or_silu(float g);
 void or_expf_array(const float* x, int64_t n, float* out);

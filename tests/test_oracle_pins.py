@@ -555,3 +555,64 @@ def test_fold_prev_linear_fp32_is_one_division(orc):
     Wp, bp = orc.fold_prev_linear(W, s, b)
     assert np.array_equal(Wp, W / s[:, None])
     assert np.array_equal(bp, b / s)
+
+
+# ---------------------------------------------------------------- f3
+def test_e4m3_codes_round_trip(orc):
+    """Every finite E4M3 code decodes to a value that rounds and re-encodes to
+    the same code; 0x7F / 0xFF (NaN) are the only codes left out; the largest
+    finite value is 448 and the smallest subnormal 2^-9."""
+    vals = {}
+    for b in range(256):
+        if (b & 0x7F) == 0x7F:
+            continue
+        v = orc.e4m3_value(b)
+        assert orc.e4m3_bits(orc.e4m3_round(np.float32(v))) == b or v == 0.0
+        vals[b] = v
+    assert max(vals.values()) == 448.0 and min(v for v in vals.values() if v > 0) == 2.0 ** -9
+    assert len(set(vals.values())) == 253  # +0 and -0 compare equal
+
+
+def test_e4m3_rounding_ties_and_saturation(orc):
+    """Midpoints between neighbouring values go to the even code; magnitudes
+    past 448 saturate; the conversion agrees with torch's float8_e4m3fn inside
+    the finite range."""
+    pos = sorted({orc.e4m3_value(b) for b in range(127)})
+    for lo, hi in zip(pos[:-1], pos[1:]):
+        mid = np.float32((lo + hi) / 2)
+        got = orc.e4m3_round(mid)
+        lo_even = orc.e4m3_bits(np.float32(lo)) % 2 == 0
+        assert got == (lo if lo_even else hi), (lo, hi, got)
+        assert orc.e4m3_round(-mid) == -got
+    for big in (448.0, 463.9, 464.0, 500.0, 1e30):
+        assert orc.e4m3_round(np.float32(big)) == 448.0 and orc.e4m3_round(np.float32(-big)) == -448.0
+    rng = np.random.default_rng(40)
+    x = (rng.normal(size=20000) * 60).astype(np.float32)
+    x = x[np.abs(x) < 440]
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).to(torch.float32).numpy()
+    got = np.array([orc.e4m3_round(v) for v in x], np.float32)
+    assert np.array_equal(got, ref)
+
+
+def test_fp8_quant_and_gemm_bruteforce(orc):
+    """Row scales 448 / max|v|, codes of v * qs, and the exact GEMM of the
+    decoded codes, against plain Python on a tiny case."""
+    rng = np.random.default_rng(41)
+    X = (rng.normal(size=(3, 16)) * 5).astype(np.float32)
+    W = (rng.normal(size=(4, 16)) * 0.1).astype(np.float32)
+    Xq, qx = orc.quantize_fp8(X, per_row=True)
+    Wq, qw = orc.quantize_fp8(W, per_row=True)
+    for i in range(3):
+        m = max(abs(float(v)) for v in X[i])
+        assert qx[i] == np.float32(448.0) / np.float32(m)
+        for j in range(16):
+            assert orc.e4m3_value(Xq[i, j]) == orc.e4m3_round(np.float32(X[i, j]) * qx[i])
+    acc = orc.gemm_fp8(Xq, Wq)
+    for i in range(3):
+        for j in range(4):
+            t = sum(orc.e4m3_value(Xq[i, k]) * orc.e4m3_value(Wq[j, k]) for k in range(16))
+            assert acc[i, j] == t
+    # the dequantised product approximates X W^T to the FP8 quantisation error
+    y = acc / (qx.astype(np.float64)[:, None] * qw.astype(np.float64)[None, :])
+    ref = X.astype(np.float64) @ W.astype(np.float64).T
+    assert np.max(np.abs(y - ref)) / np.max(np.abs(ref)) < 0.1
