@@ -266,9 +266,10 @@ float or_e4m3_round(float x) {
     return (float)(x < 0 ? -v : v);
 }
 
-/* bits of an E4M3 value (already representable) */
+/* bits of an E4M3 value (already representable); the sign bit is kept for a
+ * zero too: a negative value that rounds to zero is -0 (0x80) */
 uint8_t or_e4m3_bits(float v) {
-    uint8_t sign = v < 0 ? 0x80 : 0;
+    uint8_t sign = signbit(v) ? 0x80 : 0;
     double a = fabs((double)v);
     if (a == 0.0) return sign;
     int e;

@@ -592,6 +592,13 @@ def test_e4m3_rounding_ties_and_saturation(orc):
     ref = torch.from_numpy(x).to(torch.float8_e4m3fn).to(torch.float32).numpy()
     got = np.array([orc.e4m3_round(v) for v in x], np.float32)
     assert np.array_equal(got, ref)
+    # codes, over the whole finite range on a log scale, down past the
+    # smallest subnormal: negative values that round to zero keep the sign
+    mag = np.exp(rng.uniform(np.log(1e-5), np.log(440), 50000))
+    x = (mag * rng.choice([-1.0, 1.0], mag.size)).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([orc.e4m3_bits(orc.e4m3_round(v)) for v in x], np.uint8)
+    assert np.array_equal(got, ref)
 
 
 def test_fp8_quant_and_gemm_bruteforce(orc):
