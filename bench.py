@@ -4,14 +4,16 @@ One step = one pass of every hot-path row over one batch of synthetic input
 shaped like a Qwen3-0.6B decoder layer at 2048 tokens (hidden 1024; q/k/v
 fused 1024->4096, o 2048->1024, gate/up fused 1024->6144, down 3072->1024;
 6 activation channels x20..x100):
-  a5 norm pass producing the linear input (RMSNorm, original gamma)     x2
-  a1 calibration absmax of that input                                   x2
-  a2 weight absmax over the fused consumers                             x2
-  a3 smoothing factors, gamma' = gamma / s                              x2
-  a4 weight fold + int8 quantisation (per output channel)               x4
-  a5 fused RMSNorm + smoothing + per-token int8                         x2
-  a6 int8 GEMM + dequant epilogue to bf16                               x4
-  a7-a9 LLM.int8 decomposition of the q/k/v projection (bf16)           x1
+  norm pass producing the linear input (RMSNorm, original gamma)        x2
+  calibration absmax of that input                                      x2
+  weight absmax over the fused consumers                                x2
+  smoothing factors, gamma' = gamma / s                                 x2
+  weight fold + int8 quantisation (per output channel)                  x5
+  fused RMSNorm + smoothing + per-token int8                            x2
+  int8 GEMM + dequant epilogue to bf16                                  x4
+  1/s of down_proj's input folded into up_proj's output channels        x1
+  SwiGLU of the gate/up output + per-token int8 (down_proj's input)     x1
+  LLM.int8 decomposition of the q/k/v projection (bf16)                 x1
 The independent chains of the step (the attention-side and MLP-side
 calibration/quantisation chains, the weight-side work, the o/down GEMMs and the
 LLM.int8 call) run on their own streams inside the step, joined at its end.
@@ -41,12 +43,13 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 M_TOKENS, HIDDEN = 2048, 1024
-WORKLOAD = "qwen3-0.6b-shaped decoder layer linear stack, 2048 tokens, hidden 1024, bf16 in/out, int8 GEMMs"
+WORKLOAD = ("qwen3-0.6b-shaped decoder layer linear stack, 2048 tokens, hidden 1024, bf16 in/out, int8 GEMMs; "
+            "down_proj input from the SwiGLU of the gate/up output")
 METRIC = "W8A8 GEMM TOPS & tokens/s at 1 B200; % of INT8 TC peak / HBM GB/s"
 # GEMM (M, N, K) of one step: qkv, o, gate/up, down, LLM.int8 q/k/v
 GEMMS = [(2048, 4096, 1024), (2048, 1024, 2048), (2048, 6144, 1024), (2048, 1024, 3072), (2048, 4096, 1024)]
 # our kernels per call of each entry point used in the step
-LAUNCHES_PER_STEP = (2 * 1 + 2 * 1 + 2 * 1 + 2 * 2 + 4 * 1 + 2 * 1 + 4 * 1 + 5)
+LAUNCHES_PER_STEP = (2 * 1 + 2 * 1 + 2 * 1 + 2 * 2 + 5 * 1 + 1 + 2 * 1 + 4 * 1 + 1 + 5)
 
 
 def peaks():
@@ -152,10 +155,47 @@ class Layer:
         self.llm = sq.llmint8_weight_state(self.W["qkv"])
         self.idx = e(K, dt=torch.int32)
         self.nidx = e(1, dt=torch.int32)
+        # down_proj's input: SwiGLU of the gate/up output, smoothed by s_down
+        # folded into up_proj's output channels
+        I = self.W["down"].shape[1]
+        self.I = I
+        self.W_gate, self.W_up = self.W["gateup"][:I], self.W["gateup"][I:]
+        self.W_up_f = e(I, K)
+        self.Xq_down = e(M, I, dt=torch.int8)
+        self.qx_down = e(M)
+        self.s_down = self.calibrate_down()
         self.gemm_events = None
         self.streams = [torch.cuda.Stream(device=dev) for _ in range(5)]
         self.events = {n: torch.cuda.Event() for n in ("wmax_attn", "wmax_mlp", "V_attn", "V_mlp", "s_attn", "s_mlp",
-                                                      "wq_qkv", "wq_gateup")}
+                                                      "wq_qkv", "wq_gateup", "wq_down")}
+
+    def calibrate_down(self):
+        """s for down_proj's input, from one pass of the MLP input through the
+        unsmoothed int8 gate/up projection: running max of |silu(gate) * up|
+        (calibration mode of sq_act_quant) against down_proj's weight maxima. Done once, at
+        set-up; the step then folds it (1/s into up_proj's rows, s into
+        down_proj's columns)."""
+        sq, d, torch = self.sq, self.d, self.torch
+        M, K, I = M_TOKENS, HIDDEN, self.I
+        dev = self.h["mlp"].device
+        e = lambda *s_, dt=torch.float32: torch.empty(s_, dtype=dt, device=dev)  # noqa: E731
+        V = e(M, K, dt=torch.bfloat16)
+        sq.sq_norm_smooth_quant(self.d["h_calib"].to(dev), sq.SQ_RMSNORM, self.gamma["mlp"], None, d["eps"], True, None,
+                                None, None, None, V)
+        Xq, qx = e(M, K, dt=torch.int8), e(M)
+        sq.sq_quantize_act(V, None, True, None, Xq, qx)
+        Wq, qw = e(2 * I, K, dt=torch.int8), e(2 * I)
+        sq.sq_quantize_weight(self.W["gateup"], None, True, Wq, qw)
+        Y = e(M, 2 * I, dt=torch.bfloat16)
+        sq.sq_gemm_w8a8(Xq, Wq, qx, qw, None, Y, sq.workspace(sq.SQ_OP_GEMM, M, 2 * I, K, device=dev))
+        hmax = torch.zeros(I, device=dev)
+        sq.sq_act_quant(Y, sq.SQ_ACT_SWIGLU, True, None, None, None, hmax)
+        wmax = torch.zeros(I, device=dev)
+        sq.sq_weight_absmax(self.W["down"], wmax)
+        s = e(I)
+        sq.sq_smooth_scales(hmax, wmax, d["alpha"], s)
+        torch.cuda.synchronize()
+        return s
 
     def step(self, gemm_ev=None):
         """One pass of every row. Independent chains run on their own streams
@@ -163,6 +203,7 @@ class Layer:
         latency-bound small kernels of one chain overlap the others."""
         sq, d, torch = self.sq, self.d, self.torch
         eps = d["eps"]
+        I = self.I
         main = torch.cuda.current_stream()
         sA, sB, sC, sD, sE = self.streams
         ev = self.events
@@ -170,7 +211,7 @@ class Layer:
         for s_ in self.streams:
             s_.wait_stream(main)
 
-        def gemm(i, w, xq, qx):                                                  # a6
+        def gemm(i, w, xq, qx):
             if gemm_ev is not None:
                 gemm_ev[i][0].record()
             sq.sq_gemm_w8a8(xq, self.Wq[w], qx, self.qw[w], None, self.Y[w], self.ws_gemm[w])
@@ -178,38 +219,49 @@ class Layer:
                 gemm_ev[i][1].record()
 
         with torch.cuda.stream(sC):
-            sq.sq_weight_absmax(self.W["qkv"], self.wmax["attn"])                  # a2
+            sq.sq_weight_absmax(self.W["qkv"], self.wmax["attn"])
             ev["wmax_attn"].record()
             sq.sq_weight_absmax(self.W["gateup"], self.wmax["mlp"])
             ev["wmax_mlp"].record()
-            sq.sq_quantize_weight(self.W["o"], None, True, self.Wq["o"], self.qw["o"])  # a4
+            sq.sq_quantize_weight(self.W["o"], None, True, self.Wq["o"], self.qw["o"])
             gemm(1, "o", *self.act_in["o"])
-            sq.sq_quantize_weight(self.W["down"], None, True, self.Wq["down"], self.qw["down"])
-            gemm(3, "down", *self.act_in["down"])
+            # fold into the previous linear: 1/s_down into up_proj's output channels; down_proj takes s_down
+            sq.sq_fold_prev_linear(self.W_up, self.s_down, self.W_up_f)
+            sq.sq_quantize_weight(self.W["down"], self.s_down, True, self.Wq["down"], self.qw["down"])
+            ev["wq_down"].record()
         chains = (("attn", "qkv", sA, 0), ("mlp", "gateup", sB, 2))
         for k, w, s_, i in chains:
             with torch.cuda.stream(s_):
-                # a5 (calibration pass) -> linear input; a1 on it
+                # norm (calibration pass) -> linear input; its column absmax
                 sq.sq_norm_smooth_quant(self.h[k], sq.SQ_RMSNORM, self.gamma[k], None, eps, True, None, None,
                                         None, None, self.V[k])
                 ev["V_" + k].record()
                 sq.sq_calib_absmax(self.V[k], self.xmax[k])
                 s_.wait_event(ev["wmax_" + k])
-                sq.sq_smooth_scales(self.xmax[k], self.wmax[k], d["alpha"], self.s[k])  # a3
+                sq.sq_smooth_scales(self.xmax[k], self.wmax[k], d["alpha"], self.s[k])
                 ev["s_" + k].record()
                 sq.sq_fold_norm(self.gamma[k], None, self.s[k], self.gp[k])
-                sq.sq_norm_smooth_quant(self.h[k], sq.SQ_RMSNORM, self.gp[k], None, eps, True, None,  # a5
+                sq.sq_norm_smooth_quant(self.h[k], sq.SQ_RMSNORM, self.gp[k], None, eps, True, None,
                                         self.Xq[k], self.qx[k], None, None)
-        with torch.cuda.stream(sD):
-            for k, w, _, _ in chains:
-                sD.wait_event(ev["s_" + k])
-                sq.sq_quantize_weight(self.W[w], self.s[k], True, self.Wq[w], self.qw[w])  # a4
-                ev["wq_" + w].record()
+        with torch.cuda.stream(sD):  # weight quantisation once s is known
+            sD.wait_event(ev["s_attn"])
+            sq.sq_quantize_weight(self.W["qkv"], self.s["attn"], True, self.Wq["qkv"], self.qw["qkv"])
+            ev["wq_qkv"].record()
+            sD.wait_event(ev["s_mlp"])
+            sD.wait_stream(sC)  # the folded up_proj rows
+            sq.sq_quantize_weight(self.W_gate, self.s["mlp"], True, self.Wq["gateup"][:I], self.qw["gateup"][:I])
+            sq.sq_quantize_weight(self.W_up_f, self.s["mlp"], True, self.Wq["gateup"][I:], self.qw["gateup"][I:])
+            ev["wq_gateup"].record()
         for k, w, s_, i in chains:
             with torch.cuda.stream(s_):
                 s_.wait_event(ev["wq_" + w])
                 gemm(i, w, self.Xq[k], self.qx[k])
-        with torch.cuda.stream(sE):                                                # a7-a9
+        with torch.cuda.stream(sB):
+            # down_proj's input from the SwiGLU of the gate/up output
+            sq.sq_act_quant(self.Y["gateup"], sq.SQ_ACT_SWIGLU, True, None, self.Xq_down, self.qx_down)
+            sB.wait_event(ev["wq_down"])
+            gemm(3, "down", self.Xq_down, self.qx_down)
+        with torch.cuda.stream(sE):  # LLM.int8 decomposition
             sE.wait_event(ev["V_attn"])
             sq.sq_llmint8_matmul(self.V["attn"], self.llm, 6.0, 0.0, self.Y["llm"], self.idx, self.nidx, self.ws)
         for s_ in self.streams:
@@ -316,7 +368,9 @@ def run_ours(args, rank, world, dev):
 def cpu_step_sample(rows):
     """The oracle, as it stands, on the same step for `rows` tokens of the
     workload (weights in full). Returns (seconds of weight-side work,
-    seconds of per-token work for `rows` tokens)."""
+    seconds of per-token work for `rows` tokens). The smoothing factors of
+    down_proj's input come from an untimed calibration pass over the sample,
+    as the GPU step takes them from its set-up."""
     import torch
 
     import oracle
@@ -328,6 +382,21 @@ def cpu_step_sample(rows):
     h = {"attn": d["h_attn"][sl], "mlp": d["h_mlp"][sl]}
     gamma = {"attn": d["gamma_attn"].numpy(), "mlp": d["gamma_mlp"].numpy()}
     W = {k: oracle.f32(v) for k, v in d["W"].items()}
+    I = W["down"].shape[1]
+
+    def bf16(y):
+        return torch.from_numpy(oracle.round_bf16_bits(y).view(np.int16)).view(torch.bfloat16).float().numpy()
+
+    # set-up (untimed): s of down_proj's input
+    Vc = oracle.norm_smooth_quant(d["h_calib"][sl], oracle.RMSNORM, gamma["mlp"], None, d["eps"], quantize=False,
+                                  want_v=True)["V"]
+    Vc16 = torch.from_numpy(Vc).to(torch.bfloat16).float().numpy()
+    Xc, qc = oracle.quantize_act(Vc16, None, per_token=True)
+    Wc, qwc = oracle.quantize_weight(W["gateup"], True)
+    hmax = oracle.act_quant(bf16(oracle.dequant(oracle.gemm_i8(Xc, Wc), qc, qwc)), oracle.SWIGLU, quantize=False,
+                            absmax=np.zeros(I, np.float32))["absmax"]
+    s_down = oracle.smooth_scales(hmax, oracle.col_absmax(W["down"]), d["alpha"])
+
     t_rows = 0.0
     t_w = 0.0
     t0 = time.perf_counter()
@@ -343,9 +412,13 @@ def cpu_step_sample(rows):
         s[k] = oracle.smooth_scales(xmax[k], wmax, d["alpha"])
         gp[k], _ = oracle.fold_norm(gamma[k], None, s[k])
     Wq, qw = {}, {}
-    for w, k in (("qkv", "attn"), ("gateup", "mlp"), ("o", None), ("down", None)):
-        Wp = oracle.fold_weight(W[w], s[k]) if k else W[w]
-        Wq[w], qw[w] = oracle.quantize_weight(Wp, True)
+    Wq["qkv"], qw["qkv"] = oracle.quantize_weight(oracle.fold_weight(W["qkv"], s["attn"]), True)
+    up_f, _ = oracle.fold_prev_linear(W["gateup"][I:], s_down)
+    gate_q, gate_s = oracle.quantize_weight(oracle.fold_weight(W["gateup"][:I], s["mlp"]), True)
+    up_q, up_s = oracle.quantize_weight(oracle.fold_weight(up_f, s["mlp"]), True)
+    Wq["gateup"], qw["gateup"] = np.concatenate([gate_q, up_q]), np.concatenate([gate_s, up_s])
+    Wq["o"], qw["o"] = oracle.quantize_weight(W["o"], True)
+    Wq["down"], qw["down"] = oracle.quantize_weight(oracle.fold_weight(W["down"], s_down), True)
     t_w += time.perf_counter() - t0
     t0 = time.perf_counter()
     Xq, qx = {}, {}
@@ -353,12 +426,12 @@ def cpu_step_sample(rows):
         r = oracle.norm_smooth_quant(h[k], oracle.RMSNORM, gp[k], None, d["eps"], True)
         Xq[k], qx[k] = r["Xq"], r["qs"]
     xo, so = d["o_in"]
-    xd, sd = d["down_in"]
-    plan = [("qkv", Xq["attn"], qx["attn"]), ("o", xo[sl].numpy(), so[sl].numpy()),
-            ("gateup", Xq["mlp"], qx["mlp"]), ("down", xd[sl].numpy(), sd[sl].numpy())]
-    for w, xq, q in plan:
-        y = oracle.dequant(oracle.gemm_i8(xq, Wq[w]), q, qw[w])
-        oracle.round_bf16_bits(y)
+    Y = {}
+    for w, xq, q in (("qkv", Xq["attn"], qx["attn"]), ("o", xo[sl].numpy(), so[sl].numpy()),
+                     ("gateup", Xq["mlp"], qx["mlp"])):
+        Y[w] = bf16(oracle.dequant(oracle.gemm_i8(xq, Wq[w]), q, qw[w]))
+    a = oracle.act_quant(Y["gateup"], oracle.SWIGLU)
+    bf16(oracle.dequant(oracle.gemm_i8(a["Xq"], Wq["down"]), a["qs"], qw["down"]))
     t_rows += time.perf_counter() - t0
     # LLM.int8 of the q/k/v projection: outlier set over the sample rows,
     # row quantisation, weight requantisation, GEMM + outlier term
@@ -412,7 +485,7 @@ def run_reference(args, rank, world):
 # ------------------------------------------------------------------ single kernels
 def run_kernel(args):
     """Time one entry point alone on one shape:
-    gemm M,N,K | norm M,K | absmax M,K | quant_weight N,K | llmint8 M,K,N.
+    gemm M,N,K | gemm_fp8 M,N,K | norm M,K | absmax M,K | act M,I | quant_weight N,K | llmint8 M,K,N.
     --sets 1: every launch after an L2 flush, each launch timed on its own.
     --sets S > 1: S distinct input/output sets, launches cycling through them
     back to back (one flush before the run); the time per launch is the run's
@@ -442,8 +515,22 @@ def run_kernel(args):
             qx = torch.rand(M, generator=g, device=dev) + 1
             qw = torch.rand(N, generator=g, device=dev) + 100
             Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-            ws = sq.workspace(sq.SQ_OP_GEMM, M, N, K, device=dev)
+            # a 256-byte workspace has no room for a stream-K split: whole tiles only
+            ws = (torch.zeros(256, dtype=torch.uint8, device=dev) if args.whole_tiles
+                  else sq.workspace(sq.SQ_OP_GEMM, M, N, K, device=dev))
             return lambda: sq.sq_gemm_w8a8(Xq, Wq, qx, qw, None, Y, ws)
+        if args.kernel == "gemm_fp8":
+            M, N, K = shape
+            # random finite E4M3 codes (0x7F / 0xFF, the NaN codes, moved to 0x7E / 0xFE)
+            Xq = torch.randint(0, 256, (M, K), generator=g, device=dev, dtype=torch.int32)
+            Wq = torch.randint(0, 256, (N, K), generator=g, device=dev, dtype=torch.int32)
+            Xq = torch.where((Xq & 0x7F) == 0x7F, Xq - 1, Xq).to(torch.uint8)
+            Wq = torch.where((Wq & 0x7F) == 0x7F, Wq - 1, Wq).to(torch.uint8)
+            qx = torch.rand(M, generator=g, device=dev) + 1
+            qw = torch.rand(N, generator=g, device=dev) + 100
+            Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            ws = sq.workspace(sq.SQ_OP_GEMM, M, N, K, device=dev)
+            return lambda: sq.sq_gemm_fp8(Xq, Wq, qx, qw, None, Y, ws)
         if args.kernel == "norm":
             M, K = shape
             dt16 = torch.float16 if args.dtype == "fp16" else torch.bfloat16
@@ -459,6 +546,14 @@ def run_kernel(args):
             dtx = {"fp16": torch.float16, "bf16": torch.bfloat16, "fp32": torch.float32}[args.dtype]
             X = torch.randn((M, K), generator=g, device=dev).to(dtx)
             return lambda: sq.sq_calib_absmax(X, xmax)
+        if args.kernel == "act":
+            M, I = shape
+            dt16 = torch.float16 if args.dtype == "fp16" else torch.bfloat16
+            act = sq.SQ_ACT_RELU if args.act == "relu" else sq.SQ_ACT_SWIGLU
+            A = (torch.randn((M, 2 * I if act == sq.SQ_ACT_SWIGLU else I), generator=g, device=dev) * 2).to(dt16)
+            Xq = torch.empty((M, I), dtype=torch.int8, device=dev)
+            qs = torch.empty(M, device=dev)
+            return lambda: sq.sq_act_quant(A, act, True, None, Xq, qs)
         if args.kernel == "quant_weight":
             N, K = shape
             dtx = {"fp16": torch.float16, "bf16": torch.bfloat16, "fp32": torch.float32}[args.dtype]
@@ -480,9 +575,11 @@ def run_kernel(args):
             return lambda: sq.sq_llmint8_matmul(d["X"], st, 6.0, 0.0, Y, idx, n, ws)
         raise SystemExit(f"unknown kernel {args.kernel}")
 
-    if args.kernel == "gemm":
+    if args.kernel in ("gemm", "gemm_fp8"):
         M, N, K = shape
+        # dense int8 and fp8 peaks are both twice the bf16 one (4.5 vs 2.25 PFLOP/s nominal)
         work, unit, peak = 2.0 * M * N * K / 1e12, "TOPS", 2.0 * pk["bf16_tflops"]
+        out["whole_tiles"] = bool(args.whole_tiles)
     elif args.kernel == "norm":
         M, K = shape
         work, unit, peak = (3.0 * M * K + 4 * M) / 1e9, "GB/s", pk["hbm_gbs"]
@@ -492,6 +589,10 @@ def run_kernel(args):
         eb = 4 if args.dtype == "fp32" else 2
         work, unit, peak = eb * M * K / 1e9, "GB/s", pk["hbm_gbs"]
         xmax = torch.zeros(K, device=dev)
+    elif args.kernel == "act":
+        M, I = shape
+        work, unit, peak = ((2 if args.act == "relu" else 4) * M * I + M * I + 4 * M) / 1e9, "GB/s", pk["hbm_gbs"]
+        out["act"] = args.act
     elif args.kernel == "quant_weight":
         N, K = shape
         eb = 4 if args.dtype == "fp32" else 2
@@ -551,6 +652,8 @@ def main():
     ap.add_argument("--shape", default="4096,36864,12288")
     ap.add_argument("--dtype", default="bf16", help="input dtype of --kernel absmax|quant_weight|norm")
     ap.add_argument("--norm", default="rms", help="--kernel norm: rms|ln")
+    ap.add_argument("--act", default="swiglu", help="--kernel act: swiglu|relu")
+    ap.add_argument("--whole-tiles", action="store_true", help="--kernel gemm: a workspace without stream-K scratch")
     ap.add_argument("--sets", type=int, default=1, help="--kernel: input sets cycled back to back (1: flush each)")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)

@@ -66,6 +66,9 @@ typedef enum { SQ_F32 = 0, SQ_F16 = 1, SQ_BF16 = 2, SQ_I32 = 3, SQ_I8 = 4 } sq_d
 
 typedef enum { SQ_LAYERNORM = 0, SQ_RMSNORM = 1 } sq_norm_t;
 
+/* MLP activation feeding down_proj / FC2 (sq_act_quant). */
+typedef enum { SQ_ACT_SWIGLU = 0, SQ_ACT_RELU = 1 } sq_act_t;
+
 typedef enum {
     SQ_OP_GEMM = 0,           /* sq_gemm_w8a8                               */
     SQ_OP_QUANT_ACT = 1,      /* sq_quantize_act (per-tensor dynamic)       */
@@ -83,14 +86,25 @@ SQ_API const char* sq_last_error_string(void);
 
 /* Synchronises `stream`, reads the status word that bounded device waits
  * write into `workspace`, clears it and returns SQ_OK or SQ_ERR_TIMEOUT.
- * Applies to workspaces passed to sq_gemm_w8a8 and sq_llmint8_matmul. */
+ * Applies to workspaces passed to sq_gemm_w8a8, sq_gemm_fp8, sq_bmm_w8a8,
+ * sq_llmint8_matmul and sq_selftest_wait_timeout. */
 SQ_API sq_status_t sq_workspace_status(void* workspace, sq_stream_t stream);
+
+/* Check of the failure path of the bounded device waits: launches one block
+ * that waits on an mbarrier nothing completes, with the bounded wait every
+ * waiting kernel of the library uses, but a timeout of timeout_ns (at most
+ * 2 s) instead of 2 s. The block gives up, records the timeout code in the
+ * workspace status word and returns: sq_workspace_status then returns
+ * SQ_ERR_TIMEOUT and the context stays usable. Nothing faults, traps or
+ * hangs. The pages have no counterpart; it exists to test the failure path. */
+SQ_API sq_status_t sq_selftest_wait_timeout(void* workspace, size_t ws_bytes, uint64_t timeout_ns,
+                                            sq_stream_t stream);
 
 /* Library version as an integer (major*10000 + minor*100 + patch). */
 SQ_API int sq_version(void);
 
 /* --------------------------------------------------------------------------
- * a1 / a2  Calibration absmax                      [SQ-p2] 缩放因子;
+ * Calibration absmax                            [SQ-p2] 缩放因子;
  *          [SQ-p1] §3.2 (act.abs().amax over tokens; weight.abs().amax(dim=0));
  *          [SQ-p4] §3 (max over batch and sequence; max over output dim).
  *
@@ -111,7 +125,7 @@ SQ_API sq_status_t sq_weight_absmax(const void* W, sq_dtype_t dt, int64_t N, int
                              float* wmax_inout, sq_stream_t stream);
 
 /* --------------------------------------------------------------------------
- * a3  Smoothing factors                            [SQ-p2] 缩放因子;
+ * Smoothing factors                                [SQ-p2] 缩放因子;
  *     [SQ-p1] §2.1, §3.2; [SQ-p4] §3.
  *   s[j] = max(1e-5, x^alpha / w^(1-alpha)),  x = max(xmax[j], 1e-5),
  *   w = max(wmax[j], 1e-5), evaluated in fp64 and rounded once to fp32.
@@ -121,22 +135,34 @@ SQ_API sq_status_t sq_weight_absmax(const void* W, sq_dtype_t dt, int64_t N, int
 SQ_API sq_status_t sq_smooth_scales(const float* xmax, const float* wmax, int64_t K, double alpha,
                              float* s_out, sq_stream_t stream);
 
-/* a3 fold  W' = diag(s) W in the pages' notation: input channel k of every
+/* Weight fold  W' = diag(s) W in the pages' notation: input channel k of every
  * output row times s[k]      [SQ-p2] SmoothQuant 的原理; [SQ-p4] §3
  * (weight.mul_(s.view(1,-1))).  W: [N,K] of dt in {F16, BF16, F32};
  * Wp_out: [N,K] fp32 (one fp32 rounding per product). K % 8 == 0. */
 SQ_API sq_status_t sq_fold_weight(const void* W, sq_dtype_t dt, int64_t N, int64_t K, const float* s,
                            float* Wp_out, sq_stream_t stream);
 
-/* a3 fold into the norm  gamma' = gamma / s, beta' = beta / s  (fp32 IEEE
+/* Fold into the norm  gamma' = gamma / s, beta' = beta / s  (fp32 IEEE
  * division)                  [SQ-p2] 融入 LayerNorm.
  * beta / beta_out may both be NULL (RMSNorm). All [K] fp32. In-place
  * (gamma_out == gamma) is allowed. */
 SQ_API sq_status_t sq_fold_norm(const float* gamma, const float* beta, const float* s, int64_t K,
                          float* gamma_out, float* beta_out, sq_stream_t stream);
 
+/* Fold into the previous linear layer    [SQ-p2] 融入前序线性层的权重 and
+ * the table after it: for down_proj the smoothing goes into up_proj's output
+ * channels, for o_proj into v_proj's. Output channel n of the previous layer
+ * is divided by s[n]: Wp[n,k] = fp32(W[n,k]) / s[n], bias_out[n] = bias[n] /
+ * s[n] (fp32 IEEE division). The next layer's input channels then take s
+ * with sq_fold_weight (or sq_quantize_weight with s). W: [N,K] of dt in
+ * {F16, BF16, F32}; Wp_out: [N,K] fp32; s: [N]; bias / bias_out: [N] fp32,
+ * both NULL or both given. K % 8 == 0. With grouped KV heads, one s per
+ * v_proj output channel serves every query head that reads it. */
+SQ_API sq_status_t sq_fold_prev_linear(const void* W, sq_dtype_t dt, int64_t N, int64_t K, const float* bias,
+                                const float* s, float* Wp_out, float* bias_out, sq_stream_t stream);
+
 /* --------------------------------------------------------------------------
- * a4  Weight quantisation (offline)     [SQ-p5] §2.1; [SQ-p2]
+ * Weight quantisation (offline)     [SQ-p5] §2.1; [SQ-p2]
  *     为什么激活不能用逐通道量化 (weight scales per output channel).
  *   W' = fp32(W) * s[k]  (s may be NULL: W' = fp32(W)), then
  *   m = max |W'| over the row (per_channel != 0) or the tensor;
@@ -149,7 +175,7 @@ SQ_API sq_status_t sq_quantize_weight(const void* W, sq_dtype_t dt, int64_t N, i
                                void* workspace, size_t ws_bytes, sq_stream_t stream);
 
 /* --------------------------------------------------------------------------
- * a5'  Activation quantisation without a norm     [SQ-p4] §3 (input / s);
+ * Activation quantisation without a norm     [SQ-p4] §3 (input / s);
  *      [SQ-p1] §3.3; [SQ-p5] §2.1.
  *   v = fp32(X[i,j]) / s[j]  (IEEE division; s may be NULL: v = X),
  *   per_token != 0: qs_x[i] = 127 / max(max_j |v[i,j]|, 1e-8);
@@ -170,15 +196,16 @@ SQ_API sq_status_t sq_scale_from_absmax(const float* absmax, int64_t n, float* q
                                  sq_stream_t stream);
 
 /* --------------------------------------------------------------------------
- * a5  Fused norm + smoothing + int8           [SQ-p2] 融入 LayerNorm;
+ * Fused norm + smoothing + int8           [SQ-p2] 融入 LayerNorm;
  *     [SQ-p4] §4 item 2; [SQ-p5] §2.1.
  *   LayerNorm: mu = S(x)/K, d = x - mu, var = S(d*d)/K, r = 1/sqrt(var+eps),
  *              v = (d*r)*gamma' + beta'  (beta' may be NULL)
  *   RMSNorm:   r = 1/sqrt(S(x*x)/K + eps),  v = (x*r)*gamma'
  *   Every step is one correctly rounded fp32 operation. S() is a sum in a
- *   fixed order: 128 lanes; lane t folds 8-element chunks t, t+128, ... with
+ *   fixed order: 256 lanes; lane t folds 8-element chunks t, t+256, ... with
  *   fma in index order; each 32-lane group combines by the xor butterfly
- *   (16, 8, 4, 2, 1); the four group totals add as (G0+G1)+(G2+G3).
+ *   (16, 8, 4, 2, 1); the eight group totals add as
+ *   ((G0+G1)+(G2+G3))+((G4+G5)+(G6+G7)).
  *   Then, if Xq != NULL: per_token != 0 -> qs_x[i] = 127/max(max_j|v|,1e-8);
  *   per_token == 0 -> qs = *static_qs (required), qs_x[0] = qs;
  *   Xq = clip(rne(v*qs), -127, 127).
@@ -195,7 +222,30 @@ SQ_API sq_status_t sq_norm_smooth_quant(const void* H, sq_dtype_t dt, int64_t M,
                                  sq_stream_t stream);
 
 /* --------------------------------------------------------------------------
- * a6  INT8 GEMM with dequantisation epilogue   [SQ-p5] §2.1 (int32
+ * MLP activation + int8 for the input of down_proj / FC2
+ *     [SQ-p2] 融入前序线性层的权重 (down_proj input = act(gate) * up, its
+ *     smoothing folded into up_proj by sq_fold_prev_linear); [SQ-p5] §2.1.
+ *   SQ_ACT_SWIGLU: A is [M, 2I] (stride lda >= 2I), gate = A[:, :I],
+ *     up = A[:, I:]; h = silu(gate) * up, silu(g) = g / (1 + exp(-g)).
+ *   SQ_ACT_RELU: A is [M, I] (stride lda >= I); h = max(A, 0).
+ *   exp is a fixed sequence of correctly rounded fp32 operations: n =
+ *   rint(x * fp32(log2 e)), r = x - n*LN2_HI - n*LN2_LO (two fma, LN2_HI =
+ *   2839/4096), exp(r) by the degree-7 Taylor polynomial in Horner form with
+ *   fma, times 2^n; exp(x) = +inf above 88 and 0 below -87. The result is
+ *   within 4 ulp of exp and is reproducible bit for bit on any IEEE machine.
+ *   Then, if Xq != NULL: per_token != 0 -> qs_x[i] = 127/max(max_j|h|,1e-8);
+ *   per_token == 0 -> qs = *static_qs (required), qs_x[0] = qs;
+ *   Xq[i,j] = clip(rne(h*qs), -127, 127), Xq [M,I] contiguous.
+ *   Optional: absmax_inout [I] fp32 running max of |h| (calibration; I <=
+ *   57344), H_out [M,I] (stride I) h rounded to dt.
+ *   dt in {F16, BF16}; I % 8 == 0, lda % 8 == 0; A, Xq, H_out 16-byte aligned.
+ * ------------------------------------------------------------------------ */
+SQ_API sq_status_t sq_act_quant(const void* A, sq_dtype_t dt, int64_t M, int64_t I, int64_t lda, sq_act_t act,
+                                int per_token, const float* static_qs, int8_t* Xq, float* qs_x,
+                                float* absmax_inout, void* H_out, sq_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * INT8 GEMM with dequantisation epilogue   [SQ-p5] §2.1 (int32
  *     accumulation, out / (c_x outer c_w)); [SQ-p2] 为什么激活不能用逐通道量化
  *     (Y = diag(dX) Xq Wq diag(dW)).
  *   acc[i,j] = sum_k Xq[i,k] * Wq[j,k]   (exact int32; |acc| <= 127^2 K)
@@ -205,8 +255,15 @@ SQ_API sq_status_t sq_norm_smooth_quant(const void* H, sq_dtype_t dt, int64_t M,
  *   {F32, F16, BF16}. bias: [N] fp32 or NULL.
  *   Xq: [M,K] int8 contiguous; Wq: [N,K] int8 contiguous; Y: [M,N] stride ldy.
  *   K % 16 == 0, K <= 133144 (int32 bound); Xq, Wq 16-byte aligned.
- *   Workspace (SQ_OP_GEMM) holds the status word of the bounded waits; zero
- *   it once before first use.
+ *   Workspace (SQ_OP_GEMM, size from sq_workspace_size for the same M, N, K)
+ *   holds the status word of the bounded waits and, for shapes whose last
+ *   wave of whole tiles would be at most three quarters full, the scratch of
+ *   a stream-K split of that wave (arrival counters and parked int32 partial
+ *   sums). Zero it once before first use; every call that completes leaves
+ *   the status word and the counters at zero again (the parked sums need no
+ *   clearing). After SQ_ERR_TIMEOUT zero it again. A smaller workspace (at
+ *   least 256 bytes) is accepted and runs every tile whole. Calls sharing one
+ *   workspace must not run concurrently.
  * ------------------------------------------------------------------------ */
 SQ_API sq_status_t sq_gemm_w8a8(const int8_t* Xq, const int8_t* Wq, int64_t M, int64_t N, int64_t K,
                          const float* qs_x, int x_per_token, const float* qs_w, int w_per_channel,
@@ -214,11 +271,53 @@ SQ_API sq_status_t sq_gemm_w8a8(const int8_t* Xq, const int8_t* Wq, int64_t M, i
                          void* workspace, size_t ws_bytes, sq_stream_t stream);
 
 /* --------------------------------------------------------------------------
- * a7-a9  LLM.int8() mixed-precision decomposition     [SQ-p5] §2.2, §2.3,
+ * Batched INT8 GEMM for attention     lpnh.cn SmoothQuant practice article
+ *     §2.2 (the QK^T and PV products of attention can be quantised).
+ *   Y[b] = Aq[b] Bq[b]^T dequantised as sq_gemm_w8a8 for b < batch:
+ *   Aq: [batch, M, K] int8, Bq: [batch, N, K] int8 (each contiguous, problems
+ *   back to back); qs_a: [batch, M] (a_per_row) or [batch] scales, qs_b:
+ *   [batch, N] (b_per_row) or [batch]; Y: [batch, M, ldy] of out_dt in {I32,
+ *   F32, F16, BF16}. For QK^T: A = Q, B = K, one scale per (head, token). For
+ *   PV: A = P (per row), B = V^T (V transposed to [d, T], one scale per (head,
+ *   channel): a scale along the summed token axis would not factor out).
+ *   K % 16 == 0. Workspace as sq_gemm_w8a8.
+ * ------------------------------------------------------------------------ */
+SQ_API sq_status_t sq_bmm_w8a8(const int8_t* Aq, const int8_t* Bq, int64_t batch, int64_t M, int64_t N, int64_t K,
+                               const float* qs_a, int a_per_row, const float* qs_b, int b_per_row,
+                               sq_dtype_t out_dt, void* Y, int64_t ldy, void* workspace, size_t ws_bytes,
+                               sq_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * The same W8A8 path on FP8 units      [SQ-p3] 技術原理與特性 (the
+ *     smoothed model runs on INT8 or FP8 compute units). Format: OCP FP8
+ *     E4M3 (largest finite value 448, no infinities), codes stored one byte
+ *     per value.
+ * sq_quantize_weight_fp8 / sq_quantize_act_fp8: as sq_quantize_weight /
+ *   sq_quantize_act (same operands, s semantics, per-row or per-tensor
+ *   scales, workspace rules), with qs = 448 / max(m, 1e-8) and the code of
+ *   fl32(v * qs) rounded to the nearest E4M3 value (ties to even),
+ *   magnitudes past 448 saturated. Wq / Xq: [rows, K] uint8.
+ * sq_gemm_fp8: Y = acc / (qs_x * qs_w) (+ bias) as sq_gemm_w8a8, where acc is
+ *   the fp32 tensor-core sum of the exact E4M3 products (its error is within
+ *   K * 2^-23 * sum |a b|). out_dt in {F32, F16, BF16}. K % 16 == 0.
+ * ------------------------------------------------------------------------ */
+SQ_API sq_status_t sq_quantize_weight_fp8(const void* W, sq_dtype_t dt, int64_t N, int64_t K, const float* s,
+                                          int per_channel, uint8_t* Wq, float* qs_w, void* workspace,
+                                          size_t ws_bytes, sq_stream_t stream);
+SQ_API sq_status_t sq_quantize_act_fp8(const void* X, sq_dtype_t dt, int64_t M, int64_t K, int64_t ldx,
+                                       const float* s, int per_token, const float* static_qs, uint8_t* Xq,
+                                       float* qs_x, void* workspace, size_t ws_bytes, sq_stream_t stream);
+SQ_API sq_status_t sq_gemm_fp8(const uint8_t* Xq, const uint8_t* Wq, int64_t M, int64_t N, int64_t K,
+                               const float* qs_x, int x_per_token, const float* qs_w, int w_per_channel,
+                               const float* bias, sq_dtype_t out_dt, void* Y, int64_t ldy, void* workspace,
+                               size_t ws_bytes, sq_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * LLM.int8() mixed-precision decomposition     [SQ-p5] §2.2, §2.3,
  *        §4.1.
  * ------------------------------------------------------------------------ */
 
-/* a7: outlier dimensions O = { j : count_i(|X[i,j]| > threshold) / M >
+/* Outlier dimensions O = { j : count_i(|X[i,j]| > threshold) / M >
  * min_ratio } in ascending order (fp64 ratio and comparison; the threshold
  * test is strict, in fp32). min_ratio = 0 marks a column on any single
  * value over the threshold. X: [M,K] dt in {F16, BF16}, stride ldx.
@@ -250,7 +349,7 @@ SQ_API sq_status_t sq_llmint8_detect_noalloc(const void* X, sq_dtype_t dt, int64
                                              float threshold, double min_ratio, int32_t* outlier_idx,
                                              int32_t* n_outliers, sq_stream_t stream);
 
-/* a8: vector-wise row quantisation over the columns not in O:
+/* Vector-wise row quantisation over the columns not in O:
  * qs_x[i] = 127 / max(max_{j not in O} |X[i,j]|, 1e-8);
  * Xq[i,j] = 0 for j in O, else clip(rne(X*qs), -127, 127).
  * idx / n_idx: device outlier list (as written by sq_llmint8_detect). */
@@ -258,7 +357,7 @@ SQ_API sq_status_t sq_llmint8_quant_rows(const void* X, sq_dtype_t dt, int64_t M
                                   const int32_t* idx, const int32_t* n_idx, int8_t* Xq,
                                   float* qs_x, sq_stream_t stream);
 
-/* a9 weight side: vector-wise quantisation of W over the input channels not
+/* Weight side: vector-wise quantisation of W over the input channels not
  * in O (one scale per output channel): qs_w[n] = 127/max(max_{k not in O}
  * |W[n,k]|, 1e-8); Wq[n,k] = 0 for k in O. W: [N,K] dt in {F16, BF16}. */
 SQ_API sq_status_t sq_llmint8_quant_weight(const void* W, sq_dtype_t dt, int64_t N, int64_t K,
@@ -279,7 +378,7 @@ typedef struct {
     int32_t* cached_n;
 } sq_llmint8_weight_t;
 
-/* a7-a9 in one call: detect O on X; if O differs from the cached set,
+/* The whole decomposition in one call: detect O on X; if O differs from the cached set,
  * requantise the weight for O (on the device, no host synchronisation);
  * quantise the rows of X; then one GEMM whose epilogue forms
  *   Y[i,j] = acc[i,j] / (qs_x[i] * qs_w[j]) + sum_{o in O ascending} X[i,o] * W[j,o]

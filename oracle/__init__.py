@@ -113,7 +113,7 @@ def f32(a):
     return _c(a, np.float32)
 
 
-# ---------------------------------------------------------------- a1 / a2
+# ---------------------------------------------------------------- calibration absmax
 def col_absmax(X, running=None):
     X = f32(X)
     M, K = X.shape
@@ -122,7 +122,7 @@ def col_absmax(X, running=None):
     return io
 
 
-# ---------------------------------------------------------------- a3
+# ---------------------------------------------------------------- smoothing factors and folds
 def smooth_scales(x, w, alpha):
     x, w = f32(x), f32(w)
     s = np.empty_like(x)
@@ -151,7 +151,7 @@ def fold_norm(gamma, beta, s, round_f32=True):
     return go, bo
 
 
-# ---------------------------------------------------------------- f2
+# ---------------------------------------------------------------- fold into the previous linear
 def fold_prev_linear(W, s, bias=None, round_f32=True):
     """Output channel n of the previous layer (row n, bias_n) divided by s_n."""
     W = _c(f32(W) if round_f32 else W, np.float64)
@@ -166,7 +166,7 @@ def fold_prev_linear(W, s, bias=None, round_f32=True):
     return out, bo
 
 
-# ---------------------------------------------------------------- f1
+# ---------------------------------------------------------------- MLP activation + int8
 SWIGLU, RELU = 0, 1
 
 
@@ -199,7 +199,7 @@ def act_quant(A, act, per_token=True, static_qs=None, quantize=True, absmax=None
     return {"Xq": Xq, "qs": qs, "absmax": am, "H": H}
 
 
-# ---------------------------------------------------------------- f3
+# ---------------------------------------------------------------- FP8 variant
 def e4m3_round(x):
     return np.float32(lib().or_e4m3_round(float(x)))
 
@@ -251,7 +251,7 @@ def dequant_f64(acc, qs_x, qs_w, bias=None, rows=None):
     return y
 
 
-# ---------------------------------------------------------------- a4
+# ---------------------------------------------------------------- weight quantisation
 def quantize_weight(Wp, per_channel=True):
     Wp = f32(Wp)
     N, K = Wp.shape
@@ -261,7 +261,7 @@ def quantize_weight(Wp, per_channel=True):
     return Wq, qs
 
 
-# ---------------------------------------------------------------- a5'
+# ---------------------------------------------------------------- activation quantisation without a norm
 def quantize_act(X, s=None, per_token=True, static_qs=None):
     X = f32(X)
     M, K = X.shape
@@ -278,7 +278,7 @@ def scale_from_absmax(absmax):
     return np.float32(lib().or_scale_from_absmax(_ptr(a), a.size))
 
 
-# ---------------------------------------------------------------- a5
+# ---------------------------------------------------------------- fused norm + smoothing + int8
 LAYERNORM, RMSNORM = 0, 1
 
 
@@ -308,7 +308,7 @@ def norm_f64(H, norm, gamma, beta=None, eps=1e-5):
     return V
 
 
-# ---------------------------------------------------------------- a6
+# ---------------------------------------------------------------- int8 GEMM
 def gemm_i8(Xq, Wq, rows=None):
     Xq, Wq = _c(Xq, np.int8), _c(Wq, np.int8)
     M, K = Xq.shape
@@ -348,7 +348,27 @@ def round_fp16_bits(y):
     return out
 
 
-# ---------------------------------------------------------------- a7-a9
+# ---------------------------------------------------------------- batched int8 GEMM (attention)
+def bmm_i8(A, B, rows=None):
+    """Per problem b: the int64 product A[b] B[b]^T (the plain GEMM, problem by
+    problem: the batched product is nothing more); rows: a list of rows of
+    every A[b] to compute."""
+    A, B = _c(A, np.int8), _c(B, np.int8)
+    pick = (lambda a: a) if rows is None else (lambda a: np.ascontiguousarray(a[list(rows)]))
+    return np.stack([gemm_i8(pick(A[i]), B[i]) for i in range(A.shape[0])])
+
+
+def bmm_dequant(acc, qs_a, qs_b, rows=None):
+    """fp64 acc / (qs_a[b, i] * qs_b[b, j]) per problem b."""
+    out = []
+    for i in range(acc.shape[0]):
+        qa = np.asarray(qs_a[i])
+        qa = qa[list(rows)] if (rows is not None and qa.size > 1) else qa
+        out.append(dequant(acc[i], qa, np.asarray(qs_b[i])))
+    return np.stack(out)
+
+
+# ---------------------------------------------------------------- LLM.int8() decomposition
 def llmint8_outliers(X, thr=6.0, min_ratio=0.0):
     X = f32(X)
     M, K = X.shape

@@ -44,9 +44,9 @@
  *      any one element marks the column; the 16-bit path is exact products
  *      summed in ascending outlier order, added to the dequantised int8 path;
  *   R9 the MLP activation SiLU is evaluated with a fixed fp32 exponential
- *      (below, f1); R10 the fold into the previous linear divides its output
- *      channels by s in fp32 (f2); R11 FP8 is OCP E4M3 with the absmax rule
- *      scaled to its largest value 448 (f3).
+ *      (below); R10 the fold into the previous linear divides its output
+ *      channels by s in fp32; R11 FP8 is OCP E4M3 with the absmax rule
+ *      scaled to its largest value 448.
  */
 #include "sq_oracle.h"
 
@@ -72,7 +72,7 @@ static float scale_of(float m) {
     return 127.0f / d;
 }
 
-/* ------------------------------------------------------------------ a1/a2
+/* ------------------------------------------------------------------ calibration absmax
  * x_j = max_i |X_ij| over all calibration tokens; w_j = max over every output
  * channel of |W| in input channel j.   [SQ-p2] 缩放因子; [SQ-p1] §3.2;
  * [SQ-p4] §3.  Reading R1: running max across calls (p1's hook keeps only
@@ -85,7 +85,7 @@ void or_col_absmax(const float* X, int64_t M, int64_t K, int64_t ld, float* io) 
         }
 }
 
-/* ------------------------------------------------------------------ a3
+/* ------------------------------------------------------------------ smoothing factors and folds
  * s_j = x_j^alpha / w_j^(1-alpha)   [SQ-p2] 缩放因子, [SQ-p1] §2.1, [SQ-p4] §3.
  * Clamps at 1e-5 before and after   [SQ-p1] §3.2 (R2).
  * alpha = 0, 1/2, 1 use the page's closed forms 1/w, sqrt(x/w), x.
@@ -109,7 +109,7 @@ void or_smooth_scales(const float* x, const float* w, int64_t K, double alpha, f
     }
 }
 
-/* ------------------------------------------------------------------ a3 fold
+/* ------------------------------------------------------------------ weight fold
  * W' = S W: input channel j of the weight times s_j. With W stored [N,K]
  * that is column k of every row.  [SQ-p2] SmoothQuant 的原理; [SQ-p4] §3
  * (weight.mul_(s.view(1,-1)) on [out, in]).  Pinned by: the fp64 identity
@@ -139,7 +139,7 @@ void or_fold_norm(const double* gamma, const double* beta, const double* s, int6
     }
 }
 
-/* ------------------------------------------------------------------ f2
+/* ------------------------------------------------------------------ fold into the previous linear
  * Fold 1/s into the previous linear layer   [SQ-p2] 融入前序线性层的权重 and
  * the table after it (down_proj: up_proj's output channels; o_proj: v_proj's
  * output channels): output channel j of the previous layer (row j of W [N,K],
@@ -163,7 +163,7 @@ void or_fold_prev_linear(const double* W, int64_t N, int64_t K, const double* bi
     }
 }
 
-/* ------------------------------------------------------------------ f1
+/* ------------------------------------------------------------------ MLP activation + int8
  * The input of down_proj (FC2) is act(gate_proj(x)) * up_proj(x) ([SQ-p2]
  * 融入前序线性层的权重), or relu(fc1(x)) for a ReLU MLP; with 1/s folded into
  * up_proj's (fc1's) output channels it arrives already smoothed, and is
@@ -239,7 +239,7 @@ void or_act_quant(const float* A, int64_t M, int64_t I, int64_t ld, int act, int
     free(h);
 }
 
-/* ------------------------------------------------------------------ f3
+/* ------------------------------------------------------------------ FP8 variant
  * The same W8A8 path on FP8 units   [SQ-p3] 技術原理與特性 (the smoothed
  * model can run on INT8 or FP8 compute units). The pages give no FP8
  * details. Reading R11: the format is OCP FP8 E4M3 (1 sign bit, 4 exponent
@@ -352,7 +352,7 @@ void or_dequant_f64(const double* acc, int64_t r0, int64_t r1, int64_t N, const 
         }
 }
 
-/* ------------------------------------------------------------------ a4
+/* ------------------------------------------------------------------ weight quantisation
  * Weight int8, per output channel (row) or per tensor   [SQ-p2]
  * 为什么激活不能用逐通道量化 (weight scales per output channel factor out);
  * [SQ-p5] §2.1.  Pinned by: per-channel invariance under a power-of-two
@@ -382,7 +382,7 @@ void or_quantize_weight(const float* Wp, int64_t N, int64_t K, int per_channel,
     }
 }
 
-/* ------------------------------------------------------------------ a5'
+/* ------------------------------------------------------------------ activation quantisation without a norm
  * X' = X / s (explicit divide, [SQ-p4] §3 and §4, [SQ-p1] §3.3), then int8
  * per token or per tensor ([SQ-p5] §2.1).  Pinned by: the worked example of
  * [SQ-p2] 缩放的效果 (q = 1 before smoothing, q = 7 after). */
@@ -430,7 +430,7 @@ float or_scale_from_absmax(const float* absmax, int64_t n) {
     return scale_of(m);
 }
 
-/* ------------------------------------------------------------------ a5
+/* ------------------------------------------------------------------ fused norm + smoothing + int8
  * Fixed reduction order of the fp32 normalisation sums (reading R5; the pages
  * give the formula, not an order). With 256 lanes and chunks of 8 consecutive
  * elements:
@@ -555,7 +555,7 @@ void or_norm_f64(const double* H, int64_t M, int64_t K, int norm, const double* 
     }
 }
 
-/* ------------------------------------------------------------------ a6
+/* ------------------------------------------------------------------ int8 GEMM
  * int8 x int8 -> integer accumulation   [SQ-p5] §2.1 (int32 accumulation);
  * [SQ-p2] 为什么激活不能用逐通道量化 (Y = diag(dX) Xq Wq diag(dW)).
  * Accumulated in int64 so that a sum beyond int32 would show; the test asserts
@@ -636,7 +636,7 @@ void or_round_fp16_array(const double* y, int64_t n, uint16_t* out) {
     for (int64_t i = 0; i < n; ++i) out[i] = or_round_fp16(y[i]);
 }
 
-/* ------------------------------------------------------------------ a7
+/* ------------------------------------------------------------------ LLM.int8() decomposition
  * Outlier dimensions   [SQ-p5] §2.2 split_outliers (over = |x| > alpha;
  * ratio = over.mean(axis=0); keep ratio > min_ratio), §4.1 (any value over
  * the threshold marks the dimension). Reading R6: the garbled comparison is
@@ -661,7 +661,7 @@ static int in_set(const int32_t* idx, int64_t n, int64_t j) {
     return 0;
 }
 
-/* a8: vector-wise row quantisation of the non-outlier columns   [SQ-p5]
+/* Vector-wise row quantisation of the non-outlier columns   [SQ-p5]
  * §2.1 quantize_vectorwise(x, axis=1) applied to x[:, mask] (§2.2). */
 void or_llmint8_quant_rows(const float* X, int64_t M, int64_t K, int64_t ld,
                            const int32_t* idx, int64_t n_idx, int8_t* Xq, float* qs_x) {
@@ -681,7 +681,7 @@ void or_llmint8_quant_rows(const float* X, int64_t M, int64_t K, int64_t ld,
     free(out);
 }
 
-/* a9 (weight side): quantize_vectorwise(w[mask, :], axis=0) of [SQ-p5] §2.2;
+/* Weight side: quantize_vectorwise(w[mask, :], axis=0) of [SQ-p5] §2.2;
  * their W is [K, N], so axis 0 gives one scale per output channel. */
 void or_llmint8_quant_weight(const float* W, int64_t N, int64_t K,
                              const int32_t* idx, int64_t n_idx, int8_t* Wq, float* qs_w) {
@@ -701,7 +701,7 @@ void or_llmint8_quant_weight(const float* W, int64_t N, int64_t K,
     free(out);
 }
 
-/* a9: the two paths summed   [SQ-p5] §2.2 mixed_precision_matmul. */
+/* The two paths summed   [SQ-p5] §2.2 mixed_precision_matmul. */
 void or_llmint8_combine(const int64_t* acc, int64_t r0, int64_t r1, int64_t N, int64_t K,
                         const float* qs_x, const float* qs_w, const float* X, int64_t ldx,
                         const float* W, const int32_t* idx, int64_t n_idx, double* y) {

@@ -73,7 +73,7 @@ def rnd(shape, seed, dtype=torch.float32, scale=1.0):
     return (torch.randn(shape, generator=g) * scale).to(dtype)
 
 
-# ---------------------------------------------------------------- a1 / a2
+# ---------------------------------------------------------------- calibration absmax
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16, torch.float32])
 @pytest.mark.parametrize("M,K", [(1, 8), (37, 1000), (300, 2056), (1029, 4104)])
 def test_calib_absmax(dtype, M, K):
@@ -119,7 +119,7 @@ def test_calib_absmax_strided_and_weight():
     assert np.array_equal(npf(wmax), oracle.col_absmax(W))
 
 
-# ---------------------------------------------------------------- a3
+# ---------------------------------------------------------------- smoothing factors and folds
 @pytest.mark.parametrize("alpha", [0.0, 0.4, 0.5, 0.6, 0.75, 1.0])
 def test_smooth_scales(alpha):
     K = 12288
@@ -153,7 +153,75 @@ def test_fold_weight_and_norm():
     assert np.array_equal(npf(go), rg) and np.array_equal(npf(bo), rb)
 
 
-# ---------------------------------------------------------------- a4
+# ---------------------------------------------------------------- fold into the previous linear
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("with_bias", [True, False])
+def test_fold_prev_linear(dtype, with_bias):
+    N, K = 333, 1032
+    W = rnd((N, K), 12, dtype, 0.03)
+    s = torch.rand(N, generator=torch.Generator().manual_seed(13)) * 20 + 0.01
+    b = rnd(N, 14) if with_bias else None
+    Wp = torch.empty((N, K), device=DEV)
+    bo = torch.empty(N, device=DEV) if with_bias else None
+    sq.sq_fold_prev_linear(W.to(DEV), s.to(DEV), Wp, None if b is None else b.to(DEV), bo)
+    rW, rb = oracle.fold_prev_linear(W.float().numpy(), s.numpy(), None if b is None else b.numpy())
+    assert np.array_equal(npf(Wp), rW)
+    if with_bias:
+        assert np.array_equal(npf(bo), rb)
+
+
+# ---------------------------------------------------------------- MLP activation + int8
+def _act_input(M, I, act, dtype, seed, extra_cols=0):
+    """Gate/up (or fc1) outputs: N(0, 2), with exp-range edge values planted."""
+    width = (2 * I if act == sq.SQ_ACT_SWIGLU else I) + extra_cols
+    A = rnd((M, width), seed, torch.float32, 2.0)
+    A[0, :8] = torch.tensor([0.0, -0.0, 88.5, -88.5, 87.0, -87.0, 30.0, -30.0])
+    A[min(1, M - 1), 3] = 200.0
+    if act == sq.SQ_ACT_RELU and M > 2:
+        A[2] = -A[2].abs()  # an all-zero h row: scale from the 1e-8 floor
+    return A.to(dtype)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("act", [0, 1])
+@pytest.mark.parametrize("I,M", [(8, 5), (1000, 67), (3072, 300), (8192, 33), (9000, 21), (28672, 9)])
+def test_act_quant(dtype, act, I, M):
+    """Codes, scales, the 16-bit h and the calibration maxima bit for bit; a
+    row stride wider than the row."""
+    A = _act_input(M, I, act, dtype, I + act, extra_cols=8)
+    width = 2 * I if act == sq.SQ_ACT_SWIGLU else I
+    Ad = A.to(DEV)[:, :width]
+    Xq = torch.empty((M, I), dtype=torch.int8, device=DEV)
+    qs = torch.empty(M, device=DEV)
+    H = torch.empty((M, I), dtype=dtype, device=DEV)
+    am = torch.full((I,), 0.5, device=DEV)
+    sq.sq_act_quant(Ad, act, True, None, Xq, qs, am, H)
+    r = oracle.act_quant(A[:, :width].float().numpy(), act, want_h=True, absmax=np.full(I, 0.5, np.float32))
+    assert np.array_equal(npf(qs), r["qs"])
+    assert np.array_equal(Xq.cpu().numpy(), r["Xq"])
+    assert np.array_equal(npu16(H), npu16(torch.from_numpy(r["H"]).to(dtype)))
+    assert np.array_equal(npf(am), r["absmax"])
+    # static per-tensor scale: values beyond the range clip
+    qst = torch.tensor([11.0], device=DEV)
+    qx = torch.empty(1, device=DEV)
+    sq.sq_act_quant(Ad, act, False, qst, Xq, qx)
+    rs = oracle.act_quant(A[:, :width].float().numpy(), act, per_token=False, static_qs=11.0)
+    assert np.array_equal(Xq.cpu().numpy(), rs["Xq"])
+    assert npf(qx)[0] == np.float32(11.0)
+
+
+def test_act_quant_errors():
+    A = torch.zeros((4, 64), dtype=torch.bfloat16, device=DEV)
+    Xq = torch.empty((4, 32), dtype=torch.int8, device=DEV)
+    with pytest.raises(sq.SqError):
+        sq.sq_act_quant(A, sq.SQ_ACT_SWIGLU, False, None, Xq, torch.empty(1, device=DEV))  # no static scale
+    with pytest.raises(sq.SqError):
+        sq.sq_act_quant(A[:, :60], sq.SQ_ACT_RELU, True, None, torch.empty((4, 60), dtype=torch.int8, device=DEV),
+                        torch.empty(4, device=DEV))  # I % 8 != 0
+    sq.sq_act_quant(A[:0], sq.SQ_ACT_SWIGLU, True, None, Xq[:0], torch.empty(0, device=DEV))  # M = 0
+
+
+# ---------------------------------------------------------------- weight quantisation
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16, torch.float32])
 @pytest.mark.parametrize("per_channel", [True, False])
 @pytest.mark.parametrize("with_s", [True, False])
@@ -172,7 +240,7 @@ def test_quantize_weight(dtype, per_channel, with_s, K):
     assert np.array_equal(Wq.cpu().numpy(), rq)
 
 
-# ---------------------------------------------------------------- a5'
+# ---------------------------------------------------------------- activation quantisation without a norm
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16, torch.float32])
 @pytest.mark.parametrize("mode", ["token", "tensor_dynamic", "tensor_static"])
 @pytest.mark.parametrize("K", [256, 1040, 4096, 16400])
@@ -212,7 +280,7 @@ def test_quantize_act_config1_worked_path():
     assert np.array_equal(Xq.cpu().numpy(), rq) and np.array_equal(npf(qx), rqs)
 
 
-# ---------------------------------------------------------------- a5
+# ---------------------------------------------------------------- fused norm + smoothing + int8
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
 @pytest.mark.parametrize("norm", ["ln", "rms"])
 @pytest.mark.parametrize("K", [8, 1000, 1024, 3072, 7168, 12288, 16384])
@@ -304,7 +372,7 @@ def test_norm_static_and_calibration(norm, K):
     assert npf(qx)[0] == rqs
 
 
-# ---------------------------------------------------------------- a6
+# ---------------------------------------------------------------- int8 GEMM
 GEMM_SHAPES = [(1, 16, 16), (16, 1024, 1024), (200, 300, 272), (257, 513, 1040), (128, 256, 128),
                (640, 2048, 384), (129, 4096, 1024)]
 
@@ -394,6 +462,62 @@ def test_gemm_deterministic():
     assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
 
 
+# shapes whose last wave of whole tiles is at most three quarters full: its
+# tiles are cut by k-blocks (ragged M and K; pieces of 2 to 30 k-blocks)
+SK_SHAPES = [(1029, 7168, 2064), (260, 13000, 8192), (2560, 4096, 2048)]
+
+
+@pytest.mark.parametrize("M,N,K", SK_SHAPES)
+def test_gemm_stream_k(M, N, K):
+    assert sq.sq_workspace_size(sq.SQ_OP_GEMM, M, N, K) > 256, "the plan was expected to cut this shape"
+    Xq, Wq = rand_i8((M, K), M + 3), rand_i8((N, K), N + 4)
+    Xd, Wd = Xq.to(DEV), Wq.to(DEV)
+    ws = sq.workspace(sq.SQ_OP_GEMM, M, N, K)
+    Y = torch.empty((M, N), dtype=torch.int32, device=DEV)
+    sq.sq_gemm_w8a8(Xd, Wd, None, None, None, Y, ws)
+    sq.sq_workspace_status(ws)
+    # whole tiles (a workspace with no room for the split) agree bit for bit
+    Yw = torch.empty_like(Y)
+    sq.sq_gemm_w8a8(Xd, Wd, None, None, None, Yw, torch.zeros(256, dtype=torch.uint8, device=DEV))
+    assert torch.equal(Y, Yw)
+    Np = (N + 7) // 8 * 8
+    Wp = torch.zeros((Np, K), dtype=torch.int8, device=DEV)
+    Wp[:N] = Wd
+    assert torch.equal(Y, torch._int_mm(Xd, Wp.t())[:, :N])
+    rows = sorted({0, 127, 128, M // 2, M - 1})
+    acc = oracle.gemm_i8(Xq[rows].numpy(), Wq.numpy())
+    assert np.array_equal(Y[rows].cpu().numpy().astype(np.int64), acc)
+    # the counters are back at zero: a second call on the same workspace agrees
+    Y2 = torch.empty_like(Y)
+    sq.sq_gemm_w8a8(Xd, Wd, None, None, None, Y2, ws)
+    assert torch.equal(Y, Y2)
+    # dequantised bf16 with per-token and per-channel scales and a bias
+    g = torch.Generator().manual_seed(M + N + K)
+    qx = torch.rand(M, generator=g) * 100 + 1
+    qw = torch.rand(N, generator=g) * 5000 + 100
+    bias = torch.randn(N, generator=g)
+    Yb = torch.empty((M, N), dtype=torch.bfloat16, device=DEV)
+    sq.sq_gemm_w8a8(Xd, Wd, qx.to(DEV), qw.to(DEV), bias.to(DEV), Yb, ws)
+    y = oracle.dequant(acc, qx.numpy()[rows], qw.numpy(), bias.numpy())
+    terms = np.abs(oracle.dequant(acc, qx.numpy()[rows], qw.numpy())) + np.abs(bias.numpy().astype(np.float64))[None]
+    assert_close_16(Yb[rows].contiguous(), y, torch.bfloat16, terms)
+
+
+def test_bounded_wait_timeout():
+    """A wait that nothing completes gives up after its limit, the status word
+    says so (SQ_ERR_TIMEOUT on the host), and the context stays usable."""
+    ws = sq.workspace(sq.SQ_OP_GEMM, 1, 16, 16)
+    sq.sq_selftest_wait_timeout(ws, 20_000_000)  # 20 ms
+    with pytest.raises(sq.SqError) as e:
+        sq.sq_workspace_status(ws)
+    assert e.value.status == 5
+    sq.sq_workspace_status(ws)  # read and cleared
+    Xq, Wq = rand_i8((130, 256), 7), rand_i8((200, 256), 8)
+    Y = torch.empty((130, 200), dtype=torch.int32, device=DEV)
+    sq.sq_gemm_w8a8(Xq.to(DEV), Wq.to(DEV), None, None, None, Y, ws)
+    assert np.array_equal(Y.cpu().numpy().astype(np.int64), oracle.gemm_i8(Xq.numpy(), Wq.numpy()))
+
+
 @pytest.mark.parametrize("M,N,K", [(4096, 36864, 12288), (1024, 28672, 7168), (2048, 16384, 4096),
                                    (1024, 7168, 28672)])
 def test_gemm_full_size_sampled(M, N, K):
@@ -416,7 +540,7 @@ def test_gemm_full_size_sampled(M, N, K):
     torch.cuda.empty_cache()
 
 
-# ---------------------------------------------------------------- a7 - a9
+# ---------------------------------------------------------------- LLM.int8() decomposition
 def _llm_case(M, K, N, n_out, seed, dtype=torch.float16):
     d = inputs.c4_llmint8(device="cpu", M=M, K=K, N=N, n_out=n_out, seed=seed)
     return d["X"].to(dtype), d["W"].to(dtype), d["dims"]
@@ -560,3 +684,159 @@ def test_errors_raise():
                         torch.zeros((4, 24), dtype=torch.int8, device=DEV), None, None, None,
                         torch.empty((4, 4), dtype=torch.int32, device=DEV), sq.workspace(0, 4, 4, 24))
     assert ei.value.status == 2
+
+
+# ---------------------------------------------------------------- FP8 variant
+def _fp8_bits(t):
+    return t.cpu().numpy().view(np.uint8)
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("per_row,with_s", [(True, True), (True, False), (False, True)])
+@pytest.mark.parametrize("K", [1024, 4112, 20480])
+def test_quantize_fp8(dtype, per_row, with_s, K):
+    """E4M3 codes and scales of weights (x s) and activations (/ s), bit for bit."""
+    M = 131 if K > 4112 else 517
+    X = rnd((M, K), K + 21, dtype, 0.05)
+    X[3, 5] = 0.0
+    s = torch.rand(K, generator=torch.Generator().manual_seed(22)) * 30 + 0.05 if with_s else None
+    Q = torch.empty((M, K), dtype=torch.uint8, device=DEV)
+    qs = torch.empty(M if per_row else 1, device=DEV)
+    ws = sq.workspace(sq.SQ_OP_QUANT_WEIGHT, 0, M, K)
+    Xd, sd = X.to(DEV), None if s is None else s.to(DEV)
+    sq.sq_quantize_weight_fp8(Xd, sd, per_row, Q, qs, ws)
+    rQ, rqs = oracle.quantize_fp8(X.float().numpy(), None if s is None else s.numpy(), s_div=False, per_row=per_row)
+    assert np.array_equal(npf(qs), rqs)
+    assert np.array_equal(_fp8_bits(Q), rQ)
+    sq.sq_quantize_act_fp8(Xd, sd, per_row, None, Q, qs, ws)
+    rQ, rqs = oracle.quantize_fp8(X.float().numpy(), None if s is None else s.numpy(), s_div=True, per_row=per_row)
+    assert np.array_equal(npf(qs), rqs)
+    assert np.array_equal(_fp8_bits(Q), rQ)
+
+
+def _fp8_codes(shape, seed):
+    """Random finite E4M3 codes (NaN codes 0x7F / 0xFF redrawn)."""
+    g = torch.Generator().manual_seed(seed)
+    b = torch.randint(0, 256, shape, generator=g, dtype=torch.int32)
+    b = torch.where((b & 0x7F) == 0x7F, b ^ 0x01, b)
+    return b.to(torch.uint8)
+
+
+def _fp8_tol(A, B, rows):
+    """|error| bound of an fp32 accumulation of K products: K * 2^-23 * sum |a b|."""
+    av = np.vectorize(oracle.e4m3_value)
+    a = np.abs(av(A[rows].numpy()))
+    b = np.abs(av(B.numpy()))
+    return a @ b.T * (A.shape[1] * 2.0 ** -23)
+
+
+@pytest.mark.parametrize("M,N,K", [(16, 256, 64), (200, 300, 272), (257, 513, 1040), (129, 4096, 1024)])
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_gemm_fp8(M, N, K, out_dtype):
+    """FP8 products are exact in fp32; the tensor core sums them in fp32, so the
+    result is within K * 2^-23 * sum|a b| of the exact sum (fp32 out), plus
+    one rounding to bf16."""
+    A, B = _fp8_codes((M, K), M + 5), _fp8_codes((N, K), N + 6)
+    g = torch.Generator().manual_seed(M + N)
+    qx = torch.rand(M, generator=g) * 10 + 1
+    qw = torch.rand(N, generator=g) * 10 + 1
+    bias = torch.randn(N, generator=g)
+    Y = torch.empty((M, N), dtype=out_dtype, device=DEV)
+    sq.sq_gemm_fp8(A.to(DEV), B.to(DEV), qx.to(DEV), qw.to(DEV), bias.to(DEV), Y, sq.workspace(0, M, N, K))
+    rows = sorted({0, 1, M // 2, M - 1})
+    acc = oracle.gemm_fp8(A.numpy(), B.numpy(), rows=rows)
+    y = oracle.dequant_f64(acc, qx.numpy()[rows], qw.numpy(), bias.numpy())
+    d = (qx.numpy()[rows].astype(np.float64)[:, None] * qw.numpy().astype(np.float64)[None, :])
+    tol = _fp8_tol(A, B, rows) / d + 1e-6 * (np.abs(y) + 1e-30)
+    got = Y[rows].float().cpu().numpy().astype(np.float64)
+    if out_dtype == torch.bfloat16:
+        tol = tol + np.abs(y) * 2.0 ** -8
+    assert np.all(np.abs(got - y) <= tol)
+
+
+def test_fp8_path_end_to_end():
+    """Quantise X (/ s) and W (x s) to E4M3 with the library, multiply, and
+    compare with the oracle's chain from the same inputs."""
+    M, N, K = 256, 512, 1024
+    X = rnd((M, K), 70, torch.bfloat16, 1.0)
+    X[:, 7] *= 40
+    W = rnd((N, K), 71, torch.bfloat16, 0.02)
+    s = torch.rand(K, generator=torch.Generator().manual_seed(72)) * 4 + 0.25
+    Xq = torch.empty((M, K), dtype=torch.uint8, device=DEV)
+    Wq = torch.empty((N, K), dtype=torch.uint8, device=DEV)
+    qx, qw = torch.empty(M, device=DEV), torch.empty(N, device=DEV)
+    sq.sq_quantize_act_fp8(X.to(DEV), s.to(DEV), True, None, Xq, qx)
+    sq.sq_quantize_weight_fp8(W.to(DEV), s.to(DEV), True, Wq, qw)
+    Y = torch.empty((M, N), dtype=torch.float32, device=DEV)
+    sq.sq_gemm_fp8(Xq, Wq, qx, qw, None, Y, sq.workspace(0, M, N, K))
+    rXq, rqx = oracle.quantize_fp8(X.float().numpy(), s.numpy(), s_div=True)
+    rWq, rqw = oracle.quantize_fp8(W.float().numpy(), s.numpy(), s_div=False)
+    assert np.array_equal(_fp8_bits(Xq), rXq) and np.array_equal(_fp8_bits(Wq), rWq)
+    rows = [0, 100, 255]
+    y = oracle.dequant_f64(oracle.gemm_fp8(rXq, rWq, rows=rows), rqx[rows], rqw)
+    tol = _fp8_tol(torch.from_numpy(rXq), torch.from_numpy(rWq), rows) / (
+        rqx[rows].astype(np.float64)[:, None] * rqw.astype(np.float64)[None, :]) + 1e-6 * np.abs(y)
+    assert np.all(np.abs(Y[rows].cpu().numpy().astype(np.float64) - y) <= tol)
+    # and the FP8 W8A8 product approximates X W^T
+    ref = X.float().numpy().astype(np.float64)[rows] @ W.float().numpy().astype(np.float64).T
+    assert np.max(np.abs(y - ref)) / np.max(np.abs(ref)) < 0.1
+
+
+# ---------------------------------------------------------------- batched int8 GEMM (attention)
+@pytest.mark.parametrize("batch,M,N,K", [(3, 200, 300, 272), (4, 128, 256, 128), (2, 1, 16, 16), (16, 257, 130, 1040)])
+def test_bmm_int32_exact(batch, M, N, K):
+    """Every problem exact against torch._int_mm (library cross-check) and
+    sampled rows against the oracle; problems never bleed into each other
+    (M, N not multiples of the tile)."""
+    A = torch.stack([rand_i8((M, K), 90 + b) for b in range(batch)])
+    B = torch.stack([rand_i8((N, K), 190 + b) for b in range(batch)])
+    Ad, Bd = A.to(DEV), B.to(DEV)
+    Y = torch.empty((batch, M, N), dtype=torch.int32, device=DEV)
+    sq.sq_bmm_w8a8(Ad, Bd, None, None, Y, sq.workspace(0, M, N, K))
+    if M > 16 and N % 8 == 0:
+        for b in range(batch):
+            assert torch.equal(Y[b], torch._int_mm(Ad[b], Bd[b].t()))
+    rows = sorted({0, M // 2, M - 1})
+    ref = oracle.bmm_i8(A.numpy(), B.numpy(), rows=rows)
+    assert np.array_equal(Y[:, rows].cpu().numpy().astype(np.int64), ref)
+
+
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_bmm_attention(out_dtype):
+    """QK^T with per-(head, token) scales and PV with P per row and V^T per
+    (head, channel), quantised by the library, against the oracle's chain."""
+    H, T, d = 4, 256, 128
+    Q, Kt, V = (rnd((H, T, d), 95 + i, torch.bfloat16) for i in range(3))
+    Qq, Kq = torch.empty((H, T, d), dtype=torch.int8, device=DEV), torch.empty((H, T, d), dtype=torch.int8, device=DEV)
+    qq, qk = torch.empty((H, T), device=DEV), torch.empty((H, T), device=DEV)
+    sq.sq_quantize_act(Q.to(DEV).view(H * T, d), None, True, None, Qq.view(H * T, d), qq.view(-1))
+    sq.sq_quantize_act(Kt.to(DEV).view(H * T, d), None, True, None, Kq.view(H * T, d), qk.view(-1))
+    S = torch.empty((H, T, T), dtype=out_dtype, device=DEV)
+    sq.sq_bmm_w8a8(Qq, Kq, qq, qk, S, sq.workspace(0, T, T, d))
+    rq = [oracle.quantize_act(Q[h].float().numpy(), None, per_token=True) for h in range(H)]
+    rk = [oracle.quantize_act(Kt[h].float().numpy(), None, per_token=True) for h in range(H)]
+    assert np.array_equal(Qq.cpu().numpy(), np.stack([r[0] for r in rq]))
+    rows = [0, 17, 255]
+    ys = oracle.bmm_dequant(oracle.bmm_i8(np.stack([r[0] for r in rq]), np.stack([r[0] for r in rk]), rows=rows),
+                            [r[1] for r in rq], [r[1] for r in rk], rows=rows)
+    for h in range(H):
+        if out_dtype == torch.float32:
+            assert_close_f32(S[h, rows].contiguous(), ys[h], np.abs(ys[h]))
+        else:
+            assert_close_16(S[h, rows].contiguous(), ys[h], out_dtype)
+    # PV: P per row, V^T per (head, channel)
+    P = torch.softmax(S.float() / 16.0, dim=-1).to(torch.bfloat16)
+    Vt = V.to(DEV).transpose(1, 2).contiguous()  # [H, d, T]
+    Pq, Vq = torch.empty((H, T, T), dtype=torch.int8, device=DEV), torch.empty((H, d, T), dtype=torch.int8, device=DEV)
+    qp, qv = torch.empty((H, T), device=DEV), torch.empty((H, d), device=DEV)
+    sq.sq_quantize_act(P.view(H * T, T), None, True, None, Pq.view(H * T, T), qp.view(-1))
+    sq.sq_quantize_act(Vt.view(H * d, T), None, True, None, Vq.view(H * d, T), qv.view(-1))
+    O = torch.empty((H, T, d), dtype=out_dtype, device=DEV)
+    sq.sq_bmm_w8a8(Pq, Vq, qp, qv, O, sq.workspace(0, T, d, T))
+    acc = oracle.bmm_i8(Pq.cpu().numpy(), Vq.cpu().numpy(), rows=rows)
+    yo = oracle.bmm_dequant(acc, qp.cpu().numpy(), qv.cpu().numpy(), rows=rows)
+    for h in range(H):
+        if out_dtype == torch.float32:
+            assert_close_f32(O[h, rows].contiguous(), yo[h], np.abs(yo[h]))
+        else:
+            assert_close_16(O[h, rows].contiguous(), yo[h], out_dtype)

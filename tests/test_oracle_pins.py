@@ -21,7 +21,7 @@ def _load(name):
         return json.load(f)
 
 
-# ------------------------------------------------------------------ a3 pins
+# ------------------------------------------------------------------ smoothing factors: pins
 def test_closed_form_scales(orc):
     """"大语言模型量化技术（四）：SmoothQuant", section 缩放因子: closed forms of
     s_j = x^a / w^(1-a) at powers of two, including a = 0 and a = 1."""
@@ -416,7 +416,7 @@ def test_col_absmax_bruteforce(orc):
     assert np.array_equal(got, ref)
 
 
-# ---------------------------------------------------------------- f1 / f2
+# ---------------------------------------------------------------- MLP activation; fold into the previous linear
 def _ulps(got, ref64):
     """|got - ref| in units of the fp32 spacing at ref."""
     ref32 = ref64.astype(np.float32)
@@ -557,7 +557,7 @@ def test_fold_prev_linear_fp32_is_one_division(orc):
     assert np.array_equal(bp, b / s)
 
 
-# ---------------------------------------------------------------- f3
+# ---------------------------------------------------------------- FP8 variant
 def test_e4m3_codes_round_trip(orc):
     """Every finite E4M3 code decodes to a value that rounds and re-encodes to
     the same code; 0x7F / 0xFF (NaN) are the only codes left out; the largest
@@ -623,3 +623,36 @@ def test_fp8_quant_and_gemm_bruteforce(orc):
     y = acc / (qx.astype(np.float64)[:, None] * qw.astype(np.float64)[None, :])
     ref = X.astype(np.float64) @ W.astype(np.float64).T
     assert np.max(np.abs(y - ref)) / np.max(np.abs(ref)) < 0.1
+
+
+# ---------------------------------------------------------------- batched int8 GEMM (attention)
+def test_bmm_bruteforce(orc):
+    """Each problem of the batch is its own int64 product (einsum brute force)."""
+    rng = np.random.default_rng(50)
+    A = rng.integers(-127, 128, size=(3, 5, 7)).astype(np.int8)
+    B = rng.integers(-127, 128, size=(3, 4, 7)).astype(np.int8)
+    ref = np.einsum("bik,bjk->bij", A.astype(np.int64), B.astype(np.int64))
+    assert np.array_equal(orc.bmm_i8(A, B), ref)
+
+
+def test_bmm_attention_scores_magnitude(orc):
+    """lpnh.cn SmoothQuant practice article §2.2: QK^T in int8 with one scale
+    per (head, token) on Q and on K approximates the fp64 scores; PV with P
+    per row and V^T per (head, channel) approximates P V. Magnitude checks."""
+    rng = np.random.default_rng(51)
+    H, T, d = 2, 16, 32
+    Q, K, V = (rng.normal(size=(H, T, d)).astype(np.float32) for _ in range(3))
+    qq = [orc.quantize_act(Q[h], None, per_token=True) for h in range(H)]
+    kq = [orc.quantize_act(K[h], None, per_token=True) for h in range(H)]
+    S = orc.bmm_dequant(orc.bmm_i8(np.stack([q[0] for q in qq]), np.stack([k[0] for k in kq])),
+                        [q[1] for q in qq], [k[1] for k in kq])
+    ref = np.einsum("htd,hsd->hts", Q.astype(np.float64), K.astype(np.float64))
+    assert np.max(np.abs(S - ref)) / np.max(np.abs(ref)) < 0.03
+    P = np.exp(ref - ref.max(axis=2, keepdims=True))
+    P = (P / P.sum(axis=2, keepdims=True)).astype(np.float32)
+    pq = [orc.quantize_act(P[h], None, per_token=True) for h in range(H)]
+    vq = [orc.quantize_act(np.ascontiguousarray(V[h].T), None, per_token=True) for h in range(H)]
+    O = orc.bmm_dequant(orc.bmm_i8(np.stack([p[0] for p in pq]), np.stack([v[0] for v in vq])),
+                        [p[1] for p in pq], [v[1] for v in vq])
+    refo = np.einsum("hts,hsd->htd", P.astype(np.float64), V.astype(np.float64))
+    assert np.max(np.abs(O - refo)) / np.max(np.abs(refo)) < 0.05

@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libsq_b200.so")
 
 SQ_F32, SQ_F16, SQ_BF16, SQ_I32, SQ_I8 = 0, 1, 2, 3, 4
 SQ_LAYERNORM, SQ_RMSNORM = 0, 1
+SQ_ACT_SWIGLU, SQ_ACT_RELU = 0, 1
 SQ_OP_GEMM, SQ_OP_QUANT_ACT, SQ_OP_QUANT_WEIGHT, SQ_OP_LLMINT8_DETECT, SQ_OP_LLMINT8 = 0, 1, 2, 3, 4
 
 STATUS = {0: "SQ_OK", 1: "SQ_ERR_INVALID_ARG", 2: "SQ_ERR_UNSUPPORTED_SHAPE", 3: "SQ_ERR_ALIGNMENT",
@@ -47,15 +48,22 @@ SIGNATURES = {
     "sq_last_error_string": ([], ctypes.c_char_p),
     "sq_workspace_status": ([_p, _p], _i),
     "sq_version": ([], _i),
+    "sq_selftest_wait_timeout": ([_p, _sz, ctypes.c_uint64, _p], _i),
     "sq_calib_absmax": ([_p, _i, _i64, _i64, _i64, _p, _p], _i),
     "sq_weight_absmax": ([_p, _i, _i64, _i64, _i64, _p, _p], _i),
     "sq_smooth_scales": ([_p, _p, _i64, _d, _p, _p], _i),
     "sq_fold_weight": ([_p, _i, _i64, _i64, _p, _p, _p], _i),
     "sq_fold_norm": ([_p, _p, _p, _i64, _p, _p, _p], _i),
+    "sq_fold_prev_linear": ([_p, _i, _i64, _i64, _p, _p, _p, _p, _p], _i),
     "sq_quantize_weight": ([_p, _i, _i64, _i64, _p, _i, _p, _p, _p, _sz, _p], _i),
     "sq_quantize_act": ([_p, _i, _i64, _i64, _i64, _p, _i, _p, _p, _p, _p, _sz, _p], _i),
     "sq_scale_from_absmax": ([_p, _i64, _p, _p], _i),
     "sq_norm_smooth_quant": ([_p, _i, _i64, _i64, _i64, _i, _p, _p, _f, _i, _p, _p, _p, _p, _p, _p], _i),
+    "sq_bmm_w8a8": ([_p, _p, _i64, _i64, _i64, _i64, _p, _i, _p, _i, _i, _p, _i64, _p, _sz, _p], _i),
+    "sq_quantize_weight_fp8": ([_p, _i, _i64, _i64, _p, _i, _p, _p, _p, _sz, _p], _i),
+    "sq_quantize_act_fp8": ([_p, _i, _i64, _i64, _i64, _p, _i, _p, _p, _p, _p, _sz, _p], _i),
+    "sq_gemm_fp8": ([_p, _p, _i64, _i64, _i64, _p, _i, _p, _i, _p, _i, _p, _i64, _p, _sz, _p], _i),
+    "sq_act_quant": ([_p, _i, _i64, _i64, _i64, _i, _i, _p, _p, _p, _p, _p, _p], _i),
     "sq_gemm_w8a8": ([_p, _p, _i64, _i64, _i64, _p, _i, _p, _i, _p, _i, _p, _i64, _p, _sz, _p], _i),
     "sq_llmint8_detect": ([_p, _i, _i64, _i64, _i64, _f, _d, _p, _p, _p, _sz, _p], _i),
     "sq_llmint8_detect_noalloc": ([_p, _i, _i64, _i64, _i64, _f, _d, _p, _p, _p], _i),
@@ -134,11 +142,16 @@ def sq_workspace_status(ws, stream=None):
     _check("sq_workspace_status", lib().sq_workspace_status(_ptr(ws), _stream(stream)))
 
 
+def sq_selftest_wait_timeout(ws, timeout_ns, stream=None):
+    _check("sq_selftest_wait_timeout", lib().sq_selftest_wait_timeout(_ptr(ws), ws.numel(), int(timeout_ns),
+                                                                      _stream(stream)))
+
+
 def sq_version():
     return int(lib().sq_version())
 
 
-# ---------------------------------------------------------------- a1 / a2
+# ---------------------------------------------------------------- calibration absmax
 def sq_calib_absmax(X, xmax, stream=None):
     _check("sq_calib_absmax", lib().sq_calib_absmax(_ptr(X), _dt(X), X.shape[0], X.shape[1], _ld(X),
                                                     _vec(xmax, torch.float32, X.shape[1]), _stream(stream)))
@@ -149,7 +162,7 @@ def sq_weight_absmax(W, wmax, stream=None):
                                                       _vec(wmax, torch.float32, W.shape[1]), _stream(stream)))
 
 
-# ---------------------------------------------------------------- a3
+# ---------------------------------------------------------------- smoothing factors and folds
 def sq_smooth_scales(xmax, wmax, alpha, s_out, stream=None):
     K = xmax.numel()
     _check("sq_smooth_scales", lib().sq_smooth_scales(_vec(xmax, torch.float32, K), _vec(wmax, torch.float32, K), K,
@@ -171,7 +184,16 @@ def sq_fold_norm(gamma, beta, s, gamma_out, beta_out=None, stream=None):
                                               _vec(beta_out, torch.float32, K), _stream(stream)))
 
 
-# ---------------------------------------------------------------- a4
+def sq_fold_prev_linear(W, s, Wp_out, bias=None, bias_out=None, stream=None):
+    N, K = W.shape
+    if not W.is_contiguous() or not Wp_out.is_contiguous() or Wp_out.dtype != torch.float32:
+        raise ValueError("W and Wp_out must be contiguous; Wp_out fp32")
+    _check("sq_fold_prev_linear", lib().sq_fold_prev_linear(
+        _ptr(W), _dt(W), N, K, _vec(bias, torch.float32, N), _vec(s, torch.float32, N), _ptr(Wp_out),
+        _vec(bias_out, torch.float32, N), _stream(stream)))
+
+
+# ---------------------------------------------------------------- weight quantisation
 def sq_quantize_weight(W, s, per_channel, Wq, qs_w, ws=None, stream=None):
     N, K = W.shape
     if not W.is_contiguous() or not Wq.is_contiguous() or Wq.dtype != torch.int8:
@@ -182,7 +204,7 @@ def sq_quantize_weight(W, s, per_channel, Wq, qs_w, ws=None, stream=None):
         _stream(stream)))
 
 
-# ---------------------------------------------------------------- a5'
+# ---------------------------------------------------------------- activation quantisation without a norm
 def sq_quantize_act(X, s, per_token, static_qs, Xq, qs_x, ws=None, stream=None):
     M, K = X.shape
     if not Xq.is_contiguous() or Xq.dtype != torch.int8:
@@ -198,7 +220,7 @@ def sq_scale_from_absmax(absmax, qs_out, stream=None):
                                                               _vec(qs_out, torch.float32, 1), _stream(stream)))
 
 
-# ---------------------------------------------------------------- a5
+# ---------------------------------------------------------------- fused norm + smoothing + int8
 def sq_norm_smooth_quant(H, norm, gamma, beta, eps, per_token, static_qs, Xq, qs_x, absmax=None, V=None,
                          stream=None):
     M, K = H.shape
@@ -213,7 +235,72 @@ def sq_norm_smooth_quant(H, norm, gamma, beta, eps, per_token, static_qs, Xq, qs
         _stream(stream)))
 
 
-# ---------------------------------------------------------------- a6
+# ---------------------------------------------------------------- batched int8 GEMM (attention)
+def sq_bmm_w8a8(Aq, Bq, qs_a, qs_b, Y, ws, stream=None):
+    """Aq [batch, M, K], Bq [batch, N, K] int8; qs_a [batch, M] or [batch];
+    qs_b [batch, N] or [batch]; Y [batch, M, N] (inner stride 1)."""
+    b, M, K = Aq.shape
+    N = Bq.shape[1]
+    if Aq.dtype != torch.int8 or Bq.dtype != torch.int8 or not Aq.is_contiguous() or not Bq.is_contiguous():
+        raise ValueError("Aq and Bq must be contiguous int8")
+    if Bq.shape[0] != b or Bq.shape[2] != K or tuple(Y.shape[:2]) != (b, M) or Y.shape[2] != N:
+        raise ValueError("shape mismatch")
+    if Y.stride(2) != 1 or Y.stride(0) != M * Y.stride(1):
+        raise ValueError("Y must be [batch, M, ldy] with batches back to back")
+    _check("sq_bmm_w8a8", lib().sq_bmm_w8a8(
+        _ptr(Aq), _ptr(Bq), b, M, N, K, _vec(qs_a, torch.float32), int(qs_a is not None and qs_a.numel() == b * M),
+        _vec(qs_b, torch.float32), int(qs_b is not None and qs_b.numel() == b * N), _dt(Y), _ptr(Y), Y.stride(1),
+        _ptr(ws), ws.numel(), _stream(stream)))
+
+
+# ---------------------------------------------------------------- FP8 variant
+def sq_quantize_weight_fp8(W, s, per_channel, Wq, qs_w, ws=None, stream=None):
+    N, K = W.shape
+    if not W.is_contiguous() or not Wq.is_contiguous() or Wq.dtype != torch.uint8:
+        raise ValueError("W and Wq must be contiguous; Wq uint8 (E4M3 codes)")
+    _check("sq_quantize_weight_fp8", lib().sq_quantize_weight_fp8(
+        _ptr(W), _dt(W), N, K, _vec(s, torch.float32, K), int(per_channel), _ptr(Wq),
+        _vec(qs_w, torch.float32, N if per_channel else 1), _ptr(ws), 0 if ws is None else ws.numel(),
+        _stream(stream)))
+
+
+def sq_quantize_act_fp8(X, s, per_token, static_qs, Xq, qs_x, ws=None, stream=None):
+    M, K = X.shape
+    if not Xq.is_contiguous() or Xq.dtype != torch.uint8:
+        raise ValueError("Xq must be contiguous uint8 (E4M3 codes)")
+    _check("sq_quantize_act_fp8", lib().sq_quantize_act_fp8(
+        _ptr(X), _dt(X), M, K, _ld(X), _vec(s, torch.float32, K), int(per_token), _vec(static_qs, torch.float32, 1),
+        _ptr(Xq), _vec(qs_x, torch.float32, M if per_token else 1), _ptr(ws), 0 if ws is None else ws.numel(),
+        _stream(stream)))
+
+
+def sq_gemm_fp8(Xq, Wq, qs_x, qs_w, bias, Y, ws, stream=None):
+    M, K = Xq.shape
+    N = Wq.shape[0]
+    if Xq.dtype != torch.uint8 or Wq.dtype != torch.uint8 or not Xq.is_contiguous() or not Wq.is_contiguous():
+        raise ValueError("Xq and Wq must be contiguous uint8 (E4M3 codes)")
+    _check("sq_gemm_fp8", lib().sq_gemm_fp8(
+        _ptr(Xq), _ptr(Wq), M, N, K, _vec(qs_x, torch.float32), int(qs_x.numel() > 1), _vec(qs_w, torch.float32),
+        int(qs_w.numel() > 1), _vec(bias, torch.float32, N), _dt(Y), _ptr(Y), _ld(Y), _ptr(ws), ws.numel(),
+        _stream(stream)))
+
+
+# ---------------------------------------------------------------- MLP activation + int8
+def sq_act_quant(A, act, per_token, static_qs, Xq, qs_x, absmax=None, H=None, stream=None):
+    """A: [M, 2I] ([gate | up], SQ_ACT_SWIGLU) or [M, I] (SQ_ACT_RELU)."""
+    M, W = A.shape
+    I = W // 2 if act == SQ_ACT_SWIGLU else W
+    if Xq is not None and (not Xq.is_contiguous() or Xq.dtype != torch.int8):
+        raise ValueError("Xq must be contiguous int8")
+    if H is not None and (H.dtype != A.dtype or not H.is_contiguous()):
+        raise ValueError("H must be contiguous with the dtype of A")
+    _check("sq_act_quant", lib().sq_act_quant(
+        _ptr(A), _dt(A), M, I, _ld(A), int(act), int(per_token), _vec(static_qs, torch.float32, 1), _ptr(Xq),
+        None if qs_x is None else _vec(qs_x, torch.float32), _vec(absmax, torch.float32, I), _ptr(H),
+        _stream(stream)))
+
+
+# ---------------------------------------------------------------- int8 GEMM
 def sq_gemm_w8a8(Xq, Wq, qs_x, qs_w, bias, Y, ws, stream=None):
     M, K = Xq.shape
     N = Wq.shape[0]
@@ -227,7 +314,7 @@ def sq_gemm_w8a8(Xq, Wq, qs_x, qs_w, bias, Y, ws, stream=None):
         _dt(Y), _ptr(Y), _ld(Y), _ptr(ws), ws.numel(), _stream(stream)))
 
 
-# ---------------------------------------------------------------- a7 - a9
+# ---------------------------------------------------------------- LLM.int8() decomposition
 def sq_llmint8_detect(X, threshold, min_ratio, idx, n, ws, stream=None):
     M, K = X.shape
     _check("sq_llmint8_detect", lib().sq_llmint8_detect(

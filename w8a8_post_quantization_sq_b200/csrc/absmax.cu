@@ -1,4 +1,4 @@
-// a1 / a2: per-input-channel absmax for calibration.
+// Per-input-channel absmax for calibration.
 //
 // x_j = max_i |X_ij| over the calibration tokens and w_j = max over output
 // channels of |W| in input channel j ("大语言模型量化技术（四）：SmoothQuant",

@@ -1,5 +1,5 @@
-// a6: INT8 x INT8 -> INT32 GEMM on the 5th-generation tensor cores with a
-// dequantising epilogue, and (a9) the LLM.int8 16-bit outlier term fused into
+// INT8 x INT8 -> INT32 GEMM on the 5th-generation tensor cores with a
+// dequantising epilogue, and the LLM.int8 16-bit outlier term fused into
 // the same epilogue.
 //
 // What it computes ("8位量化：异常值与混合精度分解实战" §2.1; "大语言模型量化技术
@@ -30,6 +30,13 @@
 //     and write whole row segments, while the next tile's MMAs run in the
 //     other accumulator buffer; the buffer is released right after its
 //     last load.
+// Batched variant (lpnh.cn SmoothQuant practice article §2.2: the QK^T and PV
+// products of attention can run in int8): problem b of a [batch, M, K] x
+// [batch, N, K] pair through 3-D tensor maps, its own row scales (one per
+// (head, token) or (head, channel)), Y[b] = Y + b * M * ldy.
+// FP8 variant ("SmoothQuant" (newton wiki), 技術原理與特性: INT8 or FP8
+// units): the same kernel with tcgen05.mma kind::f8f6f4 on E4M3 operands and
+// an fp32 accumulator; the epilogue reads the fp32 sums instead of int32.
 // Every wait is bounded (about 2 s of %globaltimer); on expiry the kernel
 // records code 0x6E1 + role in the status word, drains its own TMA copies and
 // MMAs, frees its tensor memory and returns.
@@ -38,6 +45,7 @@
 
 #include "sq_common.cuh"
 #include "sq_internal.h"
+#include "sq_wait.cuh"
 
 namespace sq {
 namespace {
@@ -53,6 +61,8 @@ constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr int kStgRow = 80;
 constexpr int kStgWarpBytes = 32 * kStgRow;
 enum OutKind { kOutBF16 = 0, kOutF16 = 1, kOutF32 = 2, kOutI32 = 3 };
+// operand formats: int8 x int8 -> int32, or FP8 E4M3 x E4M3 -> fp32
+enum MmaKind { kKindI8 = 0, kKindF8 = 1 };
 
 template <int BN>
 struct Cfg {
@@ -73,19 +83,76 @@ struct Cfg {
     static constexpr uint32_t SMEM = STG_OFF + STG_BYTES;
     static constexpr uint32_t SMEM_ALLOC = SMEM + 1024;  // slack to align the base to 1024
     static constexpr uint32_t TMEM_COLS = 2 * BN;
-    // kind::i8, D = s32 (bits 4-5 = 2), A = B = signed 8-bit (bits 7-9, 10-12 = 1),
+    // kind::i8: D = s32 (bits 4-5 = 2), A = B = signed 8-bit (bits 7-9, 10-12 = 1);
+    // kind::f8f6f4: D = f32 (bits 4-5 = 1), A = B = E4M3 (format 0);
     // both K-major, N >> 3 at bit 17, M >> 4 at bit 24
-    static constexpr uint32_t IDESC =
-        (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+    static constexpr uint32_t idesc(int kind) {
+        return (kind == kKindF8 ? (1u << 4) : ((2u << 4) | (1u << 7) | (1u << 10))) |
+               ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+    }
 };
 
 struct Params {
     int M, N, K;
+    int batch;          // independent problems (heads); 1 for a plain GEMM
+    int64_t y_bstride;  // elements between the batches of Y
     int num_m, num_n, num_kb;
     int group_m;    // m-blocks per raster group
     int vec_store;  // Y rows start on 16-byte boundaries
     GemmEpilogue ep;
     int* status;
+    // Stream-K (one problem only): the first dp_tiles tiles in raster order
+    // run whole, the CTAs taking them in turn; the k-blocks of the remaining
+    // sk_tiles tiles, sk_iters in all, are cut into one contiguous range per
+    // CTA.
+    int dp_tiles, sk_tiles, sk_iters;
+    int* sk_cnt;   // [sk_tiles][kEpiWarps] k-blocks counted in per tile region (zero between launches)
+    int* sk_part;  // [grid][2][kEpiWarps][NCH][8][32] int4: parked int32 partial sums
+};
+
+// First k-iteration of CTA c's stream-K range (every CTA gets at least one:
+// sk_iters >= grid).
+__device__ __forceinline__ int sk_start(int c, const Params& p) {
+    return (int)((int64_t)c * p.sk_iters / (int64_t)gridDim.x);
+}
+// The CTA whose range holds k-iteration x.
+__device__ __forceinline__ int sk_owner(int x, const Params& p) {
+    return (int)((((int64_t)x + 1) * (int64_t)gridDim.x + p.sk_iters - 1) / p.sk_iters - 1);
+}
+
+// This CTA's work, the same sequence for its three roles: whole tiles, then
+// the pieces of its stream-K range (a piece is the part of the range inside
+// one tile). slot = -1 for a whole tile; a piece is the CTA's first (slot 0)
+// or last (slot 1) piece: a range spans at most one whole tile between them.
+template <bool SK>
+struct Segments {
+    int tile_dp, it, end;
+    bool first;
+    __device__ explicit Segments(const Params& p) {
+        tile_dp = blockIdx.x;
+        it = SK ? sk_start(blockIdx.x, p) : 0;
+        end = SK ? sk_start(blockIdx.x + 1, p) : 0;
+        first = true;
+    }
+    __device__ bool next(const Params& p, int num_tiles, int& tile, int& k0, int& k1, int& slot) {
+        if (!SK || tile_dp < p.dp_tiles) {
+            tile = tile_dp;
+            k0 = 0;
+            k1 = p.num_kb;
+            slot = -1;
+            tile_dp += gridDim.x;
+            return tile < (SK ? p.dp_tiles : num_tiles);
+        }
+        if (it >= end) return false;
+        const int u = it / p.num_kb;
+        k0 = it - u * p.num_kb;
+        k1 = min(p.num_kb, k0 + (end - it));
+        tile = p.dp_tiles + u;
+        slot = (k0 == 0 && k1 == p.num_kb) ? -1 : (first ? 0 : 1);
+        first = false;
+        it += k1 - k0;
+        return true;
+    }
 };
 
 // Raster: groups of group_m m-blocks; inside a group, n-major then m. The
@@ -102,51 +169,22 @@ __device__ __forceinline__ void tile_coords(int tile, const Params& p, int bn, i
     n0 = nb * bn;
 }
 
+// Batched problems: tile t of problem b = t / (num_m * num_n).
+__device__ __forceinline__ void tile_coords_b(int tile, const Params& p, int bn, int& b, int& m0, int& n0) {
+    const int tpb = p.num_m * p.num_n;
+    b = tile / tpb;
+    tile_coords(tile - b * tpb, p, bn, m0, n0);
+}
+
 // ---------------------------------------------------------------- PTX helpers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-__device__ __forceinline__ uint64_t global_ns() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-// Wait for the phase of `parity` to complete. Gives up when another role has
-// aborted or after kTimeoutNs, recording `code` in the status word.
-__device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          int* status, int code) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = global_ns();
-    for (uint32_t n = 1;; ++n) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if (*abort_flag) return false;
-        if ((n & 31u) == 0 && global_ns() - t0 > kTimeoutNs) {
-            *abort_flag = 1;
-            atomicExch(status, code);
-            return false;
-        }
-    }
+// Wait for the phase of `parity` to complete, giving up after kTimeoutNs or
+// when another role has aborted (the shared bounded wait of sq_wait.cuh).
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* status,
+                                             int code) {
+    return wait_bounded_ns(bar, parity, abort_flag, status, code, kTimeoutNs);
 }
 
 // Short bounded wait used while draining after an abort (ignores the flag).
@@ -156,10 +194,11 @@ __device__ __noinline__ void wait_drain(uint32_t bar, uint32_t parity) {
         if (global_ns() - t0 > kTimeoutNs / 4) return;
 }
 
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y) {
+// Tile (x = k, y = row) of problem z of a 3-D [batch, rows, K] int8 tensor.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y, int z) {
     asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
-        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
         : "memory");
 }
 
@@ -174,12 +213,21 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr) {
     return d;
 }
 
-__device__ __forceinline__ void umma_i8(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(acc));
+template <int KIND>
+__device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    if constexpr (KIND == kKindF8) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
+            ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(acc));
+    } else {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}"
+            ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(acc));
+    }
 }
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
@@ -248,10 +296,10 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
 // term and bias), stage the chunk in shared memory, then write it out as
 // whole 64-byte row segments (four lanes per row for 16-bit outputs; 32-bit
 // outputs go out in two 16-column halves).
-template <int OUT, bool OUTL>
+template <int OUT, bool OUTL, int KIND>
 __device__ __forceinline__ void epi_chunk(const Params& p, const uint32_t* r, int cw, int col0, int row0, int64_t row,
                                           bool row_ok, float rx, const float* rw_w, const float* bias_w, uint8_t* stg,
-                                          int lane, int n_out, bool compact) {
+                                          int lane, int n_out, bool compact, int prob) {
     const GemmEpilogue& ep = p.ep;
     float y[32];
     if constexpr (OUT == kOutI32) {
@@ -266,8 +314,12 @@ __device__ __forceinline__ void epi_chunk(const Params& p, const uint32_t* r, in
             const float4 w = rw4[e];
             const uint64_t d01 = mul2(rx2, pk2(w.x, w.y));
             const uint64_t d23 = mul2(rx2, pk2(w.z, w.w));
-            upk2(mul2(pk2((float)(int)r[4 * e + 0], (float)(int)r[4 * e + 1]), d01), y[4 * e + 0], y[4 * e + 1]);
-            upk2(mul2(pk2((float)(int)r[4 * e + 2], (float)(int)r[4 * e + 3]), d23), y[4 * e + 2], y[4 * e + 3]);
+            float a[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                a[i] = KIND == kKindF8 ? __uint_as_float(r[4 * e + i]) : (float)(int)r[4 * e + i];
+            upk2(mul2(pk2(a[0], a[1]), d01), y[4 * e + 0], y[4 * e + 1]);
+            upk2(mul2(pk2(a[2], a[3]), d23), y[4 * e + 2], y[4 * e + 3]);
         }
         if constexpr (OUTL) {
             // the 16-bit outlier term, added term by term in ascending o with
@@ -324,7 +376,7 @@ __device__ __forceinline__ void epi_chunk(const Params& p, const uint32_t* r, in
             const int col = col0 + part * 8;
             const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * kStgRow + part * 16);
             if (grow < p.M && col < p.N) {
-                uint16_t* out = static_cast<uint16_t*>(ep.Y) + grow * ep.ldy + col;
+                uint16_t* out = static_cast<uint16_t*>(ep.Y) + prob * p.y_bstride + grow * ep.ldy + col;
                 if (p.vec_store && col + 8 <= p.N) {
                     *reinterpret_cast<uint4*>(out) = v;
                 } else {
@@ -353,7 +405,7 @@ __device__ __forceinline__ void epi_chunk(const Params& p, const uint32_t* r, in
                 const int col = col0 + 16 * hh + part * 4;
                 const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * kStgRow + part * 16);
                 if (grow < p.M && col < p.N) {
-                    uint32_t* out = static_cast<uint32_t*>(ep.Y) + grow * ep.ldy + col;
+                    uint32_t* out = static_cast<uint32_t*>(ep.Y) + prob * p.y_bstride + grow * ep.ldy + col;
                     if (p.vec_store && col + 4 <= p.N) {
                         *reinterpret_cast<uint4*>(out) = v;
                     } else {
@@ -369,7 +421,7 @@ __device__ __forceinline__ void epi_chunk(const Params& p, const uint32_t* r, in
     }
 }
 
-template <int BN, int OUT, bool OUTL>
+template <int BN, int OUT, bool OUTL, int KIND, bool SK>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                  const Params p) {
@@ -422,7 +474,7 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
     pdl_wait();
     pdl_trigger();
 
-    const int num_tiles = p.num_m * p.num_n;
+    const int num_tiles = p.batch * p.num_m * p.num_n;
     if (warp == 0) {
         if (lane == 0) {
             // ---------------------------------------------------- TMA producer
@@ -432,17 +484,19 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
             bool issued[STAGES];
             for (int s = 0; s < STAGES; ++s) issued[s] = false, issued_phase[s] = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-                int m0, n0;
-                tile_coords(tile, p, BN, m0, n0);
-                for (int kb = 0; kb < p.num_kb; ++kb) {
+            Segments<SK> seg(p);
+            int tile, k0, k1, slot;
+            while (ok && seg.next(p, num_tiles, tile, k0, k1, slot)) {
+                int b, m0, n0;
+                tile_coords_b(tile, p, BN, b, m0, n0);
+                for (int kb = k0; kb < k1; ++kb) {
                     if (!wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, p.status, 0x6E1)) {
                         ok = false;
                         break;
                     }
                     mbar_expect_tx(full_bar(stage), C::A_BYTES + C::B_BYTES);
-                    tma_load_2d(sbase + C::A_OFF + stage * C::A_BYTES, &tmap_a, full_bar(stage), kb * BK, m0);
-                    tma_load_2d(sbase + C::B_OFF + stage * C::B_BYTES, &tmap_b, full_bar(stage), kb * BK, n0);
+                    tma_load_3d(sbase + C::A_OFF + stage * C::A_BYTES, &tmap_a, full_bar(stage), kb * BK, m0, b);
+                    tma_load_3d(sbase + C::B_OFF + stage * C::B_BYTES, &tmap_b, full_bar(stage), kb * BK, n0, b);
                     issued[stage] = true;
                     issued_phase[stage] = phase;
                     if (++stage == STAGES) stage = 0, phase ^= 1u;
@@ -461,7 +515,9 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
             uint32_t phase = 0;
             bool ok = true;
             int local = 0;
-            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
+            Segments<SK> seg(p);
+            int tile, k0, k1, slot;
+            for (; ok && seg.next(p, num_tiles, tile, k0, k1, slot); ++local) {
                 const int acc = local & 1;
                 const uint32_t acc_phase = (uint32_t)(local >> 1) & 1u;
                 if (!wait_bounded(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p.status, 0x6E2)) {
@@ -470,7 +526,7 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-                for (int kb = 0; kb < p.num_kb; ++kb) {
+                for (int kb = k0; kb < k1; ++kb) {
                     if (!wait_bounded(full_bar(stage), phase, abort_flag, p.status, 0x6E3)) {
                         ok = false;
                         break;
@@ -480,8 +536,8 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
                     const uint32_t b_addr = sbase + C::B_OFF + stage * C::B_BYTES;
 #pragma unroll
                     for (int k = 0; k < BK / UMMA_K; ++k)
-                        umma_i8(d_tmem, sdesc(a_addr + k * UMMA_K), sdesc(b_addr + k * UMMA_K), C::IDESC,
-                                (kb | k) != 0 ? 1u : 0u);
+                        umma<KIND>(d_tmem, sdesc(a_addr + k * UMMA_K), sdesc(b_addr + k * UMMA_K), C::idesc(KIND),
+                                (kb != k0 || k != 0) ? 1u : 0u);
                     umma_commit(empty_bar(stage));
                     if (++stage == STAGES) stage = 0, phase ^= 1u;
                 }
@@ -510,21 +566,23 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
         float* bias_w = rw_w + HC;
         uint8_t* stg = smem + C::STG_OFF + (warp - 2) * kStgWarpBytes;
         int local = 0;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
-            int m0, n0;
-            tile_coords(tile, p, BN, m0, n0);
+        Segments<SK> seg(p);
+        int tile, k0, k1, slot;
+        for (; seg.next(p, num_tiles, tile, k0, k1, slot); ++local) {
+            int b, m0, n0;
+            tile_coords_b(tile, p, BN, b, m0, n0);
             const int c_base = n0 + half * HC;  // first column of this warp
             if constexpr (OUT != kOutI32) {
                 __syncwarp();
                 for (int c = lane; c < HC; c += 32) {
                     const int col = c_base + c;
-                    float rw = 0.0f, b = 0.0f;
+                    float rw = 0.0f, bv = 0.0f;
                     if (col < p.N) {
-                        rw = __frcp_rn(ep.w_per_channel ? ep.qs_w[col] : ep.qs_w[0]);
-                        if (ep.bias) b = ep.bias[col];
+                        rw = __frcp_rn(ep.w_per_channel ? ep.qs_w[(int64_t)b * p.N + col] : ep.qs_w[b]);
+                        if (ep.bias) bv = ep.bias[col];
                     }
                     rw_w[c] = rw;
-                    bias_w[c] = b;
+                    bias_w[c] = bv;
                 }
                 __syncwarp();
             }
@@ -538,15 +596,69 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
             const bool row_ok = row < p.M;
             float rx = 0.0f;
             if constexpr (OUT != kOutI32)
-                if (row_ok) rx = __frcp_rn(ep.x_per_token ? ep.qs_x[row] : ep.qs_x[0]);
+                if (row_ok) rx = __frcp_rn(ep.x_per_token ? ep.qs_x[(int64_t)b * p.M + row] : ep.qs_x[b]);
             const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + half * HC);
             // chunks that hold at least one valid column; none when the rows are past M
             int nch = 0;
             if (row0 < p.M && c_base < p.N) nch = min(NCH, (p.N - c_base + 31) / 32);
             // Double-buffered TMEM loads only where the variant keeps every
             // value in registers (no spill may sit between a load and its wait).
-            constexpr bool kPipe = !OUTL && OUT != kOutF32;
+            constexpr bool kPipe = !OUTL && OUT != kOutF32 && !SK;
             uint32_t ra[32];
+            if constexpr (SK) {
+                if (slot >= 0) {
+                    // a piece of a split tile: park this warp region's partial
+                    // sums (each warp store writes 512 contiguous bytes),
+                    // release the accumulator, count the piece's k-blocks in;
+                    // the piece that completes the count adds every piece up
+                    // (int32: exact in any order) and runs the epilogue
+                    const int wr = warp - 2;
+                    int4* mine = reinterpret_cast<int4*>(p.sk_part) +
+                                 ((size_t)(blockIdx.x * 2 + slot) * kEpiWarps + wr) * (NCH * 8 * 32);
+                    for (int c = 0; c < NCH; ++c) {
+                        tmem_ld32(t_row + (uint32_t)(c * 32), ra);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            mine[(c * 8 + e) * 32 + lane] = make_int4((int)ra[4 * e], (int)ra[4 * e + 1],
+                                                                      (int)ra[4 * e + 2], (int)ra[4 * e + 3]);
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(tempty_bar(acc));  // accumulator read in full
+                    __threadfence();
+                    __syncwarp();
+                    const int u = tile - p.dp_tiles;
+                    int before = 0;
+                    if (lane == 0) before = atomicAdd(p.sk_cnt + u * kEpiWarps + wr, k1 - k0);
+                    before = __shfl_sync(0xffffffffu, before, 0);
+                    if (before + (k1 - k0) == p.num_kb) {
+                        __threadfence();
+                        const int x0 = u * p.num_kb;
+                        const int c_lo = sk_owner(x0, p), c_hi = sk_owner(x0 + p.num_kb - 1, p);
+                        for (int c = 0; c < nch; ++c) {
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) ra[e] = 0u;
+                            for (int cc = c_lo; cc <= c_hi; ++cc) {
+                                const int sl = sk_start(cc, p) >= x0 ? 0 : 1;
+                                const int4* src = reinterpret_cast<const int4*>(p.sk_part) +
+                                                  ((size_t)(cc * 2 + sl) * kEpiWarps + wr) * (NCH * 8 * 32);
+#pragma unroll
+                                for (int e = 0; e < 8; ++e) {
+                                    const int4 v = __ldcg(src + (c * 8 + e) * 32 + lane);
+                                    ra[4 * e] += (uint32_t)v.x;
+                                    ra[4 * e + 1] += (uint32_t)v.y;
+                                    ra[4 * e + 2] += (uint32_t)v.z;
+                                    ra[4 * e + 3] += (uint32_t)v.w;
+                                }
+                            }
+                            epi_chunk<OUT, OUTL, KIND>(p, ra, c * 32, c_base + c * 32, row0, row, row_ok, rx, rw_w,
+                                                       bias_w, stg, lane, n_out, compact, b);
+                        }
+                        if (lane == 0) p.sk_cnt[u * kEpiWarps + wr] = 0;  // ready for the next launch
+                    }
+                    continue;
+                }
+            }
             if constexpr (kPipe) {
                 uint32_t rb[32];
                 if (nch > 0) {
@@ -562,8 +674,8 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
                         __syncwarp();
                         if (lane == 0) mbar_arrive(tempty_bar(acc));  // accumulator read in full
                     }
-                    epi_chunk<OUT, OUTL>(p, ra, c * 32, c_base + c * 32, row0, row, row_ok, rx, rw_w, bias_w, stg,
-                                         lane, n_out, compact);
+                    epi_chunk<OUT, OUTL, KIND>(p, ra, c * 32, c_base + c * 32, row0, row, row_ok, rx, rw_w, bias_w, stg,
+                                         lane, n_out, compact, b);
                     if (!more) break;
                     tmem_wait(rb);
                     const bool more2 = c + 2 < nch;
@@ -573,8 +685,8 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
                         __syncwarp();
                         if (lane == 0) mbar_arrive(tempty_bar(acc));
                     }
-                    epi_chunk<OUT, OUTL>(p, rb, (c + 1) * 32, c_base + (c + 1) * 32, row0, row, row_ok, rx, rw_w,
-                                         bias_w, stg, lane, n_out, compact);
+                    epi_chunk<OUT, OUTL, KIND>(p, rb, (c + 1) * 32, c_base + (c + 1) * 32, row0, row, row_ok, rx, rw_w,
+                                         bias_w, stg, lane, n_out, compact, b);
                     if (more2) tmem_wait(ra);
                 }
             } else {
@@ -585,8 +697,8 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
                         __syncwarp();
                         if (lane == 0) mbar_arrive(tempty_bar(acc));  // accumulator read in full
                     }
-                    epi_chunk<OUT, OUTL>(p, ra, c * 32, c_base + c * 32, row0, row, row_ok, rx, rw_w, bias_w, stg,
-                                         lane, n_out, compact);
+                    epi_chunk<OUT, OUTL, KIND>(p, ra, c * 32, c_base + c * 32, row0, row, row_ok, rx, rw_w, bias_w, stg,
+                                         lane, n_out, compact, b);
                 }
             }
             if (nch == 0) {
@@ -624,15 +736,16 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// 2-D int8 tensor [rows, K] row-major, box BK x box_rows, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t K, int box_rows) {
+// 3-D int8 tensor [batch, rows, K] (rows of each problem contiguous, problems
+// rows * K bytes apart), box BK x box_rows x 1, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t K, int box_rows, int64_t batch) {
     auto fn = encode_fn();
     if (!fn) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)K};
-    cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+    cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)rows, (cuuint64_t)batch};
+    cuuint64_t strides[2] = {(cuuint64_t)K, (cuuint64_t)(rows * K)};
+    cuuint32_t box[3] = {(cuuint32_t)BK, (cuuint32_t)box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
@@ -640,27 +753,44 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t K, int box
 
 using KernelFn = void (*)(const CUtensorMap, const CUtensorMap, const Params);
 
-template <int BN>
-KernelFn pick_kernel(sq_dtype_t out_dt, bool outl) {
+template <int BN, bool SK>
+KernelFn pick_kernel_sk(sq_dtype_t out_dt, bool outl, int kind) {
+    if (kind == kKindF8) {
+        switch (out_dt) {
+            case SQ_BF16: return gemm_w8a8_kernel<BN, kOutBF16, false, kKindF8, SK>;
+            case SQ_F16: return gemm_w8a8_kernel<BN, kOutF16, false, kKindF8, SK>;
+            default: return gemm_w8a8_kernel<BN, kOutF32, false, kKindF8, SK>;
+        }
+    }
     switch (out_dt) {
-        case SQ_BF16: return outl ? gemm_w8a8_kernel<BN, kOutBF16, true> : gemm_w8a8_kernel<BN, kOutBF16, false>;
-        case SQ_F16: return outl ? gemm_w8a8_kernel<BN, kOutF16, true> : gemm_w8a8_kernel<BN, kOutF16, false>;
-        case SQ_F32: return gemm_w8a8_kernel<BN, kOutF32, false>;
-        default: return gemm_w8a8_kernel<BN, kOutI32, false>;
+        case SQ_BF16:
+            return outl ? gemm_w8a8_kernel<BN, kOutBF16, true, kKindI8, SK>
+                        : gemm_w8a8_kernel<BN, kOutBF16, false, kKindI8, SK>;
+        case SQ_F16:
+            return outl ? gemm_w8a8_kernel<BN, kOutF16, true, kKindI8, SK>
+                        : gemm_w8a8_kernel<BN, kOutF16, false, kKindI8, SK>;
+        case SQ_F32: return gemm_w8a8_kernel<BN, kOutF32, false, kKindI8, SK>;
+        default: return gemm_w8a8_kernel<BN, kOutI32, false, kKindI8, SK>;
     }
 }
 
 template <int BN>
+KernelFn pick_kernel(sq_dtype_t out_dt, bool outl, int kind, bool sk) {
+    return sk ? pick_kernel_sk<BN, true>(out_dt, outl, kind) : pick_kernel_sk<BN, false>(out_dt, outl, kind);
+}
+
+template <int BN>
 sq_status_t launch_bn(const int8_t* Xq, const int8_t* Wq, int64_t M, int64_t N, int64_t K, const GemmEpilogue& ep,
-                      int* status, cudaStream_t stream) {
+                      const GemmPlan& plan, int* status, void* sk_ws, cudaStream_t stream) {
     using C = Cfg<BN>;
     CUtensorMap ta, tb;
-    if (!make_map(&ta, Xq, M, K, BM) || !make_map(&tb, Wq, N, K, BN))
+    if (!make_map(&ta, Xq, M, K, BM, ep.batch) || !make_map(&tb, Wq, N, K, BN, ep.batch))
         return set_error(SQ_ERR_CUDA, "sq_gemm_w8a8: cuTensorMapEncodeTiled failed");
     const bool outl = ep.idx != nullptr;
     if (outl && ep.out_dt != SQ_BF16 && ep.out_dt != SQ_F16)
         return set_error(SQ_ERR_INVALID_ARG, "sq_gemm_w8a8: the outlier term needs a 16-bit output");
-    KernelFn fn = pick_kernel<BN>(ep.out_dt, outl);
+    const bool sk = plan.sk_tiles > 0 && sk_ws != nullptr;
+    KernelFn fn = pick_kernel<BN>(ep.out_dt, outl, ep.kind, sk);
     // the shared-memory opt-in is per kernel and per device; it is cheap, so set it every time
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM_ALLOC) != cudaSuccess)
         return check_launch("sq_gemm_w8a8: set shared memory size");
@@ -668,6 +798,8 @@ sq_status_t launch_bn(const int8_t* Xq, const int8_t* Wq, int64_t M, int64_t N, 
     p.M = (int)M;
     p.N = (int)N;
     p.K = (int)K;
+    p.batch = (int)ep.batch;
+    p.y_bstride = ep.y_bstride;
     p.num_m = (int)((M + BM - 1) / BM);
     p.num_n = (int)((N + BN - 1) / BN);
     p.num_kb = (int)((K + BK - 1) / BK);
@@ -679,24 +811,125 @@ sq_status_t launch_bn(const int8_t* Xq, const int8_t* Wq, int64_t M, int64_t N, 
     p.vec_store = ((reinterpret_cast<uintptr_t>(ep.Y) & 15u) == 0) && ((ep.ldy * eb) % 16 == 0);
     p.ep = ep;
     p.status = status;
-    const int tiles = p.num_m * p.num_n;
-    const int grid = tiles < num_sms() ? tiles : num_sms();
+    p.dp_tiles = sk ? plan.tiles - plan.sk_tiles : plan.tiles;
+    p.sk_tiles = sk ? plan.sk_tiles : 0;
+    p.sk_iters = sk ? plan.sk_tiles * p.num_kb : 0;
+    p.sk_cnt = sk ? static_cast<int*>(sk_ws) : nullptr;
+    p.sk_part = sk ? reinterpret_cast<int*>(static_cast<uint8_t*>(sk_ws) + plan.sk_cnt_bytes) : nullptr;
+    const int grid = plan.grid;
     launch_pdl(fn, dim3(grid), dim3(kThreads), C::SMEM_ALLOC, stream, ta, tb, p);
     return check_launch("sq_gemm_w8a8");
 }
 
 }  // namespace
 
-sq_status_t launch_gemm_w8a8(const int8_t* Xq, const int8_t* Wq, int64_t M, int64_t N, int64_t K,
-                             const GemmEpilogue& ep, int* status_word, cudaStream_t stream) {
+GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int64_t batch) {
+    GemmPlan pl;
+    const int sms = num_sms();
+    const int64_t num_m = (M + BM - 1) / BM;
     // narrow N tiles when wide ones would leave most SMs idle
-    const int64_t tiles256 = ((M + BM - 1) / BM) * ((N + 255) / 256);
-    if (tiles256 < (int64_t)num_sms() && N > 128)
-        return launch_bn<128>(Xq, Wq, M, N, K, ep, status_word, stream);
-    return launch_bn<256>(Xq, Wq, M, N, K, ep, status_word, stream);
+    const int64_t tiles256 = batch * num_m * ((N + 255) / 256);
+    pl.bn = (tiles256 < (int64_t)sms && N > 128) ? 128 : 256;
+    const int64_t tiles = batch * num_m * ((N + pl.bn - 1) / pl.bn);
+    pl.tiles = (int)tiles;
+    pl.grid = (int)(tiles < sms ? tiles : sms);
+    // Stream-K for the remainder: when the last wave of whole tiles would be
+    // at most three quarters full (and the waves average under 90 % busy),
+    // its tiles are cut by k-blocks into one range per CTA, every CTA
+    // starting them together after the whole waves. A k-loop of 16 blocks or
+    // more pays for parking and adding the partial sums.
+    const int64_t kb = (K + BK - 1) / BK;
+    const int64_t rem = tiles % pl.grid;
+    const double eff = (double)tiles / (double)(((tiles + pl.grid - 1) / pl.grid) * pl.grid);
+    if (batch == 1 && pl.grid == sms && tiles > pl.grid && kb >= 16 && rem > 0 && 4 * rem <= 3 * (int64_t)pl.grid &&
+        eff < 0.9 && rem * kb >= pl.grid && rem * kb < (1ll << 31)) {
+        pl.sk_tiles = (int)rem;
+        pl.sk_cnt_bytes = ((size_t)rem * kEpiWarps * sizeof(int) + 255) / 256 * 256;
+        pl.sk_bytes = pl.sk_cnt_bytes + (size_t)pl.grid * 2 * BM * pl.bn * sizeof(int);
+    }
+    return pl;
+}
+
+size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+    if (M <= 0 || N <= 0 || K <= 0) return kStatusBytes;
+    return kStatusBytes + plan_gemm(M, N, K, 1).sk_bytes;
+}
+
+sq_status_t launch_gemm_w8a8(const int8_t* Xq, const int8_t* Wq, int64_t M, int64_t N, int64_t K,
+                             const GemmEpilogue& ep, int* status_word, size_t ws_bytes, cudaStream_t stream) {
+    const GemmPlan pl = plan_gemm(M, N, K, ep.batch);
+    // a workspace without room for the split runs whole tiles only
+    void* sk_ws = (pl.sk_tiles > 0 && ws_bytes >= kStatusBytes + pl.sk_bytes)
+                      ? static_cast<void*>(reinterpret_cast<uint8_t*>(status_word) + kStatusBytes)
+                      : nullptr;
+    if (pl.bn == 128) return launch_bn<128>(Xq, Wq, M, N, K, ep, pl, status_word, sk_ws, stream);
+    return launch_bn<256>(Xq, Wq, M, N, K, ep, pl, status_word, sk_ws, stream);
 }
 
 }  // namespace sq
+
+extern "C" sq_status_t sq_gemm_fp8(const uint8_t* Xq, const uint8_t* Wq, int64_t M, int64_t N, int64_t K,
+                                   const float* qs_x, int x_per_token, const float* qs_w, int w_per_channel,
+                                   const float* bias, sq_dtype_t out_dt, void* Y, int64_t ldy, void* workspace,
+                                   size_t ws_bytes, sq_stream_t stream) {
+    const char* name = "sq_gemm_fp8";
+    SQ_REQUIRE((Xq || M == 0) && Wq && (Y || M == 0) && qs_x && qs_w, SQ_ERR_INVALID_ARG,
+               "%s: null Xq, Wq, Y or scales", name);
+    SQ_REQUIRE(out_dt == SQ_F32 || out_dt == SQ_F16 || out_dt == SQ_BF16, SQ_ERR_INVALID_ARG,
+               "%s: out dtype must be F32, F16 or BF16", name);
+    SQ_REQUIRE(workspace && ws_bytes >= sq::kStatusBytes, SQ_ERR_INVALID_ARG, "%s: needs a workspace of %zu bytes",
+               name, sq::kStatusBytes);
+    SQ_REQUIRE(M >= 0 && N > 0 && K > 0 && ldy >= N, SQ_ERR_UNSUPPORTED_SHAPE, "%s: need N > 0, K > 0, ldy >= N", name);
+    SQ_REQUIRE(K % 16 == 0, SQ_ERR_UNSUPPORTED_SHAPE, "%s: K must be a multiple of 16 (TMA row stride)", name);
+    SQ_REQUIRE(M < (1ll << 31) && N < (1ll << 31), SQ_ERR_UNSUPPORTED_SHAPE, "%s: M and N must be < 2^31", name);
+    SQ_REQUIRE(sq::aligned16(Xq) && sq::aligned16(Wq), SQ_ERR_ALIGNMENT, "%s: Xq and Wq must be 16-byte aligned", name);
+    if (M == 0) return SQ_OK;
+    sq::GemmEpilogue ep;
+    ep.qs_x = qs_x;
+    ep.x_per_token = x_per_token;
+    ep.qs_w = qs_w;
+    ep.w_per_channel = w_per_channel;
+    ep.bias = bias;
+    ep.out_dt = out_dt;
+    ep.Y = Y;
+    ep.ldy = ldy;
+    ep.kind = 1;
+    return sq::launch_gemm_w8a8(reinterpret_cast<const int8_t*>(Xq), reinterpret_cast<const int8_t*>(Wq), M, N, K, ep,
+                                static_cast<int*>(workspace), ws_bytes, sq::as_cuda(stream));
+}
+
+extern "C" sq_status_t sq_bmm_w8a8(const int8_t* Aq, const int8_t* Bq, int64_t batch, int64_t M, int64_t N,
+                                   int64_t K, const float* qs_a, int a_per_row, const float* qs_b, int b_per_row,
+                                   sq_dtype_t out_dt, void* Y, int64_t ldy, void* workspace, size_t ws_bytes,
+                                   sq_stream_t stream) {
+    const char* name = "sq_bmm_w8a8";
+    SQ_REQUIRE(batch >= 0 && M >= 0 && N > 0 && K > 0 && ldy >= N, SQ_ERR_UNSUPPORTED_SHAPE,
+               "%s: need batch, M >= 0, N, K > 0, ldy >= N", name);
+    if (batch == 0 || M == 0) return SQ_OK;
+    SQ_REQUIRE(Aq && Bq && Y, SQ_ERR_INVALID_ARG, "%s: null Aq, Bq or Y", name);
+    SQ_REQUIRE(out_dt == SQ_I32 || (qs_a && qs_b), SQ_ERR_INVALID_ARG, "%s: dequantising output needs qs_a and qs_b",
+               name);
+    SQ_REQUIRE(out_dt == SQ_I32 || out_dt == SQ_F32 || out_dt == SQ_F16 || out_dt == SQ_BF16, SQ_ERR_INVALID_ARG,
+               "%s: out dtype must be I32, F32, F16 or BF16", name);
+    SQ_REQUIRE(workspace && ws_bytes >= sq::kStatusBytes, SQ_ERR_INVALID_ARG, "%s: needs a workspace of %zu bytes",
+               name, sq::kStatusBytes);
+    SQ_REQUIRE(K % 16 == 0, SQ_ERR_UNSUPPORTED_SHAPE, "%s: K must be a multiple of 16 (TMA row stride)", name);
+    SQ_REQUIRE(K <= 133144, SQ_ERR_UNSUPPORTED_SHAPE, "%s: K > 133144 could overflow the int32 accumulator", name);
+    SQ_REQUIRE(batch * ((M + 127) / 128) * ((N + 127) / 128) < (1ll << 31) && M < (1ll << 31) && N < (1ll << 31),
+               SQ_ERR_UNSUPPORTED_SHAPE, "%s: too many tiles", name);
+    SQ_REQUIRE(sq::aligned16(Aq) && sq::aligned16(Bq), SQ_ERR_ALIGNMENT, "%s: Aq and Bq must be 16-byte aligned", name);
+    sq::GemmEpilogue ep;
+    ep.qs_x = qs_a;
+    ep.x_per_token = a_per_row;
+    ep.qs_w = qs_b;
+    ep.w_per_channel = b_per_row;
+    ep.out_dt = out_dt;
+    ep.Y = Y;
+    ep.ldy = ldy;
+    ep.batch = batch;
+    ep.y_bstride = M * ldy;
+    return sq::launch_gemm_w8a8(Aq, Bq, M, N, K, ep, static_cast<int*>(workspace), ws_bytes, sq::as_cuda(stream));
+}
 
 extern "C" sq_status_t sq_gemm_w8a8(const int8_t* Xq, const int8_t* Wq, int64_t M, int64_t N, int64_t K,
                                     const float* qs_x, int x_per_token, const float* qs_w, int w_per_channel,
@@ -725,5 +958,5 @@ extern "C" sq_status_t sq_gemm_w8a8(const int8_t* Xq, const int8_t* Wq, int64_t 
     ep.out_dt = out_dt;
     ep.Y = Y;
     ep.ldy = ldy;
-    return sq::launch_gemm_w8a8(Xq, Wq, M, N, K, ep, static_cast<int*>(workspace), sq::as_cuda(stream));
+    return sq::launch_gemm_w8a8(Xq, Wq, M, N, K, ep, static_cast<int*>(workspace), ws_bytes, sq::as_cuda(stream));
 }

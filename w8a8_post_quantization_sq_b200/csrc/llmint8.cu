@@ -1,4 +1,4 @@
-// a7-a9: the LLM.int8() mixed-precision decomposition
+// The LLM.int8() mixed-precision decomposition
 // ("8位量化：异常值与混合精度分解实战" §2.2 split_outliers / mixed_precision_matmul,
 // §2.3 threshold 6.0, §4.1 any value over the threshold marks its dimension).
 //
@@ -349,7 +349,7 @@ sq_status_t sq_llmint8_matmul(const void* X, sq_dtype_t dt, int64_t M, int64_t K
     float* wo = reinterpret_cast<float*>(wsb + off);
     const int64_t wo_ld = sq::wo_ld_of(w->N);
     int32_t* changed = reinterpret_cast<int32_t*>(wsb + 4);
-    // a7: O, and whether the cached int8 weight was built for it
+    // the outlier set O, and whether the cached int8 weight was built for it
     st = sq::launch_detect(X, dt, M, K, ldx, threshold, min_ratio, idx_out, n_out, w->cached_idx, w->cached_n, workspace,
                            s);
     if (st != SQ_OK) return st;
@@ -357,7 +357,7 @@ sq_status_t sq_llmint8_matmul(const void* X, sq_dtype_t dt, int64_t M, int64_t K
     st = sq::launch_masked_quant(w->W, dt, w->N, K, K, idx_out, n_out, changed, w->Wq, w->qs_w, s, name);
     if (st != SQ_OK) return st;
     if (M == 0) return SQ_OK;
-    // a8 (and the fp32 copy of the outlier columns of X)
+    // row quantisation outside O (and the fp32 copy of the outlier columns of X)
     st = sq::launch_masked_quant(X, dt, M, K, ldx, idx_out, n_out, nullptr, Xq, qs_x, s, name, xo);
     if (st != SQ_OK) return st;
     // fp32 copy of the outlier input channels of W, transposed, for the epilogue
@@ -373,7 +373,7 @@ sq_status_t sq_llmint8_matmul(const void* X, sq_dtype_t dt, int64_t M, int64_t K
         st = sq::check_launch(name);
         if (st != SQ_OK) return st;
     }
-    // a9: int8 GEMM + 16-bit outlier term in the epilogue
+    // int8 GEMM + 16-bit outlier term in the epilogue
     sq::GemmEpilogue ep;
     ep.qs_x = qs_x;
     ep.x_per_token = 1;
@@ -391,7 +391,8 @@ sq_status_t sq_llmint8_matmul(const void* X, sq_dtype_t dt, int64_t M, int64_t K
     ep.xo = xo;
     ep.wo = wo;
     ep.wo_ld = wo_ld;
-    return sq::launch_gemm_w8a8(Xq, w->Wq, M, w->N, K, ep, static_cast<int*>(workspace), s);
+    // the workspace past its header holds the decomposition's own buffers: no stream-K scratch
+    return sq::launch_gemm_w8a8(Xq, w->Wq, M, w->N, K, ep, static_cast<int*>(workspace), sq::kStatusBytes, s);
 }
 
 }  // extern "C"

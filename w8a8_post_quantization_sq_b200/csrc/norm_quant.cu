@@ -1,4 +1,4 @@
-// a5: LayerNorm / RMSNorm with the smoothing folded into gamma' (and beta'),
+// LayerNorm / RMSNorm with the smoothing folded into gamma' (and beta'),
 // fused with int8 quantisation of the result.
 //
 // "大语言模型量化技术（四）：SmoothQuant", section 融入 LayerNorm: the norm's
@@ -64,17 +64,17 @@ __device__ __forceinline__ float warp_max(float v) {
 }
 
 // v_j of one 8-element chunk from its fp32 inputs f (v may alias f); g holds
-// gamma'_j of the chunk, beta'_j is read from a.beta (LayerNorm with a shift)
+// gamma'_j of the chunk, beta (shared or global memory, or null) beta'
 template <bool LN>
-__device__ __forceinline__ void compute_v_f(const float* f, int ch, const NormArgs& a, const float* g, float mu,
+__device__ __forceinline__ void compute_v_f(const float* f, int ch, const float* beta, const float* g, float mu,
                                             float r, float* v) {
     const uint64_t r2 = pk2(r, r);
     if constexpr (LN) {
         const uint64_t nmu2 = pk2(-mu, -mu);  // x + (-mu) is the IEEE x - mu
-        if (a.beta) {
+        if (beta) {
             // the last product feeds an add: keep those two steps scalar
-            const float4 b0 = __ldg(reinterpret_cast<const float4*>(a.beta + ch * 8));
-            const float4 b1 = __ldg(reinterpret_cast<const float4*>(a.beta + ch * 8 + 4));
+            const float4 b0 = *reinterpret_cast<const float4*>(beta + ch * 8);
+            const float4 b1 = *reinterpret_cast<const float4*>(beta + ch * 8 + 4);
             const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
             for (int e = 0; e < 8; e += 2) {
@@ -96,11 +96,11 @@ __device__ __forceinline__ void compute_v_f(const float* f, int ch, const NormAr
 
 // the same from the chunk's 16-bit inputs
 template <typename T, bool LN>
-__device__ __forceinline__ void compute_v_g(const uint4& rw, int ch, const NormArgs& a, const float* g, float mu,
+__device__ __forceinline__ void compute_v_g(const uint4& rw, int ch, const float* beta, const float* g, float mu,
                                             float r, float* v) {
     float f[8];
     unpack<T>(rw, f);
-    compute_v_f<LN>(f, ch, a, g, mu, r, v);
+    compute_v_f<LN>(f, ch, beta, g, mu, r, v);
 }
 
 __device__ __forceinline__ void load_gamma(const NormArgs& a, int ch, float* g) {
@@ -115,7 +115,7 @@ template <typename T, bool LN>
 __device__ __forceinline__ void compute_v(const uint4& rw, int ch, const NormArgs& a, float mu, float r, float* v) {
     float g[8];
     load_gamma(a, ch, g);
-    compute_v_g<T, LN>(rw, ch, a, g, mu, r, v);
+    compute_v_g<T, LN>(rw, ch, a.beta, g, mu, r, v);
 }
 
 template <typename T>
@@ -322,6 +322,8 @@ norm_quant_bulk_kernel(const T* __restrict__ H, NormArgs a, int R) {
     const float Kf = (float)a.K;
     const uint32_t row_bytes = (uint32_t)(a.K * sizeof(T));
     float* amax_sh = reinterpret_cast<float*>(dsm + (size_t)R * row_bytes);
+    // beta' (LayerNorm with a shift) staged once per block after the maxima
+    float* beta_sh = (LN && a.beta) ? amax_sh + (!QONLY && a.absmax ? a.K : 0) : nullptr;
     const int64_t G = gridDim.x;
     auto mine = [&](int c) { return FULL || t + c * kBlock < nch; };
     float g[C][8];
@@ -336,6 +338,9 @@ norm_quant_bulk_kernel(const T* __restrict__ H, NormArgs a, int R) {
     }
     if (!QONLY && a.absmax)
         for (int j = t; j < a.K; j += kBlock) amax_sh[j] = 0.0f;
+    if (beta_sh)
+        for (int j = t; j < nch * 2; j += kBlock)
+            reinterpret_cast<float4*>(beta_sh)[j] = __ldg(reinterpret_cast<const float4*>(a.beta) + j);
     __syncwarp();
     __syncthreads();
     if (t == 0)
@@ -412,8 +417,8 @@ norm_quant_bulk_kernel(const T* __restrict__ H, NormArgs a, int R) {
                 if (mine(c)) {
                     float vl[8];
                     float* v = KEEPV ? vk[c] : vl;
-                    if constexpr (KEEPV) compute_v_f<LN>(vk[c], ch, a, g[c], mu, r, v);
-                    else compute_v_g<T, LN>(chunk(c), ch, a, g[c], mu, r, v);
+                    if constexpr (KEEPV) compute_v_f<LN>(vk[c], ch, beta_sh, g[c], mu, r, v);
+                    else compute_v_g<T, LN>(chunk(c), ch, beta_sh, g[c], mu, r, v);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(v[e]));
                     if constexpr (!QONLY) {
@@ -449,7 +454,7 @@ norm_quant_bulk_kernel(const T* __restrict__ H, NormArgs a, int R) {
                         *reinterpret_cast<uint2*>(q + ch * 8) = codes8(vk[c], qs, !a.per_token);
                     } else {
                         float v[8];
-                        compute_v_g<T, LN>(chunk(c), ch, a, g[c], mu, r, v);
+                        compute_v_g<T, LN>(chunk(c), ch, beta_sh, g[c], mu, r, v);
                         *reinterpret_cast<uint2*>(q + ch * 8) = codes8(v, qs, !a.per_token);
                     }
                 }
@@ -496,10 +501,11 @@ template <typename T, bool LN, int C, bool KEEPV, bool FULL, bool QONLY>
 void launch_block_k(const void* H, const NormArgs& a, cudaStream_t s) {
     auto kern = norm_quant_bulk_kernel<T, LN, C, KEEPV, FULL, QONLY>;
     const size_t row_bytes = (size_t)a.K * sizeof(T);
-    int R = (int)((96 * 1024) / row_bytes);  // about 96 KB of staged rows per block
+    const size_t extra = (a.absmax ? (size_t)a.K * sizeof(float) : 0) + (LN && a.beta ? (size_t)a.K * sizeof(float) : 0);
+    int R = (int)((96 * 1024 - (a.absmax ? 0 : extra)) / row_bytes);  // about 96 KB of staged rows and beta'
     if (R < 2) R = 2;
     if (R > 8) R = 8;
-    const size_t smem = (size_t)R * row_bytes + (a.absmax ? (size_t)a.K * sizeof(float) : 0);
+    const size_t smem = (size_t)R * row_bytes + extra;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     int per_sm = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kBlock, smem) != cudaSuccess || per_sm < 1)

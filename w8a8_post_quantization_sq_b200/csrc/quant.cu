@@ -1,4 +1,4 @@
-// a4 / a5': symmetric absmax int8 quantisation of weights and of activations
+// Symmetric absmax int8 quantisation of weights and of activations
 // that do not come out of a norm.
 //
 // "8位量化：异常值与混合精度分解实战" §2.1: scale = 127 / max(|x|, 1e-8) over the
@@ -11,10 +11,17 @@
 // 解决激活值离群点难题" §3). All arithmetic is fp32 with correctly rounded
 // operations, so codes and scales are bit-exact against a plain CPU loop.
 //
+// The same kernels write FP8 E4M3 codes for the FP8 variant of the path
+// ("SmoothQuant" (newton wiki), 技術原理與特性: INT8 or FP8 units): scale =
+// 448 / max(|x|, 1e-8), codes by the saturating round-to-nearest-even
+// conversion.
+//
 // Row mode: the row is read once into the registers of one warp (K <= 2048)
 // or one block (K <= 16384), reduced to its absmax and quantised from the
 // registers; longer rows stream twice through a warp. Tensor mode: a
 // grid-wide absmax into the workspace, then the quantising pass.
+#include <cuda_fp8.h>
+
 #include "sq_common.cuh"
 #include "sq_internal.h"
 
@@ -64,11 +71,33 @@ __device__ __forceinline__ float block_max(float v, float* sh) {
     return m;
 }
 
-__device__ __forceinline__ float scale_of(float m) { return __fdiv_rn(127.0f, fmaxf(m, 1e-8f)); }
+// Output formats: int8 codes, or FP8 E4M3 codes (largest finite value 448).
+enum QFmt { kI8 = 0, kE4M3 = 1 };
 
-// Eight codes; `clip` is needed only when qs does not come from the group's
-// own absmax (a static per-tensor scale).
-__device__ __forceinline__ uint2 codes8(const float* v, float qs, bool clip) {
+template <int FMT>
+__device__ __forceinline__ float scale_of(float m) {
+    return __fdiv_rn(FMT == kE4M3 ? 448.0f : 127.0f, fmaxf(m, 1e-8f));
+}
+
+// Eight E4M3 codes of v * qs: each product one fp32 rounding, then the
+// conversion rounds to the nearest E4M3 value (ties to even) and saturates
+// at +-448.
+__device__ __forceinline__ uint2 fp8codes8(const float* v, float qs) {
+    uint32_t w[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const __nv_fp8x2_storage_t a = __nv_cvt_float2_to_fp8x2(
+            make_float2(__fmul_rn(v[4 * h], qs), __fmul_rn(v[4 * h + 1], qs)), __NV_SATFINITE, __NV_E4M3);
+        const __nv_fp8x2_storage_t b = __nv_cvt_float2_to_fp8x2(
+            make_float2(__fmul_rn(v[4 * h + 2], qs), __fmul_rn(v[4 * h + 3], qs)), __NV_SATFINITE, __NV_E4M3);
+        w[h] = (uint32_t)a | ((uint32_t)b << 16);
+    }
+    return make_uint2(w[0], w[1]);
+}
+
+// Eight int8 codes; `clip` is needed only when qs does not come from the
+// group's own absmax (a static per-tensor scale).
+__device__ __forceinline__ uint2 codes8_i8(const float* v, float qs, bool clip) {
     uint32_t b[8];
     if (clip) {
 #pragma unroll
@@ -79,6 +108,12 @@ __device__ __forceinline__ uint2 codes8(const float* v, float qs, bool clip) {
     return make_uint2(pack_low_bytes(b[0], b[1], b[2], b[3]), pack_low_bytes(b[4], b[5], b[6], b[7]));
 }
 
+template <int FMT>
+__device__ __forceinline__ uint2 codes8(const float* v, float qs, bool clip) {
+    if constexpr (FMT == kE4M3) return fp8codes8(v, qs);  // saturating conversion: no separate clip
+    else return codes8_i8(v, qs, clip);
+}
+
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -87,7 +122,7 @@ __device__ __forceinline__ float warp_max(float v) {
 
 // One warp per row, rows strided over the grid. per_row != 0: the row's own
 // scale from its absmax; else *tensor_qs for every row.
-template <typename T, int SM>
+template <typename T, int SM, int FMT>
 __global__ void __launch_bounds__(kThreads)
 row_quant_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, const float* __restrict__ s,
                  int per_row, const float* __restrict__ tensor_qs, int8_t* __restrict__ Q,
@@ -109,7 +144,7 @@ row_quant_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, cons
 #pragma unroll
                 for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(f[e]));
             }
-            qs = scale_of(warp_max(m));
+            qs = scale_of<FMT>(warp_max(m));
             if (lane == 0) qs_out[row] = qs;
         } else {
             qs = *tensor_qs;
@@ -121,7 +156,7 @@ row_quant_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, cons
             float f[8];
             load8<T>(x + k0, f);
             apply_s<SM>(f, s, k0);
-            *reinterpret_cast<uint2*>(q + k0) = codes8(f, qs, !per_row);
+            *reinterpret_cast<uint2*>(q + k0) = codes8<FMT>(f, qs, !per_row);
         }
     }
 }
@@ -152,7 +187,7 @@ __device__ __forceinline__ void unpack_raw(const Raw8<T>& r, float* f) {
 // codes from the registers. The next row's loads are issued before the group
 // reduction so they land while this row is finished. Used while
 // K <= 8 * G * CH_max.
-template <typename T, int SM, int G, int CH>
+template <typename T, int SM, int G, int CH, int FMT>
 __global__ void __launch_bounds__(kThreads)
 row_quant_reg_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, const float* __restrict__ s,
                      int per_row, const float* __restrict__ tensor_qs, int8_t* __restrict__ Q,
@@ -202,7 +237,7 @@ row_quant_reg_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, 
             } else {
                 m = block_max(m, sh);
             }
-            qs = scale_of(m);
+            qs = scale_of<FMT>(m);
             if (gt == 0) qs_out[row] = qs;
         } else {
             qs = *tensor_qs;
@@ -212,7 +247,7 @@ row_quant_reg_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, 
 #pragma unroll
         for (int c = 0; c < CH; ++c) {
             const int64_t k0 = ((int64_t)gt + (int64_t)c * G) * 8;
-            if (k0 < K) *reinterpret_cast<uint2*>(q + k0) = codes8(v[c], qs, !per_row);
+            if (k0 < K) *reinterpret_cast<uint2*>(q + k0) = codes8<FMT>(v[c], qs, !per_row);
         }
     }
 }
@@ -241,7 +276,8 @@ tensor_absmax_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld,
     if (threadIdx.x == 0) atomic_max_nonneg(out, m);
 }
 
-// qs = 127 / max(max_j a[j], 1e-8) into *qs (one block).
+// qs = 127 (int8) or 448 (E4M3) / max(max_j a[j], 1e-8) into *qs (one block).
+template <int FMT>
 __global__ void __launch_bounds__(kThreads)
 scale_from_absmax_kernel(const float* __restrict__ a, int64_t n, float* __restrict__ qs) {
     pdl_wait();
@@ -250,7 +286,7 @@ scale_from_absmax_kernel(const float* __restrict__ a, int64_t n, float* __restri
     float m = 0.0f;
     for (int64_t j = threadIdx.x; j < n; j += kThreads) m = fmaxf(m, a[j]);
     m = block_max(m, sh);
-    if (threadIdx.x == 0) *qs = scale_of(m);
+    if (threadIdx.x == 0) *qs = scale_of<FMT>(m);
 }
 
 int row_grid(int64_t M) {
@@ -265,7 +301,7 @@ int vec_grid(int64_t nvec) {
     return (int)(b < 1 ? 1 : (b > cap ? cap : b));
 }
 
-template <typename T, int SM>
+template <typename T, int SM, int FMT>
 sq_status_t quantize(const void* Xv, int64_t M, int64_t K, int64_t ld, const float* s, int per_row,
                      const float* static_qs, int8_t* Q, float* qs_out, void* ws, cudaStream_t st,
                      const char* name) {
@@ -277,7 +313,7 @@ sq_status_t quantize(const void* Xv, int64_t M, int64_t K, int64_t ld, const flo
         float* wqs = wmax + 1;
         if (cudaMemsetAsync(wmax, 0, sizeof(float), st) != cudaSuccess) return check_launch(name);
         launch_pdl(tensor_absmax_kernel<T, SM>, dim3(vec_grid(M * K / 8)), dim3(kThreads), 0, st, X, M, K, ld, s, wmax);
-        launch_pdl(scale_from_absmax_kernel, dim3(1), dim3(kThreads), 0, st, wmax, 1, wqs);
+        launch_pdl(scale_from_absmax_kernel<FMT>, dim3(1), dim3(kThreads), 0, st, wmax, 1, wqs);
         tensor_qs = wqs;
     }
     // one resident wave of blocks; each group strides over the rows
@@ -291,33 +327,33 @@ sq_status_t quantize(const void* Xv, int64_t M, int64_t K, int64_t ld, const flo
         return launch_pdl(kern, dim3((unsigned)b), dim3(kThreads), 0, st, X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
     };
     if (K <= 256)
-        go(row_quant_reg_kernel<T, SM, 32, 1>, 8);
+        go(row_quant_reg_kernel<T, SM, 32, 1, FMT>, 8);
     else if (K <= 512)
-        go(row_quant_reg_kernel<T, SM, 32, 2>, 8);
+        go(row_quant_reg_kernel<T, SM, 32, 2, FMT>, 8);
     else if (K <= 1024)
-        go(row_quant_reg_kernel<T, SM, 32, 4>, 8);
+        go(row_quant_reg_kernel<T, SM, 32, 4, FMT>, 8);
     else if (K <= 2048)
-        go(row_quant_reg_kernel<T, SM, 32, 8>, 8);
+        go(row_quant_reg_kernel<T, SM, 32, 8, FMT>, 8);
     else if (K <= 4096)
-        go(row_quant_reg_kernel<T, SM, 256, 2>, 1);
+        go(row_quant_reg_kernel<T, SM, 256, 2, FMT>, 1);
     else if (K <= 8192)
-        go(row_quant_reg_kernel<T, SM, 256, 4>, 1);
+        go(row_quant_reg_kernel<T, SM, 256, 4, FMT>, 1);
     else if (K <= 16384)
-        go(row_quant_reg_kernel<T, SM, 256, 8>, 1);
+        go(row_quant_reg_kernel<T, SM, 256, 8, FMT>, 1);
     else
-        launch_pdl(row_quant_kernel<T, SM>, dim3(row_grid(M)), dim3(kThreads), 0, st, X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
+        launch_pdl(row_quant_kernel<T, SM, FMT>, dim3(row_grid(M)), dim3(kThreads), 0, st, X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
     return check_launch(name);
 }
 
-template <int SM>
+template <int SM, int FMT = kI8>
 sq_status_t quantize_dt(sq_dtype_t dt, const void* X, int64_t M, int64_t K, int64_t ld, const float* s,
                         int per_row, const float* static_qs, int8_t* Q, float* qs_out, void* ws,
                         cudaStream_t st, const char* name) {
     switch (dt) {
-        case SQ_F16: return quantize<__half, SM>(X, M, K, ld, s, per_row, static_qs, Q, qs_out, ws, st, name);
+        case SQ_F16: return quantize<__half, SM, FMT>(X, M, K, ld, s, per_row, static_qs, Q, qs_out, ws, st, name);
         case SQ_BF16:
-            return quantize<__nv_bfloat16, SM>(X, M, K, ld, s, per_row, static_qs, Q, qs_out, ws, st, name);
-        case SQ_F32: return quantize<float, SM>(X, M, K, ld, s, per_row, static_qs, Q, qs_out, ws, st, name);
+            return quantize<__nv_bfloat16, SM, FMT>(X, M, K, ld, s, per_row, static_qs, Q, qs_out, ws, st, name);
+        case SQ_F32: return quantize<float, SM, FMT>(X, M, K, ld, s, per_row, static_qs, Q, qs_out, ws, st, name);
         default: return set_error(SQ_ERR_INVALID_ARG, "%s: dtype must be F16, BF16 or F32", name);
     }
 }
@@ -364,10 +400,51 @@ sq_status_t sq_quantize_act(const void* X, sq_dtype_t dt, int64_t M, int64_t K, 
                                          name);
 }
 
+sq_status_t sq_quantize_weight_fp8(const void* W, sq_dtype_t dt, int64_t N, int64_t K, const float* s,
+                                   int per_channel, uint8_t* Wq, float* qs_w, void* workspace, size_t ws_bytes,
+                                   sq_stream_t stream) {
+    const char* name = "sq_quantize_weight_fp8";
+    SQ_REQUIRE((W && Wq && qs_w) || N == 0, SQ_ERR_INVALID_ARG, "%s: null pointer", name);
+    SQ_REQUIRE(N >= 0 && K > 0 && K % 16 == 0, SQ_ERR_UNSUPPORTED_SHAPE, "%s: need K > 0 and K %% 16 == 0", name);
+    SQ_REQUIRE(sq::aligned16(W) && sq::aligned16(Wq) && (!s || sq::aligned16(s)), SQ_ERR_ALIGNMENT,
+               "%s: W, Wq and s must be 16-byte aligned", name);
+    SQ_REQUIRE(per_channel || (workspace && ws_bytes >= sq::kStatusBytes), SQ_ERR_INVALID_ARG,
+               "%s: per-tensor quantisation needs a workspace of %zu bytes", name, sq::kStatusBytes);
+    if (N == 0) return SQ_OK;
+    cudaStream_t st = sq::as_cuda(stream);
+    int8_t* Q = reinterpret_cast<int8_t*>(Wq);
+    if (s)
+        return sq::quantize_dt<sq::kMul, sq::kE4M3>(dt, W, N, K, K, s, per_channel, nullptr, Q, qs_w, workspace, st,
+                                                   name);
+    return sq::quantize_dt<sq::kNoScale, sq::kE4M3>(dt, W, N, K, K, nullptr, per_channel, nullptr, Q, qs_w,
+                                                    workspace, st, name);
+}
+
+sq_status_t sq_quantize_act_fp8(const void* X, sq_dtype_t dt, int64_t M, int64_t K, int64_t ldx, const float* s,
+                                int per_token, const float* static_qs, uint8_t* Xq, float* qs_x, void* workspace,
+                                size_t ws_bytes, sq_stream_t stream) {
+    const char* name = "sq_quantize_act_fp8";
+    SQ_REQUIRE((X && Xq && qs_x) || M == 0, SQ_ERR_INVALID_ARG, "%s: null pointer", name);
+    SQ_REQUIRE(M >= 0 && K > 0 && K % 16 == 0 && ldx >= K && ldx % 8 == 0, SQ_ERR_UNSUPPORTED_SHAPE,
+               "%s: need K > 0, K %% 16 == 0, ldx >= K, ldx %% 8 == 0", name);
+    SQ_REQUIRE(sq::aligned16(X) && sq::aligned16(Xq) && (!s || sq::aligned16(s)), SQ_ERR_ALIGNMENT,
+               "%s: X, Xq and s must be 16-byte aligned", name);
+    SQ_REQUIRE(per_token || static_qs || (workspace && ws_bytes >= sq::kStatusBytes), SQ_ERR_INVALID_ARG,
+               "%s: dynamic per-tensor quantisation needs a workspace of %zu bytes", name, sq::kStatusBytes);
+    if (M == 0) return SQ_OK;
+    cudaStream_t st = sq::as_cuda(stream);
+    int8_t* Q = reinterpret_cast<int8_t*>(Xq);
+    if (s)
+        return sq::quantize_dt<sq::kDiv, sq::kE4M3>(dt, X, M, K, ldx, s, per_token, static_qs, Q, qs_x, workspace,
+                                                    st, name);
+    return sq::quantize_dt<sq::kNoScale, sq::kE4M3>(dt, X, M, K, ldx, nullptr, per_token, static_qs, Q, qs_x,
+                                                    workspace, st, name);
+}
+
 sq_status_t sq_scale_from_absmax(const float* absmax, int64_t n, float* qs_out, sq_stream_t stream) {
     SQ_REQUIRE(absmax && qs_out, SQ_ERR_INVALID_ARG, "sq_scale_from_absmax: null pointer");
     SQ_REQUIRE(n > 0, SQ_ERR_UNSUPPORTED_SHAPE, "sq_scale_from_absmax: n must be > 0");
-    sq::launch_pdl(sq::scale_from_absmax_kernel, dim3(1), dim3(sq::kThreads), 0, sq::as_cuda(stream), absmax, n, qs_out);
+    sq::launch_pdl(sq::scale_from_absmax_kernel<sq::kI8>, dim3(1), dim3(sq::kThreads), 0, sq::as_cuda(stream), absmax, n, qs_out);
     return sq::check_launch("sq_scale_from_absmax");
 }
 

@@ -1,4 +1,6 @@
-// a3: smoothing factors and the offline folds.
+// Smoothing factors and the offline folds, including the fold into the
+// previous linear layer ("大语言模型量化技术（四）：SmoothQuant", section
+// 融入前序线性层的权重: up_proj's output channel j, or v_proj's, divided by s_j).
 //
 // s_j = x_j^alpha / w_j^(1-alpha) ("大语言模型量化技术（四）：SmoothQuant", section
 // 缩放因子; lpnh.cn SmoothQuant article §2.1) with clamp(min=1e-5) on both
@@ -73,6 +75,32 @@ __global__ void fold_norm_kernel(const float* __restrict__ g, const float* __res
     }
 }
 
+// Fold into the previous linear: row n of the previous layer divided by s_n (and its bias).
+template <typename T>
+__global__ void fold_prev_kernel(const T* __restrict__ W, int64_t N, int64_t K, const float* __restrict__ bias,
+                                 const float* __restrict__ s, float* __restrict__ Wp, float* __restrict__ bias_out) {
+    pdl_wait();
+    pdl_trigger();
+    constexpr int V = Vec<T>::N;
+    const int64_t nvec = N * K / V;
+    for (int64_t v = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; v < nvec;
+         v += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t e0 = v * V;
+        const int64_t n = e0 / K;  // K % V == 0: a vector never crosses a row
+        const float sn = __ldg(s + n);
+        float f[V];
+        unpack<T>(ldg_nc_v4(W + e0), f);
+#pragma unroll
+        for (int e = 0; e < V; ++e) f[e] = __fdiv_rn(f[e], sn);
+#pragma unroll
+        for (int e = 0; e < V; e += 4)
+            *reinterpret_cast<float4*>(Wp + e0 + e) = make_float4(f[e], f[e + 1], f[e + 2], f[e + 3]);
+    }
+    if (bias)
+        for (int64_t n = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; n < N; n += (int64_t)gridDim.x * blockDim.x)
+            bias_out[n] = __fdiv_rn(bias[n], s[n]);
+}
+
 int grid_for(int64_t n, int threads) {
     int64_t b = (n + threads - 1) / threads;
     const int64_t cap = (int64_t)num_sms() * 16;
@@ -118,6 +146,33 @@ sq_status_t sq_fold_weight(const void* W, sq_dtype_t dt, int64_t N, int64_t K, c
         default: return sq::set_error(SQ_ERR_INVALID_ARG, "sq_fold_weight: dtype must be F16, BF16 or F32");
     }
     return sq::check_launch("sq_fold_weight");
+}
+
+sq_status_t sq_fold_prev_linear(const void* W, sq_dtype_t dt, int64_t N, int64_t K, const float* bias,
+                                const float* s, float* Wp_out, float* bias_out, sq_stream_t stream) {
+    SQ_REQUIRE(W && s && Wp_out, SQ_ERR_INVALID_ARG, "sq_fold_prev_linear: null pointer");
+    SQ_REQUIRE((bias == nullptr) == (bias_out == nullptr), SQ_ERR_INVALID_ARG,
+               "sq_fold_prev_linear: bias and bias_out must both be given or both be NULL");
+    SQ_REQUIRE(N > 0 && K > 0 && K % 8 == 0, SQ_ERR_UNSUPPORTED_SHAPE, "sq_fold_prev_linear: need N, K > 0, K %% 8 == 0");
+    SQ_REQUIRE(sq::aligned16(W) && sq::aligned16(Wp_out), SQ_ERR_ALIGNMENT, "sq_fold_prev_linear: unaligned pointer");
+    cudaStream_t st = sq::as_cuda(stream);
+    const int64_t n = N * K;
+    switch (dt) {
+        case SQ_F16:
+            sq::launch_pdl(sq::fold_prev_kernel<__half>, dim3(sq::grid_for(n / 8, 256)), dim3(256), 0, st,
+                           static_cast<const __half*>(W), N, K, bias, s, Wp_out, bias_out);
+            break;
+        case SQ_BF16:
+            sq::launch_pdl(sq::fold_prev_kernel<__nv_bfloat16>, dim3(sq::grid_for(n / 8, 256)), dim3(256), 0, st,
+                           static_cast<const __nv_bfloat16*>(W), N, K, bias, s, Wp_out, bias_out);
+            break;
+        case SQ_F32:
+            sq::launch_pdl(sq::fold_prev_kernel<float>, dim3(sq::grid_for(n / 4, 256)), dim3(256), 0, st,
+                           static_cast<const float*>(W), N, K, bias, s, Wp_out, bias_out);
+            break;
+        default: return sq::set_error(SQ_ERR_INVALID_ARG, "sq_fold_prev_linear: dtype must be F16, BF16 or F32");
+    }
+    return sq::check_launch("sq_fold_prev_linear");
 }
 
 sq_status_t sq_fold_norm(const float* gamma, const float* beta, const float* s, int64_t K,

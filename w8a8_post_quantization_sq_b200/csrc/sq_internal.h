@@ -43,9 +43,29 @@ struct GemmEpilogue {
     const float* xo = nullptr;  // [M, kOutlierCap] fp32 copies of X[:, O]
     const float* wo = nullptr;  // [kOutlierCap, wo_ld] fp32 copies of W[:, O]^T
     int64_t wo_ld = 0;          // multiple of 256, >= N
+    int kind = 0;               // 0: int8 operands, int32 sums; 1: FP8 E4M3 operands, fp32 sums
+    int64_t batch = 1;          // independent problems; operands [batch, rows, K], scales [batch, rows]
+    int64_t y_bstride = 0;      // elements between the batches of Y
 };
 
+// How the GEMM covers a problem: tile width, grid, and how many trailing
+// tiles are cut by k-blocks (stream-K), with the scratch that needs.
+struct GemmPlan {
+    int bn = 256;
+    int tiles = 0;
+    int grid = 0;
+    int sk_tiles = 0;
+    size_t sk_cnt_bytes = 0;  // arrival counters per tile region (zero between launches)
+    size_t sk_bytes = 0;      // counters + parked partial sums
+};
+GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int64_t batch);
+// Workspace of sq_gemm_w8a8 / sq_gemm_fp8: the status header plus the
+// stream-K scratch of the plan.
+size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+// status_word: the caller's workspace (ws_bytes); the stream-K scratch, if
+// the plan has one and it fits, follows the 256-byte header.
 sq_status_t launch_gemm_w8a8(const int8_t* Xq, const int8_t* Wq, int64_t M, int64_t N, int64_t K,
-                             const GemmEpilogue& ep, int* status_word, cudaStream_t stream);
+                             const GemmEpilogue& ep, int* status_word, size_t ws_bytes, cudaStream_t stream);
 
 }  // namespace sq

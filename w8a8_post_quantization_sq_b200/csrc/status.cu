@@ -57,7 +57,7 @@ int sq_version(void) { return 100; }
 
 size_t sq_workspace_size(sq_op_t op, int64_t M, int64_t N, int64_t K) {
     switch (op) {
-        case SQ_OP_GEMM: return sq::kStatusBytes;
+        case SQ_OP_GEMM: return sq::gemm_workspace_bytes(M, N, K);
         case SQ_OP_QUANT_ACT: return sq::kStatusBytes;
         case SQ_OP_QUANT_WEIGHT: return sq::kStatusBytes;
         case SQ_OP_LLMINT8_DETECT: return sq::detect_workspace_bytes(M, K);
