@@ -75,10 +75,13 @@ def test_workspace_sizes(L):
     assert full >= det + 2048 * 4096 + 2048 * 4
     assert L.sq_workspace_size(99, 1, 1, 1) == 0
     # GEMM plan on 148 SMs: 1024 x 7168 makes 224 tiles of 128 x 256, a last
-    # wave of 76 (half full), so those 76 are cut by k-blocks: arrival
-    # counters for 76 tiles x 8 epilogue regions (padded to 256 bytes) plus
-    # two parked 128 x 256 int32 partials per CTA after the 256-byte header
-    assert L.sq_workspace_size(0, 1024, 7168, 7168) == 256 + 2560 + 148 * 2 * 128 * 256 * 4
+    # wave of 76 (half full); with a k-loop of 224 blocks those 76 are cut by
+    # k-blocks: arrival counters for 76 tiles x 8 epilogue regions (padded to
+    # 256 bytes) plus two parked 128 x 256 int32 partials per CTA after the
+    # 256-byte header
+    assert L.sq_workspace_size(0, 1024, 7168, 28672) == 256 + 2560 + 148 * 2 * 128 * 256 * 4
+    # the same tiles with 56 k-blocks stay whole (measured faster)
+    assert L.sq_workspace_size(0, 1024, 7168, 7168) == 256
     # 2048 x 16384: 1024 tiles, last wave 136 of 148: whole tiles only
     assert L.sq_workspace_size(0, 2048, 16384, 4096) == 256
     # 4096 x 36864: 4608 tiles, 97 % of the waves busy: whole tiles only

@@ -462,9 +462,10 @@ def test_gemm_deterministic():
     assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
 
 
-# shapes whose last wave of whole tiles is at most three quarters full: its
-# tiles are cut by k-blocks (ragged M and K; pieces of 2 to 30 k-blocks)
-SK_SHAPES = [(1029, 7168, 2064), (260, 13000, 8192), (2560, 4096, 2048)]
+# shapes whose last wave of whole tiles is at most three quarters full, with
+# k-loops of 128 blocks or more: that wave is cut by k-blocks (ragged M and K;
+# pieces of 4 to 100 k-blocks)
+SK_SHAPES = [(1029, 7168, 16400), (260, 13000, 16384), (2560, 4096, 16384)]
 
 
 @pytest.mark.parametrize("M,N,K", SK_SHAPES)

@@ -16,7 +16,7 @@
 // 2^n. Every step is one correctly rounded fp32 operation, so h, the scales
 // and the codes are bit-equal to a CPU evaluation of the same sequence.
 //
-// One 128-thread block per row, rows strided over the grid. Up to I = 8192
+// One 256-thread block per row, rows strided over the grid. Up to I = 16384
 // the thread's h values stay in registers between the absmax and the codes;
 // longer rows compute h twice.
 #include "sq_common.cuh"
@@ -24,7 +24,7 @@
 namespace sq {
 namespace {
 
-constexpr int kT = 128;
+constexpr int kT = 256;
 
 struct ActArgs {
     int64_t M, I, lda;
@@ -73,14 +73,16 @@ __device__ __forceinline__ void act8(const T* __restrict__ A, const ActArgs& a, 
     }
 }
 
-__device__ __forceinline__ float block_max4(float v, float* sh) {
+__device__ __forceinline__ float block_max(float v, float* sh) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     if (lane == 0) sh[warp] = v;
     __syncwarp();
     __syncthreads();
-    const float r = fmaxf(fmaxf(sh[0], sh[1]), fmaxf(sh[2], sh[3]));
+    float r = sh[0];
+#pragma unroll
+    for (int w = 1; w < kT / 32; ++w) r = fmaxf(r, sh[w]);
     __syncwarp();
     __syncthreads();  // sh is free again for the next row
     return r;
@@ -105,7 +107,7 @@ act_quant_kernel(const T* __restrict__ A, ActArgs a) {
     pdl_wait();
     pdl_trigger();
     extern __shared__ float amax_sh[];  // [I] running max |h| of the block (calibration mode)
-    __shared__ float sh[4];
+    __shared__ float sh[kT / 32];
     const int t = threadIdx.x;
     const int nch = (int)(a.I / 8);
     if (a.absmax) {
@@ -141,6 +143,7 @@ act_quant_kernel(const T* __restrict__ A, ActArgs a) {
                 }
             }
         } else {
+#pragma unroll 4
             for (int ch = t; ch < nch; ch += kT) {
                 float h[8];
                 act8<T, ACT>(A, a, row, (int64_t)ch * 8, h);
@@ -150,7 +153,7 @@ act_quant_kernel(const T* __restrict__ A, ActArgs a) {
         if (!a.Xq) continue;
         float qs;
         if (a.per_token) {
-            qs = __fdiv_rn(127.0f, fmaxf(block_max4(m, sh), 1e-8f));
+            qs = __fdiv_rn(127.0f, fmaxf(block_max(m, sh), 1e-8f));
             if (t == 0) a.qs_x[row] = qs;
         } else {
             qs = *a.static_qs;
@@ -164,6 +167,7 @@ act_quant_kernel(const T* __restrict__ A, ActArgs a) {
                 if (ch < nch) *reinterpret_cast<uint2*>(q + ch * 8) = codes8(hk[i], qs, !a.per_token);
             }
         } else {
+#pragma unroll 4
             for (int ch = t; ch < nch; ch += kT) {
                 float h[8];
                 act8<T, ACT>(A, a, row, (int64_t)ch * 8, h);

@@ -836,12 +836,14 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int64_t batch) {
     // Stream-K for the remainder: when the last wave of whole tiles would be
     // at most three quarters full (and the waves average under 90 % busy),
     // its tiles are cut by k-blocks into one range per CTA, every CTA
-    // starting them together after the whole waves. A k-loop of 16 blocks or
-    // more pays for parking and adding the partial sums.
+    // starting them together after the whole waves. Measured on B200 it pays
+    // only for long k-loops (1024 x 7168 x 28672: 186 -> 178 us); at 56
+    // k-blocks the pieces' scattered k-offsets cost more L2 reuse than the
+    // idle tail they remove, so it needs 128 k-blocks or more.
     const int64_t kb = (K + BK - 1) / BK;
     const int64_t rem = tiles % pl.grid;
     const double eff = (double)tiles / (double)(((tiles + pl.grid - 1) / pl.grid) * pl.grid);
-    if (batch == 1 && pl.grid == sms && tiles > pl.grid && kb >= 16 && rem > 0 && 4 * rem <= 3 * (int64_t)pl.grid &&
+    if (batch == 1 && pl.grid == sms && tiles > pl.grid && kb >= 128 && rem > 0 && 4 * rem <= 3 * (int64_t)pl.grid &&
         eff < 0.9 && rem * kb >= pl.grid && rem * kb < (1ll << 31)) {
         pl.sk_tiles = (int)rem;
         pl.sk_cnt_bytes = ((size_t)rem * kEpiWarps * sizeof(int) + 255) / 256 * 256;
