@@ -61,6 +61,20 @@ def peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
+# ------------------------------------------------------------------ ranks
+def max_over_ranks(x, dev):
+    """The maximum of a per-rank number over all ranks (timing: the slowest
+    rank's clock decides); x itself with one rank."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ------------------------------------------------------------------ DRAM traffic
 GEMM_SOURCES = ["w8a8_post_quantization_sq_b200/csrc/gemm_w8a8.cu", "w8a8_post_quantization_sq_b200/csrc/sq_common.cuh",
                 "w8a8_post_quantization_sq_b200/csrc/sq_wait.cuh", "w8a8_post_quantization_sq_b200/csrc/sq_internal.h"]
@@ -344,11 +358,7 @@ def run_ours(args, rank, world, dev):
         dist.barrier()
     clk = clocks.stop() if clocks else None
     step_ms = [a.elapsed_time(b) for a, b in ev]
-    total_ms = sum(step_ms)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), dev)
     ms_per_step = total_ms / args.steps
 
     # e2e through the public API with host buffers: H2D of the inputs, the
@@ -373,10 +383,7 @@ def run_ours(args, rank, world, dev):
                 oh.copy_(o, non_blocking=True)
         e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = torch.tensor([e0.elapsed_time(e1) / e2e_steps], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-    e2e_ms = float(e2e_ms.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev)
 
     gm = np.array(gemm_ms)  # [steps, 4]
     gemm_ops = [2.0 * m * n * k for (m, n, k) in GEMMS[:4]]

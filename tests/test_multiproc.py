@@ -1,0 +1,72 @@
+"""Two-rank runs on CPU (gloo): the one exchange of sharded calibration and
+the benchmark's max-over-ranks timing."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _calib_rank(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        sys.path.insert(0, ROOT)
+        import oracle
+        from w8a8_post_quantization_sq_b200 import sharded
+        import bench
+
+        g = torch.Generator().manual_seed(5)
+        X = torch.randn((4 * 37, 96), generator=g)
+        X[:, 11] *= 80
+        X[3, 50] = -400.0    # the column's extreme sits in rank 0's shard ...
+        X[40, 51] = 800.0    # ... and this one in rank 1's
+        shard = X[rank * 37:(rank + 1) * 37] if rank < world - 1 else X[rank * 37:]
+        local = torch.from_numpy(oracle.col_absmax(shard.numpy()))
+        sharded.allreduce_max_(local)
+        full = oracle.col_absmax(X.numpy())
+        ok_calib = bool(np.array_equal(local.numpy(), full))
+        # the benchmark's timing: the max over the ranks of each rank's own time
+        t = bench.max_over_ranks(1.5 + rank, torch.device("cpu"))
+        out[rank] = (ok_calib, t)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_sharded_calibration_and_max_over_ranks():
+    world = 2
+    port = _free_port()
+    out = mp.Manager().dict()
+    mp.spawn(_calib_rank, args=(world, port, out), nprocs=world, join=True)
+    assert all(out[r][0] for r in range(world)), "sharded maxima differ from the maxima of all tokens"
+    assert [out[r][1] for r in range(world)] == [2.5, 2.5]
+
+
+def test_reference_arm_under_torchrun():
+    """`bench.py --impl reference` launched like the driver does for N = 2:
+    rank 0 prints one JSON line, rank 1 exits 0 without work."""
+    port = _free_port()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.join(ROOT, "bench.py"),
+           "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "0"]
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0

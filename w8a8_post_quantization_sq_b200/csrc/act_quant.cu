@@ -40,7 +40,12 @@ struct ActArgs {
 __device__ __forceinline__ float exp_fixed(float x) {
     if (x > 88.0f) return __int_as_float(0x7f800000);
     if (x < -87.0f) return 0.0f;
-    const float n = rintf(__fmul_rn(x, 0x1.715476p+0f));  // log2(e) in fp32; n in [-126, 127]
+    // n = x * log2(e) rounded to the nearest integer (ties to even): adding
+    // 1.5 * 2^23 rounds it into the low bits of the sum, which also hold n as
+    // an integer; this is rint() with two adds instead of conversions
+    const float sh = __fadd_rn(__fmul_rn(x, 0x1.715476p+0f), 12582912.0f);  // log2(e) in fp32
+    const float n = __fsub_rn(sh, 12582912.0f);                            // exact; in [-126, 127]
+    const int ni = __float_as_int(sh) - 0x4B400000;
     float r = __fmaf_rn(-n, 0x1.62e000p-1f, x);            // ln 2, high part (12 bits)
     r = __fmaf_rn(-n, 0x1.0bfbe8p-15f, r);                 // ln 2, low part
     float p = 0x1.a01a02p-13f;                             // 1/7!
@@ -51,7 +56,7 @@ __device__ __forceinline__ float exp_fixed(float x) {
     p = __fmaf_rn(p, r, 0.5f);
     p = __fmaf_rn(p, r, 1.0f);
     p = __fmaf_rn(p, r, 1.0f);
-    return __fmul_rn(p, __int_as_float(((int)n + 127) << 23));
+    return __fmul_rn(p, __int_as_float((ni + 127) << 23));
 }
 
 __device__ __forceinline__ float silu(float g) { return __fdiv_rn(g, __fadd_rn(1.0f, exp_fixed(-g))); }
