@@ -841,3 +841,111 @@ def test_bmm_attention(out_dtype):
             assert_close_f32(O[h, rows].contiguous(), yo[h], np.abs(yo[h]))
         else:
             assert_close_16(O[h, rows].contiguous(), yo[h], out_dtype)
+
+
+# ---------------------------------------------------------------- the benchmark's whole step
+def test_bench_step_against_oracle():
+    """The benchmark's step (every row, on its streams, captured in a CUDA
+    graph) against the oracle on the same inputs: the weight side in full, the
+    token side on sampled rows. Stages after a 16-bit GEMM output take the
+    device's output as their input, so each stage is held to its own bar."""
+    import bench
+
+    dev = torch.device(DEV, 0)
+    L = bench.Layer(dev)
+    L.step()
+    torch.cuda.synchronize()
+    eager = [y.clone() for y in L.outputs()]
+    stream = torch.cuda.Stream()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        L.step()  # warm-up on the capture stream
+    torch.cuda.synchronize()
+    with torch.cuda.graph(graph, stream=stream):
+        L.step()
+    for _ in range(2):
+        for y in L.outputs():
+            y.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        for a, b in zip(eager, L.outputs()):
+            assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+    d = {k: v for k, v in L.d.items() if torch.is_tensor(v)}
+    d = {k: v.cpu() for k, v in d.items()}
+    W = {k: v.cpu() for k, v in L.d["W"].items()}
+    eps, alpha, I = L.d["eps"], L.d["alpha"], L.I
+    rows = [0, 1, 127, 128, 1029, bench.M_TOKENS - 1]
+    # calibration input, maxima, smoothing factors, folded gamma
+    s, gp = {}, {}
+    V16 = {}
+    for k, w in (("attn", "qkv"), ("mlp", "gateup")):
+        V = oracle.norm_smooth_quant(d["h_" + k], oracle.RMSNORM, d["gamma_" + k].numpy(), None, eps,
+                                     quantize=False, want_v=True)["V"]
+        V16[k] = torch.from_numpy(V).to(torch.bfloat16)
+        assert np.array_equal(npu16(L.V[k]), npu16(V16[k]))
+        xmax = oracle.col_absmax(V16[k])
+        assert np.array_equal(npf(L.xmax[k]), xmax)
+        wmax = oracle.col_absmax(W[w])
+        assert np.array_equal(npf(L.wmax[k]), wmax)
+        s[k] = oracle.smooth_scales(xmax, wmax, alpha)
+        assert np.array_equal(npf(L.s[k]), s[k])
+        gp[k], _ = oracle.fold_norm(d["gamma_" + k].numpy(), None, s[k])
+        assert np.array_equal(npf(L.gp[k]), gp[k])
+    # weight side: the down_proj factors s_down are set-up state, taken from the
+    # device; checked here on sampled channels against the oracle's own
+    # calibration (through a 16-bit GEMM output, so to 1e-2 relative: a one-ulp
+    # bf16 difference of gate or up moves a column maximum by about 2^-8)
+    s_down = npf(L.s_down)
+    js = [0, 5, 1000, I - 1]
+    Vc = oracle.norm_smooth_quant(d["h_calib"], oracle.RMSNORM, d["gamma_mlp"].numpy(), None, eps,
+                                  quantize=False, want_v=True)["V"]
+    Xc, qc = oracle.quantize_act(torch.from_numpy(Vc).to(torch.bfloat16).float().numpy(), None, per_token=True)
+    Wc, qwc = oracle.quantize_weight(W["gateup"], True)
+    sel = js + [I + j for j in js]
+    yc = oracle.dequant(oracle.gemm_i8(Xc, Wc[sel]), qc, qwc[sel])
+    yc16 = torch.from_numpy(oracle.round_bf16_bits(yc).view(np.int16)).view(torch.bfloat16).float().numpy()
+    hmax = oracle.act_quant(yc16, oracle.SWIGLU, quantize=False, absmax=np.zeros(len(js), np.float32))["absmax"]
+    s_js = oracle.smooth_scales(hmax, oracle.col_absmax(W["down"])[js], alpha)
+    assert np.allclose(s_down[js], s_js, rtol=1e-2, atol=0)
+    up_f, _ = oracle.fold_prev_linear(W["gateup"][I:], s_down)
+    assert np.array_equal(npf(L.W_up_f), up_f)
+    ref_w = {
+        "qkv": oracle.fold_weight(W["qkv"], s["attn"]),
+        "gateup": np.concatenate([oracle.fold_weight(W["gateup"][:I], s["mlp"]), oracle.fold_weight(up_f, s["mlp"])]),
+        "o": oracle.f32(W["o"]),
+        "down": oracle.fold_weight(W["down"], s_down),
+    }
+    Wq, qw = {}, {}
+    for w, Wp in ref_w.items():
+        Wq[w], qw[w] = oracle.quantize_weight(Wp, True)
+        assert np.array_equal(L.Wq[w].cpu().numpy(), Wq[w]), w
+        assert np.array_equal(npf(L.qw[w]), qw[w]), w
+    # token side on sampled rows
+    for k, w in (("attn", "qkv"), ("mlp", "gateup")):
+        r = oracle.norm_smooth_quant(d["h_" + k][rows], oracle.RMSNORM, gp[k], None, eps, True)
+        assert np.array_equal(L.Xq[k][rows].cpu().numpy(), r["Xq"])
+        assert np.array_equal(npf(L.qx[k][rows]), r["qs"])
+        y = oracle.dequant(oracle.gemm_i8(r["Xq"], Wq[w]), r["qs"], qw[w])
+        assert_close_16(L.Y[w][rows], y, torch.bfloat16)
+    xo, so = L.act_in["o"]
+    xs, ss = xo[rows].cpu().numpy(), npf(so[rows])
+    assert_close_16(L.Y["o"][rows], oracle.dequant(oracle.gemm_i8(xs, Wq["o"]), ss, qw["o"]), torch.bfloat16)
+    a = oracle.act_quant(npf(L.Y["gateup"][rows]), oracle.SWIGLU)
+    assert np.array_equal(L.Xq_down[rows].cpu().numpy(), a["Xq"])
+    assert np.array_equal(npf(L.qx_down[rows]), a["qs"])
+    y = oracle.dequant(oracle.gemm_i8(a["Xq"], Wq["down"]), a["qs"], qw["down"])
+    assert_close_16(L.Y["down"][rows], y, torch.bfloat16)
+    # LLM.int8 of the q/k/v projection: outlier set over every token
+    idx = oracle.llmint8_outliers(V16["attn"], 6.0, 0.0)
+    n = int(L.nidx.item())
+    assert n == idx.size and L.idx[:n].cpu().numpy().tolist() == idx.tolist()
+    Xs = V16["attn"][rows]
+    Xq8, qx8 = oracle.llmint8_quant_rows(Xs, idx)
+    Wq8, qw8 = oracle.llmint8_quant_weight(W["qkv"], idx)
+    acc = oracle.gemm_i8(Xq8, Wq8)
+    y = oracle.llmint8_combine(acc, qx8, qw8, Xs, W["qkv"], idx)
+    Xf, Wf = npf(Xs).astype(np.float64), npf(W["qkv"]).astype(np.float64)
+    terms = np.abs(oracle.dequant(acc, qx8, qw8)) + np.abs(Xf[:, idx]) @ np.abs(Wf[:, idx]).T
+    assert_close_16(L.Y["llm"][rows], y, torch.bfloat16, terms)
+    del graph

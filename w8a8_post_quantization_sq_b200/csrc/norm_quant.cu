@@ -26,7 +26,8 @@
 //     reach shared memory through a ring of buffers, one bulk copy (TMA
 //     engine, cp.async.bulk) per row issued R rows ahead, so several rows per
 //     block are in flight while the block reduces and quantises; gamma' of a
-//     thread's chunks lives in its registers for the whole launch.
+//     thread's chunks lives in its registers for the whole launch, beta' in
+//     shared memory.
 // The codes are written 8 bytes per chunk, the per-token scale once per row.
 #include "sq_common.cuh"
 
@@ -63,44 +64,72 @@ __device__ __forceinline__ float warp_max(float v) {
     return v;
 }
 
-// v_j of one 8-element chunk from its fp32 inputs f (v may alias f); g holds
-// gamma'_j of the chunk, beta (shared or global memory, or null) beta'
-template <bool LN>
-__device__ __forceinline__ void compute_v_f(const float* f, int ch, const float* beta, const float* g, float mu,
+// max(a, b, c) in one instruction (exact; the order of a max does not matter)
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+// max(m, |v_0|, ..., |v_7|)
+__device__ __forceinline__ float absmax8(float m, const float* v) {
+    const float m0 = max3f(m, fabsf(v[0]), fabsf(v[1]));
+    const float m1 = max3f(fabsf(v[2]), fabsf(v[3]), fabsf(v[4]));
+    return max3f(max3f(m0, fabsf(v[5]), fabsf(v[6])), m1, fabsf(v[7]));
+}
+
+// v_j of one 8-element chunk from d_j = x_j - mu (LayerNorm) or x_j
+// (RMSNorm), given r: (d * r) * gamma' (+ beta'). g holds gamma'_j of the
+// chunk; b_lo / b_hi point at beta'_j of its first and last four elements
+// (null: no shift). v may alias d.
+__device__ __forceinline__ void compute_v_d(const float* d, const float4* b_lo, const float4* b_hi, const float* g,
                                             float r, float* v) {
     const uint64_t r2 = pk2(r, r);
-    if constexpr (LN) {
-        const uint64_t nmu2 = pk2(-mu, -mu);  // x + (-mu) is the IEEE x - mu
-        if (beta) {
-            // the last product feeds an add: keep those two steps scalar
-            const float4 b0 = *reinterpret_cast<const float4*>(beta + ch * 8);
-            const float4 b1 = *reinterpret_cast<const float4*>(beta + ch * 8 + 4);
-            const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+    if (b_lo) {
+        // the last product feeds an add: keep those two steps scalar
+        const float4 b0 = *b_lo, b1 = *b_hi;
+        const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-            for (int e = 0; e < 8; e += 2) {
-                float u0, u1;
-                upk2(mul2(add2(pk2(f[e], f[e + 1]), nmu2), r2), u0, u1);
-                v[e] = __fadd_rn(__fmul_rn(u0, g[e]), b[e]);
-                v[e + 1] = __fadd_rn(__fmul_rn(u1, g[e + 1]), b[e + 1]);
-            }
-        } else {
-#pragma unroll
-            for (int e = 0; e < 8; e += 2)
-                upk2(mul2(mul2(add2(pk2(f[e], f[e + 1]), nmu2), r2), pk2(g[e], g[e + 1])), v[e], v[e + 1]);
+        for (int e = 0; e < 8; e += 2) {
+            float u0, u1;
+            upk2(mul2(pk2(d[e], d[e + 1]), r2), u0, u1);
+            v[e] = __fadd_rn(__fmul_rn(u0, g[e]), b[e]);
+            v[e + 1] = __fadd_rn(__fmul_rn(u1, g[e + 1]), b[e + 1]);
         }
     } else {
 #pragma unroll
-        for (int e = 0; e < 8; e += 2) upk2(mul2(mul2(pk2(f[e], f[e + 1]), r2), pk2(g[e], g[e + 1])), v[e], v[e + 1]);
+        for (int e = 0; e < 8; e += 2) upk2(mul2(mul2(pk2(d[e], d[e + 1]), r2), pk2(g[e], g[e + 1])), v[e], v[e + 1]);
+    }
+}
+
+// d_j = x_j - mu for the eight elements of a chunk, in place
+__device__ __forceinline__ void center8(float* f, float mu) {
+    const uint64_t nmu2 = pk2(-mu, -mu);  // x + (-mu) is the IEEE x - mu
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) upk2(add2(pk2(f[e], f[e + 1]), nmu2), f[e], f[e + 1]);
+}
+
+// v_j of one chunk from its fp32 inputs f (v may alias f)
+template <bool LN>
+__device__ __forceinline__ void compute_v_f(const float* f, const float4* b_lo, const float4* b_hi, const float* g,
+                                            float mu, float r, float* v) {
+    if constexpr (LN) {
+        float d[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) d[e] = f[e];
+        center8(d, mu);
+        compute_v_d(d, b_lo, b_hi, g, r, v);
+    } else {
+        compute_v_d(f, nullptr, nullptr, g, r, v);
     }
 }
 
 // the same from the chunk's 16-bit inputs
 template <typename T, bool LN>
-__device__ __forceinline__ void compute_v_g(const uint4& rw, int ch, const float* beta, const float* g, float mu,
-                                            float r, float* v) {
+__device__ __forceinline__ void compute_v_g(const uint4& rw, const float4* b_lo, const float4* b_hi, const float* g,
+                                            float mu, float r, float* v) {
     float f[8];
     unpack<T>(rw, f);
-    compute_v_f<LN>(f, ch, beta, g, mu, r, v);
+    compute_v_f<LN>(f, b_lo, b_hi, g, mu, r, v);
 }
 
 __device__ __forceinline__ void load_gamma(const NormArgs& a, int ch, float* g) {
@@ -110,12 +139,21 @@ __device__ __forceinline__ void load_gamma(const NormArgs& a, int ch, float* g) 
     g[4] = g1.x; g[5] = g1.y; g[6] = g1.z; g[7] = g1.w;
 }
 
-// v_j of one 8-element chunk, gamma'_j read from a.gamma
+// v_j of one 8-element chunk, gamma'_j and beta'_j read from global memory
 template <typename T, bool LN>
 __device__ __forceinline__ void compute_v(const uint4& rw, int ch, const NormArgs& a, float mu, float r, float* v) {
     float g[8];
     load_gamma(a, ch, g);
-    compute_v_g<T, LN>(rw, ch, a.beta, g, mu, r, v);
+    const float4* bl = a.beta ? reinterpret_cast<const float4*>(a.beta) + ch * 2 : nullptr;
+    compute_v_g<T, LN>(rw, bl, bl + 1, g, mu, r, v);
+}
+
+// Per-chunk parameters staged in shared memory as two planes of float4 (the
+// first and last four of every chunk), so a warp reading the chunks of 32
+// consecutive lanes touches 512 consecutive bytes per plane: no bank conflicts.
+__device__ __forceinline__ void stage_planes(float4* dst, const float* src, int nch, int tid, int nthreads) {
+    for (int j = tid; j < nch * 2; j += nthreads)
+        dst[(j & 1) * nch + (j >> 1)] = __ldg(reinterpret_cast<const float4*>(src) + j);
 }
 
 template <typename T>
@@ -184,10 +222,10 @@ norm_quant_warp_kernel(const T* __restrict__ H, NormArgs a) {
                 const float d = __fsub_rn(x, m_);
                 return __fmaf_rn(d, d, c);
             }), Kf);
-            r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(var, a.eps)));
+            r = __frcp_rn(__fsqrt_rn(__fadd_rn(var, a.eps)));
         } else {
             const float ms = __fdiv_rn(canon([](float x, float c) { return __fmaf_rn(x, x, c); }), Kf);
-            r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, a.eps)));
+            r = __frcp_rn(__fsqrt_rn(__fadd_rn(ms, a.eps)));
         }
         float m = 0.0f;
         if ((a.Xq && a.per_token) || a.absmax || a.V) {
@@ -198,7 +236,7 @@ norm_quant_warp_kernel(const T* __restrict__ H, NormArgs a) {
                     float v[8];
                     compute_v<T, LN>(raw[i], ch, a, mu, r, v);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(v[e]));
+                    m = absmax8(m, v);
                     if (a.absmax) {
 #pragma unroll
                         for (int e = 0; e < 8; ++e)
@@ -323,7 +361,9 @@ norm_quant_bulk_kernel(const T* __restrict__ H, NormArgs a, int R) {
     const uint32_t row_bytes = (uint32_t)(a.K * sizeof(T));
     float* amax_sh = reinterpret_cast<float*>(dsm + (size_t)R * row_bytes);
     // beta' (LayerNorm with a shift) staged once per block after the maxima
-    float* beta_sh = (LN && a.beta) ? amax_sh + (!QONLY && a.absmax ? a.K : 0) : nullptr;
+    float4* beta_sh = (LN && a.beta) ? reinterpret_cast<float4*>(amax_sh + (!QONLY && a.absmax ? a.K : 0)) : nullptr;
+    auto b_lo = [&](int ch) { return beta_sh ? beta_sh + ch : nullptr; };
+    auto b_hi = [&](int ch) { return beta_sh ? beta_sh + nch + ch : nullptr; };
     const int64_t G = gridDim.x;
     auto mine = [&](int c) { return FULL || t + c * kBlock < nch; };
     float g[C][8];
@@ -338,9 +378,7 @@ norm_quant_bulk_kernel(const T* __restrict__ H, NormArgs a, int R) {
     }
     if (!QONLY && a.absmax)
         for (int j = t; j < a.K; j += kBlock) amax_sh[j] = 0.0f;
-    if (beta_sh)
-        for (int j = t; j < nch * 2; j += kBlock)
-            reinterpret_cast<float4*>(beta_sh)[j] = __ldg(reinterpret_cast<const float4*>(a.beta) + j);
+    if (beta_sh) stage_planes(beta_sh, a.beta, nch, t, kBlock);
     __syncwarp();
     __syncthreads();
     if (t == 0)
@@ -384,29 +422,28 @@ norm_quant_bulk_kernel(const T* __restrict__ H, NormArgs a, int R) {
                 for (int e = 0; e < 8; ++e) acc = LN ? __fmaf_rn(f[e], 1.0f, acc) : __fmaf_rn(f[e], f[e], acc);
             }
         }
-        const float sum = canon_block_sum(acc, sh[0]);
-        if constexpr (KEEPV) refill();
+        auto rstd = [&](float s_) { return __frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(s_, Kf), a.eps))); };
         float mu = 0.0f, r;
         if constexpr (LN) {
-            mu = __fdiv_rn(sum, Kf);
+            mu = __fdiv_rn(canon_block_sum(acc, sh[0]), Kf);
+            if constexpr (KEEPV) refill();
             acc = 0.0f;
 #pragma unroll
             for (int c = 0; c < C; ++c) {
                 if (mine(c)) {
+                    // d = x - mu, kept in place of x when the row is in registers
                     float fl[8];
                     if constexpr (!KEEPV) unpack<T>(chunk(c), fl);
-                    const float* f = KEEPV ? vk[c] : fl;
+                    float* d = KEEPV ? vk[c] : fl;
+                    center8(d, mu);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const float d = __fsub_rn(f[e], mu);
-                        acc = __fmaf_rn(d, d, acc);
-                    }
+                    for (int e = 0; e < 8; ++e) acc = __fmaf_rn(d[e], d[e], acc);
                 }
             }
-            const float var = __fdiv_rn(canon_block_sum(acc, sh[1]), Kf);
-            r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(var, a.eps)));
+            r = rstd(canon_block_sum(acc, sh[1]));
         } else {
-            r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(sum, Kf), a.eps)));
+            r = rstd(canon_block_sum(acc, sh[0]));
+            if constexpr (KEEPV) refill();
         }
         // pass 2: v, its absmax, the optional outputs
         float m = 0.0f;
@@ -417,10 +454,10 @@ norm_quant_bulk_kernel(const T* __restrict__ H, NormArgs a, int R) {
                 if (mine(c)) {
                     float vl[8];
                     float* v = KEEPV ? vk[c] : vl;
-                    if constexpr (KEEPV) compute_v_f<LN>(vk[c], ch, beta_sh, g[c], mu, r, v);
-                    else compute_v_g<T, LN>(chunk(c), ch, beta_sh, g[c], mu, r, v);
+                    if constexpr (KEEPV) compute_v_d(vk[c], b_lo(ch), b_hi(ch), g[c], r, v);  // vk holds d
+                    else compute_v_g<T, LN>(chunk(c), b_lo(ch), b_hi(ch), g[c], mu, r, v);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(v[e]));
+                    m = absmax8(m, v);
                     if constexpr (!QONLY) {
                         if (a.absmax) {
                             float4* am = reinterpret_cast<float4*>(amax_sh + ch * 8);
@@ -454,7 +491,7 @@ norm_quant_bulk_kernel(const T* __restrict__ H, NormArgs a, int R) {
                         *reinterpret_cast<uint2*>(q + ch * 8) = codes8(vk[c], qs, !a.per_token);
                     } else {
                         float v[8];
-                        compute_v_g<T, LN>(chunk(c), ch, beta_sh, g[c], mu, r, v);
+                        compute_v_g<T, LN>(chunk(c), b_lo(ch), b_hi(ch), g[c], mu, r, v);
                         *reinterpret_cast<uint2*>(q + ch * 8) = codes8(v, qs, !a.per_token);
                     }
                 }
