@@ -13,10 +13,9 @@
 // Design (sm_100a):
 //   - persistent: one 320-thread CTA per SM loops over 128 x BN output tiles
 //     in a grouped raster (the CTAs running together share Xq rows and weight
-//     tiles in L2); whole tiles only: a stream-K split of the k-loop was
-//     measured slower on this part (pieces at scattered k-offsets lose the
-//     L2 reuse of whole tiles running in lockstep, and cost more than the
-//     idle tail they remove);
+//     tiles in L2); when the last wave of whole tiles would be mostly idle,
+//     that wave's tiles are cut by k-blocks into one range per CTA, run
+//     before the whole tiles (stream-K, see plan_gemm);
 //   - warp 0 (one lane) issues TMA loads of 128 x 128 int8 tiles of Xq and
 //     BN x 128 tiles of Wq (128-byte swizzle) into a 4-stage shared-memory
 //     ring guarded by mbarriers;
@@ -120,10 +119,12 @@ __device__ __forceinline__ int sk_owner(int x, const Params& p) {
     return (int)((((int64_t)x + 1) * (int64_t)gridDim.x + p.sk_iters - 1) / p.sk_iters - 1);
 }
 
-// This CTA's work, the same sequence for its three roles: whole tiles, then
-// the pieces of its stream-K range (a piece is the part of the range inside
-// one tile). slot = -1 for a whole tile; a piece is the CTA's first (slot 0)
-// or last (slot 1) piece: a range spans at most one whole tile between them.
+// This CTA's work, the same sequence for its three roles: the pieces of its
+// stream-K range first (a piece is the part of the range inside one tile),
+// then its whole tiles, so the parking of partial sums and the fix-up
+// epilogues overlap the whole tiles' MMAs instead of trailing the launch.
+// slot = -1 for a whole tile; a piece is the CTA's first (slot 0) or last
+// (slot 1) piece: a range spans at most one whole tile between them.
 template <bool SK>
 struct Segments {
     int tile_dp, it, end;
@@ -135,23 +136,22 @@ struct Segments {
         first = true;
     }
     __device__ bool next(const Params& p, int num_tiles, int& tile, int& k0, int& k1, int& slot) {
-        if (!SK || tile_dp < p.dp_tiles) {
-            tile = tile_dp;
-            k0 = 0;
-            k1 = p.num_kb;
-            slot = -1;
-            tile_dp += gridDim.x;
-            return tile < (SK ? p.dp_tiles : num_tiles);
+        if (SK && it < end) {
+            const int u = it / p.num_kb;
+            k0 = it - u * p.num_kb;
+            k1 = min(p.num_kb, k0 + (end - it));
+            tile = p.dp_tiles + u;
+            slot = (k0 == 0 && k1 == p.num_kb) ? -1 : (first ? 0 : 1);
+            first = false;
+            it += k1 - k0;
+            return true;
         }
-        if (it >= end) return false;
-        const int u = it / p.num_kb;
-        k0 = it - u * p.num_kb;
-        k1 = min(p.num_kb, k0 + (end - it));
-        tile = p.dp_tiles + u;
-        slot = (k0 == 0 && k1 == p.num_kb) ? -1 : (first ? 0 : 1);
-        first = false;
-        it += k1 - k0;
-        return true;
+        tile = tile_dp;
+        k0 = 0;
+        k1 = p.num_kb;
+        slot = -1;
+        tile_dp += gridDim.x;
+        return tile < (SK ? p.dp_tiles : num_tiles);
     }
 };
 
@@ -835,16 +835,16 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int64_t batch) {
     pl.grid = (int)(tiles < sms ? tiles : sms);
     // Stream-K for the remainder: when the last wave of whole tiles would be
     // at most three quarters full (and the waves average under 90 % busy),
-    // its tiles are cut by k-blocks into one range per CTA, every CTA
-    // starting them together after the whole waves. Measured on B200 it pays
-    // only for long k-loops (1024 x 7168 x 28672: 186 -> 178 us); at 56
-    // k-blocks the pieces' scattered k-offsets cost more L2 reuse than the
-    // idle tail they remove, so it needs 128 k-blocks or more.
+    // its tiles are cut by k-blocks into one range per CTA, which every CTA
+    // runs before its whole tiles. Measured on B200: 1024 x 7168 x 7168
+    // (56 k-blocks) 54.1 -> 51.4 us, 1024 x 7168 x 28672 176 -> 174 us. Each
+    // CTA's range must hold 8 k-blocks or more, and the k-loop 32 or more,
+    // or the parking of partial sums costs more than the idle tail.
     const int64_t kb = (K + BK - 1) / BK;
     const int64_t rem = tiles % pl.grid;
     const double eff = (double)tiles / (double)(((tiles + pl.grid - 1) / pl.grid) * pl.grid);
-    if (batch == 1 && pl.grid == sms && tiles > pl.grid && kb >= 128 && rem > 0 && 4 * rem <= 3 * (int64_t)pl.grid &&
-        eff < 0.9 && rem * kb >= pl.grid && rem * kb < (1ll << 31)) {
+    if (batch == 1 && pl.grid == sms && tiles > pl.grid && kb >= 32 && rem > 0 && 4 * rem <= 3 * (int64_t)pl.grid &&
+        eff < 0.9 && rem * kb >= 8ll * pl.grid && rem * kb < (1ll << 31)) {
         pl.sk_tiles = (int)rem;
         pl.sk_cnt_bytes = ((size_t)rem * kEpiWarps * sizeof(int) + 255) / 256 * 256;
         pl.sk_bytes = pl.sk_cnt_bytes + (size_t)pl.grid * 2 * BM * pl.bn * sizeof(int);

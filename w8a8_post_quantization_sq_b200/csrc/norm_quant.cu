@@ -164,13 +164,24 @@ __device__ __forceinline__ void store_v16(const NormArgs& a, int64_t row, int ch
     *reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.V) + row * a.K + ch * 8) = make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+// int8 codes of eight values. Without a clip the products v * qs go two at a
+// time (packed multiply) into the scalar shifter add: a packed multiply feeding
+// a scalar add keeps its own rounding (the bit-exact parity tests hit many
+// exact ties here), unlike a packed multiply feeding a packed add.
 __device__ __forceinline__ uint2 codes8(const float* v, float qs, bool clip) {
     uint32_t b[8];
     if (clip) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) b[e] = quant_bits_clip(__fmul_rn(v[e], qs));
     } else {
-        quant_bits8_noclip(v, qs, b);
+        const uint64_t q2 = pk2(qs, qs);
+#pragma unroll
+        for (int e = 0; e < 8; e += 2) {
+            float t0, t1;
+            upk2(mul2(pk2(v[e], v[e + 1]), q2), t0, t1);
+            b[e] = quant_bits_noclip(t0);
+            b[e + 1] = quant_bits_noclip(t1);
+        }
     }
     return make_uint2(pack_low_bytes(b[0], b[1], b[2], b[3]), pack_low_bytes(b[4], b[5], b[6], b[7]));
 }
