@@ -368,7 +368,12 @@ SQ_API sq_status_t sq_llmint8_quant_weight(const void* W, sq_dtype_t dt, int64_t
  * (same dtype as X). Wq [N,K] int8, qs_w [N] fp32, cached_idx [K] int32 and
  * cached_n [1] int32 are caller-allocated device buffers that the library
  * maintains: they hold the int8 weight for the outlier set in cached_idx.
- * Set *cached_n = -1 (device) before the first call to mark the cache empty. */
+ * Set *cached_n = -1 (device) before the first call to mark the cache empty.
+ * wo (optional, may be NULL): a caller-allocated device buffer of
+ * 32 x ceil(N/256)*256 fp32 in which the library keeps the outlier input
+ * channels of W for the cached set, transposed (wo[o, n] = W[n, O_o]), so a
+ * call whose O is unchanged does not gather them again; with NULL they are
+ * gathered into the workspace on every call. */
 typedef struct {
     const void* W;
     int64_t N;
@@ -376,6 +381,7 @@ typedef struct {
     float* qs_w;
     int32_t* cached_idx;
     int32_t* cached_n;
+    float* wo;
 } sq_llmint8_weight_t;
 
 /* The whole decomposition in one call: detect O on X; if O differs from the cached set,

@@ -306,7 +306,8 @@ def test_norm_smooth_quant_per_token(dtype, norm, K):
 
 @pytest.mark.parametrize("norm", ["ln", "rms"])
 @pytest.mark.parametrize("K,M,dtype", [(5000, 300, torch.bfloat16), (8192, 300, torch.float16),
-                                       (12288, 2500, torch.bfloat16), (13000, 300, torch.bfloat16),
+                                       (11008, 300, torch.float16), (12288, 2500, torch.bfloat16),
+                                       (13000, 300, torch.bfloat16),
                                        (16384, 700, torch.float16)])
 def test_norm_quant_only(norm, K, M, dtype):
     """Codes and scales without the V output, per token and with a static scale:
@@ -595,12 +596,15 @@ def test_llmint8_steps_and_matmul(dtype, M, K, N, n_out):
     assert torch.equal(Y.view(torch.int16), Y2.view(torch.int16))
 
 
-def test_llmint8_cache_follows_outlier_set():
+@pytest.mark.parametrize("keep_wo", [True, False])
+def test_llmint8_cache_follows_outlier_set(keep_wo):
+    """The cached int8 weight (and, when the state keeps it, the gathered fp32
+    outlier channels of W) follows O as it changes from call to call."""
     M, K, N = 128, 512, 256
     X1, W, _ = _llm_case(M, K, N, 3, seed=1)
     X2, _, _ = _llm_case(M, K, N, 5, seed=2)
     Wd = W.to(DEV)
-    st = sq.llmint8_weight_state(Wd)
+    st = sq.llmint8_weight_state(Wd, keep_wo=keep_wo)
     ws = sq.workspace(sq.SQ_OP_LLMINT8, M, N, K)
     idx = torch.empty(K, dtype=torch.int32, device=DEV)
     n = torch.empty(1, dtype=torch.int32, device=DEV)

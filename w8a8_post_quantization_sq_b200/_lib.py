@@ -37,7 +37,8 @@ class SqError(RuntimeError):
 
 class LLMInt8Weight(ctypes.Structure):
     _fields_ = [("W", ctypes.c_void_p), ("N", ctypes.c_int64), ("Wq", ctypes.c_void_p),
-                ("qs_w", ctypes.c_void_p), ("cached_idx", ctypes.c_void_p), ("cached_n", ctypes.c_void_p)]
+                ("qs_w", ctypes.c_void_p), ("cached_idx", ctypes.c_void_p), ("cached_n", ctypes.c_void_p),
+                ("wo", ctypes.c_void_p)]
 
 
 _p, _i64, _i, _f, _d, _sz = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_double,
@@ -346,16 +347,19 @@ def sq_llmint8_quant_weight(W, idx, n, Wq, qs_w, stream=None):
         _vec(qs_w, torch.float32, N), _stream(stream)))
 
 
-def llmint8_weight_state(W):
+def llmint8_weight_state(W, keep_wo=True):
     """Device buffers of the int8 weight cache for sq_llmint8_matmul (torch
-    allocates them; cached_n = -1 marks the cache empty)."""
+    allocates them; cached_n = -1 marks the cache empty). keep_wo: also keep
+    the fp32 outlier channels of W (32 x N rounded up to 256) in the state."""
     N, K = W.shape
     st = {"W": W, "Wq": torch.empty((N, K), dtype=torch.int8, device=W.device),
           "qs_w": torch.empty(N, dtype=torch.float32, device=W.device),
           "cached_idx": torch.zeros(K, dtype=torch.int32, device=W.device),
-          "cached_n": torch.full((1,), -1, dtype=torch.int32, device=W.device)}
+          "cached_n": torch.full((1,), -1, dtype=torch.int32, device=W.device),
+          "wo": torch.zeros((32, (N + 255) // 256 * 256), dtype=torch.float32, device=W.device) if keep_wo else None}
     st["c"] = LLMInt8Weight(W.data_ptr(), N, st["Wq"].data_ptr(), st["qs_w"].data_ptr(),
-                            st["cached_idx"].data_ptr(), st["cached_n"].data_ptr())
+                            st["cached_idx"].data_ptr(), st["cached_n"].data_ptr(),
+                            st["wo"].data_ptr() if keep_wo else None)
     return st
 
 

@@ -325,9 +325,10 @@ __device__ __forceinline__ void epi_chunk(const Params& p, const uint32_t* r, in
             // the 16-bit outlier term, added term by term in ascending o with
             // fma (the 16-bit products are exact in fp32)
             if (compact) {
-                for (int o = 0; o < n_out; ++o) {
-                    const float xo = row_ok ? ep.xo[row * kOutlierCap + o] : 0.0f;
-                    const float4* w4 = reinterpret_cast<const float4*>(ep.wo + (int64_t)o * ep.wo_ld + col0);
+                // X_O is o-major (a warp's 32 rows read 128 contiguous bytes);
+                // two outliers per step so their loads are in flight together,
+                // the fmas still in ascending o
+                auto term = [&](float xo, const float4* w4) {
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const float4 w = __ldg(w4 + e);
@@ -336,6 +337,17 @@ __device__ __forceinline__ void epi_chunk(const Params& p, const uint32_t* r, in
                         y[4 * e + 2] = __fmaf_rn(xo, w.z, y[4 * e + 2]);
                         y[4 * e + 3] = __fmaf_rn(xo, w.w, y[4 * e + 3]);
                     }
+                };
+                int o = 0;
+                for (; o + 1 < n_out; o += 2) {
+                    const float xa = row_ok ? __ldg(ep.xo + (int64_t)o * p.M + row) : 0.0f;
+                    const float xb = row_ok ? __ldg(ep.xo + (int64_t)(o + 1) * p.M + row) : 0.0f;
+                    term(xa, reinterpret_cast<const float4*>(ep.wo + (int64_t)o * ep.wo_ld + col0));
+                    term(xb, reinterpret_cast<const float4*>(ep.wo + (int64_t)(o + 1) * ep.wo_ld + col0));
+                }
+                if (o < n_out) {
+                    const float xa = row_ok ? __ldg(ep.xo + (int64_t)o * p.M + row) : 0.0f;
+                    term(xa, reinterpret_cast<const float4*>(ep.wo + (int64_t)o * ep.wo_ld + col0));
                 }
             } else {
                 for (int o = 0; o < n_out; ++o) {

@@ -23,6 +23,7 @@
 // Nothing here synchronises with the host, so a whole call can be captured in
 // a CUDA graph.
 #include <mutex>
+#include <type_traits>
 
 #include "sq_common.cuh"
 #include "sq_internal.h"
@@ -38,7 +39,7 @@ size_t detect_workspace_bytes(int64_t M, int64_t K) {
 static size_t r256(size_t b) { return (b + 255) / 256 * 256; }
 static int64_t wo_ld_of(int64_t N) { return (N + 255) / 256 * 256; }
 
-// header + counts | Xq [M,K] int8 | qs_x [M] fp32 | X_O [M, cap] fp32 | W_O [cap, N256] fp32
+// header + counts | Xq [M,K] int8 | qs_x [M] fp32 | X_O [cap, M] fp32 (o-major) | W_O [cap, N256] fp32
 size_t llmint8_workspace_bytes(int64_t M, int64_t N, int64_t K) {
     return detect_workspace_bytes(M, K) + r256((size_t)M * (size_t)K) + r256((size_t)M * 4) +
            r256((size_t)M * kOutlierCap * 4) + r256((size_t)kOutlierCap * (size_t)wo_ld_of(N) * 4);
@@ -61,11 +62,24 @@ count_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, float th
     const int64_t r1 = min(M, r0 + kDetectRows);
     int32_t cnt[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     if (c0 < K) {
-        for (int64_t r = r0 + warp; r < r1; r += kWarps) {
-            float f[8];
-            unpack<T>(ldg_nc_v4(X + r * ld + c0), f);
+        // the warp's rows of the band (kDetectRows / kWarps of them), all
+        // loads issued before any is used
+        constexpr int RW = kDetectRows / kWarps;
+        uint4 v[RW];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) cnt[e] += fabsf(f[e]) > thr ? 1 : 0;
+        for (int u = 0; u < RW; ++u) {
+            const int64_t r = r0 + warp + (int64_t)u * kWarps;
+            if (r < r1) v[u] = ldg_nc_v4(X + r * ld + c0);
+        }
+#pragma unroll
+        for (int u = 0; u < RW; ++u) {
+            const int64_t r = r0 + warp + (int64_t)u * kWarps;
+            if (r < r1) {
+                float f[8];
+                unpack<T>(v[u], f);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) cnt[e] += fabsf(f[e]) > thr ? 1 : 0;
+            }
         }
     }
 #pragma unroll
@@ -100,9 +114,13 @@ compact_kernel(const int32_t* __restrict__ partial, int64_t row_blocks, int64_t 
         bool flag = false;
         if (j < K) {
             int64_t total = 0;
+#pragma unroll 8
             for (int64_t b = 0; b < row_blocks; ++b) total += partial[b * K + j];
-            const double ratio = M > 0 ? __ddiv_rn((double)total, (double)M) : 0.0;
-            flag = ratio > min_ratio;
+            // an empty column has ratio 0, never above min_ratio >= 0
+            if (total > 0) {
+                const double ratio = M > 0 ? __ddiv_rn((double)total, (double)M) : 0.0;
+                flag = ratio > min_ratio;
+            }
         }
         const unsigned bal = __ballot_sync(0xffffffffu, flag);
         const int before_in_warp = __popc(bal & ((1u << lane) - 1u));
@@ -189,7 +207,7 @@ masked_quant_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, c
                 float f[8];
                 uint4 v = make_uint4(u, 0, 0, 0);
                 unpack<T>(v, f);
-                xo[row * kOutlierCap + o] = f[0];
+                xo[(int64_t)o * M + row] = f[0];
             }
         int8_t* q = Q + row * K;
 #pragma unroll 4
@@ -206,12 +224,90 @@ masked_quant_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, c
     }
 }
 
-// W_O[o, j] = W[j, idx[o]] for o < min(n, cap), j < N; zero for N <= j < ld.
-template <typename T>
-__global__ void gather_wo_kernel(const T* __restrict__ W, int64_t N, int64_t K, const int32_t* __restrict__ idx,
-                                 const int32_t* __restrict__ n_idx, float* __restrict__ wo, int64_t ld) {
+// The same with the row in registers (K <= 256 * CH): one read of X. Lane l
+// holds chunks l, l + 32, ... of 8 columns; X_O (when asked for) is written
+// o-major, xo[o * M + row], so the GEMM epilogue's reads are coalesced.
+template <typename T, int CH>
+__global__ void __launch_bounds__(256)
+masked_quant_reg_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, const int32_t* __restrict__ idx,
+                        const int32_t* __restrict__ n_idx, const int32_t* __restrict__ only_if,
+                        int8_t* __restrict__ Q, float* __restrict__ qs_out, float* __restrict__ xo) {
     pdl_wait();
     pdl_trigger();
+    extern __shared__ uint32_t mask[];  // K bits
+    if (only_if && *only_if == 0) return;
+    const int64_t words = (K + 31) / 32;
+    for (int64_t w = threadIdx.x; w < words; w += blockDim.x) mask[w] = 0u;
+    __syncwarp();
+    __syncthreads();
+    const int n = *n_idx;
+    for (int o = threadIdx.x; o < n; o += blockDim.x) {
+        const int j = idx[o];
+        atomicOr(&mask[j >> 5], 1u << (j & 31));
+    }
+    __syncwarp();
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < M; row += nwarps) {
+        const T* x = X + row * ld;
+        uint4 raw[CH];
+#pragma unroll
+        for (int i = 0; i < CH; ++i) {
+            const int64_t k0 = (int64_t)lane * 8 + 256 * i;
+            if (k0 < K) raw[i] = ldg_nc_v4(x + k0);
+        }
+        float m = 0.0f;
+#pragma unroll
+        for (int i = 0; i < CH; ++i) {
+            const int64_t k0 = (int64_t)lane * 8 + 256 * i;
+            if (k0 < K) {
+                float f[8];
+                unpack<T>(raw[i], f);
+                const uint32_t bits = (mask[k0 >> 5] >> (k0 & 31)) & 0xffu;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) m = fmaxf(m, ((bits >> e) & 1u) ? 0.0f : fabsf(f[e]));
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        const float qs = __fdiv_rn(127.0f, fmaxf(m, 1e-8f));
+        if (lane == 0) qs_out[row] = qs;
+        if (xo)
+            for (int o = lane; o < n && o < kOutlierCap; o += 32) {
+                const uint16_t u = reinterpret_cast<const uint16_t*>(x)[idx[o]];
+                float f[8];
+                unpack<T>(make_uint4(u, 0, 0, 0), f);
+                xo[(int64_t)o * M + row] = f[0];
+            }
+        int8_t* q = Q + row * K;
+#pragma unroll
+        for (int i = 0; i < CH; ++i) {
+            const int64_t k0 = (int64_t)lane * 8 + 256 * i;
+            if (k0 < K) {
+                float f[8];
+                unpack<T>(raw[i], f);
+                const uint32_t bits = (mask[k0 >> 5] >> (k0 & 31)) & 0xffu;
+                uint32_t c[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    c[e] = ((bits >> e) & 1u) ? 0u : quant_bits_noclip(__fmul_rn(f[e], qs));
+                *reinterpret_cast<uint2*>(q + k0) =
+                    make_uint2(pack_low_bytes(c[0], c[1], c[2], c[3]), pack_low_bytes(c[4], c[5], c[6], c[7]));
+            }
+        }
+    }
+}
+
+// W_O[o, j] = W[j, idx[o]] for o < min(n, cap), j < N; zero for N <= j < ld.
+// When `only_if` is given and *only_if == 0 the kernel does nothing.
+template <typename T>
+__global__ void gather_wo_kernel(const T* __restrict__ W, int64_t N, int64_t K, const int32_t* __restrict__ idx,
+                                 const int32_t* __restrict__ n_idx, const int32_t* __restrict__ only_if,
+                                 float* __restrict__ wo, int64_t ld) {
+    pdl_wait();
+    pdl_trigger();
+    if (only_if && *only_if == 0) return;
     const int n = min(*n_idx, kOutlierCap);
     for (int64_t j = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; j < ld; j += (int64_t)gridDim.x * blockDim.x)
         for (int o = 0; o < n; ++o) {
@@ -252,17 +348,25 @@ sq_status_t launch_masked_quant(const void* X, sq_dtype_t dt, int64_t M, int64_t
                                 const char* name, float* xo = nullptr) {
     const size_t smem = (size_t)((K + 31) / 32) * 4;
     int64_t grid = (M + 7) / 8;  // one warp per row, 8 warps per block
-    if (grid > (int64_t)num_sms() * 8) grid = (int64_t)num_sms() * 8;
+    // a conditional (weight-side) pass usually returns at once: fewer blocks
+    const int64_t cap = (int64_t)num_sms() * (only_if ? 2 : 8);
+    if (grid > cap) grid = cap;
     if (grid < 1) return SQ_OK;
-    if (dt == SQ_BF16) {
-        auto k = masked_quant_kernel<__nv_bfloat16>;
+    auto go = [&](auto k, auto* x) {
         if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        launch_pdl(k, dim3((unsigned)grid), dim3(256), smem, s, static_cast<const __nv_bfloat16*>(X), M, K, ldx, idx, n_idx, only_if, Q, qs, xo);
-    } else {
-        auto k = masked_quant_kernel<__half>;
-        if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        launch_pdl(k, dim3((unsigned)grid), dim3(256), smem, s, static_cast<const __half*>(X), M, K, ldx, idx, n_idx, only_if, Q, qs, xo);
-    }
+        launch_pdl(k, dim3((unsigned)grid), dim3(256), smem, s, x, M, K, ldx, idx, n_idx, only_if, Q, qs, xo);
+    };
+    auto pick = [&](auto* x) {
+        using T = std::remove_const_t<std::remove_pointer_t<decltype(x)>>;
+        if (K <= 256) go(masked_quant_reg_kernel<T, 1>, x);
+        else if (K <= 512) go(masked_quant_reg_kernel<T, 2>, x);
+        else if (K <= 1024) go(masked_quant_reg_kernel<T, 4>, x);
+        else if (K <= 2048) go(masked_quant_reg_kernel<T, 8>, x);
+        else if (K <= 4096) go(masked_quant_reg_kernel<T, 16>, x);
+        else go(masked_quant_kernel<T>, x);
+    };
+    if (dt == SQ_BF16) pick(static_cast<const __nv_bfloat16*>(X));
+    else pick(static_cast<const __half*>(X));
     return check_launch(name);
 }
 
@@ -360,16 +464,20 @@ sq_status_t sq_llmint8_matmul(const void* X, sq_dtype_t dt, int64_t M, int64_t K
     // row quantisation outside O (and the fp32 copy of the outlier columns of X)
     st = sq::launch_masked_quant(X, dt, M, K, ldx, idx_out, n_out, nullptr, Xq, qs_x, s, name, xo);
     if (st != SQ_OK) return st;
-    // fp32 copy of the outlier input channels of W, transposed, for the epilogue
+    // fp32 copy of the outlier input channels of W, transposed, for the
+    // epilogue: kept in the weight state (gathered again only when O changed)
+    // or, without one, gathered into the workspace
     {
+        const int32_t* only_if = w->wo ? changed : nullptr;
+        if (w->wo) wo = w->wo;
         int64_t blocks = (wo_ld + 255) / 256;
         if (blocks > (int64_t)sq::num_sms() * 4) blocks = (int64_t)sq::num_sms() * 4;
         if (dt == SQ_BF16)
-            sq::launch_pdl(sq::gather_wo_kernel<__nv_bfloat16>, dim3((unsigned)blocks), dim3(256), 0, s, 
-                static_cast<const __nv_bfloat16*>(w->W), w->N, K, idx_out, n_out, wo, wo_ld);
+            sq::launch_pdl(sq::gather_wo_kernel<__nv_bfloat16>, dim3((unsigned)blocks), dim3(256), 0, s,
+                           static_cast<const __nv_bfloat16*>(w->W), w->N, K, idx_out, n_out, only_if, wo, wo_ld);
         else
-            sq::launch_pdl(sq::gather_wo_kernel<__half>, dim3((unsigned)blocks), dim3(256), 0, s, static_cast<const __half*>(w->W), w->N, K,
-                                                                         idx_out, n_out, wo, wo_ld);
+            sq::launch_pdl(sq::gather_wo_kernel<__half>, dim3((unsigned)blocks), dim3(256), 0, s,
+                           static_cast<const __half*>(w->W), w->N, K, idx_out, n_out, only_if, wo, wo_ld);
         st = sq::check_launch(name);
         if (st != SQ_OK) return st;
     }

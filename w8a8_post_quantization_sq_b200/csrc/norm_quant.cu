@@ -108,6 +108,51 @@ __device__ __forceinline__ void center8(float* f, float mu) {
     for (int e = 0; e < 8; e += 2) upk2(add2(pk2(f[e], f[e + 1]), nmu2), f[e], f[e + 1]);
 }
 
+// Mixed-precision forms (a 16-bit operand widened exactly, one fp32 rounding):
+// acc + x_e in index order over a chunk, and d_e = x_e - mu, straight from the
+// packed 16-bit row, with no separate unpack.
+template <typename T> struct Mix;
+template <> struct Mix<__nv_bfloat16> {
+    static __device__ __forceinline__ float add(uint32_t w, float acc) {
+        asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\t"
+            "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %0, hi, %0;\n\t}"
+            : "+f"(acc) : "r"(w));
+        return acc;
+    }
+    static __device__ __forceinline__ void sub(uint32_t w, float mu, float& d0, float& d1) {
+        asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+            "sub.rn.f32.bf16 %0, lo, %3;\n\tsub.rn.f32.bf16 %1, hi, %3;\n\t}"
+            : "=f"(d0), "=f"(d1) : "r"(w), "f"(mu));
+    }
+};
+template <> struct Mix<__half> {
+    static __device__ __forceinline__ float add(uint32_t w, float acc) {
+        asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\t"
+            "add.rn.f32.f16 %0, lo, %0;\n\tadd.rn.f32.f16 %0, hi, %0;\n\t}"
+            : "+f"(acc) : "r"(w));
+        return acc;
+    }
+    static __device__ __forceinline__ void sub(uint32_t w, float mu, float& d0, float& d1) {
+        asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+            "sub.rn.f32.f16 %0, lo, %3;\n\tsub.rn.f32.f16 %1, hi, %3;\n\t}"
+            : "=f"(d0), "=f"(d1) : "r"(w), "f"(mu));
+    }
+};
+template <typename T>
+__device__ __forceinline__ float add8_16(const uint4& w, float acc) {
+    acc = Mix<T>::add(w.x, acc);
+    acc = Mix<T>::add(w.y, acc);
+    acc = Mix<T>::add(w.z, acc);
+    return Mix<T>::add(w.w, acc);
+}
+template <typename T>
+__device__ __forceinline__ void sub8_16(const uint4& w, float mu, float* d) {
+    Mix<T>::sub(w.x, mu, d[0], d[1]);
+    Mix<T>::sub(w.y, mu, d[2], d[3]);
+    Mix<T>::sub(w.z, mu, d[4], d[5]);
+    Mix<T>::sub(w.w, mu, d[6], d[7]);
+}
+
 // v_j of one chunk from its fp32 inputs f (v may alias f)
 template <bool LN>
 __device__ __forceinline__ void compute_v_f(const float* f, const float4* b_lo, const float4* b_hi, const float* g,
@@ -421,16 +466,26 @@ norm_quant_bulk_kernel(const T* __restrict__ H, NormArgs a, int R) {
             }
         };
         float vk[KEEPV ? C : 1][8];
-        // pass 1: the sum (LayerNorm: of x; RMSNorm: of x^2) in the lane's order
+        // pass 1: the sum (LayerNorm: of x; RMSNorm: of x^2) in the lane's order.
+        // LayerNorm with the row in registers keeps the packed 16-bit chunks
+        // and sums them with mixed-precision adds; d = x - mu is formed from
+        // them the same way below.
+        constexpr bool kRaw = LN && KEEPV && (FULL || C <= 4);  // (the ragged C = 6 case would spill)
+        uint4 raw[kRaw ? C : 1];
         float acc = 0.0f;
 #pragma unroll
         for (int c = 0; c < C; ++c) {
             if (mine(c)) {
-                float fl[8];
-                float* f = KEEPV ? vk[c] : fl;
-                unpack<T>(chunk(c), f);
+                if constexpr (kRaw) {
+                    raw[c] = chunk(c);
+                    acc = add8_16<T>(raw[c], acc);
+                } else {
+                    float fl[8];
+                    float* f = KEEPV ? vk[c] : fl;
+                    unpack<T>(chunk(c), f);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) acc = LN ? __fmaf_rn(f[e], 1.0f, acc) : __fmaf_rn(f[e], f[e], acc);
+                    for (int e = 0; e < 8; ++e) acc = LN ? __fmaf_rn(f[e], 1.0f, acc) : __fmaf_rn(f[e], f[e], acc);
+                }
             }
         }
         auto rstd = [&](float s_) { return __frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(s_, Kf), a.eps))); };
@@ -442,11 +497,15 @@ norm_quant_bulk_kernel(const T* __restrict__ H, NormArgs a, int R) {
 #pragma unroll
             for (int c = 0; c < C; ++c) {
                 if (mine(c)) {
-                    // d = x - mu, kept in place of x when the row is in registers
+                    // d = x - mu, kept in registers from here on when the row is
                     float fl[8];
-                    if constexpr (!KEEPV) unpack<T>(chunk(c), fl);
                     float* d = KEEPV ? vk[c] : fl;
-                    center8(d, mu);
+                    if constexpr (kRaw) {
+                        sub8_16<T>(raw[c], mu, d);
+                    } else {
+                        if constexpr (!KEEPV) unpack<T>(chunk(c), fl);
+                        center8(d, mu);
+                    }
 #pragma unroll
                     for (int e = 0; e < 8; ++e) acc = __fmaf_rn(d[e], d[e], acc);
                 }

@@ -40,7 +40,7 @@ struct GemmEpilogue {
     const int32_t* idx = nullptr;
     const int32_t* n_out = nullptr;
     int in16_bf16 = 0;
-    const float* xo = nullptr;  // [M, kOutlierCap] fp32 copies of X[:, O]
+    const float* xo = nullptr;  // [kOutlierCap, M] fp32 copies of X[:, O] (o-major)
     const float* wo = nullptr;  // [kOutlierCap, wo_ld] fp32 copies of W[:, O]^T
     int64_t wo_ld = 0;          // multiple of 256, >= N
     int kind = 0;               // 0: int8 operands, int32 sums; 1: FP8 E4M3 operands, fp32 sums
