@@ -600,12 +600,25 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
             }
             const int acc = local & 1;
             const uint32_t acc_phase = (uint32_t)(local >> 1) & 1u;
-            const bool ok = wait_bounded(tfull_bar(acc), acc_phase, abort_flag, p.status, 0x6E4);
-            if (!__all_sync(0xffffffffu, ok)) break;
-            tc_fence_after();
             const int row0 = m0 + q * 32;  // first row of this warp
             const int64_t row = (int64_t)row0 + lane;
             const bool row_ok = row < p.M;
+            if constexpr (OUTL) {
+                // while this tile's MMAs run: bring its X_O rows and W_O
+                // columns into L1, so the outlier term's loads do not wait on L2
+                if (compact && row0 < p.M && c_base < p.N) {
+                    for (int o = 0; o < n_out; ++o)
+                        if (row_ok)
+                            asm volatile("prefetch.global.L1 [%0];" ::"l"(ep.xo + (int64_t)o * p.M + row));
+                    for (int i = lane; i < n_out * NCH; i += 32) {
+                        const int o = i / NCH, l = i - o * NCH;
+                        asm volatile("prefetch.global.L1 [%0];" ::"l"(ep.wo + (int64_t)o * ep.wo_ld + c_base + 32 * l));
+                    }
+                }
+            }
+            const bool ok = wait_bounded(tfull_bar(acc), acc_phase, abort_flag, p.status, 0x6E4);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc_fence_after();
             float rx = 0.0f;
             if constexpr (OUT != kOutI32)
                 if (row_ok) rx = __frcp_rn(ep.x_per_token ? ep.qs_x[(int64_t)b * p.M + row] : ep.qs_x[b]);
