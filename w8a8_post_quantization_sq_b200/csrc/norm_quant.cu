@@ -85,15 +85,17 @@ __device__ __forceinline__ void compute_v_d(const float* d, const float4* b_lo, 
                                             float r, float* v) {
     const uint64_t r2 = pk2(r, r);
     if (b_lo) {
-        // the last product feeds an add: keep those two steps scalar
+        // the last product feeds an add: the products go as packed pairs, the
+        // adds stay scalar (a packed multiply feeding a packed add has been
+        // seen fused into one rounding; feeding a scalar add it has not)
         const float4 b0 = *b_lo, b1 = *b_hi;
         const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
         for (int e = 0; e < 8; e += 2) {
-            float u0, u1;
-            upk2(mul2(pk2(d[e], d[e + 1]), r2), u0, u1);
-            v[e] = __fadd_rn(__fmul_rn(u0, g[e]), b[e]);
-            v[e + 1] = __fadd_rn(__fmul_rn(u1, g[e + 1]), b[e + 1]);
+            float t0, t1;
+            upk2(mul2(mul2(pk2(d[e], d[e + 1]), r2), pk2(g[e], g[e + 1])), t0, t1);
+            v[e] = __fadd_rn(t0, b[e]);
+            v[e + 1] = __fadd_rn(t1, b[e + 1]);
         }
     } else {
 #pragma unroll
