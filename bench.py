@@ -265,14 +265,16 @@ class Layer:
             if gemm_ev is not None:
                 gemm_ev[i][1].record()
 
+        # the MLP chain (norm -> gate/up GEMM -> SwiGLU -> down GEMM) is the
+        # longest, so the weight-side work it waits for goes first on each stream
         with torch.cuda.stream(sC):
-            sq.sq_weight_absmax(self.W["qkv"], self.wmax["attn"])
-            ev["wmax_attn"].record()
             sq.sq_weight_absmax(self.W["gateup"], self.wmax["mlp"])
             ev["wmax_mlp"].record()
             # fold into the previous linear: 1/s_down into up_proj's output channels; down_proj takes s_down
             sq.sq_fold_prev_linear(self.W_up, self.s_down, self.W_up_f)
             ev["up_folded"].record()
+            sq.sq_weight_absmax(self.W["qkv"], self.wmax["attn"])
+            ev["wmax_attn"].record()
             sq.sq_quantize_weight(self.W["down"], self.s_down, True, self.Wq["down"], self.qw["down"])
             ev["wq_down"].record()
             sq.sq_quantize_weight(self.W["o"], None, True, self.Wq["o"], self.qw["o"])
@@ -292,14 +294,14 @@ class Layer:
                 sq.sq_norm_smooth_quant(self.h[k], sq.SQ_RMSNORM, self.gp[k], None, eps, True, None,
                                         self.Xq[k], self.qx[k], None, None)
         with torch.cuda.stream(sD):  # weight quantisation once s is known
+            sD.wait_event(ev["s_mlp"])
+            sq.sq_quantize_weight(self.W_gate, self.s["mlp"], True, self.Wq["gateup"][:I], self.qw["gateup"][:I])
+            sD.wait_event(ev["up_folded"])
+            sq.sq_quantize_weight(self.W_up_f, self.s["mlp"], True, self.Wq["gateup"][I:], self.qw["gateup"][I:])
+            ev["wq_gateup"].record()
             sD.wait_event(ev["s_attn"])
             sq.sq_quantize_weight(self.W["qkv"], self.s["attn"], True, self.Wq["qkv"], self.qw["qkv"])
             ev["wq_qkv"].record()
-            sD.wait_event(ev["s_mlp"])
-            sD.wait_event(ev["up_folded"])
-            sq.sq_quantize_weight(self.W_gate, self.s["mlp"], True, self.Wq["gateup"][:I], self.qw["gateup"][:I])
-            sq.sq_quantize_weight(self.W_up_f, self.s["mlp"], True, self.Wq["gateup"][I:], self.qw["gateup"][I:])
-            ev["wq_gateup"].record()
         for k, w, s_, i in chains:
             with torch.cuda.stream(s_):
                 s_.wait_event(ev["wq_" + w])
