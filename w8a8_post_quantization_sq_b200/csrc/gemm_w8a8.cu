@@ -261,17 +261,11 @@ __device__ __forceinline__ void tmem_wait(uint32_t* r) {
                  : "memory");
 }
 
+// A 32-column TMEM load completed before return. The wait names the
+// destination registers, so none of them can be spilled or used before it.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+    tmem_ld32_async(taddr, r);
+    tmem_wait(r);
 }
 
 __device__ __forceinline__ float load16(const void* base, int64_t idx, int bf16) {
@@ -329,13 +323,12 @@ __device__ __forceinline__ void epi_chunk(const Params& p, const uint32_t* r, in
                 // two outliers per step so their loads are in flight together,
                 // the fmas still in ascending o
                 auto term = [&](float xo, const float4* w4) {
+                    const uint64_t x2 = pk2(xo, xo);  // fmas two columns at a time
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const float4 w = __ldg(w4 + e);
-                        y[4 * e + 0] = __fmaf_rn(xo, w.x, y[4 * e + 0]);
-                        y[4 * e + 1] = __fmaf_rn(xo, w.y, y[4 * e + 1]);
-                        y[4 * e + 2] = __fmaf_rn(xo, w.z, y[4 * e + 2]);
-                        y[4 * e + 3] = __fmaf_rn(xo, w.w, y[4 * e + 3]);
+                        upk2(fma2(x2, pk2(w.x, w.y), pk2(y[4 * e + 0], y[4 * e + 1])), y[4 * e + 0], y[4 * e + 1]);
+                        upk2(fma2(x2, pk2(w.z, w.w), pk2(y[4 * e + 2], y[4 * e + 3])), y[4 * e + 2], y[4 * e + 3]);
                     }
                 };
                 int o = 0;

@@ -179,6 +179,13 @@ __device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
     asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
     return r;
 }
+// fma on packed pairs: each lane one fused, correctly rounded fma (the
+// scalar __fmaf_rn of that lane)
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
 // v[e] *= s[e] for 8 values, two at a time
 __device__ __forceinline__ void mul8(float* v, const float* s) {
 #pragma unroll
