@@ -211,7 +211,6 @@ class Layer:
         self.Xq_down = e(M, I, dt=torch.int8)
         self.qx_down = e(M)
         self.s_down = self.calibrate_down()
-        self.gemm_events = None
         self.streams = [torch.cuda.Stream(device=dev) for _ in range(5)]
         self.events = {n: torch.cuda.Event() for n in ("wmax_attn", "wmax_mlp", "V_attn", "V_mlp", "s_attn", "s_mlp",
                                                       "wq_qkv", "wq_gateup", "wq_down", "up_folded")}
