@@ -88,6 +88,11 @@ def test_workspace_sizes(L):
     assert L.sq_workspace_size(0, 2048, 16384, 4096) == 256
     # 4096 x 36864: 4608 tiles, 97 % of the waves busy: whole tiles only
     assert L.sq_workspace_size(0, 4096, 36864, 12288) == 256
+    # 4096 x 12288: 1536 tiles, 94 % busy; cut with a k-loop of 384 blocks
+    # (counters for the last wave's 56 tiles), not with one of 56 blocks
+    # (1024 x 21504: 91 % busy)
+    assert L.sq_workspace_size(0, 4096, 12288, 49152) == 256 + 1792 + 148 * 2 * 128 * 256 * 4
+    assert L.sq_workspace_size(0, 1024, 21504, 7168) == 256
     # a short k-loop (8 blocks) is never cut, nor a thin remainder: 260 x
     # 13000 leaves 5 tiles of 128 k-blocks, under 8 k-blocks per CTA
     assert L.sq_workspace_size(0, 260, 13000, 16384) == 256

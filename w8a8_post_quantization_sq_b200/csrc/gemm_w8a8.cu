@@ -867,12 +867,14 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int64_t batch) {
     // runs before its whole tiles. Measured on B200: 1024 x 7168 x 7168
     // (56 k-blocks) 54.1 -> 51.4 us, 1024 x 7168 x 28672 176 -> 174 us. Each
     // CTA's range must hold 8 k-blocks or more, and the k-loop 32 or more,
-    // or the parking of partial sums costs more than the idle tail.
+    // or the parking of partial sums costs more than the idle tail. Waves
+    // between 90 and 95 % busy are cut only for k-loops of 64 blocks or more
+    // (4096 x 12288 x 49152: 1832 -> 1792 us; 1024 x 21504 x 7168 gains nothing).
     const int64_t kb = (K + BK - 1) / BK;
     const int64_t rem = tiles % pl.grid;
     const double eff = (double)tiles / (double)(((tiles + pl.grid - 1) / pl.grid) * pl.grid);
     if (batch == 1 && pl.grid == sms && tiles > pl.grid && kb >= 32 && rem > 0 && 4 * rem <= 3 * (int64_t)pl.grid &&
-        eff < 0.9 && rem * kb >= 8ll * pl.grid && rem * kb < (1ll << 31)) {
+        (eff < 0.9 || (eff < 0.95 && kb >= 64)) && rem * kb >= 8ll * pl.grid && rem * kb < (1ll << 31)) {
         pl.sk_tiles = (int)rem;
         pl.sk_cnt_bytes = ((size_t)rem * kEpiWarps * sizeof(int) + 255) / 256 * 256;
         pl.sk_bytes = pl.sk_cnt_bytes + (size_t)pl.grid * 2 * BM * pl.bn * sizeof(int);
