@@ -466,9 +466,10 @@ def test_gemm_deterministic():
 # shapes whose last wave of whole tiles is at most three quarters full, with
 # k-loops of 128 blocks or more: that wave is cut by k-blocks (ragged M and K;
 # pieces of 4 to 100 k-blocks)
-# stream-K plans on 148 SMs: last waves of 104 tiles (129 and 57 k-blocks)
-# and of 24 tiles (128 k-blocks)
-SK_SHAPES = [(1029, 7168, 16400), (1029, 7168, 7200), (2560, 4096, 16384)]
+# stream-K plans on 148 SMs: last waves of 104 tiles (129 and 57 k-blocks),
+# of 24 tiles (128 k-blocks), and of 104 tiles with the waves 90 % busy
+# (64 k-blocks)
+SK_SHAPES = [(1029, 7168, 16400), (1029, 7168, 7200), (2560, 4096, 16384), (2048, 6400, 8192)]
 
 
 @pytest.mark.parametrize("M,N,K", SK_SHAPES)
