@@ -167,7 +167,7 @@ template <typename T>
 __global__ void __launch_bounds__(256)
 masked_quant_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, const int32_t* __restrict__ idx,
                     const int32_t* __restrict__ n_idx, const int32_t* __restrict__ only_if, int8_t* __restrict__ Q,
-                    float* __restrict__ qs_out, float* __restrict__ xo) {
+                    float* __restrict__ qs_out, float* __restrict__ xo, int64_t xo_ld) {
     pdl_wait();
     pdl_trigger();
     extern __shared__ uint32_t mask[];  // K bits
@@ -207,7 +207,7 @@ masked_quant_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, c
                 float f[8];
                 uint4 v = make_uint4(u, 0, 0, 0);
                 unpack<T>(v, f);
-                xo[(int64_t)o * M + row] = f[0];
+                xo[(int64_t)o * xo_ld + row] = f[0];
             }
         int8_t* q = Q + row * K;
 #pragma unroll 4
@@ -231,7 +231,8 @@ template <typename T, int CH>
 __global__ void __launch_bounds__(256)
 masked_quant_reg_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, const int32_t* __restrict__ idx,
                         const int32_t* __restrict__ n_idx, const int32_t* __restrict__ only_if,
-                        int8_t* __restrict__ Q, float* __restrict__ qs_out, float* __restrict__ xo) {
+                        int8_t* __restrict__ Q, float* __restrict__ qs_out, float* __restrict__ xo,
+                        int64_t xo_ld) {
     pdl_wait();
     pdl_trigger();
     extern __shared__ uint32_t mask[];  // K bits
@@ -278,7 +279,7 @@ masked_quant_reg_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t l
                 const uint16_t u = reinterpret_cast<const uint16_t*>(x)[idx[o]];
                 float f[8];
                 unpack<T>(make_uint4(u, 0, 0, 0), f);
-                xo[(int64_t)o * M + row] = f[0];
+                xo[(int64_t)o * xo_ld + row] = f[0];
             }
         int8_t* q = Q + row * K;
 #pragma unroll
@@ -345,7 +346,7 @@ sq_status_t launch_detect(const void* X, sq_dtype_t dt, int64_t M, int64_t K, in
 
 sq_status_t launch_masked_quant(const void* X, sq_dtype_t dt, int64_t M, int64_t K, int64_t ldx, const int32_t* idx,
                                 const int32_t* n_idx, const int32_t* only_if, int8_t* Q, float* qs, cudaStream_t s,
-                                const char* name, float* xo = nullptr) {
+                                const char* name, float* xo = nullptr, int64_t xo_ld = 0) {
     const size_t smem = (size_t)((K + 31) / 32) * 4;
     int64_t grid = (M + 7) / 8;  // one warp per row, 8 warps per block
     // a conditional (weight-side) pass usually returns at once: fewer blocks
@@ -354,7 +355,7 @@ sq_status_t launch_masked_quant(const void* X, sq_dtype_t dt, int64_t M, int64_t
     if (grid < 1) return SQ_OK;
     auto go = [&](auto k, auto* x) {
         if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        launch_pdl(k, dim3((unsigned)grid), dim3(256), smem, s, x, M, K, ldx, idx, n_idx, only_if, Q, qs, xo);
+        launch_pdl(k, dim3((unsigned)grid), dim3(256), smem, s, x, M, K, ldx, idx, n_idx, only_if, Q, qs, xo, xo_ld);
     };
     auto pick = [&](auto* x) {
         using T = std::remove_const_t<std::remove_pointer_t<decltype(x)>>;
@@ -457,19 +458,20 @@ sq_status_t sq_llmint8_matmul(const void* X, sq_dtype_t dt, int64_t M, int64_t K
     st = sq::launch_detect(X, dt, M, K, ldx, threshold, min_ratio, idx_out, n_out, w->cached_idx, w->cached_n, workspace,
                            s);
     if (st != SQ_OK) return st;
-    // weight side for O (returns at once when O is unchanged)
-    st = sq::launch_masked_quant(w->W, dt, w->N, K, K, idx_out, n_out, changed, w->Wq, w->qs_w, s, name);
+    // weight side for O (returns at once when O is unchanged); with a W_O
+    // buffer in the weight state the same pass refreshes it (wo[o, n] is
+    // W[n, O_o], written o-major like X_O)
+    st = sq::launch_masked_quant(w->W, dt, w->N, K, K, idx_out, n_out, changed, w->Wq, w->qs_w, s, name, w->wo, wo_ld);
     if (st != SQ_OK) return st;
     if (M == 0) return SQ_OK;
     // row quantisation outside O (and the fp32 copy of the outlier columns of X)
-    st = sq::launch_masked_quant(X, dt, M, K, ldx, idx_out, n_out, nullptr, Xq, qs_x, s, name, xo);
+    st = sq::launch_masked_quant(X, dt, M, K, ldx, idx_out, n_out, nullptr, Xq, qs_x, s, name, xo, M);
     if (st != SQ_OK) return st;
-    // fp32 copy of the outlier input channels of W, transposed, for the
-    // epilogue: kept in the weight state (gathered again only when O changed)
-    // or, without one, gathered into the workspace
-    {
-        const int32_t* only_if = w->wo ? changed : nullptr;
-        if (w->wo) wo = w->wo;
+    // without a W_O buffer in the weight state: gather W_O into the workspace
+    if (w->wo) {
+        wo = w->wo;
+    } else {
+        const int32_t* only_if = nullptr;
         int64_t blocks = (wo_ld + 255) / 256;
         if (blocks > (int64_t)sq::num_sms() * 4) blocks = (int64_t)sq::num_sms() * 4;
         if (dt == SQ_BF16)
