@@ -149,6 +149,14 @@ SQ_API sq_status_t sq_fold_weight(const void* W, sq_dtype_t dt, int64_t N, int64
 SQ_API sq_status_t sq_fold_norm(const float* gamma, const float* beta, const float* s, int64_t K,
                          float* gamma_out, float* beta_out, sq_stream_t stream);
 
+/* sq_smooth_scales and sq_fold_norm in one launch: s_out as sq_smooth_scales,
+ * then gamma_out = gamma / s_out and beta_out = beta / s_out as sq_fold_norm
+ * (the same operations, so the same bits as the two calls in sequence).
+ * beta / beta_out may both be NULL. All [K] fp32; alpha in [0, 1]. */
+SQ_API sq_status_t sq_smooth_fold_norm(const float* xmax, const float* wmax, int64_t K, double alpha,
+                                       const float* gamma, const float* beta, float* s_out, float* gamma_out,
+                                       float* beta_out, sq_stream_t stream);
+
 /* Fold into the previous linear layer    [SQ-p2] 融入前序线性层的权重 and
  * the table after it: for down_proj the smoothing goes into up_proj's output
  * channels, for o_proj into v_proj's. Output channel n of the previous layer

@@ -153,6 +153,32 @@ def test_fold_weight_and_norm():
     assert np.array_equal(npf(go), rg) and np.array_equal(npf(bo), rb)
 
 
+@pytest.mark.parametrize("alpha", [0.5, 0.4, 0.0, 1.0])
+@pytest.mark.parametrize("with_beta", [True, False])
+def test_smooth_fold_norm(alpha, with_beta):
+    """The one-launch smoothing + norm fold against the oracle's two steps."""
+    K = 4104
+    g = torch.Generator().manual_seed(17)
+    xmax = torch.rand(K, generator=g) * 80
+    wmax = torch.rand(K, generator=g) * 0.3
+    xmax[:5] = 0.0  # the clamp at 1e-5
+    gamma = 1 + 0.1 * rnd(K, 18)
+    beta = 0.1 * rnd(K, 19) if with_beta else None
+    s = torch.empty(K, device=DEV)
+    go = torch.empty(K, device=DEV)
+    bo = torch.empty(K, device=DEV) if with_beta else None
+    sq.sq_smooth_fold_norm(xmax.to(DEV), wmax.to(DEV), alpha, gamma.to(DEV), None if beta is None else beta.to(DEV),
+                           s, go, bo)
+    rs = oracle.smooth_scales(xmax.numpy(), wmax.numpy(), alpha)
+    assert np.array_equal(npf(s), rs)
+    rg, rb = oracle.fold_norm(gamma.numpy(), None if beta is None else beta.numpy(), rs, round_f32=True)
+    assert np.array_equal(npf(go), rg)
+    if with_beta:
+        assert np.array_equal(npf(bo), rb)
+    with pytest.raises(sq.SqError):
+        sq.sq_smooth_fold_norm(xmax.to(DEV), wmax.to(DEV), 1.5, gamma.to(DEV), None, s, go)
+
+
 # ---------------------------------------------------------------- fold into the previous linear
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16, torch.float32])
 @pytest.mark.parametrize("with_bias", [True, False])

@@ -55,6 +55,7 @@ SIGNATURES = {
     "sq_smooth_scales": ([_p, _p, _i64, _d, _p, _p], _i),
     "sq_fold_weight": ([_p, _i, _i64, _i64, _p, _p, _p], _i),
     "sq_fold_norm": ([_p, _p, _p, _i64, _p, _p, _p], _i),
+    "sq_smooth_fold_norm": ([_p, _p, _i64, _d, _p, _p, _p, _p, _p, _p], _i),
     "sq_fold_prev_linear": ([_p, _i, _i64, _i64, _p, _p, _p, _p, _p], _i),
     "sq_quantize_weight": ([_p, _i, _i64, _i64, _p, _i, _p, _p, _p, _sz, _p], _i),
     "sq_quantize_act": ([_p, _i, _i64, _i64, _i64, _p, _i, _p, _p, _p, _p, _sz, _p], _i),
@@ -183,6 +184,14 @@ def sq_fold_norm(gamma, beta, s, gamma_out, beta_out=None, stream=None):
     _check("sq_fold_norm", lib().sq_fold_norm(_vec(gamma, torch.float32, K), _vec(beta, torch.float32, K),
                                               _vec(s, torch.float32, K), K, _vec(gamma_out, torch.float32, K),
                                               _vec(beta_out, torch.float32, K), _stream(stream)))
+
+
+def sq_smooth_fold_norm(xmax, wmax, alpha, gamma, beta, s_out, gamma_out, beta_out=None, stream=None):
+    K = xmax.numel()
+    _check("sq_smooth_fold_norm", lib().sq_smooth_fold_norm(
+        _vec(xmax, torch.float32, K), _vec(wmax, torch.float32, K), K, float(alpha), _vec(gamma, torch.float32, K),
+        _vec(beta, torch.float32, K), _vec(s_out, torch.float32, K), _vec(gamma_out, torch.float32, K),
+        _vec(beta_out, torch.float32, K), _stream(stream)))
 
 
 def sq_fold_prev_linear(W, s, Wp_out, bias=None, bias_out=None, stream=None):

@@ -18,24 +18,42 @@
 namespace sq {
 namespace {
 
+__device__ __forceinline__ float smooth_one(float x, float w, double alpha) {
+    const float xc = fmaxf(x, 1e-5f);
+    const float wc = fmaxf(w, 1e-5f);
+    double v;
+    if (alpha == 0.5)
+        v = __dsqrt_rn(__ddiv_rn((double)xc, (double)wc));
+    else if (alpha == 0.0)
+        v = __ddiv_rn(1.0, (double)wc);
+    else if (alpha == 1.0)
+        v = (double)xc;
+    else
+        v = __ddiv_rn(pow((double)xc, alpha), pow((double)wc, 1.0 - alpha));
+    return fmaxf(__double2float_rn(v), 1e-5f);
+}
+
 __global__ void smooth_scales_kernel(const float* __restrict__ x, const float* __restrict__ w,
                                      int64_t K, double alpha, float* __restrict__ s) {
     pdl_wait();
     pdl_trigger();
     for (int64_t j = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; j < K;
+         j += (int64_t)gridDim.x * blockDim.x)
+        s[j] = smooth_one(x[j], w[j], alpha);
+}
+
+// s, then gamma' = gamma / s (and beta' = beta / s), in one pass
+__global__ void smooth_fold_norm_kernel(const float* __restrict__ x, const float* __restrict__ w, int64_t K,
+                                        double alpha, const float* __restrict__ g, const float* __restrict__ b,
+                                        float* __restrict__ s, float* __restrict__ g_out, float* __restrict__ b_out) {
+    pdl_wait();
+    pdl_trigger();
+    for (int64_t j = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; j < K;
          j += (int64_t)gridDim.x * blockDim.x) {
-        const float xc = fmaxf(x[j], 1e-5f);
-        const float wc = fmaxf(w[j], 1e-5f);
-        double v;
-        if (alpha == 0.5)
-            v = __dsqrt_rn(__ddiv_rn((double)xc, (double)wc));
-        else if (alpha == 0.0)
-            v = __ddiv_rn(1.0, (double)wc);
-        else if (alpha == 1.0)
-            v = (double)xc;
-        else
-            v = __ddiv_rn(pow((double)xc, alpha), pow((double)wc, 1.0 - alpha));
-        s[j] = fmaxf(__double2float_rn(v), 1e-5f);
+        const float sj = smooth_one(x[j], w[j], alpha);
+        s[j] = sj;
+        g_out[j] = __fdiv_rn(g[j], sj);
+        if (b) b_out[j] = __fdiv_rn(b[j], sj);
     }
 }
 
@@ -173,6 +191,19 @@ sq_status_t sq_fold_prev_linear(const void* W, sq_dtype_t dt, int64_t N, int64_t
         default: return sq::set_error(SQ_ERR_INVALID_ARG, "sq_fold_prev_linear: dtype must be F16, BF16 or F32");
     }
     return sq::check_launch("sq_fold_prev_linear");
+}
+
+sq_status_t sq_smooth_fold_norm(const float* xmax, const float* wmax, int64_t K, double alpha, const float* gamma,
+                                const float* beta, float* s_out, float* gamma_out, float* beta_out, sq_stream_t stream) {
+    const char* name = "sq_smooth_fold_norm";
+    SQ_REQUIRE(xmax && wmax && s_out && gamma && gamma_out, SQ_ERR_INVALID_ARG, "%s: null pointer", name);
+    SQ_REQUIRE((beta == nullptr) == (beta_out == nullptr), SQ_ERR_INVALID_ARG,
+               "%s: beta and beta_out must both be given or both be NULL", name);
+    SQ_REQUIRE(K > 0, SQ_ERR_UNSUPPORTED_SHAPE, "%s: K must be > 0", name);
+    SQ_REQUIRE(alpha >= 0.0 && alpha <= 1.0, SQ_ERR_INVALID_ARG, "%s: alpha must be in [0, 1]", name);
+    sq::launch_pdl(sq::smooth_fold_norm_kernel, dim3(sq::grid_for(K, 256)), dim3(256), 0, sq::as_cuda(stream), xmax,
+                   wmax, K, alpha, gamma, beta, s_out, gamma_out, beta_out);
+    return sq::check_launch(name);
 }
 
 sq_status_t sq_fold_norm(const float* gamma, const float* beta, const float* s, int64_t K,
