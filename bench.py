@@ -9,9 +9,9 @@ fused 1024->4096, o 2048->1024, gate/up fused 1024->6144, down 3072->1024;
   weight absmax over the fused consumers                                x2
   smoothing factors and gamma' = gamma / s (one launch)                 x2
   weight fold + int8 quantisation (per output channel)                  x5
+    (up_proj's also takes 1/s of down_proj's input on its output channels)
   fused RMSNorm + smoothing + per-token int8                            x2
   int8 GEMM + dequant epilogue to bf16                                  x4
-  1/s of down_proj's input folded into up_proj's output channels        x1
   SwiGLU of the gate/up output + per-token int8 (down_proj's input)     x1
   LLM.int8 decomposition of the q/k/v projection (bf16)                 x1
 The independent chains of the step (the attention-side and MLP-side
@@ -53,12 +53,12 @@ METRIC = "W8A8 GEMM TOPS & tokens/s at 1 B200; % of INT8 TC peak / HBM GB/s"
 # GEMM (M, N, K) of one step: qkv, o, gate/up, down, LLM.int8 q/k/v
 GEMMS = [(2048, 4096, 1024), (2048, 1024, 2048), (2048, 6144, 1024), (2048, 1024, 3072), (2048, 4096, 1024)]
 # our kernels in one step: weight absmax 2, calibration absmax 2, smoothing +
-# gamma fold 2, norm passes 4, weight quantisation 5, fold into up_proj 1,
-# GEMMs 4, SwiGLU + int8 1, LLM.int8 5 (counts, compaction, weight-side pass,
-# row quantisation, GEMM)
+# gamma fold 2, norm passes 4, weight quantisation 5 (up_proj's with the fold
+# of down_proj's s), GEMMs 4, SwiGLU + int8 1, LLM.int8 5 (counts, compaction,
+# weight-side pass, row quantisation, GEMM)
 # steps of the instrumented copy of the step that time the GEMM launches
 GEMM_TIMED_STEPS = 200
-LAUNCHES_PER_STEP = (2 * 1 + 2 * 1 + 2 * 1 + 2 * 2 + 5 * 1 + 1 + 4 * 1 + 1 + 5)
+LAUNCHES_PER_STEP = (2 * 1 + 2 * 1 + 2 * 1 + 2 * 2 + 5 * 1 + 4 * 1 + 1 + 5)
 
 
 def peaks():
@@ -210,13 +210,12 @@ class Layer:
         I = self.W["down"].shape[1]
         self.I = I
         self.W_gate, self.W_up = self.W["gateup"][:I], self.W["gateup"][I:]
-        self.W_up_f = e(I, K)
         self.Xq_down = e(M, I, dt=torch.int8)
         self.qx_down = e(M)
         self.s_down = self.calibrate_down()
         self.streams = [torch.cuda.Stream(device=dev) for _ in range(5)]
         self.events = {n: torch.cuda.Event() for n in ("wmax_attn", "wmax_mlp", "V_attn", "V_mlp", "s_attn", "s_mlp",
-                                                      "wq_qkv", "wq_gateup", "wq_down", "up_folded")}
+                                                      "wq_qkv", "wq_gateup", "wq_down")}
 
     def calibrate_down(self):
         """s for down_proj's input, from one pass of the MLP input through the
@@ -272,9 +271,6 @@ class Layer:
         with torch.cuda.stream(sC):
             sq.sq_weight_absmax(self.W["gateup"], self.wmax["mlp"])
             ev["wmax_mlp"].record()
-            # fold into the previous linear: 1/s_down into up_proj's output channels; down_proj takes s_down
-            sq.sq_fold_prev_linear(self.W_up, self.s_down, self.W_up_f)
-            ev["up_folded"].record()
             sq.sq_weight_absmax(self.W["qkv"], self.wmax["attn"])
             ev["wmax_attn"].record()
             sq.sq_quantize_weight(self.W["down"], self.s_down, True, self.Wq["down"], self.qw["down"])
@@ -299,8 +295,10 @@ class Layer:
         with torch.cuda.stream(sD):  # weight quantisation once s is known
             sD.wait_event(ev["s_mlp"])
             sq.sq_quantize_weight(self.W_gate, self.s["mlp"], True, self.Wq["gateup"][:I], self.qw["gateup"][:I])
-            sD.wait_event(ev["up_folded"])
-            sq.sq_quantize_weight(self.W_up_f, self.s["mlp"], True, self.Wq["gateup"][I:], self.qw["gateup"][I:])
+            # up_proj: 1/s_down folded into its output channels (down_proj takes
+            # s_down) and its own s, in the quantising pass
+            sq.sq_quantize_weight_fold_prev(self.W_up, self.s_down, self.s["mlp"], self.Wq["gateup"][I:],
+                                            self.qw["gateup"][I:])
             ev["wq_gateup"].record()
             sD.wait_event(ev["s_attn"])
             sq.sq_quantize_weight(self.W["qkv"], self.s["attn"], True, self.Wq["qkv"], self.qw["qkv"])

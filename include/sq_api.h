@@ -182,6 +182,19 @@ SQ_API sq_status_t sq_quantize_weight(const void* W, sq_dtype_t dt, int64_t N, i
                                const float* s, int per_channel, int8_t* Wq, float* qs_w,
                                void* workspace, size_t ws_bytes, sq_stream_t stream);
 
+/* The fold into this layer's output channels and the int8 quantisation in one
+ * pass     [SQ-p2] 融入前序线性层的权重 with the weight step above: a layer whose
+ * output feeds a smoothed linear (up_proj before down_proj) takes 1/s_next on
+ * its output channels, and its own input smoothing s:
+ *   W'[n,k] = (W[n,k] / s_next[n]) * s[k]  (two fp32 roundings, the values
+ *   sq_fold_prev_linear then sq_quantize_weight would give), then per output
+ *   channel int8 as sq_quantize_weight with per_channel = 1.
+ * s_next: [N] fp32; s: [K] fp32 (16-byte aligned). W: [N,K] of dt in {F16,
+ * BF16, F32}. K % 16 == 0. */
+SQ_API sq_status_t sq_quantize_weight_fold_prev(const void* W, sq_dtype_t dt, int64_t N, int64_t K,
+                                                const float* s_next, const float* s, int8_t* Wq, float* qs_w,
+                                                sq_stream_t stream);
+
 /* --------------------------------------------------------------------------
  * Activation quantisation without a norm     [SQ-p4] §3 (input / s);
  *      [SQ-p1] §3.3; [SQ-p5] §2.1.

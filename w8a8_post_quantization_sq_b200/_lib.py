@@ -54,6 +54,7 @@ SIGNATURES = {
     "sq_weight_absmax": ([_p, _i, _i64, _i64, _i64, _p, _p], _i),
     "sq_smooth_scales": ([_p, _p, _i64, _d, _p, _p], _i),
     "sq_fold_weight": ([_p, _i, _i64, _i64, _p, _p, _p], _i),
+    "sq_quantize_weight_fold_prev": ([_p, _i, _i64, _i64, _p, _p, _p, _p, _p], _i),
     "sq_fold_norm": ([_p, _p, _p, _i64, _p, _p, _p], _i),
     "sq_smooth_fold_norm": ([_p, _p, _i64, _d, _p, _p, _p, _p, _p, _p], _i),
     "sq_fold_prev_linear": ([_p, _i, _i64, _i64, _p, _p, _p, _p, _p], _i),
@@ -184,6 +185,15 @@ def sq_fold_norm(gamma, beta, s, gamma_out, beta_out=None, stream=None):
     _check("sq_fold_norm", lib().sq_fold_norm(_vec(gamma, torch.float32, K), _vec(beta, torch.float32, K),
                                               _vec(s, torch.float32, K), K, _vec(gamma_out, torch.float32, K),
                                               _vec(beta_out, torch.float32, K), _stream(stream)))
+
+
+def sq_quantize_weight_fold_prev(W, s_next, s, Wq, qs_w, stream=None):
+    N, K = W.shape
+    if not W.is_contiguous() or not Wq.is_contiguous():
+        raise ValueError("W and Wq must be contiguous")
+    _check("sq_quantize_weight_fold_prev", lib().sq_quantize_weight_fold_prev(
+        _ptr(W), _dt(W), N, K, _vec(s_next, torch.float32, N), _vec(s, torch.float32, K), _ptr(Wq),
+        _vec(qs_w, torch.float32, N), _stream(stream)))
 
 
 def sq_smooth_fold_norm(xmax, wmax, alpha, gamma, beta, s_out, gamma_out, beta_out=None, stream=None):

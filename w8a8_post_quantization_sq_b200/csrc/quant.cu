@@ -29,7 +29,9 @@ namespace sq {
 namespace {
 
 constexpr int kThreads = 256;
-enum SMode { kNoScale = 0, kMul = 1, kDiv = 2 };
+// kRowDivMul: row n divided by rdiv[n] (the fold of the next layer's smoothing
+// into this one's output channels), then column k multiplied by s[k]
+enum SMode { kNoScale = 0, kMul = 1, kDiv = 2, kRowDivMul = 3 };
 
 // Load 8 consecutive elements as fp32.
 template <typename T>
@@ -43,16 +45,22 @@ __device__ __forceinline__ void load8(const T* p, float* f) {
 }
 
 template <int SM>
-__device__ __forceinline__ void apply_s(float* f, const float* __restrict__ s, int64_t k0) {
+__device__ __forceinline__ void apply_s(float* f, const float* __restrict__ s, const float* __restrict__ rdiv,
+                                        int64_t row, int64_t k0) {
+    if constexpr (SM == kRowDivMul) {
+        const float rd = __ldg(rdiv + row);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) f[e] = __fdiv_rn(f[e], rd);
+    }
     if constexpr (SM != kNoScale) {
         const float4 a = *reinterpret_cast<const float4*>(s + k0);
         const float4 b = *reinterpret_cast<const float4*>(s + k0 + 4);
         const float sv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-        if constexpr (SM == kMul) {
-            mul8(f, sv);
-        } else {
+        if constexpr (SM == kDiv) {
 #pragma unroll
             for (int e = 0; e < 8; ++e) f[e] = __fdiv_rn(f[e], sv[e]);
+        } else {
+            mul8(f, sv);
         }
     }
 }
@@ -125,8 +133,8 @@ __device__ __forceinline__ float warp_max(float v) {
 template <typename T, int SM, int FMT>
 __global__ void __launch_bounds__(kThreads)
 row_quant_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, const float* __restrict__ s,
-                 int per_row, const float* __restrict__ tensor_qs, int8_t* __restrict__ Q,
-                 float* __restrict__ qs_out) {
+                 const float* __restrict__ rdiv, int per_row, const float* __restrict__ tensor_qs,
+                 int8_t* __restrict__ Q, float* __restrict__ qs_out) {
     pdl_wait();
     pdl_trigger();
     const int lane = threadIdx.x & 31;
@@ -140,7 +148,7 @@ row_quant_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, cons
             for (int64_t k0 = lane * 8; k0 < K; k0 += 256) {
                 float f[8];
                 load8<T>(x + k0, f);
-                apply_s<SM>(f, s, k0);
+                apply_s<SM>(f, s, rdiv, row, k0);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(f[e]));
             }
@@ -155,7 +163,7 @@ row_quant_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, cons
         for (int64_t k0 = lane * 8; k0 < K; k0 += 256) {
             float f[8];
             load8<T>(x + k0, f);
-            apply_s<SM>(f, s, k0);
+            apply_s<SM>(f, s, rdiv, row, k0);
             *reinterpret_cast<uint2*>(q + k0) = codes8<FMT>(f, qs, !per_row);
         }
     }
@@ -190,8 +198,8 @@ __device__ __forceinline__ void unpack_raw(const Raw8<T>& r, float* f) {
 template <typename T, int SM, int G, int CH, int FMT>
 __global__ void __launch_bounds__(kThreads)
 row_quant_reg_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, const float* __restrict__ s,
-                     int per_row, const float* __restrict__ tensor_qs, int8_t* __restrict__ Q,
-                     float* __restrict__ qs_out) {
+                     const float* __restrict__ rdiv, int per_row, const float* __restrict__ tensor_qs,
+                     int8_t* __restrict__ Q, float* __restrict__ qs_out) {
     pdl_wait();
     pdl_trigger();
     __shared__ float sh[kThreads / 32];
@@ -217,7 +225,7 @@ row_quant_reg_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, 
             const int64_t k0 = ((int64_t)gt + (int64_t)c * G) * 8;
             if (k0 < K) {
                 unpack_raw<T>(raw[c], v[c]);
-                apply_s<SM>(v[c], s, k0);
+                apply_s<SM>(v[c], s, rdiv, row, k0);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(v[c][e]));
             }
@@ -256,7 +264,7 @@ row_quant_reg_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, 
 template <typename T, int SM>
 __global__ void __launch_bounds__(kThreads)
 tensor_absmax_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld,
-                     const float* __restrict__ s, float* __restrict__ out) {
+                     const float* __restrict__ s, const float* __restrict__ rdiv, float* __restrict__ out) {
     pdl_wait();
     pdl_trigger();
     __shared__ float sh[kThreads / 32];
@@ -268,7 +276,7 @@ tensor_absmax_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld,
         const int64_t k0 = (v - row * vecs_per_row) * 8;
         float f[8];
         load8<T>(X + row * ld + k0, f);
-        apply_s<SM>(f, s, k0);
+        apply_s<SM>(f, s, rdiv, row, k0);
 #pragma unroll
         for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(f[e]));
     }
@@ -304,7 +312,7 @@ int vec_grid(int64_t nvec) {
 template <typename T, int SM, int FMT>
 sq_status_t quantize(const void* Xv, int64_t M, int64_t K, int64_t ld, const float* s, int per_row,
                      const float* static_qs, int8_t* Q, float* qs_out, void* ws, cudaStream_t st,
-                     const char* name) {
+                     const char* name, const float* rdiv = nullptr) {
     const T* X = static_cast<const T*>(Xv);
     const float* tensor_qs = static_qs;
     if (!per_row && !static_qs) {
@@ -312,7 +320,8 @@ sq_status_t quantize(const void* Xv, int64_t M, int64_t K, int64_t ld, const flo
         float* wmax = reinterpret_cast<float*>(static_cast<char*>(ws) + 16);
         float* wqs = wmax + 1;
         if (cudaMemsetAsync(wmax, 0, sizeof(float), st) != cudaSuccess) return check_launch(name);
-        launch_pdl(tensor_absmax_kernel<T, SM>, dim3(vec_grid(M * K / 8)), dim3(kThreads), 0, st, X, M, K, ld, s, wmax);
+        launch_pdl(tensor_absmax_kernel<T, SM>, dim3(vec_grid(M * K / 8)), dim3(kThreads), 0, st, X, M, K, ld, s, rdiv,
+                   wmax);
         launch_pdl(scale_from_absmax_kernel<FMT>, dim3(1), dim3(kThreads), 0, st, wmax, 1, wqs);
         tensor_qs = wqs;
     }
@@ -324,7 +333,8 @@ sq_status_t quantize(const void* Xv, int64_t M, int64_t K, int64_t ld, const flo
         int64_t b = (M + rows_per_block - 1) / rows_per_block;
         const int64_t cap = (int64_t)num_sms() * per_sm;
         if (b > cap) b = cap;
-        return launch_pdl(kern, dim3((unsigned)b), dim3(kThreads), 0, st, X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
+        return launch_pdl(kern, dim3((unsigned)b), dim3(kThreads), 0, st, X, M, K, ld, s, rdiv, per_row, tensor_qs, Q,
+                          qs_out);
     };
     if (K <= 256)
         go(row_quant_reg_kernel<T, SM, 32, 1, FMT>, 8);
@@ -341,7 +351,8 @@ sq_status_t quantize(const void* Xv, int64_t M, int64_t K, int64_t ld, const flo
     else if (K <= 16384)
         go(row_quant_reg_kernel<T, SM, 256, 8, FMT>, 1);
     else
-        launch_pdl(row_quant_kernel<T, SM, FMT>, dim3(row_grid(M)), dim3(kThreads), 0, st, X, M, K, ld, s, per_row, tensor_qs, Q, qs_out);
+        launch_pdl(row_quant_kernel<T, SM, FMT>, dim3(row_grid(M)), dim3(kThreads), 0, st, X, M, K, ld, s, rdiv, per_row,
+                   tensor_qs, Q, qs_out);
     return check_launch(name);
 }
 
@@ -379,6 +390,29 @@ sq_status_t sq_quantize_weight(const void* W, sq_dtype_t dt, int64_t N, int64_t 
         return sq::quantize_dt<sq::kMul>(dt, W, N, K, K, s, per_channel, nullptr, Wq, qs_w, workspace, st, name);
     return sq::quantize_dt<sq::kNoScale>(dt, W, N, K, K, nullptr, per_channel, nullptr, Wq, qs_w, workspace, st,
                                          name);
+}
+
+sq_status_t sq_quantize_weight_fold_prev(const void* W, sq_dtype_t dt, int64_t N, int64_t K, const float* s_next,
+                                         const float* s, int8_t* Wq, float* qs_w, sq_stream_t stream) {
+    const char* name = "sq_quantize_weight_fold_prev";
+    SQ_REQUIRE((W && Wq && qs_w && s_next && s) || N == 0, SQ_ERR_INVALID_ARG, "%s: null pointer", name);
+    SQ_REQUIRE(N >= 0 && K > 0 && K % 16 == 0, SQ_ERR_UNSUPPORTED_SHAPE, "%s: need K > 0 and K %% 16 == 0", name);
+    SQ_REQUIRE(sq::aligned16(W) && sq::aligned16(Wq) && sq::aligned16(s), SQ_ERR_ALIGNMENT,
+               "%s: W, Wq and s must be 16-byte aligned", name);
+    if (N == 0) return SQ_OK;
+    cudaStream_t st = sq::as_cuda(stream);
+    switch (dt) {
+        case SQ_F16:
+            return sq::quantize<__half, sq::kRowDivMul, sq::kI8>(W, N, K, K, s, 1, nullptr, Wq, qs_w, nullptr, st,
+                                                                 name, s_next);
+        case SQ_BF16:
+            return sq::quantize<__nv_bfloat16, sq::kRowDivMul, sq::kI8>(W, N, K, K, s, 1, nullptr, Wq, qs_w, nullptr,
+                                                                        st, name, s_next);
+        case SQ_F32:
+            return sq::quantize<float, sq::kRowDivMul, sq::kI8>(W, N, K, K, s, 1, nullptr, Wq, qs_w, nullptr, st,
+                                                                name, s_next);
+        default: return sq::set_error(SQ_ERR_INVALID_ARG, "%s: dtype must be F16, BF16 or F32", name);
+    }
 }
 
 sq_status_t sq_quantize_act(const void* X, sq_dtype_t dt, int64_t M, int64_t K, int64_t ldx, const float* s,
