@@ -1,0 +1,66 @@
+"""The benchmark step's launch claim against its code (CPU, no kernels run).
+
+bench.py reports `gpu_launches` = LAUNCHES_PER_STEP x steps. This test runs the
+step's host code against stand-ins that record which entry points it calls,
+and adds up the kernels each entry point launches in the step's configuration
+(16-bit inputs under 16 MB for the absmax calls, per-channel weights, K = 1024
+norms, the LLM.int8 weight state keeping its W_O copy, O unchanged)."""
+from unittest import mock
+
+import bench
+
+# kernels per call of each entry point in the step's configuration
+KERNELS = {
+    "sq_weight_absmax": 1,
+    "sq_calib_absmax": 1,
+    "sq_smooth_fold_norm": 1,
+    "sq_norm_smooth_quant": 1,
+    "sq_quantize_weight": 1,
+    "sq_quantize_weight_fold_prev": 1,
+    "sq_gemm_w8a8": 1,
+    "sq_act_quant": 1,
+    # counts, compaction, weight-side pass, row quantisation, GEMM
+    "sq_llmint8_matmul": 5,
+}
+
+
+class RecordingSQ:
+    def __init__(self):
+        self.calls = []
+
+    def __getattr__(self, name):
+        if name.startswith("SQ_"):
+            return 0
+
+        def call(*args, **kwargs):
+            self.calls.append(name)
+        return call
+
+
+def run_step_host_code():
+    sq = RecordingSQ()
+    layer = mock.MagicMock()
+    layer.sq = sq
+    layer.torch = mock.MagicMock()
+    layer.d = {"eps": 1e-6, "alpha": 0.5}
+    layer.I = 3072
+    layer.streams = [mock.MagicMock() for _ in range(5)]
+    layer.act_in = {"o": (mock.MagicMock(), mock.MagicMock()), "down": (mock.MagicMock(), mock.MagicMock())}
+    bench.Layer.step(layer)
+    return sq.calls
+
+
+def test_step_calls_known_entry_points():
+    calls = run_step_host_code()
+    assert calls, "the step made no calls"
+    assert set(calls) <= set(KERNELS), set(calls) - set(KERNELS)
+
+
+def test_launch_claim_matches_the_step():
+    calls = run_step_host_code()
+    assert sum(KERNELS[c] for c in calls) == bench.LAUNCHES_PER_STEP
+    # every row of the path is in the step
+    for row in ("sq_calib_absmax", "sq_weight_absmax", "sq_smooth_fold_norm", "sq_quantize_weight",
+                "sq_norm_smooth_quant", "sq_gemm_w8a8", "sq_llmint8_matmul", "sq_act_quant",
+                "sq_quantize_weight_fold_prev"):
+        assert row in calls, row
