@@ -293,7 +293,6 @@ norm_quant_warp_kernel(const T* __restrict__ H, NormArgs a) {
                 if (ch < nch) {
                     float v[8];
                     compute_v<T, LN>(raw[i], ch, a, mu, r, v);
-#pragma unroll
                     m = absmax8(m, v);
                     if (a.absmax) {
 #pragma unroll
@@ -528,7 +527,6 @@ norm_quant_bulk_kernel(const T* __restrict__ H, NormArgs a, int R) {
                     float* v = KEEPV ? vk[c] : vl;
                     if constexpr (KEEPV) compute_v_d(vk[c], b_lo(ch), b_hi(ch), g[c], r, v);  // vk holds d
                     else compute_v_g<T, LN>(chunk(c), b_lo(ch), b_hi(ch), g[c], mu, r, v);
-#pragma unroll
                     m = absmax8(m, v);
                     if constexpr (!QONLY) {
                         if (a.absmax) {
