@@ -57,7 +57,7 @@ def test_sharded_calibration_and_max_over_ranks():
 
 
 def test_reference_arm_under_torchrun():
-    """`bench.py --impl reference` launched like the driver does for N = 2:
+    """`bench.py --impl reference` launched by torchrun with two ranks:
     rank 0 prints one JSON line, rank 1 exits 0 without work."""
     port = _free_port()
     cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
