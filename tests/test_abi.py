@@ -127,6 +127,15 @@ def test_argument_validation_without_gpu(L):
             "static")
     # smoothing: alpha out of range
     _expect(L, L.sq_smooth_scales(p, p, 16, 1.5, p, None), 1, "alpha")
+    # smoothing fused with the norm fold: alpha out of range, beta without beta_out, K = 0
+    _expect(L, L.sq_smooth_fold_norm(p, p, 16, -0.1, p, None, p, p, None, None), 1, "alpha")
+    _expect(L, L.sq_smooth_fold_norm(p, p, 16, 0.5, p, p, p, p, None, None), 1, "beta_out")
+    _expect(L, L.sq_smooth_fold_norm(p, p, 0, 0.5, p, None, p, p, None, None), 2, "K")
+    # weight quantisation with the next block's 1/s folded into its rows: K, alignment, dtype
+    _expect(L, L.sq_quantize_weight_fold_prev(p, 2, 4, 24, p, p, p, p, None), 2, "K % 16")
+    _expect(L, L.sq_quantize_weight_fold_prev(p, 2, 4, 16, p, odd, p, p, None), 3, "aligned")
+    _expect(L, L.sq_quantize_weight_fold_prev(p, 7, 4, 16, p, p, p, p, None), 1, "dtype")
+    _expect(L, L.sq_quantize_weight_fold_prev(p, 2, 4, 16, None, p, p, p, None), 1, "null")
     # absmax: stride smaller than K
     _expect(L, L.sq_calib_absmax(p, 2, 4, 16, 8, p, None), 2, "sizes")
     # quantize_act: dynamic per-tensor without workspace
