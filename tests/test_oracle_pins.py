@@ -391,6 +391,33 @@ def test_llmint8_planted_and_accuracy(orc):
     assert err < 2e-2 and err < err_v / 2
 
 
+def test_llmint8_exact_on_dyadic_grid(orc):
+    """When every row of X outside O has absmax 127/32 and every row of W
+    outside O has absmax 127/64, with all entries on those grids, the
+    vector-wise codes are the grid integers and the dequantised int8 part is
+    exact; the outlier term (whole numbers times grid values) is exact too.
+    The decomposition then returns X·Wᵀ exactly, so a dropped or doubled
+    outlier term, an outlier column left in a row's absmax, a transposed
+    operand or a wrong scale fails it (LLM.int8() decomposition, the
+    outlier/vector-wise split of "LLM.int8()" §2.2)."""
+    rng = np.random.default_rng(20)
+    M, K, N = 24, 96, 40
+    dims = [5, 47, 90]
+    X = rng.integers(-127, 128, size=(M, K)).astype(np.float32) / 32.0
+    X[:, 0] = np.where(rng.random(M) < 0.5, -127.0, 127.0) / 32.0  # row absmax outside O
+    for d in dims:
+        X[rng.permutation(M)[:6], d] = rng.choice([-40.0, -30.0, 9.0, 30.0, 40.0], 6)
+    W = rng.integers(-127, 128, size=(N, K)).astype(np.float32) / 64.0
+    W[:, 1] = np.where(rng.random(N) < 0.5, -127.0, 127.0) / 64.0
+    y, idx, Xq, qx, Wq, qw = orc.llmint8_matmul(X, W, 6.0)
+    assert idx.tolist() == dims
+    assert np.all(qx == 32.0) and np.all(qw == 64.0)
+    keep = np.setdiff1d(np.arange(K), dims)
+    assert np.array_equal(Xq[:, keep].astype(np.float64), X[:, keep].astype(np.float64) * 32)
+    assert np.array_equal(Wq[:, keep].astype(np.float64), W[:, keep].astype(np.float64) * 64)
+    assert np.array_equal(y, X.astype(np.float64) @ W.astype(np.float64).T)
+
+
 def test_vectorwise_toy_magnitude(orc):
     """"8位量化" §2.1 toy: X(4x8), W(8x16) from default_rng(0), X[0,3] = 40;
     vector-wise int8 gives a relative error of order 1e-3..1e-2. A magnitude
