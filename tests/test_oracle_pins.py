@@ -292,6 +292,39 @@ def test_dequant_closed_form(orc):
     assert y[0, 1] == -127 * 64 / (63.5 * 127) - 1.0
 
 
+def test_static_scale_from_calibration_absmax(orc):
+    """A static per-tensor scale is 127 over the largest calibrated channel
+    absmax ("8位量化" §2.1, one scale for the whole tensor): closed forms, the
+    1e-8 floor of an all-zero calibration, and agreement with the dynamic
+    per-tensor scale of a tensor whose absmax is that value."""
+    assert orc.scale_from_absmax(np.array([0.5, 2.0, 1.0], np.float32)) == np.float32(63.5)
+    assert orc.scale_from_absmax(np.array([127.0], np.float32)) == np.float32(1.0)
+    assert orc.scale_from_absmax(np.zeros(4, np.float32)) == np.float32(127.0) / np.float32(1e-8)
+    rng = np.random.default_rng(13)
+    X = rng.normal(size=(9, 48)).astype(np.float32)
+    Xq, qs = orc.quantize_act(X, None, per_token=False)
+    assert qs[0] == orc.scale_from_absmax(np.abs(X).max(0))
+    Xq2, _ = orc.quantize_act(X, None, per_token=False, static_qs=qs[0])
+    assert np.array_equal(Xq, Xq2)
+
+
+def test_dequant_f64_accumulators(orc):
+    """The fp64-accumulator dequant (for FP8 products, whose sums are not
+    integers) is the same outer-product formula: exact on power-of-two
+    scales, per-tensor and per-row/per-column indexing, bias added last."""
+    acc = np.array([[1.5, -3.0, 0.0], [96.0, 0.25, -7.75]], np.float64)
+    qx = np.array([2.0, 0.5], np.float32)
+    qw = np.array([4.0, 8.0, 0.25], np.float32)
+    b = np.array([1.0, -0.5, 0.125], np.float32)
+    y = orc.dequant_f64(acc, qx, qw, bias=b)
+    ref = acc / (qx.astype(np.float64)[:, None] * qw.astype(np.float64)[None, :]) + b.astype(np.float64)
+    assert np.array_equal(y, ref)
+    y1 = orc.dequant_f64(acc, np.array([2.0], np.float32), np.array([4.0], np.float32))
+    assert np.array_equal(y1, acc / 8.0)
+    assert np.array_equal(orc.dequant_f64(acc.astype(np.int64).astype(np.float64), qx, qw),
+                          orc.dequant(acc.astype(np.int64), qx, qw))
+
+
 def test_dequant_row_and_column_scales(orc):
     """Scales factor out only per row (token) and per column (output channel):
     Y = diag(dX) Xq Wq^T diag(dW) ("为什么激活不能用逐通道量化")."""
