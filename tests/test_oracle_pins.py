@@ -127,6 +127,22 @@ def test_fold_f32_is_one_rounding(orc):
     assert np.array_equal(Wp, (W * s[None, :]).astype(np.float32))
 
 
+def test_norm_fold_f32_is_one_division(orc):
+    """The fp32 norm fold gamma' = gamma/s, beta' = beta/s ("融入 LayerNorm")
+    is the IEEE fp32 quotient: the fp64 quotient of two fp32 values rounded
+    to fp32 is the correctly rounded fp32 quotient (53 >= 2*24 + 2, so the
+    double rounding is innocuous). RMSNorm has no beta."""
+    rng = np.random.default_rng(8)
+    K = 4099
+    gamma = (1 + 0.1 * rng.normal(size=K)).astype(np.float32)
+    beta = (0.1 * rng.normal(size=K)).astype(np.float32)
+    s = (rng.random(K) * 20 + 1e-3).astype(np.float32)
+    gp, bp = orc.fold_norm(gamma, beta, s)
+    assert np.array_equal(gp, gamma / s) and np.array_equal(bp, beta / s)
+    gp2, bp2 = orc.fold_norm(gamma, None, s)
+    assert bp2 is None and np.array_equal(gp2, gp)
+
+
 def test_norm_fold_identity_fp64(orc):
     """"融入 LayerNorm": with gamma' = gamma/s and beta' = beta/s the norm output
     is y/s (fp64, 1e-12), for LayerNorm and RMSNorm."""
