@@ -712,6 +712,23 @@ def test_bmm_bruteforce(orc):
     assert np.array_equal(orc.bmm_i8(A, B), ref)
 
 
+def test_bmm_dequant_per_problem_scales(orc):
+    """Problem b divides by its own row and column scales, and a row subset
+    picks the matching row scales; exact on power-of-two scales."""
+    rng = np.random.default_rng(52)
+    B, T, S = 3, 6, 5
+    acc = rng.integers(-2 ** 20, 2 ** 20, size=(B, T, S)).astype(np.int64)
+    qa = [(2.0 ** rng.integers(-4, 5, size=T)).astype(np.float32) for _ in range(B)]
+    qb = [(2.0 ** rng.integers(-4, 5, size=S)).astype(np.float32) for _ in range(B)]
+    y = orc.bmm_dequant(acc, qa, qb)
+    ref = np.stack([acc[b] / (qa[b].astype(np.float64)[:, None] * qb[b].astype(np.float64)[None, :])
+                    for b in range(B)])
+    assert np.array_equal(y, ref)
+    rows = [1, 4]
+    ys = orc.bmm_dequant(acc[:, rows], qa, qb, rows=rows)
+    assert np.array_equal(ys, ref[:, rows])
+
+
 def test_bmm_attention_scores_magnitude(orc):
     """lpnh.cn SmoothQuant practice article §2.2: QK^T in int8 with one scale
     per (head, token) on Q and on K approximates the fp64 scores; PV with P
