@@ -145,3 +145,57 @@ def test_argument_validation_without_gpu(L):
     # M == 0 is a valid empty call (nothing launched)
     assert L.sq_gemm_w8a8(p, p, 0, 16, 16, p, 1, p, 1, None, 2, p, 16, p, 256, None) == 0
     assert L.sq_calib_absmax(p, 2, 0, 16, 16, p, None) == 0
+
+
+def test_binding_checks_before_the_call(L):
+    """The Python binding rejects host tensors (there is no CPU path) and
+    buffers too small for what the library reads or writes, before any
+    pointer reaches the library."""
+    import torch
+
+    from w8a8_post_quantization_sq_b200 import _lib as sq
+
+    M, N, K = 8, 16, 32
+    Xq, Wq = torch.zeros((M, K), dtype=torch.int8), torch.zeros((N, K), dtype=torch.int8)
+    Y = torch.empty((M, N), dtype=torch.bfloat16)
+    ws = torch.zeros(256, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="CUDA device"):
+        sq.sq_gemm_w8a8(Xq, Wq, torch.ones(M), torch.ones(N), None, Y, ws)
+    with pytest.raises(ValueError, match="qs_x"):
+        sq.sq_gemm_w8a8(Xq, Wq, torch.ones(M - 1), torch.ones(N), None, Y, ws)
+    with pytest.raises(ValueError, match="qs_w"):
+        sq.sq_gemm_fp8(Xq.view(torch.uint8), Wq.view(torch.uint8), torch.ones(1), torch.ones(3), None, Y, ws)
+    with pytest.raises(ValueError, match="shape"):
+        sq.sq_gemm_fp8(Xq.view(torch.uint8), Wq.view(torch.uint8), None, None, None, Y[:, :4], ws)
+    H = torch.zeros((M, K), dtype=torch.bfloat16)
+    g = torch.ones(K)
+    with pytest.raises(ValueError, match="qs_x"):
+        sq.sq_norm_smooth_quant(H, sq.SQ_RMSNORM, g, None, 1e-6, True, None, Xq, torch.ones(M - 1))
+    with pytest.raises(ValueError, match="Xq"):
+        sq.sq_norm_smooth_quant(H, sq.SQ_RMSNORM, g, None, 1e-6, True, None, Xq[:, :16].contiguous(), torch.ones(M))
+    with pytest.raises(ValueError, match="Xq"):
+        sq.sq_quantize_act(H, None, True, None, Xq.float(), torch.ones(M))
+    with pytest.raises(ValueError, match="Wq"):
+        sq.sq_quantize_weight_fold_prev(H, torch.ones(M), g, Wq.view(torch.uint8), torch.ones(M))
+    with pytest.raises(ValueError, match="Xq"):
+        sq.sq_act_quant(torch.zeros((M, 2 * K), dtype=torch.bfloat16), sq.SQ_ACT_SWIGLU, True, None,
+                        torch.zeros((M, K - 8), dtype=torch.int8), torch.ones(M))
+    with pytest.raises(ValueError, match="qs_a"):
+        sq.sq_bmm_w8a8(Xq.view(1, M, K).repeat(2, 1, 1), Wq.view(1, N, K).repeat(2, 1, 1), torch.ones(1), None,
+                       torch.empty((2, M, N), dtype=torch.int32), ws)
+    st = {"W": torch.zeros((N, K), dtype=torch.float16)}
+    with pytest.raises(ValueError, match="Y must be"):
+        sq.sq_llmint8_matmul(torch.zeros((M, K), dtype=torch.float16), st, 6.0, 0.0, Y, None, None, ws)
+    with pytest.raises(ValueError, match="weight state"):
+        sq.sq_llmint8_matmul(torch.zeros((M, 2 * K), dtype=torch.float16), st, 6.0, 0.0,
+                             torch.empty((M, N), dtype=torch.float16), None, None, ws)
+
+
+def test_missing_library_raises(monkeypatch):
+    """Without the built library the first call raises; nothing falls back."""
+    from w8a8_post_quantization_sq_b200 import _lib as sq
+
+    monkeypatch.setattr(sq, "LIB_PATH", os.path.join(ROOT, "_no_such_dir", "libsq_b200.so"))
+    monkeypatch.setattr(sq, "_lib", None)
+    with pytest.raises(RuntimeError, match="not built"):
+        sq.sq_version()

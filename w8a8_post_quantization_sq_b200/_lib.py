@@ -104,6 +104,8 @@ def _ptr(t):
         return None
     if not t.is_cuda:
         raise ValueError("tensor must be on a CUDA device")
+    if t.device.index is not None and t.device.index != torch.cuda.current_device():
+        raise ValueError(f"tensor on {t.device}, but the current device is cuda:{torch.cuda.current_device()}")
     return ctypes.c_void_p(t.data_ptr())
 
 
@@ -120,6 +122,23 @@ def _ld(t):
     if t.dim() != 2 or t.stride(1) != 1:
         raise ValueError("expected a 2-D tensor with unit inner stride")
     return t.stride(0)
+
+
+def _need(ok, msg):
+    if not ok:
+        raise ValueError(msg)
+
+
+def _out(t, dtype, n, what):
+    """An output the library writes n elements of, back to back."""
+    _need(t.dtype == dtype and t.is_contiguous() and t.numel() >= n,
+          f"{what} must be a contiguous {dtype} tensor of at least {n} elements")
+
+
+def _scales(t, n, what):
+    """One scale, or one per row/column: the library reads n entries whenever
+    the tensor holds more than one."""
+    _need(t is None or t.numel() == 1 or t.numel() >= n, f"{what} must hold 1 or at least {n} scales")
 
 
 def _vec(t, dtype, n=None):
@@ -174,8 +193,8 @@ def sq_smooth_scales(xmax, wmax, alpha, s_out, stream=None):
 
 def sq_fold_weight(W, s, Wp_out, stream=None):
     N, K = W.shape
-    if not W.is_contiguous() or not Wp_out.is_contiguous() or Wp_out.dtype != torch.float32:
-        raise ValueError("W and Wp_out must be contiguous; Wp_out fp32")
+    _need(W.is_contiguous(), "W must be contiguous")
+    _out(Wp_out, torch.float32, N * K, "Wp_out")
     _check("sq_fold_weight", lib().sq_fold_weight(_ptr(W), _dt(W), N, K, _vec(s, torch.float32, K), _ptr(Wp_out),
                                                   _stream(stream)))
 
@@ -189,8 +208,8 @@ def sq_fold_norm(gamma, beta, s, gamma_out, beta_out=None, stream=None):
 
 def sq_quantize_weight_fold_prev(W, s_next, s, Wq, qs_w, stream=None):
     N, K = W.shape
-    if not W.is_contiguous() or not Wq.is_contiguous():
-        raise ValueError("W and Wq must be contiguous")
+    _need(W.is_contiguous(), "W must be contiguous")
+    _out(Wq, torch.int8, N * K, "Wq")
     _check("sq_quantize_weight_fold_prev", lib().sq_quantize_weight_fold_prev(
         _ptr(W), _dt(W), N, K, _vec(s_next, torch.float32, N), _vec(s, torch.float32, K), _ptr(Wq),
         _vec(qs_w, torch.float32, N), _stream(stream)))
@@ -206,8 +225,8 @@ def sq_smooth_fold_norm(xmax, wmax, alpha, gamma, beta, s_out, gamma_out, beta_o
 
 def sq_fold_prev_linear(W, s, Wp_out, bias=None, bias_out=None, stream=None):
     N, K = W.shape
-    if not W.is_contiguous() or not Wp_out.is_contiguous() or Wp_out.dtype != torch.float32:
-        raise ValueError("W and Wp_out must be contiguous; Wp_out fp32")
+    _need(W.is_contiguous(), "W must be contiguous")
+    _out(Wp_out, torch.float32, N * K, "Wp_out")
     _check("sq_fold_prev_linear", lib().sq_fold_prev_linear(
         _ptr(W), _dt(W), N, K, _vec(bias, torch.float32, N), _vec(s, torch.float32, N), _ptr(Wp_out),
         _vec(bias_out, torch.float32, N), _stream(stream)))
@@ -216,8 +235,8 @@ def sq_fold_prev_linear(W, s, Wp_out, bias=None, bias_out=None, stream=None):
 # ---------------------------------------------------------------- weight quantisation
 def sq_quantize_weight(W, s, per_channel, Wq, qs_w, ws=None, stream=None):
     N, K = W.shape
-    if not W.is_contiguous() or not Wq.is_contiguous() or Wq.dtype != torch.int8:
-        raise ValueError("W and Wq must be contiguous; Wq int8")
+    _need(W.is_contiguous(), "W must be contiguous")
+    _out(Wq, torch.int8, N * K, "Wq")
     _check("sq_quantize_weight", lib().sq_quantize_weight(
         _ptr(W), _dt(W), N, K, _vec(s, torch.float32, K), int(per_channel), _ptr(Wq),
         _vec(qs_w, torch.float32, N if per_channel else 1), _ptr(ws), 0 if ws is None else ws.numel(),
@@ -227,8 +246,7 @@ def sq_quantize_weight(W, s, per_channel, Wq, qs_w, ws=None, stream=None):
 # ---------------------------------------------------------------- activation quantisation without a norm
 def sq_quantize_act(X, s, per_token, static_qs, Xq, qs_x, ws=None, stream=None):
     M, K = X.shape
-    if not Xq.is_contiguous() or Xq.dtype != torch.int8:
-        raise ValueError("Xq must be contiguous int8")
+    _out(Xq, torch.int8, M * K, "Xq")
     _check("sq_quantize_act", lib().sq_quantize_act(
         _ptr(X), _dt(X), M, K, _ld(X), _vec(s, torch.float32, K), int(per_token), _vec(static_qs, torch.float32, 1),
         _ptr(Xq), _vec(qs_x, torch.float32, M if per_token else 1), _ptr(ws), 0 if ws is None else ws.numel(),
@@ -244,10 +262,12 @@ def sq_scale_from_absmax(absmax, qs_out, stream=None):
 def sq_norm_smooth_quant(H, norm, gamma, beta, eps, per_token, static_qs, Xq, qs_x, absmax=None, V=None,
                          stream=None):
     M, K = H.shape
-    if Xq is not None and (not Xq.is_contiguous() or Xq.dtype != torch.int8):
-        raise ValueError("Xq must be contiguous int8")
-    if V is not None and (V.dtype != H.dtype or not V.is_contiguous()):
-        raise ValueError("V must be contiguous with the dtype of H")
+    if Xq is not None:
+        _out(Xq, torch.int8, M * K, "Xq")
+        _need(qs_x is not None and qs_x.numel() >= (M if per_token else 1),
+              f"qs_x must hold {M if per_token else 1} scales")
+    if V is not None:
+        _out(V, H.dtype, M * K, "V")
     _check("sq_norm_smooth_quant", lib().sq_norm_smooth_quant(
         _ptr(H), _dt(H), M, K, _ld(H), int(norm), _vec(gamma, torch.float32, K), _vec(beta, torch.float32, K),
         float(eps), int(per_token), _vec(static_qs, torch.float32, 1), _ptr(Xq),
@@ -267,6 +287,8 @@ def sq_bmm_w8a8(Aq, Bq, qs_a, qs_b, Y, ws, stream=None):
         raise ValueError("shape mismatch")
     if Y.stride(2) != 1 or Y.stride(0) != M * Y.stride(1):
         raise ValueError("Y must be [batch, M, ldy] with batches back to back")
+    _need(qs_a is None or qs_a.numel() >= b, f"qs_a must hold one scale per problem ({b}) or per row")
+    _need(qs_b is None or qs_b.numel() >= b, f"qs_b must hold one scale per problem ({b}) or per row")
     _check("sq_bmm_w8a8", lib().sq_bmm_w8a8(
         _ptr(Aq), _ptr(Bq), b, M, N, K, _vec(qs_a, torch.float32), int(qs_a is not None and qs_a.numel() == b * M),
         _vec(qs_b, torch.float32), int(qs_b is not None and qs_b.numel() == b * N), _dt(Y), _ptr(Y), Y.stride(1),
@@ -276,8 +298,8 @@ def sq_bmm_w8a8(Aq, Bq, qs_a, qs_b, Y, ws, stream=None):
 # ---------------------------------------------------------------- FP8 variant
 def sq_quantize_weight_fp8(W, s, per_channel, Wq, qs_w, ws=None, stream=None):
     N, K = W.shape
-    if not W.is_contiguous() or not Wq.is_contiguous() or Wq.dtype != torch.uint8:
-        raise ValueError("W and Wq must be contiguous; Wq uint8 (E4M3 codes)")
+    _need(W.is_contiguous(), "W must be contiguous")
+    _out(Wq, torch.uint8, N * K, "Wq (E4M3 codes)")
     _check("sq_quantize_weight_fp8", lib().sq_quantize_weight_fp8(
         _ptr(W), _dt(W), N, K, _vec(s, torch.float32, K), int(per_channel), _ptr(Wq),
         _vec(qs_w, torch.float32, N if per_channel else 1), _ptr(ws), 0 if ws is None else ws.numel(),
@@ -286,8 +308,7 @@ def sq_quantize_weight_fp8(W, s, per_channel, Wq, qs_w, ws=None, stream=None):
 
 def sq_quantize_act_fp8(X, s, per_token, static_qs, Xq, qs_x, ws=None, stream=None):
     M, K = X.shape
-    if not Xq.is_contiguous() or Xq.dtype != torch.uint8:
-        raise ValueError("Xq must be contiguous uint8 (E4M3 codes)")
+    _out(Xq, torch.uint8, M * K, "Xq (E4M3 codes)")
     _check("sq_quantize_act_fp8", lib().sq_quantize_act_fp8(
         _ptr(X), _dt(X), M, K, _ld(X), _vec(s, torch.float32, K), int(per_token), _vec(static_qs, torch.float32, 1),
         _ptr(Xq), _vec(qs_x, torch.float32, M if per_token else 1), _ptr(ws), 0 if ws is None else ws.numel(),
@@ -299,6 +320,10 @@ def sq_gemm_fp8(Xq, Wq, qs_x, qs_w, bias, Y, ws, stream=None):
     N = Wq.shape[0]
     if Xq.dtype != torch.uint8 or Wq.dtype != torch.uint8 or not Xq.is_contiguous() or not Wq.is_contiguous():
         raise ValueError("Xq and Wq must be contiguous uint8 (E4M3 codes)")
+    if Wq.shape[1] != K or Y.shape[0] != M or Y.shape[1] != N:
+        raise ValueError("shape mismatch")
+    _scales(qs_x, M, "qs_x")
+    _scales(qs_w, N, "qs_w")
     _check("sq_gemm_fp8", lib().sq_gemm_fp8(
         _ptr(Xq), _ptr(Wq), M, N, K, _vec(qs_x, torch.float32), int(qs_x.numel() > 1), _vec(qs_w, torch.float32),
         int(qs_w.numel() > 1), _vec(bias, torch.float32, N), _dt(Y), _ptr(Y), _ld(Y), _ptr(ws), ws.numel(),
@@ -310,10 +335,12 @@ def sq_act_quant(A, act, per_token, static_qs, Xq, qs_x, absmax=None, H=None, st
     """A: [M, 2I] ([gate | up], SQ_ACT_SWIGLU) or [M, I] (SQ_ACT_RELU)."""
     M, W = A.shape
     I = W // 2 if act == SQ_ACT_SWIGLU else W
-    if Xq is not None and (not Xq.is_contiguous() or Xq.dtype != torch.int8):
-        raise ValueError("Xq must be contiguous int8")
-    if H is not None and (H.dtype != A.dtype or not H.is_contiguous()):
-        raise ValueError("H must be contiguous with the dtype of A")
+    if Xq is not None:
+        _out(Xq, torch.int8, M * I, "Xq")
+        _need(qs_x is not None and qs_x.numel() >= (M if per_token else 1),
+              f"qs_x must hold {M if per_token else 1} scales")
+    if H is not None:
+        _out(H, A.dtype, M * I, "H")
     _check("sq_act_quant", lib().sq_act_quant(
         _ptr(A), _dt(A), M, I, _ld(A), int(act), int(per_token), _vec(static_qs, torch.float32, 1), _ptr(Xq),
         None if qs_x is None else _vec(qs_x, torch.float32), _vec(absmax, torch.float32, I), _ptr(H),
@@ -328,6 +355,8 @@ def sq_gemm_w8a8(Xq, Wq, qs_x, qs_w, bias, Y, ws, stream=None):
         raise ValueError("Xq and Wq must be contiguous int8")
     if Wq.shape[1] != K or Y.shape[0] != M or Y.shape[1] != N:
         raise ValueError("shape mismatch")
+    _scales(qs_x, M, "qs_x")
+    _scales(qs_w, N, "qs_w")
     _check("sq_gemm_w8a8", lib().sq_gemm_w8a8(
         _ptr(Xq), _ptr(Wq), M, N, K, _vec(qs_x, torch.float32), int(qs_x is not None and qs_x.numel() > 1),
         _vec(qs_w, torch.float32), int(qs_w is not None and qs_w.numel() > 1), _vec(bias, torch.float32, N),
@@ -352,6 +381,7 @@ def sq_llmint8_detect_noalloc(X, threshold, min_ratio, idx, n, stream=None):
 
 def sq_llmint8_quant_rows(X, idx, n, Xq, qs_x, stream=None):
     M, K = X.shape
+    _out(Xq, torch.int8, M * K, "Xq")
     _check("sq_llmint8_quant_rows", lib().sq_llmint8_quant_rows(
         _ptr(X), _dt(X), M, K, _ld(X), _vec(idx, torch.int32), _vec(n, torch.int32, 1), _ptr(Xq),
         _vec(qs_x, torch.float32, M), _stream(stream)))
@@ -359,8 +389,8 @@ def sq_llmint8_quant_rows(X, idx, n, Xq, qs_x, stream=None):
 
 def sq_llmint8_quant_weight(W, idx, n, Wq, qs_w, stream=None):
     N, K = W.shape
-    if not W.is_contiguous():
-        raise ValueError("W must be contiguous")
+    _need(W.is_contiguous(), "W must be contiguous")
+    _out(Wq, torch.int8, N * K, "Wq")
     _check("sq_llmint8_quant_weight", lib().sq_llmint8_quant_weight(
         _ptr(W), _dt(W), N, K, _vec(idx, torch.int32), _vec(n, torch.int32, 1), _ptr(Wq),
         _vec(qs_w, torch.float32, N), _stream(stream)))
@@ -384,6 +414,9 @@ def llmint8_weight_state(W, keep_wo=True):
 
 def sq_llmint8_matmul(X, wstate, threshold, min_ratio, Y, idx, n, ws, stream=None):
     M, K = X.shape
+    W = wstate["W"]
+    _need(W.dtype == X.dtype and W.dim() == 2 and W.shape[1] == K, "the weight state's W must be [N, K] of X's dtype")
+    _need(Y.dtype == X.dtype and tuple(Y.shape) == (M, W.shape[0]), "Y must be [M, N] of X's dtype")
     _check("sq_llmint8_matmul", lib().sq_llmint8_matmul(
         _ptr(X), _dt(X), M, K, _ld(X), ctypes.byref(wstate["c"]), float(threshold), float(min_ratio), _ptr(Y),
         _ld(Y), _vec(idx, torch.int32, K), _vec(n, torch.int32, 1), _ptr(ws), ws.numel(), _stream(stream)))
