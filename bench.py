@@ -458,92 +458,120 @@ def run_ours(args, rank, world, dev):
 
 
 # ------------------------------------------------------------------ CPU arm
-def cpu_step_sample(rows):
-    """The oracle, as it stands, on the same step for `rows` tokens of the
-    workload (weights in full). Returns (seconds of weight-side work,
-    seconds of per-token work for `rows` tokens). The smoothing factors of
-    down_proj's input come from an untimed calibration pass over the sample,
-    as the GPU step takes them from its set-up."""
-    import torch
+class CpuStep:
+    """The oracle, as it stands, on the benchmark's step, timed on a sample.
 
-    import oracle
-    from w8a8_post_quantization_sq_b200 import inputs
+    The inputs, and the step's set-up (down_proj's smoothing factors from a
+    calibration pass, and the full int8 weights the token rows multiply), are
+    made once, untimed. Each call of ``step(rows, wfrac)`` then times the
+    whole path on a sample: the per-token work for ``rows`` tokens, and the
+    weight-side work (maxima, smoothing factors, folds, quantisation, the
+    LLM.int8 weight requantisation) on the first ``wfrac`` of every weight's
+    output channels. Both are linear in what they process, so the step time
+    of the full workload is t_weights / wfrac + t_rows * tokens / rows."""
 
-    oracle.lib()
-    d = inputs.c2_qwen3_06b(device="cpu")
-    sl = slice(0, rows)
-    h = {"attn": d["h_attn"][sl], "mlp": d["h_mlp"][sl]}
-    gamma = {"attn": d["gamma_attn"].numpy(), "mlp": d["gamma_mlp"].numpy()}
-    W = {k: oracle.f32(v) for k, v in d["W"].items()}
-    I = W["down"].shape[1]
+    def __init__(self, rows=64):
+        import torch
 
-    def bf16(y):
-        return torch.from_numpy(oracle.round_bf16_bits(y).view(np.int16)).view(torch.bfloat16).float().numpy()
+        import oracle
+        from w8a8_post_quantization_sq_b200 import inputs
 
-    # set-up (untimed): s of down_proj's input
-    Vc = oracle.norm_smooth_quant(d["h_calib"][sl], oracle.RMSNORM, gamma["mlp"], None, d["eps"], quantize=False,
-                                  want_v=True)["V"]
-    Vc16 = torch.from_numpy(Vc).to(torch.bfloat16).float().numpy()
-    Xc, qc = oracle.quantize_act(Vc16, None, per_token=True)
-    Wc, qwc = oracle.quantize_weight(W["gateup"], True)
-    hmax = oracle.act_quant(bf16(oracle.dequant(oracle.gemm_i8(Xc, Wc), qc, qwc)), oracle.SWIGLU, quantize=False,
-                            absmax=np.zeros(I, np.float32))["absmax"]
-    s_down = oracle.smooth_scales(hmax, oracle.col_absmax(W["down"]), d["alpha"])
+        oracle.lib()
+        self.o, self.torch = oracle, torch
+        d = inputs.c2_qwen3_06b(device="cpu")
+        self.d = d
+        self.gamma = {"attn": d["gamma_attn"].numpy(), "mlp": d["gamma_mlp"].numpy()}
+        self.W = W = {k: oracle.f32(v) for k, v in d["W"].items()}
+        self.I = I = W["down"].shape[1]
+        sl = slice(0, rows)
+        # down_proj's smoothing factors, from a calibration pass over the sample
+        Vc = oracle.norm_smooth_quant(d["h_calib"][sl], oracle.RMSNORM, self.gamma["mlp"], None, d["eps"],
+                                      quantize=False, want_v=True)["V"]
+        Vc16 = torch.from_numpy(Vc).to(torch.bfloat16).float().numpy()
+        Xc, qc = oracle.quantize_act(Vc16, None, per_token=True)
+        Wc, qwc = oracle.quantize_weight(W["gateup"], True)
+        hmax = oracle.act_quant(self.bf16(oracle.dequant(oracle.gemm_i8(Xc, Wc), qc, qwc)), oracle.SWIGLU,
+                                quantize=False, absmax=np.zeros(I, np.float32))["absmax"]
+        self.s_down = oracle.smooth_scales(hmax, oracle.col_absmax(W["down"]), d["alpha"])
+        # the full weight side once, for the token rows of every sampled step
+        h = {"attn": d["h_attn"][sl], "mlp": d["h_mlp"][sl]}
+        V = {k: oracle.norm_smooth_quant(h[k], oracle.RMSNORM, self.gamma[k], None, d["eps"], quantize=False,
+                                         want_v=True)["V"] for k in h}
+        V16 = {k: torch.from_numpy(V[k]).to(torch.bfloat16) for k in V}
+        self.xmax = {k: oracle.col_absmax(V16[k]) for k in V}
+        self.gp, self.Wq, self.qw, self.s = {}, {}, {}, {}
+        _, self.llm_idx = self.weight_side(1.0, self.gp, self.Wq, self.qw, self.s,
+                                           oracle.llmint8_outliers(V16["attn"], 6.0, 0.0))
 
-    t_rows = 0.0
-    t_w = 0.0
-    t0 = time.perf_counter()
-    V = {k: oracle.norm_smooth_quant(h[k], oracle.RMSNORM, gamma[k], None, d["eps"], quantize=False,
-                                     want_v=True)["V"] for k in h}
-    V16 = {k: torch.from_numpy(V[k]).to(torch.bfloat16) for k in V}
-    xmax = {k: oracle.col_absmax(V16[k]) for k in V}
-    t_rows += time.perf_counter() - t0
-    t0 = time.perf_counter()
-    s, gp = {}, {}
-    for k, w in (("attn", "qkv"), ("mlp", "gateup")):
-        wmax = oracle.col_absmax(W[w])
-        s[k] = oracle.smooth_scales(xmax[k], wmax, d["alpha"])
-        gp[k], _ = oracle.fold_norm(gamma[k], None, s[k])
-    Wq, qw = {}, {}
-    Wq["qkv"], qw["qkv"] = oracle.quantize_weight(oracle.fold_weight(W["qkv"], s["attn"]), True)
-    up_f, _ = oracle.fold_prev_linear(W["gateup"][I:], s_down)
-    gate_q, gate_s = oracle.quantize_weight(oracle.fold_weight(W["gateup"][:I], s["mlp"]), True)
-    up_q, up_s = oracle.quantize_weight(oracle.fold_weight(up_f, s["mlp"]), True)
-    Wq["gateup"], qw["gateup"] = np.concatenate([gate_q, up_q]), np.concatenate([gate_s, up_s])
-    Wq["o"], qw["o"] = oracle.quantize_weight(W["o"], True)
-    Wq["down"], qw["down"] = oracle.quantize_weight(oracle.fold_weight(W["down"], s_down), True)
-    t_w += time.perf_counter() - t0
-    t0 = time.perf_counter()
-    Xq, qx = {}, {}
-    for k in h:
-        r = oracle.norm_smooth_quant(h[k], oracle.RMSNORM, gp[k], None, d["eps"], True)
-        Xq[k], qx[k] = r["Xq"], r["qs"]
-    xo, so = d["o_in"]
-    Y = {}
-    for w, xq, q in (("qkv", Xq["attn"], qx["attn"]), ("o", xo[sl].numpy(), so[sl].numpy()),
-                     ("gateup", Xq["mlp"], qx["mlp"])):
-        Y[w] = bf16(oracle.dequant(oracle.gemm_i8(xq, Wq[w]), q, qw[w]))
-    a = oracle.act_quant(Y["gateup"], oracle.SWIGLU)
-    bf16(oracle.dequant(oracle.gemm_i8(a["Xq"], Wq["down"]), a["qs"], qw["down"]))
-    t_rows += time.perf_counter() - t0
-    # LLM.int8 of the q/k/v projection: outlier set over the sample rows,
-    # row quantisation, weight requantisation, GEMM + outlier term
-    t0 = time.perf_counter()
-    idx = oracle.llmint8_outliers(V16["attn"], 6.0, 0.0)
-    Xq8, qx8 = oracle.llmint8_quant_rows(V16["attn"], idx)
-    t_rows += time.perf_counter() - t0
-    t0 = time.perf_counter()
-    Wq8, qw8 = oracle.llmint8_quant_weight(d["W"]["qkv"], idx)
-    t_w += time.perf_counter() - t0
-    t0 = time.perf_counter()
-    y = oracle.llmint8_combine(oracle.gemm_i8(Xq8, Wq8), qx8, qw8, V16["attn"], d["W"]["qkv"], idx)
-    oracle.round_bf16_bits(y)
-    t_rows += time.perf_counter() - t0
-    return t_w, t_rows
+    def bf16(self, y):
+        torch = self.torch
+        return torch.from_numpy(self.o.round_bf16_bits(y).view(np.int16)).view(torch.bfloat16).float().numpy()
+
+    def weight_side(self, wfrac, gp, Wq, qw, s, idx):
+        """Maxima, smoothing factors, folds and int8 weights on the first
+        wfrac of every weight's output channels; returns (seconds, idx)."""
+        o, W, I, d = self.o, self.W, self.I, self.d
+        part = lambda w: w[: max(1, int(round(w.shape[0] * wfrac)))]  # noqa: E731
+        t0 = time.perf_counter()
+        for k, w in (("attn", "qkv"), ("mlp", "gateup")):
+            wmax = o.col_absmax(part(W[w]))
+            s[k] = o.smooth_scales(self.xmax[k], wmax, d["alpha"])
+            gp[k], _ = o.fold_norm(self.gamma[k], None, s[k])
+        Wq["qkv"], qw["qkv"] = o.quantize_weight(o.fold_weight(part(W["qkv"]), s["attn"]), True)
+        up_f, _ = o.fold_prev_linear(part(W["gateup"][I:]), self.s_down[: part(W["gateup"][I:]).shape[0]])
+        gate_q, gate_s = o.quantize_weight(o.fold_weight(part(W["gateup"][:I]), s["mlp"]), True)
+        up_q, up_s = o.quantize_weight(o.fold_weight(up_f, s["mlp"]), True)
+        Wq["gateup"], qw["gateup"] = np.concatenate([gate_q, up_q]), np.concatenate([gate_s, up_s])
+        Wq["o"], qw["o"] = o.quantize_weight(part(W["o"]), True)
+        Wq["down"], qw["down"] = o.quantize_weight(o.fold_weight(part(W["down"]), self.s_down), True)
+        Wq["llm"], qw["llm"] = o.llmint8_quant_weight(part(W["qkv"]), idx)
+        return time.perf_counter() - t0, idx
+
+    def step(self, rows, wfrac=1.0):
+        """(seconds of weight-side work scaled to all channels, seconds of
+        per-token work for `rows` tokens)."""
+        o, d, torch = self.o, self.d, self.torch
+        sl = slice(0, rows)
+        h = {"attn": d["h_attn"][sl], "mlp": d["h_mlp"][sl]}
+        t0 = time.perf_counter()
+        V = {k: o.norm_smooth_quant(h[k], o.RMSNORM, self.gamma[k], None, d["eps"], quantize=False,
+                                    want_v=True)["V"] for k in h}
+        V16 = {k: torch.from_numpy(V[k]).to(torch.bfloat16) for k in V}
+        for k in V:
+            o.col_absmax(V16[k])
+        t_rows = time.perf_counter() - t0
+        t_w, _ = self.weight_side(wfrac, {}, {}, {}, {}, self.llm_idx)
+        gp, Wq, qw = self.gp, self.Wq, self.qw
+        t0 = time.perf_counter()
+        Xq, qx = {}, {}
+        for k in h:
+            r = o.norm_smooth_quant(h[k], o.RMSNORM, gp[k], None, d["eps"], True)
+            Xq[k], qx[k] = r["Xq"], r["qs"]
+        xo, so = d["o_in"]
+        Y = {}
+        for w, xq, q in (("qkv", Xq["attn"], qx["attn"]), ("o", xo[sl].numpy(), so[sl].numpy()),
+                         ("gateup", Xq["mlp"], qx["mlp"])):
+            Y[w] = self.bf16(o.dequant(o.gemm_i8(xq, Wq[w]), q, qw[w]))
+        a = o.act_quant(Y["gateup"], o.SWIGLU)
+        self.bf16(o.dequant(o.gemm_i8(a["Xq"], Wq["down"]), a["qs"], qw["down"]))
+        # LLM.int8 of the q/k/v projection: outlier set over the sample rows,
+        # row quantisation, GEMM + outlier term (the weight requantisation for
+        # the set is on the weight side)
+        idx = o.llmint8_outliers(V16["attn"], 6.0, 0.0)
+        Xq8, qx8 = o.llmint8_quant_rows(V16["attn"], idx)
+        t_rows += time.perf_counter() - t0
+        if not np.array_equal(idx, self.llm_idx):  # untimed here: the weight side times the requantisation
+            Wq["llm"], qw["llm"] = o.llmint8_quant_weight(self.W["qkv"], idx)
+            self.llm_idx = idx
+        t0 = time.perf_counter()
+        y = o.llmint8_combine(o.gemm_i8(Xq8, Wq["llm"]), qx8, qw["llm"], V16["attn"], d["W"]["qkv"], idx)
+        o.round_bf16_bits(y)
+        t_rows += time.perf_counter() - t0
+        return t_w / wfrac, t_rows
 
 
 def cpu_baseline(rows):
-    t_w, t_rows = cpu_step_sample(rows)
+    t_w, t_rows = CpuStep(rows).step(rows)
     step_s = t_w + t_rows * (M_TOKENS / rows)
     return {"value": M_TOKENS / step_s, "unit": "tokens/s", "cores": 1, "kind": "oracle",
             "sample": f"{rows} of {M_TOKENS} tokens through every step (weights in full: {t_w:.2f} s; "
@@ -551,25 +579,45 @@ def cpu_baseline(rows):
             "step_s": step_s}
 
 
+REF_BUDGET_S = 150.0  # wall time of the reference arm's timed steps, whatever --steps asks for
+
+
+def ref_sample(t_w_full, t_row, per_step):
+    """Token rows (1..64) and weight fraction (1, 1/2, ..., 1/64) of one
+    reference step that fit `per_step` seconds, given the full weight side's
+    time and one token row's time: the largest sample that fits, weights in
+    full and 64 rows when there is room."""
+    rows, wfrac = 64, 1.0
+    if t_w_full + 64 * t_row <= per_step:
+        return rows, wfrac
+    while wfrac > 1 / 64 and t_w_full * wfrac > per_step / 2:
+        wfrac /= 2
+    rows = int(max(1, min(64, (per_step - t_w_full * wfrac) // max(t_row, 1e-9))))
+    return rows, wfrac
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return
-    rows = 64
+    ctx = CpuStep()
+    t_w_full, t16 = ctx.step(16)  # the first warm-up step also sizes the sample
+    rows, wfrac = ref_sample(t_w_full, t16 / 16, REF_BUDGET_S / max(args.steps, 1))
+    for _ in range(min(max(args.warmup, 1), 3) - 1):
+        ctx.step(rows, wfrac)
     times = []
-    for _ in range(max(args.warmup, 0) and 1):
-        cpu_step_sample(16)
     for _ in range(args.steps):
-        t_w, t_rows = cpu_step_sample(rows)
+        t_w, t_rows = ctx.step(rows, wfrac)
         times.append(t_w + t_rows * (M_TOKENS / rows))
     step_s = sum(times) / len(times)
     v = M_TOKENS / step_s
+    wpart = "weights in full" if wfrac == 1 else f"1/{round(1 / wfrac)} of every weight's output channels"
     line = {
         "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "i8", "data": "synthetic",
         "config": {"workload": WORKLOAD, "tokens": M_TOKENS, "hidden": HIDDEN},
         "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                         "sample": f"each step: {rows} of {M_TOKENS} tokens, weights in full, extrapolated"},
+                         "sample": f"each step: {rows} of {M_TOKENS} tokens and {wpart}, extrapolated linearly"},
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)

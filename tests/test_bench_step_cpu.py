@@ -64,3 +64,18 @@ def test_launch_claim_matches_the_step():
                 "sq_norm_smooth_quant", "sq_gemm_w8a8", "sq_llmint8_matmul", "sq_act_quant",
                 "sq_quantize_weight_fold_prev"):
         assert row in calls, row
+
+
+def test_reference_sample_fits_the_budget():
+    """The reference arm's per-step sample fits its share of the wall-time
+    budget for any --steps, and is the full 64-row, full-weight sample when
+    there is room."""
+    t_w, t_row = 0.25, 0.0066  # seconds: full weight side, one token row (oracle on one core)
+    assert bench.ref_sample(t_w, t_row, bench.REF_BUDGET_S / 20) == (64, 1.0)
+    for steps in (200, 500, 2000, 10000):
+        per_step = bench.REF_BUDGET_S / steps
+        rows, wfrac = bench.ref_sample(t_w, t_row, per_step)
+        assert 1 <= rows <= 64 and 1 / 64 <= wfrac <= 1
+        assert wfrac == 1 or t_w * wfrac <= per_step / 2 or wfrac == 1 / 64
+        if steps <= 2000:
+            assert t_w * wfrac + rows * t_row <= per_step
