@@ -236,6 +236,58 @@ def test_round_half_even_and_clip(orc):
     assert qs[0] == 1.0 and Xq.tolist() == [[127, 64, 0]]
 
 
+def _check_symmetric_int8(v, q, qs, keep=None):
+    """Invariants of absmax int8 with scale qs = 127 / max|v| per row ("8位量化"
+    §2.1): codes in [-127, 127]; the row's largest |v| maps to +-127; every
+    code is the nearest integer to v*qs (within 0.5 plus the fp32 rounding of
+    the product); codes keep the sign of v. Columns outside `keep` are 0."""
+    v = v.astype(np.float64)
+    qs = np.asarray(qs, np.float64).reshape(-1, 1)
+    q = q.astype(np.int64)
+    if keep is not None:
+        out = np.setdiff1d(np.arange(v.shape[1]), keep)
+        assert np.all(q[:, out] == 0)
+        v, q = v[:, keep], q[:, keep]
+    assert np.all(np.abs(q) <= 127)
+    am = np.argmax(np.abs(v), axis=1)
+    rows = np.arange(v.shape[0])
+    nz = np.abs(v[rows, am]) > 0
+    assert np.all(np.abs(q[rows, am])[nz] == 127)
+    assert np.max(np.abs(v * qs - q)) <= 0.5 + 127 * 2.0 ** -23
+    assert np.all((q == 0) | (np.sign(q) == np.sign(v)))
+
+
+def test_int8_quantisers_invariants(orc):
+    """Every absmax int8 quantiser of the oracle on random data with outlier
+    channels: activations per token, weights per output channel, the LLM.int8
+    rows and weight columns outside O, the fused norm output and the SwiGLU
+    output. A truncating or half-away rounding, an inverted scale or a clip at
+    128 fails here."""
+    rng = np.random.default_rng(60)
+    M, K, N = 37, 200, 29
+    X = rng.normal(size=(M, K)).astype(np.float32)
+    X[:, [3, 77]] *= 40
+    Xq, qx = orc.quantize_act(X, None, per_token=True)
+    _check_symmetric_int8(X, Xq, qx)
+    W = rng.normal(scale=0.02, size=(N, K)).astype(np.float32)
+    Wq, qw = orc.quantize_weight(W, per_channel=True)
+    _check_symmetric_int8(W, Wq, qw)
+    idx = orc.llmint8_outliers(X, 6.0, 0.0)
+    assert set(idx.tolist()) >= {3, 77}
+    keep = np.setdiff1d(np.arange(K), idx)
+    Xq8, qx8 = orc.llmint8_quant_rows(X, idx)
+    _check_symmetric_int8(X, Xq8, qx8, keep)
+    Wq8, qw8 = orc.llmint8_quant_weight(W, idx)
+    _check_symmetric_int8(W, Wq8, qw8, keep)
+    gamma = (1 + 0.1 * rng.normal(size=K)).astype(np.float32)
+    for norm in (orc.LAYERNORM, orc.RMSNORM):
+        r = orc.norm_smooth_quant(X, norm, gamma, None, 1e-5, True, want_v=True)
+        _check_symmetric_int8(r["V"], r["Xq"], r["qs"])
+    A = (rng.normal(size=(M, 2 * K)) * 3).astype(np.float32)
+    r = orc.act_quant(A, orc.SWIGLU, want_h=True)
+    _check_symmetric_int8(r["H"], r["Xq"], r["qs"])
+
+
 def test_zero_row_scale_floor(orc):
     """An all-zero row takes the 1e-8 floor of quantize_vectorwise and gives 0."""
     Xq, qs = orc.quantize_act(np.zeros((2, 16), np.float32), None, per_token=True)
