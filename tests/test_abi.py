@@ -199,3 +199,40 @@ def test_missing_library_raises(monkeypatch):
     monkeypatch.setattr(sq, "_lib", None)
     with pytest.raises(RuntimeError, match="not built"):
         sq.sq_version()
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include <string.h>
+#include "sq_api.h"
+
+int main(void) {
+    /* host-only calls: sizes, version, argument checks (nothing reaches a GPU) */
+    if (sq_version() < 100) return 1;
+    if (sq_workspace_size(SQ_OP_GEMM, 2048, 16384, 4096) != 256) return 2;
+    sq_status_t st = sq_gemm_w8a8(NULL, NULL, 16, 16, 16, NULL, 0, NULL, 0, NULL, SQ_BF16, NULL, 16, NULL, 0,
+                                  (sq_stream_t)0);
+    if (st != SQ_ERR_INVALID_ARG || strstr(sq_last_error_string(), "null") == NULL) return 3;
+    sq_llmint8_weight_t w;
+    memset(&w, 0, sizeof w);
+    printf("ok %zu\n", sizeof w);
+    return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_links(L):
+    """include/sq_api.h compiles as C99 with warnings as errors, and a C
+    program links libsq_b200.so and calls its host-side entry points."""
+    out = os.path.join(ROOT, "_build", "c_client")
+    os.makedirs(out, exist_ok=True)
+    src = os.path.join(out, "client.c")
+    with open(src, "w") as f:
+        f.write(C_CLIENT)
+    exe = os.path.join(out, "client")
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-o", str(exe), "-L", PKG, "-lsq_b200", "-Wl,-rpath," + PKG],
+                   check=True, capture_output=True, text=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
+    assert r.stdout.startswith("ok ")
