@@ -6,6 +6,7 @@ import glob
 import os
 import re
 import subprocess
+import sys
 
 import pytest
 
@@ -235,4 +236,56 @@ def test_header_is_plain_c_and_links(L):
                    check=True, capture_output=True, text=True)
     r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
     assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
+    assert r.stdout.startswith("ok ")
+
+
+FUZZ = r"""
+import ctypes, os, random, sys
+# fake pointers that pass validation must never reach a device: no GPU is visible here
+assert os.environ.get("CUDA_VISIBLE_DEVICES") == ""
+sys.path.insert(0, sys.argv[1])
+from w8a8_post_quantization_sq_b200 import _lib
+L = _lib.lib()
+rng = random.Random(int(sys.argv[2]))
+ptrs = [None, ctypes.c_void_p(4096), ctypes.c_void_p(4098)]
+def P(): return rng.choice(ptrs)
+def S(): return rng.choice([0, 1, 7, 8, 15, 16, 24, 100, 128, 1000, 1024, 4096, -1, -16, 1 << 20, 1 << 40])
+def D(): return rng.choice([0, 1, 2, 3, 4, 7, -1])
+calls = {
+    "sq_calib_absmax": lambda: (P(), D(), S(), S(), S(), P(), None),
+    "sq_weight_absmax": lambda: (P(), D(), S(), S(), S(), P(), None),
+    "sq_smooth_scales": lambda: (P(), P(), S(), rng.choice([-1.0, 0.0, 0.5, 1.0, 2.0]), P(), None),
+    "sq_quantize_act": lambda: (P(), D(), S(), S(), S(), P(), rng.randint(0, 1), P(), P(), P(), P(),
+                                rng.choice([0, 16, 256]), None),
+    "sq_quantize_weight": lambda: (P(), D(), S(), S(), P(), rng.randint(0, 1), P(), P(), P(),
+                                   rng.choice([0, 16, 256]), None),
+    "sq_norm_smooth_quant": lambda: (P(), D(), S(), S(), S(), rng.choice([0, 1, 5]), P(), P(), 1e-6,
+                                     rng.randint(0, 1), P(), P(), P(), P(), P(), None),
+    "sq_act_quant": lambda: (P(), D(), S(), S(), S(), rng.choice([0, 1, 5]), rng.randint(0, 1), P(), P(), P(),
+                             P(), P(), None),
+    "sq_gemm_w8a8": lambda: (P(), P(), S(), S(), S(), P(), rng.randint(0, 1), P(), rng.randint(0, 1), P(), D(),
+                             P(), S(), P(), rng.choice([0, 16, 256, 1 << 20]), None),
+    "sq_llmint8_detect": lambda: (P(), D(), S(), S(), S(), 6.0, 0.0, P(), P(), P(),
+                                  rng.choice([0, 16, 256, 1 << 20]), None),
+}
+seen = set()
+for i in range(3000):
+    name = rng.choice(sorted(calls))
+    st = getattr(L, name)(*calls[name]())
+    assert st in (0, 1, 2, 3, 4), (name, st)
+    seen.add((name, st))
+print("ok", len(seen), sorted({st for _, st in seen}))
+"""
+
+
+@pytest.mark.parametrize("seed", [1, 2])
+def test_random_arguments_never_crash(L, seed):
+    """3000 calls with random sizes, dtypes and null, aligned or misaligned
+    fake pointers: every call returns a status (no host crash). On a host
+    without a GPU, arguments that pass validation end in SQ_ERR_CUDA or, for
+    empty sizes, SQ_OK with nothing launched; fake pointers are never read on
+    the host."""
+    r = subprocess.run([sys.executable, "-c", FUZZ, ROOT, str(seed)], capture_output=True, text=True,
+                       timeout=300, env={**os.environ, "CUDA_VISIBLE_DEVICES": ""})
+    assert r.returncode == 0, (r.returncode, r.stdout[-2000:], r.stderr[-2000:])
     assert r.stdout.startswith("ok ")
