@@ -143,6 +143,10 @@ def test_argument_validation_without_gpu(L):
     _expect(L, L.sq_quantize_act(p, 2, 4, 16, 16, None, 0, None, p, p, None, 0, None), 1, "workspace")
     # llmint8: workspace too small
     _expect(L, L.sq_llmint8_detect(p, 1, 256, 64, 64, 6.0, 0.0, p, p, p, 16, None), 1, "workspace")
+    # an empty call still has its dtype checked
+    _expect(L, L.sq_quantize_weight(None, 7, 0, 16, None, 1, None, None, None, 0, None), 1, "dtype")
+    _expect(L, L.sq_quantize_act(None, -1, 0, 16, 16, None, 1, None, None, None, None, 0, None), 1, "dtype")
+    _expect(L, L.sq_fold_weight(p, 3, 0, 16, p, p, None), 1, "dtype")
     # M == 0 is a valid empty call (nothing launched)
     assert L.sq_gemm_w8a8(p, p, 0, 16, 16, p, 1, p, 1, None, 2, p, 16, p, 256, None) == 0
     assert L.sq_calib_absmax(p, 2, 0, 16, 16, p, None) == 0

@@ -384,6 +384,8 @@ sq_status_t sq_quantize_weight(const void* W, sq_dtype_t dt, int64_t N, int64_t 
                "%s: W, Wq and s must be 16-byte aligned", name);
     SQ_REQUIRE(per_channel || (workspace && ws_bytes >= sq::kStatusBytes), SQ_ERR_INVALID_ARG,
                "%s: per-tensor quantisation needs a workspace of %zu bytes", name, sq::kStatusBytes);
+    SQ_REQUIRE(dt == SQ_F16 || dt == SQ_BF16 || dt == SQ_F32, SQ_ERR_INVALID_ARG, "%s: dtype must be F16, BF16 or F32",
+               name);
     if (N == 0) return SQ_OK;
     cudaStream_t st = sq::as_cuda(stream);
     if (s)
@@ -399,6 +401,8 @@ sq_status_t sq_quantize_weight_fold_prev(const void* W, sq_dtype_t dt, int64_t N
     SQ_REQUIRE(N >= 0 && K > 0 && K % 16 == 0, SQ_ERR_UNSUPPORTED_SHAPE, "%s: need K > 0 and K %% 16 == 0", name);
     SQ_REQUIRE(sq::aligned16(W) && sq::aligned16(Wq) && sq::aligned16(s), SQ_ERR_ALIGNMENT,
                "%s: W, Wq and s must be 16-byte aligned", name);
+    SQ_REQUIRE(dt == SQ_F16 || dt == SQ_BF16 || dt == SQ_F32, SQ_ERR_INVALID_ARG, "%s: dtype must be F16, BF16 or F32",
+               name);
     if (N == 0) return SQ_OK;
     cudaStream_t st = sq::as_cuda(stream);
     switch (dt) {
@@ -426,6 +430,8 @@ sq_status_t sq_quantize_act(const void* X, sq_dtype_t dt, int64_t M, int64_t K, 
                "%s: X, Xq and s must be 16-byte aligned", name);
     SQ_REQUIRE(per_token || static_qs || (workspace && ws_bytes >= sq::kStatusBytes), SQ_ERR_INVALID_ARG,
                "%s: dynamic per-tensor quantisation needs a workspace of %zu bytes", name, sq::kStatusBytes);
+    SQ_REQUIRE(dt == SQ_F16 || dt == SQ_BF16 || dt == SQ_F32, SQ_ERR_INVALID_ARG, "%s: dtype must be F16, BF16 or F32",
+               name);
     if (M == 0) return SQ_OK;
     cudaStream_t st = sq::as_cuda(stream);
     if (s)
@@ -444,6 +450,8 @@ sq_status_t sq_quantize_weight_fp8(const void* W, sq_dtype_t dt, int64_t N, int6
                "%s: W, Wq and s must be 16-byte aligned", name);
     SQ_REQUIRE(per_channel || (workspace && ws_bytes >= sq::kStatusBytes), SQ_ERR_INVALID_ARG,
                "%s: per-tensor quantisation needs a workspace of %zu bytes", name, sq::kStatusBytes);
+    SQ_REQUIRE(dt == SQ_F16 || dt == SQ_BF16 || dt == SQ_F32, SQ_ERR_INVALID_ARG, "%s: dtype must be F16, BF16 or F32",
+               name);
     if (N == 0) return SQ_OK;
     cudaStream_t st = sq::as_cuda(stream);
     int8_t* Q = reinterpret_cast<int8_t*>(Wq);
@@ -465,6 +473,8 @@ sq_status_t sq_quantize_act_fp8(const void* X, sq_dtype_t dt, int64_t M, int64_t
                "%s: X, Xq and s must be 16-byte aligned", name);
     SQ_REQUIRE(per_token || static_qs || (workspace && ws_bytes >= sq::kStatusBytes), SQ_ERR_INVALID_ARG,
                "%s: dynamic per-tensor quantisation needs a workspace of %zu bytes", name, sq::kStatusBytes);
+    SQ_REQUIRE(dt == SQ_F16 || dt == SQ_BF16 || dt == SQ_F32, SQ_ERR_INVALID_ARG, "%s: dtype must be F16, BF16 or F32",
+               name);
     if (M == 0) return SQ_OK;
     cudaStream_t st = sq::as_cuda(stream);
     int8_t* Q = reinterpret_cast<int8_t*>(Xq);

@@ -145,6 +145,8 @@ sq_status_t sq_fold_weight(const void* W, sq_dtype_t dt, int64_t N, int64_t K, c
     SQ_REQUIRE(W && s && Wp_out, SQ_ERR_INVALID_ARG, "sq_fold_weight: null pointer");
     SQ_REQUIRE(N >= 0 && K > 0 && K % 8 == 0, SQ_ERR_UNSUPPORTED_SHAPE, "sq_fold_weight: need K > 0, K %% 8 == 0");
     SQ_REQUIRE(sq::aligned16(W) && sq::aligned16(Wp_out), SQ_ERR_ALIGNMENT, "sq_fold_weight: unaligned pointer");
+    SQ_REQUIRE(dt == SQ_F16 || dt == SQ_BF16 || dt == SQ_F32, SQ_ERR_INVALID_ARG,
+               "sq_fold_weight: dtype must be F16, BF16 or F32");
     if (N == 0) return SQ_OK;
     cudaStream_t st = sq::as_cuda(stream);
     const int64_t n = N * K;
