@@ -787,6 +787,36 @@ def run_kernel(args):
     print(json.dumps(out), flush=True)
 
 
+def json_line(args, world, r):
+    """The benchmark's JSON line (without the CPU baseline) from the measured
+    step: r holds the step time, the e2e time, the GEMM intervals and peaks,
+    the copy sizes and the clock record of run_ours."""
+    value = M_TOKENS * world / (r["ms_per_step"] * 1e-3)
+    e2e = M_TOKENS * world / (r["e2e_ms"] * 1e-3)
+    gemm_avg_s = sum(r["gemm_avg_ms"]) * 1e-3
+    gemm_ops = sum(2.0 * m * n * k for (m, n, k) in GEMMS[:4])
+    achieved = gemm_ops / gemm_avg_s / 1e12
+    traffic = gemm_traffic()
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": r["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "i8", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "tokens": M_TOKENS, "hidden": HIDDEN, "parallelism": f"replicas x{world}",
+                   "l2": "flushed before every timed step (256 MB write + 256 MB read, outside the timed interval)",
+                   "graph": "one CUDA graph per step"},
+        "gemm_tops": r["gemm_tops"], "gemm_avg_us": [x * 1e3 for x in r["gemm_avg_ms"]],
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": r["i8_peak"], "unit": "TOPS",
+                     "frac": achieved / r["i8_peak"], "traffic": traffic,
+                     "kernel": "gemm_w8a8_kernel", "peak_source": f"{r['peak_src']} bf16 burst x 2 (int8 nominal ratio)",
+                     "timing": f"CUDA events around each GEMM of an instrumented copy of the step's graph, "
+                               f"{r['gemm_timed_steps']} replays after the timed region, L2 flushed before each"},
+        "e2e": {"value": e2e, "unit": "tokens/s", "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
+        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "clocks": r["clocks"],
+    }
+    return line
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--kernel", default=None, help="time one entry point alone: gemm|norm|absmax|quant_weight|llmint8")
@@ -834,29 +864,7 @@ def main():
         dist.destroy_process_group()
     if rank != 0:
         return
-    value = M_TOKENS * world / (r["ms_per_step"] * 1e-3)
-    e2e = M_TOKENS * world / (r["e2e_ms"] * 1e-3)
-    gemm_avg_s = sum(r["gemm_avg_ms"]) * 1e-3
-    gemm_ops = sum(2.0 * m * n * k for (m, n, k) in GEMMS[:4])
-    achieved = gemm_ops / gemm_avg_s / 1e12
-    traffic = gemm_traffic()
-    line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": r["ms_per_step"], "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "i8", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "tokens": M_TOKENS, "hidden": HIDDEN, "parallelism": f"replicas x{world}",
-                   "l2": "flushed before every timed step (256 MB write + 256 MB read, outside the timed interval)",
-                   "graph": "one CUDA graph per step"},
-        "gemm_tops": r["gemm_tops"], "gemm_avg_us": [x * 1e3 for x in r["gemm_avg_ms"]],
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": r["i8_peak"], "unit": "TOPS",
-                     "frac": achieved / r["i8_peak"], "traffic": traffic,
-                     "kernel": "gemm_w8a8_kernel", "peak_source": f"{r['peak_src']} bf16 burst x 2 (int8 nominal ratio)",
-                     "timing": f"CUDA events around each GEMM of an instrumented copy of the step's graph, "
-                               f"{r['gemm_timed_steps']} replays after the timed region, L2 flushed before each"},
-        "e2e": {"value": e2e, "unit": "tokens/s", "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
-        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
-        "clocks": r["clocks"],
-    }
+    line = json_line(args, world, r)
     if not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = {k: v for k, v in cpu_baseline(args.cpu_rows).items() if k != "step_s"}
     print(json.dumps(line), flush=True)

@@ -79,3 +79,30 @@ def test_reference_sample_fits_the_budget():
         assert wfrac == 1 or t_w * wfrac <= per_step / 2 or wfrac == 1 / 64
         if steps <= 2000:
             assert t_w * wfrac + rows * t_row <= per_step
+
+
+def test_json_line_contract():
+    """The benchmark's JSON line from a synthetic measurement: every key the
+    line must carry, whole-job tokens/s over the ranks, the roofline fraction
+    as achieved / peak, and the launch claim as kernels per step x steps."""
+    import json
+    import types
+
+    args = types.SimpleNamespace(steps=100, warmup=5)
+    r = {"ms_per_step": 0.125, "e2e_ms": 1.25, "gemm_avg_ms": [0.03, 0.02, 0.05, 0.02], "gemm_tops": 500.0,
+         "i8_peak": 3300.0, "peak_src": "measured", "gemm_timed_steps": 200, "h2d": 8 << 20, "d2h": 64 << 20,
+         "clocks": {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}}
+    line = json.loads(json.dumps(bench.json_line(args, 2, r)))
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+              "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks"):
+        assert k in line, k
+    assert line["value"] == bench.M_TOKENS * 2 / 0.125e-3
+    assert line["e2e"]["value"] == bench.M_TOKENS * 2 / 1.25e-3
+    assert line["e2e"]["h2d_bytes_per_step"] == 8 << 20 and line["e2e"]["d2h_bytes_per_step"] == 64 << 20
+    ops = sum(2.0 * m * n * k for (m, n, k) in bench.GEMMS[:4])
+    assert abs(line["roofline"]["achieved"] - ops / 0.12e-3 / 1e12) < 1e-9 * line["roofline"]["achieved"]
+    assert line["roofline"]["frac"] == line["roofline"]["achieved"] / 3300.0
+    assert line["roofline"]["bound"] == "tensor" and line["roofline"]["unit"] == "TOPS"
+    assert line["gpu_launches"] == bench.LAUNCHES_PER_STEP * 100
+    assert line["n_gpus"] == 2 and line["scaling"] == "weak" and line["higher_is_better"] is True
+    assert "workload" in line["config"] and "l2" in line["config"]
