@@ -1,40 +1,40 @@
 """Benchmark of the SmoothQuant W8A8 linear-layer path on B200.
 
-One step = one pass of every hot-path row over one batch of synthetic input
-shaped like a Qwen3-0.6B decoder layer at 2048 tokens (hidden 1024; q/k/v
-fused 1024->4096, o 2048->1024, gate/up fused 1024->6144, down 3072->1024;
-6 activation channels x20..x100):
-  norm pass producing the linear input (RMSNorm, original gamma)        x2
-  calibration absmax of that input                                      x2
-  weight absmax over the fused consumers                                x2
-  smoothing factors and gamma' = gamma / s (one launch)                 x2
-  weight fold + int8 quantisation (per output channel)                  x5
-    (up_proj's also takes 1/s of down_proj's input on its output channels)
-  fused RMSNorm + smoothing + per-token int8                            x2
-  int8 GEMM + dequant epilogue to bf16                                  x4
-  SwiGLU of the gate/up output + per-token int8 (down_proj's input)     x1
-  LLM.int8 decomposition of the q/k/v projection (bf16)                 x1
-The independent chains of the step (the attention-side and MLP-side
-calibration/quantisation chains, the weight-side work, the o/down GEMMs and the
-LLM.int8 call) run on their own streams inside the step, joined at its end.
-The step is captured once in a CUDA graph and replayed. L2 is flushed (a
-256 MB write, then a 256 MB read of another buffer so that no dirty line of the
-flush is left to be written back) before every timed step, outside the timed
-interval; each step is bracketed by CUDA events on the stream it runs on. The
-GEMMs' launch durations come from a second capture of the step with events
-around each GEMM, replayed after the timed region (event nodes inside the
-graph cut the programmatic chaining of a GEMM to its producer, which costs the
-step 10-25 us, so they stay out of the timed graph).
+The headline workload is the 175B-shaped block (hidden 12288, 4096 tokens) in
+deploy mode: the weights are smoothed and quantised once, offline, and one
+step is the block's online linear stack
+
+  LayerNorm (gamma', beta' folded) + per-token int8 of the attention side
+  QKV GEMM 12288 -> 36864, int8 x int8 -> int32, dequantised to bf16
+  out GEMM 12288 -> 12288 on a per-token int8 input (attention is not on the path)
+  LayerNorm + per-token int8 of the MLP side
+  FC1 GEMM 12288 -> 49152
+  FC2 GEMM 49152 -> 12288 on a per-token int8 input (the activation is not on the path)
+
+tokens/s = tokens / step time. The offline work is timed on its own and
+reported beside the step, not inside it: the calibration pass (running
+per-channel absmax over 16 calibration batches of [4096, 12288] bf16), the
+weight maxima, the smoothing factors for alpha in {0.4, 0.5, 0.6} (gamma and
+beta folded for alpha = 0.5) and the per-channel int8 weights.
+
+Every timed step is one CUDA graph replay after an L2 flush (a 256 MB write,
+then a 256 MB read of another buffer, outside the timed interval), bracketed
+by CUDA events on the stream it runs on. Per-kernel durations come from a
+second capture of the same step with events around every launch, replayed
+after the timed region. The Qwen3-0.6B-, OPT-30B- and LLM.int8-shaped
+configurations are timed the same way and reported under "configs".
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py --kernel gemm --shape M,N,K     (one entry point alone)
 
-Prints one JSON line (rank 0). With torchrun (N > 1) every rank runs its own
+Prints one JSON line (rank 0). Under torchrun (N > 1) every rank runs its own
 replica of the step on its own GPU (no data-path collective; weak scaling).
 """
 from __future__ import annotations
 
 import argparse
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -46,19 +46,43 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-M_TOKENS, HIDDEN = 2048, 1024
-WORKLOAD = ("qwen3-0.6b-shaped decoder layer linear stack, 2048 tokens, hidden 1024, bf16 in/out, int8 GEMMs; "
-            "down_proj input from the SwiGLU of the gate/up output")
 METRIC = "W8A8 GEMM TOPS & tokens/s at 1 B200; % of INT8 TC peak / HBM GB/s"
-# GEMM (M, N, K) of one step: qkv, o, gate/up, down, LLM.int8 q/k/v
-GEMMS = [(2048, 4096, 1024), (2048, 1024, 2048), (2048, 6144, 1024), (2048, 1024, 3072), (2048, 4096, 1024)]
-# our kernels in one step: weight absmax 2, calibration absmax 2, smoothing +
-# gamma fold 2, norm passes 4, weight quantisation 5 (up_proj's with the fold
-# of down_proj's s), GEMMs 4, SwiGLU + int8 1, LLM.int8 5 (counts, compaction,
-# weight-side pass, row quantisation, GEMM)
-# steps of the instrumented copy of the step that time the GEMM launches
-GEMM_TIMED_STEPS = 200
-LAUNCHES_PER_STEP = (2 * 1 + 2 * 1 + 2 * 1 + 2 * 2 + 5 * 1 + 4 * 1 + 1 + 5)
+NOMINAL_INT8_TOPS = 4500.0  # B200 dense int8 (spec sheet), for context beside the measured-derived peak
+
+# Deploy-mode linear stacks. gemms: (weight, source) in launch order; source is
+# the norm side whose int8 output the GEMM reads, or "syn" for a synthetic
+# int8 input whose producer (attention, the MLP activation) is off the path.
+CONFIGS = {
+    "c5": {
+        "workload": "175B-shaped W8A8 block, hidden 12288, 4096 tokens, deploy mode: LayerNorm + smoothing + "
+                    "per-token int8 of the attention and MLP inputs, QKV/out/FC1/FC2 int8 GEMMs to bf16 "
+                    "(weights smoothed and quantised offline)",
+        "gen": "c5_175b", "tokens": 4096, "hidden": 12288, "norm": "layer", "per_token": True,
+        "calib": "absmax", "alphas": (0.4, 0.5, 0.6), "alpha": 0.5, "out": "bf16",
+        "gemms": (("qkv", "attn"), ("out", "syn"), ("fc1", "mlp"), ("fc2", "syn")),
+    },
+    "c3": {
+        "workload": "OPT-30B-shaped decoder linear stack, 4 x 256 tokens, hidden 7168, deploy mode: LayerNorm + "
+                    "smoothing + static per-tensor int8 (scales from 8 calibration batches), QKV/out/FC1/FC2 int8 "
+                    "GEMMs to fp16",
+        "gen": "c3_opt30b", "tokens": 1024, "hidden": 7168, "norm": "layer", "per_token": False,
+        "calib": "norm", "alphas": (0.5,), "alpha": 0.5, "out": "fp16",
+        "gemms": (("qkv", "attn"), ("out", "syn"), ("fc1", "mlp"), ("fc2", "syn")),
+    },
+    "c2": {
+        "workload": "Qwen3-0.6B-shaped decoder layer linear stack, 2048 tokens, hidden 1024, deploy mode: RMSNorm + "
+                    "smoothing + per-token int8, q/k/v, o, gate/up, down int8 GEMMs to bf16",
+        "gen": "c2_block", "tokens": 2048, "hidden": 1024, "norm": "rms", "per_token": True,
+        "calib": "norm", "alphas": (0.5,), "alpha": 0.5, "out": "bf16",
+        "gemms": (("qkv", "attn"), ("o", "syn"), ("gateup", "mlp"), ("down", "syn")),
+    },
+}
+C4 = {"workload": "LLM.int8() decomposition at 6.7B shapes: X fp16 [2048, 4096] with 6 outlier dims, W fp16 "
+                  "[16384, 4096], threshold 6.0, fp16 out (weight cache warm: the outlier set is unchanged)",
+      "tokens": 2048, "M": 2048, "K": 4096, "N": 16384}
+HEADLINE = "c5"
+L2_NOTE = ("L2 flushed before every timed step (256 MB write + 256 MB read, outside the timed interval); "
+           "the step's operands (1.8 GB of int8 weights) are far larger than L2 as well")
 
 
 def peaks():
@@ -68,6 +92,15 @@ def peaks():
             d = json.load(f)
         return d, "measured"
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def int8_peaks():
+    """Dense int8 peaks in TOPS: the measured bf16 GEMM (burst, sustained) x 2,
+    the nominal int8:bf16 ratio (4.5 vs 2.25 PFLOP/s), and the spec-sheet
+    nominal 4.5 POPS."""
+    pk, src = peaks()
+    return {"burst": 2.0 * pk["bf16_tflops"], "sustained": 2.0 * pk.get("bf16_tflops_sustained", pk["bf16_tflops"]),
+            "nominal": NOMINAL_INT8_TOPS, "source": src}
 
 
 # ------------------------------------------------------------------ ranks
@@ -99,16 +132,25 @@ def gemm_sources_digest():
     return h.hexdigest()
 
 
-def gemm_traffic():
-    """DRAM bytes per launch of the step's four GEMMs, from the ncu counters
-    recorded in profiles/gemm_traffic.json, or None once the kernel's sources
-    differ from those the counters were taken on."""
+def gemm_traffic(shapes):
+    """DRAM bytes (read + write) of one launch of each GEMM shape (M, N, K),
+    from the ncu counters recorded in profiles/gemm_traffic.json; None when a
+    shape is missing or the kernel's sources differ from those the counters
+    were taken on."""
     p = os.path.join(ROOT, "profiles", "gemm_traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
-    return d.get("bytes_per_launch") if d.get("sources_sha256") == gemm_sources_digest() else None
+    if d.get("sources_sha256") != gemm_sources_digest():
+        return None
+    per = d.get("bytes_per_launch")
+    if not isinstance(per, dict):
+        return None
+    keys = ["x".join(str(v) for v in s) for s in shapes]
+    if not all(k in per for k in keys):
+        return None
+    return [float(per[k]) for k in keys]
 
 
 # ------------------------------------------------------------------ clocks
@@ -136,18 +178,25 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
             out, _ = self.proc.communicate()
-        rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 8]
-        if not rows:
-            return None
-        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if "Active" in r[5 + i] and "Not" not in r[5 + i]})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+        return parse_clocks(out)
 
 
-# ------------------------------------------------------------------ GPU arm
+def parse_clocks(out):
+    rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 8]
+    if not rows:
+        return None
+    num = lambda x: x.strip().replace(".", "", 1).isdigit()  # noqa: E731
+    sm = [float(r[1]) for r in rows if num(r[1])]
+    mx = [float(r[2]) for r in rows if num(r[2])]
+    pw = [float(r[3]) for r in rows if num(r[3])]
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    reasons = sorted({names[i] for r in rows for i in range(4) if "Active" in r[5 + i] and "Not" not in r[5 + i]})
+    return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+            "sm_mhz_min": min(sm) if sm else None, "power_w_max": max(pw) if pw else None,
+            "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ GPU helpers
 class L2Flush:
     """Evicts L2 before a timed interval: a 256 MB write, then a 256 MB read of
     another buffer, so the dirty lines of the write are written back before the
@@ -167,8 +216,181 @@ class L2Flush:
         torch.sum(self.r, dim=0, out=self.out)
 
 
-class Layer:
-    """Device buffers and the step for the Qwen3-0.6B-shaped layer."""
+class EventBank:
+    """CUDA event pairs around launches captured in a graph (external events,
+    so every replay records them), each tagged with its kernel and its
+    algorithmic work."""
+
+    def __init__(self):
+        self.pairs = []
+
+    def pair(self, tag, work):
+        import torch
+
+        e = (torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
+        self.pairs.append((tag, work, e))
+        return e
+
+    def read(self):
+        return [a.elapsed_time(b) for _, _, (a, b) in self.pairs]
+
+
+def esize(t):
+    return t.element_size()
+
+
+# ------------------------------------------------------------------ the deploy-mode stacks
+class Stack:
+    """Device buffers, offline pass and online step of one deploy-mode linear
+    stack (CONFIGS). `offline()` calibrates, smooths and quantises the weights;
+    `step()` is the online linear stack. Every launch goes through `launch`,
+    which brackets it with events when an EventBank is attached."""
+
+    def __init__(self, name, dev, M=None, n_calib=None):
+        import torch
+
+        import w8a8_post_quantization_sq_b200 as sq
+        from w8a8_post_quantization_sq_b200 import inputs
+
+        cfg = CONFIGS[name]
+        self.name, self.cfg, self.sq, self.torch, self.dev = name, cfg, sq, torch, dev
+        self.M = M = M or cfg["tokens"]
+        kw = {} if n_calib is None else {"n_calib": n_calib}
+        d = getattr(inputs, cfg["gen"])(device=dev, M=M, **kw)
+        self.d = d
+        K = cfg["hidden"]
+        self.K = K
+        self.norm = sq.SQ_LAYERNORM if cfg["norm"] == "layer" else sq.SQ_RMSNORM
+        self.per_token = cfg["per_token"]
+        self.alpha, self.alphas = cfg["alpha"], cfg["alphas"]
+        self.out_dtype = torch.bfloat16 if cfg["out"] == "bf16" else torch.float16
+        f32 = lambda *s: torch.empty(s, dtype=torch.float32, device=dev)  # noqa: E731
+        self.sides = ("attn", "mlp")
+        self.consumer = {src: w for w, src in cfg["gemms"] if src != "syn"}
+        self.gamma = {k: d["gamma"][k].float().contiguous() for k in self.sides}
+        self.beta = {k: None if d["beta"][k] is None else d["beta"][k].float().contiguous() for k in self.sides}
+        self.h, self.syn, self.W = dict(d["h"]), dict(d["syn"]), d["W"]
+        # running maxima (cleared by one fill per offline pass): the linear
+        # inputs' per channel (one vector for both sides when the calibration
+        # batches are the linear inputs themselves), the consumers' weights,
+        # and the smoothed norm outputs (static per-tensor scales)
+        self.cal = torch.zeros((6, K), dtype=torch.float32, device=dev)
+        shared = cfg["calib"] == "absmax"
+        self.xmax = {"attn": self.cal[0], "mlp": self.cal[0] if shared else self.cal[1]}
+        self.wmax = {"attn": self.cal[2], "mlp": self.cal[3]}
+        self.vmax = {"attn": self.cal[4], "mlp": self.cal[5]}
+        self.s = {a: {k: f32(K) for k in self.sides} for a in self.alphas}
+        self.gp = {k: f32(K) for k in self.sides}
+        self.bp = {k: None if self.beta[k] is None else f32(K) for k in self.sides}
+        self.qs_static = {k: f32(1) for k in self.sides}
+        self.Wq = {w: torch.empty(self.W[w].shape, dtype=torch.int8, device=dev) for w, _ in cfg["gemms"]}
+        self.qw = {w: f32(self.W[w].shape[0]) for w, _ in cfg["gemms"]}
+        self.Xq = {k: torch.empty((M, K), dtype=torch.int8, device=dev) for k in self.sides}
+        self.qx = {k: f32(M if self.per_token else 1) for k in self.sides}
+        self.Y = {w: torch.empty((M, self.W[w].shape[0]), dtype=self.out_dtype, device=dev) for w, _ in cfg["gemms"]}
+        self.ws = {w: sq.workspace(sq.SQ_OP_GEMM, M, self.W[w].shape[0], self.W[w].shape[1], device=dev)
+                   for w, _ in cfg["gemms"]}
+        self.bank = None
+
+    # one launch, bracketed by events when a bank is attached
+    def launch(self, tag, work, fn, *a):
+        if self.bank is None:
+            fn(*a)
+            return
+        e0, e1 = self.bank.pair(tag, work)
+        e0.record()
+        fn(*a)
+        e1.record()
+
+    def gemm_shapes(self):
+        return [(self.M, self.W[w].shape[0], self.W[w].shape[1]) for w, _ in self.cfg["gemms"]]
+
+    def offline(self):
+        """Calibration, weight maxima, smoothing factors for every alpha (gamma
+        and beta folded for the deployed one), static per-tensor scales where
+        the configuration uses them, and the int8 weights."""
+        sq, d, M, K = self.sq, self.d, self.M, self.K
+        L = self.launch
+        eps = d["eps"]
+        self.cal.zero_()
+        for X in d["calib"]:
+            if self.cfg["calib"] == "absmax":
+                L("calib_absmax", ("hbm", X.numel() * esize(X)), sq.sq_calib_absmax, X, self.xmax["attn"])
+            else:
+                for k in self.sides:
+                    L("calib_norm", ("hbm", X.numel() * esize(X)), sq.sq_norm_smooth_quant, X, self.norm,
+                      self.gamma[k], self.beta[k], eps, True, None, None, None, self.xmax[k])
+        for k in self.sides:
+            W = self.W[self.consumer[k]]
+            L("weight_absmax", ("hbm", W.numel() * esize(W)), sq.sq_weight_absmax, W, self.wmax[k])
+        for a in self.alphas:
+            for k in self.sides:
+                if a == self.alpha:
+                    L("smooth_fold_norm", ("latency", 0), sq.sq_smooth_fold_norm, self.xmax[k], self.wmax[k], a,
+                      self.gamma[k], self.beta[k], self.s[a][k], self.gp[k], self.bp[k])
+                else:
+                    L("smooth_scales", ("latency", 0), sq.sq_smooth_scales, self.xmax[k], self.wmax[k], a,
+                      self.s[a][k])
+        if not self.per_token:
+            for X in d["calib"]:
+                for k in self.sides:
+                    L("calib_norm_smoothed", ("hbm", X.numel() * esize(X)), sq.sq_norm_smooth_quant, X, self.norm,
+                      self.gp[k], self.bp[k], eps, True, None, None, None, self.vmax[k])
+            for k in self.sides:
+                L("scale_from_absmax", ("latency", 0), sq.sq_scale_from_absmax, self.vmax[k], self.qs_static[k])
+        for w, src in self.cfg["gemms"]:
+            W = self.W[w]
+            s = None if src == "syn" else self.s[self.alpha][src]
+            L("quantize_weight", ("hbm", W.numel() * (esize(W) + 1) + 4 * W.shape[0]), sq.sq_quantize_weight, W, s,
+              True, self.Wq[w], self.qw[w])
+
+    def step(self):
+        """The online linear stack: per side, norm + smoothing + int8 then the
+        GEMM that reads it; the synthetic-input GEMMs in block order."""
+        sq, M, K = self.sq, self.M, self.K
+        L = self.launch
+        eps = self.d["eps"]
+        ob = esize(self.Y[self.cfg["gemms"][0][0]])
+        for w, src in self.cfg["gemms"]:
+            if src == "syn":
+                xq, qx = self.syn[w]
+            else:
+                h = self.h[src]
+                st = None if self.per_token else self.qs_static[src]
+                L("norm_quant", ("hbm", M * K * esize(h) + M * K + 4 * self.qx[src].numel()), sq.sq_norm_smooth_quant,
+                  h, self.norm, self.gp[src], self.bp[src], eps, self.per_token, st, self.Xq[src], self.qx[src])
+                xq, qx = self.Xq[src], self.qx[src]
+            N, Kw = self.W[w].shape
+            L("gemm_w8a8", ("tensor", 2.0 * M * N * Kw, M * Kw + N * Kw + M * N * ob), sq.sq_gemm_w8a8, xq,
+              self.Wq[w], qx, self.qw[w], None, self.Y[w], self.ws[w])
+
+    def launches_per_step(self):
+        return sum(2 if src != "syn" else 1 for _, src in self.cfg["gemms"])
+
+    # per-step inputs and outputs (the e2e leg copies them to and from the host)
+    def io(self):
+        ins = [self.h[k] for k in self.sides] + [t for w in self.syn for t in self.syn[w]]
+        outs = [self.Y[w] for w, _ in self.cfg["gemms"]]
+        return ins, outs
+
+    def swap_io(self, other=None):
+        """Point the step at another set of input/output buffers (fresh ones
+        when other is None); returns the previous set."""
+        torch = self.torch
+        old = (self.h, self.syn, self.Y)
+        if other is None:
+            other = ({k: torch.empty_like(v).copy_(v) for k, v in self.h.items()},
+                     {k: tuple(torch.empty_like(t).copy_(t) for t in v) for k, v in self.syn.items()},
+                     {k: torch.empty_like(v) for k, v in self.Y.items()})
+        self.h, self.syn, self.Y = other
+        return old
+
+
+class LlmInt8Stack:
+    """The LLM.int8() call at 6.7B shapes: offline = the weight's int8 copy for
+    the outlier set; step = one sq_llmint8_matmul (detection, row
+    quantisation, the int8 GEMM with the fused 16-bit outlier term) with the
+    weight cache warm."""
 
     def __init__(self, dev):
         import torch
@@ -176,186 +398,128 @@ class Layer:
         import w8a8_post_quantization_sq_b200 as sq
         from w8a8_post_quantization_sq_b200 import inputs
 
-        self.sq, self.torch = sq, torch
-        d = inputs.c2_qwen3_06b(device=dev)
-        self.d = d
-        M, K = M_TOKENS, HIDDEN
-        e = lambda *s, dt=torch.float32: torch.empty(s, dtype=dt, device=dev)  # noqa: E731
-        self.h = {"attn": d["h_attn"], "mlp": d["h_mlp"]}
-        self.gamma = {"attn": d["gamma_attn"].float().contiguous(), "mlp": d["gamma_mlp"].float().contiguous()}
-        self.W = d["W"]
-        self.V = {k: e(M, K, dt=torch.bfloat16) for k in ("attn", "mlp")}
-        # the four running maxima share one buffer, cleared by one fill per step
-        self.maxima = e(4, K)
-        self.xmax = {"attn": self.maxima[0], "mlp": self.maxima[1]}
-        self.wmax = {"attn": self.maxima[2], "mlp": self.maxima[3]}
-        self.s = {k: e(K) for k in ("attn", "mlp")}
-        self.gp = {k: e(K) for k in ("attn", "mlp")}
-        self.Wq = {k: e(*self.W[k].shape, dt=torch.int8) for k in self.W}
-        self.qw = {k: e(self.W[k].shape[0]) for k in self.W}
-        self.Xq = {k: e(M, K, dt=torch.int8) for k in ("attn", "mlp")}
-        self.qx = {k: e(M) for k in ("attn", "mlp")}
-        xo, so = d["o_in"]
-        xd, sd = d["down_in"]
-        self.act_in = {"o": (xo, so), "down": (xd, sd)}
-        self.Y = {k: e(M, self.W[k].shape[0], dt=torch.bfloat16) for k in self.W}
-        self.Y["llm"] = e(M, 4096, dt=torch.bfloat16)
-        self.ws = sq.workspace(sq.SQ_OP_LLMINT8, M, 4096, K, device=dev)
-        self.ws_gemm = {k: sq.workspace(sq.SQ_OP_GEMM, M, 4096, K, device=dev) for k in ("qkv", "o", "gateup", "down")}
-        self.llm = sq.llmint8_weight_state(self.W["qkv"])
-        self.idx = e(K, dt=torch.int32)
-        self.nidx = e(1, dt=torch.int32)
-        # down_proj's input: SwiGLU of the gate/up output, smoothed by s_down
-        # folded into up_proj's output channels
-        I = self.W["down"].shape[1]
-        self.I = I
-        self.W_gate, self.W_up = self.W["gateup"][:I], self.W["gateup"][I:]
-        self.Xq_down = e(M, I, dt=torch.int8)
-        self.qx_down = e(M)
-        self.s_down = self.calibrate_down()
-        self.streams = [torch.cuda.Stream(device=dev) for _ in range(5)]
-        self.events = {n: torch.cuda.Event() for n in ("wmax_attn", "wmax_mlp", "V_attn", "V_mlp", "s_attn", "s_mlp",
-                                                      "wq_qkv", "wq_gateup", "wq_down")}
+        self.sq, self.torch, self.dev = sq, torch, dev
+        M, K, N = C4["M"], C4["K"], C4["N"]
+        self.M, self.K, self.N = M, K, N
+        self.d = inputs.c4_llmint8(device=dev, M=M, K=K, N=N)
+        self.st = sq.llmint8_weight_state(self.d["W"])
+        self.Y = torch.empty((M, N), dtype=torch.float16, device=dev)
+        self.idx = torch.empty(K, dtype=torch.int32, device=dev)
+        self.n = torch.empty(1, dtype=torch.int32, device=dev)
+        self.ws = sq.workspace(sq.SQ_OP_LLMINT8, M, N, K, device=dev)
+        self.ws_det = sq.workspace(sq.SQ_OP_LLMINT8_DETECT, M, N, K, device=dev)
+        self.bank = None
 
-    def calibrate_down(self):
-        """s for down_proj's input, from one pass of the MLP input through the
-        unsmoothed int8 gate/up projection: running max of |silu(gate) * up|
-        (calibration mode of sq_act_quant) against down_proj's weight maxima. Done once, at
-        set-up; the step then folds it (1/s into up_proj's rows, s into
-        down_proj's columns)."""
-        sq, d, torch = self.sq, self.d, self.torch
-        M, K, I = M_TOKENS, HIDDEN, self.I
-        dev = self.h["mlp"].device
-        e = lambda *s_, dt=torch.float32: torch.empty(s_, dtype=dt, device=dev)  # noqa: E731
-        V = e(M, K, dt=torch.bfloat16)
-        sq.sq_norm_smooth_quant(self.d["h_calib"].to(dev), sq.SQ_RMSNORM, self.gamma["mlp"], None, d["eps"], True, None,
-                                None, None, None, V)
-        Xq, qx = e(M, K, dt=torch.int8), e(M)
-        sq.sq_quantize_act(V, None, True, None, Xq, qx)
-        Wq, qw = e(2 * I, K, dt=torch.int8), e(2 * I)
-        sq.sq_quantize_weight(self.W["gateup"], None, True, Wq, qw)
-        Y = e(M, 2 * I, dt=torch.bfloat16)
-        sq.sq_gemm_w8a8(Xq, Wq, qx, qw, None, Y, sq.workspace(sq.SQ_OP_GEMM, M, 2 * I, K, device=dev))
-        hmax = torch.zeros(I, device=dev)
-        sq.sq_act_quant(Y, sq.SQ_ACT_SWIGLU, True, None, None, None, hmax)
-        wmax = torch.zeros(I, device=dev)
-        sq.sq_weight_absmax(self.W["down"], wmax)
-        s = e(I)
-        sq.sq_smooth_scales(hmax, wmax, d["alpha"], s)
-        torch.cuda.synchronize()
-        return s
+    launch = Stack.launch
 
-    def step(self, gemm_ev=None):
-        """One pass of every row. Independent chains run on their own streams
-        (forked from and joined back into the current stream), so the
-        latency-bound small kernels of one chain overlap the others."""
-        sq, d, torch = self.sq, self.d, self.torch
-        eps = d["eps"]
-        I = self.I
-        main = torch.cuda.current_stream()
-        sA, sB, sC, sD, sE = self.streams
-        ev = self.events
-        self.maxima.zero_()
-        for s_ in self.streams:
-            s_.wait_stream(main)
+    def gemm_shapes(self):
+        return [(self.M, self.N, self.K)]
 
-        def gemm(i, w, xq, qx):
-            if gemm_ev is not None:
-                gemm_ev[i][0].record()
-            sq.sq_gemm_w8a8(xq, self.Wq[w], qx, self.qw[w], None, self.Y[w], self.ws_gemm[w])
-            if gemm_ev is not None:
-                gemm_ev[i][1].record()
+    def offline(self):
+        sq, X, W = self.sq, self.d["X"], self.d["W"]
+        self.launch("llmint8_detect", ("hbm", X.numel() * 2), sq.sq_llmint8_detect, X, 6.0, 0.0, self.idx, self.n,
+                    self.ws_det)
+        self.launch("llmint8_quant_weight", ("hbm", W.numel() * 3 + 4 * self.N), sq.sq_llmint8_quant_weight, W,
+                    self.idx, self.n, self.st["Wq"], self.st["qs_w"])
 
-        # the MLP chain (norm -> gate/up GEMM -> SwiGLU -> down GEMM) is the
-        # longest, so the weight-side work it waits for goes first on each stream
-        with torch.cuda.stream(sC):
-            sq.sq_weight_absmax(self.W["gateup"], self.wmax["mlp"])
-            ev["wmax_mlp"].record()
-            sq.sq_weight_absmax(self.W["qkv"], self.wmax["attn"])
-            ev["wmax_attn"].record()
-            sq.sq_quantize_weight(self.W["down"], self.s_down, True, self.Wq["down"], self.qw["down"])
-            ev["wq_down"].record()
-            sq.sq_quantize_weight(self.W["o"], None, True, self.Wq["o"], self.qw["o"])
-            gemm(1, "o", *self.act_in["o"])
-        chains = (("attn", "qkv", sA, 0), ("mlp", "gateup", sB, 2))
-        for k, w, s_, i in chains:
-            with torch.cuda.stream(s_):
-                # norm (calibration pass) -> linear input; its column absmax
-                sq.sq_norm_smooth_quant(self.h[k], sq.SQ_RMSNORM, self.gamma[k], None, eps, True, None, None,
-                                        None, None, self.V[k])
-                ev["V_" + k].record()
-                sq.sq_calib_absmax(self.V[k], self.xmax[k])
-                s_.wait_event(ev["wmax_" + k])
-                # s and gamma' = gamma / s in one launch
-                sq.sq_smooth_fold_norm(self.xmax[k], self.wmax[k], d["alpha"], self.gamma[k], None, self.s[k],
-                                       self.gp[k])
-                ev["s_" + k].record()
-                sq.sq_norm_smooth_quant(self.h[k], sq.SQ_RMSNORM, self.gp[k], None, eps, True, None,
-                                        self.Xq[k], self.qx[k], None, None)
-        with torch.cuda.stream(sD):  # weight quantisation once s is known
-            sD.wait_event(ev["s_mlp"])
-            sq.sq_quantize_weight(self.W_gate, self.s["mlp"], True, self.Wq["gateup"][:I], self.qw["gateup"][:I])
-            # up_proj: 1/s_down folded into its output channels (down_proj takes
-            # s_down) and its own s, in the quantising pass
-            sq.sq_quantize_weight_fold_prev(self.W_up, self.s_down, self.s["mlp"], self.Wq["gateup"][I:],
-                                            self.qw["gateup"][I:])
-            ev["wq_gateup"].record()
-            sD.wait_event(ev["s_attn"])
-            sq.sq_quantize_weight(self.W["qkv"], self.s["attn"], True, self.Wq["qkv"], self.qw["qkv"])
-            ev["wq_qkv"].record()
-        for k, w, s_, i in chains:
-            with torch.cuda.stream(s_):
-                s_.wait_event(ev["wq_" + w])
-                gemm(i, w, self.Xq[k], self.qx[k])
-        with torch.cuda.stream(sB):
-            # down_proj's input from the SwiGLU of the gate/up output
-            sq.sq_act_quant(self.Y["gateup"], sq.SQ_ACT_SWIGLU, True, None, self.Xq_down, self.qx_down)
-            sB.wait_event(ev["wq_down"])
-            gemm(3, "down", self.Xq_down, self.qx_down)
-        with torch.cuda.stream(sE):  # LLM.int8 decomposition
-            sE.wait_event(ev["V_attn"])
-            sq.sq_llmint8_matmul(self.V["attn"], self.llm, 6.0, 0.0, self.Y["llm"], self.idx, self.nidx, self.ws)
-        for s_ in self.streams:
-            main.wait_stream(s_)
+    def step(self):
+        M, N, K = self.M, self.N, self.K
+        self.launch("llmint8_matmul", ("tensor", 2.0 * M * N * K, M * K * 2 + N * K + M * N * 2),
+                    self.sq.sq_llmint8_matmul, self.d["X"], self.st, 6.0, 0.0, self.Y, self.idx, self.n, self.ws)
 
-    def outputs(self):
-        return [self.Y[k] for k in ("qkv", "o", "gateup", "down", "llm")]
+    def launches_per_step(self):
+        return 5  # counts, compaction, weight-side pass, row quantisation, GEMM
 
 
-def run_ours(args, rank, world, dev):
+def summarise(bank, per_launch_ms, ipk, hbm):
+    """Per-kernel figures from an instrumented replay: launches, mean time per
+    launch, achieved throughput from the algorithmic work, and the fraction
+    of the peak that bounds the kernel (int8 dense for the GEMMs, measured
+    copy bandwidth for the memory-bound kernels)."""
+    out = {}
+    for (tag, work, _), ms in zip(bank.pairs, per_launch_ms):
+        r = out.setdefault(tag, {"kernel": tag, "launches": 0, "ms": 0.0, "work": 0.0, "bytes": 0.0, "bound": work[0]})
+        r["launches"] += 1
+        r["ms"] += ms
+        r["work"] += work[1]
+        if work[0] == "tensor":
+            r["bytes"] += work[2]
+    rows = []
+    for r in out.values():
+        t = r["ms"] * 1e-3
+        e = {"kernel": r["kernel"], "launches": r["launches"], "us_per_launch": r["ms"] * 1e3 / r["launches"],
+             "us_total": r["ms"] * 1e3, "bound": r["bound"]}
+        if r["bound"] == "tensor":
+            a = r["work"] / t / 1e12
+            e.update({"ops_per_launch": r["work"] / r["launches"], "achieved": a, "unit": "TOPS",
+                      "peak": ipk["burst"], "frac": a / ipk["burst"], "frac_sustained": a / ipk["sustained"],
+                      "frac_nominal": a / ipk["nominal"], "algorithmic_bytes_per_launch": r["bytes"] / r["launches"]})
+        elif r["bound"] == "hbm":
+            a = r["work"] / t / 1e9
+            e.update({"bytes_per_launch": r["work"] / r["launches"], "achieved": a, "unit": "GB/s", "peak": hbm,
+                      "frac": a / hbm})
+        rows.append(e)
+    return rows
+
+
+def capture(fn, stream):
+    import torch
+
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    return g
+
+
+def timed_replays(graph, bank, n, flush, stream):
+    """Per-launch durations (ms) of an instrumented graph, averaged over n
+    replays, each after an L2 flush."""
+    import torch
+
+    acc = None
+    with torch.cuda.stream(stream):
+        for i in range(n):
+            flush(i)
+            graph.replay()
+            stream.synchronize()
+            v = np.array(bank.read())
+            acc = v if acc is None else acc + v
+    return (acc / n).tolist()
+
+
+def run_stack(st, args, rank, world, dev, flush, e2e=True):
+    """Time one stack: the offline pass (instrumented), the online step (plain
+    graph, timed; then instrumented, for per-kernel times) and, with e2e, the
+    step through the public API with pinned host buffers."""
     import torch
     import torch.distributed as dist
 
-    torch.cuda.set_device(dev)
-    L = Layer(dev)
-    stream = torch.cuda.Stream()
+    ipk = int8_peaks()
+    hbm = peaks()[0]["hbm_gbs"]
+    stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):
-        L.step()
-        L.step()
+        st.offline()
+        st.step()
     stream.synchronize()
-    # the step as timed: one CUDA graph with nothing but the step in it
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream):
-        L.step()
-    # a second capture of the same step with events around its four GEMMs, for
-    # their launch durations; event nodes break the programmatic chaining of
-    # the GEMMs with their producers, so this copy is replayed after the timed
-    # region, not inside it (external events are re-recorded by every replay)
-    n_g = 4
-    gemm_ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)] for _ in range(n_g)]
-    graph_ev = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph_ev, stream=stream):
-        L.step(gemm_ev)
-    flush = L2Flush(dev)
+    g_step = capture(st.step, stream)
+    st.bank = EventBank()
+    g_step_ev = capture(st.step, stream)
+    bank_step = st.bank
+    st.bank = EventBank()
+    g_off_ev = capture(st.offline, stream)
+    bank_off = st.bank
+    st.bank = None
     with torch.cuda.stream(stream):
         for _ in range(max(args.warmup, 3)):
-            graph.replay()
-            graph_ev.replay()
+            g_step.replay()
+        g_off_ev.replay()
+        g_step_ev.replay()
     torch.cuda.synchronize()
 
+    # the timed region: K replays of the step, each after an L2 flush
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    clocks = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    clocks = ClockSampler(dev.index if dev.index is not None else 0) if rank == 0 else None
     time.sleep(0.05)
     if world > 1:
         dist.barrier()
@@ -364,47 +528,48 @@ def run_ours(args, rank, world, dev):
         for i in range(args.steps):
             flush(i)
             ev[i][0].record(stream)
-            graph.replay()
+            g_step.replay()
             ev[i][1].record(stream)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     clk = clocks.stop() if clocks else None
     step_ms = [a.elapsed_time(b) for a, b in ev]
-    total_ms = max_over_ranks(sum(step_ms), dev)
-    ms_per_step = total_ms / args.steps
+    ms_per_step = max_over_ranks(sum(step_ms), dev) / args.steps
 
-    # GEMM launch durations: the instrumented step, L2 flushed before each
-    gemm_ms = []
-    n_ev = min(args.steps, GEMM_TIMED_STEPS)
-    with torch.cuda.stream(stream):
-        for i in range(n_ev):
-            flush(i)
-            graph_ev.replay()
-            stream.synchronize()
-            gemm_ms.append([gemm_ev[j][0].elapsed_time(gemm_ev[j][1]) for j in range(n_g)])
-    torch.cuda.synchronize()
+    n_ev = max(3, min(args.steps, 50))
+    k_step = summarise(bank_step, timed_replays(g_step_ev, bank_step, n_ev, flush, stream), ipk, hbm)
+    k_off = summarise(bank_off, timed_replays(g_off_ev, bank_off, max(3, min(args.steps, 10)), flush, stream), ipk,
+                      hbm)
+    r = {"ms_per_step": ms_per_step, "step_ms_median": statistics.median(step_ms), "clocks": clk,
+         "kernels": k_step, "offline": k_off, "instrumented_replays": n_ev, "ipk": ipk, "hbm": hbm,
+         "launches_per_step": st.launches_per_step()}
+    if e2e:
+        r.update(run_e2e(st, g_step, args, world, dev, stream))
+    del g_step, g_step_ev, g_off_ev
+    return r
 
-    # e2e through the public API with host buffers: every step copies its
-    # inputs in from pinned host memory, runs the step and copies every output
-    # back, all inside the timed region. Two buffer sets (a second capture of
-    # the step on the other set) let step i's outputs go out and step i+1's
-    # inputs come in on copy streams while step i+1 computes.
-    h_host = {k: L.h[k].cpu().pin_memory() for k in L.h}
-    h_alt = {k: torch.empty_like(v) for k, v in L.h.items()}
-    y_alt = {k: torch.empty_like(v) for k, v in L.Y.items()}
-    h_main, y_main = L.h, L.Y
-    L.h, L.Y = h_alt, y_alt
-    graph_b = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph_b, stream=stream):
-        L.step()
-    outs_b = L.outputs()
-    L.h, L.Y = h_main, y_main
-    sets = [(L.h, L.outputs(), graph), (h_alt, outs_b, graph_b)]
-    o_host = [[torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs_b] for _ in range(2)]
-    h2d = sum(v.numel() * v.element_size() for v in h_host.values())
-    d2h = sum(o.numel() * o.element_size() for o in outs_b)
-    e2e_steps = max(3, min(args.steps, 50))
+
+def run_e2e(st, graph, args, world, dev, stream):
+    """The step through the public API with host buffers: every step copies
+    its inputs in from pinned host memory, runs the step and copies every
+    output back, all inside the timed region. Two buffer sets (a second capture
+    of the step on the other set) let step i's outputs go out and step i+1's
+    inputs come in on copy streams while step i+1 computes."""
+    import torch
+    import torch.distributed as dist
+
+    ins_a, outs_a = st.io()
+    host_in = [t.cpu().pin_memory() for t in ins_a]
+    main = st.swap_io()
+    graph_b = capture(st.step, stream)
+    ins_b, outs_b = st.io()
+    st.swap_io(main)
+    sets = [(ins_a, outs_a, graph), (ins_b, outs_b, graph_b)]
+    host_out = [[torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs_a] for _ in range(2)]
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = sum(o.numel() * o.element_size() for o in outs_a)
+    n = max(3, min(args.steps, 20))
     s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
     ev_in = [torch.cuda.Event() for _ in range(2)]
     ev_done = [torch.cuda.Event() for _ in range(2)]
@@ -416,14 +581,14 @@ def run_ours(args, rank, world, dev):
     e0.record(stream)
     s_in.wait_stream(stream)
     s_out.wait_stream(stream)
-    for i in range(e2e_steps):
+    for i in range(n):
         b = i % 2
-        h_dev, outs, g = sets[b]
+        ins, outs, g = sets[b]
         with torch.cuda.stream(s_in):
             if i >= 2:
                 s_in.wait_event(ev_done[b])  # step i-2 has read this input set
-            for k in h_dev:
-                h_dev[k].copy_(h_host[k], non_blocking=True)
+            for t, th in zip(ins, host_in):
+                t.copy_(th, non_blocking=True)
             ev_in[b].record(s_in)
         with torch.cuda.stream(stream):
             stream.wait_event(ev_in[b])
@@ -433,191 +598,304 @@ def run_ours(args, rank, world, dev):
             ev_done[b].record(stream)
         with torch.cuda.stream(s_out):
             s_out.wait_event(ev_done[b])
-            for o, oh in zip(outs, o_host[b]):
+            for o, oh in zip(outs, host_out[b]):
                 oh.copy_(o, non_blocking=True)
             ev_out[b].record(s_out)
     stream.wait_stream(s_in)
     stream.wait_stream(s_out)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n, dev)
     del graph_b
+    return {"e2e_ms": e2e_ms, "h2d": h2d, "d2h": d2h, "e2e_steps": n}
 
-    gm = np.array(gemm_ms)  # [steps, 4]
-    gemm_ops = [2.0 * m * n * k for (m, n, k) in GEMMS[:4]]
-    gemm_avg_ms = gm.mean(axis=0)
-    gemm_tops = sum(gemm_ops) / (gemm_avg_ms.sum() * 1e-3) / 1e12
-    pk, src = peaks()
-    i8_peak = 2.0 * pk["bf16_tflops"]  # dense int8 = 2 x dense bf16 (nominal 4.5 vs 2.25 PFLOP/s)
-    del graph, graph_ev
-    return {
-        "ms_per_step": ms_per_step, "e2e_ms": e2e_ms, "h2d": h2d, "d2h": d2h, "clocks": clk,
-        "gemm_avg_ms": gemm_avg_ms.tolist(), "gemm_timed_steps": n_ev, "gemm_tops": gemm_tops, "i8_peak": i8_peak, "peak_src": src,
-        "step_ms_median": statistics.median(step_ms),
+
+def gemm_roofline(r, shapes):
+    """The dominant kernel's roofline: the int8 GEMM over its launches in one
+    step (sum of 2MNK over sum of launch durations)."""
+    g = [k for k in r["kernels"] if k["kernel"] in ("gemm_w8a8", "llmint8_matmul")][0]
+    ipk = r["ipk"]
+    traffic = gemm_traffic(shapes)
+    return {"bound": "tensor", "achieved": g["achieved"], "peak": ipk["burst"], "unit": "TOPS",
+            "frac": g["achieved"] / ipk["burst"], "traffic": None if traffic is None else sum(traffic),
+            "kernel": "gemm_w8a8_kernel", "launches_per_step": g["launches"],
+            "ops_per_step": g["ops_per_launch"] * g["launches"],
+            "algorithmic_bytes_per_step": g["algorithmic_bytes_per_launch"] * g["launches"],
+            "traffic_per": f"one step ({g['launches']} launches)",
+            "peak_source": f"{ipk['source']} bf16 burst x 2 (nominal int8:bf16 ratio)",
+            "peak_sustained": ipk["sustained"], "frac_sustained": g["achieved"] / ipk["sustained"],
+            "peak_nominal": ipk["nominal"], "frac_nominal": g["achieved"] / ipk["nominal"],
+            "timing": f"CUDA events around each launch of an instrumented copy of the step's graph, "
+                      f"{r['instrumented_replays']} replays after the timed region, L2 flushed before each"}
+
+
+def config_summary(name, r, tokens, world, shapes):
+    """A compact line for a non-headline configuration."""
+    g = [k for k in r["kernels"] if k["kernel"] in ("gemm_w8a8", "llmint8_matmul")][0]
+    return {"workload": (CONFIGS[name]["workload"] if name in CONFIGS else C4["workload"]),
+            "tokens": tokens, "tokens_per_s": tokens * world / (r["ms_per_step"] * 1e-3),
+            "ms_per_step": r["ms_per_step"], "gemm_tops": g["achieved"], "gemm_frac": g["frac"],
+            "gemm_frac_nominal": g["frac_nominal"], "gemm_shapes": shapes, "kernels": r["kernels"],
+            "offline": r["offline"], "clocks": r["clocks"]}
+
+
+def json_line(args, world, r, shapes, tokens=None, cfg=None):
+    """The benchmark's JSON line (without the CPU baseline) from the measured
+    headline stack."""
+    cfg = cfg or CONFIGS[HEADLINE]
+    tokens = tokens or cfg["tokens"]
+    calib = [k for k in r["offline"] if k["kernel"] == "calib_absmax"]
+    line = {
+        "metric": METRIC, "value": tokens * world / (r["ms_per_step"] * 1e-3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms_per_step"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "i8",
+        "data": "synthetic (seeded draws with the configuration's shapes and outlier channels; no dataset)",
+        "config": {"workload": cfg["workload"], "tokens": tokens, "hidden": cfg["hidden"],
+                   "parallelism": f"replicas x{world}", "l2": L2_NOTE},
+        "roofline": gemm_roofline(r, shapes),
+        "kernels": r["kernels"],
+        "offline": {"kernels": r["offline"], "ms": sum(k["us_total"] for k in r["offline"]) * 1e-3,
+                    "note": "calibration, weight maxima, smoothing factors for every alpha, int8 weights: "
+                            "timed separately, not part of the step"},
+        "calibration": None if not calib else {
+            "batches": calib[0]["launches"], "us_per_batch": calib[0]["us_per_launch"],
+            "achieved": calib[0]["achieved"], "unit": "GB/s", "peak": r["hbm"], "frac": calib[0]["frac"]},
+        "gpu_launches": r["launches_per_step"] * args.steps,
+        "clocks": r["clocks"],
     }
+    if "e2e_ms" in r:
+        line["e2e"] = {"value": tokens * world / (r["e2e_ms"] * 1e-3), "unit": "tokens/s",
+                       "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
+                       "ms_per_step": r["e2e_ms"], "steps": r["e2e_steps"]}
+    return line
 
 
-# ------------------------------------------------------------------ CPU arm
-class CpuStep:
-    """The oracle, as it stands, on the benchmark's step, timed on a sample.
+def run_ours(args, rank, world, dev):
+    import torch
 
-    The inputs, and the step's set-up (down_proj's smoothing factors from a
-    calibration pass, and the full int8 weights the token rows multiply), are
-    made once, untimed. Each call of ``step(rows, wfrac)`` then times the
-    whole path on a sample: the per-token work for ``rows`` tokens, and the
-    weight-side work (maxima, smoothing factors, folds, quantisation, the
-    LLM.int8 weight requantisation) on the first ``wfrac`` of every weight's
-    output channels. Both are linear in what they process, so the step time
-    of the full workload is t_weights / wfrac + t_rows * tokens / rows."""
+    torch.cuda.set_device(dev)
+    flush = L2Flush(dev)
+    st = Stack(args.workload, dev)
+    shapes = st.gemm_shapes()
+    r = run_stack(st, args, rank, world, dev, flush, e2e=True)
+    cfg = CONFIGS[args.workload]
+    line = json_line(args, world, r, shapes, cfg["tokens"], cfg)
+    del st
+    torch.cuda.empty_cache()
+    if args.configs:
+        extra = {}
+        for name in [c for c in args.configs.split(",") if c and c != args.workload]:
+            if name == "c4":
+                s = LlmInt8Stack(dev)
+                rr = run_stack(s, args, rank, world, dev, flush, e2e=False)
+                extra[name] = config_summary(name, rr, C4["tokens"], world, s.gemm_shapes())
+            else:
+                s = Stack(name, dev)
+                rr = run_stack(s, args, rank, world, dev, flush, e2e=False)
+                extra[name] = config_summary(name, rr, CONFIGS[name]["tokens"], world, s.gemm_shapes())
+            del s
+            torch.cuda.empty_cache()
+        line["configs"] = extra
+    return line
 
-    def __init__(self, rows=64):
+
+# ------------------------------------------------------------------ CPU arm (the oracle)
+class CpuStack:
+    """The oracle, as it stands, on the deploy-mode linear stack of a
+    configuration, on a sample: `rows` tokens through every online step and the
+    first `wfrac` of every weight's output channels. The offline part (the
+    calibration maxima, smoothing factors, folded norm parameters, static
+    scales and int8 weights of the sampled channels) is made once, untimed.
+    A step's time for the whole workload is t_norm * M / rows +
+    t_gemm * M / rows / wfrac: both parts are linear in what they process.
+    threads > 1 runs the oracle's calls on disjoint row and channel blocks in
+    a thread pool (the oracle's C calls release the GIL); the arithmetic is
+    the same."""
+
+    def __init__(self, name, rows, wfrac, threads=1):
         import torch
 
         import oracle
         from w8a8_post_quantization_sq_b200 import inputs
 
         oracle.lib()
-        self.o, self.torch = oracle, torch
-        d = inputs.c2_qwen3_06b(device="cpu")
+        cfg = CONFIGS[name]
+        self.o, self.torch, self.cfg = oracle, torch, cfg
+        self.rows, self.wfrac, self.threads = rows, wfrac, threads
+        d = getattr(inputs, cfg["gen"])(device="cpu", M=rows, w_frac=wfrac)
         self.d = d
-        self.gamma = {"attn": d["gamma_attn"].numpy(), "mlp": d["gamma_mlp"].numpy()}
-        self.W = W = {k: oracle.f32(v) for k, v in d["W"].items()}
-        self.I = I = W["down"].shape[1]
-        sl = slice(0, rows)
-        # down_proj's smoothing factors, from a calibration pass over the sample
-        Vc = oracle.norm_smooth_quant(d["h_calib"][sl], oracle.RMSNORM, self.gamma["mlp"], None, d["eps"],
-                                      quantize=False, want_v=True)["V"]
-        Vc16 = torch.from_numpy(Vc).to(torch.bfloat16).float().numpy()
-        Xc, qc = oracle.quantize_act(Vc16, None, per_token=True)
-        Wc, qwc = oracle.quantize_weight(W["gateup"], True)
-        hmax = oracle.act_quant(self.bf16(oracle.dequant(oracle.gemm_i8(Xc, Wc), qc, qwc)), oracle.SWIGLU,
-                                quantize=False, absmax=np.zeros(I, np.float32))["absmax"]
-        self.s_down = oracle.smooth_scales(hmax, oracle.col_absmax(W["down"]), d["alpha"])
-        # the full weight side once, for the token rows of every sampled step
-        h = {"attn": d["h_attn"][sl], "mlp": d["h_mlp"][sl]}
-        V = {k: oracle.norm_smooth_quant(h[k], oracle.RMSNORM, self.gamma[k], None, d["eps"], quantize=False,
-                                         want_v=True)["V"] for k in h}
-        V16 = {k: torch.from_numpy(V[k]).to(torch.bfloat16) for k in V}
-        self.xmax = {k: oracle.col_absmax(V16[k]) for k in V}
-        self.gp, self.Wq, self.qw, self.s = {}, {}, {}, {}
-        _, self.llm_idx = self.weight_side(1.0, self.gp, self.Wq, self.qw, self.s,
-                                           oracle.llmint8_outliers(V16["attn"], 6.0, 0.0))
+        o = oracle
+        self.norm = o.LAYERNORM if cfg["norm"] == "layer" else o.RMSNORM
+        eps, alpha = d["eps"], cfg["alpha"]
+        sides = ("attn", "mlp")
+        consumer = {src: w for w, src in cfg["gemms"] if src != "syn"}
+        g = {k: d["gamma"][k].numpy() for k in sides}
+        b = {k: None if d["beta"][k] is None else d["beta"][k].numpy() for k in sides}
+        xmax = {}
+        for k in sides:
+            x = np.zeros(cfg["hidden"], np.float32)
+            for X in d["calib"]:
+                if cfg["calib"] == "absmax":
+                    x = o.col_absmax(X, x)
+                else:
+                    x = o.norm_smooth_quant(X, self.norm, g[k], b[k], eps, quantize=False, absmax=x)["absmax"]
+            xmax[k] = x
+        self.gp, self.bp, self.qs = {}, {}, {}
+        s = {}
+        for k in sides:
+            s[k] = o.smooth_scales(xmax[k], o.col_absmax(d["W"][consumer[k]]), alpha)
+            self.gp[k], self.bp[k] = o.fold_norm(g[k], b[k], s[k])
+            if not cfg["per_token"]:
+                v = np.zeros(cfg["hidden"], np.float32)
+                for X in d["calib"]:
+                    v = o.norm_smooth_quant(X, self.norm, self.gp[k], self.bp[k], eps, quantize=False,
+                                            absmax=v)["absmax"]
+                self.qs[k] = float(o.scale_from_absmax(v))
+        self.Wq, self.qw = {}, {}
+        for w, src in cfg["gemms"]:
+            W = d["W"][w]
+            Wp = o.fold_weight(W, s[src]) if src != "syn" else o.f32(W)
+            self.Wq[w], self.qw[w] = o.quantize_weight(Wp, True)
+        self.h = {k: d["h"][k] for k in sides}
+        self.syn = {w: (t[0].numpy(), t[1].numpy()) for w, t in d["syn"].items()}
+        self.sides = sides
 
-    def bf16(self, y):
-        torch = self.torch
-        return torch.from_numpy(self.o.round_bf16_bits(y).view(np.int16)).view(torch.bfloat16).float().numpy()
+    def step(self, threads=None):
+        """(seconds of norm + int8 work, seconds of GEMM + dequant work) for
+        the sample's tokens and weight channels, on `threads` host threads."""
+        from concurrent.futures import ThreadPoolExecutor
 
-    def weight_side(self, wfrac, gp, Wq, qw, s, idx):
-        """Maxima, smoothing factors, folds and int8 weights on the first
-        wfrac of every weight's output channels; returns (seconds, idx)."""
-        o, W, I, d = self.o, self.W, self.I, self.d
-        part = lambda w: w[: max(1, int(round(w.shape[0] * wfrac)))]  # noqa: E731
-        t0 = time.perf_counter()
-        for k, w in (("attn", "qkv"), ("mlp", "gateup")):
-            wmax = o.col_absmax(part(W[w]))
-            s[k] = o.smooth_scales(self.xmax[k], wmax, d["alpha"])
-            gp[k], _ = o.fold_norm(self.gamma[k], None, s[k])
-        Wq["qkv"], qw["qkv"] = o.quantize_weight(o.fold_weight(part(W["qkv"]), s["attn"]), True)
-        up_f, _ = o.fold_prev_linear(part(W["gateup"][I:]), self.s_down[: part(W["gateup"][I:]).shape[0]])
-        gate_q, gate_s = o.quantize_weight(o.fold_weight(part(W["gateup"][:I]), s["mlp"]), True)
-        up_q, up_s = o.quantize_weight(o.fold_weight(up_f, s["mlp"]), True)
-        Wq["gateup"], qw["gateup"] = np.concatenate([gate_q, up_q]), np.concatenate([gate_s, up_s])
-        Wq["o"], qw["o"] = o.quantize_weight(part(W["o"]), True)
-        Wq["down"], qw["down"] = o.quantize_weight(o.fold_weight(part(W["down"]), self.s_down), True)
-        Wq["llm"], qw["llm"] = o.llmint8_quant_weight(part(W["qkv"]), idx)
-        return time.perf_counter() - t0, idx
+        o, cfg = self.o, self.cfg
+        rows = self.rows
+        eps = self.d["eps"]
+        T = threads or self.threads
+        rnd = o.round_bf16_bits if cfg["out"] == "bf16" else o.round_fp16_bits
+        pool = ThreadPoolExecutor(max_workers=T) if T > 1 else None
 
-    def step(self, rows, wfrac=1.0):
-        """(seconds of weight-side work scaled to all channels, seconds of
-        per-token work for `rows` tokens)."""
-        o, d, torch = self.o, self.d, self.torch
-        sl = slice(0, rows)
-        h = {"attn": d["h_attn"][sl], "mlp": d["h_mlp"][sl]}
-        t0 = time.perf_counter()
-        V = {k: o.norm_smooth_quant(h[k], o.RMSNORM, self.gamma[k], None, d["eps"], quantize=False,
-                                    want_v=True)["V"] for k in h}
-        V16 = {k: torch.from_numpy(V[k]).to(torch.bfloat16) for k in V}
-        for k in V:
-            o.col_absmax(V16[k])
-        t_rows = time.perf_counter() - t0
-        t_w, _ = self.weight_side(wfrac, {}, {}, {}, {}, self.llm_idx)
-        gp, Wq, qw = self.gp, self.Wq, self.qw
+        def rowblocks(n):
+            k = max(1, min(T, n))
+            return [(i * n // k, (i + 1) * n // k) for i in range(k)]
+
         t0 = time.perf_counter()
         Xq, qx = {}, {}
-        for k in h:
-            r = o.norm_smooth_quant(h[k], o.RMSNORM, gp[k], None, d["eps"], True)
-            Xq[k], qx[k] = r["Xq"], r["qs"]
-        xo, so = d["o_in"]
-        Y = {}
-        for w, xq, q in (("qkv", Xq["attn"], qx["attn"]), ("o", xo[sl].numpy(), so[sl].numpy()),
-                         ("gateup", Xq["mlp"], qx["mlp"])):
-            Y[w] = self.bf16(o.dequant(o.gemm_i8(xq, Wq[w]), q, qw[w]))
-        a = o.act_quant(Y["gateup"], o.SWIGLU)
-        self.bf16(o.dequant(o.gemm_i8(a["Xq"], Wq["down"]), a["qs"], qw["down"]))
-        # LLM.int8 of the q/k/v projection: outlier set over the sample rows,
-        # row quantisation, GEMM + outlier term (the weight requantisation for
-        # the set is on the weight side)
-        idx = o.llmint8_outliers(V16["attn"], 6.0, 0.0)
-        Xq8, qx8 = o.llmint8_quant_rows(V16["attn"], idx)
-        t_rows += time.perf_counter() - t0
-        if not np.array_equal(idx, self.llm_idx):  # untimed here: the weight side times the requantisation
-            Wq["llm"], qw["llm"] = o.llmint8_quant_weight(self.W["qkv"], idx)
-            self.llm_idx = idx
+        for k in self.sides:
+            h = self.h[k][:rows]
+            st = None if cfg["per_token"] else self.qs[k]
+
+            def nq(a, b_, h=h, k=k, st=st):
+                return o.norm_smooth_quant(h[a:b_], self.norm, self.gp[k], self.bp[k], eps, cfg["per_token"], st)
+            parts = list(pool.map(lambda ab: nq(*ab), rowblocks(rows))) if pool else [nq(0, rows)]
+            Xq[k] = np.concatenate([p["Xq"] for p in parts])
+            qx[k] = np.concatenate([p["qs"] for p in parts]) if cfg["per_token"] else parts[0]["qs"]
+        t_norm = time.perf_counter() - t0
         t0 = time.perf_counter()
-        y = o.llmint8_combine(o.gemm_i8(Xq8, Wq["llm"]), qx8, qw["llm"], V16["attn"], d["W"]["qkv"], idx)
-        o.round_bf16_bits(y)
-        t_rows += time.perf_counter() - t0
-        return t_w / wfrac, t_rows
+        for w, src in cfg["gemms"]:
+            if src == "syn":
+                xq, q = self.syn[w][0][:rows], self.syn[w][1]
+                q = q[:rows] if q.size > 1 else q
+            else:
+                xq, q = Xq[src], qx[src]
+            Wq, qw = self.Wq[w], self.qw[w]
+            N = Wq.shape[0]
+
+            def gm(a, b_, xq=xq, q=q, Wq=Wq, qw=qw):
+                return rnd(o.dequant(o.gemm_i8(xq, Wq[a:b_]), q, qw[a:b_]))
+            if pool:
+                list(pool.map(lambda ab: gm(*ab), rowblocks(N)))
+            else:
+                gm(0, N)
+        t_gemm = time.perf_counter() - t0
+        if pool:
+            pool.shutdown()
+        return t_norm, t_gemm
+
+    def full_step_s(self, t_norm, t_gemm):
+        M = self.cfg["tokens"]
+        return t_norm * M / self.rows + t_gemm * M / self.rows / self.wfrac
 
 
-def cpu_baseline(rows):
-    t_w, t_rows = CpuStep(rows).step(rows)
-    step_s = t_w + t_rows * (M_TOKENS / rows)
-    return {"value": M_TOKENS / step_s, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{rows} of {M_TOKENS} tokens through every step (weights in full: {t_w:.2f} s; "
-                      f"token rows: {t_rows:.2f} s), extrapolated linearly in tokens",
-            "step_s": step_s}
+def cpu_threads():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(name, rows, wfrac):
+    """The oracle on the headline stack, on one core and on every core of
+    this host, same sample; returns the line's cpu_baseline entry."""
+    M = CONFIGS[name]["tokens"]
+    out = {}
+    c = CpuStack(name, rows, wfrac)
+    c.step(1)  # warm-up: page in the sample
+    for T in (1, cpu_threads()):
+        tn, tg = c.step(T)
+        s = c.full_step_s(tn, tg)
+        out[T] = {"value": M / s, "unit": "tokens/s", "cores": T, "step_s": s,
+                  "sample_s": tn + tg}
+        if T == 1 and cpu_threads() == 1:
+            break
+    T = max(out)
+    smp = (f"{rows} of {M} tokens through the online stack against the first 1/{round(1 / wfrac)} of every "
+           f"weight's output channels (weights smoothed and quantised beforehand, untimed), extrapolated "
+           f"linearly in tokens and channels")
+    return {"value": out[T]["value"], "unit": "tokens/s", "cores": T, "kind": "oracle",
+            "sample": smp + f"; measured {out[T]['sample_s']:.2f} s for the sample on {T} threads",
+            "single_core": {"value": out[1]["value"], "cores": 1,
+                            "sample": f"the same sample, {out[1]['sample_s']:.2f} s on one thread"}}
 
 
 REF_BUDGET_S = 150.0  # wall time of the reference arm's timed steps, whatever --steps asks for
 
 
-def ref_sample(t_w_full, t_row, per_step):
-    """Token rows (1..64) and weight fraction (1, 1/2, ..., 1/64) of one
-    reference step that fit `per_step` seconds, given the full weight side's
-    time and one token row's time: the largest sample that fits, weights in
-    full and 64 rows when there is room."""
-    rows, wfrac = 64, 1.0
-    if t_w_full + 64 * t_row <= per_step:
-        return rows, wfrac
-    while wfrac > 1 / 64 and t_w_full * wfrac > per_step / 2:
+def ref_sample(t_row_norm, t_row_gemm_full, per_step):
+    """Token rows (1..64) and weight fraction (1/16, 1/32, ..., 1/256) of one
+    reference step that fit `per_step` seconds, given one token row's norm
+    time and one token row's GEMM time against the full weights: the largest
+    sample that fits."""
+    wfrac = 1 / 16
+    while wfrac > 1 / 256 and t_row_norm + t_row_gemm_full * wfrac > per_step:
         wfrac /= 2
-    rows = int(max(1, min(64, (per_step - t_w_full * wfrac) // max(t_row, 1e-9))))
+    rows = int(max(1, min(64, per_step // max(t_row_norm + t_row_gemm_full * wfrac, 1e-9))))
     return rows, wfrac
 
 
 def run_reference(args, rank, world):
+    """The oracle as the reference arm: the headline stack's online step on a
+    bounded sample per step, on one host core, extrapolated to the whole
+    workload (the line says so)."""
     if rank != 0:
         return
-    ctx = CpuStep()
-    t_w_full, t16 = ctx.step(16)  # the first warm-up step also sizes the sample
-    rows, wfrac = ref_sample(t_w_full, t16 / 16, REF_BUDGET_S / max(args.steps, 1))
-    for _ in range(min(max(args.warmup, 1), 3) - 1):
-        ctx.step(rows, wfrac)
-    times = []
+    name = args.workload
+    cfg = CONFIGS[name]
+    M = cfg["tokens"]
+    probe = CpuStack(name, 2, 1 / 64)
+    tn, tg = probe.step()
+    t_row_norm, t_row_gemm_full = tn / 2, tg / 2 * 64
+    n_warm = min(max(args.warmup, 1), 3)
+    rows, wfrac = ref_sample(t_row_norm, t_row_gemm_full, REF_BUDGET_S / max(args.steps + n_warm, 1))
+    c = CpuStack(name, rows, wfrac)
+    for _ in range(n_warm):
+        c.step()
+    full, meas = [], []
     for _ in range(args.steps):
-        t_w, t_rows = ctx.step(rows, wfrac)
-        times.append(t_w + t_rows * (M_TOKENS / rows))
-    step_s = sum(times) / len(times)
-    v = M_TOKENS / step_s
-    wpart = "weights in full" if wfrac == 1 else f"1/{round(1 / wfrac)} of every weight's output channels"
+        tn, tg = c.step()
+        meas.append(tn + tg)
+        full.append(c.full_step_s(tn, tg))
+    step_s = sum(full) / len(full)
+    v = M / step_s
+    sample = (f"each step: {rows} of {M} tokens against the first 1/{round(1 / wfrac)} of every weight's output "
+              f"channels, timed, then extrapolated linearly in tokens and channels")
     line = {
         "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "i8", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "tokens": M_TOKENS, "hidden": HIDDEN},
-        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                         "sample": f"each step: {rows} of {M_TOKENS} tokens and {wpart}, extrapolated linearly"},
+        "scaling": "weak", "vs_baseline": None, "dtype": "i8",
+        "data": "synthetic (seeded draws with the configuration's shapes and outlier channels; no dataset)",
+        "config": {"workload": cfg["workload"], "tokens": M, "hidden": cfg["hidden"],
+                   "parallelism": f"replicas x{args.gpus}", "l2": L2_NOTE},
+        "ms_per_step_extrapolated": True,
+        "ms_per_step_measured_sample": 1e3 * sum(meas) / len(meas),
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -632,7 +910,8 @@ def run_kernel(args):
     back to back (one flush before the run); the time per launch is the run's
     time divided by the launches. With S sets larger than L2 in all, no launch
     finds its inputs in L2 (e.g. absmax 4096,12288 --sets 16 is the 16-batch
-    calibration pass of the 175B-shaped configuration)."""
+    calibration pass of the 175B-shaped configuration). The clocks are sampled
+    during the timed replay."""
     import torch
 
     import w8a8_post_quantization_sq_b200 as sq
@@ -644,6 +923,7 @@ def run_kernel(args):
     shape = [int(x) for x in args.shape.split(",")]
     g = torch.Generator(device=dev).manual_seed(0)
     pk, src = peaks()
+    ipk = int8_peaks()
     flush = L2Flush(dev)
     out = {"kernel": args.kernel, "shape": shape, "dtype": args.dtype}
 
@@ -716,10 +996,13 @@ def run_kernel(args):
             return lambda: sq.sq_llmint8_matmul(d["X"], st, 6.0, 0.0, Y, idx, n, ws)
         raise SystemExit(f"unknown kernel {args.kernel}")
 
-    if args.kernel in ("gemm", "gemm_fp8"):
-        M, N, K = shape
+    if args.kernel in ("gemm", "gemm_fp8", "llmint8"):
+        if args.kernel == "llmint8":
+            M, K, N = shape
+        else:
+            M, N, K = shape
         # dense int8 and fp8 peaks are both twice the bf16 one (4.5 vs 2.25 PFLOP/s nominal)
-        work, unit, peak = 2.0 * M * N * K / 1e12, "TOPS", 2.0 * pk["bf16_tflops"]
+        work, unit, peak = 2.0 * M * N * K / 1e12, "TOPS", ipk["burst"]
         out["whole_tiles"] = bool(args.whole_tiles)
     elif args.kernel == "norm":
         M, K = shape
@@ -738,9 +1021,6 @@ def run_kernel(args):
         N, K = shape
         eb = 4 if args.dtype == "fp32" else 2
         work, unit, peak = ((eb + 1.0) * N * K + 4 * N) / 1e9, "GB/s", pk["hbm_gbs"]
-    elif args.kernel == "llmint8":
-        M, K, N = shape
-        work, unit, peak = 2.0 * M * N * K / 1e12, "TOPS", 2.0 * pk["bf16_tflops"]
     else:
         raise SystemExit(f"unknown kernel {args.kernel}")
     fns = [make(i) for i in range(max(args.sets, 1))]
@@ -750,6 +1030,7 @@ def run_kernel(args):
     torch.cuda.synchronize()
     stream = torch.cuda.Stream()
     graph = torch.cuda.CUDAGraph()
+    clocks = None
     if len(fns) == 1:
         # the launches, each preceded by an L2 flush, captured in one CUDA graph
         # so host launch latency stays out of the timed intervals; the events
@@ -762,8 +1043,11 @@ def run_kernel(args):
                 a.record()
                 fns[0]()
                 b.record()
+        clocks = ClockSampler(0)
+        time.sleep(0.05)
         graph.replay()
         torch.cuda.synchronize()
+        clk = clocks.stop()
         ms = [a.elapsed_time(b) for a, b in ev]
         avg, best = sum(ms) / len(ms), min(ms)
         out["timing"] = "each launch after an L2 flush"
@@ -774,47 +1058,23 @@ def run_kernel(args):
                 for f in fns:
                     f()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        clocks = ClockSampler(0)
+        time.sleep(0.05)
         with torch.cuda.stream(stream):
             flush()
             a.record(stream)
             graph.replay()
             b.record(stream)
         torch.cuda.synchronize()
+        clk = clocks.stop()
         avg = best = a.elapsed_time(b) / n
         out["timing"] = f"{n} launches back to back over {len(fns)} input sets"
-    out.update({"avg_us": avg * 1e3, "min_us": best * 1e3, "achieved": work / (avg * 1e-3), "unit": unit,
-                "peak": peak, "frac": work / (avg * 1e-3) / peak, "peak_source": src})
+    ach = work / (avg * 1e-3)
+    out.update({"avg_us": avg * 1e3, "min_us": best * 1e3, "achieved": ach, "unit": unit,
+                "peak": peak, "frac": ach / peak, "peak_source": src, "clocks": clk})
+    if unit == "TOPS":
+        out.update({"frac_sustained": ach / ipk["sustained"], "frac_nominal": ach / ipk["nominal"]})
     print(json.dumps(out), flush=True)
-
-
-def json_line(args, world, r):
-    """The benchmark's JSON line (without the CPU baseline) from the measured
-    step: r holds the step time, the e2e time, the GEMM intervals and peaks,
-    the copy sizes and the clock record of run_ours."""
-    value = M_TOKENS * world / (r["ms_per_step"] * 1e-3)
-    e2e = M_TOKENS * world / (r["e2e_ms"] * 1e-3)
-    gemm_avg_s = sum(r["gemm_avg_ms"]) * 1e-3
-    gemm_ops = sum(2.0 * m * n * k for (m, n, k) in GEMMS[:4])
-    achieved = gemm_ops / gemm_avg_s / 1e12
-    traffic = gemm_traffic()
-    line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": r["ms_per_step"], "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "i8", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "tokens": M_TOKENS, "hidden": HIDDEN, "parallelism": f"replicas x{world}",
-                   "l2": "flushed before every timed step (256 MB write + 256 MB read, outside the timed interval)",
-                   "graph": "one CUDA graph per step"},
-        "gemm_tops": r["gemm_tops"], "gemm_avg_us": [x * 1e3 for x in r["gemm_avg_ms"]],
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": r["i8_peak"], "unit": "TOPS",
-                     "frac": achieved / r["i8_peak"], "traffic": traffic,
-                     "kernel": "gemm_w8a8_kernel", "peak_source": f"{r['peak_src']} bf16 burst x 2 (int8 nominal ratio)",
-                     "timing": f"CUDA events around each GEMM of an instrumented copy of the step's graph, "
-                               f"{r['gemm_timed_steps']} replays after the timed region, L2 flushed before each"},
-        "e2e": {"value": e2e, "unit": "tokens/s", "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
-        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
-        "clocks": r["clocks"],
-    }
-    return line
 
 
 def main():
@@ -826,11 +1086,14 @@ def main():
     ap.add_argument("--act", default="swiglu", help="--kernel act: swiglu|relu")
     ap.add_argument("--whole-tiles", action="store_true", help="--kernel gemm: a workspace without stream-K scratch")
     ap.add_argument("--sets", type=int, default=1, help="--kernel: input sets cycled back to back (1: flush each)")
+    ap.add_argument("--workload", default=HEADLINE, choices=sorted(CONFIGS), help="the headline stack")
+    ap.add_argument("--configs", default="c2,c3,c4", help="other stacks timed and reported under 'configs'")
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--cpu-rows", type=int, default=256, help="token rows of the CPU baseline sample")
+    ap.add_argument("--cpu-rows", type=int, default=64, help="token rows of the CPU baseline sample")
+    ap.add_argument("--cpu-wfrac", type=float, default=1 / 16, help="fraction of weight channels in the CPU sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.kernel:
@@ -858,15 +1121,14 @@ def main():
         torch.cuda.set_device(dev)
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
         dist.barrier()
-    r = run_ours(args, rank, world, dev)
+    line = run_ours(args, rank, world, dev)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     if rank != 0:
         return
-    line = json_line(args, world, r)
     if not args.no_cpu_baseline and world == 1:
-        line["cpu_baseline"] = {k: v for k, v in cpu_baseline(args.cpu_rows).items() if k != "step_s"}
+        line["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_rows, args.cpu_wfrac)
     print(json.dumps(line), flush=True)
 
 

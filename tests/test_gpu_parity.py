@@ -15,6 +15,7 @@ import torch
 import oracle
 import w8a8_post_quantization_sq_b200 as sq
 from w8a8_post_quantization_sq_b200 import inputs
+from parity_helpers import assert_close_16, assert_close_f32, npf, npu16, ord16, ulp16  # noqa: F401
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -26,46 +27,6 @@ def _setup():
         pytest.skip("no CUDA device")
     sq.lib()
     oracle.lib()
-
-
-def npf(t):
-    return t.detach().to("cpu", torch.float32).numpy()
-
-
-def npu16(t):
-    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
-
-
-def ord16(bits):
-    b = bits.astype(np.int64)
-    return np.where(b & 0x8000, -(b & 0x7FFF), b)
-
-
-def ulp16(bits, dtype):
-    """Spacing of the 16-bit grid at each value (bits of a finite value)."""
-    v = torch.from_numpy(bits.view(np.int16)).view(dtype).double().numpy()
-    nxt = torch.from_numpy((bits.astype(np.int32) + 1).astype(np.uint16).view(np.int16)).view(dtype).double().numpy()
-    return np.abs(nxt - v)
-
-
-def assert_close_16(got, y, dtype, terms=None):
-    """got: torch 16-bit tensor; y: oracle fp64; terms: sum of |terms| (fp64)."""
-    gb = npu16(got)
-    rb = oracle.round_bf16_bits(y) if dtype == torch.bfloat16 else oracle.round_fp16_bits(y)
-    d = np.abs(ord16(gb) - ord16(rb))
-    ok = d <= 1
-    if terms is not None:
-        g = npf(got).astype(np.float64)
-        ok |= np.abs(g - y) <= ulp16(rb, dtype) + 2.0 ** -20 * terms
-    bad = np.argwhere(~ok)
-    assert bad.size == 0, f"{bad.shape[0]} outputs beyond tolerance, first {bad[:5].tolist()} d={d[~ok][:5]}"
-
-
-def assert_close_f32(got, y, terms):
-    g = npf(got).astype(np.float64)
-    err = np.abs(g - y)
-    bad = err > 1e-6 * terms
-    assert not bad.any(), f"max rel {np.max(err / np.maximum(terms, 1e-300))}"
 
 
 def rnd(shape, seed, dtype=torch.float32, scale=1.0):
@@ -895,12 +856,13 @@ def test_bmm_attention(out_dtype):
 
 
 # ---------------------------------------------------------------- the benchmark's whole step
-def test_bench_step_against_oracle():
-    """The benchmark's step (every row, on its streams, captured in a CUDA
-    graph) against the oracle on the same inputs: the weight side in full, the
-    token side on sampled rows. Stages after a 16-bit GEMM output take the
-    device's output as their input, so each stage is held to its own bar."""
-    import bench
+def test_every_row_step_against_oracle():
+    """The Qwen3-0.6B-shaped layer with every row in one step (on its streams,
+    captured in a CUDA graph) against the oracle on the same inputs: the
+    weight side in full, the token side on sampled rows. Stages after a 16-bit
+    GEMM output take the device's output as their input, so each stage is held
+    to its own bar."""
+    import c2_every_row as bench
 
     dev = torch.device(DEV, 0)
     L = bench.Layer(dev)

@@ -23,6 +23,8 @@ same device type. Large weights are drawn on the GPU when one is given.
 """
 from __future__ import annotations
 
+import math
+
 import torch
 
 
@@ -94,7 +96,38 @@ def c2_qwen3_06b(device="cpu", M=2048):
     }
 
 
-def c3_opt30b(device="cpu", M=1024, n_calib=8):
+def _weights(spec, device, std, dtype, w_frac):
+    """Weights [N, K] ~N(0, std) per name; with w_frac < 1 only the first
+    ceil(N * w_frac) output rows are drawn (a sample of the output channels)."""
+    w = {}
+    for name, (N, K, seed) in spec.items():
+        n = N if w_frac >= 1 else max(1, math.ceil(N * w_frac))
+        w[name] = randn((n, K), seed, device, std=std, dtype=dtype)
+    return w
+
+
+def c2_block(device="cpu", M=2048, w_frac=1.0):
+    """The Qwen3-0.6B-shaped layer of ``c2_qwen3_06b`` in the block layout the
+    linear-stack benchmark uses: the attention and MLP sides' pre-norm inputs,
+    one calibration batch, per-side gamma (RMSNorm, no beta), the four weights
+    and the synthetic int8 inputs of o_proj and down_proj."""
+    d = c2_qwen3_06b(device=device, M=M)
+    W = d["W"]
+    if w_frac < 1:
+        W = {k: v[: max(1, math.ceil(v.shape[0] * w_frac))].contiguous() for k, v in W.items()}
+    return {
+        "h": {"attn": d["h_attn"], "mlp": d["h_mlp"]}, "calib": [d["h_calib"]],
+        "gamma": {"attn": d["gamma_attn"], "mlp": d["gamma_mlp"]}, "beta": {"attn": None, "mlp": None},
+        "eps": d["eps"], "W": W, "syn": {"o": d["o_in"], "down": d["down_in"]},
+        "outlier_channels": d["outlier_channels"],
+    }
+
+
+def c3_opt30b(device="cpu", M=1024, n_calib=8, w_frac=1.0):
+    """OPT-30B decoder linear stack at 4 x 256 tokens: fp16 pre-norm inputs of
+    the attention and MLP sides (7 channels, 0.1% of 7168, x60), 8 calibration
+    batches of the same kind, one LayerNorm gamma/beta, fp16 weights
+    ~N(0, 0.02) and per-tensor synthetic int8 inputs of out and FC2."""
     K = 7168
     ch = outlier_channels(K, 7, 4321)
 
@@ -106,16 +139,14 @@ def c3_opt30b(device="cpu", M=1024, n_calib=8):
     g = _gen(9, device)
     gamma = 1.0 + 0.1 * torch.randn((K,), generator=g, device=device)
     beta = 0.1 * torch.randn((K,), generator=g, device=device)
-    w = {}
-    for i, (name, shape) in enumerate([("qkv", (21504, 7168)), ("out", (7168, 7168)),
-                                       ("fc1", (28672, 7168)), ("fc2", (7168, 28672))]):
-        w[name] = randn(shape, 300 + i, device, std=0.02, dtype=torch.float16)
-    xo, so = synthetic_int8(M, 7168, 400, device)
+    w = _weights({"qkv": (21504, K, 300), "out": (K, K, 301), "fc1": (28672, K, 302), "fc2": (K, 28672, 303)},
+                 device, 0.02, torch.float16, w_frac)
+    xo, so = synthetic_int8(M, K, 400, device)
     xf, sf = synthetic_int8(M, 28672, 401, device)
     return {
-        "h": act(0), "calib": [act(s) for s in range(1, n_calib + 1)],
-        "gamma": gamma, "beta": beta, "eps": 1e-5, "W": w,
-        "out_in": (xo, so[:1]), "fc2_in": (xf, sf[:1]), "alpha": 0.5,
+        "h": {"attn": act(0), "mlp": act(9)}, "calib": [act(s) for s in range(1, n_calib + 1)],
+        "gamma": {"attn": gamma, "mlp": gamma}, "beta": {"attn": beta, "mlp": beta}, "eps": 1e-5, "W": w,
+        "syn": {"out": (xo, so[:1].contiguous()), "fc2": (xf, sf[:1].contiguous())},
         "outlier_channels": ch,
     }
 
@@ -140,7 +171,12 @@ def c4_llmint8(device="cpu", M=2048, K=4096, N=16384, n_out=6, seed=0):
     return {"X": X.to(torch.float16).to(device), "W": W, "dims": dims, "threshold": 6.0}
 
 
-def c5_175b(device="cpu", M=4096, n_calib=16, with_weights=True):
+def c5_175b(device="cpu", M=4096, n_calib=16, w_frac=1.0):
+    """175B-class block, hidden 12288, at M tokens: n_calib calibration batches
+    of linear inputs (bf16 [M, 12288] ~N(0,1), 8 channels x100), the attention
+    and MLP sides' pre-norm inputs with the same outlier channels, one
+    LayerNorm gamma/beta, fp32 weights ~N(0, 0.01) (QKV, out, FC1, FC2) and
+    per-token synthetic int8 inputs of out and FC2."""
     K = 12288
     ch = outlier_channels(K, 8, 5555)
 
@@ -149,11 +185,15 @@ def c5_175b(device="cpu", M=4096, n_calib=16, with_weights=True):
         h[:, ch] *= 100.0
         return h.to(torch.bfloat16)
 
-    out = {"calib_seeds": list(range(100, 100 + n_calib)), "act": act,
-           "alphas": (0.4, 0.5, 0.6), "outlier_channels": ch}
-    if with_weights:
-        out["W_shapes"] = {"qkv": (36864, 12288), "out": (12288, 12288),
-                           "fc1": (49152, 12288), "fc2": (12288, 49152)}
-        out["W_seeds"] = {"qkv": 500, "out": 501, "fc1": 502, "fc2": 503}
-        out["W_std"] = 0.01
-    return out
+    g = _gen(11, device)
+    gamma = 1.0 + 0.1 * torch.randn((K,), generator=g, device=device)
+    beta = 0.1 * torch.randn((K,), generator=g, device=device)
+    w = _weights({"qkv": (36864, K, 500), "out": (K, K, 501), "fc1": (49152, K, 502), "fc2": (K, 49152, 503)},
+                 device, 0.01, torch.float32, w_frac)
+    xo, so = synthetic_int8(M, K, 600, device)
+    xf, sf = synthetic_int8(M, 49152, 601, device)
+    return {
+        "h": {"attn": act(200), "mlp": act(201)}, "calib": [act(s) for s in range(100, 100 + n_calib)],
+        "gamma": {"attn": gamma, "mlp": gamma}, "beta": {"attn": beta, "mlp": beta}, "eps": 1e-5, "W": w,
+        "syn": {"out": (xo, so), "fc2": (xf, sf)}, "outlier_channels": ch,
+    }
