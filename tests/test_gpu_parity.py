@@ -478,7 +478,9 @@ SK_SHAPES = [(1029, 7168, 16400), (1029, 7168, 7200), (2560, 4096, 16384), (2048
 
 
 @pytest.mark.parametrize("M,N,K", SK_SHAPES)
-def test_gemm_stream_k(M, N, K):
+def test_gemm_stream_k(M, N, K, monkeypatch):
+    # stream-K runs on single-CTA tiles: keep the plan off CTA pairs
+    monkeypatch.setenv("SQ_GEMM_CTA_PAIRS", "0")
     assert sq.sq_workspace_size(sq.SQ_OP_GEMM, M, N, K) > 256, "the plan was expected to cut this shape"
     Xq, Wq = rand_i8((M, K), M + 3), rand_i8((N, K), N + 4)
     Xd, Wd = Xq.to(DEV), Wq.to(DEV)
@@ -530,10 +532,15 @@ def test_bounded_wait_timeout():
 
 @pytest.mark.parametrize("M,N,K", [(4096, 36864, 12288), (1024, 28672, 7168), (2048, 16384, 4096),
                                    (1024, 7168, 28672)])
-def test_gemm_full_size_sampled(M, N, K):
-    """Full-size shapes in the launch configuration the benchmark times:
-    all outputs against torch._int_mm (a library cross-check, test only) and
-    sampled rows against the oracle."""
+@pytest.mark.parametrize("pairs", ["", "0"])
+def test_gemm_full_size_sampled(M, N, K, pairs, monkeypatch):
+    """Full-size shapes in the launch configuration the benchmark times (and
+    on single-CTA tiles): all outputs against torch._int_mm (a library
+    cross-check, test only) and sampled rows against the oracle."""
+    if pairs:
+        monkeypatch.setenv("SQ_GEMM_CTA_PAIRS", pairs)
+    else:
+        monkeypatch.delenv("SQ_GEMM_CTA_PAIRS", raising=False)
     g = torch.Generator(device=DEV).manual_seed(M + N)
     Xq = torch.randint(-127, 128, (M, K), generator=g, device=DEV, dtype=torch.int8)
     Wq = torch.randint(-127, 128, (N, K), generator=g, device=DEV, dtype=torch.int8)

@@ -42,6 +42,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <cstdlib>
+
 #include "sq_common.cuh"
 #include "sq_internal.h"
 #include "sq_wait.cuh"
@@ -52,7 +54,6 @@ namespace {
 constexpr int BM = 128;
 constexpr int BK = 128;  // one 128-byte swizzle row of int8
 constexpr int UMMA_K = 32;
-constexpr int STAGES = 4;
 constexpr int kEpiWarps = 8;  // two per TMEM lane quarter, each on half the tile's columns
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
@@ -63,10 +64,16 @@ enum OutKind { kOutBF16 = 0, kOutF16 = 1, kOutF32 = 2, kOutI32 = 3 };
 // operand formats: int8 x int8 -> int32, or FP8 E4M3 x E4M3 -> fp32
 enum MmaKind { kKindI8 = 0, kKindF8 = 1 };
 
-template <int BN>
+// CG = 1: one CTA computes a 128 x BN tile with cta_group::1 MMAs.
+// CG = 2: a cluster of two CTAs computes a 256 x BN tile with cta_group::2
+// MMAs issued by CTA 0: each CTA loads its own 128 rows of Xq and its own
+// BN/2 rows of the weight tile, and holds its 128 rows x BN of the
+// accumulator, so each SM streams half as many weight bytes per MMA.
+template <int BN, int CG>
 struct Cfg {
-    static constexpr uint32_t A_BYTES = BM * BK;
-    static constexpr uint32_t B_BYTES = BN * BK;
+    static constexpr int STAGES = CG == 2 ? 6 : 4;
+    static constexpr uint32_t A_BYTES = BM * BK;         // this CTA's 128 rows of Xq
+    static constexpr uint32_t B_BYTES = (BN / CG) * BK;  // this CTA's rows of the weight tile
     static constexpr uint32_t A_OFF = 0;
     static constexpr uint32_t B_OFF = STAGES * A_BYTES;
     static constexpr uint32_t BAR_OFF = B_OFF + STAGES * B_BYTES;
@@ -84,10 +91,10 @@ struct Cfg {
     static constexpr uint32_t TMEM_COLS = 2 * BN;
     // kind::i8: D = s32 (bits 4-5 = 2), A = B = signed 8-bit (bits 7-9, 10-12 = 1);
     // kind::f8f6f4: D = f32 (bits 4-5 = 1), A = B = E4M3 (format 0);
-    // both K-major, N >> 3 at bit 17, M >> 4 at bit 24
+    // both K-major, N >> 3 at bit 17, M >> 4 at bit 24 (M = 256 for a CTA pair)
     static constexpr uint32_t idesc(int kind) {
         return (kind == kKindF8 ? (1u << 4) : ((2u << 4) | (1u << 7) | (1u << 10))) |
-               ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+               ((uint32_t)(BN >> 3) << 17) | ((uint32_t)((BM * CG) >> 4) << 24);
     }
 };
 
@@ -124,13 +131,15 @@ __device__ __forceinline__ int sk_owner(int x, const Params& p) {
 // then its whole tiles, so the parking of partial sums and the fix-up
 // epilogues overlap the whole tiles' MMAs instead of trailing the launch.
 // slot = -1 for a whole tile; a piece is the CTA's first (slot 0) or last
-// (slot 1) piece: a range spans at most one whole tile between them.
-template <bool SK>
+// (slot 1) piece: a range spans at most one whole tile between them. A CTA
+// pair (CG = 2) walks the tiles as one unit: both CTAs see the same sequence.
+template <bool SK, int CG>
 struct Segments {
+    static_assert(!(SK && CG == 2), "stream-K runs on single-CTA tiles only");
     int tile_dp, it, end;
     bool first;
     __device__ explicit Segments(const Params& p) {
-        tile_dp = blockIdx.x;
+        tile_dp = blockIdx.x / CG;
         it = SK ? sk_start(blockIdx.x, p) : 0;
         end = SK ? sk_start(blockIdx.x + 1, p) : 0;
         first = true;
@@ -150,7 +159,7 @@ struct Segments {
         k0 = 0;
         k1 = p.num_kb;
         slot = -1;
-        tile_dp += gridDim.x;
+        tile_dp += gridDim.x / CG;
         return tile < (SK ? p.dp_tiles : num_tiles);
     }
 };
@@ -158,22 +167,22 @@ struct Segments {
 // Raster: groups of group_m m-blocks; inside a group, n-major then m. The
 // CTAs running together then share the group's rows of Xq (kept in L2) and a
 // few weight tiles, and each weight tile is fetched once per group.
-__device__ __forceinline__ void tile_coords(int tile, const Params& p, int bn, int& m0, int& n0) {
+__device__ __forceinline__ void tile_coords(int tile, const Params& p, int bm, int bn, int& m0, int& n0) {
     const int per_group = p.group_m * p.num_n;
     const int g = tile / per_group;
     const int r = tile - g * per_group;
     const int gm0 = g * p.group_m;
     const int gsize = min(p.group_m, p.num_m - gm0);
     const int nb = r / gsize;
-    m0 = (gm0 + (r - nb * gsize)) * BM;
+    m0 = (gm0 + (r - nb * gsize)) * bm;
     n0 = nb * bn;
 }
 
 // Batched problems: tile t of problem b = t / (num_m * num_n).
-__device__ __forceinline__ void tile_coords_b(int tile, const Params& p, int bn, int& b, int& m0, int& n0) {
+__device__ __forceinline__ void tile_coords_b(int tile, const Params& p, int bm, int bn, int& b, int& m0, int& n0) {
     const int tpb = p.num_m * p.num_n;
     b = tile / tpb;
-    tile_coords(tile - b * tpb, p, bn, m0, n0);
+    tile_coords(tile - b * tpb, p, bm, bn, m0, n0);
 }
 
 // ---------------------------------------------------------------- PTX helpers
@@ -194,12 +203,48 @@ __device__ __noinline__ void wait_drain(uint32_t bar, uint32_t parity) {
         if (global_ns() - t0 > kTimeoutNs / 4) return;
 }
 
-// Tile (x = k, y = row) of problem z of a 3-D [batch, rows, K] int8 tensor.
+// Tile (x = k, y = row) of problem z of a 3-D [batch, rows, K] int8 tensor
+// into this CTA's shared memory. CG = 2: the completion is counted on the
+// mbarrier `bar` names in the shared::cluster window, which may be the other
+// CTA's of the pair (no multicast: each CTA loads only its own tile).
+template <int CG>
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y, int z) {
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];"
-        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
-        : "memory");
+    if constexpr (CG == 2) {
+        asm volatile(
+            "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+            "[%0], [%1, {%3, %4, %5}], [%2];"
+            ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
+            : "memory");
+    } else {
+        asm volatile(
+            "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+            "[%0], [%1, {%3, %4, %5}], [%2];"
+            ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
+            : "memory");
+    }
+}
+
+// ---------------------------------------------------------------- CTA pairs
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// The shared::cluster address of this CTA's shared-memory location `a` in
+// CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t a, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
+    return r;
+}
+// Every thread of both CTAs arrives, then waits (aligned: whole warps).
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Arrive on an mbarrier given by its shared::cluster address (possibly the
+// other CTA's), releasing this thread's prior accesses at cluster scope.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 // UMMA shared-memory descriptor, K-major operand with 128-byte swizzle: rows of
@@ -213,9 +258,21 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr) {
     return d;
 }
 
-template <int KIND>
+template <int KIND, int CG>
 __device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-    if constexpr (KIND == kKindF8) {
+    if constexpr (CG == 2 && KIND == kKindF8) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
+            ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(acc));
+    } else if constexpr (CG == 2) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}"
+            ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(acc));
+    } else if constexpr (KIND == kKindF8) {
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
             "setp.ne.b32 p, %4, 0;\n\t"
@@ -229,9 +286,19 @@ __device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t a, uint64_t b, ui
             ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(acc));
     }
 }
-__device__ __forceinline__ void umma_commit(uint32_t bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-                 : "memory");
+// Arrive on `bar` once every MMA this thread has issued completes. CG = 2:
+// on the mbarrier at the same shared-memory offset in each CTA of `mask`.
+template <int CG>
+__device__ __forceinline__ void umma_commit(uint32_t bar, uint16_t mask = 3) {
+    if constexpr (CG == 2) {
+        asm volatile(
+            "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+            ::"r"(bar), "h"(mask)
+            : "memory");
+    } else {
+        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                     : "memory");
+    }
 }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -436,11 +503,12 @@ __device__ __forceinline__ void epi_chunk(const Params& p, const uint32_t* r, in
     }
 }
 
-template <int BN, int OUT, bool OUTL, int KIND, bool SK>
+template <int BN, int OUT, bool OUTL, int KIND, bool SK, int CG>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                  const Params p) {
-    using C = Cfg<BN>;
+    using C = Cfg<BN, CG>;
+    constexpr int STAGES = C::STAGES;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
@@ -455,6 +523,9 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
     float* rw_s = reinterpret_cast<float*>(smem + C::RW_OFF);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // CTA pair: CTA 0 issues the MMAs for both; its stage-full and
+    // accumulator-empty barriers count both CTAs' loads and epilogue warps
+    const uint32_t rank = CG == 2 ? cluster_rank() : 0u;
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(full_bar(s), 1);
@@ -462,7 +533,7 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(tfull_bar(a), 1);
-            mbar_init(tempty_bar(a), kEpiWarps);
+            mbar_init(tempty_bar(a), kEpiWarps * CG);
         }
         mbar_init(drain_bar, 1);
         *abort_flag = 0;
@@ -470,9 +541,16 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
     if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_holder)),
-                     "r"(C::TMEM_COLS));
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+        // a CTA pair allocates the same columns in both CTAs (one warp of each)
+        if constexpr (CG == 2) {
+            asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+                         ::"r"(smem_u32(tmem_holder)), "r"(C::TMEM_COLS));
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+        } else {
+            asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                         ::"r"(smem_u32(tmem_holder)), "r"(C::TMEM_COLS));
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+        }
     }
     if (warp == 0 && lane == 0) {
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_a)) : "memory");
@@ -482,6 +560,8 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
     __syncwarp();
     tc_fence_before();
     __syncthreads();
+    // a pair: neither CTA signals the other's barriers before both are initialised
+    if constexpr (CG == 2) cluster_sync_all();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
     // the set-up above touches only this CTA's shared and tensor memory; wait
@@ -499,38 +579,46 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
             bool issued[STAGES];
             for (int s = 0; s < STAGES; ++s) issued[s] = false, issued_phase[s] = 0;
             bool ok = true;
-            Segments<SK> seg(p);
+            Segments<SK, CG> seg(p);
             int tile, k0, k1, slot;
             while (ok && seg.next(p, num_tiles, tile, k0, k1, slot)) {
                 int b, m0, n0;
-                tile_coords_b(tile, p, BN, b, m0, n0);
+                tile_coords_b(tile, p, BM * CG, BN, b, m0, n0);
+                // this CTA's rows: of a pair, CTA r loads Xq rows m0 + 128 r and
+                // weight rows n0 + (BN / 2) r
+                m0 += (int)rank * BM;
+                n0 += (int)rank * (BN / CG);
                 for (int kb = k0; kb < k1; ++kb) {
                     if (!wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, p.status, 0x6E1)) {
                         ok = false;
                         break;
                     }
-                    mbar_expect_tx(full_bar(stage), C::A_BYTES + C::B_BYTES);
-                    tma_load_3d(sbase + C::A_OFF + stage * C::A_BYTES, &tmap_a, full_bar(stage), kb * BK, m0, b);
-                    tma_load_3d(sbase + C::B_OFF + stage * C::B_BYTES, &tmap_b, full_bar(stage), kb * BK, n0, b);
+                    // the pair's loads all count on CTA 0's barrier, which expects both
+                    const uint32_t fb = CG == 2 ? map_to_rank(full_bar(stage), 0) : full_bar(stage);
+                    if (rank == 0) mbar_expect_tx(full_bar(stage), CG * (C::A_BYTES + C::B_BYTES));
+                    tma_load_3d<CG>(sbase + C::A_OFF + stage * C::A_BYTES, &tmap_a, fb, kb * BK, m0, b);
+                    tma_load_3d<CG>(sbase + C::B_OFF + stage * C::B_BYTES, &tmap_b, fb, kb * BK, n0, b);
                     issued[stage] = true;
                     issued_phase[stage] = phase;
                     if (++stage == STAGES) stage = 0, phase ^= 1u;
                 }
             }
-            if (!ok) {
+            if (!ok && rank == 0) {
                 // make sure no copy still lands in shared memory after we leave
+                // (of a pair, CTA 0's barriers count both CTAs' copies, and both
+                // CTAs stay resident until the pair's closing cluster barrier)
                 for (int s = 0; s < STAGES; ++s)
                     if (issued[s]) wait_drain(full_bar(s), issued_phase[s]);
             }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
+        if (lane == 0 && rank == 0) {
             // ---------------------------------------------------- MMA issuer
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
             int local = 0;
-            Segments<SK> seg(p);
+            Segments<SK, CG> seg(p);
             int tile, k0, k1, slot;
             for (; ok && seg.next(p, num_tiles, tile, k0, k1, slot); ++local) {
                 const int acc = local & 1;
@@ -551,16 +639,16 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
                     const uint32_t b_addr = sbase + C::B_OFF + stage * C::B_BYTES;
 #pragma unroll
                     for (int k = 0; k < BK / UMMA_K; ++k)
-                        umma<KIND>(d_tmem, sdesc(a_addr + k * UMMA_K), sdesc(b_addr + k * UMMA_K), C::idesc(KIND),
-                                (kb != k0 || k != 0) ? 1u : 0u);
-                    umma_commit(empty_bar(stage));
+                        umma<KIND, CG>(d_tmem, sdesc(a_addr + k * UMMA_K), sdesc(b_addr + k * UMMA_K),
+                                       C::idesc(KIND), (kb != k0 || k != 0) ? 1u : 0u);
+                    umma_commit<CG>(empty_bar(stage));  // both CTAs' stage is free
                     if (++stage == STAGES) stage = 0, phase ^= 1u;
                 }
                 if (!ok) break;
-                umma_commit(tfull_bar(acc));
+                umma_commit<CG>(tfull_bar(acc));  // both CTAs' epilogues may read
             }
             // all MMAs issued by this thread complete before tensor memory is freed
-            umma_commit(drain_bar);
+            umma_commit<CG>(drain_bar, 1);
             wait_drain(drain_bar, 0);
         }
     } else {
@@ -581,11 +669,21 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
         float* bias_w = rw_w + HC;
         uint8_t* stg = smem + C::STG_OFF + (warp - 2) * kStgWarpBytes;
         int local = 0;
-        Segments<SK> seg(p);
+        Segments<SK, CG> seg(p);
         int tile, k0, k1, slot;
+        // the accumulator buffer is released on CTA 0's barrier for a pair
+        auto release_acc = [&](int a) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                if constexpr (CG == 2) mbar_arrive_cluster(map_to_rank(tempty_bar(a), 0));
+                else mbar_arrive(tempty_bar(a));
+            }
+        };
         for (; seg.next(p, num_tiles, tile, k0, k1, slot); ++local) {
             int b, m0, n0;
-            tile_coords_b(tile, p, BN, b, m0, n0);
+            tile_coords_b(tile, p, BM * CG, BN, b, m0, n0);
+            m0 += (int)rank * BM;  // this CTA's 128 rows of the pair's tile
             const int c_base = n0 + half * HC;  // first column of this warp
             if constexpr (OUT != kOutI32) {
                 __syncwarp();
@@ -650,9 +748,7 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
                             mine[(c * 8 + e) * 32 + lane] = make_int4((int)ra[4 * e], (int)ra[4 * e + 1],
                                                                       (int)ra[4 * e + 2], (int)ra[4 * e + 3]);
                     }
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(tempty_bar(acc));  // accumulator read in full
+                    release_acc(acc);  // accumulator read in full
                     __threadfence();
                     __syncwarp();
                     const int u = tile - p.dp_tiles;
@@ -698,9 +794,7 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
                     const bool more = c + 1 < nch;
                     if (more) tmem_ld32_async(t_row + (uint32_t)((c + 1) * 32), rb);
                     else {
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(tempty_bar(acc));  // accumulator read in full
+                        release_acc(acc);  // accumulator read in full
                     }
                     epi_chunk<OUT, OUTL, KIND>(p, ra, c * 32, c_base + c * 32, row0, row, row_ok, rx, rw_w, bias_w, stg,
                                          lane, n_out, compact, b);
@@ -709,9 +803,7 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
                     const bool more2 = c + 2 < nch;
                     if (more2) tmem_ld32_async(t_row + (uint32_t)((c + 2) * 32), ra);
                     else {
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(tempty_bar(acc));
+                        release_acc(acc);
                     }
                     epi_chunk<OUT, OUTL, KIND>(p, rb, (c + 1) * 32, c_base + (c + 1) * 32, row0, row, row_ok, rx, rw_w,
                                          bias_w, stg, lane, n_out, compact, b);
@@ -721,18 +813,14 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
                 for (int c = 0; c < nch; ++c) {
                     tmem_ld32(t_row + (uint32_t)(c * 32), ra);
                     if (c + 1 == nch) {
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(tempty_bar(acc));  // accumulator read in full
+                        release_acc(acc);  // accumulator read in full
                     }
                     epi_chunk<OUT, OUTL, KIND>(p, ra, c * 32, c_base + c * 32, row0, row, row_ok, rx, rw_w, bias_w, stg,
                                          lane, n_out, compact, b);
                 }
             }
             if (nch == 0) {
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(tempty_bar(acc));
+                release_acc(acc);
             }
         }
     }
@@ -744,9 +832,15 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
     __syncwarp();
     tc_fence_before();
     __syncthreads();
+    // a pair: CTA 0's MMAs write both CTAs' tensor memory, so neither frees it
+    // before both have finished (CTA 0's issuer waited for its last MMA)
+    if constexpr (CG == 2) cluster_sync_all();
     if (warp == 1) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(C::TMEM_COLS));
+        if constexpr (CG == 2)
+            asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(C::TMEM_COLS));
+        else
+            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(C::TMEM_COLS));
     }
 }
 
@@ -781,44 +875,89 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t K, int box
 
 using KernelFn = void (*)(const CUtensorMap, const CUtensorMap, const Params);
 
-template <int BN, bool SK>
+template <int BN, bool SK, int CG>
 KernelFn pick_kernel_sk(sq_dtype_t out_dt, bool outl, int kind) {
     if (kind == kKindF8) {
         switch (out_dt) {
-            case SQ_BF16: return gemm_w8a8_kernel<BN, kOutBF16, false, kKindF8, SK>;
-            case SQ_F16: return gemm_w8a8_kernel<BN, kOutF16, false, kKindF8, SK>;
-            default: return gemm_w8a8_kernel<BN, kOutF32, false, kKindF8, SK>;
+            case SQ_BF16: return gemm_w8a8_kernel<BN, kOutBF16, false, kKindF8, SK, CG>;
+            case SQ_F16: return gemm_w8a8_kernel<BN, kOutF16, false, kKindF8, SK, CG>;
+            default: return gemm_w8a8_kernel<BN, kOutF32, false, kKindF8, SK, CG>;
         }
     }
     switch (out_dt) {
         case SQ_BF16:
-            return outl ? gemm_w8a8_kernel<BN, kOutBF16, true, kKindI8, SK>
-                        : gemm_w8a8_kernel<BN, kOutBF16, false, kKindI8, SK>;
+            return outl ? gemm_w8a8_kernel<BN, kOutBF16, true, kKindI8, SK, CG>
+                        : gemm_w8a8_kernel<BN, kOutBF16, false, kKindI8, SK, CG>;
         case SQ_F16:
-            return outl ? gemm_w8a8_kernel<BN, kOutF16, true, kKindI8, SK>
-                        : gemm_w8a8_kernel<BN, kOutF16, false, kKindI8, SK>;
-        case SQ_F32: return gemm_w8a8_kernel<BN, kOutF32, false, kKindI8, SK>;
-        default: return gemm_w8a8_kernel<BN, kOutI32, false, kKindI8, SK>;
+            return outl ? gemm_w8a8_kernel<BN, kOutF16, true, kKindI8, SK, CG>
+                        : gemm_w8a8_kernel<BN, kOutF16, false, kKindI8, SK, CG>;
+        case SQ_F32: return gemm_w8a8_kernel<BN, kOutF32, false, kKindI8, SK, CG>;
+        default: return gemm_w8a8_kernel<BN, kOutI32, false, kKindI8, SK, CG>;
     }
 }
 
-template <int BN>
+template <int BN, int CG>
 KernelFn pick_kernel(sq_dtype_t out_dt, bool outl, int kind, bool sk) {
-    return sk ? pick_kernel_sk<BN, true>(out_dt, outl, kind) : pick_kernel_sk<BN, false>(out_dt, outl, kind);
+    if constexpr (CG == 2) return pick_kernel_sk<BN, false, 2>(out_dt, outl, kind);
+    else
+        return sk ? pick_kernel_sk<BN, true, 1>(out_dt, outl, kind) : pick_kernel_sk<BN, false, 1>(out_dt, outl, kind);
 }
 
-template <int BN>
+// CTA pairs of the pair kernel that can be resident at once on the current
+// device (0 if the device cannot run it), cached per device.
+int max_resident_pairs() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        cudaGetLastError();
+        return 0;
+    }
+    if (cache[dev] == 0) {
+        using C = Cfg<256, 2>;
+        KernelFn fn = gemm_w8a8_kernel<256, kOutBF16, false, kKindI8, false, 2>;
+        int n = 0;
+        if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM_ALLOC) ==
+            cudaSuccess) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(2 * num_sms());
+            cfg.blockDim = dim3(kThreads);
+            cfg.dynamicSmemBytes = C::SMEM_ALLOC;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = 2;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess) n = 0;
+        }
+        cudaGetLastError();
+        cache[dev] = n > 0 ? n : -1;
+    }
+    return cache[dev] > 0 ? cache[dev] : 0;
+}
+
+// SQ_GEMM_CTA_PAIRS: 0 never uses CTA pairs, 1 uses them wherever the plan
+// allows (256-wide tiles); unset leaves the choice to plan_gemm. Read on
+// every call (a few hundred nanoseconds), so a process can switch it.
+int pairs_mode() {
+    const char* e = getenv("SQ_GEMM_CTA_PAIRS");
+    return (e && e[0] == '0') ? 0 : (e && e[0] == '1') ? 1 : -1;
+}
+
+template <int BN, int CG>
 sq_status_t launch_bn(const int8_t* Xq, const int8_t* Wq, int64_t M, int64_t N, int64_t K, const GemmEpilogue& ep,
                       const GemmPlan& plan, int* status, void* sk_ws, cudaStream_t stream) {
-    using C = Cfg<BN>;
+    using C = Cfg<BN, CG>;
     CUtensorMap ta, tb;
-    if (!make_map(&ta, Xq, M, K, BM, ep.batch) || !make_map(&tb, Wq, N, K, BN, ep.batch))
+    // each CTA loads 128 rows of Xq and BN / CG rows of the weight per stage
+    if (!make_map(&ta, Xq, M, K, BM, ep.batch) || !make_map(&tb, Wq, N, K, BN / CG, ep.batch))
         return set_error(SQ_ERR_CUDA, "sq_gemm_w8a8: cuTensorMapEncodeTiled failed");
     const bool outl = ep.idx != nullptr;
     if (outl && ep.out_dt != SQ_BF16 && ep.out_dt != SQ_F16)
         return set_error(SQ_ERR_INVALID_ARG, "sq_gemm_w8a8: the outlier term needs a 16-bit output");
-    const bool sk = plan.sk_tiles > 0 && sk_ws != nullptr;
-    KernelFn fn = pick_kernel<BN>(ep.out_dt, outl, ep.kind, sk);
+    const bool sk = CG == 1 && plan.sk_tiles > 0 && sk_ws != nullptr;
+    KernelFn fn = pick_kernel<BN, CG>(ep.out_dt, outl, ep.kind, sk);
     // the shared-memory opt-in is per kernel and per device; it is cheap, so set it every time
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM_ALLOC) != cudaSuccess)
         return check_launch("sq_gemm_w8a8: set shared memory size");
@@ -828,11 +967,11 @@ sq_status_t launch_bn(const int8_t* Xq, const int8_t* Wq, int64_t M, int64_t N, 
     p.K = (int)K;
     p.batch = (int)ep.batch;
     p.y_bstride = ep.y_bstride;
-    p.num_m = (int)((M + BM - 1) / BM);
+    p.num_m = (int)((M + BM * CG - 1) / (BM * CG));
     p.num_n = (int)((N + BN - 1) / BN);
     p.num_kb = (int)((K + BK - 1) / BK);
     // rows of Xq per raster group kept within about 48 MB of L2
-    const int64_t per_mblock = (int64_t)BM * K;
+    const int64_t per_mblock = (int64_t)BM * CG * K;
     int64_t g = (48ll << 20) / per_mblock;
     p.group_m = (int)(g < 1 ? 1 : (g > p.num_m ? p.num_m : g));
     const int eb = (ep.out_dt == SQ_BF16 || ep.out_dt == SQ_F16) ? 2 : 4;
@@ -845,7 +984,10 @@ sq_status_t launch_bn(const int8_t* Xq, const int8_t* Wq, int64_t M, int64_t N, 
     p.sk_cnt = sk ? static_cast<int*>(sk_ws) : nullptr;
     p.sk_part = sk ? reinterpret_cast<int*>(static_cast<uint8_t*>(sk_ws) + plan.sk_cnt_bytes) : nullptr;
     const int grid = plan.grid;
-    launch_pdl(fn, dim3(grid), dim3(kThreads), C::SMEM_ALLOC, stream, ta, tb, p);
+    if constexpr (CG == 2)
+        launch_pdl_cluster(fn, dim3(grid), dim3(kThreads), C::SMEM_ALLOC, stream, 2, ta, tb, p);
+    else
+        launch_pdl(fn, dim3(grid), dim3(kThreads), C::SMEM_ALLOC, stream, ta, tb, p);
     return check_launch("sq_gemm_w8a8");
 }
 
@@ -879,6 +1021,25 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int64_t batch) {
         pl.sk_cnt_bytes = ((size_t)rem * kEpiWarps * sizeof(int) + 255) / 256 * 256;
         pl.sk_bytes = pl.sk_cnt_bytes + (size_t)pl.grid * 2 * BM * pl.bn * sizeof(int);
     }
+    // CTA pairs (256 x 256 tiles, cta_group::2: each SM streams half the
+    // weight bytes per MMA) where there are two waves of them or more and the
+    // single-CTA plan has no stream-K split of a ragged last wave. Measured
+    // on B200 (us, single CTA -> pairs): 4096 x 36864 x 12288 1285 -> 1252,
+    // 4096 x 49152 x 12288 1697 -> 1653, 1024 x 21504 x 7168 127 -> 122,
+    // 2048 x 16384 x 4096 105 -> 104; the shapes with a split are faster
+    // without pairs (1024 x 7168 x 28672: 159 split, 177 on pairs).
+    if (pl.bn == 256 && pairs_mode() != 0 && (pl.sk_tiles == 0 || pairs_mode() == 1)) {
+        const int pairs = max_resident_pairs();
+        const int64_t ptiles = batch * ((M + 2 * BM - 1) / (2 * BM)) * ((N + 255) / 256);
+        if (pairs > 0 && ptiles < (1ll << 31) && (pairs_mode() == 1 || ptiles >= 2ll * pairs)) {
+            GemmPlan pp;
+            pp.bn = 256;
+            pp.cg = 2;
+            pp.tiles = (int)ptiles;
+            pp.grid = 2 * (int)(ptiles < pairs ? ptiles : pairs);
+            return pp;
+        }
+    }
     return pl;
 }
 
@@ -894,8 +1055,9 @@ sq_status_t launch_gemm_w8a8(const int8_t* Xq, const int8_t* Wq, int64_t M, int6
     void* sk_ws = (pl.sk_tiles > 0 && ws_bytes >= kStatusBytes + pl.sk_bytes)
                       ? static_cast<void*>(reinterpret_cast<uint8_t*>(status_word) + kStatusBytes)
                       : nullptr;
-    if (pl.bn == 128) return launch_bn<128>(Xq, Wq, M, N, K, ep, pl, status_word, sk_ws, stream);
-    return launch_bn<256>(Xq, Wq, M, N, K, ep, pl, status_word, sk_ws, stream);
+    if (pl.cg == 2) return launch_bn<256, 2>(Xq, Wq, M, N, K, ep, pl, status_word, nullptr, stream);
+    if (pl.bn == 128) return launch_bn<128, 1>(Xq, Wq, M, N, K, ep, pl, status_word, sk_ws, stream);
+    return launch_bn<256, 1>(Xq, Wq, M, N, K, ep, pl, status_word, sk_ws, stream);
 }
 
 }  // namespace sq

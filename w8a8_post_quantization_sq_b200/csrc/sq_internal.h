@@ -52,6 +52,7 @@ struct GemmEpilogue {
 // tiles are cut by k-blocks (stream-K), with the scratch that needs.
 struct GemmPlan {
     int bn = 256;
+    int cg = 1;  // 2: tiles of 256 rows on CTA pairs (cta_group::2), grid = 2 x pairs
     int tiles = 0;
     int grid = 0;
     int sk_tiles = 0;
