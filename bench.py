@@ -33,6 +33,7 @@ replica of the step on its own GPU (no data-path collective; weak scaling).
 from __future__ import annotations
 
 import argparse
+import contextlib
 import json
 import math
 import os
@@ -291,15 +292,28 @@ class Stack:
         self.ws = {w: sq.workspace(sq.SQ_OP_GEMM, M, self.W[w].shape[0], self.W[w].shape[1], device=dev)
                    for w, _ in cfg["gemms"]}
         self.bank = None
+        self.by_phase = False  # with a bank: events around each phase of the offline pass, not each launch
 
-    # one launch, bracketed by events when a bank is attached
+    # one launch, bracketed by events when a bank is attached (per launch)
     def launch(self, tag, work, fn, *a):
-        if self.bank is None:
+        if self.bank is None or self.by_phase:
             fn(*a)
             return
         e0, e1 = self.bank.pair(tag, work)
         e0.record()
         fn(*a)
+        e1.record()
+
+    @contextlib.contextmanager
+    def phase(self, tag, work):
+        """A group of launches timed as one (events before the first and after
+        the last) when a bank is attached in phase mode."""
+        if self.bank is None or not self.by_phase:
+            yield
+            return
+        e0, e1 = self.bank.pair(tag, work)
+        e0.record()
+        yield
         e1.record()
 
     def gemm_shapes(self):
@@ -309,40 +323,70 @@ class Stack:
         """Calibration, weight maxima, smoothing factors for every alpha (gamma
         and beta folded for the deployed one), static per-tensor scales where
         the configuration uses them, and the int8 weights."""
-        sq, d, M, K = self.sq, self.d, self.M, self.K
+        sq, d = self.sq, self.d
         L = self.launch
         eps = d["eps"]
         self.cal.zero_()
-        for X in d["calib"]:
-            if self.cfg["calib"] == "absmax":
-                L("calib_absmax", ("hbm", X.numel() * esize(X)), sq.sq_calib_absmax, X, self.xmax["attn"])
-            else:
-                for k in self.sides:
-                    L("calib_norm", ("hbm", X.numel() * esize(X)), sq.sq_norm_smooth_quant, X, self.norm,
-                      self.gamma[k], self.beta[k], eps, True, None, None, None, self.xmax[k])
-        for k in self.sides:
-            W = self.W[self.consumer[k]]
-            L("weight_absmax", ("hbm", W.numel() * esize(W)), sq.sq_weight_absmax, W, self.wmax[k])
-        for a in self.alphas:
+        cb = sum(X.numel() * esize(X) for X in d["calib"])
+        if self.cfg["calib"] == "absmax":
+            with self.phase("calib_absmax", ("hbm", cb)):
+                for X in d["calib"]:
+                    L("calib_absmax", ("hbm", X.numel() * esize(X)), sq.sq_calib_absmax, X, self.xmax["attn"])
+        else:
+            with self.phase("calib_norm", ("hbm", cb * 2)):
+                for X in d["calib"]:
+                    for k in self.sides:
+                        L("calib_norm", ("hbm", X.numel() * esize(X)), sq.sq_norm_smooth_quant, X, self.norm,
+                          self.gamma[k], self.beta[k], eps, True, None, None, None, self.xmax[k])
+        with self.phase("weight_absmax", ("hbm", sum(self.W[self.consumer[k]].numel() *
+                                                      esize(self.W[self.consumer[k]]) for k in self.sides))):
             for k in self.sides:
-                if a == self.alpha:
-                    L("smooth_fold_norm", ("latency", 0), sq.sq_smooth_fold_norm, self.xmax[k], self.wmax[k], a,
-                      self.gamma[k], self.beta[k], self.s[a][k], self.gp[k], self.bp[k])
-                else:
-                    L("smooth_scales", ("latency", 0), sq.sq_smooth_scales, self.xmax[k], self.wmax[k], a,
-                      self.s[a][k])
+                W = self.W[self.consumer[k]]
+                L("weight_absmax", ("hbm", W.numel() * esize(W)), sq.sq_weight_absmax, W, self.wmax[k])
+        with self.phase("smoothing", ("latency", 0)):
+            for a in self.alphas:
+                for k in self.sides:
+                    if a == self.alpha:
+                        L("smooth_fold_norm", ("latency", 0), sq.sq_smooth_fold_norm, self.xmax[k], self.wmax[k], a,
+                          self.gamma[k], self.beta[k], self.s[a][k], self.gp[k], self.bp[k])
+                    else:
+                        L("smooth_scales", ("latency", 0), sq.sq_smooth_scales, self.xmax[k], self.wmax[k], a,
+                          self.s[a][k])
         if not self.per_token:
-            for X in d["calib"]:
+            with self.phase("static_scales", ("hbm", cb * 2)):
+                for X in d["calib"]:
+                    for k in self.sides:
+                        L("calib_norm_smoothed", ("hbm", X.numel() * esize(X)), sq.sq_norm_smooth_quant, X,
+                          self.norm, self.gp[k], self.bp[k], eps, True, None, None, None, self.vmax[k])
                 for k in self.sides:
-                    L("calib_norm_smoothed", ("hbm", X.numel() * esize(X)), sq.sq_norm_smooth_quant, X, self.norm,
-                      self.gp[k], self.bp[k], eps, True, None, None, None, self.vmax[k])
-            for k in self.sides:
-                L("scale_from_absmax", ("latency", 0), sq.sq_scale_from_absmax, self.vmax[k], self.qs_static[k])
-        for w, src in self.cfg["gemms"]:
-            W = self.W[w]
-            s = None if src == "syn" else self.s[self.alpha][src]
-            L("quantize_weight", ("hbm", W.numel() * (esize(W) + 1) + 4 * W.shape[0]), sq.sq_quantize_weight, W, s,
-              True, self.Wq[w], self.qw[w])
+                    L("scale_from_absmax", ("latency", 0), sq.sq_scale_from_absmax, self.vmax[k], self.qs_static[k])
+        wq = sum(self.W[w].numel() * (esize(self.W[w]) + 1) + 4 * self.W[w].shape[0] for w, _ in self.cfg["gemms"])
+        with self.phase("quantize_weight", ("hbm", wq)):
+            for w, src in self.cfg["gemms"]:
+                W = self.W[w]
+                s = None if src == "syn" else self.s[self.alpha][src]
+                L("quantize_weight", ("hbm", W.numel() * (esize(W) + 1) + 4 * W.shape[0]), sq.sq_quantize_weight,
+                  W, s, True, self.Wq[w], self.qw[w])
+
+    def norm_instances(self, n_sets=4):
+        """The norm + smoothing + int8 of this stack alone, on n_sets distinct
+        inputs (the step's two and fresh draws of the same kind), for a
+        back-to-back bandwidth figure; returns (launches, bytes per launch)."""
+        torch, sq = self.torch, self.sq
+        g = torch.Generator(device=self.dev).manual_seed(1234)
+        hs = [self.h["attn"], self.h["mlp"]]
+        while len(hs) < n_sets:
+            hs.append((torch.randn(hs[0].shape, generator=g, device=self.dev) * 3).to(hs[0].dtype))
+        outs = [(torch.empty(h.shape, dtype=torch.int8, device=self.dev),
+                 torch.empty(self.M if self.per_token else 1, device=self.dev)) for h in hs]
+        st = None if self.per_token else self.qs_static["attn"]
+        eps = self.d["eps"]
+
+        def one(h, o):
+            return lambda: sq.sq_norm_smooth_quant(h, self.norm, self.gp["attn"], self.bp["attn"], eps,
+                                                   self.per_token, st, o[0], o[1])
+        nbytes = self.M * self.K * esize(hs[0]) + self.M * self.K + 4 * outs[0][1].numel()
+        return [one(h, o) for h, o in zip(hs, outs)], nbytes
 
     def step(self):
         """The online linear stack: per side, norm + smoothing + int8 then the
@@ -409,6 +453,7 @@ class LlmInt8Stack:
         self.ws = sq.workspace(sq.SQ_OP_LLMINT8, M, N, K, device=dev)
         self.ws_det = sq.workspace(sq.SQ_OP_LLMINT8_DETECT, M, N, K, device=dev)
         self.bank = None
+        self.by_phase = False
 
     launch = Stack.launch
 
@@ -507,9 +552,10 @@ def run_stack(st, args, rank, world, dev, flush, e2e=True):
     g_step_ev = capture(st.step, stream)
     bank_step = st.bank
     st.bank = EventBank()
+    st.by_phase = hasattr(st, "phase")  # the offline pass: one interval per phase
     g_off_ev = capture(st.offline, stream)
     bank_off = st.bank
-    st.bank = None
+    st.bank, st.by_phase = None, False
     with torch.cuda.stream(stream):
         for _ in range(max(args.warmup, 3)):
             g_step.replay()
@@ -543,11 +589,50 @@ def run_stack(st, args, rank, world, dev, flush, e2e=True):
                       hbm)
     r = {"ms_per_step": ms_per_step, "step_ms_median": statistics.median(step_ms), "clocks": clk,
          "kernels": k_step, "offline": k_off, "instrumented_replays": n_ev, "ipk": ipk, "hbm": hbm,
-         "launches_per_step": st.launches_per_step()}
+         "launches_per_step": st.launches_per_step(),
+         "n_calib": len(st.d["calib"]) if isinstance(st.d, dict) and "calib" in st.d else None}
+    if hasattr(st, "norm_instances"):
+        r["norm_bandwidth"] = time_back_to_back(st.norm_instances(), args, dev, flush, hbm, stream)
     if e2e:
         r.update(run_e2e(st, g_step, args, world, dev, stream))
     del g_step, g_step_ev, g_off_ev
     return r
+
+
+def time_back_to_back(inst, args, dev, flush, hbm, stream):
+    """Launches of one kernel cycled over distinct input sets (together larger
+    than L2), back to back in one graph after one L2 flush: the mean time per
+    launch, the achieved bandwidth and its fraction of the measured copy
+    bandwidth, with the clocks sampled during the replay."""
+    import torch
+
+    fns, nbytes = inst
+    reps = max(5, min(args.steps, 20))
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for _ in range(reps):
+            for f in fns:
+                f()
+    with torch.cuda.stream(stream):
+        g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    time.sleep(0.05)
+    with torch.cuda.stream(stream):
+        flush()
+        a.record(stream)
+        g.replay()
+        b.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    n = reps * len(fns)
+    us = a.elapsed_time(b) * 1e3 / n
+    gbs = nbytes / (us * 1e-6) / 1e9
+    del g
+    return {"launches": n, "input_sets": len(fns), "us_per_launch": us, "bytes_per_launch": nbytes,
+            "achieved": gbs, "unit": "GB/s", "peak": hbm, "frac": gbs / hbm, "clocks": clk,
+            "timing": f"{n} launches back to back over {len(fns)} input sets, one L2 flush before"}
 
 
 def run_e2e(st, graph, args, world, dev, stream):
@@ -658,8 +743,12 @@ def json_line(args, world, r, shapes, tokens=None, cfg=None):
                     "note": "calibration, weight maxima, smoothing factors for every alpha, int8 weights: "
                             "timed separately, not part of the step"},
         "calibration": None if not calib else {
-            "batches": calib[0]["launches"], "us_per_batch": calib[0]["us_per_launch"],
-            "achieved": calib[0]["achieved"], "unit": "GB/s", "peak": r["hbm"], "frac": calib[0]["frac"]},
+            "batches": r.get("n_calib"), "us_total": calib[0]["us_total"],
+            "us_per_batch": calib[0]["us_total"] / max(r.get("n_calib") or 1, 1),
+            "bytes": calib[0]["bytes_per_launch"] * calib[0]["launches"], "achieved": calib[0]["achieved"],
+            "unit": "GB/s", "peak": r["hbm"], "frac": calib[0]["frac"],
+            "timing": "one interval around the whole pass (every batch back to back), L2 flushed before"},
+        "norm_bandwidth": r.get("norm_bandwidth"),
         "gpu_launches": r["launches_per_step"] * args.steps,
         "clocks": r["clocks"],
     }
@@ -682,9 +771,13 @@ def run_ours(args, rank, world, dev):
     line = json_line(args, world, r, shapes, cfg["tokens"], cfg)
     del st
     torch.cuda.empty_cache()
-    if args.configs:
+    names = [c for c in args.configs.split(",") if c and c not in ("none", args.workload)]
+    for c in names:
+        if c != "c4" and c not in CONFIGS:
+            raise SystemExit(f"unknown configuration {c}")
+    if names:
         extra = {}
-        for name in [c for c in args.configs.split(",") if c and c != args.workload]:
+        for name in names:
             if name == "c4":
                 s = LlmInt8Stack(dev)
                 rr = run_stack(s, args, rank, world, dev, flush, e2e=False)
@@ -1087,7 +1180,7 @@ def main():
     ap.add_argument("--whole-tiles", action="store_true", help="--kernel gemm: a workspace without stream-K scratch")
     ap.add_argument("--sets", type=int, default=1, help="--kernel: input sets cycled back to back (1: flush each)")
     ap.add_argument("--workload", default=HEADLINE, choices=sorted(CONFIGS), help="the headline stack")
-    ap.add_argument("--configs", default="c2,c3,c4", help="other stacks timed and reported under 'configs'")
+    ap.add_argument("--configs", default="c2,c3,c4", help="other stacks timed and reported under 'configs' (none: only the headline)")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)

@@ -85,7 +85,10 @@ SQ_API size_t sq_workspace_size(sq_op_t op, int64_t M, int64_t N, int64_t K);
 SQ_API const char* sq_last_error_string(void);
 
 /* Synchronises `stream`, reads the status word that bounded device waits
- * write into `workspace`, clears it and returns SQ_OK or SQ_ERR_TIMEOUT.
+ * write into `workspace`, clears it and returns SQ_OK or SQ_ERR_TIMEOUT. On
+ * SQ_ERR_TIMEOUT it also zeroes the stream-K counters of the last GEMM that
+ * used them on this workspace (their size is recorded in the header), so the
+ * workspace is ready for the next call without the caller zeroing it again.
  * Applies to workspaces passed to sq_gemm_w8a8, sq_gemm_fp8, sq_bmm_w8a8,
  * sq_llmint8_matmul and sq_selftest_wait_timeout. */
 SQ_API sq_status_t sq_workspace_status(void* workspace, sq_stream_t stream);
@@ -282,7 +285,8 @@ SQ_API sq_status_t sq_act_quant(const void* A, sq_dtype_t dt, int64_t M, int64_t
  *   a stream-K split of that wave (arrival counters and parked int32 partial
  *   sums). Zero it once before first use; every call that completes leaves
  *   the status word and the counters at zero again (the parked sums need no
- *   clearing). After SQ_ERR_TIMEOUT zero it again. A smaller workspace (at
+ *   clearing). After a call that timed out, sq_workspace_status (which
+ *   reports SQ_ERR_TIMEOUT) clears the counters as well. A smaller workspace (at
  *   least 256 bytes) is accepted and runs every tile whole. Calls sharing one
  *   workspace must not run concurrently.
  * ------------------------------------------------------------------------ */
@@ -343,7 +347,11 @@ SQ_API sq_status_t sq_gemm_fp8(const uint8_t* Xq, const uint8_t* Wq, int64_t M, 
  * test is strict, in fp32). min_ratio = 0 marks a column on any single
  * value over the threshold. X: [M,K] dt in {F16, BF16}, stride ldx.
  * outlier_idx: [K] int32 (first *n_outliers entries valid); n_outliers: [1]
- * int32, device. Workspace: SQ_OP_LLMINT8_DETECT. K % 8 == 0. */
+ * int32, device. Workspace: SQ_OP_LLMINT8_DETECT, zeroed once before its
+ * first use: it holds arrival counters that every completed call leaves at
+ * zero (one pass over X counts per 128-row band; the last band of each
+ * 256-column group adds the group up, the last group writes O). Calls sharing
+ * a workspace must not run concurrently. K % 8 == 0. */
 SQ_API sq_status_t sq_llmint8_detect(const void* X, sq_dtype_t dt, int64_t M, int64_t K, int64_t ldx,
                               float threshold, double min_ratio, int32_t* outlier_idx,
                               int32_t* n_outliers, void* workspace, size_t ws_bytes,
@@ -357,14 +365,20 @@ SQ_API sq_status_t sq_llmint8_detect(const void* X, sq_dtype_t dt, int64_t M, in
  * inference engine's plugin slot, a memory arena planned ahead of time with
  * nothing to spare), or a service that must not allocate once it is serving.
  * The scratch is a fixed 4 MiB device array inside this library, one per
- * device that loads it, held until the process exits. Hence
- * ceil(M / 128) * K <= 1,048,512 (for example M <= 32768 at K = 4096); larger
- * sizes return SQ_ERR_UNSUPPORTED_SHAPE and launch nothing.
- * The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * device that loads it, held until the process exits. It holds the per-band
+ * counts (4 * ceil(M / 128) * K bytes) after a 256-byte header and 36 bytes
+ * of counters and masks per 256 columns (each region rounded up to 256
+ * bytes), so for example M <= 32640 at K = 4096; larger sizes return
+ * SQ_ERR_UNSUPPORTED_SHAPE and launch nothing.
+ * The first call in a CUDA context looks up the array's device address there
+ * (cudaGetSymbolAddress), keyed by the context's unique id, so a new context
+ * (another driver-API context, or the primary context again after
+ * cudaDeviceReset) gets its own lookup; make that first call before any
+ * stream capture.
  * Every call uses the same array: calls that overlap on the GPU (other
  * streams, other host threads) race, so the caller must serialise them.
- * Nothing in the array needs clearing; each call writes every count it reads.
+ * Each call first clears the array's arrival counters on its stream (a
+ * memset, no allocation); the counts it reads it writes itself.
  * Arguments and results are those of sq_llmint8_detect. */
 SQ_API sq_status_t sq_llmint8_detect_noalloc(const void* X, sq_dtype_t dt, int64_t M, int64_t K, int64_t ldx,
                                              float threshold, double min_ratio, int32_t* outlier_idx,

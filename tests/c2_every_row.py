@@ -91,6 +91,8 @@ class Layer:
         s = e(I)
         sq.sq_smooth_scales(hmax, wmax, d["alpha"], s)
         torch.cuda.synchronize()
+        # kept for the parity test: every stage of the set-up is checked
+        self.calib = {"V": V, "Xq": Xq, "qx": qx, "Wq": Wq, "qw": qw, "Y": Y, "hmax": hmax, "wmax": wmax}
         return s
 
     def step(self, gemm_ev=None):

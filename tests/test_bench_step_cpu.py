@@ -35,6 +35,7 @@ def fake_stack(name):
     st.cfg = bench.CONFIGS[name]
     st.sq = RecordingSQ()
     st.bank = None
+    st.by_phase = False
     st.M, st.K = 8, 16
     st.d = {"eps": 1e-5}
     st.per_token = st.cfg["per_token"]
@@ -114,12 +115,13 @@ def synthetic_measurement():
          "ops_per_launch": 3.7e12, "achieved": 2846.0, "unit": "TOPS", "peak": 3306.6, "frac": 2846.0 / 3306.6,
          "frac_sustained": 2846.0 / 2779.0, "frac_nominal": 2846.0 / 4500.0, "algorithmic_bytes_per_launch": 7.6e8},
     ]
-    k_off = [{"kernel": "calib_absmax", "launches": 16, "us_per_launch": 18.0, "us_total": 288.0, "bound": "hbm",
-              "achieved": 5600.0, "unit": "GB/s", "peak": 6548.2, "frac": 5600.0 / 6548.2}]
+    k_off = [{"kernel": "calib_absmax", "launches": 1, "us_per_launch": 288.0, "us_total": 288.0, "bound": "hbm",
+              "bytes_per_launch": 1.61e9, "achieved": 5600.0, "unit": "GB/s", "peak": 6548.2, "frac": 5600.0 / 6548.2}]
     return {"ms_per_step": 5.5, "e2e_ms": 20.0, "h2d": 450 << 20, "d2h": 900 << 20, "e2e_steps": 20,
             "kernels": k_step, "offline": k_off, "instrumented_replays": 20,
             "ipk": {"burst": 3306.6, "sustained": 2779.0, "nominal": 4500.0, "source": "measured"}, "hbm": 6548.2,
-            "launches_per_step": 6, "clocks": {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}}
+            "launches_per_step": 6, "n_calib": 16, "clocks": {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []},
+            "norm_bandwidth": {"us_per_launch": 30.0, "achieved": 5033.0, "frac": 5033.0 / 6548.2}}
 
 
 def test_json_line_contract():
@@ -146,7 +148,8 @@ def test_json_line_contract():
     assert line["n_gpus"] == 2 and line["scaling"] == "weak" and line["higher_is_better"] is True
     assert line["config"]["workload"] == bench.CONFIGS["c5"]["workload"] and "l2" in line["config"]
     assert line["config"]["tokens"] == 4096 and line["config"]["hidden"] == 12288
-    assert line["calibration"]["batches"] == 16
+    assert line["calibration"]["batches"] == 16 and line["calibration"]["us_per_batch"] == 18.0
+    assert line["calibration"]["bytes"] == 1.61e9 and line["norm_bandwidth"]["us_per_launch"] == 30.0
     assert abs(line["offline"]["ms"] - 0.288) < 1e-12
 
 

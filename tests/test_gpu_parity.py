@@ -515,6 +515,37 @@ def test_gemm_stream_k(M, N, K, monkeypatch):
     assert_close_16(Yb[rows].contiguous(), y, torch.bfloat16, terms)
 
 
+def test_stream_k_workspace_recovers_after_a_timeout(monkeypatch):
+    """A stream-K GEMM that gave up part-way leaves its arrival counters
+    counted in. The failure is made on the host (no GPU fault): after a
+    normal call, garbage counts and a timeout code are written into the
+    workspace; sq_workspace_status reports the timeout and clears the
+    counters, and the next call on the same workspace is exact."""
+    monkeypatch.setenv("SQ_GEMM_CTA_PAIRS", "0")
+    M, N, K = 1029, 7168, 7200
+    Xq, Wq = rand_i8((M, K), 91), rand_i8((N, K), 92)
+    Xd, Wd = Xq.to(DEV), Wq.to(DEV)
+    ws = sq.workspace(sq.SQ_OP_GEMM, M, N, K)
+    Y = torch.empty((M, N), dtype=torch.int32, device=DEV)
+    sq.sq_gemm_w8a8(Xd, Wd, None, None, None, Y, ws)
+    sq.sq_workspace_status(ws)
+    hdr = ws[:256].view(torch.int32)
+    cnt_bytes = int(hdr[3].item())
+    assert cnt_bytes > 0 and cnt_bytes % 256 == 0  # the counters' region was recorded
+    ws[256:256 + cnt_bytes].view(torch.int32).fill_(3)  # pieces counted in, never completed
+    hdr[0] = 0x6E1
+    with pytest.raises(sq.SqError):
+        sq.sq_workspace_status(ws)
+    assert int(ws[256:256 + cnt_bytes].view(torch.int32).abs().sum().item()) == 0
+    assert int(hdr[0].item()) == 0
+    Y2 = torch.empty_like(Y)
+    sq.sq_gemm_w8a8(Xd, Wd, None, None, None, Y2, ws)
+    sq.sq_workspace_status(ws)
+    assert torch.equal(Y, Y2)
+    rows = [0, 511, 1028]
+    assert np.array_equal(Y2[rows].cpu().numpy().astype(np.int64), oracle.gemm_i8(Xq[rows].numpy(), Wq.numpy()))
+
+
 def test_bounded_wait_timeout():
     """A wait that nothing completes gives up after its limit, the status word
     says so (SQ_ERR_TIMEOUT on the host), and the context stays usable."""
@@ -634,6 +665,54 @@ def test_llmint8_cache_follows_outlier_set(keep_wo):
         Xf, Wf = npf(X).astype(np.float64), npf(W).astype(np.float64)
         terms = np.abs(oracle.dequant(acc, rqx, rqw)) + np.abs(Xf[:, ridx]) @ np.abs(Wf[:, ridx]).T
         assert_close_16(Y, y, torch.float16, terms)
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("n_out,thr", [(40, 6.0), (0, 3.0)])
+def test_llmint8_beyond_compact_cap(dtype, n_out, thr):
+    """|O| above the 32 outlier columns the epilogue keeps as compact fp32
+    copies: 40 planted dimensions at the 6.0 threshold, and a threshold of 3.0
+    on N(0, 1) data (about half of all columns). The GEMM epilogue then reads
+    the 16-bit operands of every outlier column directly."""
+    M, K, N = 256, 512, 384
+    X, W, dims = _llm_case(M, K, N, n_out, seed=77 + n_out, dtype=dtype)
+    ridx = oracle.llmint8_outliers(X, thr, 0.0)
+    assert ridx.size > 32
+    if n_out:
+        assert ridx.tolist() == dims.tolist()
+    Xd = X.to(DEV)
+    st = sq.llmint8_weight_state(W.to(DEV))
+    Y = torch.empty((M, N), dtype=dtype, device=DEV)
+    idx = torch.empty(K, dtype=torch.int32, device=DEV)
+    n = torch.empty(1, dtype=torch.int32, device=DEV)
+    ws = sq.workspace(sq.SQ_OP_LLMINT8, M, N, K)
+    sq.sq_llmint8_matmul(Xd, st, thr, 0.0, Y, idx, n, ws)
+    torch.cuda.synchronize()
+    sq.sq_workspace_status(ws)
+    assert int(n.item()) == ridx.size and idx[:ridx.size].cpu().numpy().tolist() == ridx.tolist()
+    rXq, rqx = oracle.llmint8_quant_rows(X, ridx)
+    rWq, rqw = oracle.llmint8_quant_weight(W, ridx)
+    assert np.array_equal(st["Wq"].cpu().numpy(), rWq) and np.array_equal(npf(st["qs_w"]), rqw)
+    acc = oracle.gemm_i8(rXq, rWq)
+    y = oracle.llmint8_combine(acc, rqx, rqw, X, W, ridx)
+    Xf, Wf = npf(X).astype(np.float64), npf(W).astype(np.float64)
+    terms = np.abs(oracle.dequant(acc, rqx, rqw)) + np.abs(Xf[:, ridx]) @ np.abs(Wf[:, ridx]).T
+    assert_close_16(Y, y, dtype, terms)
+
+
+def test_llmint8_detect_counters_reset():
+    """The detection's arrival counters are back at zero after every call:
+    many calls in a row on one workspace, of several sizes, all exact."""
+    ws = sq.workspace(sq.SQ_OP_LLMINT8_DETECT, 2048, 0, 4096)
+    for i, (M, K, n_out) in enumerate([(2048, 4096, 6), (300, 1024, 3), (1, 256, 0), (700, 4096, 9), (2048, 4096, 6)]):
+        X, _, dims = _llm_case(M, K, 16, n_out, seed=500 + i)
+        idx = torch.full((K,), -1, dtype=torch.int32, device=DEV)
+        n = torch.full((1,), -1, dtype=torch.int32, device=DEV)
+        sq.sq_llmint8_detect(X.to(DEV), 6.0, 0.0, idx, n, ws)
+        torch.cuda.synchronize()
+        assert int(n.item()) == n_out and idx[:n_out].cpu().tolist() == dims.tolist()
+    hdr = ws[:256].view(torch.int32).cpu()
+    assert int(hdr[2]) == 0  # the count of finished column groups
 
 
 def test_llmint8_min_ratio():
@@ -912,22 +991,28 @@ def test_every_row_step_against_oracle():
         assert np.array_equal(npf(L.s[k]), s[k])
         gp[k], _ = oracle.fold_norm(d["gamma_" + k].numpy(), None, s[k])
         assert np.array_equal(npf(L.gp[k]), gp[k])
-    # weight side: the down_proj factors s_down are set-up state, taken from the
-    # device; checked here on sampled channels against the oracle's own
-    # calibration (through a 16-bit GEMM output, so to 1e-2 relative: a one-ulp
-    # bf16 difference of gate or up moves a column maximum by about 2^-8)
-    s_down = npf(L.s_down)
-    js = [0, 5, 1000, I - 1]
+    # weight side: down_proj's factors s_down come from the set-up's
+    # calibration pass, checked stage by stage on every channel: the norm
+    # output and its per-token int8 (bit-exact), the int8 gate/up weight
+    # (bit-exact), the calibration GEMM's bf16 output (within one ulp, on
+    # sampled rows), then, from the device's own bf16 output, the SwiGLU
+    # maxima, down_proj's weight maxima and s_down (bit-exact)
+    c = L.calib
     Vc = oracle.norm_smooth_quant(d["h_calib"], oracle.RMSNORM, d["gamma_mlp"].numpy(), None, eps,
                                   quantize=False, want_v=True)["V"]
-    Xc, qc = oracle.quantize_act(torch.from_numpy(Vc).to(torch.bfloat16).float().numpy(), None, per_token=True)
+    Vc16 = torch.from_numpy(Vc).to(torch.bfloat16)
+    assert np.array_equal(npu16(c["V"]), npu16(Vc16))
+    Xc, qc = oracle.quantize_act(Vc16.float().numpy(), None, per_token=True)
+    assert np.array_equal(c["Xq"].cpu().numpy(), Xc) and np.array_equal(npf(c["qx"]), qc)
     Wc, qwc = oracle.quantize_weight(W["gateup"], True)
-    sel = js + [I + j for j in js]
-    yc = oracle.dequant(oracle.gemm_i8(Xc, Wc[sel]), qc, qwc[sel])
-    yc16 = torch.from_numpy(oracle.round_bf16_bits(yc).view(np.int16)).view(torch.bfloat16).float().numpy()
-    hmax = oracle.act_quant(yc16, oracle.SWIGLU, quantize=False, absmax=np.zeros(len(js), np.float32))["absmax"]
-    s_js = oracle.smooth_scales(hmax, oracle.col_absmax(W["down"])[js], alpha)
-    assert np.allclose(s_down[js], s_js, rtol=1e-2, atol=0)
+    assert np.array_equal(c["Wq"].cpu().numpy(), Wc) and np.array_equal(npf(c["qw"]), qwc)
+    assert_close_16(c["Y"][rows], oracle.dequant(oracle.gemm_i8(Xc[rows], Wc), qc[rows], qwc), torch.bfloat16)
+    hmax = oracle.act_quant(npf(c["Y"]), oracle.SWIGLU, quantize=False, absmax=np.zeros(I, np.float32))["absmax"]
+    assert np.array_equal(npf(c["hmax"]), hmax)
+    wmax_down = oracle.col_absmax(W["down"])
+    assert np.array_equal(npf(c["wmax"]), wmax_down)
+    s_down = oracle.smooth_scales(hmax, wmax_down, alpha)
+    assert np.array_equal(npf(L.s_down), s_down)
     up_f, _ = oracle.fold_prev_linear(W["gateup"][I:], s_down)
     ref_w = {
         "qkv": oracle.fold_weight(W["qkv"], s["attn"]),

@@ -70,3 +70,42 @@ def test_reference_arm_under_torchrun():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def _calib_rank_cuda(rank, world, port, out):
+    """The same exchange with each rank's maxima from the library's CUDA
+    column absmax over its shard (both ranks on the one visible GPU: the
+    kernels are independent launches that wait on nothing)."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        sys.path.insert(0, ROOT)
+        import oracle
+        import w8a8_post_quantization_sq_b200 as sq
+        from w8a8_post_quantization_sq_b200 import inputs, sharded
+
+        d = inputs.c5_175b(device="cpu", M=64, n_calib=4, w_frac=1 / 4096)
+        batches = d["calib"]  # bf16 [64, 12288] each, 8 channels x100
+        mine = [b for i, b in enumerate(batches) if i % world == rank]
+        xmax = torch.zeros(12288, device="cuda")
+        for b in mine:
+            sq.sq_calib_absmax(b.cuda(), xmax)
+        local = xmax.cpu()
+        sharded.allreduce_max_(local)
+        full = np.zeros(12288, np.float32)
+        for b in batches:
+            full = oracle.col_absmax(b, full)
+        out[rank] = bool(np.array_equal(local.numpy(), full))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.gpu
+def test_sharded_calibration_with_cuda_maxima():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    world = 2
+    port = _free_port()
+    out = mp.Manager().dict()
+    mp.spawn(_calib_rank_cuda, args=(world, port, out), nprocs=world, join=True)
+    assert all(out[r] for r in range(world)), "sharded CUDA maxima differ from the oracle's maxima of all tokens"

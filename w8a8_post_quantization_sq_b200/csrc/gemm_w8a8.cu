@@ -112,6 +112,7 @@ struct Params {
     // sk_tiles tiles, sk_iters in all, are cut into one contiguous range per
     // CTA.
     int dp_tiles, sk_tiles, sk_iters;
+    int sk_cnt_bytes;  // size of the counter region, recorded in header word 3 for sq_workspace_status
     int* sk_cnt;   // [sk_tiles][kEpiWarps] k-blocks counted in per tile region (zero between launches)
     int* sk_part;  // [grid][2][kEpiWarps][NCH][8][32] int4: parked int32 partial sums
 };
@@ -568,6 +569,9 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
     // here for the previous kernel in the stream before any global access
     pdl_wait();
     pdl_trigger();
+    // where this launch keeps its stream-K counters: if a bounded wait gives
+    // up, sq_workspace_status clears that region with the status word
+    if (SK && blockIdx.x == 0 && threadIdx.x == 0) p.status[3] = p.sk_cnt_bytes;
 
     const int num_tiles = p.batch * p.num_m * p.num_n;
     if (warp == 0) {
@@ -982,6 +986,7 @@ sq_status_t launch_bn(const int8_t* Xq, const int8_t* Wq, int64_t M, int64_t N, 
     p.sk_tiles = sk ? plan.sk_tiles : 0;
     p.sk_iters = sk ? plan.sk_tiles * p.num_kb : 0;
     p.sk_cnt = sk ? static_cast<int*>(sk_ws) : nullptr;
+    p.sk_cnt_bytes = sk ? (int)plan.sk_cnt_bytes : 0;
     p.sk_part = sk ? reinterpret_cast<int*>(static_cast<uint8_t*>(sk_ws) + plan.sk_cnt_bytes) : nullptr;
     const int grid = plan.grid;
     if constexpr (CG == 2)

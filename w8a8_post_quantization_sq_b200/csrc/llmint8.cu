@@ -9,19 +9,25 @@
 //   the two results are summed.
 //
 // Kernels:
-//   count_kernel      one pass over X; a block owns 256 columns x 128 rows and
+//   detect_kernel     one pass over X; a block owns 256 columns x 128 rows and
 //                     writes its per-column counts to its own slot of the
-//                     workspace (no atomics, nothing to zero beforehand);
-//   compact_kernel    one block sums the slots, applies the ratio test in
-//                     fp64, and writes O in ascending order with a block-wide
-//                     prefix sum; it also compares O with the set the cached
-//                     int8 weight was built for and updates that record;
+//                     workspace. The last block of each 256-column group to
+//                     finish (an atomic count per group) adds the group's
+//                     slots, applies the ratio test in fp64 and writes the
+//                     group's 256-bit outlier mask; the last group to finish
+//                     writes O in ascending order with a block-wide prefix sum
+//                     over the masks, and compares O with the set the cached
+//                     int8 weight was built for, updating that record. Each
+//                     block that completes a count sets it back to zero, so
+//                     the counters are zero between calls;
 //   masked_quant_kernel  row-wise absmax int8 over the columns not in O (used
 //                     for the rows of X and for the output channels of W; the
 //                     weight pass returns at once when O is unchanged);
 //   the tcgen05 GEMM, whose epilogue adds the 16-bit outlier term.
 // Nothing here synchronises with the host, so a whole call can be captured in
 // a CUDA graph.
+#include <cuda.h>
+
 #include <mutex>
 #include <type_traits>
 
@@ -30,13 +36,22 @@
 
 namespace sq {
 
+static size_t r256(size_t b) { return (b + 255) / 256 * 256; }
+
+// Detection scratch: the 256-byte header (word 0 status, word 1 "O changed",
+// word 2 the count of finished column groups), one arrival counter per
+// 256-column group, the groups' outlier masks (8 words each), then the
+// per-band column counts [row bands, K].
+static int64_t col_groups(int64_t K) { return (K + 255) / 256; }
+static size_t detect_done_off() { return kStatusBytes; }
+static size_t detect_mask_off(int64_t K) { return detect_done_off() + r256((size_t)col_groups(K) * 4); }
+static size_t detect_count_off(int64_t K) { return detect_mask_off(K) + r256((size_t)col_groups(K) * 32); }
+
 size_t detect_workspace_bytes(int64_t M, int64_t K) {
     const int64_t rb = (M + kDetectRows - 1) / kDetectRows;
     const size_t counts = (size_t)(rb > 0 ? rb : 1) * (size_t)K * sizeof(int32_t);
-    return kStatusBytes + (counts + 255) / 256 * 256;
+    return detect_count_off(K) + r256(counts);
 }
-
-static size_t r256(size_t b) { return (b + 255) / 256 * 256; }
 static int64_t wo_ld_of(int64_t N) { return (N + 255) / 256 * 256; }
 
 // header + counts | Xq [M,K] int8 | qs_x [M] fp32 | X_O [cap, M] fp32 (o-major) | W_O [cap, N256] fp32
@@ -48,15 +63,24 @@ size_t llmint8_workspace_bytes(int64_t M, int64_t N, int64_t K) {
 namespace {
 
 constexpr int kWarps = 8;
-constexpr int kCompactThreads = 1024;
 
+// Per-column counts of |x| > thr over a 128-row band, then (in the last block
+// of each column group, and of the grid) the outlier set. `done` holds one
+// arrival counter per column group, `gdone` the count of finished groups;
+// both are zero when the kernel starts and when it ends.
 template <typename T>
 __global__ void __launch_bounds__(kWarps * 32)
-count_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, float thr, int32_t* __restrict__ partial) {
+detect_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, float thr, double min_ratio,
+              int32_t* __restrict__ partial, uint32_t* __restrict__ done, uint32_t* __restrict__ masks,
+              uint32_t* __restrict__ gdone, int32_t* __restrict__ idx, int32_t* __restrict__ n_out,
+              int32_t* __restrict__ cached_idx, int32_t* __restrict__ cached_n, int32_t* __restrict__ changed) {
     pdl_wait();
     pdl_trigger();
     __shared__ int32_t red[kWarps][256];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    __shared__ int32_t warp_tot[kWarps];
+    __shared__ int32_t flag_sh;
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int64_t rb = gridDim.y;
     const int64_t c0 = (int64_t)blockIdx.x * 256 + lane * 8;
     const int64_t r0 = (int64_t)blockIdx.y * kDetectRows;
     const int64_t r1 = min(M, r0 + kDetectRows);
@@ -86,75 +110,90 @@ count_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, float th
     for (int e = 0; e < 8; ++e) red[warp][lane * 8 + e] = cnt[e];
     __syncwarp();  // lanes may have diverged above; bar.sync needs whole warps
     __syncthreads();
-    for (int c = threadIdx.x; c < 256; c += kWarps * 32) {
+    const int64_t col = (int64_t)blockIdx.x * 256 + t;  // kWarps * 32 == 256: one column per thread
+    {
         int32_t s = 0;
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) s += red[w][c];
-        const int64_t col = (int64_t)blockIdx.x * 256 + c;
+        for (int w = 0; w < kWarps; ++w) s += red[w][t];
         if (col < K) partial[(int64_t)blockIdx.y * K + col] = s;
     }
-}
-
-// flags word 1 of the workspace header: 1 when O differs from the cached set.
-__global__ void __launch_bounds__(kCompactThreads)
-compact_kernel(const int32_t* __restrict__ partial, int64_t row_blocks, int64_t M, int64_t K, double min_ratio,
-               int32_t* __restrict__ idx, int32_t* __restrict__ n_out, int32_t* __restrict__ cached_idx,
-               int32_t* __restrict__ cached_n, int32_t* __restrict__ changed) {
-    pdl_wait();
-    pdl_trigger();
-    __shared__ int32_t warp_tot[kCompactThreads / 32];
-    __shared__ int32_t base_sh;
-    __shared__ int32_t diff_sh;
-    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    if (t == 0) base_sh = 0, diff_sh = 0;
-    __syncwarp();
+    // the last band of this column group to arrive adds the group's counts
+    __threadfence();
     __syncthreads();
-    for (int64_t j0 = 0; j0 < K; j0 += kCompactThreads) {
-        const int64_t j = j0 + t;
-        bool flag = false;
-        if (j < K) {
-            int64_t total = 0;
-#pragma unroll 8
-            for (int64_t b = 0; b < row_blocks; ++b) total += partial[b * K + j];
-            // an empty column has ratio 0, never above min_ratio >= 0
-            if (total > 0) {
-                const double ratio = M > 0 ? __ddiv_rn((double)total, (double)M) : 0.0;
-                flag = ratio > min_ratio;
-            }
+    if (t == 0) flag_sh = atomicAdd(done + blockIdx.x, 1u) == (uint32_t)(rb - 1);
+    __syncthreads();
+    if (!flag_sh) return;
+    __threadfence();
+    bool flag = false;
+    if (col < K) {
+        int64_t total = 0;
+        for (int64_t b = 0; b < rb; ++b) total += __ldcg(partial + b * K + col);
+        // an empty column has ratio 0, never above min_ratio >= 0
+        if (total > 0) {
+            const double ratio = M > 0 ? __ddiv_rn((double)total, (double)M) : 0.0;
+            flag = ratio > min_ratio;
         }
-        const unsigned bal = __ballot_sync(0xffffffffu, flag);
-        const int before_in_warp = __popc(bal & ((1u << lane) - 1u));
-        if (lane == 0) warp_tot[warp] = __popc(bal);
+    }
+    const unsigned bal = __ballot_sync(0xffffffffu, flag);
+    if (lane == 0) masks[blockIdx.x * 8 + warp] = bal;
+    if (t == 0) done[blockIdx.x] = 0u;  // ready for the next call
+    // the last column group to finish writes O
+    __threadfence();
+    __syncthreads();
+    if (t == 0) flag_sh = atomicAdd(gdone, 1u) == gridDim.x - 1;
+    __syncthreads();
+    if (!flag_sh) return;
+    __threadfence();
+    const int64_t words = (int64_t)gridDim.x * 8;
+    int base = 0;
+    for (int64_t w0 = 0; w0 < words; w0 += 256) {
+        const int64_t w = w0 + t;
+        const uint32_t bits = w < words ? __ldcg(masks + w) : 0u;
+        const int c = __popc(bits);
+        // exclusive prefix of c over the block, in word order
+        int incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) warp_tot[warp] = incl;
         __syncwarp();
         __syncthreads();
-        int before = base_sh;
-        for (int w = 0; w < warp; ++w) before += warp_tot[w];
-        if (flag) idx[before + before_in_warp] = (int32_t)j;
-        __syncwarp();
-        __syncthreads();
-        if (t == 0) {
-            int s = 0;
-            for (int w = 0; w < kCompactThreads / 32; ++w) s += warp_tot[w];
-            base_sh += s;
+        int before = base + incl - c;
+        int total = 0;
+#pragma unroll
+        for (int q = 0; q < kWarps; ++q) {
+            if (q < warp) before += warp_tot[q];
+            total += warp_tot[q];
         }
+        uint32_t rest = bits;
+        while (rest) {
+            const int bpos = __ffs(rest) - 1;
+            idx[before++] = (int32_t)(w * 32 + bpos);
+            rest &= rest - 1u;
+        }
+        base += total;
         __syncwarp();
         __syncthreads();
     }
-    const int n = base_sh;
-    if (t == 0) *n_out = n;
+    const int n = base;
+    if (t == 0) {
+        *n_out = n;
+        *gdone = 0u;  // ready for the next call
+    }
     if (cached_n) {
-        const int cn = *cached_n;
-        if (cn != n) diff_sh = 1;
+        __threadfence_block();
+        if (t == 0) flag_sh = *cached_n != n;
+        __syncthreads();
+        if (!flag_sh)
+            for (int o = t; o < n; o += kWarps * 32)
+                if (cached_idx[o] != idx[o]) flag_sh = 1;
         __syncwarp();
         __syncthreads();
-        if (!diff_sh)
-            for (int o = t; o < n; o += kCompactThreads)
-                if (cached_idx[o] != idx[o]) diff_sh = 1;
-        __syncwarp();
-        __syncthreads();
-        const int d = diff_sh;
+        const int d = flag_sh;
         if (d) {
-            for (int o = t; o < n; o += kCompactThreads) cached_idx[o] = idx[o];
+            for (int o = t; o < n; o += kWarps * 32) cached_idx[o] = idx[o];
             if (t == 0) *cached_n = n;
         }
         if (t == 0) *changed = d;
@@ -328,19 +367,21 @@ sq_status_t launch_detect(const void* X, sq_dtype_t dt, int64_t M, int64_t K, in
                           void* ws, cudaStream_t s) {
     char* wsb = static_cast<char*>(ws);
     int32_t* changed = reinterpret_cast<int32_t*>(wsb + 4);
-    int32_t* partial = reinterpret_cast<int32_t*>(wsb + kStatusBytes);
-    const int64_t rb = (M + kDetectRows - 1) / kDetectRows;
-    if (rb > 0) {
-        SQ_REQUIRE(rb <= 65535, SQ_ERR_UNSUPPORTED_SHAPE, "sq_llmint8_detect: M too large");
-        dim3 grid((unsigned)((K + 255) / 256), (unsigned)rb);
-        if (dt == SQ_BF16)
-            launch_pdl(count_kernel<__nv_bfloat16>, dim3(grid), dim3(kWarps * 32), 0, s, static_cast<const __nv_bfloat16*>(X), M, K, ldx,
-                                                                      thr, partial);
-        else
-            launch_pdl(count_kernel<__half>, dim3(grid), dim3(kWarps * 32), 0, s, static_cast<const __half*>(X), M, K, ldx, thr, partial);
-    }
-    launch_pdl(compact_kernel, dim3(1), dim3(kCompactThreads), 0, s, partial, rb, M, K, min_ratio, idx, n_out, cached_idx, cached_n,
-                                                 changed);
+    uint32_t* gdone = reinterpret_cast<uint32_t*>(wsb + 8);
+    uint32_t* done = reinterpret_cast<uint32_t*>(wsb + detect_done_off());
+    uint32_t* masks = reinterpret_cast<uint32_t*>(wsb + detect_mask_off(K));
+    int32_t* partial = reinterpret_cast<int32_t*>(wsb + detect_count_off(K));
+    int64_t rb = (M + kDetectRows - 1) / kDetectRows;
+    if (rb < 1) rb = 1;  // M == 0: one band with no rows, so O is empty
+    SQ_REQUIRE(rb <= 65535, SQ_ERR_UNSUPPORTED_SHAPE, "sq_llmint8_detect: M too large");
+    SQ_REQUIRE(col_groups(K) < (1ll << 31), SQ_ERR_UNSUPPORTED_SHAPE, "sq_llmint8_detect: K too large");
+    dim3 grid((unsigned)col_groups(K), (unsigned)rb);
+    if (dt == SQ_BF16)
+        launch_pdl(detect_kernel<__nv_bfloat16>, grid, dim3(kWarps * 32), 0, s, static_cast<const __nv_bfloat16*>(X), M,
+                   K, ldx, thr, min_ratio, partial, done, masks, gdone, idx, n_out, cached_idx, cached_n, changed);
+    else
+        launch_pdl(detect_kernel<__half>, grid, dim3(kWarps * 32), 0, s, static_cast<const __half*>(X), M, K, ldx, thr,
+                   min_ratio, partial, done, masks, gdone, idx, n_out, cached_idx, cached_n, changed);
     return check_launch("sq_llmint8_detect");
 }
 
@@ -518,26 +559,67 @@ namespace {
 constexpr size_t kDetectScratchBytes = size_t(4) << 20;  // 4 MiB
 __device__ __align__(256) unsigned char g_detect_scratch[kDetectScratchBytes];
 
-constexpr int kMaxDevices = 64;
+// Device addresses of g_detect_scratch, one per CUDA context: the array's
+// name is only a host-side stand-in, and each context that loads the
+// library's module has its own copy of it. Keyed by the context's unique id
+// (cuCtxGetId), which a context created later never reuses, even when it
+// gets the same handle (the primary context after cudaDeviceReset).
+constexpr int kMaxContexts = 64;
 std::mutex g_scratch_mu;
-void* g_scratch_addr[kMaxDevices] = {};
+unsigned long long g_scratch_ctx[kMaxContexts] = {};
+void* g_scratch_addr[kMaxContexts] = {};
+int g_scratch_n = 0;
 
-// Device address of g_detect_scratch on the current device. The name is only
-// a host-side stand-in, so the address is looked up once per device.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+template <typename F>
+F driver_fn(const char* name) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion(name, &p, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+        return nullptr;
+    return reinterpret_cast<F>(p);
+}
+
 sq_status_t detect_scratch(void** out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return check_launch("sq_llmint8_detect_noalloc: cudaGetDevice");
-    if (dev < 0 || dev >= kMaxDevices)
-        return set_error(SQ_ERR_CUDA, "sq_llmint8_detect_noalloc: device %d out of range", dev);
+    static CtxGetCurrentFn get_cur = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+    static CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+    if (!get_cur || !get_id)
+        return set_error(SQ_ERR_CUDA, "sq_llmint8_detect_noalloc: cuCtxGetCurrent / cuCtxGetId unavailable");
     std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (g_scratch_addr[dev] == nullptr) {
-        void* p = nullptr;
+    void* p = nullptr;
+    CUcontext ctx = nullptr;
+    if (get_cur(&ctx) != CUDA_SUCCESS || !ctx) {
+        // no context current on this thread yet: the symbol lookup
+        // initialises the runtime's (primary) context and makes it current
         const cudaError_t e = cudaGetSymbolAddress(&p, g_detect_scratch);
         if (e != cudaSuccess || p == nullptr)
-            return set_error(SQ_ERR_CUDA, "sq_llmint8_detect_noalloc: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
-        g_scratch_addr[dev] = p;
+            return set_error(SQ_ERR_CUDA, "sq_llmint8_detect_noalloc: cudaGetSymbolAddress: %s",
+                             cudaGetErrorString(e));
+        if (get_cur(&ctx) != CUDA_SUCCESS || !ctx)
+            return set_error(SQ_ERR_CUDA, "sq_llmint8_detect_noalloc: no current CUDA context");
     }
-    *out = g_scratch_addr[dev];
+    unsigned long long id = 0;
+    if (get_id(ctx, &id) != CUDA_SUCCESS)
+        return set_error(SQ_ERR_CUDA, "sq_llmint8_detect_noalloc: cannot identify the current CUDA context");
+    for (int i = 0; i < g_scratch_n; ++i)
+        if (g_scratch_ctx[i] == id) {
+            *out = g_scratch_addr[i];
+            return SQ_OK;
+        }
+    if (!p) {
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_detect_scratch);
+        if (e != cudaSuccess || p == nullptr)
+            return set_error(SQ_ERR_CUDA, "sq_llmint8_detect_noalloc: cudaGetSymbolAddress: %s",
+                             cudaGetErrorString(e));
+    }
+    // a full table forgets the oldest context (it only costs a new lookup)
+    const int slot = g_scratch_n < kMaxContexts ? g_scratch_n++ : (int)(id % kMaxContexts);
+    g_scratch_ctx[slot] = id;
+    g_scratch_addr[slot] = p;
+    *out = p;
     return SQ_OK;
 }
 
@@ -562,8 +644,11 @@ extern "C" sq_status_t sq_llmint8_detect_noalloc(const void* X, sq_dtype_t dt, i
     void* scratch = nullptr;
     st = sq::detect_scratch(&scratch);
     if (st != SQ_OK) return st;
-    // every count slot read by the compaction is written by this call first,
-    // so nothing in the scratch has to be cleared between calls
+    // the arrival counters must start at zero: a completed call leaves them
+    // at zero, and they are cleared here too (a memset, no allocation); the
+    // counts and masks are written before they are read
+    if (cudaMemsetAsync(scratch, 0, sq::detect_mask_off(K), sq::as_cuda(stream)) != cudaSuccess)
+        return sq::check_launch("sq_llmint8_detect_noalloc: clearing the counters");
     return sq::launch_detect(X, dt, M, K, ldx, threshold, min_ratio, outlier_idx, n_outliers, nullptr, nullptr,
                              scratch, sq::as_cuda(stream));
 }

@@ -76,15 +76,22 @@ sq_status_t sq_workspace_status(void* workspace, sq_stream_t stream) {
     if (cudaStreamSynchronize(s) != cudaSuccess)
         return sq::set_error(SQ_ERR_CUDA, "sq_workspace_status: %s",
                              cudaGetErrorString(cudaGetLastError()));
-    int word = 0;
-    if (cudaMemcpy(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    // word 0: the status word; word 3: the size of the stream-K counter
+    // region that follows the header, as the last stream-K GEMM recorded it
+    int words[4] = {0, 0, 0, 0};
+    if (cudaMemcpy(words, workspace, sizeof(words), cudaMemcpyDeviceToHost) != cudaSuccess)
         return sq::set_error(SQ_ERR_CUDA, "sq_workspace_status: copy failed");
-    if (word != 0) {
-        int zero = 0;
+    if (words[0] != 0) {
+        // a call gave up part-way: its stream-K counters may be left counted
+        // in; clear them with the status word, so the next call starts clean
+        if (words[3] > 0 && words[3] <= (1 << 26))
+            cudaMemset(static_cast<char*>(workspace) + sq::kStatusBytes, 0, (size_t)words[3]);
+        const int zero = 0;
         cudaMemcpy(workspace, &zero, sizeof(int), cudaMemcpyHostToDevice);
+        cudaMemcpy(static_cast<int*>(workspace) + 3, &zero, sizeof(int), cudaMemcpyHostToDevice);
         return sq::set_error(SQ_ERR_TIMEOUT,
                              "a bounded device wait timed out (code %d); results of that call are invalid",
-                             word);
+                             words[0]);
     }
     return SQ_OK;
 }
