@@ -126,8 +126,17 @@ detect_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, float t
     __threadfence();
     bool flag = false;
     if (col < K) {
+        // the band counts of this column, eight loads in flight at a time
         int64_t total = 0;
-        for (int64_t b = 0; b < rb; ++b) total += __ldcg(partial + b * K + col);
+        int64_t b = 0;
+        for (; b + 8 <= rb; b += 8) {
+            int32_t v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v[u] = __ldcg(partial + (b + u) * K + col);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) total += v[u];
+        }
+        for (; b < rb; ++b) total += __ldcg(partial + b * K + col);
         // an empty column has ratio 0, never above min_ratio >= 0
         if (total > 0) {
             const double ratio = M > 0 ? __ddiv_rn((double)total, (double)M) : 0.0;
@@ -200,32 +209,75 @@ detect_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, float t
     }
 }
 
-// Row-wise int8 over the columns not in O (zeros in O). When `only_if` is
-// given and *only_if == 0 the kernel does nothing.
-template <typename T>
-__global__ void __launch_bounds__(256)
-masked_quant_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, const int32_t* __restrict__ idx,
-                    const int32_t* __restrict__ n_idx, const int32_t* __restrict__ only_if, int8_t* __restrict__ Q,
-                    float* __restrict__ qs_out, float* __restrict__ xo, int64_t xo_ld) {
-    pdl_wait();
-    pdl_trigger();
-    extern __shared__ uint32_t mask[];  // K bits
-    if (only_if && *only_if == 0) return;
+// One row-quantisation job of the masked kernels: row-wise int8 over the
+// columns not in O (zeros in O) of a [rows, K] 16-bit matrix, with the fp32
+// copy of its outlier columns (o-major, xo[o * xo_ld + row]) when xo is
+// given. When only_if is given and *only_if == 0 the job does nothing.
+struct MQJob {
+    const void* X;
+    int64_t rows, ld;
+    int8_t* Q;
+    float* qs;
+    float* xo;
+    int64_t xo_ld;
+    const int32_t* only_if;
+};
+
+// A launch runs up to two jobs (the rows of X and the weight's output
+// channels of one LLM.int8 call): blocks [0, split) take job 0, the rest job
+// 1. Builds the outlier bit mask in shared memory; returns false when the
+// block's job has nothing to do.
+__device__ __forceinline__ bool mq_setup(const MQJob& j0, const MQJob& j1, int split, int64_t K,
+                                         const int32_t* __restrict__ idx, const int32_t* __restrict__ n_idx,
+                                         uint32_t* mask, MQJob& job, int64_t& b0, int64_t& nb, int& n) {
+    const bool second = (int)blockIdx.x >= split;
+    job = second ? j1 : j0;
+    b0 = second ? (int64_t)blockIdx.x - split : (int64_t)blockIdx.x;
+    nb = second ? (int64_t)gridDim.x - split : (int64_t)split;
+    if (job.only_if && *job.only_if == 0) return false;  // block-uniform
     const int64_t words = (K + 31) / 32;
     for (int64_t w = threadIdx.x; w < words; w += blockDim.x) mask[w] = 0u;
     __syncwarp();
     __syncthreads();
-    const int n = *n_idx;
+    n = *n_idx;
     for (int o = threadIdx.x; o < n; o += blockDim.x) {
         const int j = idx[o];
         atomicOr(&mask[j >> 5], 1u << (j & 31));
     }
     __syncwarp();
     __syncthreads();
+    return true;
+}
+
+template <typename T>
+__device__ __forceinline__ void write_xo(const MQJob& job, const T* x, int64_t row, const int32_t* idx, int n,
+                                         int lane) {
+    if (job.xo)  // fp32 copy of the outlier columns of this row, for the GEMM epilogue
+        for (int o = lane; o < n && o < kOutlierCap; o += 32) {
+            const uint16_t u = reinterpret_cast<const uint16_t*>(x)[idx[o]];
+            float f[8];
+            unpack<T>(make_uint4(u, 0, 0, 0), f);
+            job.xo[(int64_t)o * job.xo_ld + row] = f[0];
+        }
+}
+
+// One warp per row, the row read twice (any K).
+template <typename T>
+__global__ void __launch_bounds__(256)
+masked_quant_kernel(MQJob j0, MQJob j1, int split, int64_t K, const int32_t* __restrict__ idx,
+                    const int32_t* __restrict__ n_idx) {
+    pdl_wait();
+    pdl_trigger();
+    extern __shared__ uint32_t mask[];  // K bits
+    MQJob job;
+    int64_t b0, nb;
+    int n = 0;
+    if (!mq_setup(j0, j1, split, K, idx, n_idx, mask, job, b0, nb, n)) return;
+    const T* X = static_cast<const T*>(job.X);
     const int lane = threadIdx.x & 31;
-    const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
-    for (int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < M; row += nwarps) {
-        const T* x = X + row * ld;
+    const int64_t nwarps = nb * (blockDim.x >> 5);
+    for (int64_t row = (b0 * blockDim.x + threadIdx.x) >> 5; row < job.rows; row += nwarps) {
+        const T* x = X + row * job.ld;
         float m = 0.0f;
 #pragma unroll 4
         for (int64_t k0 = lane * 8; k0 < K; k0 += 256) {
@@ -239,16 +291,9 @@ masked_quant_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, c
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         const float qs = __fdiv_rn(127.0f, fmaxf(m, 1e-8f));
-        if (lane == 0) qs_out[row] = qs;
-        if (xo)  // fp32 copy of the outlier columns of this row, for the GEMM epilogue
-            for (int o = lane; o < n && o < kOutlierCap; o += 32) {
-                const uint16_t u = reinterpret_cast<const uint16_t*>(x)[idx[o]];
-                float f[8];
-                uint4 v = make_uint4(u, 0, 0, 0);
-                unpack<T>(v, f);
-                xo[(int64_t)o * xo_ld + row] = f[0];
-            }
-        int8_t* q = Q + row * K;
+        if (lane == 0) job.qs[row] = qs;
+        write_xo<T>(job, x, row, idx, n, lane);
+        int8_t* q = job.Q + row * K;
 #pragma unroll 4
         for (int64_t k0 = lane * 8; k0 < K; k0 += 256) {
             float f[8];
@@ -264,33 +309,23 @@ masked_quant_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, c
 }
 
 // The same with the row in registers (K <= 256 * CH): one read of X. Lane l
-// holds chunks l, l + 32, ... of 8 columns; X_O (when asked for) is written
-// o-major, xo[o * M + row], so the GEMM epilogue's reads are coalesced.
+// holds chunks l, l + 32, ... of 8 columns.
 template <typename T, int CH>
 __global__ void __launch_bounds__(256)
-masked_quant_reg_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld, const int32_t* __restrict__ idx,
-                        const int32_t* __restrict__ n_idx, const int32_t* __restrict__ only_if,
-                        int8_t* __restrict__ Q, float* __restrict__ qs_out, float* __restrict__ xo,
-                        int64_t xo_ld) {
+masked_quant_reg_kernel(MQJob j0, MQJob j1, int split, int64_t K, const int32_t* __restrict__ idx,
+                        const int32_t* __restrict__ n_idx) {
     pdl_wait();
     pdl_trigger();
     extern __shared__ uint32_t mask[];  // K bits
-    if (only_if && *only_if == 0) return;
-    const int64_t words = (K + 31) / 32;
-    for (int64_t w = threadIdx.x; w < words; w += blockDim.x) mask[w] = 0u;
-    __syncwarp();
-    __syncthreads();
-    const int n = *n_idx;
-    for (int o = threadIdx.x; o < n; o += blockDim.x) {
-        const int j = idx[o];
-        atomicOr(&mask[j >> 5], 1u << (j & 31));
-    }
-    __syncwarp();
-    __syncthreads();
+    MQJob job;
+    int64_t b0, nb;
+    int n = 0;
+    if (!mq_setup(j0, j1, split, K, idx, n_idx, mask, job, b0, nb, n)) return;
+    const T* X = static_cast<const T*>(job.X);
     const int lane = threadIdx.x & 31;
-    const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
-    for (int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < M; row += nwarps) {
-        const T* x = X + row * ld;
+    const int64_t nwarps = nb * (blockDim.x >> 5);
+    for (int64_t row = (b0 * blockDim.x + threadIdx.x) >> 5; row < job.rows; row += nwarps) {
+        const T* x = X + row * job.ld;
         uint4 raw[CH];
 #pragma unroll
         for (int i = 0; i < CH; ++i) {
@@ -312,15 +347,9 @@ masked_quant_reg_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t l
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         const float qs = __fdiv_rn(127.0f, fmaxf(m, 1e-8f));
-        if (lane == 0) qs_out[row] = qs;
-        if (xo)
-            for (int o = lane; o < n && o < kOutlierCap; o += 32) {
-                const uint16_t u = reinterpret_cast<const uint16_t*>(x)[idx[o]];
-                float f[8];
-                unpack<T>(make_uint4(u, 0, 0, 0), f);
-                xo[(int64_t)o * xo_ld + row] = f[0];
-            }
-        int8_t* q = Q + row * K;
+        if (lane == 0) job.qs[row] = qs;
+        write_xo<T>(job, x, row, idx, n, lane);
+        int8_t* q = job.Q + row * K;
 #pragma unroll
         for (int i = 0; i < CH; ++i) {
             const int64_t k0 = (int64_t)lane * 8 + 256 * i;
@@ -385,31 +414,43 @@ sq_status_t launch_detect(const void* X, sq_dtype_t dt, int64_t M, int64_t K, in
     return check_launch("sq_llmint8_detect");
 }
 
-sq_status_t launch_masked_quant(const void* X, sq_dtype_t dt, int64_t M, int64_t K, int64_t ldx, const int32_t* idx,
-                                const int32_t* n_idx, const int32_t* only_if, int8_t* Q, float* qs, cudaStream_t s,
-                                const char* name, float* xo = nullptr, int64_t xo_ld = 0) {
+// Blocks for one job: one warp per row, 8 warps per block, capped; a
+// conditional (weight-side) job usually returns at once, so it gets fewer.
+int64_t mq_blocks(const MQJob& j) {
+    int64_t grid = (j.rows + 7) / 8;
+    const int64_t cap = (int64_t)num_sms() * (j.only_if ? 2 : 8);
+    return grid > cap ? cap : grid;
+}
+
+// Launch the masked row quantisation for one job, or two in one launch.
+sq_status_t launch_masked_quant(sq_dtype_t dt, int64_t K, const int32_t* idx, const int32_t* n_idx, const MQJob& j0,
+                                const MQJob* j1, cudaStream_t s, const char* name) {
     const size_t smem = (size_t)((K + 31) / 32) * 4;
-    int64_t grid = (M + 7) / 8;  // one warp per row, 8 warps per block
-    // a conditional (weight-side) pass usually returns at once: fewer blocks
-    const int64_t cap = (int64_t)num_sms() * (only_if ? 2 : 8);
-    if (grid > cap) grid = cap;
-    if (grid < 1) return SQ_OK;
-    auto go = [&](auto k, auto* x) {
+    const int64_t g0 = j0.rows > 0 ? mq_blocks(j0) : 0;
+    const int64_t g1 = (j1 && j1->rows > 0) ? mq_blocks(*j1) : 0;
+    if (g0 + g1 < 1) return SQ_OK;
+    const MQJob second = (j1 && j1->rows > 0) ? *j1 : j0;
+    auto go = [&](auto k) {
         if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        launch_pdl(k, dim3((unsigned)grid), dim3(256), smem, s, x, M, K, ldx, idx, n_idx, only_if, Q, qs, xo, xo_ld);
+        launch_pdl(k, dim3((unsigned)(g0 + g1)), dim3(256), smem, s, j0, second, (int)g0, K, idx, n_idx);
     };
-    auto pick = [&](auto* x) {
-        using T = std::remove_const_t<std::remove_pointer_t<decltype(x)>>;
-        if (K <= 256) go(masked_quant_reg_kernel<T, 1>, x);
-        else if (K <= 512) go(masked_quant_reg_kernel<T, 2>, x);
-        else if (K <= 1024) go(masked_quant_reg_kernel<T, 4>, x);
-        else if (K <= 2048) go(masked_quant_reg_kernel<T, 8>, x);
-        else if (K <= 4096) go(masked_quant_reg_kernel<T, 16>, x);
-        else go(masked_quant_kernel<T>, x);
+    auto pick = [&](auto* tag) {
+        using T = std::remove_pointer_t<decltype(tag)>;
+        if (K <= 256) go(masked_quant_reg_kernel<T, 1>);
+        else if (K <= 512) go(masked_quant_reg_kernel<T, 2>);
+        else if (K <= 1024) go(masked_quant_reg_kernel<T, 4>);
+        else if (K <= 2048) go(masked_quant_reg_kernel<T, 8>);
+        else if (K <= 4096) go(masked_quant_reg_kernel<T, 16>);
+        else go(masked_quant_kernel<T>);
     };
-    if (dt == SQ_BF16) pick(static_cast<const __nv_bfloat16*>(X));
-    else pick(static_cast<const __half*>(X));
+    if (dt == SQ_BF16) pick(static_cast<__nv_bfloat16*>(nullptr));
+    else pick(static_cast<__half*>(nullptr));
     return check_launch(name);
+}
+
+MQJob mq_job(const void* X, int64_t rows, int64_t ld, int8_t* Q, float* qs, float* xo = nullptr, int64_t xo_ld = 0,
+             const int32_t* only_if = nullptr) {
+    return MQJob{X, rows, ld, Q, qs, xo, xo_ld, only_if};
 }
 
 sq_status_t check_x(const char* name, const void* X, sq_dtype_t dt, int64_t M, int64_t K, int64_t ldx) {
@@ -451,7 +492,8 @@ sq_status_t sq_llmint8_quant_rows(const void* X, sq_dtype_t dt, int64_t M, int64
     SQ_REQUIRE(idx && n_idx && ((Xq && qs_x) || M == 0), SQ_ERR_INVALID_ARG, "%s: null pointer", name);
     SQ_REQUIRE(sq::aligned16(Xq), SQ_ERR_ALIGNMENT, "%s: Xq not 16-byte aligned", name);
     if (M == 0) return SQ_OK;
-    return sq::launch_masked_quant(X, dt, M, K, ldx, idx, n_idx, nullptr, Xq, qs_x, sq::as_cuda(stream), name);
+    return sq::launch_masked_quant(dt, K, idx, n_idx, sq::mq_job(X, M, ldx, Xq, qs_x), nullptr, sq::as_cuda(stream),
+                                   name);
 }
 
 sq_status_t sq_llmint8_quant_weight(const void* W, sq_dtype_t dt, int64_t N, int64_t K, const int32_t* idx,
@@ -462,7 +504,8 @@ sq_status_t sq_llmint8_quant_weight(const void* W, sq_dtype_t dt, int64_t N, int
     SQ_REQUIRE(idx && n_idx && ((Wq && qs_w) || N == 0), SQ_ERR_INVALID_ARG, "%s: null pointer", name);
     SQ_REQUIRE(sq::aligned16(Wq), SQ_ERR_ALIGNMENT, "%s: Wq not 16-byte aligned", name);
     if (N == 0) return SQ_OK;
-    return sq::launch_masked_quant(W, dt, N, K, K, idx, n_idx, nullptr, Wq, qs_w, sq::as_cuda(stream), name);
+    return sq::launch_masked_quant(dt, K, idx, n_idx, sq::mq_job(W, N, K, Wq, qs_w), nullptr, sq::as_cuda(stream),
+                                   name);
 }
 
 sq_status_t sq_llmint8_matmul(const void* X, sq_dtype_t dt, int64_t M, int64_t K, int64_t ldx,
@@ -499,15 +542,14 @@ sq_status_t sq_llmint8_matmul(const void* X, sq_dtype_t dt, int64_t M, int64_t K
     st = sq::launch_detect(X, dt, M, K, ldx, threshold, min_ratio, idx_out, n_out, w->cached_idx, w->cached_n, workspace,
                            s);
     if (st != SQ_OK) return st;
-    // weight side for O (returns at once when O is unchanged); with a W_O
-    // buffer in the weight state the same pass refreshes it (wo[o, n] is
-    // W[n, O_o], written o-major like X_O)
-    st = sq::launch_masked_quant(w->W, dt, w->N, K, K, idx_out, n_out, changed, w->Wq, w->qs_w, s, name, w->wo, wo_ld);
+    // one launch: the row quantisation outside O (and the fp32 copy of the
+    // outlier columns of X), and the weight side for O, whose blocks return
+    // at once when O is unchanged; with a W_O buffer in the weight state the
+    // weight side refreshes it too (wo[o, n] is W[n, O_o], o-major like X_O)
+    const sq::MQJob wjob = sq::mq_job(w->W, w->N, K, w->Wq, w->qs_w, w->wo, wo_ld, changed);
+    st = sq::launch_masked_quant(dt, K, idx_out, n_out, sq::mq_job(X, M, ldx, Xq, qs_x, xo, M), &wjob, s, name);
     if (st != SQ_OK) return st;
     if (M == 0) return SQ_OK;
-    // row quantisation outside O (and the fp32 copy of the outlier columns of X)
-    st = sq::launch_masked_quant(X, dt, M, K, ldx, idx_out, n_out, nullptr, Xq, qs_x, s, name, xo, M);
-    if (st != SQ_OK) return st;
     // without a W_O buffer in the weight state: gather W_O into the workspace
     if (w->wo) {
         wo = w->wo;
