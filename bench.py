@@ -759,6 +759,83 @@ def json_line(args, world, r, shapes, tokens=None, cfg=None):
     return line
 
 
+# MLP chains of the configurations: (name, tokens, hidden, intermediate, act,
+# static per-tensor scale for FC2's input?, output dtype)
+MLP_CHAINS = (("c2_swiglu", 2048, 1024, 3072, 0, False, "bf16"),
+              ("c3_relu_static", 1024, 7168, 28672, 1, True, "fp16"),
+              ("c5_gelu", 4096, 12288, 49152, 2, False, "bf16"))
+
+
+def time_mlp_chains(args, dev, flush):
+    """The MLP of each configuration from an int8 input to the down/FC2
+    output, unfused (GEMM to 16-bit Y, the activation + int8 kernel, GEMM)
+    and with the activation in the first GEMM's epilogue (its 16-bit h, or
+    with a static scale its int8 codes, then GEMM). Synthetic int8 operands;
+    each chain one CUDA graph, timed after an L2 flush, mean of the replays."""
+    import torch
+
+    import w8a8_post_quantization_sq_b200 as sq
+
+    out = {}
+    stream = torch.cuda.Stream(device=dev)
+    for name, M, D, I, act, static, odt in MLP_CHAINS:
+        dt = torch.bfloat16 if odt == "bf16" else torch.float16
+        g = torch.Generator(device=dev).manual_seed(I)
+        N1 = 2 * I if act == 0 else I
+        ri = lambda *sh: torch.randint(-127, 128, sh, generator=g, device=dev, dtype=torch.int8)  # noqa: E731
+        Xq, W1, W2 = ri(M, D), ri(N1, D), ri(D, I)
+        qx = torch.rand(M, generator=g, device=dev) * 30 + 20
+        q1 = torch.rand(N1, generator=g, device=dev) * 300 + 200 * (D / 1024) ** 0.5
+        q2 = torch.rand(D, generator=g, device=dev) * 300 + 200 * (I / 1024) ** 0.5
+        Y = torch.empty((M, N1), dtype=dt, device=dev)
+        H = torch.empty((M, I), dtype=dt, device=dev)
+        X2 = torch.empty((M, I), dtype=torch.int8, device=dev)
+        qa = torch.empty(M if not static else 1, device=dev)
+        st = torch.tensor([8.0], device=dev) if static else None
+        Out = torch.empty((M, D), dtype=dt, device=dev)
+        ws1 = sq.workspace(sq.SQ_OP_GEMM, M, N1, D, device=dev)
+        ws2 = sq.workspace(sq.SQ_OP_GEMM, M, D, I, device=dev)
+
+        def unfused():
+            sq.sq_gemm_w8a8(Xq, W1, qx, q1, None, Y, ws1)
+            sq.sq_act_quant(Y, act, not static, st, X2, qa)
+            sq.sq_gemm_w8a8(X2, W2, qa, q2, None, Out, ws2)
+
+        def fused():
+            if static:
+                sq.sq_gemm_w8a8_act(Xq, W1, qx, q1, None, act, X2, ws1, static_qs=st, out_dtype=dt)
+                sq.sq_gemm_w8a8(X2, W2, st, q2, None, Out, ws2)
+            else:
+                sq.sq_gemm_w8a8_act(Xq, W1, qx, q1, None, act, H, ws1)
+                sq.sq_quantize_act(H, None, True, None, X2, qa)
+                sq.sq_gemm_w8a8(X2, W2, qa, q2, None, Out, ws2)
+
+        r = {"tokens": M, "hidden": D, "intermediate": I, "act": ["swiglu", "relu", "gelu"][act],
+             "fc2_input_scale": "static per-tensor" if static else "per token"}
+        for key, fn in (("unfused", unfused), ("fused", fused)):
+            with torch.cuda.stream(stream):
+                fn()
+            stream.synchronize()
+            reps = max(3, min(args.steps, 20))
+            graph = capture(fn, stream)
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+            with torch.cuda.stream(stream):
+                graph.replay()
+                for i in range(reps):
+                    flush(i)
+                    ev[i][0].record(stream)
+                    graph.replay()
+                    ev[i][1].record(stream)
+            torch.cuda.synchronize()
+            r[key + "_us"] = 1e3 * sum(a.elapsed_time(b) for a, b in ev) / reps
+            del graph
+        r["speedup"] = r["unfused_us"] / r["fused_us"]
+        out[name] = r
+        del Xq, W1, W2, Y, H, X2, Out
+        torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args, rank, world, dev):
     import torch
 
@@ -789,6 +866,8 @@ def run_ours(args, rank, world, dev):
             del s
             torch.cuda.empty_cache()
         line["configs"] = extra
+    if args.mlp_chains:
+        line["mlp_chains"] = time_mlp_chains(args, dev, flush)
     return line
 
 
@@ -1181,6 +1260,8 @@ def main():
     ap.add_argument("--sets", type=int, default=1, help="--kernel: input sets cycled back to back (1: flush each)")
     ap.add_argument("--workload", default=HEADLINE, choices=sorted(CONFIGS), help="the headline stack")
     ap.add_argument("--configs", default="c2,c3,c4", help="other stacks timed and reported under 'configs' (none: only the headline)")
+    ap.add_argument("--no-mlp-chains", dest="mlp_chains", action="store_false",
+                    help="skip the MLP chains (activation unfused / in the GEMM epilogue)")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)

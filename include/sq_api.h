@@ -66,8 +66,8 @@ typedef enum { SQ_F32 = 0, SQ_F16 = 1, SQ_BF16 = 2, SQ_I32 = 3, SQ_I8 = 4 } sq_d
 
 typedef enum { SQ_LAYERNORM = 0, SQ_RMSNORM = 1 } sq_norm_t;
 
-/* MLP activation feeding down_proj / FC2 (sq_act_quant). */
-typedef enum { SQ_ACT_SWIGLU = 0, SQ_ACT_RELU = 1 } sq_act_t;
+/* MLP activation feeding down_proj / FC2 (sq_act_quant, sq_gemm_w8a8_act). */
+typedef enum { SQ_ACT_SWIGLU = 0, SQ_ACT_RELU = 1, SQ_ACT_GELU = 2 } sq_act_t;
 
 typedef enum {
     SQ_OP_GEMM = 0,           /* sq_gemm_w8a8                               */
@@ -252,6 +252,11 @@ SQ_API sq_status_t sq_norm_smooth_quant(const void* H, sq_dtype_t dt, int64_t M,
  *   SQ_ACT_SWIGLU: A is [M, 2I] (stride lda >= 2I), gate = A[:, :I],
  *     up = A[:, I:]; h = silu(gate) * up, silu(g) = g / (1 + exp(-g)).
  *   SQ_ACT_RELU: A is [M, I] (stride lda >= I); h = max(A, 0).
+ *   SQ_ACT_GELU: A is [M, I]; h = gelu(A), the tanh form
+ *     0.5 a (1 + tanh(u)), u = c (a + 0.044715 a^3), c = sqrt(2/pi), written
+ *     a / (1 + exp(-2u)) (the same function) and evaluated as the fp32
+ *     sequence x3 = (a*a)*a; u = c * fma(k, x3, a); h = a / (1 + exp(-2u))
+ *     with c and k = 0.044715 rounded to fp32 and exp as below.
  *   exp is a fixed sequence of correctly rounded fp32 operations: n =
  *   rint(x * fp32(log2 e)), r = x - n*LN2_HI - n*LN2_LO (two fma, LN2_HI =
  *   2839/4096), exp(r) by the degree-7 Taylor polynomial in Horner form with
@@ -294,6 +299,35 @@ SQ_API sq_status_t sq_gemm_w8a8(const int8_t* Xq, const int8_t* Wq, int64_t M, i
                          const float* qs_x, int x_per_token, const float* qs_w, int w_per_channel,
                          const float* bias, sq_dtype_t out_dt, void* Y, int64_t ldy,
                          void* workspace, size_t ws_bytes, sq_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * INT8 GEMM with the MLP activation in its epilogue   [SQ-p2]
+ *     融入前序线性层的权重 (down_proj's input is act(gate) * up of the
+ *     gate/up projection's output; FC2's is act(fc1)); [SQ-p5] §2.1.
+ *   The GEMM of sq_gemm_w8a8 (same operands, scales, bias and workspace), whose
+ *   16-bit outputs Y (out_dt F16 or BF16, each one rounding of the fp32
+ *   dequantised value) are not written; instead:
+ *   SQ_ACT_SWIGLU: the weight's output channels come in interleaved pairs,
+ *     channel 2c the gate and 2c+1 the up projection of MLP channel c (N
+ *     even); H[i, c] = silu(Y[i, 2c]) * Y[i, 2c + 1], H is [M, N/2];
+ *   SQ_ACT_RELU / SQ_ACT_GELU: H[i, j] = act(Y[i, j]), H is [M, N];
+ *   each h computed in fp32 from the 16-bit Y values exactly as sq_act_quant
+ *   computes it (for the same Y, de-interleaved for SwiGLU). Then:
+ *   static_qs == NULL: H holds h rounded once to out_dt (16-bit elements, the
+ *     H_out of sq_act_quant); per-token int8 of H then comes from
+ *     sq_quantize_act;
+ *   static_qs != NULL (a device scale): H holds the int8 codes
+ *     clip(rne(h * qs), -127, 127) with the fp32 h, the codes sq_act_quant
+ *     gives with that static scale, and nothing else is written.
+ *   H has row stride ldh (elements). The [M, N] output Y never reaches
+ *   memory: for SwiGLU half the 16-bit bytes go out, with a static scale a
+ *   quarter (one byte per MLP channel, no second pass), and the activation's
+ *   arithmetic runs while the next tile's MMAs do.
+ * ------------------------------------------------------------------------ */
+SQ_API sq_status_t sq_gemm_w8a8_act(const int8_t* Xq, const int8_t* Wq, int64_t M, int64_t N, int64_t K,
+                                    const float* qs_x, int x_per_token, const float* qs_w, int w_per_channel,
+                                    const float* bias, sq_act_t act, const float* static_qs, sq_dtype_t out_dt,
+                                    void* H, int64_t ldh, void* workspace, size_t ws_bytes, sq_stream_t stream);
 
 /* --------------------------------------------------------------------------
  * Batched INT8 GEMM for attention     lpnh.cn SmoothQuant practice article

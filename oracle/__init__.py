@@ -71,6 +71,7 @@ def _declare(L):
     L.or_dequant_f64.argtypes = [_p, _i64, _i64, _i64, _p, _i, _p, _i, _p, _p]
     L.or_expf_array.argtypes = [_p, _i64, _p]
     L.or_silu_array.argtypes = [_p, _i64, _p]
+    L.or_gelu_array.argtypes = [_p, _i64, _p]
     L.or_act_quant.argtypes = [_p, _i64, _i64, _i64, _i, _i, _p, _p, _p, _p, _p]
     L.or_quantize_weight.argtypes = [_p, _i64, _i64, _i, _p, _p]
     L.or_quantize_act.argtypes = [_p, _i64, _i64, _i64, _p, _i, _p, _p, _p]
@@ -167,7 +168,7 @@ def fold_prev_linear(W, s, bias=None, round_f32=True):
 
 
 # ---------------------------------------------------------------- MLP activation + int8
-SWIGLU, RELU = 0, 1
+SWIGLU, RELU, GELU = 0, 1, 2
 
 
 def expf(x):
@@ -184,8 +185,15 @@ def silu(x):
     return out
 
 
+def gelu(x):
+    x = f32(np.atleast_1d(x))
+    out = np.empty_like(x)
+    lib().or_gelu_array(_ptr(x), x.size, _ptr(out))
+    return out
+
+
 def act_quant(A, act, per_token=True, static_qs=None, quantize=True, absmax=None, want_h=False):
-    """SwiGLU (A = [gate | up], [M, 2I]) or ReLU (A = [M, I]) then int8."""
+    """SwiGLU (A = [gate | up], [M, 2I]), ReLU or GELU (A = [M, I]) then int8."""
     A = f32(A)
     M, W = A.shape
     I = W // 2 if act == SWIGLU else W

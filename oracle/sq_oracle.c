@@ -202,6 +202,27 @@ float or_expf(float x) {
 
 float or_silu(float g) { return g / (1.0f + or_expf(-g)); }
 
+/* GELU, the tanh form 0.5 x (1 + tanh(u)), u = sqrt(2/pi) (x + 0.044715 x^3),
+ * that GPT-class MLPs use. Reading R15: the pages name GELU beside SwiGLU for
+ * the activation in front of FC2 but give no formula or evaluation; the tanh
+ * form is evaluated as a fixed fp32 sequence on the exp above, written as
+ * x / (1 + exp(-2u)) (the same function, since 1 + tanh(u) = 2 / (1 +
+ * exp(-2u)), without the cancellation of 1 + tanh for negative x), one
+ * rounding per step (fmaf for the inner polynomial). Pinned by: a library
+ * GELU (tanh form, fp64) within a small relative bound, gelu(x) - gelu(-x) =
+ * x to rounding, gelu(0) = 0, the limits x and 0, and the codes it decides
+ * against those of the fp64 GELU away from ties. */
+float or_gelu(float x) {
+    const float c = 0.7978845608028654f; /* sqrt(2/pi), rounded to fp32 */
+    const float k = 0.044715f;           /* rounded to fp32 */
+    const float x3 = (x * x) * x;
+    const float u = c * fmaf(k, x3, x);
+    return x / (1.0f + or_expf(-2.0f * u));
+}
+void or_gelu_array(const float* x, int64_t n, float* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = or_gelu(x[i]);
+}
+
 void or_expf_array(const float* x, int64_t n, float* out) {
     for (int64_t i = 0; i < n; ++i) out[i] = or_expf(x[i]);
 }
@@ -218,6 +239,7 @@ void or_act_quant(const float* A, int64_t M, int64_t I, int64_t ld, int act, int
         for (int64_t j = 0; j < I; ++j) {
             float v;
             if (act == 0) v = or_silu(a[j]) * a[I + j]; /* gate | up halves of the row */
+            else if (act == 2) v = or_gelu(a[j]);
             else v = a[j] > 0.0f ? a[j] : 0.0f;
             h[j] = v;
             const float av = absf(v);

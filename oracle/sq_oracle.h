@@ -56,6 +56,8 @@ void or_dequant_f64(const double* acc, int64_t r0, int64_t r1, int64_t N, const 
                     const float* qs_w, int w_per_channel, const float* bias, double* y);
 float or_expf(float x);
 float or_silu(float g);
+float or_gelu(float x);
+void or_gelu_array(const float* x, int64_t n, float* out);
 void or_expf_array(const float* x, int64_t n, float* out);
 void or_silu_array(const float* x, int64_t n, float* out);
 void or_act_quant(const float* A, int64_t M, int64_t I, int64_t ld, int act, int per_token,

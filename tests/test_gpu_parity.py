@@ -182,13 +182,15 @@ def _act_input(M, I, act, dtype, seed, extra_cols=0):
     A = rnd((M, width), seed, torch.float32, 2.0)
     A[0, :8] = torch.tensor([0.0, -0.0, 88.5, -88.5, 87.0, -87.0, 30.0, -30.0])
     A[min(1, M - 1), 3] = 200.0
+    if act == sq.SQ_ACT_GELU:
+        A[min(1, M - 1), :8] = torch.tensor([-10.0, -10.5, -4.0, 1e-20, -1e-20, 5e3, -5e3, 3.0])  # exp's edges
     if act == sq.SQ_ACT_RELU and M > 2:
         A[2] = -A[2].abs()  # an all-zero h row: scale from the 1e-8 floor
     return A.to(dtype)
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
-@pytest.mark.parametrize("act", [0, 1])
+@pytest.mark.parametrize("act", [0, 1, 2])
 @pytest.mark.parametrize("I,M", [(8, 5), (1000, 67), (3072, 300), (8192, 33), (9000, 21), (28672, 9)])
 def test_act_quant(dtype, act, I, M):
     """Codes, scales, the 16-bit h and the calibration maxima bit for bit; a

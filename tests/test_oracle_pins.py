@@ -607,6 +607,62 @@ def test_swiglu_quant_against_fp64(orc):
     assert np.max(np.abs(swapped - h64)) > 1.0
 
 
+def _gelu64(x, c, k):
+    """The tanh-form GELU in fp64, written x / (1 + exp(-2u)): the same
+    function as 0.5 x (1 + tanh(u)) without its cancellation for x < 0."""
+    x = np.asarray(x, np.float64)
+    u = c * (x + k * x ** 3)
+    with np.errstate(over="ignore"):
+        return x / (1.0 + np.exp(-2.0 * u))
+
+
+def test_gelu_against_fp64_and_library(orc):
+    """The fixed fp32 GELU (reading R15) against an fp64 evaluation with the
+    same fp32 constants (few ulp: only the sequence's roundings and exp's
+    error remain), against a library GELU (torch, tanh form, fp64, exact
+    constants) to 1e-5 relative where |gelu| > 1e-6, and its identities:
+    gelu(x) - gelu(-x) = x, gelu(0) = 0, gelu(x) = x and 0 far from 0. A
+    plausible mistake (the erf form, or a dropped cubic term) is far off."""
+    import math
+
+    c32, k32 = float(np.float32(math.sqrt(2 / math.pi))), float(np.float32(0.044715))
+    x = np.concatenate([np.linspace(-12, 12, 200001), np.geomspace(1e-30, 1e3, 5001),
+                        -np.geomspace(1e-30, 9.0, 5001)]).astype(np.float32)
+    g = orc.gelu(x).astype(np.float64)
+    g64 = _gelu64(x, c32, k32)
+    big = np.abs(g64) > 1e-30
+    # exp(z) carries the relative error of z times |z|: the bound grows with
+    # |2u| where exp(-2u) dominates (x < 0)
+    z = np.abs(2 * c32 * (x.astype(np.float64) + k32 * x.astype(np.float64) ** 3))
+    assert np.all(_ulps(g[big].astype(np.float32), g64[big]) <= 16.0 + 8.0 * z[big])
+    lib = torch.nn.functional.gelu(torch.from_numpy(x.astype(np.float64)), approximate="tanh").numpy()
+    m = np.abs(lib) > 1e-6
+    assert np.max(np.abs(g[m] - lib[m]) / np.abs(lib[m])) < 1e-5
+    d = g - orc.gelu(-x).astype(np.float64) - x.astype(np.float64)
+    assert np.all(np.abs(d) <= 4 * np.spacing(np.abs(x)).astype(np.float64) + 1e-38)
+    assert orc.gelu(np.float32(0.0))[0] == 0.0
+    assert orc.gelu(np.float32(40.0))[0] == np.float32(40.0) and orc.gelu(np.float32(-40.0))[0] == 0.0
+    erf_form = torch.nn.functional.gelu(torch.from_numpy(x.astype(np.float64))).numpy()
+    assert np.max(np.abs(erf_form - g)) > 1e-4
+    assert np.max(np.abs(_gelu64(x, c32, 0.0) - g)) > 1e-2
+
+
+def test_gelu_quant_against_fp64(orc):
+    """GELU then per-token int8: the codes those of the fp64 GELU wherever the
+    fp64 value is not within 1e-3 of a rounding tie."""
+    import math
+
+    rng = np.random.default_rng(31)
+    A = (rng.normal(size=(40, 256)) * 3).astype(np.float32)
+    r = orc.act_quant(A, orc.GELU, want_h=True)
+    h64 = _gelu64(A, float(np.float32(math.sqrt(2 / math.pi))), float(np.float32(0.044715)))
+    qs64 = 127.0 / np.max(np.abs(h64), axis=1)
+    assert np.max(np.abs(r["qs"] / qs64 - 1)) < 1e-6
+    t = h64 * qs64[:, None]
+    clear = np.abs(np.abs(t - np.floor(t)) - 0.5) > 1e-3
+    assert np.array_equal(r["Xq"][clear], np.rint(t)[clear].astype(np.int8))
+
+
 def test_relu_quant_bruteforce(orc):
     """ReLU MLP input: h = max(x, 0), then int8 per token or with a static scale."""
     rng = np.random.default_rng(31)

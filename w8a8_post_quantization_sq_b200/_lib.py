@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libsq_b200.so")
 
 SQ_F32, SQ_F16, SQ_BF16, SQ_I32, SQ_I8 = 0, 1, 2, 3, 4
 SQ_LAYERNORM, SQ_RMSNORM = 0, 1
-SQ_ACT_SWIGLU, SQ_ACT_RELU = 0, 1
+SQ_ACT_SWIGLU, SQ_ACT_RELU, SQ_ACT_GELU = 0, 1, 2
 SQ_OP_GEMM, SQ_OP_QUANT_ACT, SQ_OP_QUANT_WEIGHT, SQ_OP_LLMINT8_DETECT, SQ_OP_LLMINT8 = 0, 1, 2, 3, 4
 
 STATUS = {0: "SQ_OK", 1: "SQ_ERR_INVALID_ARG", 2: "SQ_ERR_UNSUPPORTED_SHAPE", 3: "SQ_ERR_ALIGNMENT",
@@ -68,6 +68,7 @@ SIGNATURES = {
     "sq_gemm_fp8": ([_p, _p, _i64, _i64, _i64, _p, _i, _p, _i, _p, _i, _p, _i64, _p, _sz, _p], _i),
     "sq_act_quant": ([_p, _i, _i64, _i64, _i64, _i, _i, _p, _p, _p, _p, _p, _p], _i),
     "sq_gemm_w8a8": ([_p, _p, _i64, _i64, _i64, _p, _i, _p, _i, _p, _i, _p, _i64, _p, _sz, _p], _i),
+    "sq_gemm_w8a8_act": ([_p, _p, _i64, _i64, _i64, _p, _i, _p, _i, _p, _i, _p, _i, _p, _i64, _p, _sz, _p], _i),
     "sq_llmint8_detect": ([_p, _i, _i64, _i64, _i64, _f, _d, _p, _p, _p, _sz, _p], _i),
     "sq_llmint8_detect_noalloc": ([_p, _i, _i64, _i64, _i64, _f, _d, _p, _p, _p], _i),
     "sq_llmint8_quant_rows": ([_p, _i, _i64, _i64, _i64, _p, _p, _p, _p, _p], _i),
@@ -332,7 +333,7 @@ def sq_gemm_fp8(Xq, Wq, qs_x, qs_w, bias, Y, ws, stream=None):
 
 # ---------------------------------------------------------------- MLP activation + int8
 def sq_act_quant(A, act, per_token, static_qs, Xq, qs_x, absmax=None, H=None, stream=None):
-    """A: [M, 2I] ([gate | up], SQ_ACT_SWIGLU) or [M, I] (SQ_ACT_RELU)."""
+    """A: [M, 2I] ([gate | up], SQ_ACT_SWIGLU) or [M, I] (SQ_ACT_RELU, SQ_ACT_GELU)."""
     M, W = A.shape
     I = W // 2 if act == SQ_ACT_SWIGLU else W
     if Xq is not None:
@@ -361,6 +362,33 @@ def sq_gemm_w8a8(Xq, Wq, qs_x, qs_w, bias, Y, ws, stream=None):
         _ptr(Xq), _ptr(Wq), M, N, K, _vec(qs_x, torch.float32), int(qs_x is not None and qs_x.numel() > 1),
         _vec(qs_w, torch.float32), int(qs_w is not None and qs_w.numel() > 1), _vec(bias, torch.float32, N),
         _dt(Y), _ptr(Y), _ld(Y), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def sq_gemm_w8a8_act(Xq, Wq, qs_x, qs_w, bias, act, H, ws, static_qs=None, out_dtype=None, stream=None):
+    """The int8 GEMM with the MLP activation in its epilogue: H [M, N/2]
+    (SwiGLU over interleaved gate/up channel pairs) or [M, N] (ReLU, GELU).
+    Without static_qs H is 16-bit (its dtype is the dtype the GEMM rounds Y
+    to); with a static scale H is int8 codes and out_dtype gives Y's dtype."""
+    M, K = Xq.shape
+    N = Wq.shape[0]
+    if Xq.dtype != torch.int8 or Wq.dtype != torch.int8 or not Xq.is_contiguous() or not Wq.is_contiguous():
+        raise ValueError("Xq and Wq must be contiguous int8")
+    width = N // 2 if act == SQ_ACT_SWIGLU else N
+    if Wq.shape[1] != K or H.shape[0] != M or H.shape[1] != width:
+        raise ValueError(f"shape mismatch: H must be [{M}, {width}]")
+    if static_qs is None:
+        _need(H.dtype in (torch.float16, torch.bfloat16), "H must be fp16 or bf16")
+        ydt = _dt(H)
+    else:
+        _need(H.dtype == torch.int8, "with a static scale H must be int8")
+        _need(out_dtype in (torch.float16, torch.bfloat16), "out_dtype (Y's dtype) must be fp16 or bf16")
+        ydt = SQ_F16 if out_dtype == torch.float16 else SQ_BF16
+    _scales(qs_x, M, "qs_x")
+    _scales(qs_w, N, "qs_w")
+    _check("sq_gemm_w8a8_act", lib().sq_gemm_w8a8_act(
+        _ptr(Xq), _ptr(Wq), M, N, K, _vec(qs_x, torch.float32), int(qs_x.numel() > 1), _vec(qs_w, torch.float32),
+        int(qs_w.numel() > 1), _vec(bias, torch.float32, N), int(act), _vec(static_qs, torch.float32, 1), ydt,
+        _ptr(H), _ld(H), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 # ---------------------------------------------------------------- LLM.int8() decomposition

@@ -1,5 +1,5 @@
-// The input of down_proj (FC2), act(gate) * up for a SwiGLU MLP or
-// relu(fc1) for a ReLU MLP, quantised to int8 per token or with a static
+// The input of down_proj (FC2), act(gate) * up for a SwiGLU MLP, relu(fc1)
+// for a ReLU MLP or gelu(fc1) for a GELU MLP, quantised to int8 per token or with a static
 // per-tensor scale; optional 16-bit copy of h and a running per-channel max of
 // |h| for calibration.
 //
@@ -9,16 +9,14 @@
 // 异常值与混合精度分解实战" §2.1). For a SwiGLU MLP the gate/up projection
 // writes one [M, 2I] row per token: gate in columns [0, I), up in [I, 2I).
 //
-// silu(g) = g / (1 + exp(-g)) with exp evaluated by a fixed fp32 sequence:
-// Cody-Waite reduction x = n ln2 + r (ln 2 in two parts, the high part
-// 2839/4096 so that n * LN2_HI is exact), then the Taylor polynomial of
-// exp(r) to degree 7 by Horner's rule with fma, then the exact scaling by
-// 2^n. Every step is one correctly rounded fp32 operation, so h, the scales
-// and the codes are bit-equal to a CPU evaluation of the same sequence.
+// silu and gelu are fixed sequences of correctly rounded fp32 operations
+// (sq_act.cuh), so h, the scales and the codes are bit-equal to a CPU
+// evaluation of the same sequence.
 //
 // One 256-thread block per row, rows strided over the grid. Up to I = 16384
 // the thread's h values stay in registers between the absmax and the codes;
 // longer rows compute h twice.
+#include "sq_act.cuh"
 #include "sq_common.cuh"
 
 namespace sq {
@@ -28,7 +26,7 @@ constexpr int kT = 256;
 
 struct ActArgs {
     int64_t M, I, lda;
-    int act;  // SQ_ACT_SWIGLU or SQ_ACT_RELU
+    int act;  // SQ_ACT_SWIGLU, SQ_ACT_RELU or SQ_ACT_GELU
     int per_token;
     const float* static_qs;
     int8_t* Xq;
@@ -36,30 +34,6 @@ struct ActArgs {
     float* absmax;  // [I] running max |h|, or null
     void* H;        // [M, I] 16-bit copy of h, or null
 };
-
-__device__ __forceinline__ float exp_fixed(float x) {
-    if (x > 88.0f) return __int_as_float(0x7f800000);
-    if (x < -87.0f) return 0.0f;
-    // n = x * log2(e) rounded to the nearest integer (ties to even): adding
-    // 1.5 * 2^23 rounds it into the low bits of the sum, which also hold n as
-    // an integer; this is rint() with two adds instead of conversions
-    const float sh = __fadd_rn(__fmul_rn(x, 0x1.715476p+0f), 12582912.0f);  // log2(e) in fp32
-    const float n = __fsub_rn(sh, 12582912.0f);                            // exact; in [-126, 127]
-    const int ni = __float_as_int(sh) - 0x4B400000;
-    float r = __fmaf_rn(-n, 0x1.62e000p-1f, x);            // ln 2, high part (12 bits)
-    r = __fmaf_rn(-n, 0x1.0bfbe8p-15f, r);                 // ln 2, low part
-    float p = 0x1.a01a02p-13f;                             // 1/7!
-    p = __fmaf_rn(p, r, 0x1.6c16c2p-10f);                  // 1/6!
-    p = __fmaf_rn(p, r, 0x1.111112p-7f);                   // 1/5!
-    p = __fmaf_rn(p, r, 0x1.555556p-5f);                   // 1/4!
-    p = __fmaf_rn(p, r, 0x1.555556p-3f);                   // 1/3!
-    p = __fmaf_rn(p, r, 0.5f);
-    p = __fmaf_rn(p, r, 1.0f);
-    p = __fmaf_rn(p, r, 1.0f);
-    return __fmul_rn(p, __int_as_float((ni + 127) << 23));
-}
-
-__device__ __forceinline__ float silu(float g) { return __fdiv_rn(g, __fadd_rn(1.0f, exp_fixed(-g))); }
 
 // h of the 8 channels starting at column c of row `row`
 template <typename T, int ACT>
@@ -71,7 +45,10 @@ __device__ __forceinline__ void act8(const T* __restrict__ A, const ActArgs& a, 
         float u[8];
         unpack<T>(ldg_nc_v4(r + a.I + c), u);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) h[e] = __fmul_rn(silu(x[e]), u[e]);
+        for (int e = 0; e < 8; ++e) h[e] = __fmul_rn(silu_fixed(x[e]), u[e]);
+    } else if constexpr (ACT == SQ_ACT_GELU) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) h[e] = gelu_fixed(x[e]);
     } else {
 #pragma unroll
         for (int e = 0; e < 8; ++e) h[e] = x[e] > 0.0f ? x[e] : 0.0f;
@@ -219,7 +196,8 @@ extern "C" sq_status_t sq_act_quant(const void* A, sq_dtype_t dt, int64_t M, int
     const char* name = "sq_act_quant";
     SQ_REQUIRE(A || M == 0, SQ_ERR_INVALID_ARG, "%s: null A", name);
     SQ_REQUIRE(dt == SQ_F16 || dt == SQ_BF16, SQ_ERR_INVALID_ARG, "%s: dtype must be F16 or BF16", name);
-    SQ_REQUIRE(act == SQ_ACT_SWIGLU || act == SQ_ACT_RELU, SQ_ERR_INVALID_ARG, "%s: bad activation", name);
+    SQ_REQUIRE(act == SQ_ACT_SWIGLU || act == SQ_ACT_RELU || act == SQ_ACT_GELU, SQ_ERR_INVALID_ARG,
+               "%s: bad activation", name);
     const int64_t width = act == SQ_ACT_SWIGLU ? 2 * I : I;
     SQ_REQUIRE(M >= 0 && I > 0 && I % 8 == 0 && lda >= width && lda % 8 == 0 && I <= (int64_t)1 << 24,
                SQ_ERR_UNSUPPORTED_SHAPE, "%s: need I > 0, I %% 8 == 0, lda >= %s, lda %% 8 == 0", name,
@@ -236,9 +214,11 @@ extern "C" sq_status_t sq_act_quant(const void* A, sq_dtype_t dt, int64_t M, int
     cudaStream_t s = sq::as_cuda(stream);
     if (dt == SQ_BF16) {
         if (act == SQ_ACT_SWIGLU) sq::launch_t<__nv_bfloat16, SQ_ACT_SWIGLU>(A, a, s);
+        else if (act == SQ_ACT_GELU) sq::launch_t<__nv_bfloat16, SQ_ACT_GELU>(A, a, s);
         else sq::launch_t<__nv_bfloat16, SQ_ACT_RELU>(A, a, s);
     } else {
         if (act == SQ_ACT_SWIGLU) sq::launch_t<__half, SQ_ACT_SWIGLU>(A, a, s);
+        else if (act == SQ_ACT_GELU) sq::launch_t<__half, SQ_ACT_GELU>(A, a, s);
         else sq::launch_t<__half, SQ_ACT_RELU>(A, a, s);
     }
     return sq::check_launch(name);

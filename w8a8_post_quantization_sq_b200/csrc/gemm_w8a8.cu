@@ -43,7 +43,9 @@
 #include <cudaTypedefs.h>
 
 #include <cstdlib>
+#include <type_traits>
 
+#include "sq_act.cuh"
 #include "sq_common.cuh"
 #include "sq_internal.h"
 #include "sq_wait.cuh"
@@ -61,6 +63,9 @@ constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr int kStgRow = 80;
 constexpr int kStgWarpBytes = 32 * kStgRow;
 enum OutKind { kOutBF16 = 0, kOutF16 = 1, kOutF32 = 2, kOutI32 = 3 };
+// activation applied to the 16-bit output in the epilogue (sq_gemm_w8a8_act):
+// none, or the sq_act_t value (SwiGLU on interleaved gate/up columns, ReLU, GELU)
+constexpr int kActNone = -1;
 // operand formats: int8 x int8 -> int32, or FP8 E4M3 x E4M3 -> fp32
 enum MmaKind { kKindI8 = 0, kKindF8 = 1 };
 
@@ -368,7 +373,13 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
 // term and bias), stage the chunk in shared memory, then write it out as
 // whole 64-byte row segments (four lanes per row for 16-bit outputs; 32-bit
 // outputs go out in two 16-column halves).
-template <int OUT, bool OUTL, int KIND>
+template <typename T16>
+__device__ __forceinline__ float round16(float v) {
+    if constexpr (std::is_same<T16, __nv_bfloat16>::value) return __bfloat162float(__float2bfloat16_rn(v));
+    else return __half2float(__float2half_rn(v));
+}
+
+template <int OUT, bool OUTL, int KIND, int ACT = kActNone>
 __device__ __forceinline__ void epi_chunk(const Params& p, const uint32_t* r, int cw, int col0, int row0, int64_t row,
                                           bool row_ok, float rx, const float* rw_w, const float* bias_w, uint8_t* stg,
                                           int lane, int n_out, bool compact, int prob) {
@@ -444,6 +455,85 @@ __device__ __forceinline__ void epi_chunk(const Params& p, const uint32_t* r, in
             }
         }
     }
+    if constexpr (ACT != kActNone) {
+        // the MLP activation on the 16-bit outputs Y this GEMM would write:
+        // SwiGLU on interleaved (gate, up) column pairs -> 16 values h for the
+        // chunk's 32 columns, ReLU or GELU -> 32 values; each h one rounding
+        using T16 = typename std::conditional<OUT == kOutBF16, __nv_bfloat16, __half>::type;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) y[e] = round16<T16>(y[e]);
+        constexpr int NH = ACT == SQ_ACT_SWIGLU ? 16 : 32;  // activation values of the chunk
+        if constexpr (ACT == SQ_ACT_SWIGLU) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) y[e] = __fmul_rn(silu_fixed(y[2 * e]), y[2 * e + 1]);
+        } else if constexpr (ACT == SQ_ACT_RELU) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) y[e] = y[e] > 0.0f ? y[e] : 0.0f;
+        } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) y[e] = gelu_fixed(y[e]);
+        }
+        if (ep.act_qs) {
+            // static per-tensor scale: the int8 codes of h, clipped, straight
+            // from the registers (each lane writes its row's NH bytes)
+            const float qs = *ep.act_qs;
+            uint32_t w[NH / 4];
+#pragma unroll
+            for (int e = 0; e < NH / 4; ++e)
+                w[e] = pack_low_bytes(quant_bits_clip(__fmul_rn(y[4 * e], qs)),
+                                      quant_bits_clip(__fmul_rn(y[4 * e + 1], qs)),
+                                      quant_bits_clip(__fmul_rn(y[4 * e + 2], qs)),
+                                      quant_bits_clip(__fmul_rn(y[4 * e + 3], qs)));
+            const int64_t nh = ACT == SQ_ACT_SWIGLU ? p.N / 2 : p.N;
+            const int64_t col = ACT == SQ_ACT_SWIGLU ? (int64_t)col0 / 2 : (int64_t)col0;
+            if (row_ok && col < nh) {
+                uint8_t* out = static_cast<uint8_t*>(ep.Y) + prob * p.y_bstride + row * ep.ldy + col;
+                if (p.vec_store && col + NH <= nh) {
+#pragma unroll
+                    for (int e = 0; e < NH / 16; ++e)
+                        reinterpret_cast<uint4*>(out)[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < NH; ++e)
+                        if (col + e < nh) out[e] = (uint8_t)(w[e >> 2] >> (8 * (e & 3)));
+                }
+            }
+            return;
+        }
+        if constexpr (ACT == SQ_ACT_SWIGLU) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) y[e] = round16<T16>(y[e]);
+            uint4* dst = reinterpret_cast<uint4*>(stg + lane * kStgRow);
+#pragma unroll
+            for (int e = 0; e < 2; ++e)
+                dst[e] = make_uint4(pack2<OUT>(y[8 * e], y[8 * e + 1]), pack2<OUT>(y[8 * e + 2], y[8 * e + 3]),
+                                    pack2<OUT>(y[8 * e + 4], y[8 * e + 5]), pack2<OUT>(y[8 * e + 6], y[8 * e + 7]));
+            __syncwarp();
+            // 32 rows x 32 bytes: two lanes per row segment
+            const int part = lane & 1;
+            const int64_t nh = p.N / 2;
+#pragma unroll
+            for (int it = 0; it < 2; ++it) {
+                const int rr = it * 16 + (lane >> 1);
+                const int64_t grow = (int64_t)row0 + rr;
+                const int64_t col = (int64_t)col0 / 2 + part * 8;
+                const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * kStgRow + part * 16);
+                if (grow < p.M && col < nh) {
+                    uint16_t* out = static_cast<uint16_t*>(ep.Y) + prob * p.y_bstride + grow * ep.ldy + col;
+                    if (p.vec_store && col + 8 <= nh) {
+                        *reinterpret_cast<uint4*>(out) = v;
+                    } else {
+                        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            if (col + e < nh) out[e] = (uint16_t)(w[e >> 1] >> (16 * (e & 1)));
+                    }
+                }
+            }
+            __syncwarp();
+            return;
+        }
+    }
     if constexpr (OUT == kOutBF16 || OUT == kOutF16) {
         uint4* dst = reinterpret_cast<uint4*>(stg + lane * kStgRow);
 #pragma unroll
@@ -504,7 +594,7 @@ __device__ __forceinline__ void epi_chunk(const Params& p, const uint32_t* r, in
     }
 }
 
-template <int BN, int OUT, bool OUTL, int KIND, bool SK, int CG>
+template <int BN, int OUT, bool OUTL, int KIND, bool SK, int CG, int ACT = kActNone>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                  const Params p) {
@@ -779,7 +869,7 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
                                     ra[4 * e + 3] += (uint32_t)v.w;
                                 }
                             }
-                            epi_chunk<OUT, OUTL, KIND>(p, ra, c * 32, c_base + c * 32, row0, row, row_ok, rx, rw_w,
+                            epi_chunk<OUT, OUTL, KIND, ACT>(p, ra, c * 32, c_base + c * 32, row0, row, row_ok, rx, rw_w,
                                                        bias_w, stg, lane, n_out, compact, b);
                         }
                         if (lane == 0) p.sk_cnt[u * kEpiWarps + wr] = 0;  // ready for the next launch
@@ -800,7 +890,7 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
                     else {
                         release_acc(acc);  // accumulator read in full
                     }
-                    epi_chunk<OUT, OUTL, KIND>(p, ra, c * 32, c_base + c * 32, row0, row, row_ok, rx, rw_w, bias_w, stg,
+                    epi_chunk<OUT, OUTL, KIND, ACT>(p, ra, c * 32, c_base + c * 32, row0, row, row_ok, rx, rw_w, bias_w, stg,
                                          lane, n_out, compact, b);
                     if (!more) break;
                     tmem_wait(rb);
@@ -809,7 +899,7 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
                     else {
                         release_acc(acc);
                     }
-                    epi_chunk<OUT, OUTL, KIND>(p, rb, (c + 1) * 32, c_base + (c + 1) * 32, row0, row, row_ok, rx, rw_w,
+                    epi_chunk<OUT, OUTL, KIND, ACT>(p, rb, (c + 1) * 32, c_base + (c + 1) * 32, row0, row, row_ok, rx, rw_w,
                                          bias_w, stg, lane, n_out, compact, b);
                     if (more2) tmem_wait(ra);
                 }
@@ -819,7 +909,7 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
                     if (c + 1 == nch) {
                         release_acc(acc);  // accumulator read in full
                     }
-                    epi_chunk<OUT, OUTL, KIND>(p, ra, c * 32, c_base + c * 32, row0, row, row_ok, rx, rw_w, bias_w, stg,
+                    epi_chunk<OUT, OUTL, KIND, ACT>(p, ra, c * 32, c_base + c * 32, row0, row, row_ok, rx, rw_w, bias_w, stg,
                                          lane, n_out, compact, b);
                 }
             }
@@ -900,8 +990,29 @@ KernelFn pick_kernel_sk(sq_dtype_t out_dt, bool outl, int kind) {
     }
 }
 
+// the fused-activation variants: 16-bit outputs, int8 operands, no outlier term
+template <int BN, bool SK, int CG>
+KernelFn pick_kernel_act(sq_dtype_t out_dt, int act) {
+    const bool bf = out_dt == SQ_BF16;
+    switch (act) {
+        case SQ_ACT_SWIGLU:
+            return bf ? gemm_w8a8_kernel<BN, kOutBF16, false, kKindI8, SK, CG, SQ_ACT_SWIGLU>
+                      : gemm_w8a8_kernel<BN, kOutF16, false, kKindI8, SK, CG, SQ_ACT_SWIGLU>;
+        case SQ_ACT_RELU:
+            return bf ? gemm_w8a8_kernel<BN, kOutBF16, false, kKindI8, SK, CG, SQ_ACT_RELU>
+                      : gemm_w8a8_kernel<BN, kOutF16, false, kKindI8, SK, CG, SQ_ACT_RELU>;
+        default:
+            return bf ? gemm_w8a8_kernel<BN, kOutBF16, false, kKindI8, SK, CG, SQ_ACT_GELU>
+                      : gemm_w8a8_kernel<BN, kOutF16, false, kKindI8, SK, CG, SQ_ACT_GELU>;
+    }
+}
+
 template <int BN, int CG>
-KernelFn pick_kernel(sq_dtype_t out_dt, bool outl, int kind, bool sk) {
+KernelFn pick_kernel(sq_dtype_t out_dt, bool outl, int kind, bool sk, int act) {
+    if (act != kActNone) {
+        if constexpr (CG == 2) return pick_kernel_act<BN, false, 2>(out_dt, act);
+        else return sk ? pick_kernel_act<BN, true, 1>(out_dt, act) : pick_kernel_act<BN, false, 1>(out_dt, act);
+    }
     if constexpr (CG == 2) return pick_kernel_sk<BN, false, 2>(out_dt, outl, kind);
     else
         return sk ? pick_kernel_sk<BN, true, 1>(out_dt, outl, kind) : pick_kernel_sk<BN, false, 1>(out_dt, outl, kind);
@@ -961,7 +1072,7 @@ sq_status_t launch_bn(const int8_t* Xq, const int8_t* Wq, int64_t M, int64_t N, 
     if (outl && ep.out_dt != SQ_BF16 && ep.out_dt != SQ_F16)
         return set_error(SQ_ERR_INVALID_ARG, "sq_gemm_w8a8: the outlier term needs a 16-bit output");
     const bool sk = CG == 1 && plan.sk_tiles > 0 && sk_ws != nullptr;
-    KernelFn fn = pick_kernel<BN, CG>(ep.out_dt, outl, ep.kind, sk);
+    KernelFn fn = pick_kernel<BN, CG>(ep.out_dt, outl, ep.kind, sk, ep.act);
     // the shared-memory opt-in is per kernel and per device; it is cheap, so set it every time
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM_ALLOC) != cudaSuccess)
         return check_launch("sq_gemm_w8a8: set shared memory size");
@@ -978,7 +1089,9 @@ sq_status_t launch_bn(const int8_t* Xq, const int8_t* Wq, int64_t M, int64_t N, 
     const int64_t per_mblock = (int64_t)BM * CG * K;
     int64_t g = (48ll << 20) / per_mblock;
     p.group_m = (int)(g < 1 ? 1 : (g > p.num_m ? p.num_m : g));
-    const int eb = (ep.out_dt == SQ_BF16 || ep.out_dt == SQ_F16) ? 2 : 4;
+    // bytes per output element: int8 codes from a fused activation with a
+    // static scale, else the output dtype's
+    const int eb = ep.act_qs ? 1 : (ep.out_dt == SQ_BF16 || ep.out_dt == SQ_F16) ? 2 : 4;
     p.vec_store = ((reinterpret_cast<uintptr_t>(ep.Y) & 15u) == 0) && ((ep.ldy * eb) % 16 == 0);
     p.ep = ep;
     p.status = status;
@@ -1157,5 +1270,41 @@ extern "C" sq_status_t sq_gemm_w8a8(const int8_t* Xq, const int8_t* Wq, int64_t 
     ep.out_dt = out_dt;
     ep.Y = Y;
     ep.ldy = ldy;
+    return sq::launch_gemm_w8a8(Xq, Wq, M, N, K, ep, static_cast<int*>(workspace), ws_bytes, sq::as_cuda(stream));
+}
+
+extern "C" sq_status_t sq_gemm_w8a8_act(const int8_t* Xq, const int8_t* Wq, int64_t M, int64_t N, int64_t K,
+                                        const float* qs_x, int x_per_token, const float* qs_w, int w_per_channel,
+                                        const float* bias, sq_act_t act, const float* static_qs, sq_dtype_t out_dt,
+                                        void* H, int64_t ldh, void* workspace, size_t ws_bytes, sq_stream_t stream) {
+    const char* name = "sq_gemm_w8a8_act";
+    SQ_REQUIRE((Xq || M == 0) && Wq && (H || M == 0) && qs_x && qs_w, SQ_ERR_INVALID_ARG,
+               "%s: null Xq, Wq, H or scales", name);
+    SQ_REQUIRE(act == SQ_ACT_SWIGLU || act == SQ_ACT_RELU || act == SQ_ACT_GELU, SQ_ERR_INVALID_ARG,
+               "%s: bad activation", name);
+    SQ_REQUIRE(out_dt == SQ_F16 || out_dt == SQ_BF16, SQ_ERR_INVALID_ARG, "%s: out dtype must be F16 or BF16", name);
+    SQ_REQUIRE(workspace && ws_bytes >= sq::kStatusBytes, SQ_ERR_INVALID_ARG, "%s: needs a workspace of %zu bytes",
+               name, sq::kStatusBytes);
+    const int64_t width = act == SQ_ACT_SWIGLU ? N / 2 : N;
+    SQ_REQUIRE(M >= 0 && N > 0 && K > 0 && ldh >= width, SQ_ERR_UNSUPPORTED_SHAPE, "%s: need N > 0, K > 0, ldh >= %s",
+               name, act == SQ_ACT_SWIGLU ? "N/2" : "N");
+    SQ_REQUIRE(act != SQ_ACT_SWIGLU || N % 2 == 0, SQ_ERR_UNSUPPORTED_SHAPE,
+               "%s: SwiGLU needs an even N (interleaved gate/up channel pairs)", name);
+    SQ_REQUIRE(K % 16 == 0, SQ_ERR_UNSUPPORTED_SHAPE, "%s: K must be a multiple of 16 (TMA row stride)", name);
+    SQ_REQUIRE(K <= 133144, SQ_ERR_UNSUPPORTED_SHAPE, "%s: K > 133144 could overflow the int32 accumulator", name);
+    SQ_REQUIRE(M < (1ll << 31) && N < (1ll << 31), SQ_ERR_UNSUPPORTED_SHAPE, "%s: M and N must be < 2^31", name);
+    SQ_REQUIRE(sq::aligned16(Xq) && sq::aligned16(Wq), SQ_ERR_ALIGNMENT, "%s: Xq and Wq must be 16-byte aligned", name);
+    if (M == 0) return SQ_OK;
+    sq::GemmEpilogue ep;
+    ep.qs_x = qs_x;
+    ep.x_per_token = x_per_token;
+    ep.qs_w = qs_w;
+    ep.w_per_channel = w_per_channel;
+    ep.bias = bias;
+    ep.out_dt = out_dt;
+    ep.Y = H;
+    ep.ldy = ldh;
+    ep.act = (int)act;
+    ep.act_qs = static_qs;
     return sq::launch_gemm_w8a8(Xq, Wq, M, N, K, ep, static_cast<int*>(workspace), ws_bytes, sq::as_cuda(stream));
 }

@@ -44,6 +44,8 @@ struct GemmEpilogue {
     const float* wo = nullptr;  // [kOutlierCap, wo_ld] fp32 copies of W[:, O]^T
     int64_t wo_ld = 0;          // multiple of 256, >= N
     int kind = 0;               // 0: int8 operands, int32 sums; 1: FP8 E4M3 operands, fp32 sums
+    int act = -1;               // sq_act_t applied to the 16-bit output (sq_gemm_w8a8_act), -1: none
+    const float* act_qs = nullptr;  // with act: a static per-tensor scale, Y then holds the int8 codes of h
     int64_t batch = 1;          // independent problems; operands [batch, rows, K], scales [batch, rows]
     int64_t y_bstride = 0;      // elements between the batches of Y
 };
