@@ -156,3 +156,30 @@ def test_pairs_llmint8_epilogue(monkeypatch):
         sq.sq_workspace_status(ws)
         out.append(Y)
     assert torch.equal(out[0].view(torch.int16), out[1].view(torch.int16))
+
+
+@pytest.mark.parametrize("act", [0, 1, 2])
+def test_pairs_fused_activation(act, monkeypatch):
+    """The fused activation on CTA pairs equals the single-CTA kernel's bit
+    for bit (16-bit h and static-scale codes)."""
+    M, N, K = 300, 1040, 1040
+    Xq, Wq = rand_i8((M, K), 81 + act), rand_i8((N, K), 82 + act)
+    g = torch.Generator().manual_seed(83)
+    qx = torch.rand(M, generator=g) * 30 + 20
+    qw = torch.rand(N, generator=g) * 300 + 200
+    Xd, Wd, qxd, qwd = Xq.to(DEV), Wq.to(DEV), qx.to(DEV), qw.to(DEV)
+    width = N // 2 if act == 0 else N
+    outs = []
+    for mode in ("1", "0"):
+        monkeypatch.setenv("SQ_GEMM_CTA_PAIRS", mode)
+        ws = sq.workspace(sq.SQ_OP_GEMM, M, N, K)
+        H = torch.empty((M, width), dtype=torch.bfloat16, device=DEV)
+        sq.sq_gemm_w8a8_act(Xd, Wd, qxd, qwd, None, act, H, ws)
+        Q = torch.empty((M, width), dtype=torch.int8, device=DEV)
+        sq.sq_gemm_w8a8_act(Xd, Wd, qxd, qwd, None, act, Q, ws, static_qs=torch.tensor([3.0], device=DEV),
+                            out_dtype=torch.bfloat16)
+        torch.cuda.synchronize()
+        sq.sq_workspace_status(ws)
+        outs.append((H, Q))
+    assert torch.equal(outs[0][0].view(torch.int16), outs[1][0].view(torch.int16))
+    assert torch.equal(outs[0][1], outs[1][1])
