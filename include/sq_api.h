@@ -120,7 +120,10 @@ SQ_API int sq_version(void);
  *   several linears (q/k/v, gate/up) call it on each, or on their
  *   concatenation; the result is one scale per input channel.
  * Requirements: X (W) 16-byte aligned; K and ldx multiples of 8 (16-bit)
- * or 4 (fp32). NaN inputs give an unspecified result.
+ * or 4 (fp32). NaN inputs give an unspecified result. Inputs of 16 MB and
+ * more stream through shared memory with bounded waits (about 2 s); a wait
+ * that gives up (not expected: the copies read the caller's input) leaves NaN
+ * in the maxima of the columns concerned, never a silently wrong value.
  * ------------------------------------------------------------------------ */
 SQ_API sq_status_t sq_calib_absmax(const void* X, sq_dtype_t dt, int64_t M, int64_t K, int64_t ldx,
                             float* xmax_inout, sq_stream_t stream);
@@ -237,7 +240,10 @@ SQ_API sq_status_t sq_scale_from_absmax(const float* absmax, int64_t n, float* q
  *   (calibration mode); V_out [M,K] (stride K) v rounded to dt.
  *   gamma_p (and beta_p) are the folded parameters from sq_fold_norm, or the
  *   original ones to calibrate. H: [M,K] dt in {F16, BF16}, stride ldh.
- *   K % 8 == 0, 8 <= K <= 16384.
+ *   K % 8 == 0, 8 <= K <= 16384. For K > 4096 rows stream through shared
+ *   memory with bounded waits (about 2 s); a wait that gives up (not
+ *   expected) leaves NaN in the scales of the rows not finished (the static
+ *   scale's copy in qs_x[0]) and in the calibration maxima.
  * ------------------------------------------------------------------------ */
 SQ_API sq_status_t sq_norm_smooth_quant(const void* H, sq_dtype_t dt, int64_t M, int64_t K, int64_t ldh,
                                  sq_norm_t norm, const float* gamma_p, const float* beta_p,

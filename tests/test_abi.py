@@ -147,6 +147,18 @@ def test_argument_validation_without_gpu(L):
     _expect(L, L.sq_quantize_weight(None, 7, 0, 16, None, 1, None, None, None, 0, None), 1, "dtype")
     _expect(L, L.sq_quantize_act(None, -1, 0, 16, 16, None, 1, None, None, None, None, 0, None), 1, "dtype")
     _expect(L, L.sq_fold_weight(p, 3, 0, 16, p, p, None), 1, "dtype")
+    # GEMM with the activation in its epilogue: bad activation, 32-bit output,
+    # odd N for interleaved gate/up pairs, H narrower than its width, null scales
+    _expect(L, L.sq_gemm_w8a8_act(p, p, 16, 16, 16, p, 1, p, 1, None, 7, None, 2, p, 16, p, 256, None), 1,
+            "activation")
+    _expect(L, L.sq_gemm_w8a8_act(p, p, 16, 16, 16, p, 1, p, 1, None, 1, None, 0, p, 16, p, 256, None), 1, "F16")
+    _expect(L, L.sq_gemm_w8a8_act(p, p, 16, 17, 16, p, 1, p, 1, None, 0, None, 2, p, 16, p, 256, None), 2, "even")
+    _expect(L, L.sq_gemm_w8a8_act(p, p, 16, 32, 16, p, 1, p, 1, None, 2, None, 2, p, 16, p, 256, None), 2, "ldh")
+    _expect(L, L.sq_gemm_w8a8_act(p, p, 16, 32, 16, None, 1, p, 1, None, 2, None, 2, p, 32, p, 256, None), 1,
+            "null")
+    assert L.sq_gemm_w8a8_act(p, p, 0, 32, 16, p, 1, p, 1, None, 0, None, 2, p, 16, p, 256, None) == 0
+    # act_quant: an unknown activation
+    _expect(L, L.sq_act_quant(p, 2, 4, 16, 16, 5, 1, None, p, p, None, None, None), 1, "activation")
     # M == 0 is a valid empty call (nothing launched)
     assert L.sq_gemm_w8a8(p, p, 0, 16, 16, p, 1, p, 1, None, 2, p, 16, p, 256, None) == 0
     assert L.sq_calib_absmax(p, 2, 0, 16, 16, p, None) == 0

@@ -221,9 +221,13 @@ col_absmax_bulk_kernel(const T* __restrict__ X, int64_t M, int64_t K, int64_t ld
                     if (global_ns() - t0 > kWaitNs / 4) break;
         }
     }
-    if (active && !aborted) {
+    if (active) {
+        // a band that gave up (not expected) publishes NaN for its columns:
+        // NaN's bits order above every finite value, so the maxima the host
+        // reads carry the failure
 #pragma unroll
-        for (int e = 0; e < TC; ++e) atomic_max_nonneg(out + c0 + t * TC + e, m[e]);
+        for (int e = 0; e < TC; ++e)
+            atomic_max_nonneg(out + c0 + t * TC + e, aborted ? __int_as_float(0x7fc00000) : m[e]);
     }
 }
 

@@ -444,6 +444,7 @@ norm_quant_bulk_kernel(const T* __restrict__ H, NormArgs a, int R) {
             if (r < a.M) issue_row(smem_u32(dsm + (size_t)i * row_bytes), H + r * a.ldh, row_bytes, smem_u32(&bars[i]));
         }
     bool aborted = false;
+    int64_t abort_row = a.M;  // first row this block did not finish
     int it = 0;
     for (int64_t row = blockIdx.x; row < a.M; row += G, ++it) {
         const int slot = it % R;
@@ -452,6 +453,7 @@ norm_quant_bulk_kernel(const T* __restrict__ H, NormArgs a, int R) {
         __syncwarp();
         if (__syncthreads_and(ok) == 0) {  // a copy never landed: give up (not expected)
             aborted = true;
+            abort_row = row;
             break;
         }
         auto chunk = [&](int c) { return *reinterpret_cast<const uint4*>(xs + (size_t)(t + c * kBlock) * 16); };
@@ -585,6 +587,22 @@ norm_quant_bulk_kernel(const T* __restrict__ H, NormArgs a, int R) {
                 while (!mbar_try_wait(smem_u32(&bars[i]), ph))
                     if (global_ns() - t0 > kWaitNs / 4) break;
         }
+    }
+    if (aborted) {
+        // the call's results are incomplete: say so in them. The scales of the
+        // rows this block did not finish (or the static scale) become NaN, and
+        // so do the calibration maxima, so the failure reaches the host in the
+        // outputs themselves (there is no workspace to carry a status word)
+        const float nan = __int_as_float(0x7fc00000);
+        if (a.Xq) {
+            if (a.per_token) {
+                for (int64_t r = abort_row + (int64_t)t * G; r < a.M; r += (int64_t)kBlock * G) a.qs_x[r] = nan;
+            } else if (t == 0) {
+                a.qs_x[0] = nan;
+            }
+        }
+        if (!QONLY && a.absmax)
+            for (int j = t; j < a.K; j += kBlock) amax_sh[j] = nan;  // NaN bits order above every finite value
     }
     if (!QONLY && a.absmax) {
         __syncwarp();
