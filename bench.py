@@ -476,6 +476,135 @@ class LlmInt8Stack:
         return 5  # counts, compaction, weight-side pass, row quantisation, GEMM
 
 
+class Fp8Stack:
+    """The 175B-shaped block's linear stack on FP8 units (E4M3 codes,
+    per-token and per-channel scales, fp32 tensor-core accumulation): the
+    smoothed per-token FP8 quantisation of both sides' [4096, 12288] bf16
+    linear inputs and the four GEMMs (out and FC2 on synthetic E4M3 inputs).
+    Offline: the int8 stack's calibration and smoothing factors, then the FP8
+    weights."""
+
+    def __init__(self, dev):
+        import torch
+
+        import w8a8_post_quantization_sq_b200 as sq
+
+        self.sq, self.torch, self.dev = sq, torch, dev
+        base = Stack("c5", dev)
+        with torch.cuda.stream(torch.cuda.Stream(device=dev)):
+            base.offline()
+        torch.cuda.synchronize()
+        self.base = base
+        self.M, self.K = base.M, base.K
+        self.s = {k: base.s[base.alpha][k] for k in base.sides}
+        self.W = base.W
+        self.gemms = base.cfg["gemms"]
+        u8 = lambda *sh: torch.empty(sh, dtype=torch.uint8, device=dev)  # noqa: E731
+        self.Wq = {w: u8(*self.W[w].shape) for w, _ in self.gemms}
+        self.qw = {w: torch.empty(self.W[w].shape[0], device=dev) for w, _ in self.gemms}
+        self.Xq = {k: u8(self.M, self.K) for k in base.sides}
+        self.qx = {k: torch.empty(self.M, device=dev) for k in base.sides}
+        g = torch.Generator(device=dev).manual_seed(77)
+        self.syn = {}
+        for w, src in self.gemms:
+            if src == "syn":
+                c = torch.randint(0, 256, (self.M, self.W[w].shape[1]), generator=g, device=dev, dtype=torch.int32)
+                c = torch.where((c & 0x7F) == 0x7F, c - 1, c).to(torch.uint8)  # no NaN codes
+                self.syn[w] = (c, torch.rand(self.M, generator=g, device=dev) + 1.0)
+        self.Y = base.Y
+        self.ws = base.ws
+        self.d = {}
+        self.bank = None
+        self.by_phase = False
+
+    launch = Stack.launch
+
+    def gemm_shapes(self):
+        return self.base.gemm_shapes()
+
+    def offline(self):
+        for w, src in self.gemms:
+            W = self.W[w]
+            s = None if src == "syn" else self.s[src]
+            self.launch("quantize_weight_fp8", ("hbm", W.numel() * (esize(W) + 1) + 4 * W.shape[0]),
+                        self.sq.sq_quantize_weight_fp8, W, s, True, self.Wq[w], self.qw[w])
+
+    def step(self):
+        sq, M, K = self.sq, self.M, self.K
+        for w, src in self.gemms:
+            if src == "syn":
+                xq, qx = self.syn[w]
+            else:
+                h = self.base.h[src]
+                self.launch("quantize_act_fp8", ("hbm", M * K * esize(h) + M * K + 4 * M), sq.sq_quantize_act_fp8, h,
+                            self.s[src], True, None, self.Xq[src], self.qx[src])
+                xq, qx = self.Xq[src], self.qx[src]
+            N, Kw = self.W[w].shape
+            ob = esize(self.Y[w])
+            self.launch("gemm_fp8", ("tensor", 2.0 * M * N * Kw, M * Kw + N * Kw + M * N * ob), sq.sq_gemm_fp8, xq,
+                        self.Wq[w], qx, self.qw[w], None, self.Y[w], self.ws[w])
+
+    def launches_per_step(self):
+        return 6
+
+
+class AttnStack:
+    """Attention's two products in int8 at the 175B-shaped block's head
+    layout (96 heads of 128 channels, 2048 tokens of one sequence): per-(head,
+    token) int8 of Q and K, the batched QK^T to bf16, per-(head, channel) int8
+    of V^T, and the batched PV on int8 probabilities (the softmax between
+    them is not on the path: P stands as synthetic int8 codes with per-row
+    scales)."""
+
+    def __init__(self, dev, heads=96, T=2048, d=128):
+        import torch
+
+        import w8a8_post_quantization_sq_b200 as sq
+
+        self.sq, self.torch, self.dev = sq, torch, dev
+        self.H, self.T, self.dh = heads, T, d
+        g = torch.Generator(device=dev).manual_seed(5)
+        bf = lambda *sh: torch.randn(sh, generator=g, device=dev).to(torch.bfloat16)  # noqa: E731
+        self.Q, self.Kt, self.Vt = bf(heads * T, d), bf(heads * T, d), bf(heads * d, T)
+        i8 = lambda *sh: torch.empty(sh, dtype=torch.int8, device=dev)  # noqa: E731
+        self.Qq, self.Kq, self.Vq = i8(heads, T, d), i8(heads, T, d), i8(heads, d, T)
+        self.qq, self.qk, self.qv = (torch.empty(n, device=dev) for n in (heads * T, heads * T, heads * d))
+        t = torch.randn((heads, T, T), generator=g, device=dev) * 40
+        self.Pq = t.round().clamp_(-127, 127).to(torch.int8)
+        del t
+        self.qp = torch.rand(heads * T, generator=g, device=dev) * 100 + 100
+        self.S = torch.empty((heads, T, T), dtype=torch.bfloat16, device=dev)
+        self.O = torch.empty((heads, T, d), dtype=torch.bfloat16, device=dev)
+        self.ws1 = sq.workspace(sq.SQ_OP_GEMM, T, T, d, device=dev)
+        self.ws2 = sq.workspace(sq.SQ_OP_GEMM, T, d, T, device=dev)
+        self.d = {}
+        self.bank = None
+        self.by_phase = False
+
+    launch = Stack.launch
+
+    def gemm_shapes(self):
+        return [(self.T, self.T, self.dh), (self.T, self.dh, self.T)]
+
+    def offline(self):
+        pass
+
+    def step(self):
+        sq, H, T, dh = self.sq, self.H, self.T, self.dh
+        for X, Xq, qs in ((self.Q, self.Qq, self.qq), (self.Kt, self.Kq, self.qk)):
+            self.launch("quantize_act", ("hbm", X.numel() * 3 + 4 * X.shape[0]), sq.sq_quantize_act, X, None, True,
+                        None, Xq.view(H * T, dh), qs)
+        self.launch("bmm_w8a8", ("tensor", 2.0 * H * T * T * dh, H * (2 * T * dh + 2 * T * T)), sq.sq_bmm_w8a8,
+                    self.Qq, self.Kq, self.qq.view(H, T), self.qk.view(H, T), self.S, self.ws1)
+        self.launch("quantize_act", ("hbm", self.Vt.numel() * 3 + 4 * self.Vt.shape[0]), sq.sq_quantize_act, self.Vt,
+                    None, True, None, self.Vq.view(H * dh, T), self.qv)
+        self.launch("bmm_w8a8", ("tensor", 2.0 * H * T * dh * T, H * (T * T + dh * T + 2 * T * dh)), sq.sq_bmm_w8a8,
+                    self.Pq, self.Vq, self.qp.view(H, T), self.qv.view(H, dh), self.O, self.ws2)
+
+    def launches_per_step(self):
+        return 5
+
+
 def summarise(bank, per_launch_ms, ipk, hbm):
     """Per-kernel figures from an instrumented replay: launches, mean time per
     launch, achieved throughput from the algorithmic work, and the fraction
@@ -695,10 +824,21 @@ def run_e2e(st, graph, args, world, dev, stream):
     return {"e2e_ms": e2e_ms, "h2d": h2d, "d2h": d2h, "e2e_steps": n}
 
 
+GEMM_TAGS = ("gemm_w8a8", "llmint8_matmul", "gemm_fp8", "bmm_w8a8")
+EXTRA_WORKLOADS = {
+    "c4": C4["workload"],
+    "c5_fp8": "175B-shaped block on FP8 units: smoothed per-token E4M3 quantisation of both sides' [4096, 12288] "
+              "bf16 linear inputs, QKV/out/FC1/FC2 E4M3 GEMMs to bf16 (weights E4M3 per channel, offline)",
+    "attn_int8": "attention products in int8 at the 175B-shaped head layout: 96 heads x 128 channels, 2048 tokens; "
+                 "per-(head, token) int8 of Q and K, batched QK^T to bf16, per-(head, channel) int8 of V^T, batched PV "
+                 "on synthetic int8 probabilities",
+}
+
+
 def gemm_roofline(r, shapes):
     """The dominant kernel's roofline: the int8 GEMM over its launches in one
     step (sum of 2MNK over sum of launch durations)."""
-    g = [k for k in r["kernels"] if k["kernel"] in ("gemm_w8a8", "llmint8_matmul")][0]
+    g = [k for k in r["kernels"] if k["kernel"] in GEMM_TAGS][0]
     ipk = r["ipk"]
     traffic = gemm_traffic(shapes)
     return {"bound": "tensor", "achieved": g["achieved"], "peak": ipk["burst"], "unit": "TOPS",
@@ -716,8 +856,8 @@ def gemm_roofline(r, shapes):
 
 def config_summary(name, r, tokens, world, shapes):
     """A compact line for a non-headline configuration."""
-    g = [k for k in r["kernels"] if k["kernel"] in ("gemm_w8a8", "llmint8_matmul")][0]
-    return {"workload": (CONFIGS[name]["workload"] if name in CONFIGS else C4["workload"]),
+    g = [k for k in r["kernels"] if k["kernel"] in GEMM_TAGS][0]
+    return {"workload": (CONFIGS[name]["workload"] if name in CONFIGS else EXTRA_WORKLOADS[name]),
             "tokens": tokens, "tokens_per_s": tokens * world / (r["ms_per_step"] * 1e-3),
             "ms_per_step": r["ms_per_step"], "gemm_tops": g["achieved"], "gemm_frac": g["frac"],
             "gemm_frac_nominal": g["frac_nominal"], "gemm_shapes": shapes, "kernels": r["kernels"],
@@ -850,15 +990,16 @@ def run_ours(args, rank, world, dev):
     torch.cuda.empty_cache()
     names = [c for c in args.configs.split(",") if c and c not in ("none", args.workload)]
     for c in names:
-        if c != "c4" and c not in CONFIGS:
+        if c not in EXTRA_WORKLOADS and c not in CONFIGS:
             raise SystemExit(f"unknown configuration {c}")
     if names:
         extra = {}
         for name in names:
-            if name == "c4":
-                s = LlmInt8Stack(dev)
+            if name in EXTRA_WORKLOADS:
+                s = {"c4": LlmInt8Stack, "c5_fp8": Fp8Stack, "attn_int8": AttnStack}[name](dev)
                 rr = run_stack(s, args, rank, world, dev, flush, e2e=False)
-                extra[name] = config_summary(name, rr, C4["tokens"], world, s.gemm_shapes())
+                tokens = {"c4": C4["tokens"], "c5_fp8": 4096, "attn_int8": 2048}[name]
+                extra[name] = config_summary(name, rr, tokens, world, s.gemm_shapes())
             else:
                 s = Stack(name, dev)
                 rr = run_stack(s, args, rank, world, dev, flush, e2e=False)
@@ -1259,7 +1400,8 @@ def main():
     ap.add_argument("--whole-tiles", action="store_true", help="--kernel gemm: a workspace without stream-K scratch")
     ap.add_argument("--sets", type=int, default=1, help="--kernel: input sets cycled back to back (1: flush each)")
     ap.add_argument("--workload", default=HEADLINE, choices=sorted(CONFIGS), help="the headline stack")
-    ap.add_argument("--configs", default="c2,c3,c4", help="other stacks timed and reported under 'configs' (none: only the headline)")
+    ap.add_argument("--configs", default="c2,c3,c4,c5_fp8,attn_int8",
+                    help="other stacks timed and reported under 'configs' (none: only the headline)")
     ap.add_argument("--no-mlp-chains", dest="mlp_chains", action="store_false",
                     help="skip the MLP chains (activation unfused / in the GEMM epilogue)")
     ap.add_argument("--gpus", type=int, default=1)

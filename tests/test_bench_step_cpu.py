@@ -186,3 +186,74 @@ def test_cpu_stack_runs_on_a_tiny_sample(name):
         tn, tg = c.step(T)
         assert tn > 0 and tg > 0
         assert c.full_step_s(tn, tg) > tn + tg
+
+
+def _recording_stack(cls):
+    st = object.__new__(cls)
+    st.sq = RecordingSQ()
+    st.bank = None
+    st.by_phase = False
+    return st
+
+
+def _t(*shape, es=2):
+    t = mock.MagicMock()
+    t.shape = shape
+    t.element_size.return_value = es
+    n = 1
+    for s in shape:
+        n *= s
+    t.numel.return_value = n
+    t.view.return_value = t
+    return t
+
+
+def test_fp8_stack_launch_claim():
+    """The FP8 stack: one E4M3 quantisation per smoothed side and the four
+    E4M3 GEMMs, each one kernel."""
+    st = _recording_stack(bench.Fp8Stack)
+    st.M, st.K = 8, 16
+    st.gemms = bench.CONFIGS["c5"]["gemms"]
+    st.W = {w: _t(32, 16, es=4) for w, _ in st.gemms}
+    st.base = types.SimpleNamespace(h={"attn": _t(8, 16), "mlp": _t(8, 16)})
+    st.s = {"attn": _t(16), "mlp": _t(16)}
+    st.Xq = {k: _t(8, 16, es=1) for k in ("attn", "mlp")}
+    st.qx = {k: _t(8, es=4) for k in ("attn", "mlp")}
+    st.syn = {w: (_t(8, 16, es=1), _t(8, es=4)) for w, src in st.gemms if src == "syn"}
+    st.Y = {w: _t(8, 32) for w, _ in st.gemms}
+    st.Wq = {w: _t(32, 16, es=1) for w, _ in st.gemms}
+    st.qw = {w: _t(32, es=4) for w, _ in st.gemms}
+    st.ws = {w: _t(256, es=1) for w, _ in st.gemms}
+    bench.Fp8Stack.step(st)
+    c = st.sq.calls
+    assert c.count("sq_quantize_act_fp8") == 2 and c.count("sq_gemm_fp8") == 4
+    assert len(c) == bench.Fp8Stack.launches_per_step(st)
+
+
+def test_attention_stack_launch_claim():
+    """The attention products: int8 of Q, K and V^T and the two batched
+    GEMMs, each one kernel; the QK^T work is 2 H T^2 d."""
+    st = _recording_stack(bench.AttnStack)
+    H, T, d = 2, 32, 16
+    st.H, st.T, st.dh = H, T, d
+    for k in ("Q", "Kt"):
+        setattr(st, k, _t(H * T, d))
+    st.Vt = _t(H * d, T)
+    for k in ("Qq", "Kq", "Vq", "Pq", "qq", "qk", "qv", "qp", "S", "O", "ws1", "ws2"):
+        setattr(st, k, _t(4))
+
+    class Bank:
+        def __init__(self):
+            self.pairs = []
+
+        def pair(self, tag, work):
+            self.pairs.append((tag, work))
+            return mock.MagicMock(), mock.MagicMock()
+
+    st.bank = Bank()
+    bench.AttnStack.step(st)
+    c = st.sq.calls
+    assert c.count("sq_quantize_act") == 3 and c.count("sq_bmm_w8a8") == 2
+    assert len(c) == bench.AttnStack.launches_per_step(st)
+    bmm = [w for t, w in st.bank.pairs if t == "bmm_w8a8"]
+    assert bmm[0][1] == 2.0 * H * T * T * d and bmm[1][1] == 2.0 * H * T * d * T
