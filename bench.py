@@ -594,11 +594,14 @@ class AttnStack:
         for X, Xq, qs in ((self.Q, self.Qq, self.qq), (self.Kt, self.Kq, self.qk)):
             self.launch("quantize_act", ("hbm", X.numel() * 3 + 4 * X.shape[0]), sq.sq_quantize_act, X, None, True,
                         None, Xq.view(H * T, dh), qs)
-        self.launch("bmm_w8a8", ("tensor", 2.0 * H * T * T * dh, H * (2 * T * dh + 2 * T * T)), sq.sq_bmm_w8a8,
+        # both products are bound by HBM at this head dimension (2 T^2 d operations
+        # against the 2 T^2 bytes of S or the T^2 of P: 128 and 256 operations per
+        # byte, under the int8 ridge of ~500): judged by their bytes
+        self.launch("bmm_qk", ("hbm", H * (2 * T * dh + 2 * T * T + 8 * T)), sq.sq_bmm_w8a8,
                     self.Qq, self.Kq, self.qq.view(H, T), self.qk.view(H, T), self.S, self.ws1)
         self.launch("quantize_act", ("hbm", self.Vt.numel() * 3 + 4 * self.Vt.shape[0]), sq.sq_quantize_act, self.Vt,
                     None, True, None, self.Vq.view(H * dh, T), self.qv)
-        self.launch("bmm_w8a8", ("tensor", 2.0 * H * T * dh * T, H * (T * T + dh * T + 2 * T * dh)), sq.sq_bmm_w8a8,
+        self.launch("bmm_pv", ("hbm", H * (T * T + dh * T + 2 * T * dh + 4 * (T + dh))), sq.sq_bmm_w8a8,
                     self.Pq, self.Vq, self.qp.view(H, T), self.qv.view(H, dh), self.O, self.ws2)
 
     def launches_per_step(self):
@@ -824,7 +827,7 @@ def run_e2e(st, graph, args, world, dev, stream):
     return {"e2e_ms": e2e_ms, "h2d": h2d, "d2h": d2h, "e2e_steps": n}
 
 
-GEMM_TAGS = ("gemm_w8a8", "llmint8_matmul", "gemm_fp8", "bmm_w8a8")
+GEMM_TAGS = ("gemm_w8a8", "llmint8_matmul", "gemm_fp8", "bmm_qk")
 EXTRA_WORKLOADS = {
     "c4": C4["workload"],
     "c5_fp8": "175B-shaped block on FP8 units: smoothed per-token E4M3 quantisation of both sides' [4096, 12288] "
@@ -857,11 +860,15 @@ def gemm_roofline(r, shapes):
 def config_summary(name, r, tokens, world, shapes):
     """A compact line for a non-headline configuration."""
     g = [k for k in r["kernels"] if k["kernel"] in GEMM_TAGS][0]
-    return {"workload": (CONFIGS[name]["workload"] if name in CONFIGS else EXTRA_WORKLOADS[name]),
-            "tokens": tokens, "tokens_per_s": tokens * world / (r["ms_per_step"] * 1e-3),
-            "ms_per_step": r["ms_per_step"], "gemm_tops": g["achieved"], "gemm_frac": g["frac"],
-            "gemm_frac_nominal": g["frac_nominal"], "gemm_shapes": shapes, "kernels": r["kernels"],
-            "offline": r["offline"], "clocks": r["clocks"]}
+    out = {"workload": (CONFIGS[name]["workload"] if name in CONFIGS else EXTRA_WORKLOADS[name]),
+           "tokens": tokens, "tokens_per_s": tokens * world / (r["ms_per_step"] * 1e-3),
+           "ms_per_step": r["ms_per_step"], "gemm_bound": g["bound"], "gemm_frac": g["frac"],
+           "gemm_shapes": shapes, "kernels": r["kernels"], "offline": r["offline"], "clocks": r["clocks"]}
+    if g["bound"] == "tensor":
+        out.update({"gemm_tops": g["achieved"], "gemm_frac_nominal": g["frac_nominal"]})
+    else:
+        out["gemm_gbs"] = g["achieved"]
+    return out
 
 
 def json_line(args, world, r, shapes, tokens=None, cfg=None):
@@ -1217,7 +1224,8 @@ def run_reference(args, rank, world):
 # ------------------------------------------------------------------ single kernels
 def run_kernel(args):
     """Time one entry point alone on one shape:
-    gemm M,N,K | gemm_fp8 M,N,K | norm M,K | absmax M,K | act M,I | quant_weight N,K | llmint8 M,K,N.
+    gemm M,N,K | gemm_fp8 M,N,K | bmm B,M,N,K | norm M,K | absmax M,K | act M,I | quant_weight N,K |
+    llmint8 M,K,N.
     --sets 1: every launch after an L2 flush, each launch timed on its own.
     --sets S > 1: S distinct input/output sets, launches cycling through them
     back to back (one flush before the run); the time per launch is the run's
@@ -1265,6 +1273,15 @@ def run_kernel(args):
             Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
             ws = sq.workspace(sq.SQ_OP_GEMM, M, N, K, device=dev)
             return lambda: sq.sq_gemm_fp8(Xq, Wq, qx, qw, None, Y, ws)
+        if args.kernel == "bmm":
+            B, M, N, K = shape
+            Aq = torch.randint(-127, 128, (B, M, K), generator=g, device=dev, dtype=torch.int8)
+            Bq = torch.randint(-127, 128, (B, N, K), generator=g, device=dev, dtype=torch.int8)
+            qa = torch.rand(B * M, generator=g, device=dev) + 1
+            qb = torch.rand(B * N, generator=g, device=dev) + 100
+            Y = torch.empty((B, M, N), dtype=torch.bfloat16, device=dev)
+            ws = sq.workspace(sq.SQ_OP_GEMM, M, N, K, device=dev)
+            return lambda: sq.sq_bmm_w8a8(Aq, Bq, qa, qb, Y, ws)
         if args.kernel == "norm":
             M, K = shape
             dt16 = torch.float16 if args.dtype == "fp16" else torch.bfloat16
@@ -1317,6 +1334,13 @@ def run_kernel(args):
         # dense int8 and fp8 peaks are both twice the bf16 one (4.5 vs 2.25 PFLOP/s nominal)
         work, unit, peak = 2.0 * M * N * K / 1e12, "TOPS", ipk["burst"]
         out["whole_tiles"] = bool(args.whole_tiles)
+    elif args.kernel == "bmm":
+        B, M, N, K = shape
+        # int8 operands, bf16 output, fp32 row scales: the bytes that must cross HBM once
+        nbytes = B * (M * K + N * K + 2 * M * N + 4 * (M + N))
+        work, unit, peak = nbytes / 1e9, "GB/s", pk["hbm_gbs"]
+        out["ops"] = 2.0 * B * M * N * K
+        out["bytes"] = nbytes
     elif args.kernel == "norm":
         M, K = shape
         work, unit, peak = (3.0 * M * K + 4 * M) / 1e9, "GB/s", pk["hbm_gbs"]
@@ -1387,6 +1411,8 @@ def run_kernel(args):
                 "peak": peak, "frac": ach / peak, "peak_source": src, "clocks": clk})
     if unit == "TOPS":
         out.update({"frac_sustained": ach / ipk["sustained"], "frac_nominal": ach / ipk["nominal"]})
+    if "ops" in out:
+        out["tops"] = out["ops"] / (avg * 1e-3) / 1e12
     print(json.dumps(out), flush=True)
 
 

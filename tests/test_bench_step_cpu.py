@@ -232,7 +232,7 @@ def test_fp8_stack_launch_claim():
 
 def test_attention_stack_launch_claim():
     """The attention products: int8 of Q, K and V^T and the two batched
-    GEMMs, each one kernel; the QK^T work is 2 H T^2 d."""
+    GEMMs, each one kernel."""
     st = _recording_stack(bench.AttnStack)
     H, T, d = 2, 32, 16
     st.H, st.T, st.dh = H, T, d
@@ -255,5 +255,7 @@ def test_attention_stack_launch_claim():
     c = st.sq.calls
     assert c.count("sq_quantize_act") == 3 and c.count("sq_bmm_w8a8") == 2
     assert len(c) == bench.AttnStack.launches_per_step(st)
-    bmm = [w for t, w in st.bank.pairs if t == "bmm_w8a8"]
-    assert bmm[0][1] == 2.0 * H * T * T * d and bmm[1][1] == 2.0 * H * T * d * T
+    tags = dict(st.bank.pairs)
+    # both products judged by their bytes: S written in bf16, P read in int8
+    assert tags["bmm_qk"] == ("hbm", H * (2 * T * d + 2 * T * T + 8 * T))
+    assert tags["bmm_pv"] == ("hbm", H * (T * T + d * T + 2 * T * d + 4 * (T + d)))

@@ -26,9 +26,12 @@
 //   - warps 2..9 read the accumulator with tcgen05.ld (warp w owns TMEM lanes
 //     32*(w%4)..+31 = tile rows, and half of the columns), double-buffering
 //     the loads, dequantise in fp32, stage 32 x 32 chunks in shared memory
-//     and write whole row segments, while the next tile's MMAs run in the
-//     other accumulator buffer; the buffer is released right after its
-//     last load.
+//     and write them out while the next tile's MMAs run in the other
+//     accumulator buffer; the buffer is released right after its last load.
+//     16-bit outputs with 16-byte aligned rows leave by TMA store (one
+//     cp.async.bulk.tensor per chunk from a 64-byte-swizzled staging box,
+//     rows and columns past the edge clipped by the copy engine); the
+//     others by whole row segments of plain stores.
 // Batched variant (lpnh.cn SmoothQuant practice article §2.2: the QK^T and PV
 // products of attention can run in int8): problem b of a [batch, M, K] x
 // [batch, N, K] pair through 3-D tensor maps, its own row scales (one per
@@ -43,6 +46,7 @@
 #include <cudaTypedefs.h>
 
 #include <cstdlib>
+#include <cstring>
 #include <type_traits>
 
 #include "sq_act.cuh"
@@ -60,8 +64,13 @@ constexpr int kEpiWarps = 8;  // two per TMEM lane quarter, each on half the til
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 // staging: 32 rows x 64 B of data (32 16-bit or 16 32-bit values) + 16 B pad
+// for the plain stores; the TMA-store box uses the first 2 KB of the same
+// slot unpadded (64-byte swizzle), so slots start on 512-byte boundaries.
+// (Two boxes per warp, one filled while the other is read out, measured no
+// faster on B200 and need a pair's sixth ring stage.)
 constexpr int kStgRow = 80;
 constexpr int kStgWarpBytes = 32 * kStgRow;
+static_assert(kStgWarpBytes % 512 == 0, "staging slots must keep the 64-byte swizzle's 512-byte alignment");
 enum OutKind { kOutBF16 = 0, kOutF16 = 1, kOutF32 = 2, kOutI32 = 3 };
 // activation applied to the 16-bit output in the epilogue (sq_gemm_w8a8_act):
 // none, or the sq_act_t value (SwiGLU on interleaved gate/up columns, ReLU, GELU)
@@ -89,10 +98,11 @@ struct Cfg {
     static constexpr uint32_t RW_OFF = (MISC_OFF + 16 + 15) / 16 * 16;
     static constexpr uint32_t RW_BYTES = kEpiWarps * 2 * (BN / 2) * 4;
     // per epilogue warp: a 32 x 32 output chunk (rows padded to avoid bank conflicts)
-    static constexpr uint32_t STG_OFF = RW_OFF + RW_BYTES;
+    static constexpr uint32_t STG_OFF = (RW_OFF + RW_BYTES + 1023) / 1024 * 1024;
     static constexpr uint32_t STG_BYTES = kEpiWarps * kStgWarpBytes;
     static constexpr uint32_t SMEM = STG_OFF + STG_BYTES;
     static constexpr uint32_t SMEM_ALLOC = SMEM + 1024;  // slack to align the base to 1024
+    static_assert(SMEM_ALLOC <= 232448, "over the 227 KB of shared memory a block may use");
     static constexpr uint32_t TMEM_COLS = 2 * BN;
     // kind::i8: D = s32 (bits 4-5 = 2), A = B = signed 8-bit (bits 7-9, 10-12 = 1);
     // kind::f8f6f4: D = f32 (bits 4-5 = 1), A = B = E4M3 (format 0);
@@ -110,6 +120,7 @@ struct Params {
     int num_m, num_n, num_kb;
     int group_m;    // m-blocks per raster group
     int vec_store;  // Y rows start on 16-byte boundaries
+    int tma_store;  // 16-bit Y written by TMA store through the Y tensor map
     GemmEpilogue ep;
     int* status;
     // Stream-K (one problem only): the first dp_tiles tiles in raster order
@@ -230,6 +241,23 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
     }
 }
 
+// Store a 32 x 32 box of 16-bit outputs (x = column, y = row, z = problem)
+// from this CTA's shared memory; elements outside the tensor are not written.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int x, int y, int z) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];"
+                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(src), "r"(x), "r"(y), "r"(z)
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// this thread's bulk stores have finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read_all() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// this thread's bulk stores have completed
+__device__ __forceinline__ void bulk_wait_all() {
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- CTA pairs
 __device__ __forceinline__ uint32_t cluster_rank() {
     uint32_t r;
@@ -248,9 +276,16 @@ __device__ __forceinline__ void cluster_sync_all() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 // Arrive on an mbarrier given by its shared::cluster address (possibly the
-// other CTA's), releasing this thread's prior accesses at cluster scope.
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+// other CTA's), with the arrive's default semantics. It hands an accumulator
+// buffer back to the pair's MMA issuer: the tensor-memory reads it orders
+// have completed (tcgen05.wait::ld) and are fenced by
+// tcgen05.fence::before_thread_sync, and the issuer's wait is followed by
+// tcgen05.fence::after_thread_sync. A release at cluster scope would first
+// order every earlier memory access of this thread at that scope, a fence per
+// tile that showed up as membar stalls (measured on B200: the int8 QK^T
+// product at 96 x 2048 x 2048 x 128 took 302 us with it, 264 us without).
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 // UMMA shared-memory descriptor, K-major operand with 128-byte swizzle: rows of
@@ -382,7 +417,7 @@ __device__ __forceinline__ float round16(float v) {
 template <int OUT, bool OUTL, int KIND, int ACT = kActNone>
 __device__ __forceinline__ void epi_chunk(const Params& p, const uint32_t* r, int cw, int col0, int row0, int64_t row,
                                           bool row_ok, float rx, const float* rw_w, const float* bias_w, uint8_t* stg,
-                                          int lane, int n_out, bool compact, int prob) {
+                                          int lane, int n_out, bool compact, int prob, const CUtensorMap* tmap_y) {
     const GemmEpilogue& ep = p.ep;
     float y[32];
     if constexpr (OUT == kOutI32) {
@@ -535,6 +570,25 @@ __device__ __forceinline__ void epi_chunk(const Params& p, const uint32_t* r, in
         }
     }
     if constexpr (OUT == kOutBF16 || OUT == kOutF16) {
+        if (p.tma_store) {
+            // the previous chunk's store has read the box; refill it with
+            // this lane's row (16-byte unit e of row r at unit e ^ ((r >> 1) & 3),
+            // the 64-byte swizzle: the eight rows of each quarter-warp store
+            // cover all 32 banks), then one lane hands the box to the copy engine
+            if (lane == 0) bulk_wait_read_all();
+            __syncwarp();
+            uint8_t* rowp = stg + lane * 64;
+            const int sw = (lane >> 1) & 3;
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                *reinterpret_cast<uint4*>(rowp + ((e ^ sw) << 4)) =
+                    make_uint4(pack2<OUT>(y[8 * e], y[8 * e + 1]), pack2<OUT>(y[8 * e + 2], y[8 * e + 3]),
+                               pack2<OUT>(y[8 * e + 4], y[8 * e + 5]), pack2<OUT>(y[8 * e + 6], y[8 * e + 7]));
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) tma_store_3d(tmap_y, smem_u32(stg), col0, row0, prob);
+            return;
+        }
         uint4* dst = reinterpret_cast<uint4*>(stg + lane * kStgRow);
 #pragma unroll
         for (int e = 0; e < 4; ++e)
@@ -597,7 +651,7 @@ __device__ __forceinline__ void epi_chunk(const Params& p, const uint32_t* r, in
 template <int BN, int OUT, bool OUTL, int KIND, bool SK, int CG, int ACT = kActNone>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-                 const Params p) {
+                 const __grid_constant__ CUtensorMap tmap_y, const Params p) {
     using C = Cfg<BN, CG>;
     constexpr int STAGES = C::STAGES;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -646,6 +700,7 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
     if (warp == 0 && lane == 0) {
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_a)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_b)) : "memory");
+        if (p.tma_store) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_y)) : "memory");
     }
     // bar.sync is an aligned barrier: every warp must reach it converged
     __syncwarp();
@@ -770,7 +825,7 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
-                if constexpr (CG == 2) mbar_arrive_cluster(map_to_rank(tempty_bar(a), 0));
+                if constexpr (CG == 2) mbar_arrive_remote(map_to_rank(tempty_bar(a), 0));
                 else mbar_arrive(tempty_bar(a));
             }
         };
@@ -779,25 +834,37 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
             tile_coords_b(tile, p, BM * CG, BN, b, m0, n0);
             m0 += (int)rank * BM;  // this CTA's 128 rows of the pair's tile
             const int c_base = n0 + half * HC;  // first column of this warp
+            const int row0 = m0 + q * 32;  // first row of this warp
+            const int64_t row = (int64_t)row0 + lane;
+            const bool row_ok = row < p.M;
+            // the tile's scales: every load issued before the first is used
+            // (and the row scale before the wait for the accumulator), so a
+            // short k-loop does not wait on them one after another
+            float qxv = 1.0f;
             if constexpr (OUT != kOutI32) {
-                __syncwarp();
-                for (int c = lane; c < HC; c += 32) {
-                    const int col = c_base + c;
-                    float rw = 0.0f, bv = 0.0f;
+                constexpr int NL = HC / 32;
+                float qv[NL], bv[NL];
+#pragma unroll
+                for (int i = 0; i < NL; ++i) {
+                    const int col = c_base + lane + 32 * i;
+                    qv[i] = 0.0f;
+                    bv[i] = 0.0f;
                     if (col < p.N) {
-                        rw = __frcp_rn(ep.w_per_channel ? ep.qs_w[(int64_t)b * p.N + col] : ep.qs_w[b]);
-                        if (ep.bias) bv = ep.bias[col];
+                        qv[i] = ep.w_per_channel ? ep.qs_w[(int64_t)b * p.N + col] : ep.qs_w[b];
+                        if (ep.bias) bv[i] = ep.bias[col];
                     }
-                    rw_w[c] = rw;
-                    bias_w[c] = bv;
+                }
+                if (row_ok) qxv = ep.x_per_token ? ep.qs_x[(int64_t)b * p.M + row] : ep.qs_x[b];
+                __syncwarp();
+#pragma unroll
+                for (int i = 0; i < NL; ++i) {
+                    rw_w[lane + 32 * i] = c_base + lane + 32 * i < p.N ? __frcp_rn(qv[i]) : 0.0f;
+                    bias_w[lane + 32 * i] = bv[i];
                 }
                 __syncwarp();
             }
             const int acc = local & 1;
             const uint32_t acc_phase = (uint32_t)(local >> 1) & 1u;
-            const int row0 = m0 + q * 32;  // first row of this warp
-            const int64_t row = (int64_t)row0 + lane;
-            const bool row_ok = row < p.M;
             if constexpr (OUTL) {
                 // while this tile's MMAs run: bring its X_O rows and W_O
                 // columns into L1, so the outlier term's loads do not wait on L2
@@ -816,7 +883,7 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
             tc_fence_after();
             float rx = 0.0f;
             if constexpr (OUT != kOutI32)
-                if (row_ok) rx = __frcp_rn(ep.x_per_token ? ep.qs_x[(int64_t)b * p.M + row] : ep.qs_x[b]);
+                if (row_ok) rx = __frcp_rn(qxv);
             const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + half * HC);
             // chunks that hold at least one valid column; none when the rows are past M
             int nch = 0;
@@ -870,7 +937,7 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
                                 }
                             }
                             epi_chunk<OUT, OUTL, KIND, ACT>(p, ra, c * 32, c_base + c * 32, row0, row, row_ok, rx, rw_w,
-                                                       bias_w, stg, lane, n_out, compact, b);
+                                                       bias_w, stg, lane, n_out, compact, b, &tmap_y);
                         }
                         if (lane == 0) p.sk_cnt[u * kEpiWarps + wr] = 0;  // ready for the next launch
                     }
@@ -891,7 +958,7 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
                         release_acc(acc);  // accumulator read in full
                     }
                     epi_chunk<OUT, OUTL, KIND, ACT>(p, ra, c * 32, c_base + c * 32, row0, row, row_ok, rx, rw_w, bias_w, stg,
-                                         lane, n_out, compact, b);
+                                         lane, n_out, compact, b, &tmap_y);
                     if (!more) break;
                     tmem_wait(rb);
                     const bool more2 = c + 2 < nch;
@@ -900,7 +967,7 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
                         release_acc(acc);
                     }
                     epi_chunk<OUT, OUTL, KIND, ACT>(p, rb, (c + 1) * 32, c_base + (c + 1) * 32, row0, row, row_ok, rx, rw_w,
-                                         bias_w, stg, lane, n_out, compact, b);
+                                         bias_w, stg, lane, n_out, compact, b, &tmap_y);
                     if (more2) tmem_wait(ra);
                 }
             } else {
@@ -910,13 +977,16 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
                         release_acc(acc);  // accumulator read in full
                     }
                     epi_chunk<OUT, OUTL, KIND, ACT>(p, ra, c * 32, c_base + c * 32, row0, row, row_ok, rx, rw_w, bias_w, stg,
-                                         lane, n_out, compact, b);
+                                         lane, n_out, compact, b, &tmap_y);
                 }
             }
             if (nch == 0) {
                 release_acc(acc);
             }
         }
+        // the output boxes handed to the copy engine are written before the
+        // grid completes (and before the staging memory is released)
+        if (p.tma_store && lane == 0) bulk_wait_all();
     }
 
     // Lanes 1..31 of warps 0 and 1 reach this point long before their lane 0
@@ -967,7 +1037,23 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t K, int box
     return r == CUDA_SUCCESS;
 }
 
-using KernelFn = void (*)(const CUtensorMap, const CUtensorMap, const Params);
+// 3-D 16-bit output [batch, M, ldy] (problems y_bstride elements apart), box
+// 32 columns x 32 rows x 1, 64-byte swizzle (the staging layout of a chunk).
+bool make_map_y(CUtensorMap* m, void* Y, int64_t M, int64_t N, int64_t ldy, int64_t batch, int64_t y_bstride,
+                bool bf16) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)N, (cuuint64_t)M, (cuuint64_t)batch};
+    cuuint64_t strides[2] = {(cuuint64_t)(ldy * 2), (cuuint64_t)(y_bstride * 2)};
+    cuuint32_t box[3] = {32, 32, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, Y, dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                    CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+using KernelFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const Params);
 
 template <int BN, bool SK, int CG>
 KernelFn pick_kernel_sk(sq_dtype_t out_dt, bool outl, int kind) {
@@ -1102,6 +1188,14 @@ sq_status_t launch_bn(const int8_t* Xq, const int8_t* Wq, int64_t M, int64_t N, 
     // static scale, else the output dtype's
     const int eb = ep.act_qs ? 1 : (ep.out_dt == SQ_BF16 || ep.out_dt == SQ_F16) ? 2 : 4;
     p.vec_store = ((reinterpret_cast<uintptr_t>(ep.Y) & 15u) == 0) && ((ep.ldy * eb) % 16 == 0);
+    // 16-bit outputs of the plain epilogue go out by TMA store (row and
+    // problem strides multiples of 16 bytes, within the tensor map's limits)
+    CUtensorMap ty;
+    memset(&ty, 0, sizeof(ty));
+    p.tma_store = 0;
+    const int64_t ybs = ep.batch > 1 ? ep.y_bstride : M * ep.ldy;  // one problem: any stride past its rows
+    if (p.vec_store && eb == 2 && ep.act == kActNone && (ybs * 2) % 16 == 0 && ybs * 2 < (1ll << 40))
+        p.tma_store = make_map_y(&ty, ep.Y, M, N, ep.ldy, ep.batch, ybs, ep.out_dt == SQ_BF16) ? 1 : 0;
     p.ep = ep;
     p.status = status;
     p.dp_tiles = sk ? plan.tiles - plan.sk_tiles : plan.tiles;
@@ -1112,9 +1206,9 @@ sq_status_t launch_bn(const int8_t* Xq, const int8_t* Wq, int64_t M, int64_t N, 
     p.sk_part = sk ? reinterpret_cast<int*>(static_cast<uint8_t*>(sk_ws) + plan.sk_cnt_bytes) : nullptr;
     const int grid = plan.grid;
     if constexpr (CG == 2)
-        launch_pdl_cluster(fn, dim3(grid), dim3(kThreads), C::SMEM_ALLOC, stream, 2, ta, tb, p);
+        launch_pdl_cluster(fn, dim3(grid), dim3(kThreads), C::SMEM_ALLOC, stream, 2, ta, tb, ty, p);
     else
-        launch_pdl(fn, dim3(grid), dim3(kThreads), C::SMEM_ALLOC, stream, ta, tb, p);
+        launch_pdl(fn, dim3(grid), dim3(kThreads), C::SMEM_ALLOC, stream, ta, tb, ty, p);
     return check_launch("sq_gemm_w8a8");
 }
 
