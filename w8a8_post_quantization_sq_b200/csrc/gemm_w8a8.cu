@@ -241,6 +241,7 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
     }
 }
 
+
 // Store a 32 x 32 box of 16-bit outputs (x = column, y = row, z = problem)
 // from this CTA's shared memory; elements outside the tensor are not written.
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int x, int y, int z) {
@@ -745,6 +746,9 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
                     // the pair's loads all count on CTA 0's barrier, which expects both
                     const uint32_t fb = CG == 2 ? map_to_rank(full_bar(stage), 0) : full_bar(stage);
                     if (rank == 0) mbar_expect_tx(full_bar(stage), CG * (C::A_BYTES + C::B_BYTES));
+                    // (no L2 eviction hints: marking the weight tiles evict-first made the
+                    // other m-blocks of the group fetch them again, 2.8 -> 7.9 GB of DRAM
+                    // reads at 4096 x 12288 x 49152, and the step 8 % slower on B200)
                     tma_load_3d<CG>(sbase + C::A_OFF + stage * C::A_BYTES, &tmap_a, fb, kb * BK, m0, b);
                     tma_load_3d<CG>(sbase + C::B_OFF + stage * C::B_BYTES, &tmap_b, fb, kb * BK, n0, b);
                     issued[stage] = true;
@@ -1188,13 +1192,14 @@ sq_status_t launch_bn(const int8_t* Xq, const int8_t* Wq, int64_t M, int64_t N, 
     // static scale, else the output dtype's
     const int eb = ep.act_qs ? 1 : (ep.out_dt == SQ_BF16 || ep.out_dt == SQ_F16) ? 2 : 4;
     p.vec_store = ((reinterpret_cast<uintptr_t>(ep.Y) & 15u) == 0) && ((ep.ldy * eb) % 16 == 0);
-    // 16-bit outputs of the plain epilogue go out by TMA store (row and
-    // problem strides multiples of 16 bytes, within the tensor map's limits)
+    // 16-bit outputs of the plain, ReLU and GELU epilogues go out by TMA
+    // store (row and problem strides multiples of 16 bytes, within the
+    // tensor map's limits); SwiGLU's half-width rows keep the plain stores
     CUtensorMap ty;
     memset(&ty, 0, sizeof(ty));
     p.tma_store = 0;
     const int64_t ybs = ep.batch > 1 ? ep.y_bstride : M * ep.ldy;  // one problem: any stride past its rows
-    if (p.vec_store && eb == 2 && ep.act == kActNone && (ybs * 2) % 16 == 0 && ybs * 2 < (1ll << 40))
+    if (p.vec_store && eb == 2 && ep.act != SQ_ACT_SWIGLU && (ybs * 2) % 16 == 0 && ybs * 2 < (1ll << 40))
         p.tma_store = make_map_y(&ty, ep.Y, M, N, ep.ldy, ep.batch, ybs, ep.out_dt == SQ_BF16) ? 1 : 0;
     p.ep = ep;
     p.status = status;

@@ -123,6 +123,16 @@ def c2_block(device="cpu", M=2048, w_frac=1.0):
     }
 
 
+def _stacked(act, seeds, M, K, dtype, device):
+    """Calibration batches drawn one by one into one contiguous [n, M, K]
+    buffer: the list of batches (views) and the same tokens as one [n M, K]
+    matrix, for a single pass over all of them."""
+    buf = torch.empty((len(seeds), M, K), dtype=dtype, device=device)
+    for i, s in enumerate(seeds):
+        buf[i].copy_(act(s))
+    return [buf[i] for i in range(len(seeds))], buf.view(len(seeds) * M, K)
+
+
 def c3_opt30b(device="cpu", M=1024, n_calib=8, w_frac=1.0):
     """OPT-30B decoder linear stack at 4 x 256 tokens: fp16 pre-norm inputs of
     the attention and MLP sides (7 channels, 0.1% of 7168, x60), 8 calibration
@@ -143,8 +153,9 @@ def c3_opt30b(device="cpu", M=1024, n_calib=8, w_frac=1.0):
                  device, 0.02, torch.float16, w_frac)
     xo, so = synthetic_int8(M, K, 400, device)
     xf, sf = synthetic_int8(M, 28672, 401, device)
+    calib, calib_all = _stacked(act, range(1, n_calib + 1), M, K, torch.float16, device)
     return {
-        "h": {"attn": act(0), "mlp": act(9)}, "calib": [act(s) for s in range(1, n_calib + 1)],
+        "h": {"attn": act(0), "mlp": act(9)}, "calib": calib, "calib_all": calib_all,
         "gamma": {"attn": gamma, "mlp": gamma}, "beta": {"attn": beta, "mlp": beta}, "eps": 1e-5, "W": w,
         "syn": {"out": (xo, so[:1].contiguous()), "fc2": (xf, sf[:1].contiguous())},
         "outlier_channels": ch,
@@ -192,8 +203,9 @@ def c5_175b(device="cpu", M=4096, n_calib=16, w_frac=1.0):
                  device, 0.01, torch.float32, w_frac)
     xo, so = synthetic_int8(M, K, 600, device)
     xf, sf = synthetic_int8(M, 49152, 601, device)
+    calib, calib_all = _stacked(act, range(100, 100 + n_calib), M, K, torch.bfloat16, device)
     return {
-        "h": {"attn": act(200), "mlp": act(201)}, "calib": [act(s) for s in range(100, 100 + n_calib)],
+        "h": {"attn": act(200), "mlp": act(201)}, "calib": calib, "calib_all": calib_all,
         "gamma": {"attn": gamma, "mlp": gamma}, "beta": {"attn": beta, "mlp": beta}, "eps": 1e-5, "W": w,
         "syn": {"out": (xo, so), "fc2": (xf, sf)}, "outlier_channels": ch,
     }
