@@ -313,13 +313,15 @@ def test_norm_smooth_quant_per_token(dtype, norm, K):
 
 @pytest.mark.parametrize("norm", ["ln", "rms"])
 @pytest.mark.parametrize("K,M,dtype", [(5000, 300, torch.bfloat16), (8192, 300, torch.float16),
-                                       (11008, 300, torch.float16), (12288, 2500, torch.bfloat16),
-                                       (13000, 300, torch.bfloat16),
+                                       (8192, 301, torch.bfloat16), (11008, 300, torch.float16),
+                                       (12288, 2500, torch.bfloat16), (12288, 2501, torch.float16),
+                                       (12288, 1, torch.bfloat16), (13000, 300, torch.bfloat16),
                                        (16384, 700, torch.float16)])
 def test_norm_quant_only(norm, K, M, dtype):
     """Codes and scales without the V output, per token and with a static scale:
     the quantise-only kernels, with full and ragged chunk sets; at M = 2500
-    every block of the grid cycles its ring of staged rows more than once."""
+    every block of the grid cycles its ring of staged rows more than once; odd
+    M and a single row leave some blocks fewer rows than the others."""
     H = rnd((M, K), K + 7, dtype)
     H[:, K // 3] *= 50
     gamma = 1 + 0.1 * rnd(K, 5)

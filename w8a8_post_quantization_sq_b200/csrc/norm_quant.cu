@@ -58,10 +58,12 @@ __device__ __forceinline__ float tree8(const float* g) {
                      __fadd_rn(__fadd_rn(g[4], g[5]), __fadd_rn(g[6], g[7])));
 }
 
+// Warp maximum of non-negative floats (the row maxima here start at 0 and
+// are formed by max operations that drop NaN operands, so they are never
+// NaN): their bit patterns order as their values, so one integer redux
+// replaces the five-step shuffle tree.
 __device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    return v;
+    return __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(v)));
 }
 
 // max(a, b, c) in one instruction (exact; the order of a max does not matter)
@@ -645,6 +647,7 @@ template <typename T, bool LN, int C, bool KEEPV>
 void launch_block(const void* H, const NormArgs& a, cudaStream_t s) {
     const bool full = a.K == 2048 * C;
     const bool qonly = a.Xq && !a.absmax && !a.V;
+
     if (full) {
         if (qonly) launch_block_k<T, LN, C, KEEPV, true, true>(H, a, s);
         else launch_block_k<T, LN, C, KEEPV, true, false>(H, a, s);

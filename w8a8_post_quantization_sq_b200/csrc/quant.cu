@@ -122,10 +122,12 @@ __device__ __forceinline__ uint2 codes8(const float* v, float qs, bool clip) {
     else return codes8_i8(v, qs, clip);
 }
 
+// Warp maximum of non-negative floats (the row maxima here start at 0 and
+// are formed by max operations that drop NaN operands, so they are never
+// NaN): their bit patterns order as their values, so one integer redux
+// replaces the five-step shuffle tree.
 __device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    return v;
+    return __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(v)));
 }
 
 // One warp per row, rows strided over the grid. per_row != 0: the row's own
