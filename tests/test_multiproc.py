@@ -31,15 +31,20 @@ def _calib_rank(rank, world, port, out):
         import bench
 
         g = torch.Generator().manual_seed(5)
-        X = torch.randn((4 * 37, 96), generator=g)
+        X = torch.randn((5 * 37, 96), generator=g)
         X[:, 11] *= 80
-        X[3, 50] = -400.0    # the column's extreme sits in rank 0's shard ...
-        X[40, 51] = 800.0    # ... and this one in rank 1's
-        shard = X[rank * 37:(rank + 1) * 37] if rank < world - 1 else X[rank * 37:]
-        local = torch.from_numpy(oracle.col_absmax(shard.numpy()))
-        sharded.allreduce_max_(local)
+        X[3, 50] = -400.0    # the column's extreme sits in batch 0 (rank 0's shard) ...
+        X[40, 51] = 800.0    # ... and this one in batch 1 (rank 1's)
+        batches = [X[i * 37:(i + 1) * 37] for i in range(5)]  # 5 batches: the ranks' shards differ in size
+        seen = []
+
+        def update(b, m):  # the oracle's running maxima stand in for the CUDA call on CPU ranks
+            seen.append(next(i for i, c in enumerate(batches) if c is b))
+            m.copy_(torch.from_numpy(oracle.col_absmax(b.numpy(), m.numpy())))
+
+        local = sharded.calibrate_sharded(batches, torch.zeros(96), update)
         full = oracle.col_absmax(X.numpy())
-        ok_calib = bool(np.array_equal(local.numpy(), full))
+        ok_calib = bool(np.array_equal(local.numpy(), full)) and seen == list(range(rank, 5, world))
         # the benchmark's timing: the max over the ranks of each rank's own time
         t = bench.max_over_ranks(1.5 + rank, torch.device("cpu"))
         out[rank] = (ok_calib, t)
@@ -86,12 +91,9 @@ def _calib_rank_cuda(rank, world, port, out):
 
         d = inputs.c5_175b(device="cpu", M=64, n_calib=4, w_frac=1 / 4096)
         batches = d["calib"]  # bf16 [64, 12288] each, 8 channels x100
-        mine = [b for i, b in enumerate(batches) if i % world == rank]
         xmax = torch.zeros(12288, device="cuda")
-        for b in mine:
-            sq.sq_calib_absmax(b.cuda(), xmax)
+        sharded.calibrate_sharded(batches, xmax, lambda b, m: sq.sq_calib_absmax(b.cuda(), m))
         local = xmax.cpu()
-        sharded.allreduce_max_(local)
         full = np.zeros(12288, np.float32)
         for b in batches:
             full = oracle.col_absmax(b, full)
@@ -109,3 +111,15 @@ def test_sharded_calibration_with_cuda_maxima():
     out = mp.Manager().dict()
     mp.spawn(_calib_rank_cuda, args=(world, port, out), nprocs=world, join=True)
     assert all(out[r] for r in range(world)), "sharded CUDA maxima differ from the oracle's maxima of all tokens"
+
+
+def test_shard_assignment():
+    """Batch i goes to rank i mod world; the shards partition the batches."""
+    from w8a8_post_quantization_sq_b200 import sharded
+
+    for n, world in [(16, 1), (16, 2), (5, 2), (7, 3), (2, 4)]:
+        shards = [list(sharded.shard(n, r, world)) for r in range(world)]
+        assert sorted(i for s in shards for i in s) == list(range(n))
+        assert all(i % world == r for r, s in enumerate(shards) for i in s)
+    with pytest.raises(ValueError):
+        sharded.shard(4, 2, 2)
