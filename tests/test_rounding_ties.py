@@ -155,3 +155,35 @@ def test_gpu_norm_ties(K, norm, per_token):
     r = oracle.norm_smooth_quant(H, 0 if norm == "ln" else 1, gamma.numpy(), None if beta is None else beta.numpy(),
                                  0.0, per_token, None if per_token else 1.0)
     assert np.array_equal(r["Xq"], expect)
+
+
+# ---------------------------------------------------------------- all-zero rows
+@pytest.mark.gpu
+@pytest.mark.parametrize("K", [1024, 12288])
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+def test_gpu_zero_rows_take_the_floor(K, dtype):
+    """A row whose largest |v| is 0 takes the scale 127 / 1e-8 ("8位量化" §2.1:
+    the absmax guarded by a small floor) and codes 0, in the activation
+    quantiser and in the fused norm (RMSNorm, and LayerNorm without a shift,
+    where a zero row stays zero), bit for bit with the oracle; the rows around
+    it are unaffected."""
+    sq = gpu()
+    g = torch.Generator().manual_seed(K)
+    X = torch.randn((6, K), generator=g).to(dtype)
+    X[1] = 0
+    X[4] = 0
+    Xd = X.cuda()
+    Xq = torch.empty((6, K), dtype=torch.int8, device="cuda")
+    qs = torch.empty(6, device="cuda")
+    sq.sq_quantize_act(Xd, None, True, None, Xq, qs)
+    torch.cuda.synchronize()
+    rq, rqs = oracle.quantize_act(X.float().numpy(), None, per_token=True)
+    assert np.array_equal(Xq.cpu().numpy(), rq) and np.array_equal(qs.cpu().numpy(), rqs)
+    assert qs.cpu()[1] == np.float32(127.0) / np.float32(1e-8) and not Xq[1].any()
+    gamma = 1 + 0.1 * torch.randn(K, generator=g)
+    for nt, on in ((sq.SQ_RMSNORM, oracle.RMSNORM), (sq.SQ_LAYERNORM, oracle.LAYERNORM)):
+        sq.sq_norm_smooth_quant(Xd, nt, gamma.cuda(), None, 1e-5, True, None, Xq, qs)
+        torch.cuda.synchronize()
+        r = oracle.norm_smooth_quant(X, on, gamma.numpy(), None, 1e-5, True)
+        assert np.array_equal(Xq.cpu().numpy(), r["Xq"]) and np.array_equal(qs.cpu().numpy(), r["qs"])
+        assert qs.cpu()[4] == np.float32(127.0) / np.float32(1e-8) and not Xq[4].any()
