@@ -1228,7 +1228,8 @@ def run_reference(args, rank, world):
 # ------------------------------------------------------------------ single kernels
 def run_kernel(args):
     """Time one entry point alone on one shape:
-    gemm M,N,K | gemm_fp8 M,N,K | bmm B,M,N,K | norm M,K | absmax M,K | act M,I | quant_weight N,K |
+    gemm M,N,K | gemm_fp8 M,N,K | bmm B,M,N,K | norm M,K | norm_calib M,K | absmax M,K | act M,I |
+    quant_weight N,K |
     llmint8 M,K,N.
     --sets 1: every launch after an L2 flush, each launch timed on its own.
     --sets S > 1: S distinct input/output sets, launches cycling through them
@@ -1286,13 +1287,16 @@ def run_kernel(args):
             Y = torch.empty((B, M, N), dtype=torch.bfloat16, device=dev)
             ws = sq.workspace(sq.SQ_OP_GEMM, M, N, K, device=dev)
             return lambda: sq.sq_bmm_w8a8(Aq, Bq, qa, qb, Y, ws)
-        if args.kernel == "norm":
+        if args.kernel in ("norm", "norm_calib"):
             M, K = shape
             dt16 = torch.float16 if args.dtype == "fp16" else torch.bfloat16
             H = torch.randn((M, K), generator=g, device=dev).to(dt16)
             gamma = torch.rand(K, generator=g, device=dev) + 0.5
             beta = torch.randn(K, generator=g, device=dev) * 0.1 if args.norm == "ln" else None
             nt = sq.SQ_LAYERNORM if args.norm == "ln" else sq.SQ_RMSNORM
+            if args.kernel == "norm_calib":  # calibration mode: running max |v| per channel, no codes
+                am = torch.zeros(K, device=dev)
+                return lambda: sq.sq_norm_smooth_quant(H, nt, gamma, beta, 1e-5, True, None, None, None, am)
             Xq = torch.empty((M, K), dtype=torch.int8, device=dev)
             qs = torch.empty(M, device=dev)
             return lambda: sq.sq_norm_smooth_quant(H, nt, gamma, beta, 1e-5, True, None, Xq, qs)
@@ -1348,6 +1352,10 @@ def run_kernel(args):
     elif args.kernel == "norm":
         M, K = shape
         work, unit, peak = (3.0 * M * K + 4 * M) / 1e9, "GB/s", pk["hbm_gbs"]
+        out["norm"] = args.norm
+    elif args.kernel == "norm_calib":
+        M, K = shape
+        work, unit, peak = 2.0 * M * K / 1e9, "GB/s", pk["hbm_gbs"]
         out["norm"] = args.norm
     elif args.kernel == "absmax":
         M, K = shape

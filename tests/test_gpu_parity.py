@@ -347,10 +347,11 @@ def test_norm_quant_only(norm, K, M, dtype):
 
 
 @pytest.mark.parametrize("norm", ["ln", "rms"])
-@pytest.mark.parametrize("K", [1024, 7168, 12288])
+@pytest.mark.parametrize("K", [1024, 7168, 8192, 12288])
 def test_norm_static_and_calibration(norm, K):
     """Calibration mode (running per-channel max of |v| over batches) and the
-    static per-tensor scale taken from it, the OPT-30B-style path."""
+    static per-tensor scale taken from it, the OPT-30B-style path (K = 7168
+    and 8192: the maxima held in registers, ragged and full chunk sets)."""
     M = 200
     nt = sq.SQ_LAYERNORM if norm == "ln" else sq.SQ_RMSNORM
     on = oracle.LAYERNORM if norm == "ln" else oracle.RMSNORM
