@@ -1325,7 +1325,7 @@ def run_kernel(args):
             from w8a8_post_quantization_sq_b200 import inputs
 
             M, K, N = shape
-            d = inputs.c4_llmint8(device=dev, M=M, K=K, N=N, seed=i)
+            d = inputs.c4_llmint8(device=dev, M=M, K=K, N=N, n_out=args.outliers, seed=i)
             st = sq.llmint8_weight_state(d["W"])
             Y = torch.empty((M, N), dtype=torch.float16, device=dev)
             idx = torch.empty(K, dtype=torch.int32, device=dev)
@@ -1436,6 +1436,7 @@ def main():
     ap.add_argument("--norm", default="rms", help="--kernel norm: rms|ln")
     ap.add_argument("--act", default="swiglu", help="--kernel act: swiglu|relu")
     ap.add_argument("--whole-tiles", action="store_true", help="--kernel gemm: a workspace without stream-K scratch")
+    ap.add_argument("--outliers", type=int, default=6, help="--kernel llmint8: outlier dimensions in X")
     ap.add_argument("--sets", type=int, default=1, help="--kernel: input sets cycled back to back (1: flush each)")
     ap.add_argument("--workload", default=HEADLINE, choices=sorted(CONFIGS), help="the headline stack")
     ap.add_argument("--configs", default="c2,c3,c4,c5_fp8,attn_int8",
