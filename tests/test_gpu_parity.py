@@ -232,9 +232,15 @@ def test_act_quant_errors():
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16, torch.float32])
 @pytest.mark.parametrize("per_channel", [True, False])
 @pytest.mark.parametrize("with_s", [True, False])
-@pytest.mark.parametrize("K", [1024, 2064, 12288, 20480])
+@pytest.mark.parametrize("K", [1024, 2064, 11008, 12288, 20480, 49152])
 def test_quantize_weight(dtype, per_channel, with_s, K):
-    N = 517 if K <= 2064 else 131
+    """Every row kernel: warp-held rows, block-held rows (six chunks per
+    thread up to K = 12288, ragged at 11008), and rows read twice by a block
+    (K = 20480, 49152; at 49152, 1100 rows: more than the grid, which is capped
+    by the rows in flight, so blocks take several)."""
+    if K == 49152 and not per_channel:
+        pytest.skip("per-tensor scales at K = 49152 add nothing the per-channel case does not cover")
+    N = 517 if K <= 2064 else (1100 if K == 49152 else 131)
     W = rnd((N, K), 10, dtype, 0.02)
     s = torch.rand(K, generator=torch.Generator().manual_seed(11)) * 30 + 0.05 if with_s else None
     Wq = torch.empty((N, K), dtype=torch.int8, device=DEV)
