@@ -922,58 +922,62 @@ MLP_CHAINS = (("c2_swiglu", 2048, 1024, 3072, 0, False, "bf16"),
 INT8_OPS_PER_SM_CLK = 16384
 
 
-def int8_ceiling(args, dev, flush, n=8192, reps=10):
+def int8_ceiling(args, dev, flush, shapes=((8192, 8192, 8192), (4096, 36864, 12288)), reps=10):
     """The measured int8 ceiling beside the library's own GEMM: this library's
-    GEMM at n^3 (int32 and bf16 outputs) against the CUDA library int8 matmul
-    torch exposes (torch._int_mm, int32 output) on the same operands, each
-    launch after an L2 flush, with the clocks during the timing and the
-    clock-scaled dense peak (SM count x 16384 ops/clock x the median SM clock)."""
+    GEMM (int32 and bf16 outputs) against the CUDA library int8 matmul torch
+    exposes (torch._int_mm, int32 output) on the same operands, at 8192^3 and
+    at the 175B-shaped QKV shape, each launch after an L2 flush, with the
+    clocks during the timing and the clock-scaled dense peak (SM count x 16384
+    ops/clock x the median SM clock)."""
     import torch
 
     import w8a8_post_quantization_sq_b200 as sq
 
-    g = torch.Generator(device=dev).manual_seed(8)
-    A = torch.randint(-127, 128, (n, n), generator=g, device=dev, dtype=torch.int8)
-    B = torch.randint(-127, 128, (n, n), generator=g, device=dev, dtype=torch.int8)
-    qa = torch.rand(n, generator=g, device=dev) + 1
-    qb = torch.rand(n, generator=g, device=dev) + 100
-    Y32 = torch.empty((n, n), dtype=torch.int32, device=dev)
-    Y16 = torch.empty((n, n), dtype=torch.bfloat16, device=dev)
-    ws = sq.workspace(sq.SQ_OP_GEMM, n, n, n, device=dev)
-    Bt = B.t()  # [K, N] column-major view: torch._int_mm computes A @ Bt = A B^T, the same product
-    arms = {"ours_int32": lambda: sq.sq_gemm_w8a8(A, B, None, None, None, Y32, ws),
-            "ours_bf16": lambda: sq.sq_gemm_w8a8(A, B, qa, qb, None, Y16, ws),
-            "torch_int_mm_int32": lambda: torch._int_mm(A, Bt)}
-    out = {"shape": [n, n, n], "timing": f"median of {reps} launches, each after an L2 flush"}
-    ok = True
-    for f in arms.values():
-        f()
-    torch.cuda.synchronize()
-    ok = bool(torch.equal(torch._int_mm(A, Bt), Y32))
-    clocks = ClockSampler(dev.index if dev.index is not None else 0)
-    time.sleep(0.05)
-    for name, f in arms.items():
-        ms = []
-        for _ in range(reps):
-            flush(0)
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record()
+    res = {"timing": f"median of {reps} launches, each after an L2 flush", "shapes": []}
+    for M, N, K in shapes:
+        g = torch.Generator(device=dev).manual_seed(8)
+        A = torch.randint(-127, 128, (M, K), generator=g, device=dev, dtype=torch.int8)
+        B = torch.randint(-127, 128, (N, K), generator=g, device=dev, dtype=torch.int8)
+        qa = torch.rand(M, generator=g, device=dev) + 1
+        qb = torch.rand(N, generator=g, device=dev) + 100
+        Y32 = torch.empty((M, N), dtype=torch.int32, device=dev)
+        Y16 = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        ws = sq.workspace(sq.SQ_OP_GEMM, M, N, K, device=dev)
+        Bt = B.t()  # [K, N] column-major view: torch._int_mm computes A @ Bt = A B^T, the same product
+        arms = {"ours_int32": lambda: sq.sq_gemm_w8a8(A, B, None, None, None, Y32, ws),
+                "ours_bf16": lambda: sq.sq_gemm_w8a8(A, B, qa, qb, None, Y16, ws),
+                "torch_int_mm_int32": lambda: torch._int_mm(A, Bt)}
+        out = {"shape": [M, N, K]}
+        for f in arms.values():
             f()
-            b.record()
-            torch.cuda.synchronize()
-            ms.append(a.elapsed_time(b))
-        t = statistics.median(ms) * 1e-3
-        out[name] = {"us": t * 1e6, "tops": 2.0 * n ** 3 / t / 1e12}
-    clk = clocks.stop()
-    out["clocks"] = clk
-    out["int32_outputs_equal"] = ok
-    if clk and clk.get("sm_mhz"):
-        sms = torch.cuda.get_device_properties(dev).multi_processor_count
-        peak = sms * INT8_OPS_PER_SM_CLK * clk["sm_mhz"] * 1e6 / 1e12
-        out["clock_scaled_peak_tops"] = peak
-        for name in arms:
-            out[name]["frac_clock_scaled"] = out[name]["tops"] / peak
-    return out
+        torch.cuda.synchronize()
+        out["int32_outputs_equal"] = bool(torch.equal(torch._int_mm(A, Bt), Y32))
+        clocks = ClockSampler(dev.index if dev.index is not None else 0)
+        time.sleep(0.05)
+        for name, f in arms.items():
+            ms = []
+            for _ in range(reps):
+                flush(0)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                f()
+                b.record()
+                torch.cuda.synchronize()
+                ms.append(a.elapsed_time(b))
+            t = statistics.median(ms) * 1e-3
+            out[name] = {"us": t * 1e6, "tops": 2.0 * M * N * K / t / 1e12}
+        clk = clocks.stop()
+        out["clocks"] = clk
+        if clk and clk.get("sm_mhz"):
+            sms = torch.cuda.get_device_properties(dev).multi_processor_count
+            peak = sms * INT8_OPS_PER_SM_CLK * clk["sm_mhz"] * 1e6 / 1e12
+            out["clock_scaled_peak_tops"] = peak
+            for name in arms:
+                out[name]["frac_clock_scaled"] = out[name]["tops"] / peak
+        res["shapes"].append(out)
+        del A, B, Y32, Y16, ws
+        torch.cuda.empty_cache()
+    return res
 
 
 def time_mlp_chains(args, dev, flush):

@@ -213,6 +213,16 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, vola
     return wait_bounded_ns(bar, parity, abort_flag, status, code, kTimeoutNs);
 }
 
+// The same with the common case inline: one try_wait (which itself suspends
+// the thread for a while if the phase is not complete), and the call into the
+// bounded loop only when that is not enough. The producer and the MMA issuer
+// wait once per k-block; a call per wait sat on their critical path.
+__device__ __forceinline__ bool wait_fast(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* status,
+                                         int code) {
+    if (mbar_try_wait(bar, parity)) return true;
+    return wait_bounded(bar, parity, abort_flag, status, code);
+}
+
 // Short bounded wait used while draining after an abort (ignores the flag).
 __device__ __noinline__ void wait_drain(uint32_t bar, uint32_t parity) {
     const uint64_t t0 = global_ns();
@@ -739,7 +749,7 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
                 m0 += (int)rank * BM;
                 n0 += (int)rank * (BN / CG);
                 for (int kb = k0; kb < k1; ++kb) {
-                    if (!wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, p.status, 0x6E1)) {
+                    if (!wait_fast(empty_bar(stage), phase ^ 1u, abort_flag, p.status, 0x6E1)) {
                         ok = false;
                         break;
                     }
@@ -776,14 +786,14 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
             for (; ok && seg.next(p, num_tiles, tile, k0, k1, slot); ++local) {
                 const int acc = local & 1;
                 const uint32_t acc_phase = (uint32_t)(local >> 1) & 1u;
-                if (!wait_bounded(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p.status, 0x6E2)) {
+                if (!wait_fast(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p.status, 0x6E2)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
                 for (int kb = k0; kb < k1; ++kb) {
-                    if (!wait_bounded(full_bar(stage), phase, abort_flag, p.status, 0x6E3)) {
+                    if (!wait_fast(full_bar(stage), phase, abort_flag, p.status, 0x6E3)) {
                         ok = false;
                         break;
                     }
@@ -882,7 +892,7 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
                     }
                 }
             }
-            const bool ok = wait_bounded(tfull_bar(acc), acc_phase, abort_flag, p.status, 0x6E4);
+            const bool ok = wait_fast(tfull_bar(acc), acc_phase, abort_flag, p.status, 0x6E4);
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
             float rx = 0.0f;
@@ -1248,13 +1258,13 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int64_t batch) {
         pl.sk_bytes = pl.sk_cnt_bytes + (size_t)pl.grid * 2 * BM * pl.bn * sizeof(int);
     }
     // CTA pairs (256 x 256 tiles, cta_group::2: each SM streams half the
-    // weight bytes per MMA) where there are two waves of them or more and the
-    // single-CTA plan has no stream-K split of a ragged last wave. Measured
-    // on B200 (us, single CTA -> pairs): 4096 x 36864 x 12288 1285 -> 1252,
-    // 4096 x 49152 x 12288 1697 -> 1653, 1024 x 21504 x 7168 127 -> 122,
-    // 2048 x 16384 x 4096 105 -> 104; the shapes with a split are faster
-    // without pairs (1024 x 7168 x 28672: 159 split, 177 on pairs).
-    if (pl.bn == 256 && pairs_mode() != 0 && (pl.sk_tiles == 0 || pairs_mode() == 1)) {
+    // weight bytes per MMA) where there are two waves of them or more, with or
+    // without a stream-K split in the single-CTA plan. Measured on B200 (us,
+    // single CTA -> pairs): 4096 x 36864 x 12288 1285 -> 1252 (and 1178 with
+    // the inline waits), 4096 x 12288 x 12288 419 (stream-K) -> 386,
+    // 4096 x 12288 x 49152 1713 (stream-K) -> 1625; shapes with fewer pair
+    // tiles keep single CTAs and their split (1024 x 7168 x 28672: 158).
+    if (pl.bn == 256 && pairs_mode() != 0) {
         const int pairs = max_resident_pairs();
         const int64_t ptiles = batch * ((M + 2 * BM - 1) / (2 * BM)) * ((N + 255) / 256);
         if (pairs > 0 && ptiles < (1ll << 31) && (pairs_mode() == 1 || ptiles >= 2ll * pairs)) {
