@@ -120,12 +120,17 @@ __device__ __forceinline__ uint64_t global_ns() {
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
 }
-__device__ __noinline__ bool wait_stage(uint32_t bar, uint32_t parity) {
+__device__ __noinline__ bool wait_stage_slow(uint32_t bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     while (!mbar_try_wait(bar, parity))
         if (global_ns() - t0 > kWaitNs) return false;
     return true;
+}
+// the common case inline (one try_wait, which itself suspends the thread for
+// a while), the bounded loop only when that is not enough
+__device__ __forceinline__ bool wait_stage(uint32_t bar, uint32_t parity) {
+    return mbar_try_wait(bar, parity) || wait_stage_slow(bar, parity);
 }
 
 template <typename T>

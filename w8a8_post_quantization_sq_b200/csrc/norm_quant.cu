@@ -357,12 +357,17 @@ __device__ __forceinline__ uint64_t global_ns() {
     return t;
 }
 // Bounded wait for a row copy; false after about 2 s.
-__device__ __noinline__ bool wait_row(uint32_t bar, uint32_t parity) {
+__device__ __noinline__ bool wait_row_slow(uint32_t bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     while (!mbar_try_wait(bar, parity))
         if (global_ns() - t0 > kWaitNs) return false;
     return true;
+}
+// the common case inline (one try_wait, which itself suspends the thread for
+// a while), the bounded loop only when that is not enough
+__device__ __forceinline__ bool wait_row(uint32_t bar, uint32_t parity) {
+    return mbar_try_wait(bar, parity) || wait_row_slow(bar, parity);
 }
 // One row (bytes, a multiple of 16) from global into shared memory, completing
 // on the mbarrier; a plain bulk copy, no multicast.
