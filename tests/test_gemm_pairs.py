@@ -183,3 +183,43 @@ def test_pairs_fused_activation(act, monkeypatch):
         outs.append((H, Q))
     assert torch.equal(outs[0][0].view(torch.int16), outs[1][0].view(torch.int16))
     assert torch.equal(outs[0][1], outs[1][1])
+
+
+@pytest.mark.parametrize("M,N,K,dtype", [(2048, 6144, 8192, torch.bfloat16), (2000, 6100, 8320, torch.float16),
+                                         (2048, 6144, 8192, torch.float32)])
+def test_pairs_stream_k(M, N, K, dtype, monkeypatch):
+    """A ragged last wave of pair tiles cut by k-blocks, one range per CTA pair
+    (each CTA of a pair parks and counts its own half of a tile; the piece
+    that completes a half adds the parks up): 192 pair tiles over 74 pairs,
+    k-loops of 64 and 65 blocks.
+    int32 sums exact against the CUDA library's int8 matmul, the dequantised
+    output bit for bit against the single-CTA kernel (same int32 sums, same
+    epilogue arithmetic), and sampled rows against the oracle; the split's
+    counters are left at zero, so a second call on the workspace is exact too."""
+    monkeypatch.delenv("SQ_GEMM_CTA_PAIRS", raising=False)
+    if M == 2048:
+        assert sq.sq_workspace_size(sq.SQ_OP_GEMM, M, N, K) > 30 << 20, "the plan was expected to split on pairs"
+    Xq, Wq = rand_i8((M, K), M + 21), rand_i8((N, K), N + 22)
+    Xd, Wd = Xq.to(DEV), Wq.to(DEV)
+    ws = sq.workspace(sq.SQ_OP_GEMM, M, N, K)
+    Y32 = torch.empty((M, N), dtype=torch.int32, device=DEV)
+    for _ in range(2):
+        sq.sq_gemm_w8a8(Xd, Wd, None, None, None, Y32, ws)
+        torch.cuda.synchronize()
+        sq.sq_workspace_status(ws)
+        if N % 8 == 0:
+            assert torch.equal(Y32, torch._int_mm(Xd, Wd.t()))
+    rows = [0, 255, 256, M // 2, M - 1]
+    ref = oracle.gemm_i8(Xq[rows].numpy(), Wq.numpy())
+    assert np.array_equal(Y32[rows].cpu().numpy().astype(np.int64), ref)
+    g = torch.Generator().manual_seed(M + N)
+    qx = (torch.rand(M, generator=g) * 30 + 20).to(DEV)
+    qw = (torch.rand(N, generator=g) * 300 + 200).to(DEV)
+    Y2 = torch.empty((M, N), dtype=dtype, device=DEV)
+    sq.sq_gemm_w8a8(Xd, Wd, qx, qw, None, Y2, ws)
+    torch.cuda.synchronize()
+    sq.sq_workspace_status(ws)
+    Y1 = torch.empty_like(Y2)
+    run(Xd, Wd, qx, qw, None, Y1, "0", monkeypatch)
+    assert torch.equal(Y1.view(torch.int16 if dtype != torch.float32 else torch.int32),
+                       Y2.view(torch.int16 if dtype != torch.float32 else torch.int32))

@@ -128,19 +128,20 @@ struct Params {
     // sk_tiles tiles, sk_iters in all, are cut into one contiguous range per
     // CTA.
     int dp_tiles, sk_tiles, sk_iters;
+    int sk_units;      // the units the split ranges are dealt to: CTAs, or CTA pairs (grid / CG)
     int sk_cnt_bytes;  // size of the counter region, recorded in header word 3 for sq_workspace_status
-    int* sk_cnt;   // [sk_tiles][kEpiWarps] k-blocks counted in per tile region (zero between launches)
+    int* sk_cnt;   // [sk_tiles][CG][kEpiWarps] k-blocks counted in per tile region (zero between launches)
     int* sk_part;  // [grid][2][kEpiWarps][NCH][8][32] int4: parked int32 partial sums
 };
 
-// First k-iteration of CTA c's stream-K range (every CTA gets at least one:
-// sk_iters >= grid).
+// First k-iteration of unit c's stream-K range (a unit is a CTA, or a CTA
+// pair, which splits as one; every unit gets at least one: sk_iters >= units).
 __device__ __forceinline__ int sk_start(int c, const Params& p) {
-    return (int)((int64_t)c * p.sk_iters / (int64_t)gridDim.x);
+    return (int)((int64_t)c * p.sk_iters / (int64_t)p.sk_units);
 }
-// The CTA whose range holds k-iteration x.
+// The unit whose range holds k-iteration x.
 __device__ __forceinline__ int sk_owner(int x, const Params& p) {
-    return (int)((((int64_t)x + 1) * (int64_t)gridDim.x + p.sk_iters - 1) / p.sk_iters - 1);
+    return (int)((((int64_t)x + 1) * (int64_t)p.sk_units + p.sk_iters - 1) / p.sk_iters - 1);
 }
 
 // This CTA's work, the same sequence for its three roles: the pieces of its
@@ -152,13 +153,12 @@ __device__ __forceinline__ int sk_owner(int x, const Params& p) {
 // pair (CG = 2) walks the tiles as one unit: both CTAs see the same sequence.
 template <bool SK, int CG>
 struct Segments {
-    static_assert(!(SK && CG == 2), "stream-K runs on single-CTA tiles only");
     int tile_dp, it, end;
     bool first;
     __device__ explicit Segments(const Params& p) {
         tile_dp = blockIdx.x / CG;
-        it = SK ? sk_start(blockIdx.x, p) : 0;
-        end = SK ? sk_start(blockIdx.x + 1, p) : 0;
+        it = SK ? sk_start(blockIdx.x / CG, p) : 0;
+        end = SK ? sk_start(blockIdx.x / CG + 1, p) : 0;
         first = true;
     }
     __device__ bool next(const Params& p, int num_tiles, int& tile, int& k0, int& k1, int& slot) {
@@ -928,7 +928,9 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
                     __syncwarp();
                     const int u = tile - p.dp_tiles;
                     int before = 0;
-                    if (lane == 0) before = atomicAdd(p.sk_cnt + u * kEpiWarps + wr, k1 - k0);
+                    // (of a pair, each CTA counts its own half of the tile)
+                    int* cnt = p.sk_cnt + ((size_t)u * CG + rank) * kEpiWarps + wr;
+                    if (lane == 0) before = atomicAdd(cnt, k1 - k0);
                     before = __shfl_sync(0xffffffffu, before, 0);
                     if (before + (k1 - k0) == p.num_kb) {
                         __threadfence();
@@ -940,7 +942,8 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
                             for (int cc = c_lo; cc <= c_hi; ++cc) {
                                 const int sl = sk_start(cc, p) >= x0 ? 0 : 1;
                                 const int4* src = reinterpret_cast<const int4*>(p.sk_part) +
-                                                  ((size_t)(cc * 2 + sl) * kEpiWarps + wr) * (NCH * 8 * 32);
+                                                  ((size_t)((cc * CG + (int)rank) * 2 + sl) * kEpiWarps + wr) *
+                                                      (NCH * 8 * 32);
 #pragma unroll
                                 for (int e = 0; e < 8; ++e) {
                                     const int4 v = __ldcg(src + (c * 8 + e) * 32 + lane);
@@ -953,7 +956,7 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
                             epi_chunk<OUT, OUTL, KIND, ACT>(p, ra, c * 32, c_base + c * 32, row0, row, row_ok, rx, rw_w,
                                                        bias_w, stg, lane, n_out, compact, b, &tmap_y);
                         }
-                        if (lane == 0) p.sk_cnt[u * kEpiWarps + wr] = 0;  // ready for the next launch
+                        if (lane == 0) *cnt = 0;  // ready for the next launch
                     }
                     continue;
                 }
@@ -1109,13 +1112,8 @@ KernelFn pick_kernel_act(sq_dtype_t out_dt, int act) {
 
 template <int BN, int CG>
 KernelFn pick_kernel(sq_dtype_t out_dt, bool outl, int kind, bool sk, int act) {
-    if (act != kActNone) {
-        if constexpr (CG == 2) return pick_kernel_act<BN, false, 2>(out_dt, act);
-        else return sk ? pick_kernel_act<BN, true, 1>(out_dt, act) : pick_kernel_act<BN, false, 1>(out_dt, act);
-    }
-    if constexpr (CG == 2) return pick_kernel_sk<BN, false, 2>(out_dt, outl, kind);
-    else
-        return sk ? pick_kernel_sk<BN, true, 1>(out_dt, outl, kind) : pick_kernel_sk<BN, false, 1>(out_dt, outl, kind);
+    if (act != kActNone) return sk ? pick_kernel_act<BN, true, CG>(out_dt, act) : pick_kernel_act<BN, false, CG>(out_dt, act);
+    return sk ? pick_kernel_sk<BN, true, CG>(out_dt, outl, kind) : pick_kernel_sk<BN, false, CG>(out_dt, outl, kind);
 }
 
 // CTA pairs of the pair kernel that can be resident at once on the current
@@ -1171,7 +1169,7 @@ sq_status_t launch_bn(const int8_t* Xq, const int8_t* Wq, int64_t M, int64_t N, 
     const bool outl = ep.idx != nullptr;
     if (outl && ep.out_dt != SQ_BF16 && ep.out_dt != SQ_F16)
         return set_error(SQ_ERR_INVALID_ARG, "sq_gemm_w8a8: the outlier term needs a 16-bit output");
-    const bool sk = CG == 1 && plan.sk_tiles > 0 && sk_ws != nullptr;
+    const bool sk = plan.sk_tiles > 0 && sk_ws != nullptr;
     KernelFn fn = pick_kernel<BN, CG>(ep.out_dt, outl, ep.kind, sk, ep.act);
     // the shared-memory opt-in is per kernel and per device; it is cheap, so set it every time
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM_ALLOC) != cudaSuccess)
@@ -1216,6 +1214,7 @@ sq_status_t launch_bn(const int8_t* Xq, const int8_t* Wq, int64_t M, int64_t N, 
     p.dp_tiles = sk ? plan.tiles - plan.sk_tiles : plan.tiles;
     p.sk_tiles = sk ? plan.sk_tiles : 0;
     p.sk_iters = sk ? plan.sk_tiles * p.num_kb : 0;
+    p.sk_units = plan.grid / CG;
     p.sk_cnt = sk ? static_cast<int*>(sk_ws) : nullptr;
     p.sk_cnt_bytes = sk ? (int)plan.sk_cnt_bytes : 0;
     p.sk_part = sk ? reinterpret_cast<int*>(static_cast<uint8_t*>(sk_ws) + plan.sk_cnt_bytes) : nullptr;
@@ -1228,6 +1227,11 @@ sq_status_t launch_bn(const int8_t* Xq, const int8_t* Wq, int64_t M, int64_t N, 
 }
 
 }  // namespace
+
+// Arrival counters of a split: one per warp region of each CTA's part of a tile.
+static size_t sk_counter_bytes(int64_t tiles, int cg) {
+    return ((size_t)tiles * cg * kEpiWarps * sizeof(int) + 255) / 256 * 256;
+}
 
 GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int64_t batch) {
     GemmPlan pl;
@@ -1254,7 +1258,7 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int64_t batch) {
     if (batch == 1 && pl.grid == sms && tiles > pl.grid && kb >= 32 && rem > 0 && 4 * rem <= 3 * (int64_t)pl.grid &&
         (eff < 0.9 || (eff < 0.95 && kb >= 64)) && rem * kb >= 8ll * pl.grid && rem * kb < (1ll << 31)) {
         pl.sk_tiles = (int)rem;
-        pl.sk_cnt_bytes = ((size_t)rem * kEpiWarps * sizeof(int) + 255) / 256 * 256;
+        pl.sk_cnt_bytes = sk_counter_bytes(rem, 1);
         pl.sk_bytes = pl.sk_cnt_bytes + (size_t)pl.grid * 2 * BM * pl.bn * sizeof(int);
     }
     // CTA pairs (256 x 256 tiles, cta_group::2: each SM streams half the
@@ -1272,7 +1276,22 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int64_t batch) {
             pp.bn = 256;
             pp.cg = 2;
             pp.tiles = (int)ptiles;
-            pp.grid = 2 * (int)(ptiles < pairs ? ptiles : pairs);
+            const int units = (int)(ptiles < pairs ? ptiles : pairs);
+            pp.grid = 2 * units;
+            // the stream-K rule over pairs: the ragged last wave of pair tiles
+            // cut into one k-range per pair, for k-loops of 64 to 128 blocks.
+            // Measured on B200 (us, whole pair tiles -> split): 4096 x 12288 x
+            // 12288 (96 k-blocks, 10.4 waves of 74 pairs) 382 -> 368; longer or
+            // shorter k-loops lost: 4096 x 12288 x 49152 1713 -> 1734,
+            // 2048 x 6144 x 4096 45.2 -> 47.1
+            const int64_t prem = ptiles % units;
+            const double peff = (double)ptiles / (double)(((ptiles + units - 1) / units) * units);
+            if (batch == 1 && units == pairs && ptiles > units && kb >= 64 && kb <= 128 && prem > 0 &&
+                4 * prem <= 3 * (int64_t)units && peff < 0.95 && prem * kb >= 8ll * units && prem * kb < (1ll << 31)) {
+                pp.sk_tiles = (int)prem;
+                pp.sk_cnt_bytes = sk_counter_bytes(prem, 2);
+                pp.sk_bytes = pp.sk_cnt_bytes + (size_t)pp.grid * 2 * BM * pp.bn * sizeof(int);
+            }
             return pp;
         }
     }
@@ -1291,7 +1310,7 @@ sq_status_t launch_gemm_w8a8(const int8_t* Xq, const int8_t* Wq, int64_t M, int6
     void* sk_ws = (pl.sk_tiles > 0 && ws_bytes >= kStatusBytes + pl.sk_bytes)
                       ? static_cast<void*>(reinterpret_cast<uint8_t*>(status_word) + kStatusBytes)
                       : nullptr;
-    if (pl.cg == 2) return launch_bn<256, 2>(Xq, Wq, M, N, K, ep, pl, status_word, nullptr, stream);
+    if (pl.cg == 2) return launch_bn<256, 2>(Xq, Wq, M, N, K, ep, pl, status_word, sk_ws, stream);
     if (pl.bn == 128) return launch_bn<128, 1>(Xq, Wq, M, N, K, ep, pl, status_word, sk_ws, stream);
     return launch_bn<256, 1>(Xq, Wq, M, N, K, ep, pl, status_word, sk_ws, stream);
 }
