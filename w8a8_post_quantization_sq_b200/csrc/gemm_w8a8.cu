@@ -904,7 +904,8 @@ gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
             if (row0 < p.M && c_base < p.N) nch = min(NCH, (p.N - c_base + 31) / 32);
             // Double-buffered TMEM loads only where the variant keeps every
             // value in registers (no spill may sit between a load and its wait).
-            constexpr bool kPipe = !OUTL && OUT != kOutF32 && !SK;
+            // (the single-CTA GELU instance spills a few bytes, so it loads synchronously)
+            constexpr bool kPipe = !OUTL && OUT != kOutF32 && !SK && !(ACT == SQ_ACT_GELU && CG == 1);
             uint32_t ra[32];
             if constexpr (SK) {
                 if (slot >= 0) {
