@@ -443,26 +443,28 @@ norm_quant_bulk_kernel(const T* __restrict__ H, NormArgs a, int R) {
     const int64_t G = gridDim.x;
     constexpr bool FULL = CF == C;
     auto mine = [&](int c) { return c < CF || t + c * kBlock < nch; };
-    float g[C][8];
-#pragma unroll
-    for (int c = 0; c < C; ++c)
-        if (mine(c)) load_gamma(a, t + c * kBlock, g[c]);
+    // the first R rows are requested before anything else, so their DRAM
+    // latency overlaps the loads of gamma' and beta' below (the barriers are
+    // used by other threads only after the block barrier that follows)
     if (t == 0) {
         for (int i = 0; i < R; ++i)
             asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bars[i])));
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        for (int i = 0; i < R; ++i) {
+            const int64_t r = blockIdx.x + i * G;
+            if (r < a.M) issue_row(smem_u32(dsm + (size_t)i * row_bytes), H + r * a.ldh, row_bytes, smem_u32(&bars[i]));
+        }
     }
+    float g[C][8];
+#pragma unroll
+    for (int c = 0; c < C; ++c)
+        if (mine(c)) load_gamma(a, t + c * kBlock, g[c]);
     if (kAmaxSh && a.absmax)
         for (int j = t; j < a.K; j += kBlock) amax_sh[j] = 0.0f;
     if (beta_sh) stage_planes(beta_sh, a.beta, nch, t, kBlock);
     __syncwarp();
     __syncthreads();
-    if (t == 0)
-        for (int i = 0; i < R; ++i) {
-            const int64_t r = blockIdx.x + i * G;
-            if (r < a.M) issue_row(smem_u32(dsm + (size_t)i * row_bytes), H + r * a.ldh, row_bytes, smem_u32(&bars[i]));
-        }
     bool aborted = false;
     int64_t abort_row = a.M;  // first row this block did not finish
     int it = 0;
