@@ -589,6 +589,8 @@ class AttnStack:
     def gemm_shapes(self):
         return [(self.T, self.T, self.dh), (self.T, self.dh, self.T)]
 
+    has_offline = False
+
     def offline(self):
         pass
 
@@ -688,13 +690,15 @@ def run_stack(st, args, rank, world, dev, flush, e2e=True):
     bank_step = st.bank
     st.bank = EventBank()
     st.by_phase = hasattr(st, "phase")  # the offline pass: one interval per phase
-    g_off_ev = capture(st.offline, stream)
+    # (a stack with no offline work captures no graph for it: an empty graph)
+    g_off_ev = capture(st.offline, stream) if getattr(st, "has_offline", True) else None
     bank_off = st.bank
     st.bank, st.by_phase = None, False
     with torch.cuda.stream(stream):
         for _ in range(max(args.warmup, 3)):
             g_step.replay()
-        g_off_ev.replay()
+        if g_off_ev is not None:
+            g_off_ev.replay()
         g_step_ev.replay()
     torch.cuda.synchronize()
 
@@ -720,8 +724,10 @@ def run_stack(st, args, rank, world, dev, flush, e2e=True):
 
     n_ev = max(3, min(args.steps, 50))
     k_step = summarise(bank_step, timed_replays(g_step_ev, bank_step, n_ev, flush, stream), ipk, hbm)
-    k_off = summarise(bank_off, timed_replays(g_off_ev, bank_off, max(3, min(args.steps, 10)), flush, stream), ipk,
-                      hbm)
+    k_off = []
+    if g_off_ev is not None:
+        k_off = summarise(bank_off, timed_replays(g_off_ev, bank_off, max(3, min(args.steps, 10)), flush, stream),
+                          ipk, hbm)
     r = {"ms_per_step": ms_per_step, "step_ms_median": statistics.median(step_ms), "clocks": clk,
          "kernels": k_step, "offline": k_off, "instrumented_replays": n_ev, "ipk": ipk, "hbm": hbm,
          "launches_per_step": st.launches_per_step(),
