@@ -726,6 +726,28 @@ def test_llmint8_detect_counters_reset():
     assert int(hdr[2]) == 0  # the count of finished column groups
 
 
+def test_llmint8_detect_wide_rows():
+    """Rows of more than 32 column groups of 256 (more mask words than the
+    last group's block takes in one pass) with a ragged last group: outlier
+    columns at both ends, on either side of column 8192 and in the last
+    group, found in ascending order on one workspace call after call."""
+    ws = sq.workspace(sq.SQ_OP_LLMINT8_DETECT, 300, 0, 16392)
+    for i, (M, K, cols) in enumerate([(300, 8200, [0, 17, 8191, 8192, 8199]),
+                                      (129, 16392, [5, 4000, 8192, 12000, 16384, 16391]),
+                                      (300, 8200, [1, 8198])]):
+        X = rnd((M, K), 900 + i, torch.float16).clamp(-5, 5)
+        for j, c in enumerate(cols):
+            X[(7 * j) % M, c] = 6.5 + j
+        idx = torch.full((K,), -1, dtype=torch.int32, device=DEV)
+        n = torch.full((1,), -1, dtype=torch.int32, device=DEV)
+        sq.sq_llmint8_detect(X.to(DEV), 6.0, 0.0, idx, n, ws)
+        torch.cuda.synchronize()
+        ref = oracle.llmint8_outliers(X, 6.0, 0.0).tolist()
+        assert ref == cols
+        assert int(n.item()) == len(cols) and idx[:len(cols)].cpu().tolist() == cols
+    assert int(ws[:256].view(torch.int32)[2].item()) == 0  # the count of finished column groups
+
+
 def test_llmint8_min_ratio():
     M, K = 200, 256
     X = rnd((M, K), 61, torch.float16).clamp(-5, 5)
