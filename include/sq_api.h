@@ -390,8 +390,10 @@ SQ_API sq_status_t sq_gemm_fp8(const uint8_t* Xq, const uint8_t* Wq, int64_t M, 
  * int32, device. Workspace: SQ_OP_LLMINT8_DETECT, zeroed once before its
  * first use: it holds arrival counters that every completed call leaves at
  * zero (one pass over X counts per 128-row band; the last band of each
- * 256-column group adds the group up, the last group writes O). Calls sharing
- * a workspace must not run concurrently. K % 8 == 0. */
+ * 256-column group adds the group up, the last group writes O). The counters
+ * sit at the same bytes for every M and K, so a workspace serves any later
+ * call it is large enough for. Calls sharing a workspace must not run
+ * concurrently. K % 8 == 0, K <= 2^20. */
 SQ_API sq_status_t sq_llmint8_detect(const void* X, sq_dtype_t dt, int64_t M, int64_t K, int64_t ldx,
                               float threshold, double min_ratio, int32_t* outlier_idx,
                               int32_t* n_outliers, void* workspace, size_t ws_bytes,
@@ -406,9 +408,9 @@ SQ_API sq_status_t sq_llmint8_detect(const void* X, sq_dtype_t dt, int64_t M, in
  * nothing to spare), or a service that must not allocate once it is serving.
  * The scratch is a fixed 4 MiB device array inside this library, one per
  * device that loads it, held until the process exits. It holds the per-band
- * counts (4 * ceil(M / 128) * K bytes) after a 256-byte header and 36 bytes
- * of counters and masks per 256 columns (each region rounded up to 256
- * bytes), so for example M <= 32640 at K = 4096; larger sizes return
+ * counts (4 * ceil(M / 128) * K bytes) after a 256-byte header, 16 KiB of
+ * arrival counters and 32 bytes of outlier mask per 256 columns (rounded up
+ * to 256 bytes), so for example M <= 32512 at K = 4096; larger sizes return
  * SQ_ERR_UNSUPPORTED_SHAPE and launch nothing.
  * The first call in a CUDA context looks up the array's device address there
  * (cudaGetSymbolAddress), keyed by the context's unique id, so a new context

@@ -730,7 +730,10 @@ def test_llmint8_detect_wide_rows():
     """Rows of more than 32 column groups of 256 (more mask words than the
     last group's block takes in one pass) with a ragged last group: outlier
     columns at both ends, on either side of column 8192 and in the last
-    group, found in ascending order on one workspace call after call."""
+    group, found in ascending order on one workspace call after call, the
+    second call wider than the first: the arrival counters sit at the same
+    bytes for every K, so the first call's masks and counts (left behind,
+    not cleared) are never read as the second call's counters."""
     ws = sq.workspace(sq.SQ_OP_LLMINT8_DETECT, 300, 0, 16392)
     for i, (M, K, cols) in enumerate([(300, 8200, [0, 17, 8191, 8192, 8199]),
                                       (129, 16392, [5, 4000, 8192, 12000, 16384, 16391]),

@@ -41,10 +41,16 @@ static size_t r256(size_t b) { return (b + 255) / 256 * 256; }
 // Detection scratch: the 256-byte header (word 0 status, word 1 "O changed",
 // word 2 the count of finished column groups), one arrival counter per
 // 256-column group, the groups' outlier masks (8 words each), then the
-// per-band column counts [row bands, K].
+// per-band column counts [row bands, K]. The arrival counters take room for
+// the widest rows any call takes (K <= 2^20: 4096 groups), so they sit at the
+// same bytes whatever K a call has: a call that leaves them at zero leaves a
+// workspace ready for any later call, while the masks and counts a call
+// leaves behind (written before they are read) never land where a later
+// call with more columns expects a zero counter.
+constexpr int64_t kMaxDetectK = int64_t(1) << 20;
 static int64_t col_groups(int64_t K) { return (K + 255) / 256; }
 static size_t detect_done_off() { return kStatusBytes; }
-static size_t detect_mask_off(int64_t K) { return detect_done_off() + r256((size_t)col_groups(K) * 4); }
+static size_t detect_mask_off(int64_t) { return detect_done_off() + (size_t)col_groups(kMaxDetectK) * 4; }
 static size_t detect_count_off(int64_t K) { return detect_mask_off(K) + r256((size_t)col_groups(K) * 32); }
 
 size_t detect_workspace_bytes(int64_t M, int64_t K) {
@@ -403,7 +409,7 @@ sq_status_t launch_detect(const void* X, sq_dtype_t dt, int64_t M, int64_t K, in
     int64_t rb = (M + kDetectRows - 1) / kDetectRows;
     if (rb < 1) rb = 1;  // M == 0: one band with no rows, so O is empty
     SQ_REQUIRE(rb <= 65535, SQ_ERR_UNSUPPORTED_SHAPE, "sq_llmint8_detect: M too large");
-    SQ_REQUIRE(col_groups(K) < (1ll << 31), SQ_ERR_UNSUPPORTED_SHAPE, "sq_llmint8_detect: K too large");
+    SQ_REQUIRE(K <= kMaxDetectK, SQ_ERR_UNSUPPORTED_SHAPE, "sq_llmint8_detect: K too large");
     dim3 grid((unsigned)col_groups(K), (unsigned)rb);
     if (dt == SQ_BF16)
         launch_pdl(detect_kernel<__nv_bfloat16>, grid, dim3(kWarps * 32), 0, s, static_cast<const __nv_bfloat16*>(X), M,
@@ -458,7 +464,7 @@ sq_status_t check_x(const char* name, const void* X, sq_dtype_t dt, int64_t M, i
     SQ_REQUIRE(dt == SQ_F16 || dt == SQ_BF16, SQ_ERR_INVALID_ARG, "%s: dtype must be F16 or BF16", name);
     SQ_REQUIRE(M >= 0 && K > 0 && ldx >= K && K % 8 == 0 && ldx % 8 == 0, SQ_ERR_UNSUPPORTED_SHAPE,
                "%s: need K > 0, K %% 8 == 0, ldx >= K, ldx %% 8 == 0", name);
-    SQ_REQUIRE(K <= (1 << 20), SQ_ERR_UNSUPPORTED_SHAPE, "%s: K too large", name);
+    SQ_REQUIRE(K <= kMaxDetectK, SQ_ERR_UNSUPPORTED_SHAPE, "%s: K too large", name);
     SQ_REQUIRE(aligned16(X), SQ_ERR_ALIGNMENT, "%s: input not 16-byte aligned", name);
     return SQ_OK;
 }
