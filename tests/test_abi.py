@@ -77,22 +77,22 @@ def test_workspace_sizes(L):
     assert L.sq_workspace_size(99, 1, 1, 1) == 0
     # GEMM plan on 148 SMs: 2048 x 6144 makes 384 tiles of 128 x 256, a last
     # wave of 88; with a k-loop of 128 blocks those 88 are cut by k-blocks:
-    # arrival counters for 88 tiles x 8
-    # epilogue regions (a multiple of 256 bytes) plus two parked 128 x 256
-    # int32 partials per CTA after the 256-byte header
-    assert L.sq_workspace_size(0, 2048, 6144, 16384) == 256 + 2816 + 148 * 2 * 128 * 256 * 4
+    # after the 256-byte header, the arrival counters (a region of one size
+    # for every shape: 256 CTA parts x 8 epilogue regions x 4 bytes) plus two
+    # parked 128 x 256 int32 partials per CTA
+    SK_CNT = 256 * 8 * 4
+    assert L.sq_workspace_size(0, 2048, 6144, 16384) == 256 + SK_CNT + 148 * 2 * 128 * 256 * 4
     # 1024 x 7168: 224 tiles, a last wave of 76 (half full): cut at 224 and at
-    # 56 k-blocks (counters for 76 tiles x 8 regions, padded to 2560 bytes)
-    assert L.sq_workspace_size(0, 1024, 7168, 28672) == 256 + 2560 + 148 * 2 * 128 * 256 * 4
-    assert L.sq_workspace_size(0, 1024, 7168, 7168) == 256 + 2560 + 148 * 2 * 128 * 256 * 4
+    # 56 k-blocks
+    assert L.sq_workspace_size(0, 1024, 7168, 28672) == 256 + SK_CNT + 148 * 2 * 128 * 256 * 4
+    assert L.sq_workspace_size(0, 1024, 7168, 7168) == 256 + SK_CNT + 148 * 2 * 128 * 256 * 4
     # 2048 x 16384: 1024 tiles, last wave 136 of 148: whole tiles only
     assert L.sq_workspace_size(0, 2048, 16384, 4096) == 256
     # 4096 x 36864: 4608 tiles, 97 % of the waves busy: whole tiles only
     assert L.sq_workspace_size(0, 4096, 36864, 12288) == 256
     # 4096 x 12288: 1536 tiles, 94 % busy; cut with a k-loop of 384 blocks
-    # (counters for the last wave's 56 tiles), not with one of 56 blocks
-    # (1024 x 21504: 91 % busy)
-    assert L.sq_workspace_size(0, 4096, 12288, 49152) == 256 + 1792 + 148 * 2 * 128 * 256 * 4
+    # (the last wave's 56 tiles), not with one of 56 blocks (1024 x 21504: 91 % busy)
+    assert L.sq_workspace_size(0, 4096, 12288, 49152) == 256 + SK_CNT + 148 * 2 * 128 * 256 * 4
     assert L.sq_workspace_size(0, 1024, 21504, 7168) == 256
     # a short k-loop (8 blocks) is never cut, nor a thin remainder: 260 x
     # 13000 leaves 5 tiles of 128 k-blocks, under 8 k-blocks per CTA

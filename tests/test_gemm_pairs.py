@@ -223,3 +223,25 @@ def test_pairs_stream_k(M, N, K, dtype, monkeypatch):
     run(Xd, Wd, qx, qw, None, Y1, "0", monkeypatch)
     assert torch.equal(Y1.view(torch.int16 if dtype != torch.float32 else torch.int32),
                        Y2.view(torch.int16 if dtype != torch.float32 else torch.int32))
+
+
+def test_stream_k_workspace_shared_between_shapes(monkeypatch):
+    """One workspace, sized for the larger of two shapes that both split their
+    last wave, used by each in turn: single CTAs cutting 76 tiles
+    (1024 x 7168 x 7168), then CTA pairs cutting 44 pair tiles
+    (2048 x 6144 x 8192), then the first shape again. The arrival counters sit
+    at the same bytes for every shape, so the partial sums one shape parks
+    are never read as the other's counters: every call exact against the
+    CUDA library's int8 matmul."""
+    monkeypatch.delenv("SQ_GEMM_CTA_PAIRS", raising=False)
+    shapes = [(1024, 7168, 7168), (2048, 6144, 8192), (1024, 7168, 7168)]
+    size = max(sq.sq_workspace_size(sq.SQ_OP_GEMM, M, N, K) for M, N, K in shapes)
+    assert all(sq.sq_workspace_size(sq.SQ_OP_GEMM, M, N, K) > 256 for M, N, K in shapes), "both shapes split"
+    ws = torch.zeros(size, dtype=torch.uint8, device=DEV)
+    for i, (M, N, K) in enumerate(shapes):
+        Xd, Wd = rand_i8((M, K), 700 + i).to(DEV), rand_i8((N, K), 800 + i).to(DEV)
+        Y32 = torch.empty((M, N), dtype=torch.int32, device=DEV)
+        sq.sq_gemm_w8a8(Xd, Wd, None, None, None, Y32, ws)
+        torch.cuda.synchronize()
+        sq.sq_workspace_status(ws)
+        assert torch.equal(Y32, torch._int_mm(Xd, Wd.t())), f"call {i}: {M} x {N} x {K}"

@@ -1229,10 +1229,16 @@ sq_status_t launch_bn(const int8_t* Xq, const int8_t* Wq, int64_t M, int64_t N, 
 
 }  // namespace
 
-// Arrival counters of a split: one per warp region of each CTA's part of a tile.
-static size_t sk_counter_bytes(int64_t tiles, int cg) {
-    return ((size_t)tiles * cg * kEpiWarps * sizeof(int) + 255) / 256 * 256;
-}
+// Arrival counters of a split: one per warp region of each CTA's part of a
+// tile, in a region of one size for every shape (room for kSkMaxParts CTA
+// parts of tiles; a split covers less than one wave, so fewer parts than
+// SMs). The counters thus sit at the same bytes whatever the shape: a call
+// that leaves them at zero leaves the workspace ready for a call of any other
+// shape it is large enough for, and the partial sums one shape parks after
+// its counters are never read as another shape's counters.
+constexpr int64_t kSkMaxParts = 256;
+static size_t sk_counter_bytes() { return (size_t)kSkMaxParts * kEpiWarps * sizeof(int); }
+static_assert((kSkMaxParts * kEpiWarps * sizeof(int)) % 256 == 0, "the parked sums start 256-byte aligned");
 
 GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int64_t batch) {
     GemmPlan pl;
@@ -1257,9 +1263,10 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int64_t batch) {
     const int64_t rem = tiles % pl.grid;
     const double eff = (double)tiles / (double)(((tiles + pl.grid - 1) / pl.grid) * pl.grid);
     if (batch == 1 && pl.grid == sms && tiles > pl.grid && kb >= 32 && rem > 0 && 4 * rem <= 3 * (int64_t)pl.grid &&
-        (eff < 0.9 || (eff < 0.95 && kb >= 64)) && rem * kb >= 8ll * pl.grid && rem * kb < (1ll << 31)) {
+        (eff < 0.9 || (eff < 0.95 && kb >= 64)) && rem * kb >= 8ll * pl.grid && rem * kb < (1ll << 31) &&
+        rem <= kSkMaxParts) {
         pl.sk_tiles = (int)rem;
-        pl.sk_cnt_bytes = sk_counter_bytes(rem, 1);
+        pl.sk_cnt_bytes = sk_counter_bytes();
         pl.sk_bytes = pl.sk_cnt_bytes + (size_t)pl.grid * 2 * BM * pl.bn * sizeof(int);
     }
     // CTA pairs (256 x 256 tiles, cta_group::2: each SM streams half the
@@ -1288,9 +1295,10 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int64_t batch) {
             const int64_t prem = ptiles % units;
             const double peff = (double)ptiles / (double)(((ptiles + units - 1) / units) * units);
             if (batch == 1 && units == pairs && ptiles > units && kb >= 64 && kb <= 128 && prem > 0 &&
-                4 * prem <= 3 * (int64_t)units && peff < 0.95 && prem * kb >= 8ll * units && prem * kb < (1ll << 31)) {
+                4 * prem <= 3 * (int64_t)units && peff < 0.95 && prem * kb >= 8ll * units && prem * kb < (1ll << 31) &&
+                2 * prem <= kSkMaxParts) {
                 pp.sk_tiles = (int)prem;
-                pp.sk_cnt_bytes = sk_counter_bytes(prem, 2);
+                pp.sk_cnt_bytes = sk_counter_bytes();
                 pp.sk_bytes = pp.sk_cnt_bytes + (size_t)pp.grid * 2 * BM * pp.bn * sizeof(int);
             }
             return pp;
