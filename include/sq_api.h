@@ -298,7 +298,8 @@ SQ_API sq_status_t sq_act_quant(const void* A, sq_dtype_t dt, int64_t M, int64_t
  *   the status word and the counters at zero again (the parked sums need no
  *   clearing). The counters sit at the same bytes (an 8 KiB region after the
  *   256-byte header) for every shape, so one workspace, sized for the largest,
- *   serves calls of several shapes in turn. After a call that timed out, sq_workspace_status (which
+ *   serves GEMM calls of several shapes in turn (not calls of other ops,
+ *   whose counters sit elsewhere). After a call that timed out, sq_workspace_status (which
  *   reports SQ_ERR_TIMEOUT) clears the counters as well. A smaller workspace (at
  *   least 256 bytes) is accepted and runs every tile whole. Calls sharing one
  *   workspace must not run concurrently.
