@@ -72,6 +72,13 @@ def test_workspace_sizes(L):
     assert L.sq_workspace_size(0, 2048, 4096, 1024) >= 256
     det = L.sq_workspace_size(3, 2048, 0, 4096)
     assert det >= 256 + 16 * 4096 * 4
+    # detection: the header, arrival counters for the 4096 column groups of the
+    # widest rows (at the same bytes for every K), 32 bytes of mask per group,
+    # then the per-band counts
+    r256 = lambda b: (b + 255) // 256 * 256
+    for M, K in [(2048, 4096), (300, 8200), (129, 16392), (1, 1 << 20)]:
+        groups, bands = (K + 255) // 256, (M + 127) // 128
+        assert L.sq_workspace_size(3, M, 0, K) == 256 + 4096 * 4 + r256(groups * 32) + r256(bands * K * 4)
     full = L.sq_workspace_size(4, 2048, 16384, 4096)
     assert full >= det + 2048 * 4096 + 2048 * 4
     assert L.sq_workspace_size(99, 1, 1, 1) == 0
